@@ -1,0 +1,284 @@
+"""CPU oracle for the packed-sequence pre-norm encoder layer (numpy, float64).
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports this module;
+only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may call it.  It shares no code, table or helper with the CUDA
+path: it is a plain, slow, direct restatement of what the layer computes,
+written so that it can be checked against the pages by eye.
+
+Sources (web pages, cited by title and section):
+  * "Days-gone/cti2026" README -- TransformerEncoder section (per-layer
+    pseudo-code: LayerNorm, Linear_qkv, FlashAttention_Varlen(qkv,
+    user_offsets), residual + Linear_out, LayerNorm, Gate -> (topk_idx,
+    topk_weight), FusedMoE, residual), the FlashAttention_Varlen operator
+    design (segment boundaries from cu_seqlens, query i sees keys 0..i of its
+    own user, online softmax in fp32), the SMoE structure (Gate Linear(512->8)
+    then softmax -> top-2 -> renormalise; 8 experts Linear(512->1024) + ReLU
+    + Linear(1024->512); each token weighted over its 2 experts), the fused
+    MoE routing notes (per-expert counts, token reordering, route-major rows
+    token_id*top_k + k_idx, per-token weighted sum) and the Prediction Head
+    section (Linear(512->1) -> clamp(-15, 15) -> sigmoid, pred_mask select).
+  * "CTI-Inference-Opt" optimisation plan -- attention as softmax(QK^T/sqrt(d))V.
+  * "CTI-Inference-Opt" AUC-recovery plan -- the dense block-diagonal causal
+    mask built from user_offsets (same user AND lower triangle), the
+    FlexAttention mask_mod restatement of it, and the vectorised SMoE that
+    evaluates all experts for all tokens and then gathers the top-k.
+
+Readings taken where the pages are silent:
+  * every Linear has a bias; LayerNorm eps = 1e-5 with biased variance;
+  * QKV columns split as [Q | K | V], head h = 64-column block h of each;
+  * softmax scale 1/sqrt(64) = 0.125;
+  * top-2 ties go to the lower expert index, slot 0 holds the larger weight;
+  * renormalised weights w_k = p_k / (p_e0 + p_e1) with no epsilon;
+  * route id r = 2 t + k; within an expert, routes are ordered by ascending r
+    (a stable counting sort);
+  * the head applies a final LayerNorm before Linear(512->1).
+
+Parity status: every function below is pinned by tests/test_oracle_pins.py
+(closed forms, library routines, brute force and invariants); the composed
+random layer beyond those pins is checked only through its pinned parts.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+LN_EPS = 1e-5
+N_HEADS = 8
+D_HEAD = 64
+TOP_K = 2
+LOGIT_CLAMP = 15.0
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# LayerNorm and Linear (cti2026 README, TransformerEncoder section)
+# --------------------------------------------------------------------------
+def layer_norm(x, gamma, beta, eps=LN_EPS):
+    """Per-row LayerNorm: (x - mean) / sqrt(biased var + eps) * gamma + beta."""
+    x = _f64(x)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * _f64(gamma) + _f64(beta)
+
+
+def linear(x, weight, bias=None):
+    """nn.Linear: y = x W^T + b with W stored [out, in]."""
+    y = _f64(x) @ _f64(weight).T
+    if bias is not None:
+        y = y + _f64(bias)
+    return y
+
+
+def split_qkv(qkv):
+    """[T, 3*H*Dh] -> q, k, v each [T, H, Dh]; columns are [Q | K | V] and
+    head h owns columns h*Dh .. h*Dh+Dh-1 of each block."""
+    qkv = _f64(qkv)
+    T = qkv.shape[0]
+    hd = qkv.shape[1] // 3
+    H = hd // D_HEAD
+    q = qkv[:, :hd].reshape(T, H, D_HEAD)
+    k = qkv[:, hd:2 * hd].reshape(T, H, D_HEAD)
+    v = qkv[:, 2 * hd:].reshape(T, H, D_HEAD)
+    return q, k, v
+
+
+# --------------------------------------------------------------------------
+# Attention (cti2026 README, FlashAttention_Varlen operator design)
+# --------------------------------------------------------------------------
+def _softmax_rows(s):
+    s = s - s.max(axis=-1, keepdims=True)
+    p = np.exp(s)
+    return p / p.sum(axis=-1, keepdims=True)
+
+
+def jagged_causal_attention(q, k, v, cu_seqlens, scale=None):
+    """Block-diagonal causal attention over a packed stream.
+
+    q, k, v: [T, H, Dh].  For user u (tokens cu[u] .. cu[u+1]-1) and head h,
+    S = Q_u K_u^T * scale with S[i, j] = -inf for j > i, P = row softmax(S),
+    O_u = P V_u.  Tokens of other users are never seen.  Returns [T, H, Dh].
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, H, Dh = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dh)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    out = np.zeros_like(q)
+    for u in range(len(cu) - 1):
+        s, e = int(cu[u]), int(cu[u + 1])
+        L = e - s
+        if L <= 0:
+            continue
+        future = np.triu(np.ones((L, L), dtype=bool), k=1)
+        for h in range(H):
+            S = q[s:e, h, :] @ k[s:e, h, :].T * scale
+            S[future] = -np.inf
+            out[s:e, h, :] = _softmax_rows(S) @ v[s:e, h, :]
+    return out
+
+
+def dense_block_causal_mask(cu_seqlens):
+    """[T, T] boolean mask: key j visible to query i iff same user and j <= i
+    (the AUC-recovery plan's dense mask and its FlexAttention mask_mod)."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    lengths = np.diff(cu)
+    user_of = np.repeat(np.arange(len(lengths)), lengths)
+    T = int(cu[-1])
+    same = user_of[:, None] == user_of[None, :]
+    causal = np.tril(np.ones((T, T), dtype=bool))
+    return same & causal
+
+
+def dense_masked_attention(q, k, v, cu_seqlens, scale=None):
+    """Second formulation: one [T, T] score matrix per head with the dense
+    block-diagonal causal mask applied (tiny inputs only)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, H, Dh = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dh)
+    mask = dense_block_causal_mask(cu_seqlens)
+    out = np.zeros_like(q)
+    for h in range(H):
+        S = q[:, h, :] @ k[:, h, :].T * scale
+        S = np.where(mask, S, -np.inf)
+        out[:, h, :] = _softmax_rows(S) @ v[:, h, :]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Gate (cti2026 README, SMoE structure: softmax -> top-2 -> renormalise)
+# --------------------------------------------------------------------------
+def gate_probs(xn2, w_gate, b_gate):
+    """p = softmax(xn2 Wg^T + bg) over the experts, [T, E]."""
+    return _softmax_rows(linear(xn2, w_gate, b_gate))
+
+
+def top2(p):
+    """Top-2 experts by descending probability (ties: lower expert index
+    first), and their renormalised weights.  Returns idx [T,2] int64, w [T,2]."""
+    p = _f64(p)
+    order = np.argsort(-p, axis=-1, kind="stable")
+    idx = order[:, :TOP_K]
+    pt = np.take_along_axis(p, idx, axis=-1)
+    w = pt / pt.sum(axis=-1, keepdims=True)
+    return idx.astype(np.int64), w
+
+
+def top2_gap(p):
+    """p_(2) - p_(3): how far the chosen pair sits from the first left out."""
+    ps = -np.sort(-_f64(p), axis=-1)
+    return ps[:, 1] - ps[:, 2]
+
+
+# --------------------------------------------------------------------------
+# Route builder (cti2026 README, fused MoE routing preparation)
+# --------------------------------------------------------------------------
+def route_build(idx, num_experts):
+    """Counting sort of the routes r = 2 t + k by expert.
+
+    Returns cnt [E] (routes per expert), off [E+1] (exclusive prefix of cnt),
+    perm [2T] (perm[off[e] + j] = j-th route of expert e, ascending r) and
+    pos [2T] (the inverse: the slot of route r).
+    """
+    r_expert = np.asarray(idx, dtype=np.int64).reshape(-1)
+    cnt = np.bincount(r_expert, minlength=num_experts).astype(np.int64)
+    off = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int64)
+    perm = np.argsort(r_expert, kind="stable").astype(np.int64)
+    pos = np.empty_like(perm)
+    pos[perm] = np.arange(perm.size)
+    return cnt, off, perm, pos
+
+
+# --------------------------------------------------------------------------
+# Experts and combine (cti2026 README, SMoE + fused MoE; AUC-recovery plan)
+# --------------------------------------------------------------------------
+def expert_ffn(x, w1, b1, w2, b2):
+    """One expert: Linear(D->F) + ReLU + Linear(F->D)."""
+    return linear(np.maximum(linear(x, w1, b1), 0.0), w2, b2)
+
+
+def moe_routed(xn2, idx, w, w1, b1, w2, b2):
+    """Sparse top-2 MoE.  Routes are grouped per expert with ``route_build``;
+    each expert runs its FFN on its gathered tokens; route r's result is kept
+    in route-major row r = 2 t + k; token t's output is w[t,0] y[2t] +
+    w[t,1] y[2t+1].  Returns (moe_out [T, D], y [2T, D], hidden per route
+    [2T, F] in slot order)."""
+    xn2 = _f64(xn2)
+    T, D = xn2.shape
+    E = np.asarray(w1).shape[0]
+    F = np.asarray(w1).shape[1]
+    cnt, off, perm, _ = route_build(idx, E)
+    y = np.zeros((2 * T, D))
+    hidden = np.zeros((2 * T, F))
+    for e in range(E):
+        routes = perm[off[e]:off[e + 1]]
+        if routes.size == 0:
+            continue
+        tok = routes // TOP_K
+        h = np.maximum(linear(xn2[tok], w1[e], b1[e]), 0.0)
+        hidden[off[e]:off[e + 1]] = h
+        y[routes] = linear(h, w2[e], b2[e])
+    w = _f64(w)
+    out = w[:, 0:1] * y[0::2] + w[:, 1:2] * y[1::2]
+    return out, y, hidden
+
+
+def moe_dense_all_experts(xn2, idx, w, w1, b1, w2, b2):
+    """Second formulation: every expert on every token, then gather the two
+    selected outputs and weight them."""
+    xn2 = _f64(xn2)
+    E = np.asarray(w1).shape[0]
+    allout = np.stack([expert_ffn(xn2, w1[e], b1[e], w2[e], b2[e]) for e in range(E)], axis=1)
+    sel = np.take_along_axis(allout, np.asarray(idx)[:, :, None], axis=1)  # [T, 2, D]
+    return (sel * _f64(w)[:, :, None]).sum(axis=1)
+
+
+# --------------------------------------------------------------------------
+# Layer, stack, head (cti2026 README, TransformerEncoder + Prediction Head)
+# --------------------------------------------------------------------------
+def layer_forward(x, cu_seqlens, wts, return_intermediates=False):
+    """One pre-norm layer over the packed stream x [T, D]."""
+    x = _f64(x)
+    T, D = x.shape
+    xn = layer_norm(x, wts["ln1_g"], wts["ln1_b"])
+    qkv = linear(xn, wts["w_qkv"], wts.get("b_qkv"))
+    q, k, v = split_qkv(qkv)
+    attn = jagged_causal_attention(q, k, v, cu_seqlens).reshape(T, D)
+    x1 = x + linear(attn, wts["w_o"], wts.get("b_o"))
+    xn2 = layer_norm(x1, wts["ln2_g"], wts["ln2_b"])
+    p = gate_probs(xn2, wts["w_gate"], wts.get("b_gate"))
+    idx, w = top2(p)
+    moe, y, hidden = moe_routed(xn2, idx, w, wts["w1"], wts["b1"], wts["w2"], wts["b2"])
+    out = x1 + moe
+    if not return_intermediates:
+        return out
+    E = np.asarray(wts["w1"]).shape[0]
+    cnt, off, perm, pos = route_build(idx, E)
+    return out, dict(xn=xn, qkv=qkv, attn=attn, x1=x1, xn2=xn2, p=p, idx=idx, w=w,
+                     gap=top2_gap(p), cnt=cnt, off=off, perm=perm, pos=pos, y=y,
+                     hidden=hidden, moe=moe)
+
+
+def head_forward(x, head, pred_mask=None):
+    """Final LayerNorm, Linear(D->1), clamp to [-15, 15], sigmoid; keep the
+    tokens whose pred_mask is set, in ascending token order."""
+    z = linear(layer_norm(x, head["lnf_g"], head["lnf_b"]),
+               _f64(head["w"]).reshape(1, -1), head.get("b")).reshape(-1)
+    z = np.clip(z, -LOGIT_CLAMP, LOGIT_CLAMP)
+    probs = 1.0 / (1.0 + np.exp(-z))
+    if pred_mask is None:
+        return probs
+    return probs[np.asarray(pred_mask).astype(bool)]
+
+
+def stack_forward(x, cu_seqlens, layers, head=None, pred_mask=None):
+    """L layers in sequence, each with its own weights, then the optional head."""
+    h = _f64(x)
+    for wts in layers:
+        h = layer_forward(h, cu_seqlens, wts)
+    if head is None:
+        return h
+    return h, head_forward(h, head, pred_mask)

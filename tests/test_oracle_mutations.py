@@ -1,0 +1,112 @@
+"""Plant plausible mistakes in the oracle (on the CPU, by monkeypatching) and
+check that at least one pin in test_oracle_pins fails for each.  This shows
+the pins constrain every step rather than restating the oracle."""
+import numpy as np
+import pytest
+
+from oracle import ptl_oracle as O
+import tests.test_oracle_pins as P
+
+
+def _fails(fn):
+    try:
+        fn()
+    except AssertionError:
+        return True
+    return False
+
+
+def test_wrong_softmax_scale_is_caught(monkeypatch):
+    orig = O.jagged_causal_attention
+    monkeypatch.setattr(O, "jagged_causal_attention",
+                        lambda q, k, v, cu, scale=None: orig(q, k, v, cu, scale=1.0 / 64))
+    assert _fails(P.test_attention_closed_form_golden)
+    assert _fails(P.test_attention_single_user_is_torch_causal_sdpa)
+
+
+def test_missing_causal_mask_is_caught(monkeypatch):
+    def no_causal(q, k, v, cu, scale=None):
+        q, k, v = (np.asarray(a, np.float64) for a in (q, k, v))
+        out = np.zeros_like(q)
+        for u in range(len(cu) - 1):
+            s, e = int(cu[u]), int(cu[u + 1])
+            if e == s:
+                continue
+            for h in range(q.shape[1]):
+                S = q[s:e, h] @ k[s:e, h].T / 8.0
+                out[s:e, h] = O._softmax_rows(S) @ v[s:e, h]
+        return out
+    monkeypatch.setattr(O, "jagged_causal_attention", no_causal)
+    assert _fails(P.test_attention_first_token_outputs_its_own_v)
+    assert _fails(P.test_attention_matches_dense_block_causal_mask)
+
+
+def test_cross_user_leak_is_caught(monkeypatch):
+    orig = O.jagged_causal_attention
+    monkeypatch.setattr(O, "jagged_causal_attention",
+                        lambda q, k, v, cu, scale=None: orig(q, k, v, [0, int(cu[-1])], scale))
+    assert _fails(P.test_attention_user_permutation_and_isolation)
+    assert _fails(P.test_attention_closed_form_golden)
+
+
+def test_swapped_k_and_v_blocks_are_caught(monkeypatch):
+    orig = O.split_qkv
+
+    def swapped(qkv):
+        q, k, v = orig(qkv)
+        return q, v, k
+    monkeypatch.setattr(O, "split_qkv", swapped)
+    assert _fails(P.test_layer_zero_query_weights_give_prefix_mean_of_v)
+
+
+def test_tie_break_to_higher_index_is_caught(monkeypatch):
+    def top2_hi(p):
+        p = np.asarray(p, np.float64)
+        E = p.shape[1]
+        order = E - 1 - np.argsort(-p[:, ::-1], axis=-1, kind="stable")
+        idx = order[:, :2]
+        pt = np.take_along_axis(p, idx, axis=-1)
+        return idx, pt / pt.sum(-1, keepdims=True)
+    monkeypatch.setattr(O, "top2", top2_hi)
+    assert _fails(P.test_top2_golden_ties_and_weights)
+
+
+def test_missing_renormalisation_is_caught(monkeypatch):
+    def top2_raw(p):
+        p = np.asarray(p, np.float64)
+        idx = np.argsort(-p, axis=-1, kind="stable")[:, :2]
+        return idx, np.take_along_axis(p, idx, axis=-1)
+    monkeypatch.setattr(O, "top2", top2_raw)
+    assert _fails(P.test_layer_constant_expert_output_adds_constant)
+    assert _fails(P.test_top2_golden_ties_and_weights)
+
+
+def test_unstable_route_order_is_caught(monkeypatch):
+    orig = O.route_build
+
+    def unstable(idx, E):
+        cnt, off, perm, pos = orig(idx, E)
+        perm = perm.copy()
+        for e in range(E):
+            perm[off[e]:off[e + 1]] = perm[off[e]:off[e + 1]][::-1]
+        pos = np.empty_like(perm)
+        pos[perm] = np.arange(perm.size)
+        return cnt, off, perm, pos
+    monkeypatch.setattr(O, "route_build", unstable)
+    assert _fails(P.test_route_build_golden)
+    assert _fails(P.test_route_build_brute_force)
+
+
+def test_dropped_expert_bias_is_caught(monkeypatch):
+    orig = O.moe_routed
+
+    def no_b2(xn2, idx, w, w1, b1, w2, b2):
+        return orig(xn2, idx, w, w1, b1, w2, np.zeros_like(np.asarray(b2, np.float64)))
+    monkeypatch.setattr(O, "moe_routed", no_b2)
+    assert _fails(P.test_moe_golden)
+    assert _fails(P.test_layer_constant_expert_output_adds_constant)
+
+
+def test_missing_logit_clamp_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "LOGIT_CLAMP", 1e9)
+    assert _fails(P.test_head_clamp_and_sigmoid_values)
