@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the packed-sequence encoder stack on B200.
+
+Metric: packed tokens/s per layer forward (jagged causal attention + top-2
+MoE) on the 60-user / 6823-token packing, and its fraction of the tensor
+core roofline.  One step = the whole hot path once over one batch: the
+attention work list, 8 layers (LayerNorm1 + QKV GEMM, jagged attention,
+output projection + residual, LayerNorm2 + gate + top-2, route counting
+sort, expert GEMM1 + ReLU, expert GEMM2 + combine + residual) and the
+prediction head.  value = tokens x layers / step time, summed over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload stack8|layer]
+
+N > 1 runs under torch.distributed.run: every rank processes its own batch
+of the same shape (weak scaling, no collective on the data path); the step
+time is the max over ranks.  --impl reference times the CPU oracle (numpy
+fp64) on this host on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed tokens/s per layer fwd (attn+top-2 MoE), 6823 tok/60 users; % TC peak"
+GEMM_FLOPS_PER_TOKEN = 2 * 512 * 1536 + 2 * 512 * 512 + 2 * 512 * 8 + 2 * 2 * (2 * 512 * 1024)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["stack8", "layer"], default="stack8")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def make_workload(name, rank):
+    from packed_sequence_transformer_b200 import synthetic as S
+    lengths = S.config1_lengths()
+    if name == "stack8":
+        c = S.make_case("stack8_6823tok_60u", lengths=lengths, seed=2 + 1000 * rank, dtype="bf16",
+                        num_layers=8, with_head=True)
+    else:
+        c = S.make_case("layer_6823tok_60u", lengths=lengths, seed=1 + 1000 * rank, dtype="bf16",
+                        gate_std=0.1)
+    return c
+
+
+def attention_flops(lengths):
+    L = np.asarray(lengths, np.int64)
+    return 2048 * int((L * (L + 1) // 2).sum())
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_id)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        mhz, maxm, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxm = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": maxm, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- oracle
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = [i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def time_oracle_layers(case, budget_s=12.0, max_reps=8, min_reps=1, layer_offset=0):
+    """Time the oracle's full-batch layer forward (layers of the case in turn);
+    returns (seconds per layer, reps)."""
+    from oracle import ptl_oracle as O
+    times = []
+    h = case.x
+    t_all = time.perf_counter()
+    i = 0
+    while i < max_reps and (i < min_reps or time.perf_counter() - t_all < budget_s):
+        w = case.layers[(layer_offset + i) % len(case.layers)]
+        t0 = time.perf_counter()
+        O.layer_forward(h, case.cu_seqlens, w)
+        times.append(time.perf_counter() - t0)
+        i += 1
+    return statistics.mean(times), len(times)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    case = make_workload(args.workload, 0)
+    T = case.total_tokens
+    # warm-up and timed steps: one oracle layer over the full batch each
+    for i in range(args.warmup):
+        time_oracle_layers(case, max_reps=1, layer_offset=i)
+    secs = []
+    for i in range(args.steps):
+        s, _ = time_oracle_layers(case, max_reps=1, layer_offset=i)
+        secs.append(s)
+    sec = statistics.mean(secs)
+    value = T / sec
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": case.name + (" (one layer per step)" if args.workload == "stack8" else ""),
+                   "tokens": T, "users": case.num_users, "layers_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"numpy fp64 oracle, one full-batch layer ({T} tokens) per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from packed_sequence_transformer_b200 import ptl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ptl.lib()  # no library, no benchmark
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    case = make_workload(args.workload, rank)
+    T, U = case.total_tokens, case.num_users
+    n_layers = len(case.layers)
+    layers = [ptl.to_device_layer(w, "bf16", dev) for w in case.layers]
+    head = ptl.to_device_head(case.head, dev) if case.head is not None else None
+    x = torch.as_tensor(case.x).to(dev, torch.bfloat16).contiguous()
+    cu = torch.as_tensor(case.cu_seqlens).to(dev, torch.int32)
+    mask = torch.as_tensor(case.pred_mask).to(dev, torch.uint8) if head is not None else None
+    out = torch.empty_like(x)
+    probs = torch.empty(T, dtype=torch.float32, device=dev) if head is not None else None
+    n_pred = torch.zeros(1, dtype=torch.int32, device=dev) if head is not None else None
+    ws = ptl.alloc_workspace(T, U, "bf16", dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MiB > L2
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        if head is not None:
+            ptl.stack_forward(x, out, cu, layers, ws, head=head, pred_mask=mask, probs=probs,
+                              n_pred=n_pred)
+        else:
+            ptl.layer_forward(x, out, cu, layers[0], ws)
+
+    # eager warm-up (configures kernels), error check, then graph capture
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    st = ptl.last_device_error(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device error {ptl.STATUS.get(st)}")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = 1 + 8 * n_layers + (2 if head is not None else 0)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            graph.replay()
+            flush.fill_(1.0)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K graph replays, L2 flushed between them
+    gpu_index = torch.cuda.current_device()
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = str(gpu_index)
+    clocks = ClockSampler(uuid)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            evs[i][0].record(stream)
+            graph.replay()
+            evs[i][1].record(stream)
+            flush.fill_(float(i))
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = statistics.mean(step_ms)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens_layers = T * n_layers * world
+    value = tokens_layers / (ms_max / 1e3)
+
+    # ---- per-kernel device times (eager, traced; L2 flushed between steps)
+    trace_steps = min(args.steps, 10)
+    kt = ptl.KernelTrace(capacity=trace_steps * (launches_per_step + 8) + 16)
+    with torch.cuda.stream(stream):
+        with kt:
+            for i in range(trace_steps):
+                step()
+                flush.fill_(float(i))
+    per_kind = {}
+    for kind, t_ms in kt.launches():
+        d = per_kind.setdefault(kind, [0.0, 0])
+        d[0] += t_ms
+        d[1] += 1
+    kinds = {k: {"launches_per_step": v[1] / trace_steps, "avg_us": 1e3 * v[0] / v[1],
+                 "share": 0.0} for k, v in per_kind.items()}
+    tot = sum(v[0] for v in per_kind.values())
+    for k, v in per_kind.items():
+        kinds[k]["share"] = v[0] / tot if tot else 0.0
+
+    peaks, peak_src = load_peaks()
+    lengths = case.lengths
+    attn_fl = attention_flops(lengths)
+    alg = {
+        "gemm_qkv": ("tensor", 2 * T * 512 * 1536),
+        "attention": ("tensor", attn_fl),
+        "gemm_out": ("tensor", 2 * T * 512 * 512),
+        "gemm_expert1": ("tensor", 2 * (2 * T) * 512 * 1024),
+        "gemm_expert2_combine": ("tensor", 2 * (2 * T) * 1024 * 512),
+        "gate": ("hbm", T * (1024 + 1024 + 16)),
+        "layernorm": ("hbm", T * 2048),
+        "route": ("hbm", T * 24),
+    }
+    dom = max((k for k in kinds if k in alg), key=lambda k: kinds[k]["avg_us"] * kinds[k]["launches_per_step"])
+    bound, work = alg[dom]
+    t_s = kinds[dom]["avg_us"] / 1e6
+    if bound == "tensor":
+        achieved = work / t_s / 1e12
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        unit = "TFLOP/s"
+    else:
+        achieved = work / t_s / 1e9
+        peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        unit = "GB/s"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": None, "kernel": dom,
+                "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs'})",
+                "algorithmic_per_launch": work}
+    step_flops = n_layers * (GEMM_FLOPS_PER_TOKEN * T + attn_fl)
+    whole_step_tflops = step_flops / (ms_max / 1e3) / 1e12
+
+    # ---- end to end through the public API: host (pinned) inputs in, result out
+    x_h = torch.as_tensor(case.x).to(torch.bfloat16).pin_memory()
+    cu_h = torch.as_tensor(case.cu_seqlens).to(torch.int32).pin_memory()
+    mask_h = torch.as_tensor(case.pred_mask).to(torch.uint8).pin_memory() if head is not None else None
+    res_h = (torch.empty(T, dtype=torch.float32).pin_memory() if head is not None
+             else torch.empty(T, 512, dtype=torch.bfloat16).pin_memory())
+    n_h = torch.zeros(1, dtype=torch.int32).pin_memory()
+    h2d = x_h.numel() * 2 + cu_h.numel() * 4 + (mask_h.numel() if mask_h is not None else 0)
+    d2h = res_h.numel() * res_h.element_size() + (4 if head is not None else 0)
+    e2e_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup + args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            x.copy_(x_h, non_blocking=True)
+            cu.copy_(cu_h, non_blocking=True)
+            if mask is not None:
+                mask.copy_(mask_h, non_blocking=True)
+            graph.replay()
+            if head is not None:
+                res_h.copy_(probs, non_blocking=True)
+                n_h.copy_(n_pred, non_blocking=True)
+            else:
+                res_h.copy_(out, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            if i >= args.warmup:
+                e2e_ms.append(a.elapsed_time(b))
+            flush.fill_(float(i))
+    e2e = statistics.mean(e2e_ms)
+    e2e_t = torch.tensor([e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens_layers / (float(e2e_t.item()) / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        sec, reps = time_oracle_layers(case, budget_s=15.0, max_reps=6, min_reps=2)
+        cpu = {"value": T / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"numpy fp64 oracle, {reps} full-batch layers of this workload ({T} tokens each)"}
+
+    graph.reset()
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; lognormal user lengths, random-init weights)",
+            "config": {"workload": case.name, "tokens": T, "users": U, "layers": n_layers,
+                       "head": head is not None, "parallelism": f"dp{world} (independent batches)",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "timing": "CUDA graph replay, CUDA events per step"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "detail": {"step_tflops": whole_step_tflops,
+                       "step_frac_of_peak": whole_step_tflops / float(peaks.get("bf16_tflops", 1590.0)),
+                       "us_per_layer": ms_max * 1e3 / n_layers,
+                       "kernels": kinds, "attention_flops_per_layer": attn_fl,
+                       "gemm_flops_per_layer": GEMM_FLOPS_PER_TOKEN * T},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

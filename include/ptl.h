@@ -1,0 +1,239 @@
+/*
+ * ptl.h -- C ABI of the packed-sequence Transformer layer library (libptl.so).
+ *
+ * The library runs the forward pass of a pre-norm encoder layer over many
+ * users' behaviour sequences packed end to end into one jagged token stream,
+ * as described in the "Days-gone/cti2026" README (TransformerEncoder
+ * section):
+ *
+ *     x1  = x  + Linear_out( Attn( LayerNorm1(x) Wqkv^T + b_qkv, user_offsets ) )
+ *     out = x1 + FusedMoE( LayerNorm2(x1), Gate(LayerNorm2(x1)) )
+ *
+ * Attention is block-diagonal causal: token i of a user attends to that
+ * user's tokens 0..i only (README, FlashAttention_Varlen operator design).
+ * The gate is Linear(512->8) followed by softmax, top-2 and renormalisation
+ * (README, SMoE structure); each token's two experts Linear(512->1024) +
+ * ReLU + Linear(1024->512) are combined with the renormalised weights
+ * (README, fused MoE routing and weighted sum).  The prediction head is a
+ * final LayerNorm, Linear(512->1), clamp to [-15, 15] and sigmoid on the
+ * tokens whose pred_mask is set (README, Prediction Head section).
+ *
+ * Layer shape is fixed: d_model 512, 8 heads x 64, QKV 512->1536, gate
+ * 512->8, 8 experts 512->1024->512, top-2.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise,
+ *     row-major, and must be 16-byte aligned (PTL_ERR_ALIGN otherwise).
+ *     Weight matrices use the nn.Linear layout W[out][in].
+ *   - Activations and the big matrices (w_qkv, w_o, w1, w2) are stored in
+ *     the build dtype `dt`: PTL_BF16 (bfloat16 storage, fp32 accumulation)
+ *     or PTL_F32 (fp32 storage and arithmetic).  LayerNorm parameters, the
+ *     gate weight and every bias are float32 in both builds.  Bias pointers
+ *     may be NULL (treated as zero); LayerNorm gamma/beta may not.
+ *   - cu_seqlens (user_offsets) is int32 [num_users + 1] with cu[0] = 0,
+ *     non-decreasing, cu[num_users] = total_tokens.  Zero-length users are
+ *     allowed anywhere and produce nothing.  These properties are checked on
+ *     the device; a violation sets the workspace error word to
+ *     PTL_ERR_BAD_OFFSETS, later kernels of the call skip their work, the
+ *     outputs are undefined, and ptl_last_device_error() reports it.
+ *   - The caller owns every buffer.  The library allocates nothing inside
+ *     the forward calls, never synchronises `stream` and keeps no state
+ *     between calls, so a sequence of calls can be captured into a CUDA
+ *     graph (TMA descriptors are built on the host at call time and passed
+ *     by value, so a captured graph keeps the buffers it was captured on).
+ *     `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *   - workspace: a device buffer of at least ptl_workspace_size(T, U, dt)
+ *     bytes, 256-byte aligned, used only by the calls that receive it.  Two
+ *     calls that run concurrently must not share a workspace.
+ *   - Host-checkable problems (NULL pointers, misalignment, sizes, a too
+ *     small workspace, an unknown dtype) return a status immediately and
+ *     launch nothing.  total_tokens == 0 returns PTL_OK with no launches.
+ *     No entry point traps, prints or throws across the ABI.
+ */
+#ifndef PTL_H
+#define PTL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PTL_D_MODEL 512
+#define PTL_N_HEADS 8
+#define PTL_D_HEAD 64
+#define PTL_D_FF 1024
+#define PTL_N_EXPERTS 8
+#define PTL_TOP_K 2
+
+typedef enum {
+  PTL_OK = 0,
+  PTL_ERR_NULL = 1,        /* a required pointer is NULL */
+  PTL_ERR_ALIGN = 2,       /* a pointer is not 16-byte aligned (workspace: 256) */
+  PTL_ERR_SHAPE = 3,       /* num_users < 1, total_tokens < 0 or >= 2^31, num_layers < 1 */
+  PTL_ERR_BAD_OFFSETS = 4, /* cu_seqlens not 0-based, not monotone, or not ending at T */
+  PTL_ERR_WORKSPACE = 5,   /* workspace smaller than ptl_workspace_size() */
+  PTL_ERR_DTYPE = 6,       /* unknown ptl_dtype */
+  PTL_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed */
+  PTL_ERR_TIMEOUT = 8,     /* a bounded device-side wait ran out (kernel returned early) */
+  PTL_ERR_UNSUPPORTED = 9  /* no sm_100 device, or a feature not built */
+} ptl_status;
+
+typedef enum { PTL_F32 = 0, PTL_BF16 = 1 } ptl_dtype;
+
+/* One layer's parameters (device pointers). */
+typedef struct {
+  const void* ln1_g;  /* [512] f32 */
+  const void* ln1_b;  /* [512] f32 */
+  const void* w_qkv;  /* [1536][512] dt; rows 0-511 Q, 512-1023 K, 1024-1535 V; head h = rows 64h..64h+63 of each */
+  const void* b_qkv;  /* [1536] f32 or NULL */
+  const void* w_o;    /* [512][512] dt */
+  const void* b_o;    /* [512] f32 or NULL */
+  const void* ln2_g;  /* [512] f32 */
+  const void* ln2_b;  /* [512] f32 */
+  const void* w_gate; /* [8][512] f32 */
+  const void* b_gate; /* [8] f32 or NULL */
+  const void* w1;     /* [8][1024][512] dt */
+  const void* b1;     /* [8][1024] f32 or NULL */
+  const void* w2;     /* [8][512][1024] dt */
+  const void* b2;     /* [8][512] f32 or NULL */
+} ptl_layer_weights;
+
+/* Prediction head parameters (device pointers, all f32). */
+typedef struct {
+  const void* lnf_g; /* [512] */
+  const void* lnf_b; /* [512] */
+  const void* w;     /* [512] */
+  const void* b;     /* [1] or NULL */
+} ptl_head_weights;
+
+/* Optional debug outputs of ptl_layer_forward (device pointers; any may be NULL). */
+typedef struct {
+  int32_t* topk_idx;   /* [T][2] chosen experts, slot 0 = larger probability */
+  float* topk_w;       /* [T][2] renormalised weights */
+  int32_t* perm;       /* [2T] routes r = 2t+k sorted by expert, ascending r within an expert */
+  int32_t* expert_off; /* [9] exclusive prefix of routes per expert */
+} ptl_debug_out;
+
+/* Bytes of workspace needed for calls with up to max_tokens tokens and
+ * max_users users in build dtype dt (0 for invalid arguments). */
+size_t ptl_workspace_size(int64_t max_tokens, int32_t max_users, ptl_dtype dt);
+
+/* One encoder layer: out[T][512] = layer(x[T][512]).  x and out may not
+ * alias.  dbg may be NULL. */
+ptl_status ptl_layer_forward(const void* x, void* out, const int32_t* cu_seqlens,
+                             int32_t num_users, int64_t total_tokens, ptl_dtype dt,
+                             const ptl_layer_weights* w, void* workspace, size_t ws_bytes,
+                             const ptl_debug_out* dbg, void* stream);
+
+/* num_layers layers in sequence (layers: HOST array of num_layers structs
+ * holding device pointers), then, when head != NULL, the prediction head:
+ * probs[0 .. n_pred-1] = sigmoid(clamp(LN_f(h) w + b)) for the tokens with
+ * pred_mask[t] != 0 in ascending t; *n_pred (device int32) receives the
+ * count.  out[T][512] always receives the final hidden state.  With head ==
+ * NULL, pred_mask/probs/n_pred are ignored.  x and out may not alias. */
+ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens,
+                             int32_t num_users, int64_t total_tokens, int32_t num_layers,
+                             ptl_dtype dt, const ptl_layer_weights* layers,
+                             const ptl_head_weights* head, const uint8_t* pred_mask,
+                             float* probs, int32_t* n_pred, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* ---- The layer's steps, one entry point each (the pages' operator
+ * interface: Linear_qkv, FlashAttention_Varlen(qkv, user_offsets),
+ * Linear_out + residual, Gate(x) -> (topk_idx, topk_weight),
+ * FusedMoE(x, topk_idx, topk_weight) + residual, Prediction Head). ---- */
+
+/* qkv[T][1536] = LayerNorm1(x) Wqkv^T + b_qkv (uses ln1_g, ln1_b, w_qkv, b_qkv of w). */
+ptl_status ptl_qkv_projection(const void* x, void* qkv, int64_t total_tokens, ptl_dtype dt,
+                              const ptl_layer_weights* w, void* workspace, size_t ws_bytes,
+                              void* stream);
+
+/* attn[T][512] = block-diagonal causal softmax(Q K^T / 8) V per user and head,
+ * Q/K/V read from qkv[T][1536] as [Q|K|V]. */
+ptl_status ptl_attention(const void* qkv, void* attn, const int32_t* cu_seqlens,
+                         int32_t num_users, int64_t total_tokens, ptl_dtype dt,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/* x1[T][512] = x + attn Wo^T + b_o. */
+ptl_status ptl_out_projection(const void* attn, const void* x, void* x1, int64_t total_tokens,
+                              ptl_dtype dt, const ptl_layer_weights* w, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* xn2[T][512] = LayerNorm2(x1) (dt); p = softmax(xn2 Wg^T + bg) in fp32;
+ * topk_idx[T][2] (int32) = the two largest p (ties to the lower expert
+ * index, slot 0 the larger), topk_w[T][2] (f32) = p / (p0 + p1). */
+ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w,
+                    int64_t total_tokens, ptl_dtype dt, const ptl_layer_weights* w,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* Counting sort of the 2T routes r = 2t+k by topk_idx: expert_off[9] is the
+ * exclusive prefix of the per-expert counts and perm[2T] lists the routes of
+ * expert 0, then expert 1, ..., each in ascending r.  Either output may be
+ * NULL.  topk_idx values must be in [0, 8). */
+ptl_status ptl_route_build(const int32_t* topk_idx, int64_t total_tokens, int32_t* perm,
+                           int32_t* expert_off, void* workspace, size_t ws_bytes, void* stream);
+
+/* out[t] = residual[t] + topk_w[t][0] y(t, topk_idx[t][0]) + topk_w[t][1] y(t, topk_idx[t][1]),
+ * y(t, e) = ReLU(xn2[t] W1[e]^T + b1[e]) W2[e]^T + b2[e]  (uses w1, b1, w2, b2 of w).
+ * The k = 0 term is added first, in fp32, and rounded once. */
+ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w,
+                   const void* residual, void* out, int64_t total_tokens, ptl_dtype dt,
+                   const ptl_layer_weights* w, void* workspace, size_t ws_bytes, void* stream);
+
+/* Prediction head on h[T][512] (dt), see ptl_stack_forward. */
+ptl_status ptl_head(const void* h, const ptl_head_weights* head, const uint8_t* pred_mask,
+                    float* probs, int32_t* n_pred, int64_t total_tokens, ptl_dtype dt,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- Per-kernel tracing (for profiling; off by default). ----
+ * While a trace is installed on the calling host thread, every entry point
+ * records events[count] on its stream just before each kernel (or memset)
+ * it enqueues, stores that launch's kind in kinds[count] and increments
+ * count; after its last launch it records one more event with kind
+ * PTL_KERNEL_END.  The time of launch i is the elapsed time between
+ * events[i] and events[i + 1].  events are cudaEvent_t handles created by
+ * the caller (with timing enabled); kinds is a host array.  Recording stops
+ * silently when count reaches capacity.  The trace is owned by the caller
+ * and must outlive the calls it observes; pass NULL to remove it. */
+typedef enum {
+  PTL_KERNEL_CLEAR = 0,        /* error-word / counter memsets */
+  PTL_KERNEL_WORKLIST = 1,     /* cu_seqlens validation + attention work list */
+  PTL_KERNEL_LAYERNORM = 2,    /* LayerNorm1 */
+  PTL_KERNEL_GEMM_QKV = 3,     /* QKV projection */
+  PTL_KERNEL_ATTENTION = 4,    /* jagged causal attention */
+  PTL_KERNEL_GEMM_OUT = 5,     /* output projection + residual */
+  PTL_KERNEL_GATE = 6,         /* LayerNorm2 + gate + top-2 */
+  PTL_KERNEL_ROUTE = 7,        /* route counting sort (and per-chunk counts) */
+  PTL_KERNEL_GEMM_EXPERT1 = 8, /* expert GEMM1 + ReLU (gathered rows) */
+  PTL_KERNEL_GEMM_EXPERT2 = 9, /* expert GEMM2 + top-2 combine + residual */
+  PTL_KERNEL_HEAD = 10,        /* prediction head + compaction */
+  PTL_KERNEL_COPY = 11,        /* debug-output copies */
+  PTL_KERNEL_END = 99
+} ptl_kernel_kind;
+
+typedef struct {
+  void** events;    /* cudaEvent_t[capacity] */
+  int32_t* kinds;   /* host [capacity] */
+  int32_t capacity;
+  int32_t count;
+} ptl_trace;
+
+/* Installs (or, with NULL, removes) the calling thread's trace. */
+void ptl_set_trace(ptl_trace* trace);
+
+/* Synchronises `stream`, returns the status recorded in the workspace error
+ * word by earlier calls on that workspace (PTL_OK if none) and clears it. */
+ptl_status ptl_last_device_error(void* workspace, size_t ws_bytes, void* stream);
+
+/* Static text for a status code. */
+const char* ptl_status_string(ptl_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t ptl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PTL_H */

@@ -1,0 +1,485 @@
+// api.cu -- the C ABI of libptl: argument validation, workspace carving,
+// TMA descriptor encoding and the launch sequence of the layer, the stack
+// and the individual steps.  No allocation, no stream synchronisation (except
+// in ptl_last_device_error), no state kept between calls.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/ptl.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+using namespace ptl;
+
+// ------------------------------------------------------------ driver entry
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor map: `rows` rows of `cols` elements, `stride_bytes` apart;
+// box = box_rows x box_cols (box_cols * 2 bytes = 128, the swizzle span).
+bool map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride_bytes,
+              uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+ptl_status device_ok() {
+  static int cache[64];  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PTL_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev] == 1 ? PTL_OK : PTL_ERR_UNSUPPORTED;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return PTL_ERR_CUDA;
+  const int ok = major == 10 ? 1 : 2;
+  if (dev >= 0 && dev < 64) cache[dev] = ok;
+  return ok == 1 ? PTL_OK : PTL_ERR_UNSUPPORTED;
+}
+
+inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool a4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+inline bool opt16(const void* p) { return p == nullptr || a16(p); }
+
+ptl_status check_common(int64_t T, ptl_dtype dt, void* ws, size_t ws_bytes, int32_t U, WsLayout* L) {
+  if (dt != PTL_F32 && dt != PTL_BF16) return PTL_ERR_DTYPE;
+  if (T < 0 || T >= (int64_t(1) << 31) || U < 1) return PTL_ERR_SHAPE;
+  if (!ws) return PTL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return PTL_ERR_ALIGN;
+  if (!make_layout(T, U, dt, L)) return PTL_ERR_SHAPE;
+  if (ws_bytes < L->total) return PTL_ERR_WORKSPACE;
+  return PTL_OK;
+}
+
+ptl_status check_weights(const ptl_layer_weights* w) {
+  if (!w) return PTL_ERR_NULL;
+  const void* req[] = {w->ln1_g, w->ln1_b, w->w_qkv, w->w_o, w->ln2_g, w->ln2_b, w->w_gate, w->w1, w->w2};
+  for (const void* p : req) {
+    if (!p) return PTL_ERR_NULL;
+    if (!a16(p)) return PTL_ERR_ALIGN;
+  }
+  const void* opt[] = {w->b_qkv, w->b_o, w->b_gate, w->b1, w->b2};
+  for (const void* p : opt)
+    if (!opt16(p)) return PTL_ERR_ALIGN;
+  return PTL_OK;
+}
+
+ptl_status check_head(const ptl_head_weights* h) {
+  if (!h->lnf_g || !h->lnf_b || !h->w) return PTL_ERR_NULL;
+  if (!a16(h->lnf_g) || !a16(h->lnf_b) || !a16(h->w) || !opt16(h->b)) return PTL_ERR_ALIGN;
+  return PTL_OK;
+}
+
+thread_local ptl_trace* g_trace = nullptr;
+
+// Records the trace event that opens a launch of `kind` (no-op without a trace).
+inline void mark(cudaStream_t st, int kind) {
+  ptl_trace* t = g_trace;
+  if (!t || !t->events || t->count >= t->capacity) return;
+  cudaEventRecord(static_cast<cudaEvent_t>(t->events[t->count]), st);
+  if (t->kinds) t->kinds[t->count] = kind;
+  ++t->count;
+}
+
+// Records the closing PTL_KERNEL_END event when an entry point returns.
+struct EndMark {
+  cudaStream_t st;
+  ~EndMark() { mark(st, PTL_KERNEL_END); }
+};
+
+struct Call {
+  WsLayout L;
+  char* ws;
+  int32_t* err;
+  cudaStream_t st;
+  ptl_dtype dt;
+  int T;
+  int U;
+};
+
+inline const float* F32(const void* p) { return static_cast<const float*>(p); }
+template <typename T>
+inline T* at(const Call& c, size_t off) { return reinterpret_cast<T*>(c.ws + off); }
+
+#define PTL_TRY(expr)                 \
+  do {                                \
+    if ((expr) != 0) return PTL_ERR_CUDA; \
+  } while (0)
+
+// Clears the error word: every top-level call reports only its own errors.
+ptl_status begin(const Call& c) {
+  mark(c.st, PTL_KERNEL_CLEAR);
+  return cudaMemsetAsync(c.err, 0, sizeof(int32_t), c.st) == cudaSuccess ? PTL_OK : PTL_ERR_CUDA;
+}
+
+ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_weights* w) {
+  const int T = c.T;
+  if (c.dt == PTL_BF16) {
+    mark(c.st, PTL_KERNEL_LAYERNORM);
+    PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));
+    CUtensorMap ma, mb;
+    if (!map_bf16(&ma, c.ws + c.L.xn, D, T, D * 2, 64, 128)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mb, w->w_qkv, D, QKV_N, D * 2, 64, QKV_BN)) return PTL_ERR_CUDA;
+    mark(c.st, PTL_KERNEL_GEMM_QKV);
+    PTL_TRY(launch_gemm_qkv(ma, mb, F32(w->b_qkv), qkv, T, c.err, c.st));
+  } else {
+    mark(c.st, PTL_KERNEL_LAYERNORM);
+    PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));
+    mark(c.st, PTL_KERNEL_GEMM_QKV);
+    PTL_TRY(launch_gemm_f32(0, at<float>(c, c.L.xn), D, F32(w->w_qkv), F32(w->b_qkv), nullptr,
+                            static_cast<float*>(qkv), QKV_N, T, QKV_N, D, c.L, c.ws, c.st));
+  }
+  return PTL_OK;
+}
+
+ptl_status step_attention(const Call& c, const void* qkv, void* attn, const int32_t* cu) {
+  if (c.dt == PTL_BF16) {
+    CUtensorMap m;
+    if (!map_bf16(&m, qkv, QKV_N, c.T, QKV_N * 2, 64, 128)) return PTL_ERR_CUDA;
+    mark(c.st, PTL_KERNEL_ATTENTION);
+    PTL_TRY(launch_attn_tc(m, attn, cu, c.L, c.ws, c.st));
+  } else {
+    mark(c.st, PTL_KERNEL_ATTENTION);
+    PTL_TRY(launch_attn_f32(static_cast<const float*>(qkv), static_cast<float*>(attn), cu, c.L, c.ws,
+                            c.st));
+  }
+  return PTL_OK;
+}
+
+ptl_status step_out(const Call& c, const void* attn, const void* x, void* x1, const ptl_layer_weights* w) {
+  if (c.dt == PTL_BF16) {
+    CUtensorMap ma, mb;
+    if (!map_bf16(&ma, attn, D, c.T, D * 2, 64, 128)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mb, w->w_o, D, D, D * 2, 64, OUT_BN)) return PTL_ERR_CUDA;
+    mark(c.st, PTL_KERNEL_GEMM_OUT);
+    PTL_TRY(launch_gemm_out(ma, mb, F32(w->b_o), x, x1, c.T, c.err, c.st));
+  } else {
+    mark(c.st, PTL_KERNEL_GEMM_OUT);
+    PTL_TRY(launch_gemm_f32(1, static_cast<const float*>(attn), D, F32(w->w_o), F32(w->b_o),
+                            static_cast<const float*>(x), static_cast<float*>(x1), D, c.T, D, D, c.L,
+                            c.ws, c.st));
+  }
+  return PTL_OK;
+}
+
+ptl_status step_gate(const Call& c, const void* x1, void* xn2, int32_t* idx, float* wout,
+                     const ptl_layer_weights* w) {
+  mark(c.st, PTL_KERNEL_GATE);
+  PTL_TRY(launch_gate(x1, F32(w->ln2_g), F32(w->ln2_b), F32(w->w_gate), F32(w->b_gate), xn2, idx, wout,
+                      at<int32_t>(c, c.L.chunk_cnt), at<int32_t>(c, c.L.comb_cnt), c.T, c.dt, c.st));
+  return PTL_OK;
+}
+
+// Routes + both expert GEMMs + combine + residual.  chunk counts and the
+// cleared combine counters must already be in the workspace.
+ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const float* wts,
+                    const void* resid, void* out, const ptl_layer_weights* w, int32_t* dbg_perm,
+                    int32_t* dbg_off) {
+  mark(c.st, PTL_KERNEL_ROUTE);
+  PTL_TRY(launch_route(idx, c.T, c.L, c.ws, dbg_perm, dbg_off, c.st));
+  if (c.dt == PTL_BF16) {
+    CUtensorMap m1, m2, mh;
+    if (!map_bf16(&m1, w->w1, D, uint64_t(E) * F, D * 2, 64, MOE1_BN)) return PTL_ERR_CUDA;
+    if (!map_bf16(&m2, w->w2, F, uint64_t(E) * D, F * 2, 64, GEMM2_BN)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mh, c.ws + c.L.hbuf, F, c.L.padded_rows, F * 2, 64, 128)) return PTL_ERR_CUDA;
+    mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
+    PTL_TRY(launch_gemm_moe1(m1, m1, F32(w->b1), xn2, c.L, c.ws, c.st));
+    mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
+    PTL_TRY(launch_gemm_moe2(mh, m2, F32(w->b2), resid, wts, out, c.L, c.ws, c.st));
+  } else {
+    mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
+    PTL_TRY(launch_gemm_f32(2, static_cast<const float*>(xn2), D, F32(w->w1), F32(w->b1), nullptr,
+                            at<float>(c, c.L.hbuf), F, 0, F, D, c.L, c.ws, c.st));
+    mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
+    PTL_TRY(launch_gemm_f32(3, at<float>(c, c.L.hbuf), F, F32(w->w2), F32(w->b2), nullptr,
+                            at<float>(c, c.L.ystage), D, 0, D, F, c.L, c.ws, c.st));
+    PTL_TRY(launch_combine_f32(at<float>(c, c.L.ystage), wts, static_cast<const float*>(resid),
+                               static_cast<float*>(out), c.T, c.err, c.st));
+  }
+  return PTL_OK;
+}
+
+ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu,
+                      const ptl_layer_weights* w, const ptl_debug_out* dbg) {
+  ptl_status s;
+  if ((s = step_qkv(c, x, c.ws + c.L.qkv, w)) != PTL_OK) return s;
+  if ((s = step_attention(c, c.ws + c.L.qkv, c.ws + c.L.attn, cu)) != PTL_OK) return s;
+  if ((s = step_out(c, c.ws + c.L.attn, x, c.ws + c.L.x1, w)) != PTL_OK) return s;
+  int32_t* idx = at<int32_t>(c, c.L.idx);
+  float* wts = at<float>(c, c.L.wgt);
+  if ((s = step_gate(c, c.ws + c.L.x1, c.ws + c.L.xn2, idx, wts, w)) != PTL_OK) return s;
+  if ((s = step_moe(c, c.ws + c.L.xn2, idx, wts, c.ws + c.L.x1, out, w, dbg ? dbg->perm : nullptr,
+                    dbg ? dbg->expert_off : nullptr)) != PTL_OK)
+    return s;
+  if (dbg && (dbg->topk_idx || dbg->topk_w)) mark(c.st, PTL_KERNEL_COPY);
+  if (dbg && dbg->topk_idx &&
+      cudaMemcpyAsync(dbg->topk_idx, idx, sizeof(int32_t) * 2 * c.T, cudaMemcpyDeviceToDevice, c.st) !=
+          cudaSuccess)
+    return PTL_ERR_CUDA;
+  if (dbg && dbg->topk_w &&
+      cudaMemcpyAsync(dbg->topk_w, wts, sizeof(float) * 2 * c.T, cudaMemcpyDeviceToDevice, c.st) !=
+          cudaSuccess)
+    return PTL_ERR_CUDA;
+  return PTL_OK;
+}
+
+ptl_status setup(Call* c, int64_t T, int32_t U, ptl_dtype dt, void* ws, size_t ws_bytes, void* stream) {
+  ptl_status s = check_common(T, dt, ws, ws_bytes, U, &c->L);
+  if (s != PTL_OK) return s;
+  c->ws = static_cast<char*>(ws);
+  c->err = reinterpret_cast<int32_t*>(c->ws + c->L.err);
+  c->st = static_cast<cudaStream_t>(stream);
+  c->dt = dt;
+  c->T = int(T);
+  c->U = U;
+  return PTL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t ptl_version(void) { return 100; }
+
+void ptl_set_trace(ptl_trace* trace) { g_trace = trace; }
+
+const char* ptl_status_string(ptl_status s) {
+  switch (s) {
+    case PTL_OK: return "ok";
+    case PTL_ERR_NULL: return "a required pointer is NULL";
+    case PTL_ERR_ALIGN: return "a pointer is not aligned (16 bytes; workspace 256 bytes)";
+    case PTL_ERR_SHAPE: return "invalid size or index (num_users < 1, total_tokens out of [0, 2^31), expert id out of range)";
+    case PTL_ERR_BAD_OFFSETS: return "cu_seqlens is not 0-based, non-decreasing and ending at total_tokens";
+    case PTL_ERR_WORKSPACE: return "workspace smaller than ptl_workspace_size()";
+    case PTL_ERR_DTYPE: return "unknown dtype";
+    case PTL_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case PTL_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case PTL_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
+  }
+  return "unknown status";
+}
+
+size_t ptl_workspace_size(int64_t max_tokens, int32_t max_users, ptl_dtype dt) {
+  WsLayout L;
+  if (!make_layout(max_tokens, max_users, dt, &L)) return 0;
+  return L.total;
+}
+
+ptl_status ptl_layer_forward(const void* x, void* out, const int32_t* cu_seqlens, int32_t num_users,
+                             int64_t total_tokens, ptl_dtype dt, const ptl_layer_weights* w,
+                             void* workspace, size_t ws_bytes, const ptl_debug_out* dbg, void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!x || !out || !cu_seqlens) return PTL_ERR_NULL;
+  if (!a16(x) || !a16(out) || !a4(cu_seqlens)) return PTL_ERR_ALIGN;
+  if ((s = check_weights(w)) != PTL_OK) return s;
+  if (x == out) return PTL_ERR_SHAPE;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_WORKLIST);
+  PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
+  return layer_body(c, x, out, cu_seqlens, w, dbg);
+}
+
+ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens, int32_t num_users,
+                             int64_t total_tokens, int32_t num_layers, ptl_dtype dt,
+                             const ptl_layer_weights* layers, const ptl_head_weights* head,
+                             const uint8_t* pred_mask, float* probs, int32_t* n_pred, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (num_layers < 1) return PTL_ERR_SHAPE;
+  if (!x || !out || !cu_seqlens || !layers) return PTL_ERR_NULL;
+  if (!a16(x) || !a16(out) || !a4(cu_seqlens)) return PTL_ERR_ALIGN;
+  if (x == out) return PTL_ERR_SHAPE;
+  for (int i = 0; i < num_layers; ++i)
+    if ((s = check_weights(&layers[i])) != PTL_OK) return s;
+  if (head) {
+    if ((s = check_head(head)) != PTL_OK) return s;
+    if (!pred_mask || !probs) return PTL_ERR_NULL;
+    if (!a4(probs) || (n_pred && !a4(n_pred))) return PTL_ERR_ALIGN;
+  }
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_WORKLIST);
+  PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
+  const void* h_in = x;
+  for (int i = 0; i < num_layers; ++i) {
+    void* h_out = (i == num_layers - 1) ? out : c.ws + ((i & 1) ? c.L.act1 : c.L.act0);
+    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr)) != PTL_OK) return s;
+    h_in = h_out;
+  }
+  if (head) mark(c.st, PTL_KERNEL_HEAD);
+  if (head) PTL_TRY(launch_head(out, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st));
+  return PTL_OK;
+}
+
+ptl_status ptl_qkv_projection(const void* x, void* qkv, int64_t total_tokens, ptl_dtype dt,
+                              const ptl_layer_weights* w, void* workspace, size_t ws_bytes, void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!x || !qkv || !w || !w->ln1_g || !w->ln1_b || !w->w_qkv) return PTL_ERR_NULL;
+  if (!a16(x) || !a16(qkv) || !a16(w->ln1_g) || !a16(w->ln1_b) || !a16(w->w_qkv) || !opt16(w->b_qkv))
+    return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  return step_qkv(c, x, qkv, w);
+}
+
+ptl_status ptl_attention(const void* qkv, void* attn, const int32_t* cu_seqlens, int32_t num_users,
+                         int64_t total_tokens, ptl_dtype dt, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!qkv || !attn || !cu_seqlens) return PTL_ERR_NULL;
+  if (!a16(qkv) || !a16(attn) || !a4(cu_seqlens)) return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_WORKLIST);
+  PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
+  return step_attention(c, qkv, attn, cu_seqlens);
+}
+
+ptl_status ptl_out_projection(const void* attn, const void* x, void* x1, int64_t total_tokens,
+                              ptl_dtype dt, const ptl_layer_weights* w, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!attn || !x || !x1 || !w || !w->w_o) return PTL_ERR_NULL;
+  if (!a16(attn) || !a16(x) || !a16(x1) || !a16(w->w_o) || !opt16(w->b_o)) return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  return step_out(c, attn, x, x1, w);
+}
+
+ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w, int64_t total_tokens,
+                    ptl_dtype dt, const ptl_layer_weights* w, void* workspace, size_t ws_bytes,
+                    void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!x1 || !xn2 || !topk_idx || !topk_w || !w || !w->ln2_g || !w->ln2_b || !w->w_gate)
+    return PTL_ERR_NULL;
+  if (!a16(x1) || !a16(xn2) || !a4(topk_idx) || !a4(topk_w) || !a16(w->ln2_g) || !a16(w->ln2_b) ||
+      !a16(w->w_gate) || !opt16(w->b_gate))
+    return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  return step_gate(c, x1, xn2, topk_idx, topk_w, w);
+}
+
+ptl_status ptl_route_build(const int32_t* topk_idx, int64_t total_tokens, int32_t* perm,
+                           int32_t* expert_off, void* workspace, size_t ws_bytes, void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, 1, PTL_BF16, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!topk_idx) return PTL_ERR_NULL;
+  if (!a4(topk_idx) || (perm && !a4(perm)) || (expert_off && !a4(expert_off))) return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_ROUTE);
+  PTL_TRY(launch_chunk_hist(topk_idx, c.T, at<int32_t>(c, c.L.chunk_cnt), c.err, c.st));
+  PTL_TRY(launch_route(topk_idx, c.T, c.L, c.ws, perm, expert_off, c.st));
+  return PTL_OK;
+}
+
+ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w, const void* residual,
+                   void* out, int64_t total_tokens, ptl_dtype dt, const ptl_layer_weights* w,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!xn2 || !topk_idx || !topk_w || !residual || !out || !w || !w->w1 || !w->w2) return PTL_ERR_NULL;
+  if (!a16(xn2) || !a4(topk_idx) || !a4(topk_w) || !a16(residual) || !a16(out) || !a16(w->w1) ||
+      !a16(w->w2) || !opt16(w->b1) || !opt16(w->b2))
+    return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_ROUTE);
+  PTL_TRY(launch_chunk_hist(topk_idx, c.T, at<int32_t>(c, c.L.chunk_cnt), c.err, c.st));
+  mark(c.st, PTL_KERNEL_CLEAR);
+  if (cudaMemsetAsync(c.ws + c.L.comb_cnt, 0, sizeof(int32_t) * size_t(c.T) * GEMM2_NT, c.st) !=
+      cudaSuccess)
+    return PTL_ERR_CUDA;
+  return step_moe(c, xn2, topk_idx, topk_w, residual, out, w, nullptr, nullptr);
+}
+
+ptl_status ptl_head(const void* h, const ptl_head_weights* head, const uint8_t* pred_mask, float* probs,
+                    int32_t* n_pred, int64_t total_tokens, ptl_dtype dt, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (total_tokens == 0) return PTL_OK;
+  if (!h || !head || !pred_mask || !probs) return PTL_ERR_NULL;
+  if ((s = check_head(head)) != PTL_OK) return s;
+  if (!a16(h) || !a4(probs) || (n_pred && !a4(n_pred))) return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_HEAD);
+  PTL_TRY(launch_head(h, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st));
+  return PTL_OK;
+}
+
+ptl_status ptl_last_device_error(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace) return PTL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PTL_ERR_ALIGN;
+  if (ws_bytes < 256) return PTL_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PTL_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return PTL_ERR_CUDA;
+  if (cudaMemset(workspace, 0, sizeof(v)) != cudaSuccess) return PTL_ERR_CUDA;
+  return static_cast<ptl_status>(v);
+}
+
+}  // extern "C"

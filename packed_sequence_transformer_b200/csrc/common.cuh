@@ -1,0 +1,135 @@
+// common.cuh -- layer constants, workspace layout and small device helpers
+// shared by the kernels of the packed-sequence encoder layer.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/ptl.h"
+
+namespace ptl {
+
+constexpr int D = PTL_D_MODEL;     // 512
+constexpr int H = PTL_N_HEADS;     // 8
+constexpr int DH = PTL_D_HEAD;     // 64
+constexpr int F = PTL_D_FF;        // 1024
+constexpr int E = PTL_N_EXPERTS;   // 8
+constexpr int K = PTL_TOP_K;       // 2
+constexpr int QKV_N = 3 * D;       // 1536
+constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
+constexpr int MOE_BM = 128;        // rows per expert tile (padding granule)
+constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
+constexpr int GEMM2_BN = 256;      // N tile of the second expert GEMM
+constexpr int GEMM2_NT = D / GEMM2_BN;  // combine counters per token
+constexpr float LN_EPS = 1e-5f;
+constexpr float LOGIT_CLAMP = 15.0f;
+
+// Error word values are ptl_status codes; 0 = no error.
+struct WsLayout {
+  size_t err;         // int32 error word
+  size_t items;       // int2 [max_items]   (user, query block) pairs, heaviest first
+  size_t item_count;  // int32
+  size_t lvl_hist;    // int32 [max_levels + 1]
+  size_t lvl_start;   // int32 [max_levels + 1]
+  size_t lvl_fill;    // int32 [max_levels + 1]
+  size_t xn;          // dt [T][512]    LayerNorm1 output
+  size_t qkv;         // dt [T][1536]
+  size_t attn;        // dt [T][512]
+  size_t x1;          // dt [T][512]
+  size_t xn2;         // dt [T][512]
+  size_t act0, act1;  // dt [T][512]    stack ping-pong
+  size_t idx;         // int32 [T][2]
+  size_t wgt;         // f32 [T][2]
+  size_t chunk_cnt;   // int32 [n_chunks][8]
+  size_t perm;        // int32 [2T]
+  size_t rowroute;    // int32 [2T + 8*128]   padded expert rows -> route (or -1)
+  size_t tiles;       // int2 [max_tiles]     (expert, first padded row)
+  size_t route_meta;  // int32 [32]: [0] n_tiles, [1..9] off, [10..18] padded off
+  size_t hbuf;        // dt [2T + 8*128][1024]  expert hidden rows (padded layout)
+  size_t ystage;      // f32 [2T][512]      per-route expert outputs awaiting combine
+  size_t comb_cnt;    // int32 [T][GEMM2_NT] combine arrival counters
+  size_t head_p;      // f32 [T]            head probabilities before compaction
+  size_t total;
+  int64_t T;
+  int32_t U;
+  int64_t max_items, max_levels, n_chunks, max_tiles, padded_rows;
+};
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+__host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L) {
+  if (T < 0 || T >= (int64_t(1) << 31) || U < 1) return false;
+  if (dt != PTL_F32 && dt != PTL_BF16) return false;
+  const size_t es = dt == PTL_BF16 ? 2 : 4;
+  L->T = T;
+  L->U = U;
+  const int64_t nonempty_users = U < T ? U : T;
+  L->max_items = (T + ATT_BLK - 1) / ATT_BLK + nonempty_users + 1;
+  L->max_levels = (T + ATT_BLK - 1) / ATT_BLK + 1;
+  L->n_chunks = (2 * T + ROUTE_CHUNK - 1) / ROUTE_CHUNK + 1;
+  L->max_tiles = (2 * T + MOE_BM - 1) / MOE_BM + E + 1;
+  L->padded_rows = 2 * T + E * MOE_BM;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + (bytes ? bytes : 1), 256);
+    return at;
+  };
+  L->err = take(256);
+  L->items = take(sizeof(int2) * L->max_items);
+  L->item_count = take(4);
+  L->lvl_hist = take(4 * (L->max_levels + 1));
+  L->lvl_start = take(4 * (L->max_levels + 1));
+  L->lvl_fill = take(4 * (L->max_levels + 1));
+  L->xn = take(es * T * D);
+  L->qkv = take(es * T * QKV_N);
+  L->attn = take(es * T * D);
+  L->x1 = take(es * T * D);
+  L->xn2 = take(es * T * D);
+  L->act0 = take(es * T * D);
+  L->act1 = take(es * T * D);
+  L->idx = take(4 * T * K);
+  L->wgt = take(4 * T * K);
+  L->chunk_cnt = take(4 * L->n_chunks * E);
+  L->perm = take(4 * 2 * T);
+  L->rowroute = take(4 * L->padded_rows);
+  L->tiles = take(sizeof(int2) * L->max_tiles);
+  L->route_meta = take(4 * 32);
+  L->hbuf = take(es * L->padded_rows * F);
+  L->ystage = take(4 * 2 * T * D);
+  L->comb_cnt = take(4 * T * GEMM2_NT);
+  L->head_p = take(4 * T);
+  L->total = o;
+  return true;
+}
+
+// ---------------------------------------------------------------- device
+__device__ __forceinline__ void set_error(int32_t* err, int32_t code) {
+  atomicCAS(err, 0, code);
+}
+__device__ __forceinline__ bool has_error(const int32_t* err) {
+  return *reinterpret_cast<const volatile int32_t*>(err) != 0;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace ptl

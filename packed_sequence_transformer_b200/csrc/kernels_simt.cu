@@ -1,0 +1,698 @@
+// kernels_simt.cu -- the bandwidth- and latency-bound steps of the layer
+// (work-list build + offset validation, LayerNorm, gate, route builder,
+// prediction head) and the fp32 build's CUDA-core GEMM / attention /
+// combine.  All of them are warp- or block-level SIMT kernels with 16-byte
+// vector access to rows of 512 elements.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace ptl {
+
+// ------------------------------------------------------------------ rows
+// One warp owns one row of 512 elements; lane l holds 16 of them.  For bf16
+// rows the lane's elements are two 8-element (16-byte) chunks at l*8 and
+// 256+l*8; for fp32 rows four 4-element chunks at l*4 + 128*i.
+template <typename T>
+struct Row16;
+
+template <>
+struct Row16<__nv_bfloat16> {
+  __device__ static __forceinline__ int elem(int lane, int j) { return (j >> 3) * 256 + lane * 8 + (j & 7); }
+  __device__ static __forceinline__ void load(const __nv_bfloat16* row, int lane, float (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint4 u = __ldg(reinterpret_cast<const uint4*>(row + c * 256 + lane * 8));
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        v[c * 8 + 2 * i] = f.x;
+        v[c * 8 + 2 * i + 1] = f.y;
+      }
+    }
+  }
+  __device__ static __forceinline__ void store(__nv_bfloat16* row, int lane, const float (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint4 u;
+      __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(v[c * 8 + 2 * i], v[c * 8 + 2 * i + 1]);
+      *reinterpret_cast<uint4*>(row + c * 256 + lane * 8) = u;
+    }
+  }
+};
+
+template <>
+struct Row16<float> {
+  __device__ static __forceinline__ int elem(int lane, int j) { return (j >> 2) * 128 + lane * 4 + (j & 3); }
+  __device__ static __forceinline__ void load(const float* row, int lane, float (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float4 f = __ldg(reinterpret_cast<const float4*>(row + c * 128 + lane * 4));
+      v[c * 4 + 0] = f.x;
+      v[c * 4 + 1] = f.y;
+      v[c * 4 + 2] = f.z;
+      v[c * 4 + 3] = f.w;
+    }
+  }
+  __device__ static __forceinline__ void store(float* row, int lane, const float (&v)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<float4*>(row + c * 128 + lane * 4) =
+          make_float4(v[c * 4 + 0], v[c * 4 + 1], v[c * 4 + 2], v[c * 4 + 3]);
+  }
+};
+
+// LayerNorm of the lane's 16 values of a 512-element row (two passes over
+// registers: mean, then biased variance of the centred values).
+template <typename T>
+__device__ __forceinline__ void layer_norm16(float (&v)[16], const float* __restrict__ g,
+                                             const float* __restrict__ b, int lane) {
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) s += v[j];
+  const float mean = warp_sum(s) * (1.0f / D);
+  float q = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    v[j] -= mean;
+    q += v[j] * v[j];
+  }
+  const float rstd = rsqrtf(warp_sum(q) * (1.0f / D) + LN_EPS);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int c = Row16<T>::elem(lane, j);
+    v[j] = v[j] * rstd * __ldg(g + c) + __ldg(b + c);
+  }
+}
+
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256) ln_rows_kernel(const TI* __restrict__ x, const float* __restrict__ g,
+                                                      const float* __restrict__ b, TO* __restrict__ y,
+                                                      int T) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= T) return;
+  float v[16];
+  Row16<TI>::load(x + size_t(row) * D, lane, v);
+  layer_norm16<TI>(v, g, b, lane);
+  Row16<TO>::store(y + size_t(row) * D, lane, v);
+}
+
+// ------------------------------------------------------------- work list
+// Validates cu_seqlens and lists the (user, query block) pairs of the
+// jagged attention, heaviest first: a pair (u, b) needs b + 1 key blocks,
+// so pairs are grouped by b in descending order (any order inside a group).
+// One block of 1024 threads.
+__device__ void block_suffix_exclusive(int32_t* a, int n) {
+  // a[i] <- sum_{j > i} a[j] for i in [0, n), done in chunks of blockDim from
+  // the top so that the running carry flows downward.
+  __shared__ int32_t s_scan[1024];
+  __shared__ int32_t s_carry;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = n - 1; base >= 0; base -= blockDim.x) {
+    const int i = base - int(threadIdx.x);
+    const int32_t v = i >= 0 ? a[i] : 0;
+    s_scan[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < int(blockDim.x); o <<= 1) {
+      int32_t t = threadIdx.x >= unsigned(o) ? s_scan[threadIdx.x - o] : 0;
+      __syncthreads();
+      s_scan[threadIdx.x] += t;
+      __syncthreads();
+    }
+    if (i >= 0) a[i] = s_carry + s_scan[threadIdx.x] - v;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) s_carry += s_scan[threadIdx.x];
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restrict__ cu, int U, int T,
+                                                        int2* __restrict__ items, int32_t* item_count,
+                                                        int32_t* lvl_hist, int32_t* lvl_start,
+                                                        int32_t* lvl_fill, int max_levels, int32_t* err) {
+  __shared__ int s_bad;
+  __shared__ int s_total;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_bad = (cu[0] != 0 || cu[U] != T) ? 1 : 0;
+    s_total = 0;
+  }
+  for (int i = tid; i <= max_levels; i += blockDim.x) {
+    lvl_hist[i] = 0;
+    lvl_fill[i] = 0;
+  }
+  __syncthreads();
+  for (int u = tid; u < U; u += blockDim.x)
+    if (cu[u + 1] < cu[u]) s_bad = 1;
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      *item_count = 0;
+      set_error(err, PTL_ERR_BAD_OFFSETS);
+    }
+    return;
+  }
+  int local = 0;
+  for (int u = tid; u < U; u += blockDim.x) {
+    const int nb = (cu[u + 1] - cu[u] + ATT_BLK - 1) / ATT_BLK;
+    if (nb > 0) atomicAdd(&lvl_hist[nb], 1);
+    local += nb;
+  }
+  atomicAdd(&s_total, local);
+  __syncthreads();
+  // lvl_start[b] <- #users with nb > b (pairs at level b) ...
+  for (int i = tid; i <= max_levels; i += blockDim.x) lvl_start[i] = lvl_hist[i];
+  __syncthreads();
+  block_suffix_exclusive(lvl_start, max_levels + 1);
+  // ... then the first slot of level b: sum over the deeper levels b' > b.
+  block_suffix_exclusive(lvl_start, max_levels + 1);
+  for (int u = tid; u < U; u += blockDim.x) {
+    const int nb = (cu[u + 1] - cu[u] + ATT_BLK - 1) / ATT_BLK;
+    for (int b = 0; b < nb; ++b) {
+      const int slot = lvl_start[b] + atomicAdd(&lvl_fill[b], 1);
+      items[slot] = make_int2(u, b);
+    }
+  }
+  if (tid == 0) *item_count = s_total;
+}
+
+// ------------------------------------------------------------------ gate
+// One warp per token: LayerNorm2 of x1, the 8 gate logits in fp32, softmax,
+// top-2 (ties to the lower index), renormalised weights.  A block owns 128
+// tokens (= one 256-route chunk) and writes that chunk's per-expert route
+// counts; it also clears the token's combine counters for the MoE.
+template <typename T>
+__global__ void __launch_bounds__(256) gate_kernel(const T* __restrict__ x1, const float* __restrict__ g,
+                                                   const float* __restrict__ b,
+                                                   const float* __restrict__ wg,
+                                                   const float* __restrict__ bg, T* __restrict__ xn2,
+                                                   int32_t* __restrict__ idx, float* __restrict__ wout,
+                                                   int32_t* __restrict__ chunk_cnt,
+                                                   int32_t* __restrict__ comb_cnt, int T_) {
+  __shared__ int32_t s_hist[E];
+  if (threadIdx.x < E) s_hist[threadIdx.x] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int i = 0; i < 16; ++i) {
+    const int t = blockIdx.x * 128 + warp * 16 + i;
+    if (t >= T_) break;
+    float v[16];
+    Row16<T>::load(x1 + size_t(t) * D, lane, v);
+    layer_norm16<T>(v, g, b, lane);
+    Row16<T>::store(xn2 + size_t(t) * D, lane, v);
+    float lg[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) s += v[j] * __ldg(wg + e * D + Row16<T>::elem(lane, j));
+      lg[e] = warp_sum(s) + (bg ? __ldg(bg + e) : 0.f);
+    }
+    if (lane == 0) {
+      float m = lg[0];
+#pragma unroll
+      for (int e = 1; e < E; ++e) m = fmaxf(m, lg[e]);
+      float p[E], sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        p[e] = expf(lg[e] - m);
+        sum += p[e];
+      }
+      int e0 = -1, e1 = -1;
+      float p0 = -1.f, p1 = -1.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float pe = p[e] / sum;
+        if (pe > p0) {
+          e1 = e0;
+          p1 = p0;
+          e0 = e;
+          p0 = pe;
+        } else if (pe > p1) {
+          e1 = e;
+          p1 = pe;
+        }
+      }
+      const float den = p0 + p1;
+      idx[2 * t] = e0;
+      idx[2 * t + 1] = e1;
+      wout[2 * t] = p0 / den;
+      wout[2 * t + 1] = p1 / den;
+      atomicAdd(&s_hist[e0], 1);
+      atomicAdd(&s_hist[e1], 1);
+    }
+    if (comb_cnt && lane < GEMM2_NT) comb_cnt[size_t(t) * GEMM2_NT + lane] = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x < E) chunk_cnt[blockIdx.x * E + threadIdx.x] = s_hist[threadIdx.x];
+}
+
+// Per-chunk route counts for a caller-supplied topk_idx (standalone route
+// build); out-of-range expert ids set PTL_ERR_SHAPE and are skipped.
+__global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ idx, int n_routes,
+                                                         int32_t* __restrict__ chunk_cnt, int32_t* err) {
+  __shared__ int32_t s_hist[E];
+  if (threadIdx.x < E) s_hist[threadIdx.x] = 0;
+  __syncthreads();
+  const int r = blockIdx.x * ROUTE_CHUNK + threadIdx.x;
+  if (r < n_routes) {
+    const int e = idx[r];
+    if (e >= 0 && e < E)
+      atomicAdd(&s_hist[e], 1);
+    else
+      set_error(err, PTL_ERR_SHAPE);
+  }
+  __syncthreads();
+  if (threadIdx.x < E) chunk_cnt[blockIdx.x * E + threadIdx.x] = s_hist[threadIdx.x];
+}
+
+// ---------------------------------------------------------- route builder
+// One block per chunk of 256 routes (one thread per route r = 2t + k).
+// Stable counting sort: slot of r inside expert e = routes of e in earlier
+// chunks + routes of e in earlier warps of this chunk + earlier lanes of
+// this warp with the same expert.  Writes perm (compact slots), rowroute
+// (padded slots: every expert's rows start on a 128-row boundary) and, in
+// block 0, the padding (-1), the expert tile list and the offsets.
+__global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
+    const int32_t* __restrict__ idx, int n_routes, const int32_t* __restrict__ chunk_cnt,
+    int32_t* __restrict__ perm, int32_t* __restrict__ rowroute, int2* __restrict__ tiles,
+    int32_t* __restrict__ meta, int32_t* __restrict__ dbg_perm, int32_t* __restrict__ dbg_off,
+    const int32_t* err) {
+  __shared__ int32_t s_red[ROUTE_CHUNK / 32][2 * E];
+  __shared__ int32_t s_pre[E], s_tot[E], s_off[E + 1], s_poff[E + 1];
+  __shared__ int32_t s_wcnt[ROUTE_CHUNK / 32][E];
+  if (has_error(err)) return;
+  const int c = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n_chunks = (n_routes + ROUTE_CHUNK - 1) / ROUTE_CHUNK;
+  int acc[2 * E];
+#pragma unroll
+  for (int e = 0; e < 2 * E; ++e) acc[e] = 0;
+  for (int cc = tid; cc < n_chunks; cc += ROUTE_CHUNK) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int v = chunk_cnt[cc * E + e];
+      acc[E + e] += v;
+      if (cc < c) acc[e] += v;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 2 * E; ++e) {
+    int v = acc[e];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) s_red[warp][e] = v;
+  }
+  if (tid < E) {
+#pragma unroll
+    for (int w = 0; w < ROUTE_CHUNK / 32; ++w) s_wcnt[w][tid] = 0;
+  }
+  __syncthreads();
+  if (tid < 2 * E) {
+    int v = 0;
+#pragma unroll
+    for (int w = 0; w < ROUTE_CHUNK / 32; ++w) v += s_red[w][tid];
+    if (tid < E) s_pre[tid] = v; else s_tot[tid - E] = v;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    s_off[0] = 0;
+    s_poff[0] = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e + 1] = s_off[e] + s_tot[e];
+      s_poff[e + 1] = s_poff[e] + (s_tot[e] + MOE_BM - 1) / MOE_BM * MOE_BM;
+    }
+  }
+  const int r = c * ROUTE_CHUNK + tid;
+  bool valid = r < n_routes;
+  int e = valid ? idx[r] : E;
+  if (e < 0 || e >= E) {  // never index with an id outside [0, E)
+    e = E;
+    valid = false;
+  }
+  const unsigned same = __match_any_sync(0xffffffffu, e);
+  const int rank = __popc(same & ((1u << lane) - 1u));
+  if (valid && rank == 0) s_wcnt[warp][e] = __popc(same);
+  __syncthreads();
+  if (valid) {
+    int j = s_pre[e] + rank;
+    for (int w = 0; w < warp; ++w) j += s_wcnt[w][e];
+    perm[s_off[e] + j] = r;
+    if (dbg_perm) dbg_perm[s_off[e] + j] = r;
+    rowroute[s_poff[e] + j] = r;
+  }
+  if (c == 0) {
+    for (int ee = 0; ee < E; ++ee) {
+      for (int i = s_off[ee + 1] - s_off[ee] + tid; i < s_poff[ee + 1] - s_poff[ee]; i += ROUTE_CHUNK)
+        rowroute[s_poff[ee] + i] = -1;
+      const int nt = (s_poff[ee + 1] - s_poff[ee]) / MOE_BM;
+      for (int j = tid; j < nt; j += ROUTE_CHUNK)
+        tiles[s_poff[ee] / MOE_BM + j] = make_int2(ee, s_poff[ee] + j * MOE_BM);
+    }
+    if (tid == 0) meta[0] = s_poff[E] / MOE_BM;
+    if (tid <= E) {
+      meta[1 + tid] = s_off[tid];
+      meta[10 + tid] = s_poff[tid];
+      if (dbg_off) dbg_off[tid] = s_off[tid];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ head
+template <typename T>
+__global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, const float* __restrict__ g,
+                                                   const float* __restrict__ b,
+                                                   const float* __restrict__ w,
+                                                   const float* __restrict__ bias,
+                                                   float* __restrict__ p, int T_) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T_) return;
+  float v[16];
+  Row16<T>::load(h + size_t(t) * D, lane, v);
+  layer_norm16<T>(v, g, b, lane);
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) s += v[j] * __ldg(w + Row16<T>::elem(lane, j));
+  s = warp_sum(s) + (bias ? __ldg(bias) : 0.f);
+  if (lane == 0) {
+    const float z = fminf(fmaxf(s, -LOGIT_CLAMP), LOGIT_CLAMP);
+    p[t] = 1.0f / (1.0f + expf(-z));
+  }
+}
+
+// Keeps p[t] for the tokens with pred_mask[t] != 0, in ascending t.
+__global__ void __launch_bounds__(1024) head_compact_kernel(const float* __restrict__ p,
+                                                            const uint8_t* __restrict__ mask,
+                                                            float* __restrict__ probs,
+                                                            int32_t* __restrict__ n_pred, int T_) {
+  __shared__ int32_t s_scan[1024];
+  __shared__ int32_t s_carry;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < T_; base += 1024) {
+    const int t = base + threadIdx.x;
+    const int f = (t < T_ && mask[t]) ? 1 : 0;
+    s_scan[threadIdx.x] = f;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int v = threadIdx.x >= unsigned(o) ? s_scan[threadIdx.x - o] : 0;
+      __syncthreads();
+      s_scan[threadIdx.x] += v;
+      __syncthreads();
+    }
+    if (f) probs[s_carry + s_scan[threadIdx.x] - 1] = p[t];
+    __syncthreads();
+    if (threadIdx.x == 1023) s_carry += s_scan[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && n_pred) *n_pred = s_carry;
+}
+
+// ------------------------------------------------- fp32 build: CUDA cores
+// C tile 64 x 64, K step 16, 256 threads with 4 x 4 outputs each.
+// Modes: 0 = A rows direct, out = acc + bias (QKV projection)
+//        1 = A rows direct, out = acc + bias + R (output projection + residual)
+//        2 = A rows gathered through rowroute (token = route / 2), per-tile
+//            expert weights, out = ReLU(acc + b1[e]) into the padded hidden rows
+//        3 = A = padded hidden rows, per-tile expert weights, y[route] = acc + b2[e]
+template <int MODE>
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, int lda,
+                                                       const float* __restrict__ W,
+                                                       const float* __restrict__ bias,
+                                                       const float* __restrict__ R,
+                                                       float* __restrict__ C, int ldc, int M, int N,
+                                                       int Kd, const int32_t* __restrict__ rowroute,
+                                                       const int2* __restrict__ tiles,
+                                                       const int32_t* __restrict__ meta,
+                                                       const int32_t* err) {
+  __shared__ float sA[16][64 + 4];
+  __shared__ float sB[16][64 + 4];
+  __shared__ int s_arow[64];
+  if (has_error(err)) return;
+  const int tid = threadIdx.x;
+  int row0, expert = 0;
+  if (MODE >= 2) {
+    const int tile = blockIdx.x >> 1;
+    if (tile >= meta[0]) return;
+    const int2 tl = tiles[tile];
+    expert = tl.x;
+    row0 = tl.y + (blockIdx.x & 1) * 64;
+  } else {
+    row0 = blockIdx.x * 64;
+  }
+  const int n0 = blockIdx.y * 64;
+  if (tid < 64) {
+    const int m = row0 + tid;
+    int ar;
+    if (MODE == 2) {
+      const int r = rowroute[m];
+      ar = r < 0 ? -1 : r / K;
+    } else if (MODE == 3) {
+      ar = m;
+    } else {
+      ar = m < M ? m : -1;
+    }
+    s_arow[tid] = ar;
+  }
+  __syncthreads();
+  const float* Wt = W + size_t(expert) * N * Kd;
+  const int tr = tid / 16, tc = tid % 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < Kd; k0 += 16) {
+    for (int i = tid; i < 64 * 16; i += 256) {
+      const int r = i / 16, kk = i % 16;
+      const int ar = s_arow[r];
+      sA[kk][r] = ar >= 0 ? A[size_t(ar) * lda + k0 + kk] : 0.f;
+      sB[kk][r] = (n0 + r < N) ? Wt[size_t(n0 + r) * Kd + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = sA[kk][tr * 4 + i];
+        bb[i] = sB[kk][tc * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = row0 + tr * 4 + i;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tc * 4 + j;
+      if (n >= N) continue;
+      float v = acc[i][j];
+      if (MODE == 0) {
+        if (m >= M) continue;
+        C[size_t(m) * ldc + n] = v + (bias ? bias[n] : 0.f);
+      } else if (MODE == 1) {
+        if (m >= M) continue;
+        C[size_t(m) * ldc + n] = v + (bias ? bias[n] : 0.f) + R[size_t(m) * ldc + n];
+      } else if (MODE == 2) {
+        v += bias ? bias[expert * N + n] : 0.f;
+        C[size_t(m) * ldc + n] = fmaxf(v, 0.f);
+      } else {
+        const int r = rowroute[m];
+        if (r < 0) continue;
+        C[size_t(r) * ldc + n] = v + (bias ? bias[expert * N + n] : 0.f);
+      }
+    }
+  }
+}
+
+// out[t] = (x1[t] + w[t][0] * y[2t]) + w[t][1] * y[2t+1], fp32.
+__global__ void __launch_bounds__(256) combine_f32_kernel(const float* __restrict__ y,
+                                                          const float* __restrict__ w,
+                                                          const float* __restrict__ x1,
+                                                          float* __restrict__ out, int T_,
+                                                          const int32_t* err) {
+  if (has_error(err)) return;
+  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= size_t(T_) * D) return;
+  const size_t t = i / D, n = i % D;
+  const float a = x1[i] + w[2 * t] * y[(2 * t) * D + n];
+  out[i] = a + w[2 * t + 1] * y[(2 * t + 1) * D + n];
+}
+
+// Jagged causal attention on CUDA cores (fp32 build).  One block of 128
+// threads per (user, query block, head) work item; thread i owns query row
+// i of the block and runs an fp32 online softmax over the user's keys
+// 0..q, staged 64 at a time in shared memory.
+__global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__ qkv,
+                                                       float* __restrict__ out,
+                                                       const int32_t* __restrict__ cu,
+                                                       const int2* __restrict__ items,
+                                                       const int32_t* __restrict__ item_count,
+                                                       const int32_t* err) {
+  __shared__ float sK[64][DH + 1];
+  __shared__ float sV[64][DH + 1];
+  if (has_error(err)) return;
+  const int item = blockIdx.x / H, h = blockIdx.x % H;
+  if (item >= *item_count) return;
+  const int2 it = items[item];
+  const int s0 = cu[it.x], L = cu[it.x + 1] - s0;
+  const int qi = it.y * ATT_BLK + threadIdx.x;
+  const bool valid = qi < L;
+  float q[DH], o[DH];
+  const float scale = 0.125f;
+#pragma unroll
+  for (int d = 0; d < DH; ++d) {
+    q[d] = valid ? qkv[size_t(s0 + qi) * QKV_N + h * DH + d] * scale : 0.f;
+    o[d] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const int kend = min(L, (it.y + 1) * ATT_BLK);
+  for (int k0 = 0; k0 < kend; k0 += 64) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 64 * DH; i += 128) {
+      const int r = i / DH, d = i % DH;
+      const int kj = k0 + r;
+      sK[r][d] = kj < L ? qkv[size_t(s0 + kj) * QKV_N + D + h * DH + d] : 0.f;
+      sV[r][d] = kj < L ? qkv[size_t(s0 + kj) * QKV_N + 2 * D + h * DH + d] : 0.f;
+    }
+    __syncthreads();
+    if (!valid) continue;
+    for (int r = 0; r < 64 && k0 + r <= qi; ++r) {
+      float s = 0.f;
+#pragma unroll
+      for (int d = 0; d < DH; ++d) s = fmaf(q[d], sK[r][d], s);
+      const float mn = fmaxf(m, s);
+      const float alpha = expf(m - mn);
+      const float p = expf(s - mn);
+      l = l * alpha + p;
+#pragma unroll
+      for (int d = 0; d < DH; ++d) o[d] = o[d] * alpha + p * sV[r][d];
+      m = mn;
+    }
+  }
+  if (!valid) return;
+  const float inv = 1.0f / l;
+#pragma unroll
+  for (int d = 0; d < DH; ++d) out[size_t(s0 + qi) * D + h * DH + d] = o[d] * inv;
+}
+
+// ------------------------------------------------------------- launchers
+#define PTL_LAUNCH_CHECK() (cudaPeekAtLastError() == cudaSuccess ? 0 : -1)
+
+int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st) {
+  worklist_kernel<<<1, 1024, 0, st>>>(cu, U, T, reinterpret_cast<int2*>(ws + L.items),
+                                      reinterpret_cast<int32_t*>(ws + L.item_count),
+                                      reinterpret_cast<int32_t*>(ws + L.lvl_hist),
+                                      reinterpret_cast<int32_t*>(ws + L.lvl_start),
+                                      reinterpret_cast<int32_t*>(ws + L.lvl_fill), int(L.max_levels),
+                                      reinterpret_cast<int32_t*>(ws + L.err));
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
+                     cudaStream_t st) {
+  const int blocks = (T + 7) / 8;
+  if (dt == PTL_BF16)
+    ln_rows_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T);
+  else
+    ln_rows_kernel<float, float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), g, b,
+                                                         static_cast<float*>(y), T);
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
+                void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int32_t* comb_cnt, int T,
+                ptl_dtype dt, cudaStream_t st) {
+  const int blocks = (T + 127) / 128;
+  if (dt == PTL_BF16)
+    gate_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x1), g, b, wg, bg, static_cast<__nv_bfloat16*>(xn2), idx,
+        w, chunk_cnt, comb_cnt, T);
+  else
+    gate_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x1), g, b, wg, bg,
+                                               static_cast<float*>(xn2), idx, w, chunk_cnt,
+                                               comb_cnt, T);
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_chunk_hist(const int32_t* idx, int T, int32_t* chunk_cnt, int32_t* err, cudaStream_t st) {
+  const int n = 2 * T;
+  chunk_hist_kernel<<<(n + ROUTE_CHUNK - 1) / ROUTE_CHUNK, ROUTE_CHUNK, 0, st>>>(idx, n, chunk_cnt, err);
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
+                 int32_t* dbg_off, cudaStream_t st) {
+  const int n = 2 * T;
+  route_kernel<<<(n + ROUTE_CHUNK - 1) / ROUTE_CHUNK, ROUTE_CHUNK, 0, st>>>(
+      idx, n, reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
+      reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.rowroute),
+      reinterpret_cast<int2*>(ws + L.tiles), reinterpret_cast<int32_t*>(ws + L.route_meta),
+      dbg_perm, dbg_off, reinterpret_cast<const int32_t*>(ws + L.err));
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, float* probs,
+                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st) {
+  float* p = reinterpret_cast<float*>(ws + L.head_p);
+  const int blocks = (T + 7) / 8;
+  const float* g = static_cast<const float*>(hw->lnf_g);
+  const float* b = static_cast<const float*>(hw->lnf_b);
+  const float* w = static_cast<const float*>(hw->w);
+  const float* bias = static_cast<const float*>(hw->b);
+  if (dt == PTL_BF16)
+    head_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), g, b, w,
+                                                       bias, p, T);
+  else
+    head_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(h), g, b, w, bias, p, T);
+  if (PTL_LAUNCH_CHECK() != 0) return -1;
+  head_compact_kernel<<<1, 1024, 0, st>>>(p, mask, probs, n_pred, T);
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const float* bias,
+                    const float* R, float* C, int ldc, int M, int N, int Kd, const WsLayout& L,
+                    const char* ws, cudaStream_t st) {
+  const int32_t* rr = reinterpret_cast<const int32_t*>(ws + L.rowroute);
+  const int2* tiles = reinterpret_cast<const int2*>(ws + L.tiles);
+  const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
+  const int32_t* err = reinterpret_cast<const int32_t*>(ws + L.err);
+  dim3 grid(mode >= 2 ? unsigned(2 * L.max_tiles) : unsigned((M + 63) / 64), unsigned((N + 63) / 64));
+  switch (mode) {
+    case 0: gemm_f32_kernel<0><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    case 1: gemm_f32_kernel<1><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    case 2: gemm_f32_kernel<2><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    default: gemm_f32_kernel<3><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+  }
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_combine_f32(const float* y, const float* w, const float* x1, float* out, int T,
+                       const int32_t* err, cudaStream_t st) {
+  const size_t n = size_t(T) * D;
+  combine_f32_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(y, w, x1, out, T, err);
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
+                    const char* ws, cudaStream_t st) {
+  attn_f32_kernel<<<unsigned(L.max_items * H), 128, 0, st>>>(
+      qkv, out, cu, reinterpret_cast<const int2*>(ws + L.items),
+      reinterpret_cast<const int32_t*>(ws + L.item_count), reinterpret_cast<const int32_t*>(ws + L.err));
+  return PTL_LAUNCH_CHECK();
+}
+
+}  // namespace ptl
