@@ -53,6 +53,29 @@ def _f64(a):
     return np.asarray(a, dtype=np.float64)
 
 
+def round_bf16(a):
+    """Round to the nearest bfloat16 value (ties to even), returned as float64:
+    keep the top 16 bits of the float32 encoding after adding half of the
+    dropped part (0x7FFF plus the lowest kept bit, which breaks ties to even).
+    Used only by the storage='bf16' mode below."""
+    f = np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    keep = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return keep.astype(np.uint32).view(np.float32).astype(np.float64).reshape(f.shape)
+
+
+def _storage(storage):
+    """Rounding applied where the bf16 pipeline stores an activation: the
+    identity for the exact fp64 oracle (storage=None), bfloat16 rounding for
+    storage='bf16' (the cti2026 README runs inference in bf16 with fp32
+    accumulation and fp32 softmax statistics, writing results back as bf16)."""
+    if storage is None:
+        return lambda a: _f64(a)
+    if storage == "bf16":
+        return round_bf16
+    raise ValueError(storage)
+
+
 # --------------------------------------------------------------------------
 # LayerNorm and Linear (cti2026 README, TransformerEncoder section)
 # --------------------------------------------------------------------------
@@ -173,6 +196,12 @@ def top2_gap(p):
     return ps[:, 1] - ps[:, 2]
 
 
+def top1_gap(p):
+    """p_(1) - p_(2): how far apart the two chosen experts are (slot order)."""
+    ps = -np.sort(-_f64(p), axis=-1)
+    return ps[:, 0] - ps[:, 1]
+
+
 # --------------------------------------------------------------------------
 # Route builder (cti2026 README, fused MoE routing preparation)
 # --------------------------------------------------------------------------
@@ -200,12 +229,13 @@ def expert_ffn(x, w1, b1, w2, b2):
     return linear(np.maximum(linear(x, w1, b1), 0.0), w2, b2)
 
 
-def moe_routed(xn2, idx, w, w1, b1, w2, b2):
+def moe_routed(xn2, idx, w, w1, b1, w2, b2, hidden_round=None):
     """Sparse top-2 MoE.  Routes are grouped per expert with ``route_build``;
     each expert runs its FFN on its gathered tokens; route r's result is kept
     in route-major row r = 2 t + k; token t's output is w[t,0] y[2t] +
     w[t,1] y[2t+1].  Returns (moe_out [T, D], y [2T, D], hidden per route
-    [2T, F] in slot order)."""
+    [2T, F] in slot order).  hidden_round, if given, is applied to the
+    hidden layer (the bf16 storage mode of layer_forward)."""
     xn2 = _f64(xn2)
     T, D = xn2.shape
     E = np.asarray(w1).shape[0]
@@ -219,6 +249,8 @@ def moe_routed(xn2, idx, w, w1, b1, w2, b2):
             continue
         tok = routes // TOP_K
         h = np.maximum(linear(xn2[tok], w1[e], b1[e]), 0.0)
+        if hidden_round is not None:
+            h = hidden_round(h)
         hidden[off[e]:off[e + 1]] = h
         y[routes] = linear(h, w2[e], b2[e])
     w = _f64(w)
@@ -239,27 +271,38 @@ def moe_dense_all_experts(xn2, idx, w, w1, b1, w2, b2):
 # --------------------------------------------------------------------------
 # Layer, stack, head (cti2026 README, TransformerEncoder + Prediction Head)
 # --------------------------------------------------------------------------
-def layer_forward(x, cu_seqlens, wts, return_intermediates=False):
-    """One pre-norm layer over the packed stream x [T, D]."""
+def layer_forward(x, cu_seqlens, wts, return_intermediates=False, storage=None):
+    """One pre-norm layer over the packed stream x [T, D].
+
+    storage=None computes everything in float64.  storage='bf16' rounds to
+    bfloat16 the activations a bf16 pipeline stores between its steps -- the
+    LayerNorm1 output, q/k/v, the attention output, x1, the LayerNorm2 output
+    fed to the experts, the expert hidden layer and the layer output -- while
+    the gate still sees the unrounded LayerNorm2 output and all arithmetic
+    stays float64.  It follows the same definition; only the stored values
+    carry the bf16 rounding."""
+    rnd = _storage(storage)
     x = _f64(x)
     T, D = x.shape
-    xn = layer_norm(x, wts["ln1_g"], wts["ln1_b"])
-    qkv = linear(xn, wts["w_qkv"], wts.get("b_qkv"))
+    xn = rnd(layer_norm(x, wts["ln1_g"], wts["ln1_b"]))
+    qkv = rnd(linear(xn, wts["w_qkv"], wts.get("b_qkv")))
     q, k, v = split_qkv(qkv)
-    attn = jagged_causal_attention(q, k, v, cu_seqlens).reshape(T, D)
-    x1 = x + linear(attn, wts["w_o"], wts.get("b_o"))
-    xn2 = layer_norm(x1, wts["ln2_g"], wts["ln2_b"])
-    p = gate_probs(xn2, wts["w_gate"], wts.get("b_gate"))
+    attn = rnd(jagged_causal_attention(q, k, v, cu_seqlens).reshape(T, D))
+    x1 = rnd(x + linear(attn, wts["w_o"], wts.get("b_o")))
+    xn2_exact = layer_norm(x1, wts["ln2_g"], wts["ln2_b"])
+    xn2 = rnd(xn2_exact)
+    p = gate_probs(xn2_exact, wts["w_gate"], wts.get("b_gate"))
     idx, w = top2(p)
-    moe, y, hidden = moe_routed(xn2, idx, w, wts["w1"], wts["b1"], wts["w2"], wts["b2"])
-    out = x1 + moe
+    moe, y, hidden = moe_routed(xn2, idx, w, wts["w1"], wts["b1"], wts["w2"], wts["b2"],
+                                hidden_round=rnd)
+    out = rnd(x1 + moe)
     if not return_intermediates:
         return out
     E = np.asarray(wts["w1"]).shape[0]
     cnt, off, perm, pos = route_build(idx, E)
     return out, dict(xn=xn, qkv=qkv, attn=attn, x1=x1, xn2=xn2, p=p, idx=idx, w=w,
-                     gap=top2_gap(p), cnt=cnt, off=off, perm=perm, pos=pos, y=y,
-                     hidden=hidden, moe=moe)
+                     gap=top2_gap(p), gap12=top1_gap(p), cnt=cnt, off=off, perm=perm, pos=pos,
+                     y=y, hidden=hidden, moe=moe, out=out)
 
 
 def head_forward(x, head, pred_mask=None):
@@ -274,11 +317,19 @@ def head_forward(x, head, pred_mask=None):
     return probs[np.asarray(pred_mask).astype(bool)]
 
 
-def stack_forward(x, cu_seqlens, layers, head=None, pred_mask=None):
-    """L layers in sequence, each with its own weights, then the optional head."""
+def stack_forward(x, cu_seqlens, layers, head=None, pred_mask=None, storage=None,
+                  return_intermediates=False):
+    """L layers in sequence, each with its own weights, then the optional head.
+    With return_intermediates, also returns each layer's intermediates."""
     h = _f64(x)
+    per_layer = []
     for wts in layers:
-        h = layer_forward(h, cu_seqlens, wts)
-    if head is None:
-        return h
-    return h, head_forward(h, head, pred_mask)
+        if return_intermediates:
+            h, it = layer_forward(h, cu_seqlens, wts, return_intermediates=True, storage=storage)
+            per_layer.append(it)
+        else:
+            h = layer_forward(h, cu_seqlens, wts, storage=storage)
+    res = (h,) if head is None else (h, head_forward(h, head, pred_mask))
+    if return_intermediates:
+        res = res + (per_layer,)
+    return res[0] if len(res) == 1 else res

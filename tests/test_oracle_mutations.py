@@ -100,8 +100,8 @@ def test_unstable_route_order_is_caught(monkeypatch):
 def test_dropped_expert_bias_is_caught(monkeypatch):
     orig = O.moe_routed
 
-    def no_b2(xn2, idx, w, w1, b1, w2, b2):
-        return orig(xn2, idx, w, w1, b1, w2, np.zeros_like(np.asarray(b2, np.float64)))
+    def no_b2(xn2, idx, w, w1, b1, w2, b2, **kw):
+        return orig(xn2, idx, w, w1, b1, w2, np.zeros_like(np.asarray(b2, np.float64)), **kw)
     monkeypatch.setattr(O, "moe_routed", no_b2)
     assert _fails(P.test_moe_golden)
     assert _fails(P.test_layer_constant_expert_output_adds_constant)

@@ -360,3 +360,25 @@ def test_generated_packings():
     assert L.sum() == 6823 and len(L) == 60 and L.min() >= 1 and L.max() <= 1024
     c = S.config0()
     assert c.cu_seqlens.tolist() == [0, 3, 10, 22, 42]
+
+
+# ---------------------------------------------------- bf16 storage precision
+def test_round_bf16_matches_torch_conversion():
+    rng = np.random.default_rng(41)
+    a = np.concatenate([rng.standard_normal(20000) * 7, [0.0, -0.0, 1.0, 1.00390625, 1.01171875,
+                                                          65504.0, 1e-30, -3.3e38]])
+    ref = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(a), ref)
+    np.testing.assert_array_equal(O.round_bf16(O.round_bf16(a)), O.round_bf16(a))
+
+
+def test_bf16_storage_mode_stays_within_bf16_error_of_exact():
+    c = S.make_case("st", lengths=[30, 1, 70], seed=42, dtype="bf16", gate_std=0.1, random_bias=True)
+    ex, it = O.layer_forward(c.x, c.cu_seqlens, c.layers[0], return_intermediates=True)
+    bf, itb = O.layer_forward(c.x, c.cu_seqlens, c.layers[0], return_intermediates=True,
+                              storage="bf16")
+    same = np.all(it["idx"] == itb["idx"], axis=1)
+    assert same.mean() > 0.95
+    assert np.max(np.abs(bf[same] - ex[same])) < 3e-2
+    assert np.array_equal(bf, O.round_bf16(bf))          # stored output is on the bf16 grid
+    assert not np.array_equal(bf, ex)
