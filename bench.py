@@ -285,16 +285,27 @@ def run_ours(args):
     tokens_layers = T * n_layers * world
     value = tokens_layers / (ms_max / 1e3)
 
-    # ---- per-kernel device times (eager, traced; L2 flushed between steps)
+    # ---- per-kernel device times: the same step captured with a CUDA event
+    # before every launch (event nodes inside the graph), replayed with the
+    # L2 flushed in between; launch i takes events[i] -> events[i + 1].
     trace_steps = min(args.steps, 10)
-    kt = ptl.KernelTrace(capacity=trace_steps * (launches_per_step + 8) + 16)
+    kt = ptl.KernelTrace(capacity=2 * launches_per_step + 16)
+    tgraph = torch.cuda.CUDAGraph()
+    with kt:
+        with torch.cuda.graph(tgraph, stream=stream):
+            step()
+    torch.cuda.synchronize()
+    recorded = []
     with torch.cuda.stream(stream):
-        with kt:
-            for i in range(trace_steps):
-                step()
-                flush.fill_(float(i))
+        for i in range(trace_steps):
+            tgraph.replay()
+            torch.cuda.synchronize()
+            recorded.extend(kt.launches())
+            flush.fill_(float(i))
+    torch.cuda.synchronize()
+    tgraph.reset()
     per_kind = {}
-    for kind, t_ms in kt.launches():
+    for kind, t_ms in recorded:
         d = per_kind.setdefault(kind, [0.0, 0])
         d[0] += t_ms
         d[1] += 1
@@ -388,7 +399,7 @@ def run_ours(args):
             "config": {"workload": case.name, "tokens": T, "users": U, "layers": n_layers,
                        "head": head is not None, "parallelism": f"dp{world} (independent batches)",
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "timing": "CUDA graph replay, CUDA events per step"},
+                       "timing": "CUDA graph replay, CUDA events per step; per-kernel times from event nodes in a second captured graph"},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),

@@ -22,9 +22,12 @@
  * 512->8, 8 experts 512->1024->512, top-2.
  *
  * Conventions for every entry point
- *   - All tensor pointers are DEVICE pointers unless stated otherwise,
- *     row-major, and must be 16-byte aligned (PTL_ERR_ALIGN otherwise).
- *     Weight matrices use the nn.Linear layout W[out][in].
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise and
+ *     row-major.  Activations, weights, biases and LayerNorm parameters must
+ *     be 16-byte aligned; topk_idx / topk_w written by ptl_gate 8-byte
+ *     aligned; cu_seqlens, perm, expert_off, probs and n_pred 4-byte
+ *     aligned (PTL_ERR_ALIGN otherwise).  Weight matrices use the nn.Linear
+ *     layout W[out][in].
  *   - Activations and the big matrices (w_qkv, w_o, w1, w2) are stored in
  *     the build dtype `dt`: PTL_BF16 (bfloat16 storage, fp32 accumulation)
  *     or PTL_F32 (fp32 storage and arithmetic).  LayerNorm parameters, the
@@ -156,12 +159,15 @@ ptl_status ptl_attention(const void* qkv, void* attn, const int32_t* cu_seqlens,
                          int32_t num_users, int64_t total_tokens, ptl_dtype dt,
                          void* workspace, size_t ws_bytes, void* stream);
 
-/* x1[T][512] = x + attn Wo^T + b_o. */
+/* x1[T][512] = x + attn Wo^T + b_o.  x1 is float32 in both builds: the
+ * residual stream inside a layer is kept in fp32 so that the layer output is
+ * rounded to the build dtype once. */
 ptl_status ptl_out_projection(const void* attn, const void* x, void* x1, int64_t total_tokens,
                               ptl_dtype dt, const ptl_layer_weights* w, void* workspace,
                               size_t ws_bytes, void* stream);
 
-/* xn2[T][512] = LayerNorm2(x1) (dt); p = softmax(xn2 Wg^T + bg) in fp32;
+/* x1: float32 [T][512] (see ptl_out_projection).
+ * xn2[T][512] = LayerNorm2(x1) (dt); p = softmax(xn2 Wg^T + bg) in fp32;
  * topk_idx[T][2] (int32) = the two largest p (ties to the lower expert
  * index, slot 0 the larger), topk_w[T][2] (f32) = p / (p0 + p1). */
 ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w,
@@ -175,7 +181,8 @@ ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w,
 ptl_status ptl_route_build(const int32_t* topk_idx, int64_t total_tokens, int32_t* perm,
                            int32_t* expert_off, void* workspace, size_t ws_bytes, void* stream);
 
-/* out[t] = residual[t] + topk_w[t][0] y(t, topk_idx[t][0]) + topk_w[t][1] y(t, topk_idx[t][1]),
+/* residual: float32 [T][512] (x1 of the layer); out: [T][512] in dt.
+ * out[t] = residual[t] + topk_w[t][0] y(t, topk_idx[t][0]) + topk_w[t][1] y(t, topk_idx[t][1]),
  * y(t, e) = ReLU(xn2[t] W1[e]^T + b1[e]) W2[e]^T + b2[e]  (uses w1, b1, w2, b2 of w).
  * The k = 0 term is added first, in fp32, and rounded once. */
 ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w,

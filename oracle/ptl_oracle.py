@@ -271,16 +271,21 @@ def moe_dense_all_experts(xn2, idx, w, w1, b1, w2, b2):
 # --------------------------------------------------------------------------
 # Layer, stack, head (cti2026 README, TransformerEncoder + Prediction Head)
 # --------------------------------------------------------------------------
-def layer_forward(x, cu_seqlens, wts, return_intermediates=False, storage=None):
+def layer_forward(x, cu_seqlens, wts, return_intermediates=False, storage=None, choose=None):
     """One pre-norm layer over the packed stream x [T, D].
 
     storage=None computes everything in float64.  storage='bf16' rounds to
     bfloat16 the activations a bf16 pipeline stores between its steps -- the
-    LayerNorm1 output, q/k/v, the attention output, x1, the LayerNorm2 output
-    fed to the experts, the expert hidden layer and the layer output -- while
-    the gate still sees the unrounded LayerNorm2 output and all arithmetic
-    stays float64.  It follows the same definition; only the stored values
-    carry the bf16 rounding."""
+    LayerNorm1 output, q/k/v, the attention output, the LayerNorm2 output fed
+    to the experts, the expert hidden layer and the layer output -- while the
+    residual x1 inside the layer stays unrounded (an fp32 buffer in such a
+    pipeline), the gate sees the unrounded LayerNorm2 output and all
+    arithmetic stays float64.  It follows the same definition; only the stored values
+    carry the bf16 rounding.
+
+    choose(p, idx) -> idx, if given, may replace the top-2 pairs before
+    routing (the weights are renormalised from p for the pairs it returns).
+    Tests use it to follow another valid branch where two experts tie."""
     rnd = _storage(storage)
     x = _f64(x)
     T, D = x.shape
@@ -288,11 +293,15 @@ def layer_forward(x, cu_seqlens, wts, return_intermediates=False, storage=None):
     qkv = rnd(linear(xn, wts["w_qkv"], wts.get("b_qkv")))
     q, k, v = split_qkv(qkv)
     attn = rnd(jagged_causal_attention(q, k, v, cu_seqlens).reshape(T, D))
-    x1 = rnd(x + linear(attn, wts["w_o"], wts.get("b_o")))
+    x1 = x + linear(attn, wts["w_o"], wts.get("b_o"))
     xn2_exact = layer_norm(x1, wts["ln2_g"], wts["ln2_b"])
     xn2 = rnd(xn2_exact)
     p = gate_probs(xn2_exact, wts["w_gate"], wts.get("b_gate"))
     idx, w = top2(p)
+    if choose is not None:
+        idx = np.asarray(choose(p, idx), dtype=np.int64)
+        pt = np.take_along_axis(p, idx, axis=-1)
+        w = pt / pt.sum(axis=-1, keepdims=True)
     moe, y, hidden = moe_routed(xn2, idx, w, wts["w1"], wts["b1"], wts["w2"], wts["b2"],
                                 hidden_round=rnd)
     out = rnd(x1 + moe)
@@ -318,17 +327,20 @@ def head_forward(x, head, pred_mask=None):
 
 
 def stack_forward(x, cu_seqlens, layers, head=None, pred_mask=None, storage=None,
-                  return_intermediates=False):
+                  return_intermediates=False, choose=None):
     """L layers in sequence, each with its own weights, then the optional head.
-    With return_intermediates, also returns each layer's intermediates."""
+    With return_intermediates, also returns each layer's intermediates.
+    choose(layer, p, idx) -> idx is passed to each layer (see layer_forward)."""
     h = _f64(x)
     per_layer = []
-    for wts in layers:
+    for li, wts in enumerate(layers):
+        ch = None if choose is None else (lambda p, idx, li=li: choose(li, p, idx))
         if return_intermediates:
-            h, it = layer_forward(h, cu_seqlens, wts, return_intermediates=True, storage=storage)
+            h, it = layer_forward(h, cu_seqlens, wts, return_intermediates=True, storage=storage,
+                                  choose=ch)
             per_layer.append(it)
         else:
-            h = layer_forward(h, cu_seqlens, wts, storage=storage)
+            h = layer_forward(h, cu_seqlens, wts, storage=storage, choose=ch)
     res = (h,) if head is None else (h, head_forward(h, head, pred_mask))
     if return_intermediates:
         res = res + (per_layer,)

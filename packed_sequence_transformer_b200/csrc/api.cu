@@ -66,6 +66,7 @@ ptl_status device_ok() {
 
 inline bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool a4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+inline bool a8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 inline bool opt16(const void* p) { return p == nullptr || a16(p); }
 
 ptl_status check_common(int64_t T, ptl_dtype dt, void* ws, size_t ws_bytes, int32_t U, WsLayout* L) {
@@ -103,7 +104,14 @@ thread_local ptl_trace* g_trace = nullptr;
 inline void mark(cudaStream_t st, int kind) {
   ptl_trace* t = g_trace;
   if (!t || !t->events || t->count >= t->capacity) return;
-  cudaEventRecord(static_cast<cudaEvent_t>(t->events[t->count]), st);
+  // inside a stream capture only an external record becomes an event node
+  // that can be timed after the graph runs
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cap);
+  if (cap == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(t->events[t->count]), st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(static_cast<cudaEvent_t>(t->events[t->count]), st);
   if (t->kinds) t->kinds[t->count] = kind;
   ++t->count;
 }
@@ -403,7 +411,7 @@ ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w,
   if (total_tokens == 0) return PTL_OK;
   if (!x1 || !xn2 || !topk_idx || !topk_w || !w || !w->ln2_g || !w->ln2_b || !w->w_gate)
     return PTL_ERR_NULL;
-  if (!a16(x1) || !a16(xn2) || !a4(topk_idx) || !a4(topk_w) || !a16(w->ln2_g) || !a16(w->ln2_b) ||
+  if (!a16(x1) || !a16(xn2) || !a8(topk_idx) || !a8(topk_w) || !a16(w->ln2_g) || !a16(w->ln2_b) ||
       !a16(w->w_gate) || !opt16(w->b_gate))
     return PTL_ERR_ALIGN;
   if ((s = device_ok()) != PTL_OK) return s;

@@ -36,7 +36,7 @@ struct WsLayout {
   size_t xn;          // dt [T][512]    LayerNorm1 output
   size_t qkv;         // dt [T][1536]
   size_t attn;        // dt [T][512]
-  size_t x1;          // dt [T][512]
+  size_t x1;          // f32 [T][512]   residual stream inside the layer
   size_t xn2;         // dt [T][512]
   size_t act0, act1;  // dt [T][512]    stack ping-pong
   size_t idx;         // int32 [T][2]
@@ -85,7 +85,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->xn = take(es * T * D);
   L->qkv = take(es * T * QKV_N);
   L->attn = take(es * T * D);
-  L->x1 = take(es * T * D);
+  L->x1 = take(4 * T * D);
   L->xn2 = take(es * T * D);
   L->act0 = take(es * T * D);
   L->act1 = take(es * T * D);

@@ -15,7 +15,7 @@
 //               permutation) into the swizzled ring themselves.
 // Modes:
 //   QKV   qkv = xn Wqkv^T + b_qkv                         (A by TMA)
-//   OUT   x1  = x + attn Wo^T + b_o                       (A by TMA)
+//   OUT   x1  = x + attn Wo^T + b_o, kept in fp32         (A by TMA)
 //   MOE1  H[row] = ReLU(xn2[token(row)] W1[e]^T + b1[e])  (A gathered)
 //   MOE2  y = H W2[e]^T + b2[e], then the top-2 combine   (A by TMA)
 //         out[t] = (x1[t] + w[t,0] y(t,0)) + w[t,1] y(t,1): both routes of
@@ -39,8 +39,10 @@ struct GemmTcParams {
   int N_total;                   // output columns (per expert in the MoE modes)
   int num_kb;                    // K / 64
   const float* bias;             // [N] or [E][N]; may be NULL
-  const __nv_bfloat16* resid;    // OUT: x; MOE2: x1 (row stride 512)
+  const __nv_bfloat16* resid;    // OUT: x (row stride 512)
+  const float* resid_f32;        // MOE2: x1 in fp32 (row stride 512)
   __nv_bfloat16* out;            // output rows
+  float* out_f32;                // OUT: x1 in fp32
   int ldo;                       // output row stride (elements)
   const int32_t* rowroute;       // padded expert row -> route (or -1)
   const int2* tiles;             // (expert, first padded row) per M tile
@@ -249,7 +251,14 @@ __global__ void __launch_bounds__(192, 1)
             for (int j = 0; j < BN / 32; ++j) {
               const int n = n0 + 32 * j;
               float xr[32], o[32];
-              load_bf16x32(p.resid + size_t(t) * D + n, xr);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 r4 = *(reinterpret_cast<const float4*>(p.resid_f32 + size_t(t) * D + n) + q);
+                xr[4 * q + 0] = r4.x;
+                xr[4 * q + 1] = r4.y;
+                xr[4 * q + 2] = r4.z;
+                xr[4 * q + 3] = r4.w;
+              }
 #pragma unroll
               for (int q = 0; q < 8; ++q) {
                 const float4 a = __ldcg(reinterpret_cast<const float4*>(y0 + n) + q);
@@ -282,10 +291,14 @@ __global__ void __launch_bounds__(192, 1)
             if (MODE == G_OUT) {
               float xr[32];
               load_bf16x32(p.resid + size_t(row) * D + n, xr);
+              float4* dst = reinterpret_cast<float4*>(p.out_f32 + size_t(row) * p.ldo + n);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += xr[i];
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(v[4 * q] + xr[4 * q], v[4 * q + 1] + xr[4 * q + 1],
+                                     v[4 * q + 2] + xr[4 * q + 2], v[4 * q + 3] + xr[4 * q + 3]);
+            } else {
+              store_bf16x32(p.out + size_t(row) * p.ldo + n, v);
             }
-            store_bf16x32(p.out + size_t(row) * p.ldo + n, v);
           }
         }
       }
@@ -336,7 +349,7 @@ int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const float* 
   p.num_kb = D / 64;
   p.bias = bias;
   p.resid = static_cast<const __nv_bfloat16*>(x);
-  p.out = static_cast<__nv_bfloat16*>(x1);
+  p.out_f32 = static_cast<float*>(x1);
   p.ldo = D;
   p.err = err;
   return launch_one<OUT_BN, G_OUT>(attn, w, p, dim3((T + 127) / 128, D / OUT_BN), st);
@@ -364,7 +377,7 @@ int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const float
   p.N_total = D;
   p.num_kb = F / 64;
   p.bias = b2;
-  p.resid = static_cast<const __nv_bfloat16*>(x1);
+  p.resid_f32 = static_cast<const float*>(x1);
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ldo = D;
   p.rowroute = reinterpret_cast<const int32_t*>(ws + L.rowroute);

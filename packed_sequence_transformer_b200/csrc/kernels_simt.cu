@@ -185,38 +185,83 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
 }
 
 // ------------------------------------------------------------------ gate
-// One warp per token: LayerNorm2 of x1, the 8 gate logits in fp32, softmax,
-// top-2 (ties to the lower index), renormalised weights.  A block owns 128
-// tokens (= one 256-route chunk) and writes that chunk's per-expert route
-// counts; it also clears the token's combine counters for the MoE.
+// One warp per token (grid-stride): LayerNorm2 of x1, the 8 gate logits in
+// fp32 (w_gate staged once per block in shared memory), softmax, top-2 (ties
+// to the lower index), renormalised weights.  Per-chunk route counts (128
+// tokens = 256 routes per chunk, zeroed beforehand) are accumulated with
+// atomics; the token's combine counters for the MoE are cleared.
+constexpr int GATE_WARPS = 16;
+
+// Sums a[0..7] over the warp and leaves expert (lane >> 2)'s total in a[0]:
+// each exchange hands half of the remaining partial sums to the partner lane
+// (4 + 2 + 1 shuffles), then two more butterflies finish the sum.
+__device__ __forceinline__ float warp_reduce_scatter8(float (&a)[E], int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 16;
+    const float send = hi ? a[i] : a[i + 4];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+    a[i] = (hi ? a[i + 4] : a[i]) + recv;
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 8;
+    const float send = hi ? a[i] : a[i + 2];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+    a[i] = (hi ? a[i + 2] : a[i]) + recv;
+  }
+  {
+    const bool hi = lane & 4;
+    const float send = hi ? a[0] : a[1];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+    a[0] = (hi ? a[1] : a[0]) + recv;
+  }
+  a[0] += __shfl_xor_sync(0xffffffffu, a[0], 2);
+  a[0] += __shfl_xor_sync(0xffffffffu, a[0], 1);
+  return a[0];
+}
+
 template <typename T>
-__global__ void __launch_bounds__(256) gate_kernel(const T* __restrict__ x1, const float* __restrict__ g,
-                                                   const float* __restrict__ b,
-                                                   const float* __restrict__ wg,
-                                                   const float* __restrict__ bg, T* __restrict__ xn2,
-                                                   int32_t* __restrict__ idx, float* __restrict__ wout,
-                                                   int32_t* __restrict__ chunk_cnt,
-                                                   int32_t* __restrict__ comb_cnt, int T_) {
-  __shared__ int32_t s_hist[E];
-  if (threadIdx.x < E) s_hist[threadIdx.x] = 0;
+__global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
+    const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
+    const float* __restrict__ wg, const float* __restrict__ bg, T* __restrict__ xn2,
+    int32_t* __restrict__ idx, float* __restrict__ wout, int32_t* __restrict__ chunk_cnt,
+    int32_t* __restrict__ comb_cnt, int T_) {
+  __shared__ __align__(16) float s_wg[E * D];
+  for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  for (int i = 0; i < 16; ++i) {
-    const int t = blockIdx.x * 128 + warp * 16 + i;
-    if (t >= T_) break;
+  for (int t = blockIdx.x * GATE_WARPS + warp; t < T_; t += gridDim.x * GATE_WARPS) {
+    // x1 (fp32) is read in the output dtype's lane layout so that the LN2
+    // values land in the registers the xn2 store and the gate dots expect
     float v[16];
-    Row16<T>::load(x1 + size_t(t) * D, lane, v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<T>::elem(lane, 4 * q)));
+      v[4 * q] = f.x;
+      v[4 * q + 1] = f.y;
+      v[4 * q + 2] = f.z;
+      v[4 * q + 3] = f.w;
+    }
     layer_norm16<T>(v, g, b, lane);
     Row16<T>::store(xn2 + size_t(t) * D, lane, v);
-    float lg[E];
+    float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       float s = 0.f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) s += v[j] * __ldg(wg + e * D + Row16<T>::elem(lane, j));
-      lg[e] = warp_sum(s) + (bg ? __ldg(bg + e) : 0.f);
+      for (int q = 0; q < 4; ++q) {
+        const float4 w4 = *reinterpret_cast<const float4*>(s_wg + e * D + Row16<T>::elem(lane, 4 * q));
+        s += v[4 * q] * w4.x + v[4 * q + 1] * w4.y + v[4 * q + 2] * w4.z + v[4 * q + 3] * w4.w;
+      }
+      acc[e] = s;
     }
+    float mine = warp_reduce_scatter8(acc, lane) + (bg ? __ldg(bg + (lane >> 2)) : 0.f);
+    float lg[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) lg[e] = __shfl_sync(0xffffffffu, mine, 4 * e);
     if (lane == 0) {
       float m = lg[0];
 #pragma unroll
@@ -243,17 +288,13 @@ __global__ void __launch_bounds__(256) gate_kernel(const T* __restrict__ x1, con
         }
       }
       const float den = p0 + p1;
-      idx[2 * t] = e0;
-      idx[2 * t + 1] = e1;
-      wout[2 * t] = p0 / den;
-      wout[2 * t + 1] = p1 / den;
-      atomicAdd(&s_hist[e0], 1);
-      atomicAdd(&s_hist[e1], 1);
+      *reinterpret_cast<int2*>(idx + 2 * t) = make_int2(e0, e1);
+      *reinterpret_cast<float2*>(wout + 2 * t) = make_float2(p0 / den, p1 / den);
+      atomicAdd(&chunk_cnt[(t >> 7) * E + e0], 1);
+      atomicAdd(&chunk_cnt[(t >> 7) * E + e1], 1);
     }
     if (comb_cnt && lane < GEMM2_NT) comb_cnt[size_t(t) * GEMM2_NT + lane] = 0;
   }
-  __syncthreads();
-  if (threadIdx.x < E) chunk_cnt[blockIdx.x * E + threadIdx.x] = s_hist[threadIdx.x];
 }
 
 // Per-chunk route counts for a caller-supplied topk_idx (standalone route
@@ -616,15 +657,19 @@ int launch_layernorm(const void* x, const float* g, const float* b, void* y, int
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int32_t* comb_cnt, int T,
                 ptl_dtype dt, cudaStream_t st) {
-  const int blocks = (T + 127) / 128;
+  // chunk counts are accumulated with atomics: clear them first
+  const size_t n_chunk_bytes = sizeof(int32_t) * E * size_t((T + 127) / 128);
+  if (cudaMemsetAsync(chunk_cnt, 0, n_chunk_bytes, st) != cudaSuccess) return -1;
+  int blocks = (T + GATE_WARPS - 1) / GATE_WARPS;
+  if (blocks > 148 * 2) blocks = 148 * 2;
   if (dt == PTL_BF16)
-    gate_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x1), g, b, wg, bg, static_cast<__nv_bfloat16*>(xn2), idx,
-        w, chunk_cnt, comb_cnt, T);
+    gate_kernel<__nv_bfloat16><<<blocks, GATE_WARPS * 32, 0, st>>>(
+        static_cast<const float*>(x1), g, b, wg, bg, static_cast<__nv_bfloat16*>(xn2), idx, w,
+        chunk_cnt, comb_cnt, T);
   else
-    gate_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x1), g, b, wg, bg,
-                                               static_cast<float*>(xn2), idx, w, chunk_cnt,
-                                               comb_cnt, T);
+    gate_kernel<float><<<blocks, GATE_WARPS * 32, 0, st>>>(static_cast<const float*>(x1), g, b, wg,
+                                                           bg, static_cast<float*>(xn2), idx, w,
+                                                           chunk_cnt, comb_cnt, T);
   return PTL_LAUNCH_CHECK();
 }
 

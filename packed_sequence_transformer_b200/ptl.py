@@ -258,7 +258,7 @@ def out_projection(attn, x, x1, weights, workspace, stream=None):
 def gate(x1, xn2, topk_idx, topk_w, weights, workspace, stream=None):
     w = layer_struct(weights)
     _check(lib().ptl_gate(_ptr(x1), _ptr(xn2), _ptr(topk_idx), _ptr(topk_w), x1.shape[0],
-                          _dt(x1.dtype), ctypes.byref(w), _ptr(workspace), workspace.numel(),
+                          _dt(xn2.dtype), ctypes.byref(w), _ptr(workspace), workspace.numel(),
                           _stream(stream)), "ptl_gate")
     return xn2, topk_idx, topk_w
 

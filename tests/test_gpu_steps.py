@@ -114,7 +114,7 @@ def test_out_projection(dt, T):
     w = _weights(201, dt)
     td = BF if dt == "bf16" else F32
     ws = poisoned_workspace(T, 1, dt)
-    x1 = torch.empty(T, 512, dtype=td, device="cuda")
+    x1 = torch.empty(T, 512, dtype=F32, device="cuda")  # the residual stream stays fp32
     ptl.out_projection(dev(attn, td), dev(x, td), x1, ptl.to_device_layer(w, dt), ws)
     torch.cuda.synchronize()
     ref = x + O.linear(attn, w["w_o"], w["b_o"])
@@ -125,16 +125,14 @@ def test_out_projection(dt, T):
 @pytest.mark.parametrize("dt,T", [("bf16", 1), ("bf16", 1000), ("bf16", 6823), ("fp32", 300)])
 def test_gate(dt, T):
     rng = np.random.default_rng(300 + T)
-    x1 = rng.standard_normal((T, 512)).astype(np.float32) * 1.3 + 0.2
-    if dt == "bf16":
-        x1 = S.round_to_bf16(x1)
+    x1 = rng.standard_normal((T, 512)).astype(np.float32) * 1.3 + 0.2   # fp32 residual
     w = _weights(301, dt)
     td = BF if dt == "bf16" else F32
     ws = poisoned_workspace(T, 1, dt)
     xn2 = torch.empty(T, 512, dtype=td, device="cuda")
     idx = torch.empty(T, 2, dtype=torch.int32, device="cuda")
     wt = torch.empty(T, 2, dtype=F32, device="cuda")
-    ptl.gate(dev(x1, td), xn2, idx, wt, ptl.to_device_layer(w, dt), ws)
+    ptl.gate(dev(x1, F32), xn2, idx, wt, ptl.to_device_layer(w, dt), ws)
     torch.cuda.synchronize()
     xn2_ref = O.layer_norm(x1, w["ln2_g"], w["ln2_b"])
     p = O.gate_probs(xn2_ref, w["w_gate"], w["b_gate"])
@@ -197,9 +195,9 @@ def test_route_build_rejects_bad_expert_id():
 def test_moe(dt, T, kind):
     rng = np.random.default_rng(500 + T)
     xn2 = rng.standard_normal((T, 512)).astype(np.float32)
-    res = rng.standard_normal((T, 512)).astype(np.float32)
+    res = rng.standard_normal((T, 512)).astype(np.float32)       # fp32 residual (x1)
     if dt == "bf16":
-        xn2, res = S.round_to_bf16(xn2), S.round_to_bf16(res)
+        xn2 = S.round_to_bf16(xn2)
     idx, wts = random_topk(rng, T)
     if kind == "skewed":
         idx[:, 0] = 0
@@ -208,7 +206,7 @@ def test_moe(dt, T, kind):
     td = BF if dt == "bf16" else F32
     ws = poisoned_workspace(T, 1, dt)
     out = torch.full((T, 512), float("nan"), dtype=td, device="cuda")
-    ptl.moe(dev(xn2, td), dev(idx, torch.int32), dev(wts, F32), dev(res, td), out,
+    ptl.moe(dev(xn2, td), dev(idx, torch.int32), dev(wts, F32), dev(res, F32), out,
             ptl.to_device_layer(w, dt), ws)
     torch.cuda.synchronize()
     assert ptl.last_device_error(ws) == 0
