@@ -230,6 +230,37 @@ typedef struct {
 /* Installs (or, with NULL, removes) the calling thread's trace. */
 void ptl_set_trace(ptl_trace* trace);
 
+/* ---- Attention without any device allocation. ----
+ * Some callers cannot allocate device memory: host programs that own all of
+ * device memory through their own pool or budget and hand a library no
+ * allocator, and latency-critical loops that cannot afford cudaMalloc, which
+ * may synchronise the whole device.  ptl_attention_noalloc computes what
+ * ptl_attention computes (same arguments, no workspace): its only scratch,
+ * the device error word and the attention work list, lives in one fixed
+ * array of PTL_NOALLOC_SCRATCH_BYTES bytes in the library's device memory,
+ * which every GPU that loads the library holds until the process exits.
+ * It allocates nothing and calls no allocating routine.
+ *   - Limits: total_tokens <= PTL_NOALLOC_MAX_TOKENS and num_users <=
+ *     PTL_NOALLOC_MAX_USERS; larger requests return PTL_ERR_SHAPE and launch
+ *     nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device uses the same array, which keeps the previous
+ *     call's contents (each call clears what must start at zero).  Calls
+ *     that can overlap on the GPU -- on different streams with no ordering
+ *     between them -- race on the array; do not issue them.
+ *   - device_status (nullable, device int32, 4-byte aligned) receives the
+ *     call's device-side status: PTL_OK, or PTL_ERR_BAD_OFFSETS for a
+ *     cu_seqlens that is not 0-based, non-decreasing and ending at T.
+ * The pages describe no such entry point; it has no counterpart there. */
+#define PTL_NOALLOC_MAX_TOKENS 65536
+#define PTL_NOALLOC_MAX_USERS 4096
+#define PTL_NOALLOC_SCRATCH_BYTES 49152
+ptl_status ptl_attention_noalloc(const void* qkv, void* attn, const int32_t* cu_seqlens,
+                                 int32_t num_users, int64_t total_tokens, ptl_dtype dt,
+                                 int32_t* device_status, void* stream);
+
 /* Synchronises `stream`, returns the status recorded in the workspace error
  * word by earlier calls on that workspace (PTL_OK if none) and clears it. */
 ptl_status ptl_last_device_error(void* workspace, size_t ws_bytes, void* stream);

@@ -98,6 +98,9 @@ _SIGS = {
                   ctypes.c_void_p], ctypes.c_int),
     "ptl_last_device_error": ([ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
     "ptl_set_trace": ([ctypes.POINTER(Trace)], None),
+    "ptl_attention_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                               ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
+                              ctypes.c_int),
 }
 
 
@@ -284,6 +287,18 @@ def head(h, head_weights, pred_mask, probs, n_pred, workspace, stream=None):
                           h.shape[0], _dt(h.dtype), _ptr(workspace), workspace.numel(),
                           _stream(stream)), "ptl_head")
     return probs
+
+
+def attention_noalloc(qkv, attn, cu_seqlens, device_status=None, stream=None):
+    """ptl_attention_noalloc: the attention step for callers that cannot
+    allocate device memory (no workspace; scratch in a fixed array inside the
+    library).  device_status, if given, is a device int32 tensor that
+    receives the call's device-side status."""
+    _check(lib().ptl_attention_noalloc(_ptr(qkv), _ptr(attn), _ptr(cu_seqlens),
+                                       cu_seqlens.numel() - 1, qkv.shape[0], _dt(qkv.dtype),
+                                       _ptr(device_status), _stream(stream)),
+           "ptl_attention_noalloc")
+    return attn
 
 
 def last_device_error(workspace, stream=None) -> int:
