@@ -77,9 +77,10 @@ class NearTieChooser:
     slot 0 not below slot 1 by more than `margin`.  Any other difference is
     recorded as a violation: the result there is unique and must match."""
 
-    def __init__(self, gpu_idx_per_layer, margin):
+    def __init__(self, gpu_idx_per_layer, margin, later_margin=None):
         self.gpu = [np.asarray(g) for g in gpu_idx_per_layer]
         self.margin = margin
+        self.later_margin = margin if later_margin is None else later_margin
         self.violations = []
         self.followed = []
 
@@ -89,13 +90,16 @@ class NearTieChooser:
         if not diff.any():
             self.followed.append(0)
             return idx
+        margin = self.margin if layer == 0 else self.later_margin
         ps = -np.sort(-p, axis=1)
         pg = np.take_along_axis(p, g, axis=1)
-        valid = np.all(pg >= ps[:, 1:2] - self.margin, axis=1) & (pg[:, 0] >= pg[:, 1] - self.margin)
+        valid = np.all(pg >= ps[:, 1:2] - margin, axis=1) & (pg[:, 0] >= pg[:, 1] - margin)
         valid &= g[:, 0] != g[:, 1]
         bad = diff & ~valid
         if bad.any():
-            self.violations.append((layer, np.where(bad)[0][:10].tolist(), int(bad.sum())))
+            gap = (ps[:, 1] - ps[:, 2])[bad]
+            self.violations.append((layer, np.where(bad)[0][:10].tolist(), int(bad.sum()),
+                                    float(gap.max())))
         use = diff & valid
         self.followed.append(int(use.sum()))
         out = idx.copy()
