@@ -247,7 +247,7 @@ def run_ours(args):
     with torch.cuda.graph(graph, stream=stream):
         step()
     torch.cuda.synchronize()
-    launches_per_step = 1 + 8 * n_layers + (2 if head is not None else 0)
+    launches_per_step = 1 + 9 * n_layers + (2 if head is not None else 0)
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
@@ -323,7 +323,8 @@ def run_ours(args):
         "attention": ("tensor", attn_fl),
         "gemm_out": ("tensor", 2 * T * 512 * 512),
         "gemm_expert1": ("tensor", 2 * (2 * T) * 512 * 1024),
-        "gemm_expert2_combine": ("tensor", 2 * (2 * T) * 1024 * 512),
+        "gemm_expert2": ("tensor", 2 * (2 * T) * 1024 * 512),
+        "combine": ("hbm", T * (2 * 1024 + 2048 + 1024 + 16)),
         "gate": ("hbm", T * (1024 + 1024 + 16)),
         "layernorm": ("hbm", T * 2048),
         "route": ("hbm", T * 24),

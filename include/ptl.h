@@ -214,9 +214,10 @@ typedef enum {
   PTL_KERNEL_GATE = 6,         /* LayerNorm2 + gate + top-2 */
   PTL_KERNEL_ROUTE = 7,        /* route counting sort (and per-chunk counts) */
   PTL_KERNEL_GEMM_EXPERT1 = 8, /* expert GEMM1 + ReLU (gathered rows) */
-  PTL_KERNEL_GEMM_EXPERT2 = 9, /* expert GEMM2 + top-2 combine + residual */
+  PTL_KERNEL_GEMM_EXPERT2 = 9, /* expert GEMM2 (per-route outputs) */
   PTL_KERNEL_HEAD = 10,        /* prediction head + compaction */
   PTL_KERNEL_COPY = 11,        /* debug-output copies */
+  PTL_KERNEL_COMBINE = 12,     /* weighted top-2 combine + residual */
   PTL_KERNEL_END = 99
 } ptl_kernel_kind;
 

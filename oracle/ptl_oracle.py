@@ -235,7 +235,8 @@ def moe_routed(xn2, idx, w, w1, b1, w2, b2, hidden_round=None):
     in route-major row r = 2 t + k; token t's output is w[t,0] y[2t] +
     w[t,1] y[2t+1].  Returns (moe_out [T, D], y [2T, D], hidden per route
     [2T, F] in slot order).  hidden_round, if given, is applied to the
-    hidden layer (the bf16 storage mode of layer_forward)."""
+    hidden layer and to each route's output before the weighted sum (the
+    bf16 storage mode of layer_forward)."""
     xn2 = _f64(xn2)
     T, D = xn2.shape
     E = np.asarray(w1).shape[0]
@@ -252,7 +253,8 @@ def moe_routed(xn2, idx, w, w1, b1, w2, b2, hidden_round=None):
         if hidden_round is not None:
             h = hidden_round(h)
         hidden[off[e]:off[e + 1]] = h
-        y[routes] = linear(h, w2[e], b2[e])
+        ye = linear(h, w2[e], b2[e])
+        y[routes] = ye if hidden_round is None else hidden_round(ye)
     w = _f64(w)
     out = w[:, 0:1] * y[0::2] + w[:, 1:2] * y[1::2]
     return out, y, hidden
@@ -277,7 +279,8 @@ def layer_forward(x, cu_seqlens, wts, return_intermediates=False, storage=None, 
     storage=None computes everything in float64.  storage='bf16' rounds to
     bfloat16 the activations a bf16 pipeline stores between its steps -- the
     LayerNorm1 output, q/k/v, the attention output, the LayerNorm2 output fed
-    to the experts, the expert hidden layer and the layer output -- while the
+    to the experts, the expert hidden layer, each route's expert output and
+    the layer output -- while the
     residual x1 inside the layer stays unrounded (an fp32 buffer in such a
     pipeline), the gate sees the unrounded LayerNorm2 output and all
     arithmetic stays float64.  It follows the same definition; only the stored values

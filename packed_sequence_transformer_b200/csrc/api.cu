@@ -51,6 +51,20 @@ bool map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D fp32 tensor map, box = box_rows x box_cols (box_cols * 4 bytes = 128).
+bool map_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride_bytes,
+             uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 ptl_status device_ok() {
   static int cache[64];  // 0 unknown, 1 ok, 2 unsupported
   int dev = 0;
@@ -152,11 +166,12 @@ ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_wei
   if (c.dt == PTL_BF16) {
     mark(c.st, PTL_KERNEL_LAYERNORM);
     PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mo;
     if (!map_bf16(&ma, c.ws + c.L.xn, D, T, D * 2, 64, 128)) return PTL_ERR_CUDA;
     if (!map_bf16(&mb, w->w_qkv, D, QKV_N, D * 2, 64, QKV_BN)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mo, qkv, QKV_N, T, QKV_N * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_QKV);
-    PTL_TRY(launch_gemm_qkv(ma, mb, F32(w->b_qkv), qkv, T, c.err, c.st));
+    PTL_TRY(launch_gemm_qkv(ma, mb, mo, F32(w->b_qkv), qkv, T, c.err, c.st));
   } else {
     mark(c.st, PTL_KERNEL_LAYERNORM);
     PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));
@@ -183,11 +198,12 @@ ptl_status step_attention(const Call& c, const void* qkv, void* attn, const int3
 
 ptl_status step_out(const Call& c, const void* attn, const void* x, void* x1, const ptl_layer_weights* w) {
   if (c.dt == PTL_BF16) {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mo;
     if (!map_bf16(&ma, attn, D, c.T, D * 2, 64, 128)) return PTL_ERR_CUDA;
     if (!map_bf16(&mb, w->w_o, D, D, D * 2, 64, OUT_BN)) return PTL_ERR_CUDA;
+    if (!map_f32(&mo, x1, D, c.T, D * 4, 32, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_OUT);
-    PTL_TRY(launch_gemm_out(ma, mb, F32(w->b_o), x, x1, c.T, c.err, c.st));
+    PTL_TRY(launch_gemm_out(ma, mb, mo, F32(w->b_o), x, x1, c.T, c.err, c.st));
   } else {
     mark(c.st, PTL_KERNEL_GEMM_OUT);
     PTL_TRY(launch_gemm_f32(1, static_cast<const float*>(attn), D, F32(w->w_o), F32(w->b_o),
@@ -201,34 +217,39 @@ ptl_status step_gate(const Call& c, const void* x1, void* xn2, int32_t* idx, flo
                      const ptl_layer_weights* w) {
   mark(c.st, PTL_KERNEL_GATE);
   PTL_TRY(launch_gate(x1, F32(w->ln2_g), F32(w->ln2_b), F32(w->w_gate), F32(w->b_gate), xn2, idx, wout,
-                      at<int32_t>(c, c.L.chunk_cnt), at<int32_t>(c, c.L.comb_cnt), c.T, c.dt, c.st));
+                      at<int32_t>(c, c.L.chunk_cnt), c.T, c.dt, c.st));
   return PTL_OK;
 }
 
-// Routes + both expert GEMMs + combine + residual.  chunk counts and the
-// cleared combine counters must already be in the workspace.
+// Routes + both expert GEMMs + combine + residual.  The per-chunk expert
+// counts must already be in the workspace.
 ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const float* wts,
                     const void* resid, void* out, const ptl_layer_weights* w, int32_t* dbg_perm,
                     int32_t* dbg_off) {
   mark(c.st, PTL_KERNEL_ROUTE);
   PTL_TRY(launch_route(idx, c.T, c.L, c.ws, dbg_perm, dbg_off, c.st));
   if (c.dt == PTL_BF16) {
-    CUtensorMap m1, m2, mh;
+    CUtensorMap m1, m2, mh, my;
     if (!map_bf16(&m1, w->w1, D, uint64_t(E) * F, D * 2, 64, MOE1_BN)) return PTL_ERR_CUDA;
     if (!map_bf16(&m2, w->w2, F, uint64_t(E) * D, F * 2, 64, GEMM2_BN)) return PTL_ERR_CUDA;
     if (!map_bf16(&mh, c.ws + c.L.hbuf, F, c.L.padded_rows, F * 2, 64, 128)) return PTL_ERR_CUDA;
+    if (!map_bf16(&my, c.ws + c.L.ybuf, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
-    PTL_TRY(launch_gemm_moe1(m1, m1, F32(w->b1), xn2, c.L, c.ws, c.st));
+    PTL_TRY(launch_gemm_moe1(m1, mh, F32(w->b1), xn2, c.L, c.ws, c.st));
     mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
-    PTL_TRY(launch_gemm_moe2(mh, m2, F32(w->b2), resid, wts, out, c.L, c.ws, c.st));
+    PTL_TRY(launch_gemm_moe2(mh, m2, my, F32(w->b2), c.L, c.ws, c.st));
+    mark(c.st, PTL_KERNEL_COMBINE);
+    PTL_TRY(launch_combine_bf16(c.ws + c.L.ybuf, at<int32_t>(c, c.L.pos), wts,
+                                static_cast<const float*>(resid), out, c.T, c.err, c.st));
   } else {
     mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
     PTL_TRY(launch_gemm_f32(2, static_cast<const float*>(xn2), D, F32(w->w1), F32(w->b1), nullptr,
                             at<float>(c, c.L.hbuf), F, 0, F, D, c.L, c.ws, c.st));
     mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
     PTL_TRY(launch_gemm_f32(3, at<float>(c, c.L.hbuf), F, F32(w->w2), F32(w->b2), nullptr,
-                            at<float>(c, c.L.ystage), D, 0, D, F, c.L, c.ws, c.st));
-    PTL_TRY(launch_combine_f32(at<float>(c, c.L.ystage), wts, static_cast<const float*>(resid),
+                            at<float>(c, c.L.ybuf), D, 0, D, F, c.L, c.ws, c.st));
+    mark(c.st, PTL_KERNEL_COMBINE);
+    PTL_TRY(launch_combine_f32(at<float>(c, c.L.ybuf), wts, static_cast<const float*>(resid),
                                static_cast<float*>(out), c.T, c.err, c.st));
   }
   return PTL_OK;
@@ -453,10 +474,6 @@ ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w
   EndMark end_mark{c.st};
   mark(c.st, PTL_KERNEL_ROUTE);
   PTL_TRY(launch_chunk_hist(topk_idx, c.T, at<int32_t>(c, c.L.chunk_cnt), c.err, c.st));
-  mark(c.st, PTL_KERNEL_CLEAR);
-  if (cudaMemsetAsync(c.ws + c.L.comb_cnt, 0, sizeof(int32_t) * size_t(c.T) * GEMM2_NT, c.st) !=
-      cudaSuccess)
-    return PTL_ERR_CUDA;
   return step_moe(c, xn2, topk_idx, topk_w, residual, out, w, nullptr, nullptr);
 }
 

@@ -20,8 +20,7 @@ constexpr int QKV_N = 3 * D;       // 1536
 constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
 constexpr int MOE_BM = 128;        // rows per expert tile (padding granule)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
-constexpr int GEMM2_BN = 256;      // N tile of the second expert GEMM
-constexpr int GEMM2_NT = D / GEMM2_BN;  // combine counters per token
+constexpr int GEMM2_BN = 128;      // N tile of the second expert GEMM
 constexpr float LN_EPS = 1e-5f;
 constexpr float LOGIT_CLAMP = 15.0f;
 
@@ -43,12 +42,14 @@ struct WsLayout {
   size_t wgt;         // f32 [T][2]
   size_t chunk_cnt;   // int32 [n_chunks][8]
   size_t perm;        // int32 [2T]
+  size_t pos;         // int32 [2T]          route -> padded expert row
   size_t rowroute;    // int32 [2T + 8*128]   padded expert rows -> route (or -1)
   size_t tiles;       // int2 [max_tiles]     (expert, first padded row)
   size_t route_meta;  // int32 [32]: [0] n_tiles, [1..9] off, [10..18] padded off
   size_t hbuf;        // dt [2T + 8*128][1024]  expert hidden rows (padded layout)
-  size_t ystage;      // f32 [2T][512]      per-route expert outputs awaiting combine
-  size_t comb_cnt;    // int32 [T][GEMM2_NT] combine arrival counters
+  size_t ybuf;        // per-route expert outputs awaiting the combine: bf16 build
+                      // [2T + 8*128][512] bf16 in padded row order, fp32 build
+                      // [2T][512] f32 in route order
   size_t head_p;      // f32 [T]            head probabilities before compaction
   size_t total;
   int64_t T;
@@ -93,12 +94,12 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->wgt = take(4 * T * K);
   L->chunk_cnt = take(4 * L->n_chunks * E);
   L->perm = take(4 * 2 * T);
+  L->pos = take(4 * 2 * T);
   L->rowroute = take(4 * L->padded_rows);
   L->tiles = take(sizeof(int2) * L->max_tiles);
   L->route_meta = take(4 * 32);
   L->hbuf = take(es * L->padded_rows * F);
-  L->ystage = take(4 * 2 * T * D);
-  L->comb_cnt = take(4 * T * GEMM2_NT);
+  L->ybuf = take(dt == PTL_BF16 ? 2 * L->padded_rows * D : 4 * 2 * T * D);
   L->head_p = take(4 * T);
   L->total = o;
   return true;

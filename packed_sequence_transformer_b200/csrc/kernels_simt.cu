@@ -84,10 +84,16 @@ __device__ __forceinline__ void layer_norm16(float (&v)[16], const float* __rest
     q += v[j] * v[j];
   }
   const float rstd = rsqrtf(warp_sum(q) * (1.0f / D) + LN_EPS);
+  // the lane's elements come in groups of 4 consecutive columns
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int c = Row16<T>::elem(lane, j);
-    v[j] = v[j] * rstd * __ldg(g + c) + __ldg(b + c);
+  for (int qd = 0; qd < 4; ++qd) {
+    const int c = Row16<T>::elem(lane, 4 * qd);
+    const float4 g4 = __ldg(reinterpret_cast<const float4*>(g + c));
+    const float4 b4 = __ldg(reinterpret_cast<const float4*>(b + c));
+    v[4 * qd + 0] = v[4 * qd + 0] * rstd * g4.x + b4.x;
+    v[4 * qd + 1] = v[4 * qd + 1] * rstd * g4.y + b4.y;
+    v[4 * qd + 2] = v[4 * qd + 2] * rstd * g4.z + b4.z;
+    v[4 * qd + 3] = v[4 * qd + 3] * rstd * g4.w + b4.w;
   }
 }
 
@@ -192,6 +198,11 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
 // atomics; the token's combine counters for the MoE are cleared.
 constexpr int GATE_WARPS = 16;
 
+__device__ __forceinline__ uint32_t sm_pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 // Sums a[0..7] over the warp and leaves expert (lane >> 2)'s total in a[0]:
 // each exchange hands half of the remaining partial sums to the partner lane
 // (4 + 2 + 1 shuffles), then two more butterflies finish the sum.
@@ -221,12 +232,29 @@ __device__ __forceinline__ float warp_reduce_scatter8(float (&a)[E], int lane) {
   return a[0];
 }
 
+// Stores the lane's 16 LayerNorm2 values (fp32 lane layout: 4 groups of 4
+// consecutive columns at q*128 + lane*4) in the output dtype; a warp writes
+// each group as one contiguous 256-byte (bf16) or 512-byte (fp32) segment.
+__device__ __forceinline__ void store_row16_groups(__nv_bfloat16* row, int lane, const float (&v)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint2 u;
+    u.x = sm_pack_bf16x2(v[4 * q], v[4 * q + 1]);
+    u.y = sm_pack_bf16x2(v[4 * q + 2], v[4 * q + 3]);
+    *reinterpret_cast<uint2*>(row + q * 128 + lane * 4) = u;
+  }
+}
+__device__ __forceinline__ void store_row16_groups(float* row, int lane, const float (&v)[16]) {
+  Row16<float>::store(row, lane, v);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
     const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
     const float* __restrict__ wg, const float* __restrict__ bg, T* __restrict__ xn2,
-    int32_t* __restrict__ idx, float* __restrict__ wout, int32_t* __restrict__ chunk_cnt,
-    int32_t* __restrict__ comb_cnt, int T_) {
+    int32_t* __restrict__ idx, float* __restrict__ wout, int32_t* __restrict__ chunk_cnt, int T_) {
+  // gate weights [8][512] in shared memory; lane l reads columns q*128 + 4l..4l+3,
+  // i.e. consecutive 16-byte words across the warp (no bank conflicts)
   __shared__ __align__(16) float s_wg[E * D];
   for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
     reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
@@ -234,26 +262,17 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   for (int t = blockIdx.x * GATE_WARPS + warp; t < T_; t += gridDim.x * GATE_WARPS) {
-    // x1 (fp32) is read in the output dtype's lane layout so that the LN2
-    // values land in the registers the xn2 store and the gate dots expect
     float v[16];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<T>::elem(lane, 4 * q)));
-      v[4 * q] = f.x;
-      v[4 * q + 1] = f.y;
-      v[4 * q + 2] = f.z;
-      v[4 * q + 3] = f.w;
-    }
-    layer_norm16<T>(v, g, b, lane);
-    Row16<T>::store(xn2 + size_t(t) * D, lane, v);
+    Row16<float>::load(x1 + size_t(t) * D, lane, v);
+    layer_norm16<float>(v, g, b, lane);
+    store_row16_groups(xn2 + size_t(t) * D, lane, v);
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       float s = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float4 w4 = *reinterpret_cast<const float4*>(s_wg + e * D + Row16<T>::elem(lane, 4 * q));
+        const float4 w4 = *reinterpret_cast<const float4*>(s_wg + e * D + q * 128 + lane * 4);
         s += v[4 * q] * w4.x + v[4 * q + 1] * w4.y + v[4 * q + 2] * w4.z + v[4 * q + 3] * w4.w;
       }
       acc[e] = s;
@@ -293,7 +312,6 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
       atomicAdd(&chunk_cnt[(t >> 7) * E + e0], 1);
       atomicAdd(&chunk_cnt[(t >> 7) * E + e1], 1);
     }
-    if (comb_cnt && lane < GEMM2_NT) comb_cnt[size_t(t) * GEMM2_NT + lane] = 0;
   }
 }
 
@@ -325,9 +343,9 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restri
 // block 0, the padding (-1), the expert tile list and the offsets.
 __global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
     const int32_t* __restrict__ idx, int n_routes, const int32_t* __restrict__ chunk_cnt,
-    int32_t* __restrict__ perm, int32_t* __restrict__ rowroute, int2* __restrict__ tiles,
-    int32_t* __restrict__ meta, int32_t* __restrict__ dbg_perm, int32_t* __restrict__ dbg_off,
-    const int32_t* err) {
+    int32_t* __restrict__ perm, int32_t* __restrict__ pos, int32_t* __restrict__ rowroute,
+    int2* __restrict__ tiles, int32_t* __restrict__ meta, int32_t* __restrict__ dbg_perm,
+    int32_t* __restrict__ dbg_off, const int32_t* err) {
   __shared__ int32_t s_red[ROUTE_CHUNK / 32][2 * E];
   __shared__ int32_t s_pre[E], s_tot[E], s_off[E + 1], s_poff[E + 1];
   __shared__ int32_t s_wcnt[ROUTE_CHUNK / 32][E];
@@ -390,6 +408,7 @@ __global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
     perm[s_off[e] + j] = r;
     if (dbg_perm) dbg_perm[s_off[e] + j] = r;
     rowroute[s_poff[e] + j] = r;
+    pos[r] = s_poff[e] + j;
   }
   if (c == 0) {
     for (int ee = 0; ee < E; ++ee) {
@@ -558,7 +577,38 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
   }
 }
 
-// out[t] = (x1[t] + w[t][0] * y[2t]) + w[t][1] * y[2t+1], fp32.
+// bf16 build: out[t] = (x1[t] + w[t][0] y(2t)) + w[t][1] y(2t+1) in fp32,
+// rounded once; y(r) is row pos[r] of the padded per-route expert outputs
+// (bf16).  One warp per token, 16-byte loads.
+__global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* __restrict__ ybuf,
+                                                           const int32_t* __restrict__ pos,
+                                                           const float* __restrict__ w,
+                                                           const float* __restrict__ x1,
+                                                           __nv_bfloat16* __restrict__ out, int T_,
+                                                           const int32_t* err) {
+  if (has_error(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T_) return;
+  const int2 pr = __ldg(reinterpret_cast<const int2*>(pos) + t);
+  const float2 wt = __ldg(reinterpret_cast<const float2*>(w) + t);
+  float y0[16], y1[16], xr[16], o[16];
+  Row16<__nv_bfloat16>::load(ybuf + size_t(pr.x) * D, lane, y0);
+  Row16<__nv_bfloat16>::load(ybuf + size_t(pr.y) * D, lane, y1);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<__nv_bfloat16>::elem(lane, 4 * q)));
+    xr[4 * q] = f.x;
+    xr[4 * q + 1] = f.y;
+    xr[4 * q + 2] = f.z;
+    xr[4 * q + 3] = f.w;
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j] = (xr[j] + wt.x * y0[j]) + wt.y * y1[j];
+  Row16<__nv_bfloat16>::store(out + size_t(t) * D, lane, o);
+}
+
+// fp32 build: out[t] = (x1[t] + w[t][0] * y[2t]) + w[t][1] * y[2t+1].
 __global__ void __launch_bounds__(256) combine_f32_kernel(const float* __restrict__ y,
                                                           const float* __restrict__ w,
                                                           const float* __restrict__ x1,
@@ -655,8 +705,8 @@ int launch_layernorm(const void* x, const float* g, const float* b, void* y, int
 }
 
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
-                void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int32_t* comb_cnt, int T,
-                ptl_dtype dt, cudaStream_t st) {
+                void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
+                cudaStream_t st) {
   // chunk counts are accumulated with atomics: clear them first
   const size_t n_chunk_bytes = sizeof(int32_t) * E * size_t((T + 127) / 128);
   if (cudaMemsetAsync(chunk_cnt, 0, n_chunk_bytes, st) != cudaSuccess) return -1;
@@ -665,11 +715,11 @@ int launch_gate(const void* x1, const float* g, const float* b, const float* wg,
   if (dt == PTL_BF16)
     gate_kernel<__nv_bfloat16><<<blocks, GATE_WARPS * 32, 0, st>>>(
         static_cast<const float*>(x1), g, b, wg, bg, static_cast<__nv_bfloat16*>(xn2), idx, w,
-        chunk_cnt, comb_cnt, T);
+        chunk_cnt, T);
   else
     gate_kernel<float><<<blocks, GATE_WARPS * 32, 0, st>>>(static_cast<const float*>(x1), g, b, wg,
                                                            bg, static_cast<float*>(xn2), idx, w,
-                                                           chunk_cnt, comb_cnt, T);
+                                                           chunk_cnt, T);
   return PTL_LAUNCH_CHECK();
 }
 
@@ -684,7 +734,8 @@ int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t
   const int n = 2 * T;
   route_kernel<<<(n + ROUTE_CHUNK - 1) / ROUTE_CHUNK, ROUTE_CHUNK, 0, st>>>(
       idx, n, reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
-      reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.rowroute),
+      reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.pos),
+      reinterpret_cast<int32_t*>(ws + L.rowroute),
       reinterpret_cast<int2*>(ws + L.tiles), reinterpret_cast<int32_t*>(ws + L.route_meta),
       dbg_perm, dbg_off, reinterpret_cast<const int32_t*>(ws + L.err));
   return PTL_LAUNCH_CHECK();
@@ -722,6 +773,13 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
     case 2: gemm_f32_kernel<2><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
     default: gemm_f32_kernel<3><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
   }
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
+                        int T, const int32_t* err, cudaStream_t st) {
+  combine_bf16_kernel<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(ybuf), pos, w, x1,
+                                                  static_cast<__nv_bfloat16*>(out), T, err);
   return PTL_LAUNCH_CHECK();
 }
 

@@ -10,7 +10,7 @@
 
 namespace ptl {
 
-constexpr int QKV_BN = 256;
+constexpr int QKV_BN = 192;
 constexpr int OUT_BN = 128;
 constexpr int MOE1_BN = 256;
 
@@ -19,8 +19,8 @@ int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st);
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
-                void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int32_t* comb_cnt, int T,
-                ptl_dtype dt, cudaStream_t st);
+                void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
+                cudaStream_t st);
 int launch_chunk_hist(const int32_t* idx, int T, int32_t* chunk_cnt, int32_t* err, cudaStream_t st);
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
                  int32_t* dbg_off, cudaStream_t st);
@@ -29,20 +29,22 @@ int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, 
 int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const float* bias,
                     const float* R, float* C, int ldc, int M, int N, int Kd, const WsLayout& L,
                     const char* ws, cudaStream_t st);
+int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
+                        int T, const int32_t* err, cudaStream_t st);
 int launch_combine_f32(const float* y, const float* w, const float* x1, float* out, int T,
                        const int32_t* err, cudaStream_t st);
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
                     const char* ws, cudaStream_t st);
 
 // gemm_tc.cu (bf16, tcgen05)
-int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const float* bias, void* qkv, int T,
-                    int32_t* err, cudaStream_t st);
-int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const float* bias, const void* x,
-                    void* x1, int T, int32_t* err, cudaStream_t st);
-int launch_gemm_moe1(const CUtensorMap& dummyA, const CUtensorMap& w1, const float* b1, const void* xn2,
+int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorMap& qkv_out,
+                    const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st);
+int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
+                    const float* bias, const void* x, void* x1, int T, int32_t* err, cudaStream_t st);
+int launch_gemm_moe1(const CUtensorMap& w1, const CUtensorMap& hbuf_out, const float* b1, const void* xn2,
                      const WsLayout& L, char* ws, cudaStream_t st);
-int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const float* b2, const void* x1,
-                     const float* topk_w, void* out, const WsLayout& L, char* ws, cudaStream_t st);
+int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUtensorMap& ybuf_out,
+                     const float* b2, const WsLayout& L, char* ws, cudaStream_t st);
 
 // attn_tc.cu (bf16, tcgen05)
 int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,

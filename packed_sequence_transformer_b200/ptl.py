@@ -59,8 +59,8 @@ class Trace(ctypes.Structure):
 
 
 KERNEL_KINDS = {0: "clear", 1: "worklist", 2: "layernorm", 3: "gemm_qkv", 4: "attention",
-                5: "gemm_out", 6: "gate", 7: "route", 8: "gemm_expert1", 9: "gemm_expert2_combine",
-                10: "head", 11: "copy", 99: "end"}
+                5: "gemm_out", 6: "gate", 7: "route", 8: "gemm_expert1", 9: "gemm_expert2",
+                10: "head", 11: "copy", 12: "combine", 99: "end"}
 
 _lib = None
 _SIGS = {
