@@ -155,10 +155,13 @@ inline T* at(const Call& c, size_t off) { return reinterpret_cast<T*>(c.ws + off
     if ((expr) != 0) return PTL_ERR_CUDA; \
   } while (0)
 
-// Clears the error word: every top-level call reports only its own errors.
+// Clears the error word (every top-level call reports only its own errors)
+// and the per-chunk expert counts that the gate accumulates into (laid out
+// right behind the error word; the first expert GEMM clears them again once
+// the route builder has used them).
 ptl_status begin(const Call& c) {
   mark(c.st, PTL_KERNEL_CLEAR);
-  return cudaMemsetAsync(c.err, 0, sizeof(int32_t), c.st) == cudaSuccess ? PTL_OK : PTL_ERR_CUDA;
+  return cudaMemsetAsync(c.ws, 0, c.L.items, c.st) == cudaSuccess ? PTL_OK : PTL_ERR_CUDA;
 }
 
 ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_weights* w) {

@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(128, 2)
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int item = blockIdx.x / H, h = blockIdx.x % H;
+  pdl_trigger();
+  pdl_wait();  // qkv, the work list and the error word come from earlier kernels
   if (tid == 0) {
     const int skip = (has_error(err) || item >= *item_count) ? 1 : 0;
     s_skip = skip;
@@ -229,10 +231,10 @@ int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, con
       return -1;
     configured = true;
   }
-  attn_tc_kernel<<<unsigned(L.max_items * H), 128, ATT_SMEM, st>>>(
-      qkv_map, cu, reinterpret_cast<const int2*>(ws + L.items),
-      reinterpret_cast<const int32_t*>(ws + L.item_count), static_cast<__nv_bfloat16*>(out),
-      reinterpret_cast<int32_t*>(ws + L.err));
+  if (launch_k(attn_tc_kernel, dim3(unsigned(L.max_items * H)), dim3(128), ATT_SMEM, st, qkv_map, cu,
+               reinterpret_cast<const int2*>(ws + L.items), reinterpret_cast<const int32_t*>(ws + L.item_count),
+               static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err)) != 0)
+    return -1;
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 

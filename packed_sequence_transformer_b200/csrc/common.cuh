@@ -78,6 +78,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
     return at;
   };
   L->err = take(256);
+  L->chunk_cnt = take(4 * L->n_chunks * E);  // right after the error word: cleared together
   L->items = take(sizeof(int2) * L->max_items);
   L->item_count = take(4);
   L->lvl_hist = take(4 * (L->max_levels + 1));
@@ -92,7 +93,6 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->act1 = take(es * T * D);
   L->idx = take(4 * T * K);
   L->wgt = take(4 * T * K);
-  L->chunk_cnt = take(4 * L->n_chunks * E);
   L->perm = take(4 * 2 * T);
   L->pos = take(4 * 2 * T);
   L->rowroute = take(4 * L->padded_rows);
@@ -106,6 +106,15 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
 }
 
 // ---------------------------------------------------------------- device
+// Programmatic dependent launch.  Every kernel of the library is launched so
+// that the next kernel in the stream may start its prologue while this one
+// drains: each kernel first allows its dependents to launch (trigger), and
+// waits for its own predecessor to complete (and its writes to be visible)
+// before it reads anything the predecessor produced.  Every kernel executes
+// the wait on every path, so completion stays transitive along the stream.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void set_error(int32_t* err, int32_t code) {
   atomicCAS(err, 0, code);
 }

@@ -51,6 +51,8 @@ struct GemmTcParams {
   const int32_t* rowroute;       // padded expert row -> route (or -1)
   const int2* tiles;             // (expert, first padded row) per M tile
   const int32_t* meta;           // [0] = number of M tiles
+  int32_t* zero_ptr;             // cleared by CTA 0 once the predecessor is done (may be NULL)
+  int zero_n;
   const __nv_bfloat16* gatherA;  // MOE1: xn2 [T][512]
   int32_t* err;
 };
@@ -140,10 +142,9 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
   __shared__ int s_ntiles;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  // prologue (overlaps the previous kernel's tail): barriers, TMEM, descriptors
   if (threadIdx.x == 0) {
-    int nt = MODE >= G_MOE1 ? p.meta[0] * (p.N_total / BN) : p.n_tiles_dense;
-    if (has_error(p.err)) nt = 0;
-    s_ntiles = nt;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], MODE == G_MOE1 ? 1 + 128 : 1);
       mbar_init(&empty[s], 1);
@@ -154,9 +155,11 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
     }
     fence_mbar_init();
   }
-  __syncthreads();
-  const int ntiles = s_ntiles;
-  if (int(blockIdx.x) >= ntiles) return;
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmOut);
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
@@ -164,13 +167,21 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // inputs, route tables and the error word come from earlier kernels
+  if (threadIdx.x == 0) {
+    int nt = MODE >= G_MOE1 ? p.meta[0] * (p.N_total / BN) : p.n_tiles_dense;
+    if (has_error(p.err)) nt = 0;
+    s_ntiles = nt;
+  }
+  if (p.zero_ptr && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.zero_n; i += blockDim.x) p.zero_ptr[i] = 0;
+  __syncthreads();
+  const int ntiles = s_ntiles;
   const uint32_t tmem = *tmem_slot;
   const int nkb = p.num_kb;
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmB);
       const uint32_t tx = (MODE == G_MOE1 ? 0u : uint32_t(Cfg::A_BYTES)) + uint32_t(Cfg::B_BYTES);
       int it = 0;
       bool ok = true;
@@ -373,7 +384,9 @@ static int launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   }
   int grid = tiles_bound < num_sms() ? tiles_bound : num_sms();
   if (grid < 1) grid = 1;
-  gemm_tc_kernel<BN, MODE><<<grid, MODE == G_MOE1 ? 320 : 192, smem, st>>>(a, b, out, p);
+  if (launch_k(gemm_tc_kernel<BN, MODE>, dim3(grid), dim3(MODE == G_MOE1 ? 320 : 192), smem, st, a, b, out,
+               p) != 0)
+    return -1;
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -419,6 +432,10 @@ int launch_gemm_moe1(const CUtensorMap& w1, const CUtensorMap& hbuf_out, const f
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
   p.gatherA = static_cast<const __nv_bfloat16*>(xn2);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
+  // the route builder (the previous kernel) has consumed the per-chunk expert
+  // counts: clear them for the next gate
+  p.zero_ptr = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
+  p.zero_n = int(L.n_chunks * E);
   // A is gathered by the kernel; the A descriptor slot is unused
   return launch_one<MOE1_BN, G_MOE1>(w1, w1, hbuf_out, p, int(L.max_tiles) * (F / MOE1_BN), st);
 }

@@ -101,6 +101,8 @@ template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) ln_rows_kernel(const TI* __restrict__ x, const float* __restrict__ g,
                                                       const float* __restrict__ b, TO* __restrict__ y,
                                                       int T) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= T) return;
@@ -144,6 +146,8 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
                                                         int2* __restrict__ items, int32_t* item_count,
                                                         int32_t* lvl_hist, int32_t* lvl_start,
                                                         int32_t* lvl_fill, int max_levels, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_bad;
   __shared__ int s_total;
   const int tid = threadIdx.x;
@@ -256,9 +260,11 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
   // gate weights [8][512] in shared memory; lane l reads columns q*128 + 4l..4l+3,
   // i.e. consecutive 16-byte words across the warp (no bank conflicts)
   __shared__ __align__(16) float s_wg[E * D];
+  pdl_trigger();
   for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
     reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
   __syncthreads();
+  pdl_wait();  // x1 comes from the previous kernel
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   for (int t = blockIdx.x * GATE_WARPS + warp; t < T_; t += gridDim.x * GATE_WARPS) {
@@ -319,6 +325,8 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
 // build); out-of-range expert ids set PTL_ERR_SHAPE and are skipped.
 __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ idx, int n_routes,
                                                          int32_t* __restrict__ chunk_cnt, int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t s_hist[E];
   if (threadIdx.x < E) s_hist[threadIdx.x] = 0;
   __syncthreads();
@@ -346,6 +354,8 @@ __global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
     int32_t* __restrict__ perm, int32_t* __restrict__ pos, int32_t* __restrict__ rowroute,
     int2* __restrict__ tiles, int32_t* __restrict__ meta, int32_t* __restrict__ dbg_perm,
     int32_t* __restrict__ dbg_off, const int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t s_red[ROUTE_CHUNK / 32][2 * E];
   __shared__ int32_t s_pre[E], s_tot[E], s_off[E + 1], s_poff[E + 1];
   __shared__ int32_t s_wcnt[ROUTE_CHUNK / 32][E];
@@ -434,6 +444,8 @@ __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, cons
                                                    const float* __restrict__ w,
                                                    const float* __restrict__ bias,
                                                    float* __restrict__ p, int T_) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T_) return;
@@ -455,6 +467,8 @@ __global__ void __launch_bounds__(1024) head_compact_kernel(const float* __restr
                                                             const uint8_t* __restrict__ mask,
                                                             float* __restrict__ probs,
                                                             int32_t* __restrict__ n_pred, int T_) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t s_scan[1024];
   __shared__ int32_t s_carry;
   if (threadIdx.x == 0) s_carry = 0;
@@ -495,6 +509,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        const int2* __restrict__ tiles,
                                                        const int32_t* __restrict__ meta,
                                                        const int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sA[16][64 + 4];
   __shared__ float sB[16][64 + 4];
   __shared__ int s_arow[64];
@@ -586,6 +602,8 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
                                                            const float* __restrict__ x1,
                                                            __nv_bfloat16* __restrict__ out, int T_,
                                                            const int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   if (has_error(err)) return;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -614,6 +632,8 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const float* __restric
                                                           const float* __restrict__ x1,
                                                           float* __restrict__ out, int T_,
                                                           const int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   if (has_error(err)) return;
   const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= size_t(T_) * D) return;
@@ -632,6 +652,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
                                                        const int2* __restrict__ items,
                                                        const int32_t* __restrict__ item_count,
                                                        const int32_t* err) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float sK[64][DH + 1];
   __shared__ float sV[64][DH + 1];
   if (has_error(err)) return;
@@ -683,61 +705,60 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
 #define PTL_LAUNCH_CHECK() (cudaPeekAtLastError() == cudaSuccess ? 0 : -1)
 
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st) {
-  worklist_kernel<<<1, 1024, 0, st>>>(cu, U, T, reinterpret_cast<int2*>(ws + L.items),
+  if (launch_k(worklist_kernel, dim3(1), dim3(1024), 0, st, cu, U, T, reinterpret_cast<int2*>(ws + L.items),
                                       reinterpret_cast<int32_t*>(ws + L.item_count),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_hist),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_start),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_fill), int(L.max_levels),
-                                      reinterpret_cast<int32_t*>(ws + L.err));
+                                      reinterpret_cast<int32_t*>(ws + L.err))) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st) {
   const int blocks = (T + 7) / 8;
-  if (dt == PTL_BF16)
-    ln_rows_kernel<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T);
-  else
-    ln_rows_kernel<float, float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), g, b,
-                                                         static_cast<float*>(y), T);
+  if (dt == PTL_BF16) {
+    if (launch_k(ln_rows_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(blocks), dim3(256), 0, st, 
+        static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T)) return -1;
+  } else {
+    if (launch_k(ln_rows_kernel<float, float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(x), g, b,
+                                                         static_cast<float*>(y), T)) return -1;
+  }
   return PTL_LAUNCH_CHECK();
 }
 
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
                 cudaStream_t st) {
-  // chunk counts are accumulated with atomics: clear them first
-  const size_t n_chunk_bytes = sizeof(int32_t) * E * size_t((T + 127) / 128);
-  if (cudaMemsetAsync(chunk_cnt, 0, n_chunk_bytes, st) != cudaSuccess) return -1;
   int blocks = (T + GATE_WARPS - 1) / GATE_WARPS;
   if (blocks > 148 * 2) blocks = 148 * 2;
-  if (dt == PTL_BF16)
-    gate_kernel<__nv_bfloat16><<<blocks, GATE_WARPS * 32, 0, st>>>(
+  if (dt == PTL_BF16) {
+    if (launch_k(gate_kernel<__nv_bfloat16>, dim3(blocks), dim3(GATE_WARPS * 32), 0, st, 
         static_cast<const float*>(x1), g, b, wg, bg, static_cast<__nv_bfloat16*>(xn2), idx, w,
-        chunk_cnt, T);
-  else
-    gate_kernel<float><<<blocks, GATE_WARPS * 32, 0, st>>>(static_cast<const float*>(x1), g, b, wg,
+        chunk_cnt, T)) return -1;
+  } else {
+    if (launch_k(gate_kernel<float>, dim3(blocks), dim3(GATE_WARPS * 32), 0, st, static_cast<const float*>(x1), g, b, wg,
                                                            bg, static_cast<float*>(xn2), idx, w,
-                                                           chunk_cnt, T);
+                                                           chunk_cnt, T)) return -1;
+  }
   return PTL_LAUNCH_CHECK();
 }
 
 int launch_chunk_hist(const int32_t* idx, int T, int32_t* chunk_cnt, int32_t* err, cudaStream_t st) {
   const int n = 2 * T;
-  chunk_hist_kernel<<<(n + ROUTE_CHUNK - 1) / ROUTE_CHUNK, ROUTE_CHUNK, 0, st>>>(idx, n, chunk_cnt, err);
+  if (launch_k(chunk_hist_kernel, dim3((n + ROUTE_CHUNK - 1) / ROUTE_CHUNK), dim3(ROUTE_CHUNK), 0, st, idx, n, chunk_cnt, err)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
                  int32_t* dbg_off, cudaStream_t st) {
   const int n = 2 * T;
-  route_kernel<<<(n + ROUTE_CHUNK - 1) / ROUTE_CHUNK, ROUTE_CHUNK, 0, st>>>(
+  if (launch_k(route_kernel, dim3((n + ROUTE_CHUNK - 1) / ROUTE_CHUNK), dim3(ROUTE_CHUNK), 0, st, 
       idx, n, reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
       reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.pos),
       reinterpret_cast<int32_t*>(ws + L.rowroute),
       reinterpret_cast<int2*>(ws + L.tiles), reinterpret_cast<int32_t*>(ws + L.route_meta),
-      dbg_perm, dbg_off, reinterpret_cast<const int32_t*>(ws + L.err));
+      dbg_perm, dbg_off, reinterpret_cast<const int32_t*>(ws + L.err))) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
@@ -749,13 +770,14 @@ int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, 
   const float* b = static_cast<const float*>(hw->lnf_b);
   const float* w = static_cast<const float*>(hw->w);
   const float* bias = static_cast<const float*>(hw->b);
-  if (dt == PTL_BF16)
-    head_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(h), g, b, w,
-                                                       bias, p, T);
-  else
-    head_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(h), g, b, w, bias, p, T);
+  if (dt == PTL_BF16) {
+    if (launch_k(head_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(h), g, b, w,
+                                                       bias, p, T)) return -1;
+  } else {
+    if (launch_k(head_kernel<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(h), g, b, w, bias, p, T)) return -1;
+  }
   if (PTL_LAUNCH_CHECK() != 0) return -1;
-  head_compact_kernel<<<1, 1024, 0, st>>>(p, mask, probs, n_pred, T);
+  if (launch_k(head_compact_kernel, dim3(1), dim3(1024), 0, st, p, mask, probs, n_pred, T)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
@@ -767,34 +789,35 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
   const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
   const int32_t* err = reinterpret_cast<const int32_t*>(ws + L.err);
   dim3 grid(mode >= 2 ? unsigned(2 * L.max_tiles) : unsigned((M + 63) / 64), unsigned((N + 63) / 64));
+  int rc = 0;
   switch (mode) {
-    case 0: gemm_f32_kernel<0><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
-    case 1: gemm_f32_kernel<1><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
-    case 2: gemm_f32_kernel<2><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
-    default: gemm_f32_kernel<3><<<grid, 256, 0, st>>>(A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    case 0: rc = launch_k(gemm_f32_kernel<0>, dim3(grid), dim3(256), 0, st, A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    case 1: rc = launch_k(gemm_f32_kernel<1>, dim3(grid), dim3(256), 0, st, A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    case 2: rc = launch_k(gemm_f32_kernel<2>, dim3(grid), dim3(256), 0, st, A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
+    default: rc = launch_k(gemm_f32_kernel<3>, dim3(grid), dim3(256), 0, st, A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;
   }
-  return PTL_LAUNCH_CHECK();
+  return rc != 0 ? -1 : PTL_LAUNCH_CHECK();
 }
 
 int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
                         int T, const int32_t* err, cudaStream_t st) {
-  combine_bf16_kernel<<<(T + 7) / 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(ybuf), pos, w, x1,
-                                                  static_cast<__nv_bfloat16*>(out), T, err);
+  if (launch_k(combine_bf16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(ybuf), pos, w, x1,
+                                                  static_cast<__nv_bfloat16*>(out), T, err)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
 int launch_combine_f32(const float* y, const float* w, const float* x1, float* out, int T,
                        const int32_t* err, cudaStream_t st) {
   const size_t n = size_t(T) * D;
-  combine_f32_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(y, w, x1, out, T, err);
+  if (launch_k(combine_f32_kernel, dim3(unsigned((n + 255) / 256)), dim3(256), 0, st, y, w, x1, out, T, err)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
                     const char* ws, cudaStream_t st) {
-  attn_f32_kernel<<<unsigned(L.max_items * H), 128, 0, st>>>(
+  if (launch_k(attn_f32_kernel, dim3(unsigned(L.max_items * H)), dim3(128), 0, st, 
       qkv, out, cu, reinterpret_cast<const int2*>(ws + L.items),
-      reinterpret_cast<const int32_t*>(ws + L.item_count), reinterpret_cast<const int32_t*>(ws + L.err));
+      reinterpret_cast<const int32_t*>(ws + L.item_count), reinterpret_cast<const int32_t*>(ws + L.err))) return -1;
   return PTL_LAUNCH_CHECK();
 }
 

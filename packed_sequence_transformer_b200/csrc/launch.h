@@ -10,6 +10,25 @@
 
 namespace ptl {
 
+// Launches `kernel` on `st` with programmatic stream serialization, so a
+// captured graph gets programmatic edges and the kernel may launch while its
+// predecessor drains (the kernels call pdl_trigger / pdl_wait).
+template <typename... KArgs, typename... Args>
+inline int launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                    Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? 0 : -1;
+}
+
 constexpr int QKV_BN = 192;
 constexpr int OUT_BN = 128;
 constexpr int MOE1_BN = 256;
