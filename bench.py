@@ -70,6 +70,24 @@ def make_workload(name, rank):
     return c
 
 
+def max_over_ranks(x, world, device="cpu"):
+    """The largest of each rank's `x` (every rank gets it); `x` itself at world 1.
+    The collective runs on `device` (cuda for NCCL, cpu for gloo)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(tokens_per_rank, layers, world, ms_max):
+    """Whole-job throughput: the token-layers all ranks processed (each rank
+    runs its own batch) over the slowest rank's step time."""
+    return tokens_per_rank * layers * world / (ms_max / 1e3)
+
+
 def attention_flops(lengths):
     L = np.asarray(lengths, np.int64)
     return 2048 * int((L * (L + 1) // 2).sum())
@@ -247,7 +265,9 @@ def run_ours(args):
     with torch.cuda.graph(graph, stream=stream):
         step()
     torch.cuda.synchronize()
-    launches_per_step = 1 + 9 * n_layers + (2 if head is not None else 0)
+    # work list + LayerNorm1 of layer 0 + 8 kernels per layer (each layer's
+    # combine writes the next layer's LayerNorm1) + head and its compaction
+    launches_per_step = 1 + 1 + 8 * n_layers + (2 if head is not None else 0)
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
@@ -277,13 +297,8 @@ def run_ours(args):
     barrier()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    ms = statistics.mean(step_ms)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    tokens_layers = T * n_layers * world
-    value = tokens_layers / (ms_max / 1e3)
+    ms_max = max_over_ranks(statistics.mean(step_ms), world, dev)
+    value = job_value(T, n_layers, world, ms_max)
 
     # ---- per-kernel device times: the same step captured with a CUDA event
     # before every launch (event nodes inside the graph), replayed with the
@@ -376,11 +391,7 @@ def run_ours(args):
             if i >= args.warmup:
                 e2e_ms.append(a.elapsed_time(b))
             flush.fill_(float(i))
-    e2e = statistics.mean(e2e_ms)
-    e2e_t = torch.tensor([e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = tokens_layers / (float(e2e_t.item()) / 1e3)
+    e2e_value = job_value(T, n_layers, world, max_over_ranks(statistics.mean(e2e_ms), world, dev))
 
     cpu = None
     if rank == 0 and world == 1:

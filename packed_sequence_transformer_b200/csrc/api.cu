@@ -164,11 +164,16 @@ ptl_status begin(const Call& c) {
   return cudaMemsetAsync(c.ws, 0, c.L.items, c.st) == cudaSuccess ? PTL_OK : PTL_ERR_CUDA;
 }
 
-ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_weights* w) {
+// xn_ready: LayerNorm1 of x is already in the workspace (the previous
+// layer's combine wrote it).
+ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_weights* w,
+                    bool xn_ready = false) {
   const int T = c.T;
   if (c.dt == PTL_BF16) {
-    mark(c.st, PTL_KERNEL_LAYERNORM);
-    PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));
+    if (!xn_ready) {
+      mark(c.st, PTL_KERNEL_LAYERNORM);
+      PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));
+    }
     CUtensorMap ma, mb, mo;
     if (!map_bf16(&ma, c.ws + c.L.xn, D, T, D * 2, 64, 128)) return PTL_ERR_CUDA;
     if (!map_bf16(&mb, w->w_qkv, D, QKV_N, D * 2, 64, QKV_BN)) return PTL_ERR_CUDA;
@@ -226,9 +231,11 @@ ptl_status step_gate(const Call& c, const void* x1, void* xn2, int32_t* idx, flo
 
 // Routes + both expert GEMMs + combine + residual.  The per-chunk expert
 // counts must already be in the workspace.
+// next (bf16 build, nullable): the following layer, whose LayerNorm1 of `out`
+// the combine also writes into the workspace.
 ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const float* wts,
                     const void* resid, void* out, const ptl_layer_weights* w, int32_t* dbg_perm,
-                    int32_t* dbg_off) {
+                    int32_t* dbg_off, const ptl_layer_weights* next = nullptr) {
   mark(c.st, PTL_KERNEL_ROUTE);
   PTL_TRY(launch_route(idx, c.T, c.L, c.ws, dbg_perm, dbg_off, c.st));
   if (c.dt == PTL_BF16) {
@@ -243,7 +250,9 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
     PTL_TRY(launch_gemm_moe2(mh, m2, my, F32(w->b2), c.L, c.ws, c.st));
     mark(c.st, PTL_KERNEL_COMBINE);
     PTL_TRY(launch_combine_bf16(c.ws + c.L.ybuf, at<int32_t>(c, c.L.pos), wts,
-                                static_cast<const float*>(resid), out, c.T, c.err, c.st));
+                                static_cast<const float*>(resid), out, c.T,
+                                next ? F32(next->ln1_g) : nullptr, next ? F32(next->ln1_b) : nullptr,
+                                next ? c.ws + c.L.xn : nullptr, c.err, c.st));
   } else {
     mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
     PTL_TRY(launch_gemm_f32(2, static_cast<const float*>(xn2), D, F32(w->w1), F32(w->b1), nullptr,
@@ -258,17 +267,21 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
   return PTL_OK;
 }
 
+// xn_ready: LayerNorm1 of x is already in the workspace; next (nullable,
+// bf16 build): the following layer of a stack, whose LayerNorm1 the combine
+// computes on the way out.
 ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu,
-                      const ptl_layer_weights* w, const ptl_debug_out* dbg) {
+                      const ptl_layer_weights* w, const ptl_debug_out* dbg, bool xn_ready = false,
+                      const ptl_layer_weights* next = nullptr) {
   ptl_status s;
-  if ((s = step_qkv(c, x, c.ws + c.L.qkv, w)) != PTL_OK) return s;
+  if ((s = step_qkv(c, x, c.ws + c.L.qkv, w, xn_ready)) != PTL_OK) return s;
   if ((s = step_attention(c, c.ws + c.L.qkv, c.ws + c.L.attn, cu)) != PTL_OK) return s;
   if ((s = step_out(c, c.ws + c.L.attn, x, c.ws + c.L.x1, w)) != PTL_OK) return s;
   int32_t* idx = at<int32_t>(c, c.L.idx);
   float* wts = at<float>(c, c.L.wgt);
   if ((s = step_gate(c, c.ws + c.L.x1, c.ws + c.L.xn2, idx, wts, w)) != PTL_OK) return s;
   if ((s = step_moe(c, c.ws + c.L.xn2, idx, wts, c.ws + c.L.x1, out, w, dbg ? dbg->perm : nullptr,
-                    dbg ? dbg->expert_off : nullptr)) != PTL_OK)
+                    dbg ? dbg->expert_off : nullptr, next)) != PTL_OK)
     return s;
   if (dbg && (dbg->topk_idx || dbg->topk_w)) mark(c.st, PTL_KERNEL_COPY);
   if (dbg && dbg->topk_idx &&
@@ -371,7 +384,11 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
   const void* h_in = x;
   for (int i = 0; i < num_layers; ++i) {
     void* h_out = (i == num_layers - 1) ? out : c.ws + ((i & 1) ? c.L.act1 : c.L.act0);
-    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr)) != PTL_OK) return s;
+    // bf16: layer i's combine also writes LayerNorm1 of its output for layer i + 1
+    const bool fuse = c.dt == PTL_BF16;
+    const ptl_layer_weights* next = (fuse && i + 1 < num_layers) ? &layers[i + 1] : nullptr;
+    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr, fuse && i > 0, next)) != PTL_OK)
+      return s;
     h_in = h_out;
   }
   if (head) mark(c.st, PTL_KERNEL_HEAD);

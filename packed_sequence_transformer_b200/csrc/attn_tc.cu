@@ -1,25 +1,36 @@
 // attn_tc.cu -- jagged block-diagonal causal attention on tcgen05.
 //
-// Work item = (user u, query block b, head h): 128 query rows of one user.
-// The items are listed on the device from cu_seqlens, heaviest first (a
-// block b needs b + 1 key blocks: the key loop stops at the diagonal block,
-// so no [S,S] mask and no block above the diagonal is ever touched).
+// A unit of work is (user u, 128-query block b, head h).  Units are listed on
+// the device from cu_seqlens, heaviest first (block b needs b + 1 key blocks:
+// the key loop stops at the diagonal block, so no [S,S] mask is built and no
+// block above the diagonal is touched).  A persistent CTA per SM takes its
+// units in snake order over the grid and splits them between two streams
+// (each unit to the stream with fewer key-block steps so far), one per
+// softmax warpgroup; a stream is a sequence of steps (unit, key block kb) and
+// the two streams' steps are interleaved:
 //
-// Per item (4 warps, thread i <-> query row i <-> TMEM lane i):
-//   TMA: Q tile [128 x 64] once, then per key block K and V tiles [128 x 64]
-//        straight out of the packed qkv rows (128-byte swizzle);
-//   S = Q K^T    tcgen05.mma M=128 N=128 K=16 x4 into TMEM columns [0,128);
-//   softmax      each thread reads its S row from TMEM, masks keys beyond
-//                its own position (and beyond the user), keeps the running
-//                max m and sum l in fp32 (base-2 exponent, scale folded in),
-//                and writes P = exp2(s - m) in bf16 into shared memory in the
-//                K-major swizzled layout the tensor core reads;
-//   PV = P V     tcgen05.mma M=128 N=64 K=16 x8 (V is the MN-major operand)
-//                into TMEM columns [128,192); the thread folds it into its
-//                fp32 output row, O = O * exp2(m_old - m_new) + PV.
-// Finally O / l is written as bf16 for the rows that belong to the user.
-// Tiles that run past the user (into the next user or past T) are masked;
-// TMA zero-fills rows past T.  All waits are bounded.
+//   warp 0      TMA producer: the Q tile [128 x 64] of each stream's current
+//               unit, and per step the K and V tiles [128 x 64] through a
+//               3-deep ring, straight from the packed qkv rows (128-byte
+//               swizzle);
+//   warp 1      MMA issuer: for a step of stream g, S = Q K^T (M=128, N = the
+//               keys of this block rounded up to 16) into TMEM S[g], then --
+//               once warpgroup g has written P for its previous step -- that
+//               step's O[g] += P V (M=128, N=64, K = its key count; V is the
+//               MN-major operand) into TMEM; a unit's first PV overwrites O;
+//   warps 2..5  softmax warpgroup 0, warps 6..9 warpgroup 1: thread r owns
+//               query row r (TMEM lane r) of its stream's unit; per step it
+//               reads its S row, masks keys past its position and past the
+//               user, keeps the running max m and sum l in fp32 (base-2,
+//               scale folded in) and writes P = exp2(s - m) as bf16 into the
+//               K-major swizzled layout the tensor core reads.  m is raised
+//               lazily (only when a block's max exceeds it by 2^8), and then
+//               the row of O in TMEM is rescaled in place.  Before writing P
+//               it waits for the previous PV (the stream's P buffer is
+//               single); at the end of a unit it stores O / l in bf16.
+// Fully masked 32-key chunks of the diagonal block are skipped (their P is
+// written as zeros); rows past the user end are computed but not stored; TMA
+// zero-fills rows past T.  Every wait is bounded.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,193 +44,423 @@ namespace ptl {
 using namespace sm100;
 
 constexpr int ATT_TILE_BYTES = ATT_BLK * DH * 2;  // 16 KB
-constexpr int ATT_SMEM = 5 * ATT_TILE_BYTES + 1024 + 128;
+constexpr int ATT_KV_STAGES = 3;
+// Q[2] + (K,V)[3] + P[2][2 column blocks]
+constexpr int ATT_SMEM_TILES = 2 + 2 * ATT_KV_STAGES + 4;
+constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 256;
+constexpr int ATT_THREADS = 320;  // producer, MMA, two softmax warpgroups
 
-__global__ void __launch_bounds__(128, 2)
+struct AttnUnit {
+  int s0, L, b, h;
+};
+
+__device__ __forceinline__ AttnUnit attn_unit(const int2* items, const int32_t* cu, int unit) {
+  const int2 it = items[unit >> 3];
+  AttnUnit a;
+  a.s0 = cu[it.x];
+  a.L = cu[it.x + 1] - a.s0;
+  a.b = it.y;
+  a.h = unit & 7;
+  return a;
+}
+
+// Units go to CTAs in snake order over the grid (0..G-1, then G-1..0, ...),
+// so each CTA gets a mix of heavy and light units (the list is heaviest
+// first).  Inside a CTA, each unit in turn goes to the stream (of two) with
+// fewer key-block steps so far; every role of the CTA replays this same
+// deterministic walk, so no assignment is stored or exchanged.
+struct CtaWalker {
+  int k = 0, acc0 = 0, acc1 = 0;
+  // the next unit of stream g, or -1 when the CTA's list is exhausted
+  __device__ int next(const int2* items, int nunits, int g) {
+    const int G = gridDim.x, c = blockIdx.x;
+    for (;;) {
+      const int u = k * G + ((k & 1) ? G - 1 - c : c);
+      if (u >= nunits) return -1;
+      ++k;
+      const int st = items[u >> 3].y + 1;
+      const int to = acc0 <= acc1 ? 0 : 1;
+      if (to == 0) acc0 += st; else acc1 += st;
+      if (to == g) return u;
+    }
+  }
+};
+
+// keys of block kb that exist for this user, rounded up to the MMA's 16
+__device__ __forceinline__ int keys16(int L, int kb) {
+  const int k = min(L - kb * ATT_BLK, ATT_BLK);
+  return (k + 15) & ~15;
+}
+
+// The interleaved step sequence both the producer and the MMA issuer walk.
+// Each stream's next unit is looked up one unit ahead, so switching units
+// does not wait on the work-list and offset loads.
+struct AttnStepGen {
+  int nunits;
+  int kb[2], n[2], uc[2];  // uc: units started by the stream
+  AttnUnit u[2], nxt[2];
+  bool live[2], nxt_live[2];
+  CtaWalker walk[2];
+  int turn;
+  __device__ void fetch_next(const int2* items, const int32_t* cu, int g) {
+    const int un = walk[g].next(items, nunits, g);
+    nxt_live[g] = un >= 0;
+    if (nxt_live[g]) nxt[g] = attn_unit(items, cu, un);
+  }
+  __device__ void init(const int2* items, const int32_t* cu, int nunits_) {
+    nunits = nunits_;
+    turn = 0;
+    for (int g = 0; g < 2; ++g) {
+      kb[g] = 0;
+      n[g] = 0;
+      uc[g] = 0;
+      walk[g] = CtaWalker();
+      fetch_next(items, cu, g);
+      live[g] = nxt_live[g];
+      u[g] = nxt[g];
+      if (live[g]) fetch_next(items, cu, g);
+    }
+  }
+  // picks the stream of the next step; false when both streams are done
+  __device__ bool pick(int& g) {
+    if (!live[0] && !live[1]) return false;
+    g = live[turn] ? turn : turn ^ 1;
+    return true;
+  }
+  __device__ void advance(const int2* items, const int32_t* cu, int g) {
+    ++n[g];
+    if (++kb[g] > u[g].b) {
+      ++uc[g];
+      kb[g] = 0;
+      live[g] = nxt_live[g];
+      u[g] = nxt[g];
+      if (live[g]) fetch_next(items, cu, g);
+    }
+    turn = g ^ 1;
+  }
+};
+
+__global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int32_t* __restrict__ cu,
                    const int2* __restrict__ items, const int32_t* __restrict__ item_count,
                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + ATT_TILE_BYTES;
-  uint8_t* sV = smem + 2 * ATT_TILE_BYTES;
-  uint8_t* sP = smem + 3 * ATT_TILE_BYTES;  // two 64-key column blocks
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * ATT_TILE_BYTES);
-  uint64_t* bar_q = bars + 0;
-  uint64_t* bar_kv = bars + 1;
-  uint64_t* bar_s = bars + 2;
-  uint64_t* bar_o = bars + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  __shared__ int s_skip;
+  uint8_t* sQ = smem;                                      // [stream]
+  uint8_t* sKV = smem + 2 * ATT_TILE_BYTES;                // [stage]: K then V
+  uint8_t* sP = sKV + 2 * ATT_KV_STAGES * ATT_TILE_BYTES;  // [stream]: two 64-key column blocks each
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);
+  uint64_t* q_full = bars;          // [stream]
+  uint64_t* q_empty = bars + 2;     // [stream]
+  uint64_t* kv_full = bars + 4;     // [stage]
+  uint64_t* kv_empty = bars + 7;    // [stage]
+  uint64_t* s_full = bars + 10;     // [stream]
+  uint64_t* s_empty = bars + 12;    // [stream]
+  uint64_t* p_full = bars + 14;     // [stream]
+  uint64_t* pv_done = bars + 16;    // [stream]
+  uint64_t* pv_empty = bars + 18;   // [stream]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  __shared__ int s_units;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int item = blockIdx.x / H, h = blockIdx.x % H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  pdl_wait();  // qkv, the work list and the error word come from earlier kernels
-  if (tid == 0) {
-    const int skip = (has_error(err) || item >= *item_count) ? 1 : 0;
-    s_skip = skip;
-    if (!skip) {
-      mbar_init(bar_q, 1);
-      mbar_init(bar_kv, 1);
-      mbar_init(bar_s, 1);
-      mbar_init(bar_o, 1);
-      fence_mbar_init();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&pv_empty[i], 128);
     }
+    for (int i = 0; i < ATT_KV_STAGES; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
   }
-  __syncthreads();
-  if (s_skip) return;
-  const int2 it = items[item];
-  const int s0 = cu[it.x];
-  const int L = cu[it.x + 1] - s0;
-  const int qb = it.y;
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // qkv, the work list and the error word come from earlier kernels
+  if (threadIdx.x == 0) s_units = has_error(err) ? 0 : (*item_count) * H;
+  __syncthreads();
+  const int nunits = s_units;
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;
-  const uint32_t tO = tmem + 128;
-  const uint32_t lane_off = uint32_t(32 * warp) << 16;
+  // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383
 
-  const int qi = qb * ATT_BLK + tid;      // query position inside the user
-  const int qlim = min(qi, L - 1);        // keys 0..qlim are visible
-  const float c2 = 0.125f * 1.4426950408889634f;  // softmax scale * log2(e)
-  constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128);
-  constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
-
-  if (tid == 0) {
-    tma_prefetch_desc(&tm_qkv);
-    mbar_arrive_expect_tx(bar_q, ATT_TILE_BYTES);
-    tma_load_2d(sQ, &tm_qkv, bar_q, h * DH, s0 + qb * ATT_BLK);
-  }
-  float o[DH];
-#pragma unroll
-  for (int d = 0; d < DH; ++d) o[d] = 0.f;
-  float m = -INFINITY, l = 0.f;
-  bool ok = true;
-
-  for (int kb = 0; kb <= qb && ok; ++kb) {
-    const uint32_t ph = kb & 1;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(bar_kv, 2 * ATT_TILE_BYTES);
-      tma_load_2d(sK, &tm_qkv, bar_kv, D + h * DH, s0 + kb * ATT_BLK);
-      tma_load_2d(sV, &tm_qkv, bar_kv, 2 * D + h * DH, s0 + kb * ATT_BLK);
-      if (mbar_wait(bar_q, 0) && mbar_wait(bar_kv, ph)) {
+  if (warp == 0) {
+    if (lane == 0) {
+      AttnStepGen gen;
+      gen.init(items, cu, nunits);
+      int step = 0, g;
+      bool ok = true;
+      while (ok && gen.pick(g)) {
+        const AttnUnit a = gen.u[g];
+        if (gen.kb[g] == 0) {  // a new unit of stream g: its Q tile
+          const int uc = gen.uc[g];
+          if (!mbar_wait(&q_empty[g], (uc & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&q_full[g], ATT_TILE_BYTES);
+          tma_load_2d(sQ + g * ATT_TILE_BYTES, &tm_qkv, &q_full[g], a.h * DH, a.s0 + a.b * ATT_BLK);
+        }
+        const int st = step % ATT_KV_STAGES;
+        if (!mbar_wait(&kv_empty[st], ((step / ATT_KV_STAGES) & 1) ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&kv_full[st], 2 * ATT_TILE_BYTES);
+        uint8_t* kbuf = sKV + (2 * st) * ATT_TILE_BYTES;
+        const int row = a.s0 + gen.kb[g] * ATT_BLK;
+        tma_load_2d(kbuf, &tm_qkv, &kv_full[st], D + a.h * DH, row);
+        tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, &kv_full[st], 2 * D + a.h * DH, row);
+        ++step;
+        gen.advance(items, cu, g);
+      }
+      if (!ok) set_error(err, PTL_ERR_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      AttnStepGen gen;
+      gen.init(items, cu, nunits);
+      int step = 0, g;
+      // the previous step of each stream, whose PV is still to be issued
+      int pv_n[2] = {-1, -1}, pv_st[2] = {0, 0}, pv_k16[2] = {0, 0}, pv_uc[2] = {0, 0};
+      bool pv_first[2] = {false, false};
+      bool ok = true;
+      // O[g] += P V; a unit's first PV overwrites O, once warpgroup g has
+      // read the previous unit's O
+      auto issue_pv = [&](int gs) -> bool {
+        const int nn = pv_n[gs];
+        if (nn < 0) return true;
+        if (!mbar_wait(&p_full[gs], nn & 1)) return false;
+        if (pv_first[gs] && !mbar_wait(&pv_empty[gs], (pv_uc[gs] & 1) ^ 1)) return false;
         tc_fence_after();
-        const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK);
+        const uint32_t p0 = smem_u32(sP + gs * 2 * ATT_TILE_BYTES);
+        const uint32_t v0 = smem_u32(sKV + (2 * pv_st[gs] + 1) * ATT_TILE_BYTES);
+        const uint32_t d = tmem + 256 + 64 * gs;
+        constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
+        for (int k = 0; k < pv_k16[gs] / 16; ++k)
+          umma_bf16_ss(d, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
+                       umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !pv_first[gs]);
+        umma_commit(&pv_done[gs]);
+        umma_commit(&kv_empty[pv_st[gs]]);
+        pv_n[gs] = -1;
+        return true;
+      };
+      while (ok && gen.pick(g)) {
+        const AttnUnit a = gen.u[g];
+        const int kb = gen.kb[g];
+        const int nn = gen.n[g];
+        if (kb == 0 && !mbar_wait(&q_full[g], gen.uc[g] & 1)) { ok = false; break; }
+        const int st = step % ATT_KV_STAGES;
+        if (!mbar_wait(&kv_full[st], (step / ATT_KV_STAGES) & 1) || !mbar_wait(&s_empty[g], (nn & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int k16 = keys16(a.L, kb);
+        const uint32_t q0 = smem_u32(sQ + g * ATT_TILE_BYTES);
+        const uint32_t k0 = smem_u32(sKV + (2 * st) * ATT_TILE_BYTES);
+        const uint32_t idesc_qk = umma_idesc_bf16(128, k16);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma_bf16_ss(tS, umma_desc_sw128(q0 + 32 * k, 1024), umma_desc_sw128(k0 + 32 * k, 1024),
+          umma_bf16_ss(tmem + 128 * g, umma_desc_sw128(q0 + 32 * k, 1024), umma_desc_sw128(k0 + 32 * k, 1024),
                        idesc_qk, k != 0);
-        umma_commit(bar_s);
-      } else {
-        set_error(err, PTL_ERR_TIMEOUT);
+        umma_commit(&s_full[g]);
+        if (kb == a.b) umma_commit(&q_empty[g]);
+        if (!issue_pv(g)) { ok = false; break; }
+        pv_n[g] = nn;
+        pv_st[g] = st;
+        pv_k16[g] = k16;
+        pv_first[g] = kb == 0;
+        pv_uc[g] = gen.uc[g];
+        ++step;
+        gen.advance(items, cu, g);
+        // a stream with no further steps must not hold its K/V ring stage
+        if (!gen.live[g] && !issue_pv(g)) { ok = false; break; }
       }
+      if (ok) ok = issue_pv(0) && issue_pv(1);
+      if (!ok) set_error(err, PTL_ERR_TIMEOUT);
     }
-    if (!mbar_wait(bar_s, ph)) {
-      set_error(err, PTL_ERR_TIMEOUT);
-      ok = false;
-    }
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    tc_fence_after();
-
-    // pass 1: row maximum over the visible keys of this block
-    const int kbase = kb * ATT_BLK;
-    float mx = -INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t raw[32];
-      tmem_ld32(tS + lane_off + 32 * c, raw);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (kbase + 32 * c + i <= qlim) mx = fmaxf(mx, __uint_as_float(raw[i]));
-    }
-    const float m_new = fmaxf(m, mx * c2);
-    const float alpha = exp2f(m - m_new);
-    // pass 2: probabilities -> bf16 P in shared memory (K-major, swizzled)
-    float lsum = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t raw[32];
-      tmem_ld32(tS + lane_off + 32 * c, raw);
-      tmem_ld_wait();
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const int j = kbase + 32 * c + i;
-        const float p0 = (j <= qlim) ? exp2f(__uint_as_float(raw[i]) * c2 - m_new) : 0.f;
-        const float p1 = (j + 1 <= qlim) ? exp2f(__uint_as_float(raw[i + 1]) * c2 - m_new) : 0.f;
-        lsum += p0 + p1;
-        pk[i >> 1] = pack_bf16x2(p0, p1);
-      }
-      // keys 32c..32c+31 live in column block c/2, 16-byte chunks (c%2)*4 .. +3
-      const uint32_t row_addr = smem_u32(sP + (c >> 1) * ATT_TILE_BYTES) + tid * 128;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int chunk = (c & 1) * 4 + q;
-        st_shared_v4(row_addr + ((chunk ^ (tid & 7)) << 4), pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
-                     pk[4 * q + 3]);
-      }
-    }
-    l = l * alpha + lsum;
-    m = m_new;
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
+  } else {
+    // softmax warpgroup g (warps 2..5 -> 0, 6..9 -> 1); thread r <-> query row r
+    // of the unit <-> TMEM lane r
+    const int g = (warp - 2) >> 2;
+    const int wq = warp & 3;
+    const int r = 32 * wq + lane;
+    const uint32_t lane_off = uint32_t(32 * wq) << 16;
+    const uint32_t tS = tmem + 128 * g + lane_off;
+    const uint32_t tPV = tmem + 256 + 64 * g + lane_off;
+    const float c2 = 0.125f * 1.4426950408889634f;  // softmax scale * log2(e)
+    // Running max m (base 2, scale folded in) and sum l of this row.  O lives
+    // in TMEM and the PV products accumulate into it; m is raised (and O, l
+    // rescaled) only when a block's max exceeds it by more than RESCALE_LOG2,
+    // so P = exp2(s - m) stays below 2^RESCALE_LOG2 and O / l is unchanged.
+    constexpr float RESCALE_LOG2 = 8.f;
+    float m = 0.f, l = 0.f;
+    // the previous step of this stream: its PV may still be running
+    int pn = -1;
+    bool plast = false;
+    float pl = 1.f;
+    int pdst = -1;  // output row offset (elements) of this thread for the previous step's unit, or -1
+    bool ok = true;
+    // waits for the previous step's PV; at a unit's end, stores O / l and
+    // releases O for the next unit's first PV
+    auto finish_prev = [&]() -> bool {
+      if (!mbar_wait(&pv_done[g], pn & 1)) return false;
       tc_fence_after();
-      const uint32_t p0 = smem_u32(sP), v0 = smem_u32(sV);
+      if (plast) {
+        const float inv = 1.0f / pl;
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        umma_bf16_ss(tO, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
-                     umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0);
-      umma_commit(bar_o);
-    }
-    if (!mbar_wait(bar_o, ph)) {
-      set_error(err, PTL_ERR_TIMEOUT);
-      ok = false;
-    }
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    tc_fence_after();
+        for (int c = 0; c < 2; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(tPV + 32 * c, raw);
+          tmem_ld_wait();
+          if (pdst >= 0) {
+            uint4* dst = reinterpret_cast<uint4*>(out + pdst + 32 * c);
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t raw[32];
-      tmem_ld32(tO + lane_off + 32 * c, raw);
-      tmem_ld_wait();
+            for (int q = 0; q < 4; ++q) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(raw[8 * q + 0]) * inv, __uint_as_float(raw[8 * q + 1]) * inv);
+              u.y = pack_bf16x2(__uint_as_float(raw[8 * q + 2]) * inv, __uint_as_float(raw[8 * q + 3]) * inv);
+              u.z = pack_bf16x2(__uint_as_float(raw[8 * q + 4]) * inv, __uint_as_float(raw[8 * q + 5]) * inv);
+              u.w = pack_bf16x2(__uint_as_float(raw[8 * q + 6]) * inv, __uint_as_float(raw[8 * q + 7]) * inv);
+              dst[q] = u;
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&pv_empty[g]);
+      }
+      return true;
+    };
+    int n = 0;  // steps of this stream
+    CtaWalker walk;
+    int unit = walk.next(items, nunits, g);
+    AttnUnit nxt = unit >= 0 ? attn_unit(items, cu, unit) : AttnUnit{0, 0, 0, 0};
+    while (unit >= 0 && ok) {
+      const AttnUnit a = nxt;
+      unit = walk.next(items, nunits, g);
+      if (unit >= 0) nxt = attn_unit(items, cu, unit);  // prefetch the next unit
+      const int qi = a.b * ATT_BLK + r;   // query position inside the user
+      const int qlim = min(qi, a.L - 1);  // keys 0..qlim are visible
+      for (int kb = 0; kb <= a.b; ++kb, ++n) {
+        if (!mbar_wait(&s_full[g], n & 1)) { ok = false; break; }
+        tc_fence_after();
+        const int k16 = keys16(a.L, kb);
+        const int kbase = kb * ATT_BLK;
+        // 32-key chunks this warp needs: those inside the block's key count,
+        // and on the diagonal block only chunks not wholly above the warp's
+        // rows; loads take 64 columns, the keys past qlim are masked
+        const int nch = (k16 + 31) >> 5;
+        const int nuse = (kb == a.b) ? min(nch, wq + 1) : nch;
+        // pass 1: the row maximum over the visible keys (four independent chains)
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int hh = 0; 2 * hh < nuse; ++hh) {
+          uint32_t raw[32];
+          tmem_ld32(tS + 64 * hh, raw);
+          uint32_t raw2[32];
+          tmem_ld32(tS + 64 * hh + 32, raw2);
+          tmem_ld_wait();
+          const int lim = qlim - (kbase + 64 * hh);  // keys i <= lim are visible
 #pragma unroll
-      for (int i = 0; i < 32; ++i) o[32 * c + i] = o[32 * c + i] * alpha + __uint_as_float(raw[i]);
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
-
-  if (ok && qi < L) {
-    const float inv = 1.0f / l;
-    uint4* dst = reinterpret_cast<uint4*>(out + size_t(s0 + qi) * D + h * DH);
+          for (int i = 0; i < 32; ++i) {
+            if (i <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
+            if (i + 32 <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw2[i]));
+          }
+        }
+        const float mblk = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c2;
+        // the previous PV must be done before O is touched or P rewritten
+        if (pn >= 0 && !finish_prev()) { ok = false; break; }
+        if (kb == 0) {
+          m = mblk;  // the unit's first PV overwrites O
+          l = 0.f;
+        } else if (__any_sync(0xffffffffu, mblk > m + RESCALE_LOG2)) {
+          const float m_new = fmaxf(m, mblk);
+          const float alpha = ex2_approx(m - m_new);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint4 u;
-      u.x = pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-      u.y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-      u.z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-      u.w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-      dst[q] = u;
+          for (int c = 0; c < 2; ++c) {
+            uint32_t raw[32];
+            tmem_ld32(tPV + 32 * c, raw);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+            tmem_st32(tPV + 32 * c, raw);
+          }
+          tmem_st_wait();
+          l *= alpha;
+          m = m_new;
+        }
+        // pass 2: probabilities -> bf16 P (K-major, swizzled); masked and
+        // skipped columns give p = 0
+        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t pbase = smem_u32(sP + g * 2 * ATT_TILE_BYTES) + r * 128;
+#pragma unroll 1
+        for (int hh = 0; 2 * hh < nch; ++hh) {
+          const uint32_t row_addr = pbase + hh * ATT_TILE_BYTES;  // column block hh: keys 64hh..64hh+63
+          if (2 * hh < nuse) {
+            uint32_t raw[32];
+            tmem_ld32(tS + 64 * hh, raw);
+            uint32_t raw2[32];
+            tmem_ld32(tS + 64 * hh + 32, raw2);
+            tmem_ld_wait();
+            const int lim = qlim - (kbase + 64 * hh);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {  // 16-byte chunk q = keys 8q..8q+7
+              uint32_t pk[4];
+#pragma unroll
+              for (int j = 0; j < 8; j += 2) {
+                const int i = 8 * q + j;
+                const float s0 = __uint_as_float(q < 4 ? raw[i] : raw2[i - 32]);
+                const float s1 = __uint_as_float(q < 4 ? raw[i + 1] : raw2[i - 31]);
+                const float p0 = (i <= lim) ? ex2_approx(s0 * c2 - m) : 0.f;
+                const float p1 = (i + 1 <= lim) ? ex2_approx(s1 * c2 - m) : 0.f;
+                ls4[j >> 1] += p0 + p1;
+                pk[j >> 1] = pack_bf16x2(p0, p1);
+              }
+              st_shared_v4(row_addr + ((q ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) st_shared_v4(row_addr + ((q ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+          }
+        }
+        l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+        // S is read and P written (and O rescaled): the next QK^T and this PV may start
+        tc_fence_before();
+        mbar_arrive(&s_empty[g]);
+        fence_proxy_async_smem();
+        mbar_arrive(&p_full[g]);
+        pn = n;
+        pl = l;
+        plast = kb == a.b;
+        pdst = qi < a.L ? (a.s0 + qi) * D + a.h * DH : -1;
+      }
     }
+    if (ok && pn >= 0) ok = finish_prev();
+    if (!ok) set_error(err, PTL_ERR_TIMEOUT);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
+}
+
+static int num_sms_attn() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
 }
 
 int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
@@ -231,7 +472,9 @@ int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, con
       return -1;
     configured = true;
   }
-  if (launch_k(attn_tc_kernel, dim3(unsigned(L.max_items * H)), dim3(128), ATT_SMEM, st, qkv_map, cu,
+  const int64_t bound = L.max_items * H;
+  const int grid = int(bound < num_sms_attn() ? bound : num_sms_attn());
+  if (launch_k(attn_tc_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map, cu,
                reinterpret_cast<const int2*>(ws + L.items), reinterpret_cast<const int32_t*>(ws + L.item_count),
                static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err)) != 0)
     return -1;

@@ -595,12 +595,17 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
 
 // bf16 build: out[t] = (x1[t] + w[t][0] y(2t)) + w[t][1] y(2t+1) in fp32,
 // rounded once; y(r) is row pos[r] of the padded per-route expert outputs
-// (bf16).  One warp per token, 16-byte loads.
+// (bf16).  One warp per token, 16-byte loads.  Inside a stack, the next
+// layer's LayerNorm1 is applied to the rounded row as well (ln_g != NULL):
+// xn = LN(out) with exactly the arithmetic of the standalone LayerNorm.
 __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* __restrict__ ybuf,
                                                            const int32_t* __restrict__ pos,
                                                            const float* __restrict__ w,
                                                            const float* __restrict__ x1,
                                                            __nv_bfloat16* __restrict__ out, int T_,
+                                                           const float* __restrict__ ln_g,
+                                                           const float* __restrict__ ln_b,
+                                                           __nv_bfloat16* __restrict__ xn,
                                                            const int32_t* err) {
   pdl_trigger();
   pdl_wait();
@@ -624,6 +629,13 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
 #pragma unroll
   for (int j = 0; j < 16; ++j) o[j] = (xr[j] + wt.x * y0[j]) + wt.y * y1[j];
   Row16<__nv_bfloat16>::store(out + size_t(t) * D, lane, o);
+  if (ln_g != nullptr) {
+    // the values the next layer reads back: o rounded to bf16
+#pragma unroll
+    for (int j = 0; j < 16; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
+    layer_norm16<__nv_bfloat16>(o, ln_g, ln_b, lane);
+    Row16<__nv_bfloat16>::store(xn + size_t(t) * D, lane, o);
+  }
 }
 
 // fp32 build: out[t] = (x1[t] + w[t][0] * y[2t]) + w[t][1] * y[2t+1].
@@ -800,9 +812,10 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
 }
 
 int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
-                        int T, const int32_t* err, cudaStream_t st) {
+                        int T, const float* ln_g, const float* ln_b, void* xn, const int32_t* err,
+                        cudaStream_t st) {
   if (launch_k(combine_bf16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(ybuf), pos, w, x1,
-                                                  static_cast<__nv_bfloat16*>(out), T, err)) return -1;
+               static_cast<__nv_bfloat16*>(out), T, ln_g, ln_b, static_cast<__nv_bfloat16*>(xn), err)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
