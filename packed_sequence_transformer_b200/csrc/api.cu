@@ -176,7 +176,7 @@ ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_wei
     }
     CUtensorMap ma, mb, mo;
     if (!map_bf16(&ma, c.ws + c.L.xn, D, T, D * 2, 64, 128)) return PTL_ERR_CUDA;
-    if (!map_bf16(&mb, w->w_qkv, D, QKV_N, D * 2, 64, QKV_BN)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mb, w->w_qkv, D, QKV_N, D * 2, 64, QKV_BN / 2)) return PTL_ERR_CUDA;
     if (!map_bf16(&mo, qkv, QKV_N, T, QKV_N * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_QKV);
     PTL_TRY(launch_gemm_qkv(ma, mb, mo, F32(w->b_qkv), qkv, T, c.err, c.st));
@@ -208,7 +208,7 @@ ptl_status step_out(const Call& c, const void* attn, const void* x, void* x1, co
   if (c.dt == PTL_BF16) {
     CUtensorMap ma, mb, mo;
     if (!map_bf16(&ma, attn, D, c.T, D * 2, 64, 128)) return PTL_ERR_CUDA;
-    if (!map_bf16(&mb, w->w_o, D, D, D * 2, 64, OUT_BN)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mb, w->w_o, D, D, D * 2, 64, OUT_BN / 2)) return PTL_ERR_CUDA;
     if (!map_f32(&mo, x1, D, c.T, D * 4, 32, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_OUT);
     PTL_TRY(launch_gemm_out(ma, mb, mo, F32(w->b_o), x, x1, c.T, c.err, c.st));

@@ -11,7 +11,7 @@
 //
 //   warp 0      TMA producer: the Q tile [128 x 64] of each stream's current
 //               unit, and per step the K and V tiles [128 x 64] through a
-//               3-deep ring, straight from the packed qkv rows (128-byte
+//               4-deep ring, straight from the packed qkv rows (128-byte
 //               swizzle);
 //   warp 1      MMA issuer: for a step of stream g, S = Q K^T (M=128, N = the
 //               keys of this block rounded up to 16) into TMEM S[g], then --
@@ -44,7 +44,9 @@ namespace ptl {
 using namespace sm100;
 
 constexpr int ATT_TILE_BYTES = ATT_BLK * DH * 2;  // 16 KB
-constexpr int ATT_KV_STAGES = 3;
+// Four stages: each stream holds one K/V stage until its deferred PV is done
+// and needs the next one loaded before its next QK^T can start.
+constexpr int ATT_KV_STAGES = 4;
 // Q[2] + (K,V)[3] + P[2][2 column blocks]
 constexpr int ATT_SMEM_TILES = 2 + 2 * ATT_KV_STAGES + 4;
 constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 256;
@@ -95,50 +97,73 @@ __device__ __forceinline__ int keys16(int L, int kb) {
 // The interleaved step sequence both the producer and the MMA issuer walk.
 // Each stream's next unit is looked up one unit ahead, so switching units
 // does not wait on the work-list and offset loads.
+// One stream's position in its step sequence, plus (for the MMA issuer) its
+// deferred PV.  The two streams are held in named registers and swapped, never
+// indexed by the stream number, so nothing lands in local memory.
+struct StreamPos {
+  int g;             // the stream (softmax warpgroup)
+  int kb, n, uc;     // key block of the current unit, steps so far, units started
+  bool live, nxt_live;
+  AttnUnit u, nxt;   // current unit, the next one (looked up one unit ahead)
+  CtaWalker walk;
+  int pv_n, pv_st, pv_k16, pv_uc;  // the step whose PV is still to be issued (-1: none)
+  bool pv_first;
+};
+
+// The interleaved step sequence both the producer and the MMA issuer walk:
+// `a` is the stream whose turn it is; after each step the streams swap while
+// both have steps left.
 struct AttnStepGen {
   int nunits;
-  int kb[2], n[2], uc[2];  // uc: units started by the stream
-  AttnUnit u[2], nxt[2];
-  bool live[2], nxt_live[2];
-  CtaWalker walk[2];
-  int turn;
-  __device__ void fetch_next(const int2* items, const int32_t* cu, int g) {
-    const int un = walk[g].next(items, nunits, g);
-    nxt_live[g] = un >= 0;
-    if (nxt_live[g]) nxt[g] = attn_unit(items, cu, un);
+  StreamPos a, b;
+  __device__ void fetch_next(const int2* items, const int32_t* cu, StreamPos& sp) {
+    const int un = sp.walk.next(items, nunits, sp.g);
+    sp.nxt_live = un >= 0;
+    if (sp.nxt_live) sp.nxt = attn_unit(items, cu, un);
+  }
+  __device__ void init_stream(const int2* items, const int32_t* cu, StreamPos& sp, int g) {
+    sp.g = g;
+    sp.kb = 0;
+    sp.n = 0;
+    sp.uc = 0;
+    sp.walk = CtaWalker();
+    sp.pv_n = -1;
+    sp.pv_st = sp.pv_k16 = sp.pv_uc = 0;
+    sp.pv_first = false;
+    fetch_next(items, cu, sp);
+    sp.live = sp.nxt_live;
+    sp.u = sp.nxt;
+    if (sp.live) fetch_next(items, cu, sp);
   }
   __device__ void init(const int2* items, const int32_t* cu, int nunits_) {
     nunits = nunits_;
-    turn = 0;
-    for (int g = 0; g < 2; ++g) {
-      kb[g] = 0;
-      n[g] = 0;
-      uc[g] = 0;
-      walk[g] = CtaWalker();
-      fetch_next(items, cu, g);
-      live[g] = nxt_live[g];
-      u[g] = nxt[g];
-      if (live[g]) fetch_next(items, cu, g);
-    }
+    init_stream(items, cu, a, 0);
+    init_stream(items, cu, b, 1);
   }
-  // picks the stream of the next step; false when both streams are done
-  __device__ bool pick(int& g) {
-    if (!live[0] && !live[1]) return false;
-    g = live[turn] ? turn : turn ^ 1;
-    return true;
+  __device__ void swap_streams() {
+    const StreamPos t = a;
+    a = b;
+    b = t;
   }
-  __device__ void advance(const int2* items, const int32_t* cu, int g) {
-    ++n[g];
-    if (++kb[g] > u[g].b) {
-      ++uc[g];
-      kb[g] = 0;
-      live[g] = nxt_live[g];
-      u[g] = nxt[g];
-      if (live[g]) fetch_next(items, cu, g);
+  // makes `a` the stream of the next step; false when both streams are done
+  __device__ bool pick() {
+    if (!a.live) swap_streams();
+    return a.live;
+  }
+  // advances `a` by one step, then hands the turn to the other stream
+  __device__ void advance(const int2* items, const int32_t* cu) {
+    ++a.n;
+    if (++a.kb > a.u.b) {
+      ++a.uc;
+      a.kb = 0;
+      a.live = a.nxt_live;
+      a.u = a.nxt;
+      if (a.live) fetch_next(items, cu, a);
     }
-    turn = g ^ 1;
+    if (b.live) swap_streams();
   }
 };
+
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int32_t* __restrict__ cu,
@@ -152,14 +177,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);
   uint64_t* q_full = bars;          // [stream]
   uint64_t* q_empty = bars + 2;     // [stream]
-  uint64_t* kv_full = bars + 4;     // [stage]
-  uint64_t* kv_empty = bars + 7;    // [stage]
-  uint64_t* s_full = bars + 10;     // [stream]
-  uint64_t* s_empty = bars + 12;    // [stream]
-  uint64_t* p_full = bars + 14;     // [stream]
-  uint64_t* pv_done = bars + 16;    // [stream]
-  uint64_t* pv_empty = bars + 18;   // [stream]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* kv_full = bars + 4;                   // [stage]
+  uint64_t* kv_empty = kv_full + ATT_KV_STAGES;   // [stage]
+  uint64_t* s_full = kv_empty + ATT_KV_STAGES;    // [stream]
+  uint64_t* s_empty = s_full + 2;                 // [stream]
+  uint64_t* p_full = s_full + 4;                  // [stream]
+  uint64_t* pv_done = s_full + 6;                 // [stream]
+  uint64_t* pv_empty = s_full + 8;                // [stream]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
   __shared__ int s_units;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -199,13 +224,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (lane == 0) {
       AttnStepGen gen;
       gen.init(items, cu, nunits);
-      int step = 0, g;
+      int step = 0;
       bool ok = true;
-      while (ok && gen.pick(g)) {
-        const AttnUnit a = gen.u[g];
-        if (gen.kb[g] == 0) {  // a new unit of stream g: its Q tile
-          const int uc = gen.uc[g];
-          if (!mbar_wait(&q_empty[g], (uc & 1) ^ 1)) { ok = false; break; }
+      while (ok && gen.pick()) {
+        const int g = gen.a.g;
+        const AttnUnit a = gen.a.u;
+        if (gen.a.kb == 0) {  // a new unit of stream g: its Q tile
+          if (!mbar_wait(&q_empty[g], (gen.a.uc & 1) ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&q_full[g], ATT_TILE_BYTES);
           tma_load_2d(sQ + g * ATT_TILE_BYTES, &tm_qkv, &q_full[g], a.h * DH, a.s0 + a.b * ATT_BLK);
         }
@@ -213,11 +238,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (!mbar_wait(&kv_empty[st], ((step / ATT_KV_STAGES) & 1) ^ 1)) { ok = false; break; }
         mbar_arrive_expect_tx(&kv_full[st], 2 * ATT_TILE_BYTES);
         uint8_t* kbuf = sKV + (2 * st) * ATT_TILE_BYTES;
-        const int row = a.s0 + gen.kb[g] * ATT_BLK;
+        const int row = a.s0 + gen.a.kb * ATT_BLK;
         tma_load_2d(kbuf, &tm_qkv, &kv_full[st], D + a.h * DH, row);
         tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, &kv_full[st], 2 * D + a.h * DH, row);
         ++step;
-        gen.advance(items, cu, g);
+        gen.advance(items, cu);
       }
       if (!ok) set_error(err, PTL_ERR_TIMEOUT);
     }
@@ -225,36 +250,36 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (lane == 0) {
       AttnStepGen gen;
       gen.init(items, cu, nunits);
-      int step = 0, g;
-      // the previous step of each stream, whose PV is still to be issued
-      int pv_n[2] = {-1, -1}, pv_st[2] = {0, 0}, pv_k16[2] = {0, 0}, pv_uc[2] = {0, 0};
-      bool pv_first[2] = {false, false};
+      int step = 0;
       bool ok = true;
-      // O[g] += P V; a unit's first PV overwrites O, once warpgroup g has
-      // read the previous unit's O
-      auto issue_pv = [&](int gs) -> bool {
-        const int nn = pv_n[gs];
+      // O[g] += P V for the stream's deferred step; a unit's first PV
+      // overwrites O, once warpgroup g has read the previous unit's O
+      auto issue_pv = [&](StreamPos& sp) -> bool {
+        const int nn = sp.pv_n;
         if (nn < 0) return true;
+        const int gs = sp.g;
         if (!mbar_wait(&p_full[gs], nn & 1)) return false;
-        if (pv_first[gs] && !mbar_wait(&pv_empty[gs], (pv_uc[gs] & 1) ^ 1)) return false;
+        if (sp.pv_first && !mbar_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
         tc_fence_after();
         const uint32_t p0 = smem_u32(sP + gs * 2 * ATT_TILE_BYTES);
-        const uint32_t v0 = smem_u32(sKV + (2 * pv_st[gs] + 1) * ATT_TILE_BYTES);
+        const uint32_t v0 = smem_u32(sKV + (2 * sp.pv_st + 1) * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256 + 64 * gs;
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
-        for (int k = 0; k < pv_k16[gs] / 16; ++k)
+        for (int k = 0; k < sp.pv_k16 / 16; ++k)
           umma_bf16_ss(d, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
-                       umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !pv_first[gs]);
+                       umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !sp.pv_first);
         umma_commit(&pv_done[gs]);
-        umma_commit(&kv_empty[pv_st[gs]]);
-        pv_n[gs] = -1;
+        umma_commit(&kv_empty[sp.pv_st]);
+        sp.pv_n = -1;
         return true;
       };
-      while (ok && gen.pick(g)) {
-        const AttnUnit a = gen.u[g];
-        const int kb = gen.kb[g];
-        const int nn = gen.n[g];
-        if (kb == 0 && !mbar_wait(&q_full[g], gen.uc[g] & 1)) { ok = false; break; }
+      while (ok && gen.pick()) {
+        StreamPos& sp = gen.a;
+        const int g = sp.g;
+        const AttnUnit a = sp.u;
+        const int kb = sp.kb;
+        const int nn = sp.n;
+        if (kb == 0 && !mbar_wait(&q_full[g], sp.uc & 1)) { ok = false; break; }
         const int st = step % ATT_KV_STAGES;
         if (!mbar_wait(&kv_full[st], (step / ATT_KV_STAGES) & 1) || !mbar_wait(&s_empty[g], (nn & 1) ^ 1)) {
           ok = false;
@@ -271,18 +296,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                        idesc_qk, k != 0);
         umma_commit(&s_full[g]);
         if (kb == a.b) umma_commit(&q_empty[g]);
-        if (!issue_pv(g)) { ok = false; break; }
-        pv_n[g] = nn;
-        pv_st[g] = st;
-        pv_k16[g] = k16;
-        pv_first[g] = kb == 0;
-        pv_uc[g] = gen.uc[g];
+        if (!issue_pv(sp)) { ok = false; break; }
+        sp.pv_n = nn;
+        sp.pv_st = st;
+        sp.pv_k16 = k16;
+        sp.pv_first = kb == 0;
+        sp.pv_uc = sp.uc;
         ++step;
-        gen.advance(items, cu, g);
         // a stream with no further steps must not hold its K/V ring stage
-        if (!gen.live[g] && !issue_pv(g)) { ok = false; break; }
+        const bool last = sp.kb == a.b && !sp.nxt_live;
+        if (last && !issue_pv(sp)) { ok = false; break; }
+        gen.advance(items, cu);
       }
-      if (ok) ok = issue_pv(0) && issue_pv(1);
+      if (ok) ok = issue_pv(gen.a) && issue_pv(gen.b);
       if (!ok) set_error(err, PTL_ERR_TIMEOUT);
     }
   } else {
@@ -314,11 +340,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tc_fence_after();
       if (plast) {
         const float inv = 1.0f / pl;
+        uint32_t oraw[2][32];
+        tmem_ld32(tPV, oraw[0]);
+        tmem_ld32(tPV + 32, oraw[1]);
+        tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(tPV + 32 * c, raw);
-          tmem_ld_wait();
+          const uint32_t (&raw)[32] = oraw[c];
           if (pdst >= 0) {
             uint4* dst = reinterpret_cast<uint4*>(out + pdst + 32 * c);
 #pragma unroll
@@ -367,10 +395,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           tmem_ld32(tS + 64 * hh + 32, raw2);
           tmem_ld_wait();
           const int lim = qlim - (kbase + 64 * hh);  // keys i <= lim are visible
+          if (lim >= 63) {  // all 64 visible (every block but the diagonal / the user's last)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
-            if (i + 32 <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw2[i]));
+            for (int i = 0; i < 32; ++i) {
+              mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
+              mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw2[i]));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
+              if (i + 32 <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw2[i]));
+            }
           }
         }
         const float mblk = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c2;
@@ -408,7 +444,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             uint32_t raw2[32];
             tmem_ld32(tS + 64 * hh + 32, raw2);
             tmem_ld_wait();
+            // keys i <= lim are visible; all 64 on every block but the
+            // diagonal / the user's last (no selects there)
             const int lim = qlim - (kbase + 64 * hh);
+            const int lim_eff = lim >= 63 ? 63 : lim;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {  // 16-byte chunk q = keys 8q..8q+7
               uint32_t pk[4];
@@ -417,8 +456,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 const int i = 8 * q + j;
                 const float s0 = __uint_as_float(q < 4 ? raw[i] : raw2[i - 32]);
                 const float s1 = __uint_as_float(q < 4 ? raw[i + 1] : raw2[i - 31]);
-                const float p0 = (i <= lim) ? ex2_approx(s0 * c2 - m) : 0.f;
-                const float p1 = (i + 1 <= lim) ? ex2_approx(s1 * c2 - m) : 0.f;
+                float p0 = ex2_approx(s0 * c2 - m);
+                float p1 = ex2_approx(s1 * c2 - m);
+                if (lim < 63) {
+                  p0 = (i <= lim_eff) ? p0 : 0.f;
+                  p1 = (i + 1 <= lim_eff) ? p1 : 0.f;
+                }
                 ls4[j >> 1] += p0 + p1;
                 pk[j >> 1] = pack_bf16x2(p0, p1);
               }

@@ -70,10 +70,11 @@ struct GemmCfg {
   static constexpr int STAGING = TMA_OUT ? 128 * BN * OUT_ELEM : 0;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = BN * 64 * 2;
-  static constexpr int USABLE = 232448 - 1024 - 256;
-  static constexpr int STAGES_FIT = (USABLE - STAGING) / (A_BYTES + B_BYTES);
+  static constexpr int BIAS = BN * 4;                              // the tile's bias slice
+  static constexpr int USABLE = 232448 - 1024 - 256 - 64;          // minus align, barriers, static
+  static constexpr int STAGES_FIT = (USABLE - STAGING - BIAS) / (A_BYTES + B_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES) + STAGING + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES) + STAGING + BIAS + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;     // power of two >= 2 accumulators
   static_assert(2 * BN <= 512, "two accumulators must fit in TMEM");
   static_assert(STAGES >= 2, "operand ring too small");
@@ -134,7 +135,8 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
   uint8_t* sOut = sB + STAGES * Cfg::B_BYTES;  // staging tile (TMA-stored modes)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg::STAGING);
+  float* s_bias = reinterpret_cast<float*>(sOut + Cfg::STAGING);  // the current tile's bias slice
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg::STAGING + Cfg::BIAS);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;   // [2] accumulator ready for the epilogue
   uint64_t* tempty = tfull + 2;       // [2] accumulator drained by the epilogue
@@ -238,19 +240,28 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
     // with the 64-element K slice of its token's LayerNorm2 row, 16 bytes at
     // a time, at the 128-byte-swizzled position TMA would have used.
     const int r = threadIdx.x - 192;
+    constexpr int NKB = D / 64;  // K slices per tile (K = 512)
+    constexpr int DEPTH = 3;     // K slices in flight per thread
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       int expert, m0, n0;
       decode_tile<BN, MODE>(p, tile, expert, m0, n0);
       const int route = p.rowroute[m0 + r];
-      const __nv_bfloat16* src = route >= 0 ? p.gatherA + size_t(route >> 1) * D : nullptr;
-      for (int kb = 0; kb < nkb; ++kb, ++it) {
-        const int s = it % STAGES;
-        uint4 v[8];
+      const uint4* src = route >= 0 ? reinterpret_cast<const uint4*>(p.gatherA + size_t(route >> 1) * D) : nullptr;
+      uint4 v[DEPTH][8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          v[c] = src ? __ldg(reinterpret_cast<const uint4*>(src + kb * 64) + c) : make_uint4(0, 0, 0, 0);
+      for (int kb = 0; kb < DEPTH - 1; ++kb)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[kb][c] = src ? __ldg(src + kb * 8 + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int kb = 0; kb < NKB; ++kb, ++it) {
+        if (kb + DEPTH - 1 < NKB) {  // the load DEPTH - 1 slices ahead
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            v[(kb + DEPTH - 1) % DEPTH][c] = src ? __ldg(src + (kb + DEPTH - 1) * 8 + c) : make_uint4(0, 0, 0, 0);
+        }
+        const int s = it % STAGES;
         if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
           set_error(p.err, PTL_ERR_TIMEOUT);
           ok = false;
@@ -259,7 +270,8 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
         const uint32_t row_addr = smem_u32(sA + s * Cfg::A_BYTES) + r * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          st_shared_v4(row_addr + ((c ^ (r & 7)) << 4), v[c].x, v[c].y, v[c].z, v[c].w);
+          st_shared_v4(row_addr + ((c ^ (r & 7)) << 4), v[kb % DEPTH][c].x, v[kb % DEPTH][c].y, v[kb % DEPTH][c].z,
+                       v[kb % DEPTH][c].w);
         fence_proxy_async_smem();
         mbar_arrive(&full[s]);
       }
@@ -273,24 +285,42 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
       int expert, m0, n0;
       decode_tile<BN, MODE>(p, tile, expert, m0, n0);
       const int acc = j & 1;
+      const int row = m0 + r;
+      // Everything the epilogue reads besides the accumulator is fetched
+      // while the tile's MMAs run: the bias slice (into shared memory) and,
+      // for the output projection, this thread's residual row (registers).
+      const float* bb = p.bias ? p.bias + (MODE >= G_MOE1 ? expert * p.N_total : 0) + n0 : nullptr;
+      float bv[(BN + 127) / 128];
+#pragma unroll
+      for (int i = 0; i < (BN + 127) / 128; ++i)
+        bv[i] = (bb && r + 128 * i < BN) ? __ldg(bb + r + 128 * i) : 0.f;
+      constexpr int NRES = MODE == G_OUT ? BN / 8 : 1;
+      uint4 res[NRES];
+      if (MODE == G_OUT) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0);
+#pragma unroll
+        for (int q = 0; q < NRES; ++q) res[q] = row < p.M ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
+      }
+      const bool leader = warp == 2 && lane == 0;
+      // the previous tile's epilogue is done with s_bias (it passed the
+      // closing barrier) and its TMA store must have finished reading the
+      // staging tile
+      if (j > 0 && leader) tma_store_wait_read();
+#pragma unroll
+      for (int i = 0; i < (BN + 127) / 128; ++i)
+        if (r + 128 * i < BN) s_bias[r + 128 * i] = bv[i];
+      named_barrier(1, 128);
       if (!mbar_wait(&tfull[acc], (j >> 1) & 1)) {
         set_error(p.err, PTL_ERR_TIMEOUT);
         break;
       }
       tc_fence_after();
       const uint32_t taddr = tmem + uint32_t(acc * BN) + lane_off;
-      const int row = m0 + r;
       {
         // Tile epilogue: bias (+ReLU / +residual), written into the swizzled
         // staging tile, then TMA-stored by one thread (rows past the tensor
         // end are clipped by the store).
-        const bool leader = warp == 2 && lane == 0;
-        if (j > 0) {  // the previous tile's store must have finished reading the staging tile
-          if (leader) tma_store_wait_read();
-          named_barrier(1, 128);
-        }
-        const float* bb = p.bias ? p.bias + (MODE >= G_MOE1 ? expert * p.N_total : 0) + n0 : nullptr;
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t raw[32];
           tmem_ld32(taddr + 32 * c, raw);
@@ -298,26 +328,29 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-          if (bb) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 b4 = __ldg(reinterpret_cast<const float4*>(bb + 32 * c) + q);
-              v[4 * q] += b4.x;
-              v[4 * q + 1] += b4.y;
-              v[4 * q + 2] += b4.z;
-              v[4 * q + 3] += b4.w;
-            }
+          for (int q = 0; q < 8; ++q) {
+            const float4 b4 = *reinterpret_cast<const float4*>(s_bias + 32 * c + 4 * q);
+            v[4 * q] += b4.x;
+            v[4 * q + 1] += b4.y;
+            v[4 * q + 2] += b4.z;
+            v[4 * q + 3] += b4.w;
           }
           if (MODE == G_MOE1) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
           }
           if (MODE == G_OUT) {
-            if (row < p.M) {
-              float xr[32];
-              load_bf16x32(p.resid + size_t(row) * D + n0 + 32 * c, xr);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += xr[i];
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = res[4 * c + q];
+              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h2[i]);
+                v[8 * q + 2 * i] += f.x;
+                v[8 * q + 2 * i + 1] += f.y;
+              }
             }
             // 32 fp32 = one 128-byte box row: box c, chunks 0..7
             const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
@@ -359,6 +392,247 @@ __global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
   }
 }
 
+// ------------------------------------------------------------- CTA pairs
+// The dense GEMMs (QKV, output projection) on CTA pairs: a cluster of two
+// CTAs computes 256 x BN output tiles with M=256 tcgen05.mma (cta_group::2).
+// CTA c of the pair loads rows m0 + 128c of A and rows n0 + c*BN/2 of B into
+// its own shared memory; both loads count on CTA 0's `full` barrier; CTA 0's
+// single MMA thread issues the MMAs, which read both CTAs' operands and
+// write each CTA's 128 rows of D into its own TMEM; its commits arrive on
+// both CTAs' barriers.  Each CTA's epilogue drains its own TMEM and releases
+// the accumulator on CTA 0's `tempty` (one arrival per epilogue warp).  Per
+// SM a K slice costs 16 KB of A and BN/2 x 128 B of B (half the B bytes of a
+// 128-row tile for the same MMA time), so the same ring covers more of the
+// L2 latency.
+template <int BN, int MODE>
+struct PairCfg {
+  static constexpr int OUT_ELEM = MODE == G_OUT ? 4 : 2;
+  static constexpr int BOX_COLS = 128 / OUT_ELEM;
+  static constexpr int STAGING = 128 * BN * OUT_ELEM;
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = (BN / 2) * 64 * 2;
+  static constexpr int BIAS = BN * 4;
+  static constexpr int USABLE = 232448 - 1024 - 256 - 64;
+  static constexpr int STAGES_FIT = (USABLE - STAGING - BIAS) / (A_BYTES + B_BYTES);
+  static constexpr int STAGES = STAGES_FIT > 10 ? 10 : STAGES_FIT;
+  static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES) + STAGING + BIAS + 1024 + 256;
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static_assert(2 * BN <= 512 && BN % 32 == 0 && B_BYTES % 1024 == 0, "tile width");
+  static_assert(STAGES >= 2, "operand ring too small");
+};
+
+template <int BN, int MODE>
+__global__ void __launch_bounds__(192, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmOut, const GemmTcParams p) {
+  static_assert(MODE == G_QKV || MODE == G_OUT, "dense modes only");
+  using Cfg = PairCfg<BN, MODE>;
+  constexpr int STAGES = Cfg::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
+  uint8_t* sOut = sB + STAGES * Cfg::B_BYTES;
+  float* s_bias = reinterpret_cast<float*>(sOut + Cfg::STAGING);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg::STAGING + Cfg::BIAS);  // [stage] (CTA 0's counts)
+  uint64_t* empty = full + STAGES;    // [stage] ring slot free (both CTAs)
+  uint64_t* tfull = empty + STAGES;   // [2] accumulator ready (both CTAs)
+  uint64_t* tempty = tfull + 2;       // [2] accumulator drained (CTA 0's counts: 8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  __shared__ int s_ntiles;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t cr = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmOut);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  pdl_wait();
+  if (threadIdx.x == 0) s_ntiles = has_error(p.err) ? 0 : p.n_tiles_dense;
+  __syncthreads();
+  const int ntiles = s_ntiles;
+  const uint32_t tmem = *tmem_slot;
+  const int nkb = p.num_kb;
+  const int nN = p.N_total / BN;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // both CTAs: own halves of A and B, counted on CTA 0's full[s]
+      const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < ntiles && ok; tile += npairs) {
+        const int mt = tile / nN;
+        const int m0 = mt * 256 + 128 * int(cr), n0 = (tile - mt * nN) * BN + int(cr) * (BN / 2);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
+            set_error(p.err, PTL_ERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          if (cr == 0) mbar_arrive_expect_tx(&full[s], 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES));
+          const uint32_t fb = full0 + uint32_t(s) * 8u;
+          tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tmA, fb, kb * 64, m0);
+          tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tmB, fb, kb * 64, n0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && cr == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(256, BN);
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int tile = pair; tile < ntiles && ok; tile += npairs, ++j) {
+        const int acc = j & 1;
+        if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1)) {
+          set_error(p.err, PTL_ERR_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + uint32_t(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1)) {
+            set_error(p.err, PTL_ERR_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * Cfg::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + s * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16_ss_pair(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
+                              (kb | k) != 0);
+          umma_commit_pair(&empty[s], 0x3);
+        }
+        umma_commit_pair(&tfull[acc], 0x3);
+      }
+    }
+  } else {
+    // Epilogue warps 2..5 of each CTA: row r of this CTA's 128 rows.
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
+    const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
+    int j = 0;
+    for (int tile = pair; tile < ntiles; tile += npairs, ++j) {
+      const int mt = tile / nN;
+      const int m0 = mt * 256 + 128 * int(cr), n0 = (tile - mt * nN) * BN;
+      const int acc = j & 1;
+      const int row = m0 + r;
+      const float* bb = p.bias ? p.bias + n0 : nullptr;
+      float bv[(BN + 127) / 128];
+#pragma unroll
+      for (int i = 0; i < (BN + 127) / 128; ++i)
+        bv[i] = (bb && r + 128 * i < BN) ? __ldg(bb + r + 128 * i) : 0.f;
+      constexpr int NRES = MODE == G_OUT ? BN / 8 : 1;
+      uint4 res[NRES];
+      if (MODE == G_OUT) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0);
+#pragma unroll
+        for (int q = 0; q < NRES; ++q) res[q] = row < p.M ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
+      }
+      const bool leader = warp == 2 && lane == 0;
+      if (j > 0 && leader) tma_store_wait_read();
+#pragma unroll
+      for (int i = 0; i < (BN + 127) / 128; ++i)
+        if (r + 128 * i < BN) s_bias[r + 128 * i] = bv[i];
+      named_barrier(1, 128);
+      if (!mbar_wait(&tfull[acc], (j >> 1) & 1)) {
+        set_error(p.err, PTL_ERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + uint32_t(acc * BN) + lane_off;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(taddr + 32 * c, raw);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 b4 = *reinterpret_cast<const float4*>(s_bias + 32 * c + 4 * q);
+          v[4 * q] += b4.x;
+          v[4 * q + 1] += b4.y;
+          v[4 * q + 2] += b4.z;
+          v[4 * q + 3] += b4.w;
+        }
+        if (MODE == G_OUT) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u = res[4 * c + q];
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h2[i]);
+              v[8 * q + 2 * i] += f.x;
+              v[8 * q + 2 * i + 1] += f.y;
+            }
+          }
+          const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                         __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+        } else {
+          const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (c & 1) * 4 + q;
+            st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pack_bf16x2(v[8 * q], v[8 * q + 1]),
+                         pack_bf16x2(v[8 * q + 2], v[8 * q + 3]), pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                         pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          }
+        }
+      }
+      // this warp's rows of the accumulator are read: release it on CTA 0
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+      fence_proxy_async_smem();
+      named_barrier(1, 128);
+      if (leader) {
+#pragma unroll 1
+        for (int bx = 0; bx < BN / Cfg::BOX_COLS; ++bx)
+          tma_store_2d(&tmOut, sOut + bx * 16384, n0 + bx * Cfg::BOX_COLS, m0);
+        tma_store_commit();
+      }
+    }
+    if (warp == 2 && lane == 0) tma_store_wait_all();
+  }
+  tc_fence_before();
+  cluster_sync();  // no MMA, TMEM read or remote arrival of either CTA is outstanding
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, Cfg::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host
 static int num_sms() {
   static int n = 0;
@@ -390,18 +664,55 @@ static int launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
+// Launches the CTA-pair kernel: clusters of two CTAs, one pair per two SMs.
+template <int BN, int MODE>
+static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
+                       const GemmTcParams& p, cudaStream_t st) {
+  static int max_pairs = 0;  // co-resident clusters of two (one CTA per SM)
+  const int smem = PairCfg<BN, MODE>::SMEM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (max_pairs == 0) {
+    if (cudaFuncSetAttribute(gemm_pair_kernel<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return -1;
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, MODE>, &cfg) != cudaSuccess || n < 1)
+      n = num_sms() / 2;
+    max_pairs = n;
+  }
+  int pairs = max_pairs;
+  if (p.n_tiles_dense < pairs) pairs = p.n_tiles_dense;
+  if (pairs < 1) pairs = 1;
+  cfg.gridDim = dim3(2 * pairs);
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, MODE>, a, b, out, p) != cudaSuccess) return -1;
+  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+}
+
 int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorMap& qkv_out,
                     const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st) {
   GemmTcParams p{};
   p.M = T;
   p.N_total = QKV_N;
   p.num_kb = D / 64;
-  p.n_tiles_dense = ((T + 127) / 128) * (QKV_N / QKV_BN);
+  p.n_tiles_dense = ((T + 255) / 256) * (QKV_N / QKV_BN);  // 256-row pair tiles
   p.bias = bias;
   p.out = static_cast<__nv_bfloat16*>(qkv);
   p.ldo = QKV_N;
   p.err = err;
-  return launch_one<QKV_BN, G_QKV>(xn, w, qkv_out, p, p.n_tiles_dense, st);
+  return launch_pair<QKV_BN, G_QKV>(xn, w, qkv_out, p, st);
 }
 
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
@@ -410,13 +721,13 @@ int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtenso
   p.M = T;
   p.N_total = D;
   p.num_kb = D / 64;
-  p.n_tiles_dense = ((T + 127) / 128) * (D / OUT_BN);
+  p.n_tiles_dense = ((T + 255) / 256) * (D / OUT_BN);  // 256-row pair tiles
   p.bias = bias;
   p.resid = static_cast<const __nv_bfloat16*>(x);
   p.out_f32 = static_cast<float*>(x1);
   p.ldo = D;
   p.err = err;
-  return launch_one<OUT_BN, G_OUT>(attn, w, x1_out, p, p.n_tiles_dense, st);
+  return launch_pair<OUT_BN, G_OUT>(attn, w, x1_out, p, st);
 }
 
 int launch_gemm_moe1(const CUtensorMap& w1, const CUtensorMap& hbuf_out, const float* b1, const void* xn2,

@@ -742,8 +742,10 @@ int launch_layernorm(const void* x, const float* g, const float* b, void* y, int
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
                 cudaStream_t st) {
+  // one token per warp: every token's row load is in flight at once (the
+  // grid-stride loop only matters past 3 resident blocks per SM)
   int blocks = (T + GATE_WARPS - 1) / GATE_WARPS;
-  if (blocks > 148 * 2) blocks = 148 * 2;
+  if (blocks > 148 * 3 * 8) blocks = 148 * 3 * 8;
   if (dt == PTL_BF16) {
     if (launch_k(gate_kernel<__nv_bfloat16>, dim3(blocks), dim3(GATE_WARPS * 32), 0, st, 
         static_cast<const float*>(x1), g, b, wg, bg, static_cast<__nv_bfloat16*>(xn2), idx, w,

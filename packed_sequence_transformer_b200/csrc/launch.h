@@ -57,7 +57,8 @@ int launch_combine_f32(const float* y, const float* w, const float* x1, float* o
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
                     const char* ws, cudaStream_t st);
 
-// gemm_tc.cu (bf16, tcgen05)
+// gemm_tc.cu (bf16, tcgen05).  QKV and the output projection run on CTA
+// pairs: their B (weight) tensor maps have boxes of BN/2 rows.
 int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorMap& qkv_out,
                     const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st);
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
