@@ -237,15 +237,16 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
                     const void* resid, void* out, const ptl_layer_weights* w, int32_t* dbg_perm,
                     int32_t* dbg_off, const ptl_layer_weights* next = nullptr) {
   mark(c.st, PTL_KERNEL_ROUTE);
-  PTL_TRY(launch_route(idx, c.T, c.L, c.ws, dbg_perm, dbg_off, c.st));
+  PTL_TRY(launch_route(idx, c.T, c.L, c.ws, dbg_perm, dbg_off, c.dt == PTL_BF16 ? xn2 : nullptr, c.st));
   if (c.dt == PTL_BF16) {
-    CUtensorMap m1, m2, mh, my;
-    if (!map_bf16(&m1, w->w1, D, uint64_t(E) * F, D * 2, 64, MOE1_BN)) return PTL_ERR_CUDA;
-    if (!map_bf16(&m2, w->w2, F, uint64_t(E) * D, F * 2, 64, GEMM2_BN)) return PTL_ERR_CUDA;
+    CUtensorMap mx, m1, m2, mh, my;
+    if (!map_bf16(&mx, c.ws + c.L.xperm, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
+    if (!map_bf16(&m1, w->w1, D, uint64_t(E) * F, D * 2, 64, MOE1_BN / 2)) return PTL_ERR_CUDA;
+    if (!map_bf16(&m2, w->w2, F, uint64_t(E) * D, F * 2, 64, GEMM2_BN / 2)) return PTL_ERR_CUDA;
     if (!map_bf16(&mh, c.ws + c.L.hbuf, F, c.L.padded_rows, F * 2, 64, 128)) return PTL_ERR_CUDA;
     if (!map_bf16(&my, c.ws + c.L.ybuf, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
-    PTL_TRY(launch_gemm_moe1(m1, mh, F32(w->b1), xn2, c.L, c.ws, c.st));
+    PTL_TRY(launch_gemm_moe1(mx, m1, mh, F32(w->b1), c.L, c.ws, c.st));
     mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
     PTL_TRY(launch_gemm_moe2(mh, m2, my, F32(w->b2), c.L, c.ws, c.st));
     mark(c.st, PTL_KERNEL_COMBINE);
@@ -474,7 +475,7 @@ ptl_status ptl_route_build(const int32_t* topk_idx, int64_t total_tokens, int32_
   EndMark end_mark{c.st};
   mark(c.st, PTL_KERNEL_ROUTE);
   PTL_TRY(launch_chunk_hist(topk_idx, c.T, at<int32_t>(c, c.L.chunk_cnt), c.err, c.st));
-  PTL_TRY(launch_route(topk_idx, c.T, c.L, c.ws, perm, expert_off, c.st));
+  PTL_TRY(launch_route(topk_idx, c.T, c.L, c.ws, perm, expert_off, nullptr, c.st));
   return PTL_OK;
 }
 

@@ -188,7 +188,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __shared__ int s_units;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
@@ -214,6 +213,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   pdl_wait();  // qkv, the work list and the error word come from earlier kernels
+  pdl_trigger();  // dependents launch once this grid has passed its own wait
   if (threadIdx.x == 0) s_units = has_error(err) ? 0 : (*item_count) * H;
   __syncthreads();
   const int nunits = s_units;

@@ -18,9 +18,9 @@ constexpr int E = PTL_N_EXPERTS;   // 8
 constexpr int K = PTL_TOP_K;       // 2
 constexpr int QKV_N = 3 * D;       // 1536
 constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
-constexpr int MOE_BM = 128;        // rows per expert tile (padding granule)
+constexpr int MOE_BM = 256;        // rows per expert tile (padding granule; one CTA pair's M)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
-constexpr int GEMM2_BN = 128;      // N tile of the second expert GEMM
+constexpr int GEMM2_BN = 256;      // expert GEMM2 output columns per tile
 constexpr float LN_EPS = 1e-5f;
 constexpr float LOGIT_CLAMP = 15.0f;
 
@@ -46,7 +46,8 @@ struct WsLayout {
   size_t rowroute;    // int32 [2T + 8*128]   padded expert rows -> route (or -1)
   size_t tiles;       // int2 [max_tiles]     (expert, first padded row)
   size_t route_meta;  // int32 [32]: [0] n_tiles, [1..9] off, [10..18] padded off
-  size_t hbuf;        // dt [2T + 8*128][1024]  expert hidden rows (padded layout)
+  size_t xperm;       // bf16 build: [padded_rows][512] LayerNorm2 rows in expert (padded) order
+  size_t hbuf;        // dt [padded_rows][1024]  expert hidden rows (padded layout)
   size_t ybuf;        // per-route expert outputs awaiting the combine: bf16 build
                       // [2T + 8*128][512] bf16 in padded row order, fp32 build
                       // [2T][512] f32 in route order
@@ -98,6 +99,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->rowroute = take(4 * L->padded_rows);
   L->tiles = take(sizeof(int2) * L->max_tiles);
   L->route_meta = take(4 * 32);
+  L->xperm = take(dt == PTL_BF16 ? 2 * L->padded_rows * D : 0);
   L->hbuf = take(es * L->padded_rows * F);
   L->ybuf = take(dt == PTL_BF16 ? 2 * L->padded_rows * D : 4 * 2 * T * D);
   L->head_p = take(4 * T);
@@ -108,10 +110,12 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
 // ---------------------------------------------------------------- device
 // Programmatic dependent launch.  Every kernel of the library is launched so
 // that the next kernel in the stream may start its prologue while this one
-// drains: each kernel first allows its dependents to launch (trigger), and
-// waits for its own predecessor to complete (and its writes to be visible)
-// before it reads anything the predecessor produced.  Every kernel executes
-// the wait on every path, so completion stays transitive along the stream.
+// runs: each kernel waits for its own predecessor to complete (and its writes
+// to be visible) before it reads anything the predecessor produced, and only
+// then allows its dependents to launch (trigger).  So at most one kernel runs
+// ahead: a persistent kernel's CTAs cannot occupy SMs while a kernel two
+// places earlier still needs them.  Every kernel executes the wait on every
+// path, so completion stays transitive along the stream.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

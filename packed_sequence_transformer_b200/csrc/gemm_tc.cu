@@ -1,30 +1,38 @@
 // gemm_tc.cu -- tcgen05 GEMMs of the layer (bf16 in, fp32 accumulate in TMEM).
 //
-// Persistent kernel: one CTA per SM walks a static round-robin list of
-// 128 x BN output tiles, D = A B^T with A [M][K] and B = W [N][K] (nn.Linear
-// layout), both K-major in shared memory with the 128-byte swizzle.  Two TMEM
-// accumulators (2 x BN columns) let the epilogue of one tile run while the
-// tensor core works on the next.  Warp roles:
+// D = A B^T with A [M][K] and B = W [N][K] (nn.Linear layout), both K-major
+// in shared memory with the 128-byte swizzle, on CTA pairs: a cluster of two
+// CTAs (two SMs) computes 256 x BN output tiles with M=256 tcgen05.mma
+// (cta_group::2).  Each pair is persistent and walks a static round-robin list
+// of tiles.  CTA c of the pair holds rows m0 + 128c of A and rows
+// n0 + c*BN/2 of B in its own shared memory; both CTAs' loads count on CTA 0's
+// `full` barrier; CTA 0's single MMA thread issues the MMAs, which read both
+// CTAs' operands and write each CTA's 128 rows of D into its own TMEM; its
+// commits arrive on both CTAs' barriers.  Two TMEM accumulators (2 x BN
+// columns) let the epilogue of one tile run while the tensor core works on
+// the next.  Warp roles in each CTA:
 //   warp 0      TMA producer: one elected thread streams 64-wide K slices of
 //               A and B through a STAGES-deep ring of shared-memory buffers;
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
-//               K=16), commits each ring stage back to the producer and each
-//               finished accumulator to the epilogue;
+//   warp 1      allocates TMEM (both CTAs); in CTA 0 one thread issues the
+//               MMAs (M=256, N=BN, K=16), commits each ring stage back to both
+//               producers and each finished accumulator to both epilogues;
 //   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane),
-//               reads it with tcgen05.ld, frees the accumulator and applies
-//               the fused epilogue;
-//   warps 6..9  (expert GEMM1 only) gather the A rows -- token rows of the
-//               LayerNorm2 output picked through the route permutation --
-//               into the swizzled ring with 16-byte loads.
+//               reads it with tcgen05.ld, releases the accumulator on CTA 0
+//               (one arrival per warp), applies the fused epilogue and stages
+//               the tile for a TMA bulk-tensor store.
+// Sharing B across the pair halves B's shared-memory traffic per output: at
+// this problem size the GEMMs are bound by L2 -> SM operand traffic, so the
+// tile shape is chosen for bytes per FLOP.
 // Modes:
 //   QKV   qkv = xn Wqkv^T + b_qkv                         (A by TMA)
 //   OUT   x1  = x + attn Wo^T + b_o, kept in fp32         (A by TMA)
-//   MOE1  H[row] = ReLU(xn2[token(row)] W1[e]^T + b1[e])  (A gathered)
+//   MOE1  H[row] = ReLU(xperm[row] W1[e]^T + b1[e])       (A by TMA: the route
+//         builder copies each route's LayerNorm2 row to its padded row)
 //   MOE2  Y[row] = H[row] W2[e]^T + b2[e]                 (A by TMA)
 //         (per-route expert outputs in padded row order, bf16; the top-2
 //         weighted combine + residual runs in combine_bf16_kernel)
-// Every mode stages its output tile in shared memory (128-byte swizzle) and
-// writes it with TMA bulk-tensor stores.
+// The expert GEMMs' rows are padded per expert to 256 (one pair tile never
+// straddles two experts).
 // Every wait is bounded; a timeout sets PTL_ERR_TIMEOUT and unwinds.
 #include <cstdint>
 #include <cuda.h>
@@ -42,368 +50,23 @@ struct GemmTcParams {
   int M;                         // rows of A (dense modes)
   int N_total;                   // output columns (per expert in the MoE modes)
   int num_kb;                    // K / 64
-  int n_tiles_dense;             // dense modes: ceil(M / 128) * (N_total / BN)
+  int n_tiles_dense;             // dense modes: ceil(M / 256) * (N_total / BN)
   const float* bias;             // [N] or [E][N]; may be NULL
   const __nv_bfloat16* resid;    // OUT: x (row stride 512)
   __nv_bfloat16* out;            // output rows
   float* out_f32;                // OUT: x1 in fp32
   int ldo;                       // output row stride (elements)
-  const int32_t* rowroute;       // padded expert row -> route (or -1)
-  const int2* tiles;             // (expert, first padded row) per M tile
+  const int2* tiles;             // (expert, first padded row) per 256-row M tile
   const int32_t* meta;           // [0] = number of M tiles
   int32_t* zero_ptr;             // cleared by CTA 0 once the predecessor is done (may be NULL)
   int zero_n;
-  const __nv_bfloat16* gatherA;  // MOE1: xn2 [T][512]
   int32_t* err;
 };
 
 enum { G_QKV = 0, G_OUT = 1, G_MOE1 = 2, G_MOE2 = 3 };
 
-// Shared-memory plan per instantiation: the operand ring plus, for the
-// modes whose output is a plain tile, a staging tile that the epilogue fills
-// in the 128-byte-swizzled layout and TMA stores (boxes of 128 rows x 128 B).
-template <int BN, int MODE>
-struct GemmCfg {
-  static constexpr bool TMA_OUT = true;
-  static constexpr int OUT_ELEM = MODE == G_OUT ? 4 : 2;          // x1 is fp32, the rest bf16
-  static constexpr int BOX_COLS = 128 / OUT_ELEM;                  // columns per 128-byte box row
-  static constexpr int STAGING = TMA_OUT ? 128 * BN * OUT_ELEM : 0;
-  static constexpr int A_BYTES = 128 * 64 * 2;
-  static constexpr int B_BYTES = BN * 64 * 2;
-  static constexpr int BIAS = BN * 4;                              // the tile's bias slice
-  static constexpr int USABLE = 232448 - 1024 - 256 - 64;          // minus align, barriers, static
-  static constexpr int STAGES_FIT = (USABLE - STAGING - BIAS) / (A_BYTES + B_BYTES);
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int SMEM = STAGES * (A_BYTES + B_BYTES) + STAGING + BIAS + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;     // power of two >= 2 accumulators
-  static_assert(2 * BN <= 512, "two accumulators must fit in TMEM");
-  static_assert(STAGES >= 2, "operand ring too small");
-  static_assert(BN % 32 == 0 && (BN * OUT_ELEM) % 128 == 0, "tile width");
-};
-
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 u;
-    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    d[q] = u;
-  }
-}
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 u = s[q];
-    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 f = __bfloat1622float2(p[i]);
-      v[8 * q + 2 * i] = f.x;
-      v[8 * q + 2 * i + 1] = f.y;
-    }
-  }
-}
-
-template <int BN, int MODE>
-__device__ __forceinline__ void decode_tile(const GemmTcParams& p, int tile, int& expert, int& m0,
-                                            int& n0) {
-  const int nN = p.N_total / BN;
-  const int mt = tile / nN;
-  n0 = (tile - mt * nN) * BN;
-  if (MODE >= G_MOE1) {
-    const int2 tl = p.tiles[mt];
-    expert = tl.x;
-    m0 = tl.y;
-  } else {
-    expert = 0;
-    m0 = mt * 128;
-  }
-}
-
-template <int BN, int MODE>
-__global__ void __launch_bounds__(MODE == G_MOE1 ? 320 : 192, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmOut, const GemmTcParams p) {
-  using Cfg = GemmCfg<BN, MODE>;
-  constexpr int STAGES = Cfg::STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * Cfg::A_BYTES;
-  uint8_t* sOut = sB + STAGES * Cfg::B_BYTES;  // staging tile (TMA-stored modes)
-  float* s_bias = reinterpret_cast<float*>(sOut + Cfg::STAGING);  // the current tile's bias slice
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg::STAGING + Cfg::BIAS);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;   // [2] accumulator ready for the epilogue
-  uint64_t* tempty = tfull + 2;       // [2] accumulator drained by the epilogue
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  __shared__ int s_ntiles;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-  // prologue (overlaps the previous kernel's tail): barriers, TMEM, descriptors
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], MODE == G_MOE1 ? 1 + 128 : 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-    }
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    tma_prefetch_desc(&tmOut);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  pdl_wait();  // inputs, route tables and the error word come from earlier kernels
-  if (threadIdx.x == 0) {
-    int nt = MODE >= G_MOE1 ? p.meta[0] * (p.N_total / BN) : p.n_tiles_dense;
-    if (has_error(p.err)) nt = 0;
-    s_ntiles = nt;
-  }
-  if (p.zero_ptr && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < p.zero_n; i += blockDim.x) p.zero_ptr[i] = 0;
-  __syncthreads();
-  const int ntiles = s_ntiles;
-  const uint32_t tmem = *tmem_slot;
-  const int nkb = p.num_kb;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint32_t tx = (MODE == G_MOE1 ? 0u : uint32_t(Cfg::A_BYTES)) + uint32_t(Cfg::B_BYTES);
-      int it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-        int expert, m0, n0;
-        decode_tile<BN, MODE>(p, tile, expert, m0, n0);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
-            set_error(p.err, PTL_ERR_TIMEOUT);
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[s], tx);
-          if (MODE != G_MOE1) tma_load_2d(sA + s * Cfg::A_BYTES, &tmA, &full[s], kb * 64, m0);
-          tma_load_2d(sB + s * Cfg::B_BYTES, &tmB, &full[s], kb * 64, expert * p.N_total + n0);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(128, BN);
-      int it = 0, j = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++j) {
-        const int acc = j & 1;
-        if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1)) {
-          set_error(p.err, PTL_ERR_TIMEOUT);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d = tmem + uint32_t(acc * BN);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1)) {
-            set_error(p.err, PTL_ERR_TIMEOUT);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * Cfg::A_BYTES);
-          const uint32_t b0 = smem_u32(sB + s * Cfg::B_BYTES);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ss(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
-                         (kb | k) != 0);
-          umma_commit(&empty[s]);
-        }
-        umma_commit(&tfull[acc]);
-      }
-    }
-  } else if (warp >= 6) {
-    // Gather producer (expert GEMM1): thread r fills row r of each A stage
-    // with the 64-element K slice of its token's LayerNorm2 row, 16 bytes at
-    // a time, at the 128-byte-swizzled position TMA would have used.
-    const int r = threadIdx.x - 192;
-    constexpr int NKB = D / 64;  // K slices per tile (K = 512)
-    constexpr int DEPTH = 3;     // K slices in flight per thread
-    int it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
-      int expert, m0, n0;
-      decode_tile<BN, MODE>(p, tile, expert, m0, n0);
-      const int route = p.rowroute[m0 + r];
-      const uint4* src = route >= 0 ? reinterpret_cast<const uint4*>(p.gatherA + size_t(route >> 1) * D) : nullptr;
-      uint4 v[DEPTH][8];
-#pragma unroll
-      for (int kb = 0; kb < DEPTH - 1; ++kb)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) v[kb][c] = src ? __ldg(src + kb * 8 + c) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int kb = 0; kb < NKB; ++kb, ++it) {
-        if (kb + DEPTH - 1 < NKB) {  // the load DEPTH - 1 slices ahead
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            v[(kb + DEPTH - 1) % DEPTH][c] = src ? __ldg(src + (kb + DEPTH - 1) * 8 + c) : make_uint4(0, 0, 0, 0);
-        }
-        const int s = it % STAGES;
-        if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
-          set_error(p.err, PTL_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
-        const uint32_t row_addr = smem_u32(sA + s * Cfg::A_BYTES) + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(row_addr + ((c ^ (r & 7)) << 4), v[kb % DEPTH][c].x, v[kb % DEPTH][c].y, v[kb % DEPTH][c].z,
-                       v[kb % DEPTH][c].w);
-        fence_proxy_async_smem();
-        mbar_arrive(&full[s]);
-      }
-    }
-  } else {
-    // Epilogue warps 2..5: accumulator row r = TMEM lane r.
-    const int r = 32 * (warp & 3) + lane;
-    const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
-    int j = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
-      int expert, m0, n0;
-      decode_tile<BN, MODE>(p, tile, expert, m0, n0);
-      const int acc = j & 1;
-      const int row = m0 + r;
-      // Everything the epilogue reads besides the accumulator is fetched
-      // while the tile's MMAs run: the bias slice (into shared memory) and,
-      // for the output projection, this thread's residual row (registers).
-      const float* bb = p.bias ? p.bias + (MODE >= G_MOE1 ? expert * p.N_total : 0) + n0 : nullptr;
-      float bv[(BN + 127) / 128];
-#pragma unroll
-      for (int i = 0; i < (BN + 127) / 128; ++i)
-        bv[i] = (bb && r + 128 * i < BN) ? __ldg(bb + r + 128 * i) : 0.f;
-      constexpr int NRES = MODE == G_OUT ? BN / 8 : 1;
-      uint4 res[NRES];
-      if (MODE == G_OUT) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0);
-#pragma unroll
-        for (int q = 0; q < NRES; ++q) res[q] = row < p.M ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
-      }
-      const bool leader = warp == 2 && lane == 0;
-      // the previous tile's epilogue is done with s_bias (it passed the
-      // closing barrier) and its TMA store must have finished reading the
-      // staging tile
-      if (j > 0 && leader) tma_store_wait_read();
-#pragma unroll
-      for (int i = 0; i < (BN + 127) / 128; ++i)
-        if (r + 128 * i < BN) s_bias[r + 128 * i] = bv[i];
-      named_barrier(1, 128);
-      if (!mbar_wait(&tfull[acc], (j >> 1) & 1)) {
-        set_error(p.err, PTL_ERR_TIMEOUT);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t taddr = tmem + uint32_t(acc * BN) + lane_off;
-      {
-        // Tile epilogue: bias (+ReLU / +residual), written into the swizzled
-        // staging tile, then TMA-stored by one thread (rows past the tensor
-        // end are clipped by the store).
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(taddr + 32 * c, raw);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 b4 = *reinterpret_cast<const float4*>(s_bias + 32 * c + 4 * q);
-            v[4 * q] += b4.x;
-            v[4 * q + 1] += b4.y;
-            v[4 * q + 2] += b4.z;
-            v[4 * q + 3] += b4.w;
-          }
-          if (MODE == G_MOE1) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
-          }
-          if (MODE == G_OUT) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 u = res[4 * c + q];
-              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(h2[i]);
-                v[8 * q + 2 * i] += f.x;
-                v[8 * q + 2 * i + 1] += f.y;
-              }
-            }
-            // 32 fp32 = one 128-byte box row: box c, chunks 0..7
-            const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                           __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
-          } else {
-            // 32 bf16 = half a box row: box c/2, chunks (c%2)*4 .. +3
-            const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int chunk = (c & 1) * 4 + q;
-              st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pack_bf16x2(v[8 * q], v[8 * q + 1]),
-                           pack_bf16x2(v[8 * q + 2], v[8 * q + 3]), pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                           pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&tempty[acc]);
-        fence_proxy_async_smem();
-        named_barrier(1, 128);
-        if (leader) {
-#pragma unroll 1
-          for (int bx = 0; bx < BN / Cfg::BOX_COLS; ++bx)
-            tma_store_2d(&tmOut, sOut + bx * 16384, n0 + bx * Cfg::BOX_COLS, m0);
-          tma_store_commit();
-        }
-      }
-    }
-    if (Cfg::TMA_OUT && warp == 2 && lane == 0) tma_store_wait_all();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, Cfg::TMEM_COLS);
-  }
-}
-
-// ------------------------------------------------------------- CTA pairs
-// The dense GEMMs (QKV, output projection) on CTA pairs: a cluster of two
-// CTAs computes 256 x BN output tiles with M=256 tcgen05.mma (cta_group::2).
-// CTA c of the pair loads rows m0 + 128c of A and rows n0 + c*BN/2 of B into
-// its own shared memory; both loads count on CTA 0's `full` barrier; CTA 0's
-// single MMA thread issues the MMAs, which read both CTAs' operands and
-// write each CTA's 128 rows of D into its own TMEM; its commits arrive on
-// both CTAs' barriers.  Each CTA's epilogue drains its own TMEM and releases
-// the accumulator on CTA 0's `tempty` (one arrival per epilogue warp).  Per
-// SM a K slice costs 16 KB of A and BN/2 x 128 B of B (half the B bytes of a
-// 128-row tile for the same MMA time), so the same ring covers more of the
-// L2 latency.
+// Shared-memory plan: the operand ring, the output staging tile and the
+// tile's bias slice.
 template <int BN, int MODE>
 struct PairCfg {
   static constexpr int OUT_ELEM = MODE == G_OUT ? 4 : 2;
@@ -421,11 +84,27 @@ struct PairCfg {
   static_assert(STAGES >= 2, "operand ring too small");
 };
 
+// Pair tile `tile` -> (expert, first row of the pair's 256 rows, first column).
+template <int BN, int MODE>
+__device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile, int& expert, int& m0,
+                                                 int& n0) {
+  const int nN = p.N_total / BN;
+  const int mt = tile / nN;
+  n0 = (tile - mt * nN) * BN;
+  if (MODE >= G_MOE1) {
+    const int2 tl = p.tiles[mt];
+    expert = tl.x;
+    m0 = tl.y;
+  } else {
+    expert = 0;
+    m0 = mt * 256;
+  }
+}
+
 template <int BN, int MODE>
 __global__ void __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmOut, const GemmTcParams p) {
-  static_assert(MODE == G_QKV || MODE == G_OUT, "dense modes only");
   using Cfg = PairCfg<BN, MODE>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -444,7 +123,6 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t cr = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  pdl_trigger();
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -468,13 +146,18 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
-  pdl_wait();
-  if (threadIdx.x == 0) s_ntiles = has_error(p.err) ? 0 : p.n_tiles_dense;
+  pdl_wait();  // inputs, route tables and the error word come from earlier kernels
+  pdl_trigger();  // dependents launch once this grid has passed its own wait
+  if (threadIdx.x == 0) {
+    int nt = MODE >= G_MOE1 ? p.meta[0] * (p.N_total / BN) : p.n_tiles_dense;
+    s_ntiles = has_error(p.err) ? 0 : nt;
+  }
+  if (p.zero_ptr && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.zero_n; i += blockDim.x) p.zero_ptr[i] = 0;
   __syncthreads();
   const int ntiles = s_ntiles;
   const uint32_t tmem = *tmem_slot;
   const int nkb = p.num_kb;
-  const int nN = p.N_total / BN;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -482,9 +165,12 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);
       int it = 0;
       bool ok = true;
+      constexpr uint32_t tx = 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES);
       for (int tile = pair; tile < ntiles && ok; tile += npairs) {
-        const int mt = tile / nN;
-        const int m0 = mt * 256 + 128 * int(cr), n0 = (tile - mt * nN) * BN + int(cr) * (BN / 2);
+        int expert, m0, n0;
+        decode_pair_tile<BN, MODE>(p, tile, expert, m0, n0);
+        const int arow = m0 + 128 * int(cr);
+        const int brow = expert * p.N_total + n0 + int(cr) * (BN / 2);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
@@ -492,10 +178,10 @@ __global__ void __launch_bounds__(192, 1)
             ok = false;
             break;
           }
-          if (cr == 0) mbar_arrive_expect_tx(&full[s], 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES));
+          if (cr == 0) mbar_arrive_expect_tx(&full[s], tx);
           const uint32_t fb = full0 + uint32_t(s) * 8u;
-          tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tmA, fb, kb * 64, m0);
-          tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tmB, fb, kb * 64, n0);
+          tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tmA, fb, kb * 64, arow);
+          tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tmB, fb, kb * 64, brow);
         }
       }
     }
@@ -538,11 +224,12 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
     int j = 0;
     for (int tile = pair; tile < ntiles; tile += npairs, ++j) {
-      const int mt = tile / nN;
-      const int m0 = mt * 256 + 128 * int(cr), n0 = (tile - mt * nN) * BN;
+      int expert, m0, n0;
+      decode_pair_tile<BN, MODE>(p, tile, expert, m0, n0);
+      m0 += 128 * int(cr);  // this CTA's rows
       const int acc = j & 1;
       const int row = m0 + r;
-      const float* bb = p.bias ? p.bias + n0 : nullptr;
+      const float* bb = p.bias ? p.bias + (MODE >= G_MOE1 ? expert * p.N_total : 0) + n0 : nullptr;
       float bv[(BN + 127) / 128];
 #pragma unroll
       for (int i = 0; i < (BN + 127) / 128; ++i)
@@ -581,6 +268,10 @@ __global__ void __launch_bounds__(192, 1)
           v[4 * q + 1] += b4.y;
           v[4 * q + 2] += b4.z;
           v[4 * q + 3] += b4.w;
+        }
+        if (MODE == G_MOE1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
         }
         if (MODE == G_OUT) {
 #pragma unroll
@@ -645,29 +336,10 @@ static int num_sms() {
   return n;
 }
 
-template <int BN, int MODE>
-static int launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
-                      const GemmTcParams& p, int tiles_bound, cudaStream_t st) {
-  static bool configured = false;
-  const int smem = GemmCfg<BN, MODE>::SMEM;
-  if (!configured) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-      return -1;
-    configured = true;
-  }
-  int grid = tiles_bound < num_sms() ? tiles_bound : num_sms();
-  if (grid < 1) grid = 1;
-  if (launch_k(gemm_tc_kernel<BN, MODE>, dim3(grid), dim3(MODE == G_MOE1 ? 320 : 192), smem, st, a, b, out,
-               p) != 0)
-    return -1;
-  return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
-}
-
 // Launches the CTA-pair kernel: clusters of two CTAs, one pair per two SMs.
 template <int BN, int MODE>
 static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
-                       const GemmTcParams& p, cudaStream_t st) {
+                       const GemmTcParams& p, int tiles_bound, cudaStream_t st) {
   static int max_pairs = 0;  // co-resident clusters of two (one CTA per SM)
   const int smem = PairCfg<BN, MODE>::SMEM;
   cudaLaunchConfig_t cfg = {};
@@ -694,7 +366,7 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
     max_pairs = n;
   }
   int pairs = max_pairs;
-  if (p.n_tiles_dense < pairs) pairs = p.n_tiles_dense;
+  if (tiles_bound < pairs) pairs = tiles_bound;
   if (pairs < 1) pairs = 1;
   cfg.gridDim = dim3(2 * pairs);
   if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, MODE>, a, b, out, p) != cudaSuccess) return -1;
@@ -712,7 +384,7 @@ int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorM
   p.out = static_cast<__nv_bfloat16*>(qkv);
   p.ldo = QKV_N;
   p.err = err;
-  return launch_pair<QKV_BN, G_QKV>(xn, w, qkv_out, p, st);
+  return launch_pair<QKV_BN, G_QKV>(xn, w, qkv_out, p, p.n_tiles_dense, st);
 }
 
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
@@ -727,28 +399,25 @@ int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtenso
   p.out_f32 = static_cast<float*>(x1);
   p.ldo = D;
   p.err = err;
-  return launch_pair<OUT_BN, G_OUT>(attn, w, x1_out, p, st);
+  return launch_pair<OUT_BN, G_OUT>(attn, w, x1_out, p, p.n_tiles_dense, st);
 }
 
-int launch_gemm_moe1(const CUtensorMap& w1, const CUtensorMap& hbuf_out, const float* b1, const void* xn2,
-                     const WsLayout& L, char* ws, cudaStream_t st) {
+int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf_out,
+                     const float* b1, const WsLayout& L, char* ws, cudaStream_t st) {
   GemmTcParams p{};
   p.N_total = F;
   p.num_kb = D / 64;
   p.bias = b1;
   p.out = reinterpret_cast<__nv_bfloat16*>(ws + L.hbuf);
   p.ldo = F;
-  p.rowroute = reinterpret_cast<const int32_t*>(ws + L.rowroute);
   p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
-  p.gatherA = static_cast<const __nv_bfloat16*>(xn2);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
   // the route builder (the previous kernel) has consumed the per-chunk expert
   // counts: clear them for the next gate
   p.zero_ptr = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
   p.zero_n = int(L.n_chunks * E);
-  // A is gathered by the kernel; the A descriptor slot is unused
-  return launch_one<MOE1_BN, G_MOE1>(w1, w1, hbuf_out, p, int(L.max_tiles) * (F / MOE1_BN), st);
+  return launch_pair<MOE1_BN, G_MOE1>(xperm, w1, hbuf_out, p, int(L.max_tiles) * (F / MOE1_BN), st);
 }
 
 int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUtensorMap& ybuf_out,
@@ -759,11 +428,10 @@ int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUten
   p.bias = b2;
   p.out = reinterpret_cast<__nv_bfloat16*>(ws + L.ybuf);
   p.ldo = D;
-  p.rowroute = reinterpret_cast<const int32_t*>(ws + L.rowroute);
   p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
-  return launch_one<GEMM2_BN, G_MOE2>(hbuf, w2, ybuf_out, p, int(L.max_tiles) * (D / GEMM2_BN), st);
+  return launch_pair<GEMM2_BN, G_MOE2>(hbuf, w2, ybuf_out, p, int(L.max_tiles) * (D / GEMM2_BN), st);
 }
 
 }  // namespace ptl

@@ -101,8 +101,8 @@ template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) ln_rows_kernel(const TI* __restrict__ x, const float* __restrict__ g,
                                                       const float* __restrict__ b, TO* __restrict__ y,
                                                       int T) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= T) return;
@@ -146,8 +146,8 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
                                                         int2* __restrict__ items, int32_t* item_count,
                                                         int32_t* lvl_hist, int32_t* lvl_start,
                                                         int32_t* lvl_fill, int max_levels, int32_t* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ int s_bad;
   __shared__ int s_total;
   const int tid = threadIdx.x;
@@ -260,11 +260,11 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
   // gate weights [8][512] in shared memory; lane l reads columns q*128 + 4l..4l+3,
   // i.e. consecutive 16-byte words across the warp (no bank conflicts)
   __shared__ __align__(16) float s_wg[E * D];
-  pdl_trigger();
   for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
     reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
   __syncthreads();
   pdl_wait();  // x1 comes from the previous kernel
+  pdl_trigger();  // dependents launch once this grid has passed its own wait
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   for (int t = blockIdx.x * GATE_WARPS + warp; t < T_; t += gridDim.x * GATE_WARPS) {
@@ -325,8 +325,8 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
 // build); out-of-range expert ids set PTL_ERR_SHAPE and are skipped.
 __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restrict__ idx, int n_routes,
                                                          int32_t* __restrict__ chunk_cnt, int32_t* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ int32_t s_hist[E];
   if (threadIdx.x < E) s_hist[threadIdx.x] = 0;
   __syncthreads();
@@ -347,26 +347,37 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int32_t* __restri
 // Stable counting sort: slot of r inside expert e = routes of e in earlier
 // chunks + routes of e in earlier warps of this chunk + earlier lanes of
 // this warp with the same expert.  Writes perm (compact slots), rowroute
-// (padded slots: every expert's rows start on a 128-row boundary) and, in
-// block 0, the padding (-1), the expert tile list and the offsets.
-__global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
+// (padded slots: every expert's rows start on a MOE_BM-row boundary) and, in
+// block 0, the padding (-1), the expert tile list and the offsets.  In the
+// bf16 build (xn2 != NULL) it also copies each route's LayerNorm2 row to its
+// padded slot of xperm, so the first expert GEMM reads its A rows by TMA
+// (padding rows are left unwritten: their products land in padding rows of
+// the expert outputs, which nothing reads).
+constexpr int ROUTE_THREADS = 1024;  // the sort uses the first ROUTE_CHUNK threads, the row copy all
+
+__global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(
     const int32_t* __restrict__ idx, int n_routes, const int32_t* __restrict__ chunk_cnt,
     int32_t* __restrict__ perm, int32_t* __restrict__ pos, int32_t* __restrict__ rowroute,
     int2* __restrict__ tiles, int32_t* __restrict__ meta, int32_t* __restrict__ dbg_perm,
-    int32_t* __restrict__ dbg_off, const int32_t* err) {
-  pdl_trigger();
+    int32_t* __restrict__ dbg_off, const __nv_bfloat16* __restrict__ xn2,
+    __nv_bfloat16* __restrict__ xperm, const int32_t* err) {
   pdl_wait();
-  __shared__ int32_t s_red[ROUTE_CHUNK / 32][2 * E];
+  pdl_trigger();
+  constexpr int NW = ROUTE_THREADS / 32;
+  __shared__ int32_t s_red[NW][2 * E];
   __shared__ int32_t s_pre[E], s_tot[E], s_off[E + 1], s_poff[E + 1];
   __shared__ int32_t s_wcnt[ROUTE_CHUNK / 32][E];
+  __shared__ int32_t s_slot[ROUTE_CHUNK];  // padded slot of each route of the chunk (-1: none)
   if (has_error(err)) return;
   const int c = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n_chunks = (n_routes + ROUTE_CHUNK - 1) / ROUTE_CHUNK;
+  // routes of each expert in the chunks before this one (acc[0..E)) and in all
+  // chunks (acc[E..2E))
   int acc[2 * E];
 #pragma unroll
   for (int e = 0; e < 2 * E; ++e) acc[e] = 0;
-  for (int cc = tid; cc < n_chunks; cc += ROUTE_CHUNK) {
+  for (int cc = tid; cc < n_chunks; cc += ROUTE_THREADS) {
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int v = chunk_cnt[cc * E + e];
@@ -389,7 +400,7 @@ __global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
   if (tid < 2 * E) {
     int v = 0;
 #pragma unroll
-    for (int w = 0; w < ROUTE_CHUNK / 32; ++w) v += s_red[w][tid];
+    for (int w = 0; w < NW; ++w) v += s_red[w][tid];
     if (tid < E) s_pre[tid] = v; else s_tot[tid - E] = v;
   }
   __syncthreads();
@@ -401,31 +412,68 @@ __global__ void __launch_bounds__(ROUTE_CHUNK) route_kernel(
       s_poff[e + 1] = s_poff[e] + (s_tot[e] + MOE_BM - 1) / MOE_BM * MOE_BM;
     }
   }
+  // threads 0..ROUTE_CHUNK-1: one route each (whole warps, so the warp match is uniform)
+  const bool sorter = tid < ROUTE_CHUNK;
   const int r = c * ROUTE_CHUNK + tid;
-  bool valid = r < n_routes;
+  bool valid = sorter && r < n_routes;
   int e = valid ? idx[r] : E;
   if (e < 0 || e >= E) {  // never index with an id outside [0, E)
     e = E;
     valid = false;
   }
-  const unsigned same = __match_any_sync(0xffffffffu, e);
-  const int rank = __popc(same & ((1u << lane) - 1u));
-  if (valid && rank == 0) s_wcnt[warp][e] = __popc(same);
+  int rank = 0;
+  if (sorter) {
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    rank = __popc(same & ((1u << lane) - 1u));
+    if (valid && rank == 0) s_wcnt[warp][e] = __popc(same);
+  }
   __syncthreads();
-  if (valid) {
-    int j = s_pre[e] + rank;
-    for (int w = 0; w < warp; ++w) j += s_wcnt[w][e];
-    perm[s_off[e] + j] = r;
-    if (dbg_perm) dbg_perm[s_off[e] + j] = r;
-    rowroute[s_poff[e] + j] = r;
-    pos[r] = s_poff[e] + j;
+  if (sorter) {
+    int slot = -1;
+    if (valid) {
+      int j = s_pre[e] + rank;
+      for (int w = 0; w < warp; ++w) j += s_wcnt[w][e];
+      perm[s_off[e] + j] = r;
+      if (dbg_perm) dbg_perm[s_off[e] + j] = r;
+      slot = s_poff[e] + j;
+      rowroute[slot] = r;
+      pos[r] = slot;
+    }
+    s_slot[tid] = slot;
+  }
+  if (xn2 != nullptr) {
+    // every warp copies 8 of the chunk's 256 rows (1 KB each): lane l moves
+    // 16-byte words l and l + 32 of each
+    __syncthreads();
+    constexpr int RPW = ROUTE_CHUNK / NW;  // rows per warp
+#pragma unroll
+    for (int h = 0; h < RPW; h += 4) {  // four rows (8 loads per lane) in flight
+      uint4 v[4][2];
+      int dst[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = warp * RPW + h + q;
+        dst[q] = s_slot[k];
+        const uint4* src = reinterpret_cast<const uint4*>(xn2 + size_t((c * ROUTE_CHUNK + k) >> 1) * D);
+        v[q][0] = dst[q] >= 0 ? __ldg(src + lane) : make_uint4(0, 0, 0, 0);
+        v[q][1] = dst[q] >= 0 ? __ldg(src + 32 + lane) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (dst[q] < 0) continue;
+        uint4* d = reinterpret_cast<uint4*>(xperm + size_t(dst[q]) * D);
+        d[lane] = v[q][0];
+        d[32 + lane] = v[q][1];
+      }
+    }
   }
   if (c == 0) {
+    __syncthreads();  // s_off / s_poff are written by thread 0
     for (int ee = 0; ee < E; ++ee) {
-      for (int i = s_off[ee + 1] - s_off[ee] + tid; i < s_poff[ee + 1] - s_poff[ee]; i += ROUTE_CHUNK)
+      for (int i = s_off[ee + 1] - s_off[ee] + tid; i < s_poff[ee + 1] - s_poff[ee]; i += ROUTE_THREADS)
         rowroute[s_poff[ee] + i] = -1;
       const int nt = (s_poff[ee + 1] - s_poff[ee]) / MOE_BM;
-      for (int j = tid; j < nt; j += ROUTE_CHUNK)
+      for (int j = tid; j < nt; j += ROUTE_THREADS)
         tiles[s_poff[ee] / MOE_BM + j] = make_int2(ee, s_poff[ee] + j * MOE_BM);
     }
     if (tid == 0) meta[0] = s_poff[E] / MOE_BM;
@@ -444,8 +492,8 @@ __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, cons
                                                    const float* __restrict__ w,
                                                    const float* __restrict__ bias,
                                                    float* __restrict__ p, int T_) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T_) return;
@@ -467,8 +515,8 @@ __global__ void __launch_bounds__(1024) head_compact_kernel(const float* __restr
                                                             const uint8_t* __restrict__ mask,
                                                             float* __restrict__ probs,
                                                             int32_t* __restrict__ n_pred, int T_) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ int32_t s_scan[1024];
   __shared__ int32_t s_carry;
   if (threadIdx.x == 0) s_carry = 0;
@@ -509,8 +557,8 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
                                                        const int2* __restrict__ tiles,
                                                        const int32_t* __restrict__ meta,
                                                        const int32_t* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float sA[16][64 + 4];
   __shared__ float sB[16][64 + 4];
   __shared__ int s_arow[64];
@@ -518,11 +566,11 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
   const int tid = threadIdx.x;
   int row0, expert = 0;
   if (MODE >= 2) {
-    const int tile = blockIdx.x >> 1;
+    const int tile = blockIdx.x / (MOE_BM / 64);
     if (tile >= meta[0]) return;
     const int2 tl = tiles[tile];
     expert = tl.x;
-    row0 = tl.y + (blockIdx.x & 1) * 64;
+    row0 = tl.y + (blockIdx.x % (MOE_BM / 64)) * 64;
   } else {
     row0 = blockIdx.x * 64;
   }
@@ -607,8 +655,8 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
                                                            const float* __restrict__ ln_b,
                                                            __nv_bfloat16* __restrict__ xn,
                                                            const int32_t* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   if (has_error(err)) return;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -644,8 +692,8 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const float* __restric
                                                           const float* __restrict__ x1,
                                                           float* __restrict__ out, int T_,
                                                           const int32_t* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   if (has_error(err)) return;
   const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= size_t(T_) * D) return;
@@ -664,8 +712,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
                                                        const int2* __restrict__ items,
                                                        const int32_t* __restrict__ item_count,
                                                        const int32_t* err) {
-  pdl_trigger();
   pdl_wait();
+  pdl_trigger();
   __shared__ float sK[64][DH + 1];
   __shared__ float sV[64][DH + 1];
   if (has_error(err)) return;
@@ -765,14 +813,16 @@ int launch_chunk_hist(const int32_t* idx, int T, int32_t* chunk_cnt, int32_t* er
 }
 
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
-                 int32_t* dbg_off, cudaStream_t st) {
+                 int32_t* dbg_off, const void* xn2, cudaStream_t st) {
   const int n = 2 * T;
-  if (launch_k(route_kernel, dim3((n + ROUTE_CHUNK - 1) / ROUTE_CHUNK), dim3(ROUTE_CHUNK), 0, st, 
+  if (launch_k(route_kernel, dim3((n + ROUTE_CHUNK - 1) / ROUTE_CHUNK), dim3(ROUTE_THREADS), 0, st, 
       idx, n, reinterpret_cast<const int32_t*>(ws + L.chunk_cnt),
       reinterpret_cast<int32_t*>(ws + L.perm), reinterpret_cast<int32_t*>(ws + L.pos),
       reinterpret_cast<int32_t*>(ws + L.rowroute),
       reinterpret_cast<int2*>(ws + L.tiles), reinterpret_cast<int32_t*>(ws + L.route_meta),
-      dbg_perm, dbg_off, reinterpret_cast<const int32_t*>(ws + L.err))) return -1;
+      dbg_perm, dbg_off, static_cast<const __nv_bfloat16*>(xn2),
+      xn2 ? reinterpret_cast<__nv_bfloat16*>(ws + L.xperm) : nullptr,
+      reinterpret_cast<const int32_t*>(ws + L.err))) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
@@ -802,7 +852,7 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
   const int2* tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
   const int32_t* err = reinterpret_cast<const int32_t*>(ws + L.err);
-  dim3 grid(mode >= 2 ? unsigned(2 * L.max_tiles) : unsigned((M + 63) / 64), unsigned((N + 63) / 64));
+  dim3 grid(mode >= 2 ? unsigned((MOE_BM / 64) * L.max_tiles) : unsigned((M + 63) / 64), unsigned((N + 63) / 64));
   int rc = 0;
   switch (mode) {
     case 0: rc = launch_k(gemm_f32_kernel<0>, dim3(grid), dim3(256), 0, st, A, lda, W, bias, R, C, ldc, M, N, Kd, rr, tiles, meta, err); break;

@@ -41,8 +41,10 @@ int launch_gate(const void* x1, const float* g, const float* b, const float* wg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
                 cudaStream_t st);
 int launch_chunk_hist(const int32_t* idx, int T, int32_t* chunk_cnt, int32_t* err, cudaStream_t st);
+// xn2 (bf16 build, nullable): also copy each route's LayerNorm2 row to its
+// padded slot of the workspace's xperm
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
-                 int32_t* dbg_off, cudaStream_t st);
+                 int32_t* dbg_off, const void* xn2, cudaStream_t st);
 int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, float* probs,
                 int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st);
 int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const float* bias,
@@ -63,8 +65,8 @@ int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorM
                     const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st);
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
                     const float* bias, const void* x, void* x1, int T, int32_t* err, cudaStream_t st);
-int launch_gemm_moe1(const CUtensorMap& w1, const CUtensorMap& hbuf_out, const float* b1, const void* xn2,
-                     const WsLayout& L, char* ws, cudaStream_t st);
+int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf_out,
+                     const float* b1, const WsLayout& L, char* ws, cudaStream_t st);
 int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUtensorMap& ybuf_out,
                      const float* b2, const WsLayout& L, char* ws, cudaStream_t st);
 
