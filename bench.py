@@ -265,9 +265,10 @@ def run_ours(args):
     with torch.cuda.graph(graph, stream=stream):
         step()
     torch.cuda.synchronize()
-    # work list + LayerNorm1 of layer 0 + 8 kernels per layer (each layer's
+    # work list + LayerNorm1 of layer 0 + 7 kernels per layer (QKV, attention,
+    # out-projection, gate + route, two expert GEMMs, combine; each layer's
     # combine writes the next layer's LayerNorm1) + head and its compaction
-    launches_per_step = 1 + 1 + 8 * n_layers + (2 if head is not None else 0)
+    launches_per_step = 1 + 1 + 7 * n_layers + (2 if head is not None else 0)
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
@@ -339,8 +340,8 @@ def run_ours(args):
         "gemm_out": ("tensor", 2 * T * 512 * 512),
         "gemm_expert1": ("tensor", 2 * (2 * T) * 512 * 1024),
         "gemm_expert2": ("tensor", 2 * (2 * T) * 1024 * 512),
-        "combine": ("hbm", T * (2 * 1024 + 2048 + 1024 + 16)),
-        "gate": ("hbm", T * (1024 + 1024 + 16)),
+        "combine": ("hbm", T * (2 * 1024 + 2048 + 1024 + 1024 + 16)),
+        "gate": ("hbm", T * (2048 + 2 * 1024 + 24)),
         "layernorm": ("hbm", T * 2048),
         "route": ("hbm", T * 24),
     }

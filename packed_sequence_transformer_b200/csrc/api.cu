@@ -156,12 +156,13 @@ inline T* at(const Call& c, size_t off) { return reinterpret_cast<T*>(c.ws + off
   } while (0)
 
 // Clears the error word (every top-level call reports only its own errors)
-// and the per-chunk expert counts that the gate accumulates into (laid out
-// right behind the error word; the first expert GEMM clears them again once
-// the route builder has used them).
+// and the routing state the gate starts from (per-chunk expert counts, the
+// fused gate + route look-back state; the first expert GEMM of each layer
+// clears them again once they are used).  The work list in between is
+// rewritten by the work-list kernel.
 ptl_status begin(const Call& c) {
   mark(c.st, PTL_KERNEL_CLEAR);
-  return cudaMemsetAsync(c.ws, 0, c.L.items, c.st) == cudaSuccess ? PTL_OK : PTL_ERR_CUDA;
+  return cudaMemsetAsync(c.ws, 0, c.L.clear_end, c.st) == cudaSuccess ? PTL_OK : PTL_ERR_CUDA;
 }
 
 // xn_ready: LayerNorm1 of x is already in the workspace (the previous
@@ -231,6 +232,9 @@ ptl_status step_gate(const Call& c, const void* x1, void* xn2, int32_t* idx, flo
 
 // Routes + both expert GEMMs + combine + residual.  The per-chunk expert
 // counts must already be in the workspace.
+ptl_status step_experts(const Call& c, const float* wts, const void* resid, void* out,
+                        const ptl_layer_weights* w, const ptl_layer_weights* next);
+
 // next (bf16 build, nullable): the following layer, whose LayerNorm1 of `out`
 // the combine also writes into the workspace.
 ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const float* wts,
@@ -238,7 +242,29 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
                     int32_t* dbg_off, const ptl_layer_weights* next = nullptr) {
   mark(c.st, PTL_KERNEL_ROUTE);
   PTL_TRY(launch_route(idx, c.T, c.L, c.ws, dbg_perm, dbg_off, c.dt == PTL_BF16 ? xn2 : nullptr, c.st));
-  if (c.dt == PTL_BF16) {
+  if (c.dt == PTL_BF16) return step_experts(c, wts, resid, out, w, next);
+  // the route builder has consumed the per-chunk expert counts: clear them
+  // for the next gate (the bf16 path's first expert GEMM does this)
+  if (cudaMemsetAsync(c.ws + c.L.chunk_cnt, 0, sizeof(int32_t) * size_t(c.L.n_chunks) * E, c.st) != cudaSuccess)
+    return PTL_ERR_CUDA;
+  mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
+  PTL_TRY(launch_gemm_f32(2, static_cast<const float*>(xn2), D, F32(w->w1), F32(w->b1), nullptr,
+                          at<float>(c, c.L.hbuf), F, 0, F, D, c.L, c.ws, c.st));
+  mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
+  PTL_TRY(launch_gemm_f32(3, at<float>(c, c.L.hbuf), F, F32(w->w2), F32(w->b2), nullptr,
+                          at<float>(c, c.L.ybuf), D, 0, D, F, c.L, c.ws, c.st));
+  mark(c.st, PTL_KERNEL_COMBINE);
+  PTL_TRY(launch_combine_f32(at<float>(c, c.L.ybuf), wts, static_cast<const float*>(resid),
+                             static_cast<float*>(out), c.T, c.err, c.st));
+  return PTL_OK;
+}
+
+// bf16: both expert GEMMs over the routed rows already in the workspace
+// (xperm, tiles, meta, pos), then the combine + residual (+ the next layer's
+// LayerNorm1 inside a stack).
+ptl_status step_experts(const Call& c, const float* wts, const void* resid, void* out,
+                        const ptl_layer_weights* w, const ptl_layer_weights* next) {
+  {
     CUtensorMap mx, m1, m2, mh, my;
     if (!map_bf16(&mx, c.ws + c.L.xperm, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
     if (!map_bf16(&m1, w->w1, D, uint64_t(E) * F, D * 2, 64, MOE1_BN / 2)) return PTL_ERR_CUDA;
@@ -254,16 +280,6 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
                                 static_cast<const float*>(resid), out, c.T,
                                 next ? F32(next->ln1_g) : nullptr, next ? F32(next->ln1_b) : nullptr,
                                 next ? c.ws + c.L.xn : nullptr, c.err, c.st));
-  } else {
-    mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
-    PTL_TRY(launch_gemm_f32(2, static_cast<const float*>(xn2), D, F32(w->w1), F32(w->b1), nullptr,
-                            at<float>(c, c.L.hbuf), F, 0, F, D, c.L, c.ws, c.st));
-    mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
-    PTL_TRY(launch_gemm_f32(3, at<float>(c, c.L.hbuf), F, F32(w->w2), F32(w->b2), nullptr,
-                            at<float>(c, c.L.ybuf), D, 0, D, F, c.L, c.ws, c.st));
-    mark(c.st, PTL_KERNEL_COMBINE);
-    PTL_TRY(launch_combine_f32(at<float>(c, c.L.ybuf), wts, static_cast<const float*>(resid),
-                               static_cast<float*>(out), c.T, c.err, c.st));
   }
   return PTL_OK;
 }
@@ -280,10 +296,22 @@ ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu
   if ((s = step_out(c, c.ws + c.L.attn, x, c.ws + c.L.x1, w)) != PTL_OK) return s;
   int32_t* idx = at<int32_t>(c, c.L.idx);
   float* wts = at<float>(c, c.L.wgt);
-  if ((s = step_gate(c, c.ws + c.L.x1, c.ws + c.L.xn2, idx, wts, w)) != PTL_OK) return s;
-  if ((s = step_moe(c, c.ws + c.L.xn2, idx, wts, c.ws + c.L.x1, out, w, dbg ? dbg->perm : nullptr,
-                    dbg ? dbg->expert_off : nullptr, next)) != PTL_OK)
-    return s;
+  if (c.dt == PTL_BF16) {
+    // gate + route builder in one kernel, then the experts and the combine
+    mark(c.st, PTL_KERNEL_GATE);
+    PTL_TRY(launch_gate_route(c.ws + c.L.x1, F32(w->ln2_g), F32(w->ln2_b), F32(w->w_gate), F32(w->b_gate), c.T,
+                              c.L, c.ws, c.st));
+    if (dbg && (dbg->perm || dbg->expert_off)) {
+      mark(c.st, PTL_KERNEL_ROUTE);
+      PTL_TRY(launch_route_debug(c.T, c.L, c.ws, dbg->perm, dbg->expert_off, c.st));
+    }
+    if ((s = step_experts(c, wts, c.ws + c.L.x1, out, w, next)) != PTL_OK) return s;
+  } else {
+    if ((s = step_gate(c, c.ws + c.L.x1, c.ws + c.L.xn2, idx, wts, w)) != PTL_OK) return s;
+    if ((s = step_moe(c, c.ws + c.L.xn2, idx, wts, c.ws + c.L.x1, out, w, dbg ? dbg->perm : nullptr,
+                      dbg ? dbg->expert_off : nullptr, next)) != PTL_OK)
+      return s;
+  }
   if (dbg && (dbg->topk_idx || dbg->topk_w)) mark(c.st, PTL_KERNEL_COPY);
   if (dbg && dbg->topk_idx &&
       cudaMemcpyAsync(dbg->topk_idx, idx, sizeof(int32_t) * 2 * c.T, cudaMemcpyDeviceToDevice, c.st) !=

@@ -6,18 +6,20 @@
 // block above the diagonal is touched).  A persistent CTA per SM takes its
 // units in snake order over the grid and splits them between two streams
 // (each unit to the stream with fewer key-block steps so far), one per
-// softmax warpgroup; a stream is a sequence of steps (unit, key block kb) and
-// the two streams' steps are interleaved:
+// softmax warpgroup; a stream is a sequence of steps (unit, key block kb).
+// The producer and the MMA issuer serve the two streams independently (each
+// polls both and advances whichever is ready), so a stream never waits for
+// the other's softmax:
 //
 //   warp 0      TMA producer: the Q tile [128 x 64] of each stream's current
 //               unit, and per step the K and V tiles [128 x 64] through a
-//               4-deep ring, straight from the packed qkv rows (128-byte
-//               swizzle);
+//               per-stream 2-deep ring, straight from the packed qkv rows
+//               (128-byte swizzle);
 //   warp 1      MMA issuer: for a step of stream g, S = Q K^T (M=128, N = the
-//               keys of this block rounded up to 16) into TMEM S[g], then --
-//               once warpgroup g has written P for its previous step -- that
-//               step's O[g] += P V (M=128, N=64, K = its key count; V is the
-//               MN-major operand) into TMEM; a unit's first PV overwrites O;
+//               keys of this block rounded up to 16) into TMEM S[g], and --
+//               once warpgroup g has written P for that step -- O[g] += P V
+//               (M=128, N=64, K = its key count; V is the MN-major operand)
+//               into TMEM; a unit's first PV overwrites O;
 //   warps 2..5  softmax warpgroup 0, warps 6..9 warpgroup 1: thread r owns
 //               query row r (TMEM lane r) of its stream's unit; per step it
 //               reads its S row, masks keys past its position and past the
@@ -44,11 +46,11 @@ namespace ptl {
 using namespace sm100;
 
 constexpr int ATT_TILE_BYTES = ATT_BLK * DH * 2;  // 16 KB
-// Four stages: each stream holds one K/V stage until its deferred PV is done
-// and needs the next one loaded before its next QK^T can start.
-constexpr int ATT_KV_STAGES = 4;
-// Q[2] + (K,V)[3] + P[2][2 column blocks]
-constexpr int ATT_SMEM_TILES = 2 + 2 * ATT_KV_STAGES + 4;
+// K/V ring stages per stream: a stream holds one stage until its deferred
+// PV is done and needs the next one loaded before its next QK^T can start.
+constexpr int ATT_KV_STAGES = 2;
+// Q[2] + (K,V)[2 streams][stages] + P[2][2 column blocks]
+constexpr int ATT_SMEM_TILES = 2 + 2 * 2 * ATT_KV_STAGES + 4;
 constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 256;
 constexpr int ATT_THREADS = 320;  // producer, MMA, two softmax warpgroups
 
@@ -98,8 +100,9 @@ __device__ __forceinline__ int keys16(int L, int kb) {
 // Each stream's next unit is looked up one unit ahead, so switching units
 // does not wait on the work-list and offset loads.
 // One stream's position in its step sequence, plus (for the MMA issuer) its
-// deferred PV.  The two streams are held in named registers and swapped, never
-// indexed by the stream number, so nothing lands in local memory.
+// deferred PV and (for the producer) whether the unit's Q load is issued.
+// The two streams are held in named registers, never indexed by the stream
+// number, so nothing lands in local memory.
 struct StreamPos {
   int g;             // the stream (softmax warpgroup)
   int kb, n, uc;     // key block of the current unit, steps so far, units started
@@ -108,11 +111,12 @@ struct StreamPos {
   CtaWalker walk;
   int pv_n, pv_st, pv_k16, pv_uc;  // the step whose PV is still to be issued (-1: none)
   bool pv_first;
+  bool q_sent;       // producer: the current unit's Q tile load is issued
 };
 
-// The interleaved step sequence both the producer and the MMA issuer walk:
-// `a` is the stream whose turn it is; after each step the streams swap while
-// both have steps left.
+// Both streams' step sequences as the producer and the MMA issuer walk them
+// (`a` = stream 0, `b` = stream 1); each role advances a stream when that
+// stream's next step can proceed.
 struct AttnStepGen {
   int nunits;
   StreamPos a, b;
@@ -130,6 +134,7 @@ struct AttnStepGen {
     sp.pv_n = -1;
     sp.pv_st = sp.pv_k16 = sp.pv_uc = 0;
     sp.pv_first = false;
+    sp.q_sent = false;
     fetch_next(items, cu, sp);
     sp.live = sp.nxt_live;
     sp.u = sp.nxt;
@@ -140,27 +145,17 @@ struct AttnStepGen {
     init_stream(items, cu, a, 0);
     init_stream(items, cu, b, 1);
   }
-  __device__ void swap_streams() {
-    const StreamPos t = a;
-    a = b;
-    b = t;
-  }
-  // makes `a` the stream of the next step; false when both streams are done
-  __device__ bool pick() {
-    if (!a.live) swap_streams();
-    return a.live;
-  }
-  // advances `a` by one step, then hands the turn to the other stream
-  __device__ void advance(const int2* items, const int32_t* cu) {
-    ++a.n;
-    if (++a.kb > a.u.b) {
-      ++a.uc;
-      a.kb = 0;
-      a.live = a.nxt_live;
-      a.u = a.nxt;
-      if (a.live) fetch_next(items, cu, a);
+  // advances stream `sp` by one step
+  __device__ void step(const int2* items, const int32_t* cu, StreamPos& sp) {
+    ++sp.n;
+    if (++sp.kb > sp.u.b) {
+      ++sp.uc;
+      sp.kb = 0;
+      sp.q_sent = false;
+      sp.live = sp.nxt_live;
+      sp.u = sp.nxt;
+      if (sp.live) fetch_next(items, cu, sp);
     }
-    if (b.live) swap_streams();
   }
 };
 
@@ -171,15 +166,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                      // [stream]
-  uint8_t* sKV = smem + 2 * ATT_TILE_BYTES;                // [stage]: K then V
-  uint8_t* sP = sKV + 2 * ATT_KV_STAGES * ATT_TILE_BYTES;  // [stream]: two 64-key column blocks each
+  uint8_t* sQ = smem;                                          // [stream]
+  uint8_t* sKV = smem + 2 * ATT_TILE_BYTES;                    // [stream][stage]: K then V
+  uint8_t* sP = sKV + 2 * 2 * ATT_KV_STAGES * ATT_TILE_BYTES;  // [stream]: two 64-key column blocks each
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);
   uint64_t* q_full = bars;          // [stream]
   uint64_t* q_empty = bars + 2;     // [stream]
-  uint64_t* kv_full = bars + 4;                   // [stage]
-  uint64_t* kv_empty = kv_full + ATT_KV_STAGES;   // [stage]
-  uint64_t* s_full = kv_empty + ATT_KV_STAGES;    // [stream]
+  uint64_t* kv_full = bars + 4;                       // [stream][stage]
+  uint64_t* kv_empty = kv_full + 2 * ATT_KV_STAGES;   // [stream][stage]
+  uint64_t* s_full = kv_empty + 2 * ATT_KV_STAGES;    // [stream]
   uint64_t* s_empty = s_full + 2;                 // [stream]
   uint64_t* p_full = s_full + 4;                  // [stream]
   uint64_t* pv_done = s_full + 6;                 // [stream]
@@ -198,7 +193,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&pv_done[i], 1);
       mbar_init(&pv_empty[i], 128);
     }
-    for (int i = 0; i < ATT_KV_STAGES; ++i) {
+    for (int i = 0; i < 2 * ATT_KV_STAGES; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
@@ -220,75 +215,85 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383
 
+  // The producer and the MMA issuer serve the two streams independently:
+  // each polls both streams (non-blocking barrier tests) and advances
+  // whichever is ready, so neither stream waits for the other's softmax.
+  // They give up (PTL_ERR_TIMEOUT) after a second without progress.
   if (warp == 0) {
     if (lane == 0) {
-      AttnStepGen gen;
+      AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
       gen.init(items, cu, nunits);
-      int step = 0;
-      bool ok = true;
-      while (ok && gen.pick()) {
-        const int g = gen.a.g;
-        const AttnUnit a = gen.a.u;
-        if (gen.a.kb == 0) {  // a new unit of stream g: its Q tile
-          if (!mbar_wait(&q_empty[g], (gen.a.uc & 1) ^ 1)) { ok = false; break; }
+      auto produce = [&](StreamPos& sp) -> bool {
+        const int g = sp.g;
+        const AttnUnit a = sp.u;
+        if (sp.kb == 0 && !sp.q_sent) {  // a new unit of stream g: its Q tile
+          if (!mbar_try_wait(&q_empty[g], (sp.uc & 1) ^ 1)) return false;
           mbar_arrive_expect_tx(&q_full[g], ATT_TILE_BYTES);
           tma_load_2d(sQ + g * ATT_TILE_BYTES, &tm_qkv, &q_full[g], a.h * DH, a.s0 + a.b * ATT_BLK);
+          sp.q_sent = true;
         }
-        const int st = step % ATT_KV_STAGES;
-        if (!mbar_wait(&kv_empty[st], ((step / ATT_KV_STAGES) & 1) ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&kv_full[st], 2 * ATT_TILE_BYTES);
-        uint8_t* kbuf = sKV + (2 * st) * ATT_TILE_BYTES;
-        const int row = a.s0 + gen.a.kb * ATT_BLK;
-        tma_load_2d(kbuf, &tm_qkv, &kv_full[st], D + a.h * DH, row);
-        tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, &kv_full[st], 2 * D + a.h * DH, row);
-        ++step;
-        gen.advance(items, cu);
+        const int st = sp.n % ATT_KV_STAGES, use = sp.n / ATT_KV_STAGES;
+        uint64_t* ke = &kv_empty[g * ATT_KV_STAGES + st];
+        uint64_t* kf = &kv_full[g * ATT_KV_STAGES + st];
+        if (!mbar_try_wait(ke, (use & 1) ^ 1)) return false;
+        mbar_arrive_expect_tx(kf, 2 * ATT_TILE_BYTES);
+        uint8_t* kbuf = sKV + (2 * (g * ATT_KV_STAGES + st)) * ATT_TILE_BYTES;
+        const int row = a.s0 + sp.kb * ATT_BLK;
+        tma_load_2d(kbuf, &tm_qkv, kf, D + a.h * DH, row);
+        tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, kf, 2 * D + a.h * DH, row);
+        gen.step(items, cu, sp);
+        return true;
+      };
+      uint64_t t_prog = globaltimer_ns();
+      while (gen.a.live || gen.b.live) {
+        bool prog = false;
+        if (gen.a.live) prog |= produce(gen.a);
+        if (gen.b.live) prog |= produce(gen.b);
+        if (prog) {
+          t_prog = globaltimer_ns();
+        } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
+          set_error(err, PTL_ERR_TIMEOUT);
+          break;
+        }
       }
-      if (!ok) set_error(err, PTL_ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      AttnStepGen gen;
+      AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
       gen.init(items, cu, nunits);
-      int step = 0;
-      bool ok = true;
       // O[g] += P V for the stream's deferred step; a unit's first PV
       // overwrites O, once warpgroup g has read the previous unit's O
       auto issue_pv = [&](StreamPos& sp) -> bool {
         const int nn = sp.pv_n;
-        if (nn < 0) return true;
         const int gs = sp.g;
-        if (!mbar_wait(&p_full[gs], nn & 1)) return false;
-        if (sp.pv_first && !mbar_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
+        if (!mbar_try_wait(&p_full[gs], nn & 1)) return false;
+        if (sp.pv_first && !mbar_try_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
         tc_fence_after();
         const uint32_t p0 = smem_u32(sP + gs * 2 * ATT_TILE_BYTES);
-        const uint32_t v0 = smem_u32(sKV + (2 * sp.pv_st + 1) * ATT_TILE_BYTES);
+        const uint32_t v0 = smem_u32(sKV + (2 * (gs * ATT_KV_STAGES + sp.pv_st) + 1) * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256 + 64 * gs;
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
         for (int k = 0; k < sp.pv_k16 / 16; ++k)
           umma_bf16_ss(d, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
                        umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !sp.pv_first);
         umma_commit(&pv_done[gs]);
-        umma_commit(&kv_empty[sp.pv_st]);
+        umma_commit(&kv_empty[gs * ATT_KV_STAGES + sp.pv_st]);
         sp.pv_n = -1;
         return true;
       };
-      while (ok && gen.pick()) {
-        StreamPos& sp = gen.a;
+      // S = Q K^T for the stream's next step (its previous PV already issued)
+      auto issue_s = [&](StreamPos& sp) -> bool {
         const int g = sp.g;
         const AttnUnit a = sp.u;
-        const int kb = sp.kb;
-        const int nn = sp.n;
-        if (kb == 0 && !mbar_wait(&q_full[g], sp.uc & 1)) { ok = false; break; }
-        const int st = step % ATT_KV_STAGES;
-        if (!mbar_wait(&kv_full[st], (step / ATT_KV_STAGES) & 1) || !mbar_wait(&s_empty[g], (nn & 1) ^ 1)) {
-          ok = false;
-          break;
-        }
+        const int kb = sp.kb, nn = sp.n;
+        const int st = nn % ATT_KV_STAGES, use = nn / ATT_KV_STAGES;
+        if (kb == 0 && !mbar_try_wait(&q_full[g], sp.uc & 1)) return false;
+        if (!mbar_try_wait(&kv_full[g * ATT_KV_STAGES + st], use & 1)) return false;
+        if (!mbar_try_wait(&s_empty[g], (nn & 1) ^ 1)) return false;
         tc_fence_after();
         const int k16 = keys16(a.L, kb);
         const uint32_t q0 = smem_u32(sQ + g * ATT_TILE_BYTES);
-        const uint32_t k0 = smem_u32(sKV + (2 * st) * ATT_TILE_BYTES);
+        const uint32_t k0 = smem_u32(sKV + (2 * (g * ATT_KV_STAGES + st)) * ATT_TILE_BYTES);
         const uint32_t idesc_qk = umma_idesc_bf16(128, k16);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -296,20 +301,31 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                        idesc_qk, k != 0);
         umma_commit(&s_full[g]);
         if (kb == a.b) umma_commit(&q_empty[g]);
-        if (!issue_pv(sp)) { ok = false; break; }
         sp.pv_n = nn;
         sp.pv_st = st;
         sp.pv_k16 = k16;
         sp.pv_first = kb == 0;
         sp.pv_uc = sp.uc;
-        ++step;
-        // a stream with no further steps must not hold its K/V ring stage
-        const bool last = sp.kb == a.b && !sp.nxt_live;
-        if (last && !issue_pv(sp)) { ok = false; break; }
-        gen.advance(items, cu);
+        gen.step(items, cu, sp);
+        return true;
+      };
+      auto serve = [&](StreamPos& sp) -> bool {
+        bool prog = false;
+        if (sp.pv_n >= 0 && issue_pv(sp)) prog = true;
+        if (sp.pv_n < 0 && sp.live && issue_s(sp)) prog = true;
+        return prog;
+      };
+      uint64_t t_prog = globaltimer_ns();
+      while (gen.a.live || gen.a.pv_n >= 0 || gen.b.live || gen.b.pv_n >= 0) {
+        bool prog = serve(gen.a);
+        prog |= serve(gen.b);
+        if (prog) {
+          t_prog = globaltimer_ns();
+        } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
+          set_error(err, PTL_ERR_TIMEOUT);
+          break;
+        }
       }
-      if (ok) ok = issue_pv(gen.a) && issue_pv(gen.b);
-      if (!ok) set_error(err, PTL_ERR_TIMEOUT);
     }
   } else {
     // softmax warpgroup g (warps 2..5 -> 0, 6..9 -> 1); thread r <-> query row r

@@ -20,6 +20,7 @@ constexpr int QKV_N = 3 * D;       // 1536
 constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
 constexpr int MOE_BM = 256;        // rows per expert tile (padding granule; one CTA pair's M)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
+constexpr int GR_TOK = 16;         // tokens per block of the fused gate + route kernel
 constexpr int GEMM2_BN = 256;      // expert GEMM2 output columns per tile
 constexpr float LN_EPS = 1e-5f;
 constexpr float LOGIT_CLAMP = 15.0f;
@@ -41,21 +42,26 @@ struct WsLayout {
   size_t idx;         // int32 [T][2]
   size_t wgt;         // f32 [T][2]
   size_t chunk_cnt;   // int32 [n_chunks][8]
+  size_t lb;          // int32 [32 + 32 * n_gchunks]  fused gate + route: ticket, per-chunk look-back state
   size_t perm;        // int32 [2T]
   size_t pos;         // int32 [2T]          route -> padded expert row
-  size_t rowroute;    // int32 [2T + 8*128]   padded expert rows -> route (or -1)
+  size_t rowroute;    // int32 [padded_rows]   padded expert rows -> route (or -1)
   size_t tiles;       // int2 [max_tiles]     (expert, first padded row)
-  size_t route_meta;  // int32 [32]: [0] n_tiles, [1..9] off, [10..18] padded off
+  size_t route_meta;  // int32 [32]: [0] n_tiles, [1..9] off, [10..18] first row of each expert
   size_t xperm;       // bf16 build: [padded_rows][512] LayerNorm2 rows in expert (padded) order
   size_t hbuf;        // dt [padded_rows][1024]  expert hidden rows (padded layout)
   size_t ybuf;        // per-route expert outputs awaiting the combine: bf16 build
-                      // [2T + 8*128][512] bf16 in padded row order, fp32 build
+                      // [padded_rows][512] bf16 in padded row order, fp32 build
                       // [2T][512] f32 in route order
   size_t head_p;      // f32 [T]            head probabilities before compaction
+  size_t wl_end;      // end of the error word + work list (the no-alloc scratch holds these)
+  size_t clear_end;   // end of the routing state that each call starts from zero
   size_t total;
   int64_t T;
   int32_t U;
   int64_t max_items, max_levels, n_chunks, max_tiles, padded_rows;
+  int64_t n_gchunks;  // fused gate + route chunks (GR_TOK tokens each)
+  int64_t cap;        // fused path: expert e's rows start at e * cap (T rounded up to MOE_BM)
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -71,7 +77,11 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->max_levels = (T + ATT_BLK - 1) / ATT_BLK + 1;
   L->n_chunks = (2 * T + ROUTE_CHUNK - 1) / ROUTE_CHUNK + 1;
   L->max_tiles = (2 * T + MOE_BM - 1) / MOE_BM + E + 1;
+  L->n_gchunks = (T + GR_TOK - 1) / GR_TOK + 1;
+  L->cap = (T + MOE_BM - 1) / MOE_BM * MOE_BM;
+  // expert rows: compact-padded (route builder) or at fixed e * cap (fused path)
   L->padded_rows = 2 * T + E * MOE_BM;
+  if (E * L->cap > L->padded_rows) L->padded_rows = E * L->cap;
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t at = o;
@@ -79,12 +89,15 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
     return at;
   };
   L->err = take(256);
-  L->chunk_cnt = take(4 * L->n_chunks * E);  // right after the error word: cleared together
   L->items = take(sizeof(int2) * L->max_items);
   L->item_count = take(4);
   L->lvl_hist = take(4 * (L->max_levels + 1));
   L->lvl_start = take(4 * (L->max_levels + 1));
   L->lvl_fill = take(4 * (L->max_levels + 1));
+  L->wl_end = o;  // error word + attention work list
+  L->chunk_cnt = take(4 * L->n_chunks * E);
+  L->lb = take(4 * (32 + 32 * L->n_gchunks));
+  L->clear_end = o;  // [0, clear_end) is cleared by one memset per call
   L->xn = take(es * T * D);
   L->qkv = take(es * T * QKV_N);
   L->attn = take(es * T * D);

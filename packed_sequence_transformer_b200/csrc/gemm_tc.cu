@@ -58,7 +58,7 @@ struct GemmTcParams {
   int ldo;                       // output row stride (elements)
   const int2* tiles;             // (expert, first padded row) per 256-row M tile
   const int32_t* meta;           // [0] = number of M tiles
-  int32_t* zero_ptr;             // cleared by CTA 0 once the predecessor is done (may be NULL)
+  int32_t* zero_ptr;             // cleared by the grid once the predecessor is done (may be NULL)
   int zero_n;
   int32_t* err;
 };
@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(192, 1)
     int nt = MODE >= G_MOE1 ? p.meta[0] * (p.N_total / BN) : p.n_tiles_dense;
     s_ntiles = has_error(p.err) ? 0 : nt;
   }
-  if (p.zero_ptr && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < p.zero_n; i += blockDim.x) p.zero_ptr[i] = 0;
+  if (p.zero_ptr)
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_n; i += gridDim.x * blockDim.x)
+      p.zero_ptr[i] = 0;
   __syncthreads();
   const int ntiles = s_ntiles;
   const uint32_t tmem = *tmem_slot;
@@ -413,10 +414,11 @@ int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUte
   p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
-  // the route builder (the previous kernel) has consumed the per-chunk expert
-  // counts: clear them for the next gate
+  // the routing state of this layer (per-chunk expert counts, look-back
+  // state, contiguous in the workspace) is consumed: clear it for the next
+  // layer's gate
   p.zero_ptr = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
-  p.zero_n = int(L.n_chunks * E);
+  p.zero_n = int((L.clear_end - L.chunk_cnt) / 4);
   return launch_pair<MOE1_BN, G_MOE1>(xperm, w1, hbuf_out, p, int(L.max_tiles) * (F / MOE1_BN), st);
 }
 

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "sm100.cuh"
 
 namespace ptl {
 
@@ -252,16 +253,77 @@ __device__ __forceinline__ void store_row16_groups(float* row, int lane, const f
   Row16<float>::store(row, lane, v);
 }
 
+// The gate for one token, by one warp: LayerNorm2 of the x1 row into v (the
+// lane's 16 values in the fp32 lane layout: 4 groups of 4 consecutive columns
+// at q*128 + lane*4), the 8 logits in fp32 against the staged gate weights,
+// softmax, top-2 (ties to the lower index) and the renormalised weights.
+// Every lane returns the same e0, e1, w0, w1.
+__device__ __forceinline__ void gate_token(const float* __restrict__ x1_row, const float* __restrict__ g,
+                                           const float* __restrict__ b, const float* __restrict__ s_wg,
+                                           const float* __restrict__ bg, int lane, float (&v)[16], int& e0,
+                                           int& e1, float& w0, float& w1) {
+  Row16<float>::load(x1_row, lane, v);
+  layer_norm16<float>(v, g, b, lane);
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 w4 = *reinterpret_cast<const float4*>(s_wg + e * D + q * 128 + lane * 4);
+      s += v[4 * q] * w4.x + v[4 * q + 1] * w4.y + v[4 * q + 2] * w4.z + v[4 * q + 3] * w4.w;
+    }
+    acc[e] = s;
+  }
+  float mine = warp_reduce_scatter8(acc, lane) + (bg ? __ldg(bg + (lane >> 2)) : 0.f);
+  float lg[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) lg[e] = __shfl_sync(0xffffffffu, mine, 4 * e);
+  // every lane evaluates the same (tiny) softmax / top-2
+  float m = lg[0];
+#pragma unroll
+  for (int e = 1; e < E; ++e) m = fmaxf(m, lg[e]);
+  float p[E], sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    p[e] = expf(lg[e] - m);
+    sum += p[e];
+  }
+  e0 = -1;
+  e1 = -1;
+  float p0 = -1.f, p1 = -1.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float pe = p[e] / sum;
+    if (pe > p0) {
+      e1 = e0;
+      p1 = p0;
+      e0 = e;
+      p0 = pe;
+    } else if (pe > p1) {
+      e1 = e;
+      p1 = pe;
+    }
+  }
+  const float den = p0 + p1;
+  w0 = p0 / den;
+  w1 = p1 / den;
+}
+
+// Stages the gate weights [8][512] in shared memory; lane l later reads
+// columns q*128 + 4l..4l+3, i.e. consecutive 16-byte words across the warp.
+__device__ __forceinline__ void stage_gate_weights(float* s_wg, const float* __restrict__ wg) {
+  for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
     const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
     const float* __restrict__ wg, const float* __restrict__ bg, T* __restrict__ xn2,
     int32_t* __restrict__ idx, float* __restrict__ wout, int32_t* __restrict__ chunk_cnt, int T_) {
-  // gate weights [8][512] in shared memory; lane l reads columns q*128 + 4l..4l+3,
-  // i.e. consecutive 16-byte words across the warp (no bank conflicts)
   __shared__ __align__(16) float s_wg[E * D];
-  for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
-    reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
+  stage_gate_weights(s_wg, wg);
   __syncthreads();
   pdl_wait();  // x1 comes from the previous kernel
   pdl_trigger();  // dependents launch once this grid has passed its own wait
@@ -269,56 +331,187 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
   const int warp = threadIdx.x >> 5;
   for (int t = blockIdx.x * GATE_WARPS + warp; t < T_; t += gridDim.x * GATE_WARPS) {
     float v[16];
-    Row16<float>::load(x1 + size_t(t) * D, lane, v);
-    layer_norm16<float>(v, g, b, lane);
+    int e0, e1;
+    float w0, w1;
+    gate_token(x1 + size_t(t) * D, g, b, s_wg, bg, lane, v, e0, e1, w0, w1);
     store_row16_groups(xn2 + size_t(t) * D, lane, v);
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 w4 = *reinterpret_cast<const float4*>(s_wg + e * D + q * 128 + lane * 4);
-        s += v[4 * q] * w4.x + v[4 * q + 1] * w4.y + v[4 * q + 2] * w4.z + v[4 * q + 3] * w4.w;
-      }
-      acc[e] = s;
-    }
-    float mine = warp_reduce_scatter8(acc, lane) + (bg ? __ldg(bg + (lane >> 2)) : 0.f);
-    float lg[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) lg[e] = __shfl_sync(0xffffffffu, mine, 4 * e);
     if (lane == 0) {
-      float m = lg[0];
-#pragma unroll
-      for (int e = 1; e < E; ++e) m = fmaxf(m, lg[e]);
-      float p[E], sum = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        p[e] = expf(lg[e] - m);
-        sum += p[e];
-      }
-      int e0 = -1, e1 = -1;
-      float p0 = -1.f, p1 = -1.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float pe = p[e] / sum;
-        if (pe > p0) {
-          e1 = e0;
-          p1 = p0;
-          e0 = e;
-          p0 = pe;
-        } else if (pe > p1) {
-          e1 = e;
-          p1 = pe;
-        }
-      }
-      const float den = p0 + p1;
       *reinterpret_cast<int2*>(idx + 2 * t) = make_int2(e0, e1);
-      *reinterpret_cast<float2*>(wout + 2 * t) = make_float2(p0 / den, p1 / den);
+      *reinterpret_cast<float2*>(wout + 2 * t) = make_float2(w0, w1);
       atomicAdd(&chunk_cnt[(t >> 7) * E + e0], 1);
       atomicAdd(&chunk_cnt[(t >> 7) * E + e1], 1);
     }
   }
+}
+
+// ------------------------------------------------------- gate + route
+// The layer path's gate and route builder in one kernel (bf16 build).  A
+// block takes the next chunk of GR_TOK tokens (a ticket, so chunks start in
+// order), runs the gate for one token per warp, ranks the chunk's 2*GR_TOK
+// routes per expert (stable: ascending route id r = 2t + k), publishes the
+// chunk's counts (flag 1) and sums the published counts of every earlier
+// chunk (one thread per earlier chunk, in parallel; an earlier chunk's block
+// took its ticket first, so it is running and will publish).  Expert e's rows start at e * cap (cap = T
+// rounded up to 256 >= any expert's route count), so a route's row
+// e * cap + (routes of e before it) needs no global totals: each warp writes
+// pos[r] and stores its token's LayerNorm2 row (bf16) straight into both of
+// its rows of xperm.  The last chunk also writes the expert tile list and
+// the offsets.  Waits on predecessors are bounded (PTL_ERR_TIMEOUT).
+// lb: [0] ticket, then per chunk 32 ints: [0] flag, [4..11] counts; all
+// zero before the kernel.
+__global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
+    const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
+    const float* __restrict__ wg, const float* __restrict__ bg, int32_t* __restrict__ idx,
+    float* __restrict__ wout, int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ xperm, int cap,
+    int32_t* __restrict__ lb, int2* __restrict__ tiles, int32_t* __restrict__ meta, int T_,
+    int32_t* err) {
+  __shared__ __align__(16) float s_wg[E * D];
+  __shared__ int s_chunk, s_e[2 * GR_TOK], s_rank[2 * GR_TOK], s_cnt[E], s_excl[E], s_tot[E];
+  __shared__ int s_red[GR_TOK][E];
+  stage_gate_weights(s_wg, wg);
+  __syncthreads();
+  pdl_wait();  // x1 comes from the previous kernel
+  pdl_trigger();  // dependents launch once this grid has passed its own wait
+  if (has_error(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) s_chunk = atomicAdd(lb, 1);
+  __syncthreads();
+  const int c = s_chunk;
+  const int nchunks = (T_ + GR_TOK - 1) / GR_TOK;
+  const int t = c * GR_TOK + warp;
+  const bool valid = t < T_;
+  float v[16];
+  int e0 = E, e1 = E;
+  float w0 = 0.f, w1 = 0.f;
+  if (valid) {
+    gate_token(x1 + size_t(t) * D, g, b, s_wg, bg, lane, v, e0, e1, w0, w1);
+    if (lane == 0) {
+      *reinterpret_cast<int2*>(idx + 2 * t) = make_int2(e0, e1);
+      *reinterpret_cast<float2*>(wout + 2 * t) = make_float2(w0, w1);
+    }
+  }
+  if (lane == 0) {
+    s_e[2 * warp] = e0;
+    s_e[2 * warp + 1] = e1;
+  }
+  __syncthreads();
+  // chunk-local stable ranks and counts (the chunk's 2 * GR_TOK = 32 routes
+  // are one warp's lanes)
+  static_assert(2 * GR_TOK == 32, "one lane per route of the chunk");
+  if (warp == 0) {
+    const int e = s_e[lane];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    s_rank[lane] = __popc(same & ((1u << lane) - 1u));
+#pragma unroll
+    for (int x = 0; x < E; ++x) {
+      const unsigned bal = __ballot_sync(0xffffffffu, e == x);
+      if (lane == x) s_cnt[x] = __popc(bal);
+    }
+  }
+  __syncthreads();
+  // publish this chunk's counts, then sum the counts of every earlier chunk
+  // (one thread per earlier chunk, all read in parallel: no chain of
+  // prefixes to wait for)
+  int32_t* me = lb + 32 + 32 * c;
+  if (threadIdx.x < E) me[4 + threadIdx.x] = s_cnt[threadIdx.x];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    *reinterpret_cast<volatile int32_t*>(me) = 1;
+  }
+  int part[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) part[e] = 0;
+  for (int pc = threadIdx.x; pc < c; pc += blockDim.x) {
+    const volatile int32_t* pf = lb + 32 + 32 * pc;
+    int f = *pf;
+    if (f == 0) {
+      const uint64_t t0 = sm100::globaltimer_ns();
+      while ((f = *pf) == 0) {
+        if (sm100::globaltimer_ns() - t0 > sm100::kWaitLimitNs) break;
+      }
+    }
+    if (f == 0) {
+      set_error(err, PTL_ERR_TIMEOUT);
+      break;
+    }
+    __threadfence();
+    const int4* src = reinterpret_cast<const int4*>(lb + 32 + 32 * pc + 4);
+    const int4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
+    part[0] += v0.x;
+    part[1] += v0.y;
+    part[2] += v0.z;
+    part[3] += v0.w;
+    part[4] += v1.x;
+    part[5] += v1.y;
+    part[6] += v1.z;
+    part[7] += v1.w;
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int w = __reduce_add_sync(0xffffffffu, part[e]);
+    if (lane == 0) s_red[warp][e] = w;
+  }
+  __syncthreads();
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    int excl = 0;
+#pragma unroll
+    for (int w = 0; w < GR_TOK; ++w) excl += s_red[w][e];
+    s_excl[e] = excl;
+    s_tot[e] = excl + s_cnt[e];
+  }
+  __syncthreads();
+  if (valid) {
+    // this token's two routes: rows e * cap + (routes of e before it)
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = k == 0 ? e0 : e1;
+      const int row = e * cap + s_excl[e] + s_rank[2 * warp + k];
+      if (lane == 0) pos[2 * t + k] = row;
+      store_row16_groups(xperm + size_t(row) * D, lane, v);
+    }
+  }
+  if (c == nchunks - 1) {
+    // the last chunk's inclusive prefix holds every expert's total
+    int nt_before = 0;
+    for (int e = 0; e < E; ++e) {
+      const int nt = (s_tot[e] + MOE_BM - 1) / MOE_BM;
+      for (int j = threadIdx.x; j < nt; j += blockDim.x) tiles[nt_before + j] = make_int2(e, e * cap + j * MOE_BM);
+      nt_before += nt;
+    }
+    if (threadIdx.x == 0) {
+      meta[0] = nt_before;
+      int off = 0;
+      for (int e = 0; e < E; ++e) {
+        meta[1 + e] = off;
+        meta[10 + e] = e * cap;
+        off += s_tot[e];
+      }
+      meta[1 + E] = off;
+      meta[10 + E] = E * cap;
+    }
+  }
+}
+
+// Debug outputs of the fused path: perm (compact, stable) and expert_off from
+// the rows gate_route_kernel assigned.  One thread per route.
+__global__ void __launch_bounds__(256) route_debug_kernel(const int32_t* __restrict__ idx,
+                                                          const int32_t* __restrict__ pos,
+                                                          const int32_t* __restrict__ meta, int cap,
+                                                          int n_routes, int32_t* __restrict__ perm,
+                                                          int32_t* __restrict__ expert_off,
+                                                          const int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
+  if (has_error(err)) return;
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r <= E && blockIdx.x == 0 && expert_off) expert_off[r] = meta[1 + r];
+  if (r >= n_routes || !perm) return;
+  const int e = idx[r];
+  perm[meta[1 + e] + (pos[r] - e * cap)] = r;
 }
 
 // Per-chunk route counts for a caller-supplied topk_idx (standalone route
@@ -803,6 +996,29 @@ int launch_gate(const void* x1, const float* g, const float* b, const float* wg,
                                                            bg, static_cast<float*>(xn2), idx, w,
                                                            chunk_cnt, T)) return -1;
   }
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_gate_route(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
+                      int T, const WsLayout& L, char* ws, cudaStream_t st) {
+  const int blocks = (T + GR_TOK - 1) / GR_TOK;
+  if (launch_k(gate_route_kernel, dim3(blocks), dim3(GR_TOK * 32), 0, st, static_cast<const float*>(x1), g, b,
+               wg, bg, reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<float*>(ws + L.wgt),
+               reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<__nv_bfloat16*>(ws + L.xperm),
+               int(L.cap), reinterpret_cast<int32_t*>(ws + L.lb), reinterpret_cast<int2*>(ws + L.tiles),
+               reinterpret_cast<int32_t*>(ws + L.route_meta), T, reinterpret_cast<int32_t*>(ws + L.err)))
+    return -1;
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_route_debug(int T, const WsLayout& L, const char* ws, int32_t* perm, int32_t* expert_off,
+                       cudaStream_t st) {
+  const int n = 2 * T;
+  if (launch_k(route_debug_kernel, dim3((n + 255) / 256), dim3(256), 0, st,
+               reinterpret_cast<const int32_t*>(ws + L.idx), reinterpret_cast<const int32_t*>(ws + L.pos),
+               reinterpret_cast<const int32_t*>(ws + L.route_meta), int(L.cap), n, perm, expert_off,
+               reinterpret_cast<const int32_t*>(ws + L.err)))
+    return -1;
   return PTL_LAUNCH_CHECK();
 }
 

@@ -41,6 +41,13 @@ int launch_gate(const void* x1, const float* g, const float* b, const float* wg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
                 cudaStream_t st);
 int launch_chunk_hist(const int32_t* idx, int T, int32_t* chunk_cnt, int32_t* err, cudaStream_t st);
+// bf16 layer path: gate + route builder in one kernel (idx, wgt, pos, xperm,
+// tiles, meta in the workspace; the look-back state must be zero)
+int launch_gate_route(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
+                      int T, const WsLayout& L, char* ws, cudaStream_t st);
+// perm / expert_off (either may be NULL) of the fused path
+int launch_route_debug(int T, const WsLayout& L, const char* ws, int32_t* perm, int32_t* expert_off,
+                       cudaStream_t st);
 // xn2 (bf16 build, nullable): also copy each route's LayerNorm2 row to its
 // padded slot of the workspace's xperm
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,

@@ -91,7 +91,7 @@ extern "C" ptl_status ptl_attention_noalloc(const void* qkv, void* attn, const i
     return PTL_ERR_ALIGN;
   WsLayout L;
   if (!make_layout(total_tokens, num_users, dt, &L)) return PTL_ERR_SHAPE;
-  if (L.xn > sizeof(g_noalloc_scratch)) return PTL_ERR_SHAPE;  // work list must fit the array
+  if (L.wl_end > sizeof(g_noalloc_scratch)) return PTL_ERR_SHAPE;  // work list must fit the array
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)

@@ -244,6 +244,23 @@ def test_stack_of_one_equals_layer():
     assert torch.equal(o_layer, o_stack)
 
 
+@pytest.mark.parametrize("dt", ["bf16", "fp32"])
+def test_three_layer_stack_equals_chain_and_oracle(dt):
+    """Every layer of a stack starts from cleared per-layer routing state:
+    the stack equals the chain of single-layer calls bit for bit, and the
+    fp32 build stays within its bar of the fp64 oracle after three layers."""
+    c = S.make_case("s3", lengths=[3, 7, 12, 20, 130, 257, 1], seed=5, dtype=dt, num_layers=3,
+                    gate_std=0.1)
+    out, _, _ = _run_stack(c)
+    chain_out, gidx = _chain_idx(c)
+    assert torch.equal(chain_out, out), "stack differs from the chain of single layers"
+    if dt == "fp32":
+        ch = NearTieChooser(gidx, EXACT_MARGIN)
+        ref = O.stack_forward(c.x, c.cu_seqlens, c.layers, choose=ch)
+        ch.assert_ok()
+        assert_close(host(out), ref, 3 * LAYER_F32[0], LAYER_F32[1], what=c.name)
+
+
 @pytest.mark.parametrize("bad", ["not_monotone", "first_not_zero", "last_not_T"])
 def test_bad_offsets_reported(bad):
     c = S.make_case("bad", lengths=[5, 6, 7], seed=3, dtype="bf16")
