@@ -14,7 +14,8 @@
 //   warp 0      TMA producer: the Q tile [128 x 64] of each stream's current
 //               unit, and per step the K and V tiles [128 x 64] through a
 //               per-stream 2-deep ring, straight from the packed qkv rows
-//               (128-byte swizzle);
+//               (128-byte swizzle); K and V have separate barriers, so the
+//               next K loads as soon as its slot's QK^T is done;
 //   warp 1      MMA issuer: for a step of stream g, S = Q K^T (M=128, N = the
 //               keys of this block rounded up to 16) into TMEM S[g], and --
 //               once warpgroup g has written P for that step -- O[g] += P V
@@ -51,8 +52,8 @@ constexpr int ATT_TILE_BYTES = ATT_BLK * DH * 2;  // 16 KB
 constexpr int ATT_KV_STAGES = 2;
 // Q[2] + (K,V)[2 streams][stages] + P[2][2 column blocks]
 constexpr int ATT_SMEM_TILES = 2 + 2 * 2 * ATT_KV_STAGES + 4;
-constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 256;
-constexpr int ATT_THREADS = 320;  // producer, MMA, two softmax warpgroups
+constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 512;  // + alignment, barriers
+constexpr int ATT_THREADS = 576;  // producer, MMA, four softmax warpgroups (two per stream)
 
 struct AttnUnit {
   int s0, L, b, h;
@@ -112,6 +113,7 @@ struct StreamPos {
   int pv_n, pv_st, pv_k16, pv_uc;  // the step whose PV is still to be issued (-1: none)
   bool pv_first;
   bool q_sent;       // producer: the current unit's Q tile load is issued
+  bool k_sent;       // producer: the current step's K tile load is issued
 };
 
 // Both streams' step sequences as the producer and the MMA issuer walk them
@@ -135,6 +137,7 @@ struct AttnStepGen {
     sp.pv_st = sp.pv_k16 = sp.pv_uc = 0;
     sp.pv_first = false;
     sp.q_sent = false;
+    sp.k_sent = false;
     fetch_next(items, cu, sp);
     sp.live = sp.nxt_live;
     sp.u = sp.nxt;
@@ -172,14 +175,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);
   uint64_t* q_full = bars;          // [stream]
   uint64_t* q_empty = bars + 2;     // [stream]
-  uint64_t* kv_full = bars + 4;                       // [stream][stage]
-  uint64_t* kv_empty = kv_full + 2 * ATT_KV_STAGES;   // [stream][stage]
-  uint64_t* s_full = kv_empty + 2 * ATT_KV_STAGES;    // [stream]
+  // K and V have their own barriers: a K tile is free once its QK^T is done,
+  // long before the step's PV frees the V tile, so the next K load can start
+  // early
+  uint64_t* k_full = bars + 4;                        // [stream][stage]
+  uint64_t* k_empty = k_full + 2 * ATT_KV_STAGES;     // [stream][stage]
+  uint64_t* v_full = k_empty + 2 * ATT_KV_STAGES;     // [stream][stage]
+  uint64_t* v_empty = v_full + 2 * ATT_KV_STAGES;     // [stream][stage]
+  uint64_t* s_full = v_empty + 2 * ATT_KV_STAGES;     // [stream]
   uint64_t* s_empty = s_full + 2;                 // [stream]
   uint64_t* p_full = s_full + 4;                  // [stream]
   uint64_t* pv_done = s_full + 6;                 // [stream]
   uint64_t* pv_empty = s_full + 8;                // [stream]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
+  uint64_t* x_bar = s_full + 10;                  // [stream] the two softmax halves meet
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 12);
   __shared__ int s_units;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,14 +197,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&s_empty[i], 256);
+      mbar_init(&p_full[i], 256);
       mbar_init(&pv_done[i], 1);
-      mbar_init(&pv_empty[i], 128);
+      mbar_init(&pv_empty[i], 256);
+      mbar_init(&x_bar[i], 256);
     }
     for (int i = 0; i < 2 * ATT_KV_STAGES; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
@@ -213,7 +225,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   const int nunits = s_units;
   const uint32_t tmem = *tmem_slot;
-  // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383
+  // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383,
+  // softmax exchange 384..399
 
   // The producer and the MMA issuer serve the two streams independently:
   // each polls both streams (non-blocking barrier tests) and advances
@@ -233,14 +246,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           sp.q_sent = true;
         }
         const int st = sp.n % ATT_KV_STAGES, use = sp.n / ATT_KV_STAGES;
-        uint64_t* ke = &kv_empty[g * ATT_KV_STAGES + st];
-        uint64_t* kf = &kv_full[g * ATT_KV_STAGES + st];
-        if (!mbar_try_wait(ke, (use & 1) ^ 1)) return false;
-        mbar_arrive_expect_tx(kf, 2 * ATT_TILE_BYTES);
-        uint8_t* kbuf = sKV + (2 * (g * ATT_KV_STAGES + st)) * ATT_TILE_BYTES;
+        const int slot = g * ATT_KV_STAGES + st;
+        uint8_t* kbuf = sKV + (2 * slot) * ATT_TILE_BYTES;
         const int row = a.s0 + sp.kb * ATT_BLK;
-        tma_load_2d(kbuf, &tm_qkv, kf, D + a.h * DH, row);
-        tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, kf, 2 * D + a.h * DH, row);
+        if (!sp.k_sent) {  // the step's K tile, once the slot's previous QK^T is done
+          if (!mbar_try_wait(&k_empty[slot], (use & 1) ^ 1)) return false;
+          mbar_arrive_expect_tx(&k_full[slot], ATT_TILE_BYTES);
+          tma_load_2d(kbuf, &tm_qkv, &k_full[slot], D + a.h * DH, row);
+          sp.k_sent = true;
+        }
+        // its V tile, once the slot's previous PV is done
+        if (!mbar_try_wait(&v_empty[slot], (use & 1) ^ 1)) return false;
+        mbar_arrive_expect_tx(&v_full[slot], ATT_TILE_BYTES);
+        tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, &v_full[slot], 2 * D + a.h * DH, row);
+        sp.k_sent = false;
         gen.step(items, cu, sp);
         return true;
       };
@@ -268,6 +287,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int gs = sp.g;
         if (!mbar_try_wait(&p_full[gs], nn & 1)) return false;
         if (sp.pv_first && !mbar_try_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
+        if (!mbar_try_wait(&v_full[gs * ATT_KV_STAGES + sp.pv_st], (nn / ATT_KV_STAGES) & 1)) return false;
         tc_fence_after();
         const uint32_t p0 = smem_u32(sP + gs * 2 * ATT_TILE_BYTES);
         const uint32_t v0 = smem_u32(sKV + (2 * (gs * ATT_KV_STAGES + sp.pv_st) + 1) * ATT_TILE_BYTES);
@@ -277,7 +297,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           umma_bf16_ss(d, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
                        umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !sp.pv_first);
         umma_commit(&pv_done[gs]);
-        umma_commit(&kv_empty[gs * ATT_KV_STAGES + sp.pv_st]);
+        umma_commit(&v_empty[gs * ATT_KV_STAGES + sp.pv_st]);
         sp.pv_n = -1;
         return true;
       };
@@ -288,7 +308,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int kb = sp.kb, nn = sp.n;
         const int st = nn % ATT_KV_STAGES, use = nn / ATT_KV_STAGES;
         if (kb == 0 && !mbar_try_wait(&q_full[g], sp.uc & 1)) return false;
-        if (!mbar_try_wait(&kv_full[g * ATT_KV_STAGES + st], use & 1)) return false;
+        if (!mbar_try_wait(&k_full[g * ATT_KV_STAGES + st], use & 1)) return false;
         if (!mbar_try_wait(&s_empty[g], (nn & 1) ^ 1)) return false;
         tc_fence_after();
         const int k16 = keys16(a.L, kb);
@@ -300,6 +320,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           umma_bf16_ss(tmem + 128 * g, umma_desc_sw128(q0 + 32 * k, 1024), umma_desc_sw128(k0 + 32 * k, 1024),
                        idesc_qk, k != 0);
         umma_commit(&s_full[g]);
+        umma_commit(&k_empty[g * ATT_KV_STAGES + st]);
         if (kb == a.b) umma_commit(&q_empty[g]);
         sp.pv_n = nn;
         sp.pv_st = st;
@@ -328,19 +349,27 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
     }
   } else {
-    // softmax warpgroup g (warps 2..5 -> 0, 6..9 -> 1); thread r <-> query row r
-    // of the unit <-> TMEM lane r
-    const int g = (warp - 2) >> 2;
+    // Softmax: four warpgroups, two per stream.  Warpgroup (g, h) (warps
+    // 2 + 8g + 4h .. +3) handles keys 64h .. 64h + 63 of every S row of stream
+    // g, column block h of P and columns 32h .. 32h + 31 of O; thread r <->
+    // query row r <-> TMEM lane r.  The two halves of a row combine their
+    // maxima (every step) and their sums (at a unit's end) through spare TMEM
+    // columns, synchronised by a per-stream mbarrier (bounded waits).
+    const int sw = (warp - 2) >> 2;
+    const int g = sw >> 1, h = sw & 1;
     const int wq = warp & 3;
     const int r = 32 * wq + lane;
     const uint32_t lane_off = uint32_t(32 * wq) << 16;
-    const uint32_t tS = tmem + 128 * g + lane_off;
-    const uint32_t tPV = tmem + 256 + 64 * g + lane_off;
+    const uint32_t tS = tmem + 128 * g + 64 * h + lane_off;       // this half's 64 S columns
+    const uint32_t tO = tmem + 256 + 64 * g + 32 * h + lane_off;  // this half's 32 O columns
+    const uint32_t tX = tmem + 384 + 8 * g + lane_off;            // exchange: [half][parity][max, l]
+    auto xcol = [](int hh, int par, int what) { return uint32_t(4 * hh + 2 * par + what); };
     const float c2 = 0.125f * 1.4426950408889634f;  // softmax scale * log2(e)
-    // Running max m (base 2, scale folded in) and sum l of this row.  O lives
-    // in TMEM and the PV products accumulate into it; m is raised (and O, l
-    // rescaled) only when a block's max exceeds it by more than RESCALE_LOG2,
-    // so P = exp2(s - m) stays below 2^RESCALE_LOG2 and O / l is unchanged.
+    // Running max m (base 2, scale folded in) of the row and this half's sum l.
+    // O lives in TMEM and the PV products accumulate into it; m is raised (and
+    // O, l rescaled) only when a block's max exceeds it by more than
+    // RESCALE_LOG2, so P = exp2(s - m) stays below 2^RESCALE_LOG2 and O / l is
+    // unchanged.  Both halves see the same maxima, so they keep the same m.
     constexpr float RESCALE_LOG2 = 8.f;
     float m = 0.f, l = 0.f;
     // the previous step of this stream: its PV may still be running
@@ -348,32 +377,37 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     bool plast = false;
     float pl = 1.f;
     int pdst = -1;  // output row offset (elements) of this thread for the previous step's unit, or -1
+    int nx = 0;     // exchanges of this stream so far
     bool ok = true;
-    // waits for the previous step's PV; at a unit's end, stores O / l and
-    // releases O for the next unit's first PV
-    auto finish_prev = [&]() -> bool {
+    // both halves of the stream meet (every thread arrives, then waits)
+    auto meet = [&]() -> bool {
+      tc_fence_before();
+      mbar_arrive(&x_bar[g]);
+      const bool met = mbar_wait(&x_bar[g], nx & 1);
+      ++nx;
+      tc_fence_after();
+      return met;
+    };
+    // waits for the previous step's PV; at a unit's end, stores this half's
+    // columns of O / l and releases O for the next unit's first PV
+    auto finish_prev = [&](float l_row) -> bool {
       if (!mbar_wait(&pv_done[g], pn & 1)) return false;
       tc_fence_after();
       if (plast) {
-        const float inv = 1.0f / pl;
-        uint32_t oraw[2][32];
-        tmem_ld32(tPV, oraw[0]);
-        tmem_ld32(tPV + 32, oraw[1]);
+        const float inv = 1.0f / l_row;
+        uint32_t raw[32];
+        tmem_ld32(tO, raw);
         tmem_ld_wait();
+        if (pdst >= 0) {
+          uint4* dst = reinterpret_cast<uint4*>(out + pdst + 32 * h);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t (&raw)[32] = oraw[c];
-          if (pdst >= 0) {
-            uint4* dst = reinterpret_cast<uint4*>(out + pdst + 32 * c);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(raw[8 * q + 0]) * inv, __uint_as_float(raw[8 * q + 1]) * inv);
-              u.y = pack_bf16x2(__uint_as_float(raw[8 * q + 2]) * inv, __uint_as_float(raw[8 * q + 3]) * inv);
-              u.z = pack_bf16x2(__uint_as_float(raw[8 * q + 4]) * inv, __uint_as_float(raw[8 * q + 5]) * inv);
-              u.w = pack_bf16x2(__uint_as_float(raw[8 * q + 6]) * inv, __uint_as_float(raw[8 * q + 7]) * inv);
-              dst[q] = u;
-            }
+          for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(raw[8 * q + 0]) * inv, __uint_as_float(raw[8 * q + 1]) * inv);
+            u.y = pack_bf16x2(__uint_as_float(raw[8 * q + 2]) * inv, __uint_as_float(raw[8 * q + 3]) * inv);
+            u.z = pack_bf16x2(__uint_as_float(raw[8 * q + 4]) * inv, __uint_as_float(raw[8 * q + 5]) * inv);
+            u.w = pack_bf16x2(__uint_as_float(raw[8 * q + 6]) * inv, __uint_as_float(raw[8 * q + 7]) * inv);
+            dst[q] = u;
           }
         }
         tc_fence_before();
@@ -398,97 +432,97 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int kbase = kb * ATT_BLK;
         // 32-key chunks this warp needs: those inside the block's key count,
         // and on the diagonal block only chunks not wholly above the warp's
-        // rows; loads take 64 columns, the keys past qlim are masked
+        // rows; this half owns chunks 2h and 2h + 1 (keys past qlim masked)
         const int nch = (k16 + 31) >> 5;
         const int nuse = (kb == a.b) ? min(nch, wq + 1) : nch;
-        // pass 1: the row maximum over the visible keys (four independent chains)
+        const bool mine = 2 * h < nuse;
+        const int lim = qlim - (kbase + 64 * h);  // this half's keys i <= lim are visible
+        // pass 1: this half's row maximum over the visible keys
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (mine) {
 #pragma unroll 1
-        for (int hh = 0; 2 * hh < nuse; ++hh) {
-          uint32_t raw[32];
-          tmem_ld32(tS + 64 * hh, raw);
-          uint32_t raw2[32];
-          tmem_ld32(tS + 64 * hh + 32, raw2);
-          tmem_ld_wait();
-          const int lim = qlim - (kbase + 64 * hh);  // keys i <= lim are visible
-          if (lim >= 63) {  // all 64 visible (every block but the diagonal / the user's last)
+          for (int c = 0; c < 2; ++c) {  // 32 columns per TMEM load
+            uint32_t raw[32];
+            tmem_ld32(tS + 32 * c, raw);
+            tmem_ld_wait();
+            const int lc = lim - 32 * c;
+            if (lc >= 31) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
-              mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw2[i]));
-            }
-          } else {
+              for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (i <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
-              if (i + 32 <= lim) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw2[i]));
+              for (int i = 0; i < 32; ++i)
+                if (i <= lc) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
             }
           }
         }
-        const float mblk = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c2;
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        // exchange the halves' maxima (and the previous step's sums)
+        tmem_st1(tX + xcol(h, n & 1, 0), __float_as_uint(mx));
+        tmem_st_wait();
+        if (!meet()) { ok = false; break; }
+        uint32_t xo, lo = 0;
+        tmem_ld1(tX + xcol(h ^ 1, n & 1, 0), xo);
+        if (pn >= 0 && plast) tmem_ld1(tX + xcol(h ^ 1, pn & 1, 1), lo);
+        tmem_ld_wait();
+        const float mblk = fmaxf(mx, __uint_as_float(xo)) * c2;
         // the previous PV must be done before O is touched or P rewritten
-        if (pn >= 0 && !finish_prev()) { ok = false; break; }
+        if (pn >= 0 && !finish_prev(pl + __uint_as_float(lo))) { ok = false; break; }
         if (kb == 0) {
           m = mblk;  // the unit's first PV overwrites O
           l = 0.f;
         } else if (__any_sync(0xffffffffu, mblk > m + RESCALE_LOG2)) {
           const float m_new = fmaxf(m, mblk);
           const float alpha = ex2_approx(m - m_new);
+          uint32_t o[32];
+          tmem_ld32(tO, o);
+          tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t raw[32];
-            tmem_ld32(tPV + 32 * c, raw);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-            tmem_st32(tPV + 32 * c, raw);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO, o);
           tmem_st_wait();
           l *= alpha;
           m = m_new;
         }
-        // pass 2: probabilities -> bf16 P (K-major, swizzled); masked and
-        // skipped columns give p = 0
-        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t pbase = smem_u32(sP + g * 2 * ATT_TILE_BYTES) + r * 128;
+        // pass 2: this half's probabilities -> bf16 P column block h
+        // (K-major, swizzled); masked and skipped columns give p = 0
+        const uint32_t row_addr = smem_u32(sP + g * 2 * ATT_TILE_BYTES + h * ATT_TILE_BYTES) + r * 128;
+        if (mine) {
+          float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-        for (int hh = 0; 2 * hh < nch; ++hh) {
-          const uint32_t row_addr = pbase + hh * ATT_TILE_BYTES;  // column block hh: keys 64hh..64hh+63
-          if (2 * hh < nuse) {
+          for (int c = 0; c < 2; ++c) {  // keys 32c..32c+31 of the half: 16-byte chunks 4c..4c+3
             uint32_t raw[32];
-            tmem_ld32(tS + 64 * hh, raw);
-            uint32_t raw2[32];
-            tmem_ld32(tS + 64 * hh + 32, raw2);
+            tmem_ld32(tS + 32 * c, raw);
             tmem_ld_wait();
-            // keys i <= lim are visible; all 64 on every block but the
-            // diagonal / the user's last (no selects there)
-            const int lim = qlim - (kbase + 64 * hh);
-            const int lim_eff = lim >= 63 ? 63 : lim;
+            const int lc = lim - 32 * c;
+            const int lc_eff = lc >= 31 ? 31 : lc;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {  // 16-byte chunk q = keys 8q..8q+7
+            for (int q = 0; q < 4; ++q) {
               uint32_t pk[4];
 #pragma unroll
               for (int j = 0; j < 8; j += 2) {
                 const int i = 8 * q + j;
-                const float s0 = __uint_as_float(q < 4 ? raw[i] : raw2[i - 32]);
-                const float s1 = __uint_as_float(q < 4 ? raw[i + 1] : raw2[i - 31]);
-                float p0 = ex2_approx(s0 * c2 - m);
-                float p1 = ex2_approx(s1 * c2 - m);
-                if (lim < 63) {
-                  p0 = (i <= lim_eff) ? p0 : 0.f;
-                  p1 = (i + 1 <= lim_eff) ? p1 : 0.f;
+                float p0 = ex2_approx(__uint_as_float(raw[i]) * c2 - m);
+                float p1 = ex2_approx(__uint_as_float(raw[i + 1]) * c2 - m);
+                if (lc < 31) {
+                  p0 = (i <= lc_eff) ? p0 : 0.f;
+                  p1 = (i + 1 <= lc_eff) ? p1 : 0.f;
                 }
                 ls4[j >> 1] += p0 + p1;
                 pk[j >> 1] = pack_bf16x2(p0, p1);
               }
-              st_shared_v4(row_addr + ((q ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+              const int qc = 4 * c + q;
+              st_shared_v4(row_addr + ((qc ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
             }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) st_shared_v4(row_addr + ((q ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
           }
+          l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+        } else if (2 * h < nch) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) st_shared_v4(row_addr + ((q ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
         }
-        l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+        // this half's sum so far, for the other half at the unit's end
+        tmem_st1(tX + xcol(h, n & 1, 1), __float_as_uint(l));
+        tmem_st_wait();
         // S is read and P written (and O rescaled): the next QK^T and this PV may start
         tc_fence_before();
         mbar_arrive(&s_empty[g]);
@@ -500,7 +534,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         pdst = qi < a.L ? (a.s0 + qi) * D + a.h * DH : -1;
       }
     }
-    if (ok && pn >= 0) ok = finish_prev();
+    if (ok && pn >= 0) {
+      // the stream's last unit: the other half's sum, then O / l
+      uint32_t lo = 0;
+      ok = meet();
+      if (ok) {
+        tmem_ld1(tX + xcol(h ^ 1, pn & 1, 1), lo);
+        tmem_ld_wait();
+        ok = finish_prev(pl + __uint_as_float(lo));
+      }
+    }
     if (!ok) set_error(err, PTL_ERR_TIMEOUT);
   }
   tc_fence_before();

@@ -224,6 +224,14 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// One 32-bit column of the warp's 32 TMEM lanes (one value per thread).
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& v) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr) : "memory");
+}
+
 // ------------------------------------------------- CTA pairs (cta_group::2)
 // A cluster of two CTAs on two SMs runs one M=256 MMA: each CTA holds 128
 // rows of A and half of B's N rows in its own shared memory at the same
