@@ -11,11 +11,13 @@
 // polls both and advances whichever is ready), so a stream never waits for
 // the other's softmax:
 //
-//   warp 0      TMA producer: the Q tile [128 x 64] of each stream's current
-//               unit, and per step the K and V tiles [128 x 64] through a
-//               per-stream 2-deep ring, straight from the packed qkv rows
-//               (128-byte swizzle); K and V have separate barriers, so the
-//               next K loads as soon as its slot's QK^T is done;
+//   warp 0      TMA producer, straight from the packed qkv rows (128-byte
+//               swizzle): the Q tile [128 x 64] of each stream's units
+//               (double-buffered, so the next unit's Q loads while the
+//               current unit runs), per step the K tile through a per-stream
+//               2-deep ring (a slot frees when its QK^T is done) and the V
+//               tile into the stream's single V buffer (freed by the
+//               previous step's PV);
 //   warp 1      MMA issuer: for a step of stream g, S = Q K^T (M=128, N = the
 //               keys of this block rounded up to 16) into TMEM S[g], and --
 //               once warpgroup g has written P for that step -- O[g] += P V
@@ -47,11 +49,11 @@ namespace ptl {
 using namespace sm100;
 
 constexpr int ATT_TILE_BYTES = ATT_BLK * DH * 2;  // 16 KB
-// K/V ring stages per stream: a stream holds one stage until its deferred
-// PV is done and needs the next one loaded before its next QK^T can start.
+// K ring stages per stream: a K tile is held until its QK^T is done and the
+// next one must be loaded before the stream's next QK^T can start.
 constexpr int ATT_KV_STAGES = 2;
-// Q[2] + (K,V)[2 streams][stages] + P[2][2 column blocks]
-constexpr int ATT_SMEM_TILES = 2 + 2 * 2 * ATT_KV_STAGES + 4;
+// per stream: Q[2] + K[stages] + V[1] + P[2 column blocks]
+constexpr int ATT_SMEM_TILES = 2 * (2 + ATT_KV_STAGES + 1 + 2);
 constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 512;  // + alignment, barriers
 constexpr int ATT_THREADS = 576;  // producer, MMA, four softmax warpgroups (two per stream)
 
@@ -169,20 +171,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                                          // [stream]
-  uint8_t* sKV = smem + 2 * ATT_TILE_BYTES;                    // [stream][stage]: K then V
-  uint8_t* sP = sKV + 2 * 2 * ATT_KV_STAGES * ATT_TILE_BYTES;  // [stream]: two 64-key column blocks each
+  // per stream: Q[2 units], K[ATT_KV_STAGES steps], V[1 step], P[2 column blocks]
+  uint8_t* sQ = smem;                                       // [stream][unit slot]
+  uint8_t* sK = sQ + 2 * 2 * ATT_TILE_BYTES;                // [stream][stage]
+  uint8_t* sV = sK + 2 * ATT_KV_STAGES * ATT_TILE_BYTES;    // [stream]
+  uint8_t* sP = sV + 2 * ATT_TILE_BYTES;                    // [stream][column block]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);
-  uint64_t* q_full = bars;          // [stream]
-  uint64_t* q_empty = bars + 2;     // [stream]
-  // K and V have their own barriers: a K tile is free once its QK^T is done,
-  // long before the step's PV frees the V tile, so the next K load can start
-  // early
-  uint64_t* k_full = bars + 4;                        // [stream][stage]
+  // Q is double-buffered (the next unit's Q loads while the current unit
+  // runs); K is a ring whose slot frees once its QK^T is done; V (needed
+  // only by the step's PV, a softmax step later) has one buffer per stream.
+  uint64_t* q_full = bars;                            // [stream][unit slot]
+  uint64_t* q_empty = bars + 4;                       // [stream][unit slot]
+  uint64_t* k_full = bars + 8;                        // [stream][stage]
   uint64_t* k_empty = k_full + 2 * ATT_KV_STAGES;     // [stream][stage]
-  uint64_t* v_full = k_empty + 2 * ATT_KV_STAGES;     // [stream][stage]
-  uint64_t* v_empty = v_full + 2 * ATT_KV_STAGES;     // [stream][stage]
-  uint64_t* s_full = v_empty + 2 * ATT_KV_STAGES;     // [stream]
+  uint64_t* v_full = k_empty + 2 * ATT_KV_STAGES;     // [stream]
+  uint64_t* v_empty = v_full + 2;                     // [stream]
+  uint64_t* s_full = v_empty + 2;                     // [stream]
   uint64_t* s_empty = s_full + 2;                 // [stream]
   uint64_t* p_full = s_full + 4;                  // [stream]
   uint64_t* pv_done = s_full + 6;                 // [stream]
@@ -193,9 +197,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 256);
       mbar_init(&p_full[i], 256);
@@ -206,8 +214,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     for (int i = 0; i < 2 * ATT_KV_STAGES; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
@@ -229,45 +235,65 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // softmax exchange 384..399
 
   // The producer and the MMA issuer serve the two streams independently:
-  // each polls both streams (non-blocking barrier tests) and advances
+  // each polls both streams (non-blocking barrier tests: test_wait, which
+  // never suspends the thread) and advances
   // whichever is ready, so neither stream waits for the other's softmax.
   // They give up (PTL_ERR_TIMEOUT) after a second without progress.
   if (warp == 0) {
     if (lane == 0) {
       AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
       gen.init(items, cu, nunits);
+      // V tiles wait in a small per-stream queue (row of the step's keys,
+      // head): V of step n loads once the stream's PV of step n - 1 is done
+      int vq0_row[2], vq0_col[2], vq1_row[2], vq1_col[2];  // [queue entry][stream]
+      int vq_n[2] = {0, 0}, vq_len[2] = {0, 0};           // next V step, queued entries
       auto produce = [&](StreamPos& sp) -> bool {
         const int g = sp.g;
-        const AttnUnit a = sp.u;
-        if (sp.kb == 0 && !sp.q_sent) {  // a new unit of stream g: its Q tile
-          if (!mbar_try_wait(&q_empty[g], (sp.uc & 1) ^ 1)) return false;
-          mbar_arrive_expect_tx(&q_full[g], ATT_TILE_BYTES);
-          tma_load_2d(sQ + g * ATT_TILE_BYTES, &tm_qkv, &q_full[g], a.h * DH, a.s0 + a.b * ATT_BLK);
-          sp.q_sent = true;
+        bool prog = false;
+        // the oldest queued V
+        if (vq_len[g] > 0 && mbar_test_wait(&v_empty[g], (vq_n[g] & 1) ^ 1)) {
+          mbar_arrive_expect_tx(&v_full[g], ATT_TILE_BYTES);
+          tma_load_2d(sV + g * ATT_TILE_BYTES, &tm_qkv, &v_full[g], vq0_col[g], vq0_row[g]);
+          ++vq_n[g];
+          --vq_len[g];
+          vq0_row[g] = vq1_row[g];
+          vq0_col[g] = vq1_col[g];
+          prog = true;
         }
+        if (!sp.live || vq_len[g] == 2) return prog;
+        const AttnUnit a = sp.u;
+        const int qs = sp.uc & 1;  // the unit's Q slot
+        if (sp.kb == 0 && !sp.q_sent) {  // a new unit of stream g: its Q tile
+          if (!mbar_test_wait(&q_empty[2 * g + qs], ((sp.uc >> 1) & 1) ^ 1)) return prog;
+          mbar_arrive_expect_tx(&q_full[2 * g + qs], ATT_TILE_BYTES);
+          tma_load_2d(sQ + (2 * g + qs) * ATT_TILE_BYTES, &tm_qkv, &q_full[2 * g + qs], a.h * DH,
+                      a.s0 + a.b * ATT_BLK);
+          sp.q_sent = true;
+          prog = true;
+        }
+        // the step's K tile, once the slot's previous QK^T is done
         const int st = sp.n % ATT_KV_STAGES, use = sp.n / ATT_KV_STAGES;
         const int slot = g * ATT_KV_STAGES + st;
-        uint8_t* kbuf = sKV + (2 * slot) * ATT_TILE_BYTES;
+        if (!mbar_test_wait(&k_empty[slot], (use & 1) ^ 1)) return prog;
+        mbar_arrive_expect_tx(&k_full[slot], ATT_TILE_BYTES);
         const int row = a.s0 + sp.kb * ATT_BLK;
-        if (!sp.k_sent) {  // the step's K tile, once the slot's previous QK^T is done
-          if (!mbar_try_wait(&k_empty[slot], (use & 1) ^ 1)) return false;
-          mbar_arrive_expect_tx(&k_full[slot], ATT_TILE_BYTES);
-          tma_load_2d(kbuf, &tm_qkv, &k_full[slot], D + a.h * DH, row);
-          sp.k_sent = true;
+        tma_load_2d(sK + slot * ATT_TILE_BYTES, &tm_qkv, &k_full[slot], D + a.h * DH, row);
+        // queue its V
+        if (vq_len[g] == 0) {
+          vq0_row[g] = row;
+          vq0_col[g] = 2 * D + a.h * DH;
+        } else {
+          vq1_row[g] = row;
+          vq1_col[g] = 2 * D + a.h * DH;
         }
-        // its V tile, once the slot's previous PV is done
-        if (!mbar_try_wait(&v_empty[slot], (use & 1) ^ 1)) return false;
-        mbar_arrive_expect_tx(&v_full[slot], ATT_TILE_BYTES);
-        tma_load_2d(kbuf + ATT_TILE_BYTES, &tm_qkv, &v_full[slot], 2 * D + a.h * DH, row);
-        sp.k_sent = false;
+        ++vq_len[g];
         gen.step(items, cu, sp);
         return true;
       };
       uint64_t t_prog = globaltimer_ns();
-      while (gen.a.live || gen.b.live) {
-        bool prog = false;
-        if (gen.a.live) prog |= produce(gen.a);
-        if (gen.b.live) prog |= produce(gen.b);
+      while (gen.a.live || gen.b.live || vq_len[0] > 0 || vq_len[1] > 0) {
+        bool prog = produce(gen.a);
+        prog |= produce(gen.b);
         if (prog) {
           t_prog = globaltimer_ns();
         } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
@@ -285,19 +311,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       auto issue_pv = [&](StreamPos& sp) -> bool {
         const int nn = sp.pv_n;
         const int gs = sp.g;
-        if (!mbar_try_wait(&p_full[gs], nn & 1)) return false;
-        if (sp.pv_first && !mbar_try_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
-        if (!mbar_try_wait(&v_full[gs * ATT_KV_STAGES + sp.pv_st], (nn / ATT_KV_STAGES) & 1)) return false;
+        if (!mbar_test_wait(&p_full[gs], nn & 1)) return false;
+        if (sp.pv_first && !mbar_test_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
+        if (!mbar_test_wait(&v_full[gs], nn & 1)) return false;
         tc_fence_after();
         const uint32_t p0 = smem_u32(sP + gs * 2 * ATT_TILE_BYTES);
-        const uint32_t v0 = smem_u32(sKV + (2 * (gs * ATT_KV_STAGES + sp.pv_st) + 1) * ATT_TILE_BYTES);
+        const uint32_t v0 = smem_u32(sV + gs * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256 + 64 * gs;
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
         for (int k = 0; k < sp.pv_k16 / 16; ++k)
           umma_bf16_ss(d, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
                        umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !sp.pv_first);
         umma_commit(&pv_done[gs]);
-        umma_commit(&v_empty[gs * ATT_KV_STAGES + sp.pv_st]);
+        umma_commit(&v_empty[gs]);
         sp.pv_n = -1;
         return true;
       };
@@ -307,13 +333,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const AttnUnit a = sp.u;
         const int kb = sp.kb, nn = sp.n;
         const int st = nn % ATT_KV_STAGES, use = nn / ATT_KV_STAGES;
-        if (kb == 0 && !mbar_try_wait(&q_full[g], sp.uc & 1)) return false;
-        if (!mbar_try_wait(&k_full[g * ATT_KV_STAGES + st], use & 1)) return false;
-        if (!mbar_try_wait(&s_empty[g], (nn & 1) ^ 1)) return false;
+        const int qs = sp.uc & 1;
+        if (kb == 0 && !mbar_test_wait(&q_full[2 * g + qs], (sp.uc >> 1) & 1)) return false;
+        if (!mbar_test_wait(&k_full[g * ATT_KV_STAGES + st], use & 1)) return false;
+        if (!mbar_test_wait(&s_empty[g], (nn & 1) ^ 1)) return false;
         tc_fence_after();
         const int k16 = keys16(a.L, kb);
-        const uint32_t q0 = smem_u32(sQ + g * ATT_TILE_BYTES);
-        const uint32_t k0 = smem_u32(sKV + (2 * (g * ATT_KV_STAGES + st)) * ATT_TILE_BYTES);
+        const uint32_t q0 = smem_u32(sQ + (2 * g + qs) * ATT_TILE_BYTES);
+        const uint32_t k0 = smem_u32(sK + (g * ATT_KV_STAGES + st) * ATT_TILE_BYTES);
         const uint32_t idesc_qk = umma_idesc_bf16(128, k16);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -321,7 +348,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                        idesc_qk, k != 0);
         umma_commit(&s_full[g]);
         umma_commit(&k_empty[g * ATT_KV_STAGES + st]);
-        if (kb == a.b) umma_commit(&q_empty[g]);
+        if (kb == a.b) umma_commit(&q_empty[2 * g + qs]);
         sp.pv_n = nn;
         sp.pv_st = st;
         sp.pv_k16 = k16;

@@ -256,7 +256,7 @@ __device__ __forceinline__ void store_row16_groups(float* row, int lane, const f
 // The gate for one token, by one warp: LayerNorm2 of the x1 row into v (the
 // lane's 16 values in the fp32 lane layout: 4 groups of 4 consecutive columns
 // at q*128 + lane*4), the 8 logits in fp32 against the staged gate weights,
-// softmax, top-2 (ties to the lower index) and the renormalised weights.
+// top-2 of the softmax (ties to the lower index) and the renormalised weights.
 // Every lane returns the same e0, e1, w0, w1.
 __device__ __forceinline__ void gate_token(const float* __restrict__ x1_row, const float* __restrict__ g,
                                            const float* __restrict__ b, const float* __restrict__ s_wg,
@@ -279,35 +279,29 @@ __device__ __forceinline__ void gate_token(const float* __restrict__ x1_row, con
   float lg[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) lg[e] = __shfl_sync(0xffffffffu, mine, 4 * e);
-  // every lane evaluates the same (tiny) softmax / top-2
-  float m = lg[0];
+  // softmax is monotonic, so the top-2 of p are the top-2 logits (ties to the
+  // lower index), and the renormalised pair p0 / (p0 + p1), p1 / (p0 + p1)
+  // depends only on their difference: w0 = 1 / (1 + t), w1 = t / (1 + t)
+  // with t = exp(l1 - l0) <= 1.  Every lane evaluates the same values.
+  e0 = 0;
+  float l0 = lg[0];
 #pragma unroll
-  for (int e = 1; e < E; ++e) m = fmaxf(m, lg[e]);
-  float p[E], sum = 0.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    p[e] = expf(lg[e] - m);
-    sum += p[e];
-  }
-  e0 = -1;
-  e1 = -1;
-  float p0 = -1.f, p1 = -1.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const float pe = p[e] / sum;
-    if (pe > p0) {
-      e1 = e0;
-      p1 = p0;
+  for (int e = 1; e < E; ++e)
+    if (lg[e] > l0) {
+      l0 = lg[e];
       e0 = e;
-      p0 = pe;
-    } else if (pe > p1) {
-      e1 = e;
-      p1 = pe;
     }
-  }
-  const float den = p0 + p1;
-  w0 = p0 / den;
-  w1 = p1 / den;
+  e1 = -1;
+  float l1 = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (e != e0 && (e1 < 0 || lg[e] > l1)) {
+      l1 = lg[e];
+      e1 = e;
+    }
+  const float t = expf(l1 - l0);
+  w0 = 1.0f / (1.0f + t);
+  w1 = t * w0;
 }
 
 // Stages the gate weights [8][512] in shared memory; lane l later reads
@@ -342,6 +336,16 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
       atomicAdd(&chunk_cnt[(t >> 7) * E + e1], 1);
     }
   }
+}
+
+// Flag store / load with release / acquire semantics at GPU scope.
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------- gate + route
@@ -381,11 +385,13 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
   const int nchunks = (T_ + GR_TOK - 1) / GR_TOK;
   const int t = c * GR_TOK + warp;
   const bool valid = t < T_;
-  float v[16];
+  uint32_t vp[8];  // the token's LN2 values, packed bf16 pairs (fp32 lane layout)
   int e0 = E, e1 = E;
-  float w0 = 0.f, w1 = 0.f;
   if (valid) {
+    float v[16], w0, w1;
     gate_token(x1 + size_t(t) * D, g, b, s_wg, bg, lane, v, e0, e1, w0, w1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) vp[i] = sm_pack_bf16x2(v[2 * i], v[2 * i + 1]);
     if (lane == 0) {
       *reinterpret_cast<int2*>(idx + 2 * t) = make_int2(e0, e1);
       *reinterpret_cast<float2*>(wout + 2 * t) = make_float2(w0, w1);
@@ -414,30 +420,30 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
   // (one thread per earlier chunk, all read in parallel: no chain of
   // prefixes to wait for)
   int32_t* me = lb + 32 + 32 * c;
-  if (threadIdx.x < E) me[4 + threadIdx.x] = s_cnt[threadIdx.x];
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < E) {
+    me[4 + threadIdx.x] = s_cnt[threadIdx.x];
     __threadfence();
-    *reinterpret_cast<volatile int32_t*>(me) = 1;
   }
+  __syncthreads();
+  if (threadIdx.x == 0) st_release_gpu(me, 1);
   int part[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) part[e] = 0;
   for (int pc = threadIdx.x; pc < c; pc += blockDim.x) {
-    const volatile int32_t* pf = lb + 32 + 32 * pc;
-    int f = *pf;
+    const int32_t* pf = lb + 32 + 32 * pc;
+    int f = ld_acquire_gpu(pf);
     if (f == 0) {
       const uint64_t t0 = sm100::globaltimer_ns();
-      while ((f = *pf) == 0) {
+      while ((f = ld_acquire_gpu(pf)) == 0) {
         if (sm100::globaltimer_ns() - t0 > sm100::kWaitLimitNs) break;
+        __nanosleep(64);
       }
     }
     if (f == 0) {
       set_error(err, PTL_ERR_TIMEOUT);
       break;
     }
-    __threadfence();
+    // the acquire load orders these after the flag
     const int4* src = reinterpret_cast<const int4*>(lb + 32 + 32 * pc + 4);
     const int4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
     part[0] += v0.x;
@@ -471,7 +477,10 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
       const int e = k == 0 ? e0 : e1;
       const int row = e * cap + s_excl[e] + s_rank[2 * warp + k];
       if (lane == 0) pos[2 * t + k] = row;
-      store_row16_groups(xperm + size_t(row) * D, lane, v);
+      __nv_bfloat16* dst = xperm + size_t(row) * D;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)  // the layout of store_row16_groups
+        *reinterpret_cast<uint2*>(dst + q * 128 + lane * 4) = make_uint2(vp[2 * q], vp[2 * q + 1]);
     }
   }
   if (c == nchunks - 1) {
