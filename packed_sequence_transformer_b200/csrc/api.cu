@@ -233,7 +233,7 @@ ptl_status step_gate(const Call& c, const void* x1, void* xn2, int32_t* idx, flo
 // Routes + both expert GEMMs + combine + residual.  The per-chunk expert
 // counts must already be in the workspace.
 ptl_status step_experts(const Call& c, const float* wts, const void* resid, void* out,
-                        const ptl_layer_weights* w, const ptl_layer_weights* next);
+                        const ptl_layer_weights* w, const ptl_layer_weights* next, bool fused = false);
 
 // next (bf16 build, nullable): the following layer, whose LayerNorm1 of `out`
 // the combine also writes into the workspace.
@@ -262,8 +262,10 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
 // bf16: both expert GEMMs over the routed rows already in the workspace
 // (xperm, tiles, meta, pos), then the combine + residual (+ the next layer's
 // LayerNorm1 inside a stack).
+// fused: both expert GEMMs in one launch (the layer path, whose gate +
+// route kernel cleared the per-tile counters).
 ptl_status step_experts(const Call& c, const float* wts, const void* resid, void* out,
-                        const ptl_layer_weights* w, const ptl_layer_weights* next) {
+                        const ptl_layer_weights* w, const ptl_layer_weights* next, bool fused) {
   {
     CUtensorMap mx, m1, m2, mh, my;
     if (!map_bf16(&mx, c.ws + c.L.xperm, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
@@ -271,10 +273,15 @@ ptl_status step_experts(const Call& c, const float* wts, const void* resid, void
     if (!map_bf16(&m2, w->w2, F, uint64_t(E) * D, F * 2, 64, GEMM2_BN / 2)) return PTL_ERR_CUDA;
     if (!map_bf16(&mh, c.ws + c.L.hbuf, F, c.L.padded_rows, F * 2, 64, 128)) return PTL_ERR_CUDA;
     if (!map_bf16(&my, c.ws + c.L.ybuf, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
-    mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
-    PTL_TRY(launch_gemm_moe1(mx, m1, mh, F32(w->b1), c.L, c.ws, c.st));
-    mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
-    PTL_TRY(launch_gemm_moe2(mh, m2, my, F32(w->b2), c.L, c.ws, c.st));
+    if (fused) {
+      mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
+      PTL_TRY(launch_gemm_moe12(mx, m1, mh, m2, my, F32(w->b1), F32(w->b2), c.L, c.ws, c.st));
+    } else {
+      mark(c.st, PTL_KERNEL_GEMM_EXPERT1);
+      PTL_TRY(launch_gemm_moe1(mx, m1, mh, F32(w->b1), c.L, c.ws, c.st));
+      mark(c.st, PTL_KERNEL_GEMM_EXPERT2);
+      PTL_TRY(launch_gemm_moe2(mh, m2, my, F32(w->b2), c.L, c.ws, c.st));
+    }
     mark(c.st, PTL_KERNEL_COMBINE);
     PTL_TRY(launch_combine_bf16(c.ws + c.L.ybuf, at<int32_t>(c, c.L.pos), wts,
                                 static_cast<const float*>(resid), out, c.T,
@@ -305,7 +312,7 @@ ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu
       mark(c.st, PTL_KERNEL_ROUTE);
       PTL_TRY(launch_route_debug(c.T, c.L, c.ws, dbg->perm, dbg->expert_off, c.st));
     }
-    if ((s = step_experts(c, wts, c.ws + c.L.x1, out, w, next)) != PTL_OK) return s;
+    if ((s = step_experts(c, wts, c.ws + c.L.x1, out, w, next, true)) != PTL_OK) return s;
   } else {
     if ((s = step_gate(c, c.ws + c.L.x1, c.ws + c.L.xn2, idx, wts, w)) != PTL_OK) return s;
     if ((s = step_moe(c, c.ws + c.L.xn2, idx, wts, c.ws + c.L.x1, out, w, dbg ? dbg->perm : nullptr,

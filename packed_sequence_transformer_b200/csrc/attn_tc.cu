@@ -112,8 +112,12 @@ struct StreamPos {
   bool live, nxt_live;
   AttnUnit u, nxt;   // current unit, the next one (looked up one unit ahead)
   CtaWalker walk;
-  int pv_n, pv_st, pv_k16, pv_uc;  // the step whose PV is still to be issued (-1: none)
+  // the MMA issuer's queue of steps whose PV is still to be issued (oldest
+  // first; -1: none): a step's QK^T may go ahead of the previous step's PV
+  int pv_n, pv_k16, pv_uc;
   bool pv_first;
+  int pv2_n, pv2_k16, pv2_uc;
+  bool pv2_first;
   bool q_sent;       // producer: the current unit's Q tile load is issued
   bool k_sent;       // producer: the current step's K tile load is issued
 };
@@ -135,9 +139,9 @@ struct AttnStepGen {
     sp.n = 0;
     sp.uc = 0;
     sp.walk = CtaWalker();
-    sp.pv_n = -1;
-    sp.pv_st = sp.pv_k16 = sp.pv_uc = 0;
-    sp.pv_first = false;
+    sp.pv_n = sp.pv2_n = -1;
+    sp.pv_k16 = sp.pv_uc = sp.pv2_k16 = sp.pv2_uc = 0;
+    sp.pv_first = sp.pv2_first = false;
     sp.q_sent = false;
     sp.k_sent = false;
     fetch_next(items, cu, sp);
@@ -299,6 +303,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
           set_error(err, PTL_ERR_TIMEOUT);
           break;
+        } else {
+          __nanosleep(20);  // leave issue slots to the softmax warps while idle
         }
       }
     }
@@ -324,10 +330,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                        umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !sp.pv_first);
         umma_commit(&pv_done[gs]);
         umma_commit(&v_empty[gs]);
-        sp.pv_n = -1;
+        sp.pv_n = sp.pv2_n;  // pop the queue
+        sp.pv_k16 = sp.pv2_k16;
+        sp.pv_uc = sp.pv2_uc;
+        sp.pv_first = sp.pv2_first;
+        sp.pv2_n = -1;
         return true;
       };
-      // S = Q K^T for the stream's next step (its previous PV already issued)
+      // S = Q K^T for the stream's next step; queues the step's PV
       auto issue_s = [&](StreamPos& sp) -> bool {
         const int g = sp.g;
         const AttnUnit a = sp.u;
@@ -349,18 +359,27 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         umma_commit(&s_full[g]);
         umma_commit(&k_empty[g * ATT_KV_STAGES + st]);
         if (kb == a.b) umma_commit(&q_empty[2 * g + qs]);
-        sp.pv_n = nn;
-        sp.pv_st = st;
-        sp.pv_k16 = k16;
-        sp.pv_first = kb == 0;
-        sp.pv_uc = sp.uc;
+        if (sp.pv_n < 0) {
+          sp.pv_n = nn;
+          sp.pv_k16 = k16;
+          sp.pv_first = kb == 0;
+          sp.pv_uc = sp.uc;
+        } else {
+          sp.pv2_n = nn;
+          sp.pv2_k16 = k16;
+          sp.pv2_first = kb == 0;
+          sp.pv2_uc = sp.uc;
+        }
         gen.step(items, cu, sp);
         return true;
       };
+      // a stream's next QK^T needs no PV of it issued first: the softmax of
+      // that step waits for the previous PV before it writes P, so at most
+      // two PVs are ever queued
       auto serve = [&](StreamPos& sp) -> bool {
         bool prog = false;
         if (sp.pv_n >= 0 && issue_pv(sp)) prog = true;
-        if (sp.pv_n < 0 && sp.live && issue_s(sp)) prog = true;
+        if (sp.pv2_n < 0 && sp.live && issue_s(sp)) prog = true;
         return prog;
       };
       uint64_t t_prog = globaltimer_ns();
@@ -372,6 +391,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
           set_error(err, PTL_ERR_TIMEOUT);
           break;
+        } else {
+          __nanosleep(20);  // leave issue slots to the softmax warps while idle
         }
       }
     }

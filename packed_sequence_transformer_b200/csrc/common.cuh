@@ -43,6 +43,7 @@ struct WsLayout {
   size_t wgt;         // f32 [T][2]
   size_t chunk_cnt;   // int32 [n_chunks][8]
   size_t lb;          // int32 [32 + 32 * n_gchunks]  fused gate + route: ticket, per-chunk look-back state
+  size_t moe_done;    // int32 [max_tiles]  fused expert GEMMs: first-GEMM tiles done per M tile
   size_t perm;        // int32 [2T]
   size_t pos;         // int32 [2T]          route -> padded expert row
   size_t rowroute;    // int32 [padded_rows]   padded expert rows -> route (or -1)
@@ -97,6 +98,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->wl_end = o;  // error word + attention work list
   L->chunk_cnt = take(4 * L->n_chunks * E);
   L->lb = take(4 * (32 + 32 * L->n_gchunks));
+  L->moe_done = take(4 * L->max_tiles);
   L->clear_end = o;  // [0, clear_end) is cleared by one memset per call
   L->xn = take(es * T * D);
   L->qkv = take(es * T * QKV_N);

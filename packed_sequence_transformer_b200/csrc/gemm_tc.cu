@@ -60,10 +60,15 @@ struct GemmTcParams {
   const int32_t* meta;           // [0] = number of M tiles
   int32_t* zero_ptr;             // cleared by the grid once the predecessor is done (may be NULL)
   int zero_n;
+  // MOE12 (both expert GEMMs in one launch): the second GEMM's width, bias
+  // and per-M-tile completion counters of the first GEMM (zero at launch)
+  int N2;
+  const float* bias2;
+  int32_t* done;
   int32_t* err;
 };
 
-enum { G_QKV = 0, G_OUT = 1, G_MOE1 = 2, G_MOE2 = 3 };
+enum { G_QKV = 0, G_OUT = 1, G_MOE1 = 2, G_MOE2 = 3, G_MOE12 = 4 };
 
 // Shared-memory plan: the operand ring, the output staging tile and the
 // tile's bias slice.
@@ -71,7 +76,10 @@ template <int BN, int MODE>
 struct PairCfg {
   static constexpr int OUT_ELEM = MODE == G_OUT ? 4 : 2;
   static constexpr int BOX_COLS = 128 / OUT_ELEM;
-  static constexpr int STAGING = 128 * BN * OUT_ELEM;
+  // columns staged (and stored) at a time: the fp32 output of a wide tile
+  // goes out in two 128-column parts through one 64 KB staging buffer
+  static constexpr int PART = (MODE == G_OUT && BN > 128) ? 128 : BN;
+  static constexpr int STAGING = 128 * PART * OUT_ELEM;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = (BN / 2) * 64 * 2;
   static constexpr int BIAS = BN * 4;
@@ -85,11 +93,20 @@ struct PairCfg {
 };
 
 // Pair tile `tile` -> (expert, first row of the pair's 256 rows, first column).
+// For MOE12 the tiles of the first expert GEMM come first (M tiles x F/BN),
+// then those of the second (M tiles x D/BN); `second` tells them apart and
+// `mt` is the tile's M tile.
 template <int BN, int MODE>
-__device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile, int& expert, int& m0,
-                                                 int& n0) {
-  const int nN = p.N_total / BN;
-  const int mt = tile / nN;
+__device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile, int n_mt, int& expert,
+                                                 int& m0, int& n0, bool& second, int& mt) {
+  second = false;
+  int nN = p.N_total / BN;
+  if (MODE == G_MOE12 && tile >= n_mt * nN) {
+    tile -= n_mt * nN;
+    nN = p.N2 / BN;
+    second = true;
+  }
+  mt = tile / nN;
   n0 = (tile - mt * nN) * BN;
   if (MODE >= G_MOE1) {
     const int2 tl = p.tiles[mt];
@@ -101,10 +118,25 @@ __device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile
   }
 }
 
+// Release / acquire on a GPU-scope counter (MOE12 tile dependencies).
+__device__ __forceinline__ void red_release_gpu_add(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t ld_acquire_gpu_s32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 template <int BN, int MODE>
 __global__ void __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmOut, const GemmTcParams p) {
+                     const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmA2,
+                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut2,
+                     const GemmTcParams p) {
   using Cfg = PairCfg<BN, MODE>;
   constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -138,6 +170,11 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmOut);
+    if (MODE == G_MOE12) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB2);
+      tma_prefetch_desc(&tmOut2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
@@ -148,17 +185,21 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   pdl_wait();  // inputs, route tables and the error word come from earlier kernels
   pdl_trigger();  // dependents launch once this grid has passed its own wait
+  __shared__ int s_nmt;
   if (threadIdx.x == 0) {
-    int nt = MODE >= G_MOE1 ? p.meta[0] * (p.N_total / BN) : p.n_tiles_dense;
+    const int nmt = MODE >= G_MOE1 ? p.meta[0] : 0;
+    int nt = MODE >= G_MOE1 ? nmt * (p.N_total / BN) : p.n_tiles_dense;
+    if (MODE == G_MOE12) nt += nmt * (p.N2 / BN);
     s_ntiles = has_error(p.err) ? 0 : nt;
+    s_nmt = nmt;
   }
   if (p.zero_ptr)
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.zero_n; i += gridDim.x * blockDim.x)
       p.zero_ptr[i] = 0;
   __syncthreads();
   const int ntiles = s_ntiles;
+  const int n_mt = s_nmt;
   const uint32_t tmem = *tmem_slot;
-  const int nkb = p.num_kb;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -168,10 +209,30 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       constexpr uint32_t tx = 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES);
       for (int tile = pair; tile < ntiles && ok; tile += npairs) {
-        int expert, m0, n0;
-        decode_pair_tile<BN, MODE>(p, tile, expert, m0, n0);
+        int expert, m0, n0, mt;
+        bool second;
+        decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt);
         const int arow = m0 + 128 * int(cr);
-        const int brow = expert * p.N_total + n0 + int(cr) * (BN / 2);
+        const int brow = expert * (second ? p.N2 : p.N_total) + n0 + int(cr) * (BN / 2);
+        const int nkb = second ? p.N_total / 64 : p.num_kb;
+        const CUtensorMap* ma = second ? &tmA2 : &tmA;
+        const CUtensorMap* mb = second ? &tmB2 : &tmB;
+        if (MODE == G_MOE12 && second) {
+          // the tile's A rows (H) come from every first-GEMM tile of this M
+          // tile, each stored by both CTAs of its pair
+          const int need = 2 * (p.N_total / BN);
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu_s32(p.done + mt) < need) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              set_error(p.err, PTL_ERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+            __nanosleep(64);
+          }
+          if (!ok) break;
+          fence_proxy_async_global();  // the H rows were written by TMA stores
+        }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
@@ -181,8 +242,8 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (cr == 0) mbar_arrive_expect_tx(&full[s], tx);
           const uint32_t fb = full0 + uint32_t(s) * 8u;
-          tma_load_2d_pair(sA + s * Cfg::A_BYTES, &tmA, fb, kb * 64, arow);
-          tma_load_2d_pair(sB + s * Cfg::B_BYTES, &tmB, fb, kb * 64, brow);
+          tma_load_2d_pair(sA + s * Cfg::A_BYTES, ma, fb, kb * 64, arow);
+          tma_load_2d_pair(sB + s * Cfg::B_BYTES, mb, fb, kb * 64, brow);
         }
       }
     }
@@ -192,6 +253,10 @@ __global__ void __launch_bounds__(192, 1)
       int it = 0, j = 0;
       bool ok = true;
       for (int tile = pair; tile < ntiles && ok; tile += npairs, ++j) {
+        int expert, m0, n0, mt;
+        bool second;
+        decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt);
+        const int nkb = second ? p.N_total / 64 : p.num_kb;
         const int acc = j & 1;
         if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1)) {
           set_error(p.err, PTL_ERR_TIMEOUT);
@@ -224,26 +289,49 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
     int j = 0;
+    int pending_mt = -1;  // MOE12: M tile of the first-GEMM tile whose store is in flight
+    // MOE12: once this CTA's store of a first-GEMM tile is complete, count it
+    // for the second GEMM's producers (leader thread, right after the store:
+    // a pair's own later second-GEMM tiles may be the ones waiting for it)
+    auto publish = [&]() {
+      if (MODE == G_MOE12 && pending_mt >= 0) {
+        tma_store_wait_all();
+        fence_proxy_async_global();
+        red_release_gpu_add(p.done + pending_mt, 1);
+        pending_mt = -1;
+      }
+    };
     for (int tile = pair; tile < ntiles; tile += npairs, ++j) {
-      int expert, m0, n0;
-      decode_pair_tile<BN, MODE>(p, tile, expert, m0, n0);
+      int expert, m0, n0, mt;
+      bool second;
+      decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt);
       m0 += 128 * int(cr);  // this CTA's rows
       const int acc = j & 1;
       const int row = m0 + r;
-      const float* bb = p.bias ? p.bias + (MODE >= G_MOE1 ? expert * p.N_total : 0) + n0 : nullptr;
+      const float* bias_base = second ? p.bias2 : p.bias;
+      const float* bb = bias_base ? bias_base + (MODE >= G_MOE1 ? expert * (second ? p.N2 : p.N_total) : 0) + n0
+                                  : nullptr;
+      const bool relu = MODE == G_MOE1 || (MODE == G_MOE12 && !second);
       float bv[(BN + 127) / 128];
 #pragma unroll
       for (int i = 0; i < (BN + 127) / 128; ++i)
         bv[i] = (bb && r + 128 * i < BN) ? __ldg(bb + r + 128 * i) : 0.f;
-      constexpr int NRES = MODE == G_OUT ? BN / 8 : 1;
-      uint4 res[NRES];
-      if (MODE == G_OUT) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0);
+      constexpr int PART = Cfg::PART, NPART = BN / PART;
+      constexpr int NRES = MODE == G_OUT ? PART / 8 : 1;
+      uint4 res[NRES];  // this thread's residual row, one part at a time
+      auto load_res = [&](int pt) {
+        if (MODE == G_OUT) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0 + pt * PART);
 #pragma unroll
-        for (int q = 0; q < NRES; ++q) res[q] = row < p.M ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
-      }
+          for (int q = 0; q < NRES; ++q) res[q] = row < p.M ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
+        }
+      };
+      load_res(0);
       const bool leader = warp == 2 && lane == 0;
-      if (j > 0 && leader) tma_store_wait_read();
+      if (j > 0 && leader) {
+        tma_store_wait_read();
+        publish();
+      }
 #pragma unroll
       for (int i = 0; i < (BN + 127) / 128; ++i)
         if (r + 128 * i < BN) s_bias[r + 128 * i] = bv[i];
@@ -254,68 +342,90 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem + uint32_t(acc * BN) + lane_off;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(taddr + 32 * c, raw);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 b4 = *reinterpret_cast<const float4*>(s_bias + 32 * c + 4 * q);
-          v[4 * q] += b4.x;
-          v[4 * q + 1] += b4.y;
-          v[4 * q + 2] += b4.z;
-          v[4 * q + 3] += b4.w;
+#pragma unroll 1
+      for (int pt = 0; pt < NPART; ++pt) {
+        if (pt > 0) {  // the previous part's store must have read the staging tile
+          load_res(pt);
+          if (leader) tma_store_wait_read();
+          named_barrier(1, 128);
         }
-        if (MODE == G_MOE1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
-        }
-        if (MODE == G_OUT) {
+        for (int c = 0; c < PART / 32; ++c) {
+          const int col = pt * PART + 32 * c;  // column within the tile
+          uint32_t raw[32];
+          tmem_ld32(taddr + col, raw);
+          tmem_ld_wait();
+          float v[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 u = res[4 * c + q];
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = __bfloat1622float2(h2[i]);
-              v[8 * q + 2 * i] += f.x;
-              v[8 * q + 2 * i + 1] += f.y;
+          for (int q = 0; q < 8; ++q) {
+            const float4 b4 = *reinterpret_cast<const float4*>(s_bias + col + 4 * q);
+            v[4 * q] += b4.x;
+            v[4 * q + 1] += b4.y;
+            v[4 * q + 2] += b4.z;
+            v[4 * q + 3] += b4.w;
+          }
+          if (relu) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
+          }
+          if (MODE == G_OUT) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = res[4 * c + q];
+              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h2[i]);
+                v[8 * q + 2 * i] += f.x;
+                v[8 * q + 2 * i + 1] += f.y;
+              }
+            }
+            // 32 fp32 = one 128-byte box row: box c of the part, chunks 0..7
+            const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                           __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+          } else {
+            // 32 bf16 = half a box row: box c/2, chunks (c%2)*4 .. +3
+            const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int chunk = (c & 1) * 4 + q;
+              st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pack_bf16x2(v[8 * q], v[8 * q + 1]),
+                           pack_bf16x2(v[8 * q + 2], v[8 * q + 3]), pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                           pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
             }
           }
-          const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                         __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
-        } else {
-          const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = (c & 1) * 4 + q;
-            st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pack_bf16x2(v[8 * q], v[8 * q + 1]),
-                         pack_bf16x2(v[8 * q + 2], v[8 * q + 3]), pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                         pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-          }
+        }
+        if (pt == NPART - 1) {
+          // this warp's rows of the accumulator are read: release it on CTA 0
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+        }
+        fence_proxy_async_smem();
+        named_barrier(1, 128);
+        if (leader) {
+          const CUtensorMap* mo = second ? &tmOut2 : &tmOut;
+#pragma unroll 1
+          for (int bx = 0; bx < PART / Cfg::BOX_COLS; ++bx)
+            tma_store_2d(mo, sOut + bx * 16384, n0 + pt * PART + bx * Cfg::BOX_COLS, m0);
+          tma_store_commit();
         }
       }
-      // this warp's rows of the accumulator are read: release it on CTA 0
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
-      fence_proxy_async_smem();
-      named_barrier(1, 128);
-      if (leader) {
-#pragma unroll 1
-        for (int bx = 0; bx < BN / Cfg::BOX_COLS; ++bx)
-          tma_store_2d(&tmOut, sOut + bx * 16384, n0 + bx * Cfg::BOX_COLS, m0);
-        tma_store_commit();
+      if (leader && MODE == G_MOE12 && !second) {
+        // publish right away: this pair's own second-GEMM tiles may wait on it
+        pending_mt = mt;
+        publish();
       }
     }
-    if (warp == 2 && lane == 0) tma_store_wait_all();
+    if (warp == 2 && lane == 0) {
+      tma_store_wait_all();
+      publish();
+    }
   }
   tc_fence_before();
   cluster_sync();  // no MMA, TMEM read or remote arrival of either CTA is outstanding
@@ -340,7 +450,8 @@ static int num_sms() {
 // Launches the CTA-pair kernel: clusters of two CTAs, one pair per two SMs.
 template <int BN, int MODE>
 static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
-                       const GemmTcParams& p, int tiles_bound, cudaStream_t st) {
+                       const GemmTcParams& p, int tiles_bound, cudaStream_t st, const CUtensorMap* a2 = nullptr,
+                       const CUtensorMap* b2 = nullptr, const CUtensorMap* out2 = nullptr) {
   static int max_pairs = 0;  // co-resident clusters of two (one CTA per SM)
   const int smem = PairCfg<BN, MODE>::SMEM;
   cudaLaunchConfig_t cfg = {};
@@ -370,7 +481,9 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   if (tiles_bound < pairs) pairs = tiles_bound;
   if (pairs < 1) pairs = 1;
   cfg.gridDim = dim3(2 * pairs);
-  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, MODE>, a, b, out, p) != cudaSuccess) return -1;
+  if (cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, MODE>, a, b, out, a2 ? *a2 : a, b2 ? *b2 : b,
+                         out2 ? *out2 : out, p) != cudaSuccess)
+    return -1;
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
@@ -420,6 +533,27 @@ int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUte
   p.zero_ptr = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
   p.zero_n = int((L.clear_end - L.chunk_cnt) / 4);
   return launch_pair<MOE1_BN, G_MOE1>(xperm, w1, hbuf_out, p, int(L.max_tiles) * (F / MOE1_BN), st);
+}
+
+int launch_gemm_moe12(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf,
+                      const CUtensorMap& w2, const CUtensorMap& ybuf_out, const float* b1, const float* b2,
+                      const WsLayout& L, char* ws, cudaStream_t st) {
+  static_assert(MOE1_BN == GEMM2_BN, "both expert GEMMs share one tile shape");
+  GemmTcParams p{};
+  p.N_total = F;
+  p.num_kb = D / 64;
+  p.bias = b1;
+  p.N2 = D;
+  p.bias2 = b2;
+  p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
+  p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
+  p.err = reinterpret_cast<int32_t*>(ws + L.err);
+  p.done = reinterpret_cast<int32_t*>(ws + L.moe_done);
+  // the routing state of this layer is consumed: clear it for the next layer
+  p.zero_ptr = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
+  p.zero_n = int((L.lb - L.chunk_cnt) / 4 + 32 + 32 * L.n_gchunks);
+  return launch_pair<MOE1_BN, G_MOE12>(xperm, w1, hbuf, p, int(L.max_tiles) * (F + D) / MOE1_BN, st, &hbuf, &w2,
+                                       &ybuf_out);
 }
 
 int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUtensorMap& ybuf_out,

@@ -367,8 +367,8 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
     const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
     const float* __restrict__ wg, const float* __restrict__ bg, int32_t* __restrict__ idx,
     float* __restrict__ wout, int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ xperm, int cap,
-    int32_t* __restrict__ lb, int2* __restrict__ tiles, int32_t* __restrict__ meta, int T_,
-    int32_t* err) {
+    int32_t* __restrict__ lb, int2* __restrict__ tiles, int32_t* __restrict__ meta,
+    int32_t* __restrict__ moe_done, int T_, int32_t* err) {
   __shared__ __align__(16) float s_wg[E * D];
   __shared__ int s_chunk, s_e[2 * GR_TOK], s_rank[2 * GR_TOK], s_cnt[E], s_excl[E], s_tot[E];
   __shared__ int s_red[GR_TOK][E];
@@ -488,7 +488,10 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
     int nt_before = 0;
     for (int e = 0; e < E; ++e) {
       const int nt = (s_tot[e] + MOE_BM - 1) / MOE_BM;
-      for (int j = threadIdx.x; j < nt; j += blockDim.x) tiles[nt_before + j] = make_int2(e, e * cap + j * MOE_BM);
+      for (int j = threadIdx.x; j < nt; j += blockDim.x) {
+        tiles[nt_before + j] = make_int2(e, e * cap + j * MOE_BM);
+        moe_done[nt_before + j] = 0;  // the fused expert GEMMs' per-tile counters
+      }
       nt_before += nt;
     }
     if (threadIdx.x == 0) {
@@ -1015,7 +1018,8 @@ int launch_gate_route(const void* x1, const float* g, const float* b, const floa
                wg, bg, reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<float*>(ws + L.wgt),
                reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<__nv_bfloat16*>(ws + L.xperm),
                int(L.cap), reinterpret_cast<int32_t*>(ws + L.lb), reinterpret_cast<int2*>(ws + L.tiles),
-               reinterpret_cast<int32_t*>(ws + L.route_meta), T, reinterpret_cast<int32_t*>(ws + L.err)))
+               reinterpret_cast<int32_t*>(ws + L.route_meta), reinterpret_cast<int32_t*>(ws + L.moe_done), T,
+               reinterpret_cast<int32_t*>(ws + L.err)))
     return -1;
   return PTL_LAUNCH_CHECK();
 }

@@ -30,7 +30,7 @@ inline int launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem
 }
 
 constexpr int QKV_BN = 192;
-constexpr int OUT_BN = 128;
+constexpr int OUT_BN = 256;
 constexpr int MOE1_BN = 256;
 
 // kernels_simt.cu
@@ -74,6 +74,12 @@ int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtenso
                     const float* bias, const void* x, void* x1, int T, int32_t* err, cudaStream_t st);
 int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf_out,
                      const float* b1, const WsLayout& L, char* ws, cudaStream_t st);
+// Both expert GEMMs in one persistent launch (first-GEMM tiles, then
+// second-GEMM tiles, each waiting for its M tile's hidden rows); the
+// workspace's per-M-tile counters (moe_done) must be zero.
+int launch_gemm_moe12(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf,
+                      const CUtensorMap& w2, const CUtensorMap& ybuf_out, const float* b1, const float* b2,
+                      const WsLayout& L, char* ws, cudaStream_t st);
 int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUtensorMap& ybuf_out,
                      const float* b2, const WsLayout& L, char* ws, cudaStream_t st);
 
