@@ -237,7 +237,8 @@ void ptl_set_trace(ptl_trace* trace);
  * allocator, and latency-critical loops that cannot afford cudaMalloc, which
  * may synchronise the whole device.  ptl_attention_noalloc computes what
  * ptl_attention computes (same arguments, no workspace): its only scratch,
- * the device error word and the attention work list, lives in one fixed
+ * the device error word and the attention work list (the (user, query
+ * block) pairs and each attention CTA's unit lists), lives in one fixed
  * array of PTL_NOALLOC_SCRATCH_BYTES bytes in the library's device memory,
  * which every GPU that loads the library holds until the process exits.
  * It allocates nothing and calls no allocating routine.
@@ -257,7 +258,7 @@ void ptl_set_trace(ptl_trace* trace);
  * The pages describe no such entry point; it has no counterpart there. */
 #define PTL_NOALLOC_MAX_TOKENS 65536
 #define PTL_NOALLOC_MAX_USERS 4096
-#define PTL_NOALLOC_SCRATCH_BYTES 49152
+#define PTL_NOALLOC_SCRATCH_BYTES 655360
 ptl_status ptl_attention_noalloc(const void* qkv, void* attn, const int32_t* cu_seqlens,
                                  int32_t num_users, int64_t total_tokens, ptl_dtype dt,
                                  int32_t* device_status, void* stream);

@@ -5,8 +5,10 @@
 // the key loop stops at the diagonal block, so no [S,S] mask is built and no
 // block above the diagonal is touched).  A persistent CTA per SM takes its
 // units in snake order over the grid and splits them between two streams
-// (each unit to the stream with fewer key-block steps so far), one per
-// softmax warpgroup; a stream is a sequence of steps (unit, key block kb).
+// (each unit to the stream with fewer key-block steps so far); the work-list
+// kernel writes each (CTA, stream) list of unit descriptors, so the CTA reads
+// one independent descriptor per unit.  A stream is a sequence of steps
+// (unit, key block kb).
 // The producer and the MMA issuer serve the two streams independently (each
 // polls both and advances whichever is ready), so a stream never waits for
 // the other's softmax:
@@ -61,37 +63,9 @@ struct AttnUnit {
   int s0, L, b, h;
 };
 
-__device__ __forceinline__ AttnUnit attn_unit(const int2* items, const int32_t* cu, int unit) {
-  const int2 it = items[unit >> 3];
-  AttnUnit a;
-  a.s0 = cu[it.x];
-  a.L = cu[it.x + 1] - a.s0;
-  a.b = it.y;
-  a.h = unit & 7;
-  return a;
-}
-
-// Units go to CTAs in snake order over the grid (0..G-1, then G-1..0, ...),
-// so each CTA gets a mix of heavy and light units (the list is heaviest
-// first).  Inside a CTA, each unit in turn goes to the stream (of two) with
-// fewer key-block steps so far; every role of the CTA replays this same
-// deterministic walk, so no assignment is stored or exchanged.
-struct CtaWalker {
-  int k = 0, acc0 = 0, acc1 = 0;
-  // the next unit of stream g, or -1 when the CTA's list is exhausted
-  __device__ int next(const int2* items, int nunits, int g) {
-    const int G = gridDim.x, c = blockIdx.x;
-    for (;;) {
-      const int u = k * G + ((k & 1) ? G - 1 - c : c);
-      if (u >= nunits) return -1;
-      ++k;
-      const int st = items[u >> 3].y + 1;
-      const int to = acc0 <= acc1 ? 0 : 1;
-      if (to == 0) acc0 += st; else acc1 += st;
-      if (to == g) return u;
-    }
-  }
-};
+// One unit of a (CTA, stream) list written by the work-list kernel:
+// (first token of the user, its length, query block, head).
+__device__ __forceinline__ AttnUnit unit_from(const int4 d) { return AttnUnit{d.x, d.y, d.z, d.w}; }
 
 // keys of block kb that exist for this user, rounded up to the MMA's 16
 __device__ __forceinline__ int keys16(int L, int kb) {
@@ -111,7 +85,8 @@ struct StreamPos {
   int kb, n, uc;     // key block of the current unit, steps so far, units started
   bool live, nxt_live;
   AttnUnit u, nxt;   // current unit, the next one (looked up one unit ahead)
-  CtaWalker walk;
+  const int4* list;  // this stream's units, in order
+  int n_list, k_list;  // list length, next entry to read
   // the MMA issuer's queue of steps whose PV is still to be issued (oldest
   // first; -1: none): a step's QK^T may go ahead of the previous step's PV
   int pv_n, pv_k16, pv_uc;
@@ -126,36 +101,36 @@ struct StreamPos {
 // (`a` = stream 0, `b` = stream 1); each role advances a stream when that
 // stream's next step can proceed.
 struct AttnStepGen {
-  int nunits;
-  StreamPos a, b;
-  __device__ void fetch_next(const int2* items, const int32_t* cu, StreamPos& sp) {
-    const int un = sp.walk.next(items, nunits, sp.g);
-    sp.nxt_live = un >= 0;
-    if (sp.nxt_live) sp.nxt = attn_unit(items, cu, un);
+  __device__ void fetch_next(StreamPos& sp) {
+    sp.nxt_live = sp.k_list < sp.n_list;
+    if (sp.nxt_live) sp.nxt = unit_from(sp.list[sp.k_list++]);
   }
-  __device__ void init_stream(const int2* items, const int32_t* cu, StreamPos& sp, int g) {
+  __device__ void init_stream(const int4* ulist, const int32_t* uoff, const int32_t* ucnt, int n_ok,
+                              StreamPos& sp, int g) {
     sp.g = g;
     sp.kb = 0;
     sp.n = 0;
     sp.uc = 0;
-    sp.walk = CtaWalker();
+    sp.list = ulist + uoff[2 * blockIdx.x + g];
+    sp.n_list = n_ok ? ucnt[2 * blockIdx.x + g] : 0;
+    sp.k_list = 0;
     sp.pv_n = sp.pv2_n = -1;
     sp.pv_k16 = sp.pv_uc = sp.pv2_k16 = sp.pv2_uc = 0;
     sp.pv_first = sp.pv2_first = false;
     sp.q_sent = false;
     sp.k_sent = false;
-    fetch_next(items, cu, sp);
+    fetch_next(sp);
     sp.live = sp.nxt_live;
     sp.u = sp.nxt;
-    if (sp.live) fetch_next(items, cu, sp);
+    if (sp.live) fetch_next(sp);
   }
-  __device__ void init(const int2* items, const int32_t* cu, int nunits_) {
-    nunits = nunits_;
-    init_stream(items, cu, a, 0);
-    init_stream(items, cu, b, 1);
+  StreamPos a, b;
+  __device__ void init(const int4* ulist, const int32_t* uoff, const int32_t* ucnt, int n_ok) {
+    init_stream(ulist, uoff, ucnt, n_ok, a, 0);
+    init_stream(ulist, uoff, ucnt, n_ok, b, 1);
   }
   // advances stream `sp` by one step
-  __device__ void step(const int2* items, const int32_t* cu, StreamPos& sp) {
+  __device__ void step(StreamPos& sp) {
     ++sp.n;
     if (++sp.kb > sp.u.b) {
       ++sp.uc;
@@ -163,15 +138,15 @@ struct AttnStepGen {
       sp.q_sent = false;
       sp.live = sp.nxt_live;
       sp.u = sp.nxt;
-      if (sp.live) fetch_next(items, cu, sp);
+      if (sp.live) fetch_next(sp);
     }
   }
 };
 
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int32_t* __restrict__ cu,
-                   const int2* __restrict__ items, const int32_t* __restrict__ item_count,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int4* __restrict__ ulist,
+                   const int32_t* __restrict__ uoff, const int32_t* __restrict__ ucnt,
                    __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -231,9 +206,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   tc_fence_after();
   pdl_wait();  // qkv, the work list and the error word come from earlier kernels
   pdl_trigger();  // dependents launch once this grid has passed its own wait
-  if (threadIdx.x == 0) s_units = has_error(err) ? 0 : (*item_count) * H;
+  if (threadIdx.x == 0) s_units = has_error(err) ? 0 : 1;
   __syncthreads();
-  const int nunits = s_units;
+  const int n_ok = s_units;  // 0: an earlier kernel reported an error, no units
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383,
   // softmax exchange 384..399
@@ -246,7 +221,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
-      gen.init(items, cu, nunits);
+      gen.init(ulist, uoff, ucnt, n_ok);
       // V tiles wait in a small per-stream queue (row of the step's keys,
       // head): V of step n loads once the stream's PV of step n - 1 is done
       int vq0_row[2], vq0_col[2], vq1_row[2], vq1_col[2];  // [queue entry][stream]
@@ -291,7 +266,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           vq1_col[g] = 2 * D + a.h * DH;
         }
         ++vq_len[g];
-        gen.step(items, cu, sp);
+        gen.step(sp);
         return true;
       };
       uint64_t t_prog = globaltimer_ns();
@@ -311,7 +286,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
-      gen.init(items, cu, nunits);
+      gen.init(ulist, uoff, ucnt, n_ok);
       // O[g] += P V for the stream's deferred step; a unit's first PV
       // overwrites O, once warpgroup g has read the previous unit's O
       auto issue_pv = [&](StreamPos& sp) -> bool {
@@ -370,7 +345,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           sp.pv2_first = kb == 0;
           sp.pv2_uc = sp.uc;
         }
-        gen.step(items, cu, sp);
+        gen.step(sp);
         return true;
       };
       // a stream's next QK^T needs no PV of it issued first: the softmax of
@@ -464,13 +439,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       return true;
     };
     int n = 0;  // steps of this stream
-    CtaWalker walk;
-    int unit = walk.next(items, nunits, g);
-    AttnUnit nxt = unit >= 0 ? attn_unit(items, cu, unit) : AttnUnit{0, 0, 0, 0};
-    while (unit >= 0 && ok) {
+    const int4* list = ulist + uoff[2 * blockIdx.x + g];
+    const int n_list = n_ok ? ucnt[2 * blockIdx.x + g] : 0;
+    int k_list = 0;
+    AttnUnit nxt = k_list < n_list ? unit_from(list[k_list]) : AttnUnit{0, 0, 0, 0};
+    while (k_list < n_list && ok) {
       const AttnUnit a = nxt;
-      unit = walk.next(items, nunits, g);
-      if (unit >= 0) nxt = attn_unit(items, cu, unit);  // prefetch the next unit
+      ++k_list;
+      if (k_list < n_list) nxt = unit_from(list[k_list]);  // prefetch the next unit
       const int qi = a.b * ATT_BLK + r;   // query position inside the user
       const int qlim = min(qi, a.L - 1);  // keys 0..qlim are visible
       for (int kb = 0; kb <= a.b; ++kb, ++n) {
@@ -602,17 +578,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   }
 }
 
-static int num_sms_attn() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  }
-  return n;
-}
-
 int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
                    char* ws, cudaStream_t st) {
   static bool configured = false;
@@ -622,10 +587,11 @@ int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, con
       return -1;
     configured = true;
   }
-  const int64_t bound = L.max_items * H;
-  const int grid = int(bound < num_sms_attn() ? bound : num_sms_attn());
-  if (launch_k(attn_tc_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map, cu,
-               reinterpret_cast<const int2*>(ws + L.items), reinterpret_cast<const int32_t*>(ws + L.item_count),
+  // the work-list kernel laid out each CTA's units for this grid
+  const int grid = attn_grid(L.max_items, num_sms());
+  if (launch_k(attn_tc_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map,
+               reinterpret_cast<const int4*>(ws + L.ulist), reinterpret_cast<const int32_t*>(ws + L.uoff),
+               reinterpret_cast<const int32_t*>(ws + L.ucnt),
                static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err)) != 0)
     return -1;
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;

@@ -21,6 +21,7 @@ constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
 constexpr int MOE_BM = 256;        // rows per expert tile (padding granule; one CTA pair's M)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
 constexpr int GR_TOK = 16;         // tokens per block of the fused gate + route kernel
+constexpr int ATT_MAX_CTAS = 1024;  // bound on the persistent attention grid
 constexpr int GEMM2_BN = 256;      // expert GEMM2 output columns per tile
 constexpr float LN_EPS = 1e-5f;
 constexpr float LOGIT_CLAMP = 15.0f;
@@ -33,6 +34,9 @@ struct WsLayout {
   size_t lvl_hist;    // int32 [max_levels + 1]
   size_t lvl_start;   // int32 [max_levels + 1]
   size_t lvl_fill;    // int32 [max_levels + 1]
+  size_t ulist;       // int4 [max_items * 8]  attention units per (CTA, stream): (s0, L, block, head)
+  size_t uoff;        // int32 [2 * ATT_MAX_CTAS]  first entry of each (CTA, stream) list
+  size_t ucnt;        // int32 [2 * ATT_MAX_CTAS]  entries of each (CTA, stream) list
   size_t xn;          // dt [T][512]    LayerNorm1 output
   size_t qkv;         // dt [T][1536]
   size_t attn;        // dt [T][512]
@@ -67,6 +71,15 @@ struct WsLayout {
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// The persistent attention grid: one CTA per SM, at most one per unit (the
+// work-list kernel lays out each CTA's units for exactly this grid).
+__host__ inline int attn_grid(int64_t max_items, int num_sms) {
+  int64_t g = max_items * H;
+  if (g > num_sms) g = num_sms;
+  if (g > ATT_MAX_CTAS) g = ATT_MAX_CTAS;
+  return g < 1 ? 1 : int(g);
+}
+
 __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L) {
   if (T < 0 || T >= (int64_t(1) << 31) || U < 1) return false;
   if (dt != PTL_F32 && dt != PTL_BF16) return false;
@@ -95,6 +108,9 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->lvl_hist = take(4 * (L->max_levels + 1));
   L->lvl_start = take(4 * (L->max_levels + 1));
   L->lvl_fill = take(4 * (L->max_levels + 1));
+  L->ulist = take(16 * L->max_items * H);
+  L->uoff = take(4 * 2 * ATT_MAX_CTAS);
+  L->ucnt = take(4 * 2 * ATT_MAX_CTAS);
   L->wl_end = o;  // error word + attention work list
   L->chunk_cnt = take(4 * L->n_chunks * E);
   L->lb = take(4 * (32 + 32 * L->n_gchunks));

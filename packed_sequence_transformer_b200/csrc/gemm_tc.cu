@@ -436,16 +436,6 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ------------------------------------------------------------------ host
-static int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  }
-  return n;
-}
 
 // Launches the CTA-pair kernel: clusters of two CTAs, one pair per two SMs.
 template <int BN, int MODE>

@@ -146,7 +146,9 @@ __device__ void block_suffix_exclusive(int32_t* a, int n) {
 __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restrict__ cu, int U, int T,
                                                         int2* __restrict__ items, int32_t* item_count,
                                                         int32_t* lvl_hist, int32_t* lvl_start,
-                                                        int32_t* lvl_fill, int max_levels, int32_t* err) {
+                                                        int32_t* lvl_fill, int max_levels, int G,
+                                                        int4* __restrict__ ulist, int32_t* __restrict__ uoff,
+                                                        int32_t* __restrict__ ucnt, int32_t* err) {
   pdl_wait();
   pdl_trigger();
   __shared__ int s_bad;
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
       *item_count = 0;
       set_error(err, PTL_ERR_BAD_OFFSETS);
     }
+    for (int i = tid; i < 2 * G; i += blockDim.x) ucnt[i] = 0;
     return;
   }
   int local = 0;
@@ -193,6 +196,69 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
     }
   }
   if (tid == 0) *item_count = s_total;
+  __syncthreads();
+  // The tensor-core attention's unit lists.  Unit u = 8 * item + head; CTA c
+  // of the G-CTA grid takes units in snake order over the grid (0..G-1, then
+  // G-1..0, ...: a mix of heavy and light units, the list being heaviest
+  // first) and gives each to the stream (of two) with fewer key-block steps
+  // so far.  Each (CTA, stream) list holds (s0, L, block, head) per unit in
+  // order, so the kernel reads one independent descriptor per unit.
+  const int nunits = s_total * H;
+  __shared__ int32_t s_off[2 * ATT_MAX_CTAS];
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int c = tid; c < G; c += blockDim.x) {
+      int acc0 = 0, acc1 = 0, n0 = 0, n1 = 0;
+      for (int k = 0;; ++k) {
+        const int u = k * G + ((k & 1) ? G - 1 - c : c);
+        if (u >= nunits) break;
+        const int2 it = items[u >> 3];
+        const int steps = it.y + 1;
+        const int to = acc0 <= acc1 ? 0 : 1;
+        if (pass == 1) {
+          const int s0 = cu[it.x];
+          ulist[s_off[2 * c + to] + (to == 0 ? n0 : n1)] = make_int4(s0, cu[it.x + 1] - s0, it.y, u & 7);
+        }
+        if (to == 0) {
+          acc0 += steps;
+          ++n0;
+        } else {
+          acc1 += steps;
+          ++n1;
+        }
+      }
+      if (pass == 0) {
+        s_off[2 * c] = n0;
+        s_off[2 * c + 1] = n1;
+        ucnt[2 * c] = n0;
+        ucnt[2 * c + 1] = n1;
+      }
+    }
+    __syncthreads();
+    if (pass == 0) {
+      // exclusive prefix of the 2G list lengths, by warp 0: lane l owns a
+      // contiguous run of entries
+      if (tid < 32) {
+        const int n = 2 * G, per = (n + 31) / 32;
+        const int lo = tid * per, hi = min(n, lo + per);
+        int sum = 0;
+        for (int i = lo; i < hi; ++i) sum += s_off[i];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int i = lo; i < hi; ++i) {
+          const int len = s_off[i];
+          s_off[i] = run;
+          uoff[i] = run;
+          run += len;
+        }
+      }
+      __syncthreads();
+    }
+  }
 }
 
 // ------------------------------------------------------------------ gate
@@ -969,12 +1035,25 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
 // ------------------------------------------------------------- launchers
 #define PTL_LAUNCH_CHECK() (cudaPeekAtLastError() == cudaSuccess ? 0 : -1)
 
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st) {
   if (launch_k(worklist_kernel, dim3(1), dim3(1024), 0, st, cu, U, T, reinterpret_cast<int2*>(ws + L.items),
                                       reinterpret_cast<int32_t*>(ws + L.item_count),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_hist),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_start),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_fill), int(L.max_levels),
+                                      attn_grid(L.max_items, num_sms()), reinterpret_cast<int4*>(ws + L.ulist),
+                                      reinterpret_cast<int32_t*>(ws + L.uoff), reinterpret_cast<int32_t*>(ws + L.ucnt),
                                       reinterpret_cast<int32_t*>(ws + L.err))) return -1;
   return PTL_LAUNCH_CHECK();
 }

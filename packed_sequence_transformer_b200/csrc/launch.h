@@ -34,6 +34,7 @@ constexpr int OUT_BN = 256;
 constexpr int MOE1_BN = 256;
 
 // kernels_simt.cu
+int num_sms();  // of the current device (148 when it cannot be queried)
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st);
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st);
