@@ -54,9 +54,13 @@ constexpr int ATT_TILE_BYTES = ATT_BLK * DH * 2;  // 16 KB
 // K ring stages per stream: a K tile is held until its QK^T is done and the
 // next one must be loaded before the stream's next QK^T can start.
 constexpr int ATT_KV_STAGES = 2;
-// per stream: Q[2] + K[stages] + V[1] + P[2 column blocks]
-constexpr int ATT_SMEM_TILES = 2 * (2 + ATT_KV_STAGES + 1 + 2);
-constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + 1024 + 512;  // + alignment, barriers
+// V buffers per stream: V of step n loads once the PV of step n - 2 is done.
+constexpr int ATT_V_STAGES = 2;
+// per stream: Q[2] + K[stages] + V[stages] (P lives in TMEM)
+constexpr int ATT_SMEM_TILES = 2 * (2 + ATT_KV_STAGES + ATT_V_STAGES);
+// the softmax halves' exchange: [parity][stream][half][row] maxima and sums
+constexpr int ATT_XCHG_BYTES = 2 * (2 * 2 * 2 * 128 * 4);
+constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + ATT_XCHG_BYTES + 1024 + 512;  // + alignment, barriers
 constexpr int ATT_THREADS = 576;  // producer, MMA, four softmax warpgroups (two per stream)
 
 struct AttnUnit {
@@ -153,9 +157,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // per stream: Q[2 units], K[ATT_KV_STAGES steps], V[1 step], P[2 column blocks]
   uint8_t* sQ = smem;                                       // [stream][unit slot]
   uint8_t* sK = sQ + 2 * 2 * ATT_TILE_BYTES;                // [stream][stage]
-  uint8_t* sV = sK + 2 * ATT_KV_STAGES * ATT_TILE_BYTES;    // [stream]
-  uint8_t* sP = sV + 2 * ATT_TILE_BYTES;                    // [stream][column block]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);
+  uint8_t* sV = sK + 2 * ATT_KV_STAGES * ATT_TILE_BYTES;    // [stream][stage]
+  float* s_xm = reinterpret_cast<float*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES);  // [parity][stream][half][row]
+  float* s_xl = s_xm + 2 * 2 * 2 * 128;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATT_SMEM_TILES * ATT_TILE_BYTES + ATT_XCHG_BYTES);
   // Q is double-buffered (the next unit's Q loads while the current unit
   // runs); K is a ring whose slot frees once its QK^T is done; V (needed
   // only by the step's PV, a softmax step later) has one buffer per stream.
@@ -163,9 +168,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* q_empty = bars + 4;                       // [stream][unit slot]
   uint64_t* k_full = bars + 8;                        // [stream][stage]
   uint64_t* k_empty = k_full + 2 * ATT_KV_STAGES;     // [stream][stage]
-  uint64_t* v_full = k_empty + 2 * ATT_KV_STAGES;     // [stream]
-  uint64_t* v_empty = v_full + 2;                     // [stream]
-  uint64_t* s_full = v_empty + 2;                     // [stream]
+  uint64_t* v_full = k_empty + 2 * ATT_KV_STAGES;     // [stream][stage]
+  uint64_t* v_empty = v_full + 2 * ATT_V_STAGES;      // [stream][stage]
+  uint64_t* s_full = v_empty + 2 * ATT_V_STAGES;      // [stream]
   uint64_t* s_empty = s_full + 2;                 // [stream]
   uint64_t* p_full = s_full + 4;                  // [stream]
   uint64_t* pv_done = s_full + 6;                 // [stream]
@@ -180,9 +185,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * ATT_V_STAGES; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 256);
       mbar_init(&p_full[i], 256);
@@ -211,7 +218,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   const int n_ok = s_units;  // 0: an earlier kernel reported an error, no units
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383,
-  // softmax exchange 384..399
+  // P[0] 384..447, P[1] 448..511 (bf16 pairs)
 
   // The producer and the MMA issuer serve the two streams independently:
   // each polls both streams (non-blocking barrier tests: test_wait, which
@@ -230,9 +237,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int g = sp.g;
         bool prog = false;
         // the oldest queued V
-        if (vq_len[g] > 0 && mbar_test_wait(&v_empty[g], (vq_n[g] & 1) ^ 1)) {
-          mbar_arrive_expect_tx(&v_full[g], ATT_TILE_BYTES);
-          tma_load_2d(sV + g * ATT_TILE_BYTES, &tm_qkv, &v_full[g], vq0_col[g], vq0_row[g]);
+        const int vs = g * ATT_V_STAGES + vq_n[g] % ATT_V_STAGES;
+        if (vq_len[g] > 0 && mbar_test_wait(&v_empty[vs], ((vq_n[g] / ATT_V_STAGES) & 1) ^ 1)) {
+          mbar_arrive_expect_tx(&v_full[vs], ATT_TILE_BYTES);
+          tma_load_2d(sV + vs * ATT_TILE_BYTES, &tm_qkv, &v_full[vs], vq0_col[g], vq0_row[g]);
           ++vq_n[g];
           --vq_len[g];
           vq0_row[g] = vq1_row[g];
@@ -294,17 +302,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int gs = sp.g;
         if (!mbar_test_wait(&p_full[gs], nn & 1)) return false;
         if (sp.pv_first && !mbar_test_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
-        if (!mbar_test_wait(&v_full[gs], nn & 1)) return false;
+        const int vs = gs * ATT_V_STAGES + nn % ATT_V_STAGES;
+        if (!mbar_test_wait(&v_full[vs], (nn / ATT_V_STAGES) & 1)) return false;
         tc_fence_after();
-        const uint32_t p0 = smem_u32(sP + gs * 2 * ATT_TILE_BYTES);
-        const uint32_t v0 = smem_u32(sV + gs * ATT_TILE_BYTES);
+        const uint32_t pt = tmem + 384 + 64 * gs;  // P: 128 keys as bf16 pairs, 64 columns
+        const uint32_t v0 = smem_u32(sV + vs * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256 + 64 * gs;
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
-        for (int k = 0; k < sp.pv_k16 / 16; ++k)
-          umma_bf16_ss(d, umma_desc_sw128(p0 + (k >> 2) * ATT_TILE_BYTES + 32 * (k & 3), 1024),
-                       umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv, k != 0 || !sp.pv_first);
+        for (int k = 0; k < sp.pv_k16 / 16; ++k)  // keys 16k..16k+15: P columns 8k..8k+7
+          umma_bf16_ts(d, pt + 8 * k, umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv,
+                       k != 0 || !sp.pv_first);
         umma_commit(&pv_done[gs]);
-        umma_commit(&v_empty[gs]);
+        umma_commit(&v_empty[vs]);
         sp.pv_n = sp.pv2_n;  // pop the queue
         sp.pv_k16 = sp.pv2_k16;
         sp.pv_uc = sp.pv2_uc;
@@ -385,8 +394,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const uint32_t lane_off = uint32_t(32 * wq) << 16;
     const uint32_t tS = tmem + 128 * g + 64 * h + lane_off;       // this half's 64 S columns
     const uint32_t tO = tmem + 256 + 64 * g + 32 * h + lane_off;  // this half's 32 O columns
-    const uint32_t tX = tmem + 384 + 8 * g + lane_off;            // exchange: [half][parity][max, l]
-    auto xcol = [](int hh, int par, int what) { return uint32_t(4 * hh + 2 * par + what); };
+    const uint32_t tP = tmem + 384 + 64 * g + 32 * h + lane_off;  // this half's 32 P columns (64 keys)
+    // exchange slots: [parity][stream][half][row]
+    auto xidx = [&](int par, int hh) { return ((par * 2 + g) * 2 + hh) * 128 + r; };
     const float c2 = 0.125f * 1.4426950408889634f;  // softmax scale * log2(e)
     // Running max m (base 2, scale folded in) of the row and this half's sum l.
     // O lives in TMEM and the PV products accumulate into it; m is raised (and
@@ -482,16 +492,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
         // exchange the halves' maxima (and the previous step's sums)
-        tmem_st1(tX + xcol(h, n & 1, 0), __float_as_uint(mx));
-        tmem_st_wait();
+        s_xm[xidx(n & 1, h)] = mx;
         if (!meet()) { ok = false; break; }
-        uint32_t xo, lo = 0;
-        tmem_ld1(tX + xcol(h ^ 1, n & 1, 0), xo);
-        if (pn >= 0 && plast) tmem_ld1(tX + xcol(h ^ 1, pn & 1, 1), lo);
-        tmem_ld_wait();
-        const float mblk = fmaxf(mx, __uint_as_float(xo)) * c2;
+        const float xo = s_xm[xidx(n & 1, h ^ 1)];
+        const float lo = (pn >= 0 && plast) ? s_xl[xidx(pn & 1, h ^ 1)] : 0.f;
+        const float mblk = fmaxf(mx, xo) * c2;
         // the previous PV must be done before O is touched or P rewritten
-        if (pn >= 0 && !finish_prev(pl + __uint_as_float(lo))) { ok = false; break; }
+        if (pn >= 0 && !finish_prev(pl + lo)) { ok = false; break; }
         if (kb == 0) {
           m = mblk;  // the unit's first PV overwrites O
           l = 0.f;
@@ -508,49 +515,45 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           l *= alpha;
           m = m_new;
         }
-        // pass 2: this half's probabilities -> bf16 P column block h
-        // (K-major, swizzled); masked and skipped columns give p = 0
-        const uint32_t row_addr = smem_u32(sP + g * 2 * ATT_TILE_BYTES + h * ATT_TILE_BYTES) + r * 128;
+        // pass 2: this half's probabilities -> bf16 pairs in TMEM (P columns
+        // 32h..32h+31); masked and skipped keys give p = 0
         if (mine) {
           float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {  // keys 32c..32c+31 of the half: 16-byte chunks 4c..4c+3
+          for (int c = 0; c < 2; ++c) {  // keys 32c..32c+31 of the half: P columns 16c..16c+15
             uint32_t raw[32];
             tmem_ld32(tS + 32 * c, raw);
             tmem_ld_wait();
             const int lc = lim - 32 * c;
             const int lc_eff = lc >= 31 ? 31 : lc;
+            uint32_t pk[16];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int j = 0; j < 8; j += 2) {
-                const int i = 8 * q + j;
-                float p0 = ex2_approx(__uint_as_float(raw[i]) * c2 - m);
-                float p1 = ex2_approx(__uint_as_float(raw[i + 1]) * c2 - m);
-                if (lc < 31) {
-                  p0 = (i <= lc_eff) ? p0 : 0.f;
-                  p1 = (i + 1 <= lc_eff) ? p1 : 0.f;
-                }
-                ls4[j >> 1] += p0 + p1;
-                pk[j >> 1] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 32; i += 2) {
+              float p0 = ex2_approx(__uint_as_float(raw[i]) * c2 - m);
+              float p1 = ex2_approx(__uint_as_float(raw[i + 1]) * c2 - m);
+              if (lc < 31) {
+                p0 = (i <= lc_eff) ? p0 : 0.f;
+                p1 = (i + 1 <= lc_eff) ? p1 : 0.f;
               }
-              const int qc = 4 * c + q;
-              st_shared_v4(row_addr + ((qc ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+              ls4[(i >> 1) & 3] += p0 + p1;
+              pk[i >> 1] = pack_bf16x2(p0, p1);
             }
+            tmem_st16(tP + 16 * c, pk);
           }
           l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
         } else if (2 * h < nch) {
+          uint32_t z[16];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) st_shared_v4(row_addr + ((q ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+          for (int i = 0; i < 16; ++i) z[i] = 0u;
+          tmem_st16(tP, z);
+          tmem_st16(tP + 16, z);
         }
-        // this half's sum so far, for the other half at the unit's end
-        tmem_st1(tX + xcol(h, n & 1, 1), __float_as_uint(l));
         tmem_st_wait();
+        // this half's sum so far, for the other half at the unit's end
+        s_xl[xidx(n & 1, h)] = l;
         // S is read and P written (and O rescaled): the next QK^T and this PV may start
         tc_fence_before();
         mbar_arrive(&s_empty[g]);
-        fence_proxy_async_smem();
         mbar_arrive(&p_full[g]);
         pn = n;
         pl = l;
@@ -560,13 +563,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     if (ok && pn >= 0) {
       // the stream's last unit: the other half's sum, then O / l
-      uint32_t lo = 0;
       ok = meet();
-      if (ok) {
-        tmem_ld1(tX + xcol(h ^ 1, pn & 1, 1), lo);
-        tmem_ld_wait();
-        ok = finish_prev(pl + __uint_as_float(lo));
-      }
+      if (ok) ok = finish_prev(pl + s_xl[xidx(pn & 1, h ^ 1)]);
     }
     if (!ok) set_error(err, PTL_ERR_TIMEOUT);
   }
