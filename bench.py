@@ -37,6 +37,19 @@ sys.path.insert(0, ROOT)
 METRIC = "packed tokens/s per layer fwd (attn+top-2 MoE), 6823 tok/60 users; % TC peak"
 GEMM_FLOPS_PER_TOKEN = 2 * 512 * 1536 + 2 * 512 * 512 + 2 * 512 * 8 + 2 * 2 * (2 * 512 * 1024)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each
+# kernel kind, from one ncu --set full capture of this workload's layer 0
+# (profiles/*_stack8_6823tok.md; ncu flushes caches between replays, so these
+# are cold-cache figures).  A kernel changed since its capture must be
+# recaptured or dropped from this table.
+NCU_DRAM_BYTES = {
+    "gemm_expert1": 31.801856e6 + 3.954432e6,  # both expert GEMMs in one launch
+    "attention": 21.015040e6,
+    "gate": 14.079488e6 + 0.037376e6,          # gate + route builder
+    "gemm_qkv": 8.589312e6,
+    "gemm_out": 14.527488e6,
+    "combine": 28.068096e6 + 0.002048e6,
+}
 
 
 def parse():
@@ -360,7 +373,7 @@ def run_ours(args):
         peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         unit = "GB/s"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": None, "kernel": dom,
+                "frac": achieved / peak, "traffic": NCU_DRAM_BYTES.get(dom), "kernel": dom,
                 "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs'})",
                 "algorithmic_per_launch": work}
     step_flops = n_layers * (GEMM_FLOPS_PER_TOKEN * T + attn_fl)

@@ -20,21 +20,23 @@
 //               2-deep ring (a slot frees when its QK^T is done) and the V
 //               tile into the stream's single V buffer (freed by the
 //               previous step's PV);
-//   warp 1      MMA issuer: for a step of stream g, S = Q K^T (M=128, N = the
-//               keys of this block rounded up to 16) into TMEM S[g], and --
-//               once warpgroup g has written P for that step -- O[g] += P V
-//               (M=128, N=64, K = its key count; V is the MN-major operand)
-//               into TMEM; a unit's first PV overwrites O;
-//   warps 2..5  softmax warpgroup 0, warps 6..9 warpgroup 1: thread r owns
-//               query row r (TMEM lane r) of its stream's unit; per step it
-//               reads its S row, masks keys past its position and past the
-//               user, keeps the running max m and sum l in fp32 (base-2,
-//               scale folded in) and writes P = exp2(s - m) as bf16 into the
-//               K-major swizzled layout the tensor core reads.  m is raised
-//               lazily (only when a block's max exceeds it by 2^8), and then
-//               the row of O in TMEM is rescaled in place.  Before writing P
-//               it waits for the previous PV (the stream's P buffer is
-//               single); at the end of a unit it stores O / l in bf16.
+//   warps 1, 2  MMA issuers, one per stream: per step S = Q K^T (M=128, N =
+//               the keys of this block rounded up to 16) into TMEM S[g], then
+//               the previous step's O[g] += P V (M=128, N=64, K = its key
+//               count; P is read from TMEM, V is the MN-major operand); a
+//               unit's first PV overwrites O;
+//   warps 3..18 softmax, four warpgroups, two per stream: thread r owns query
+//               row r (TMEM lane r) of its stream's unit and half of the
+//               block's 128 keys; per step it reads its half of the S row,
+//               masks keys past its position and past the user, combines the
+//               row maximum with the other half (shared memory + mbarrier),
+//               keeps the running max m and its half's sum l in fp32 (base-2,
+//               scale folded in) and writes P = exp2(s - m) as bf16 pairs into
+//               TMEM.  m is raised lazily (only when a block's max exceeds it
+//               by 2^8), and then its half of the O row in TMEM is rescaled in
+//               place.  Before writing P it waits for the previous PV (the
+//               stream's P buffer is single); at the end of a unit it stores
+//               its half of O / l in bf16.
 // Fully masked 32-key chunks of the diagonal block are skipped (their P is
 // written as zeros); rows past the user end are computed but not stored; TMA
 // zero-fills rows past T.  Every wait is bounded.
@@ -61,7 +63,7 @@ constexpr int ATT_SMEM_TILES = 2 * (2 + ATT_KV_STAGES + ATT_V_STAGES);
 // the softmax halves' exchange: [parity][stream][half][row] maxima and sums
 constexpr int ATT_XCHG_BYTES = 2 * (2 * 2 * 2 * 128 * 4);
 constexpr int ATT_SMEM = ATT_SMEM_TILES * ATT_TILE_BYTES + ATT_XCHG_BYTES + 1024 + 512;  // + alignment, barriers
-constexpr int ATT_THREADS = 576;  // producer, MMA, four softmax warpgroups (two per stream)
+constexpr int ATT_THREADS = 608;  // producer, two MMA issuers, four softmax warpgroups (two per stream)
 
 struct AttnUnit {
   int s0, L, b, h;
@@ -291,46 +293,49 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // MMA issuer of stream g = warp - 1 (one thread; the two streams' issuers
+    // run independently): per step n, S(n) = Q K^T, then the previous step's
+    // O += P V (a unit's first PV overwrites O, once warpgroup g has read the
+    // previous unit's O).  The PV of step n - 1 is ready when S(n) can start
+    // (both wait for the end of softmax step n - 1).
     if (lane == 0) {
-      AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
-      gen.init(ulist, uoff, ucnt, n_ok);
-      // O[g] += P V for the stream's deferred step; a unit's first PV
-      // overwrites O, once warpgroup g has read the previous unit's O
-      auto issue_pv = [&](StreamPos& sp) -> bool {
-        const int nn = sp.pv_n;
-        const int gs = sp.g;
-        if (!mbar_test_wait(&p_full[gs], nn & 1)) return false;
-        if (sp.pv_first && !mbar_test_wait(&pv_empty[gs], (sp.pv_uc & 1) ^ 1)) return false;
-        const int vs = gs * ATT_V_STAGES + nn % ATT_V_STAGES;
-        if (!mbar_test_wait(&v_full[vs], (nn / ATT_V_STAGES) & 1)) return false;
+      const int g = warp - 1;
+      AttnStepGen gen;
+      StreamPos& sp = g == 0 ? gen.a : gen.b;
+      gen.init_stream(ulist, uoff, ucnt, n_ok, sp, g);
+      bool ok = true;
+      int pvn = -1, pvk16 = 0, pvuc = 0;
+      bool pvfirst = false;
+      auto issue_pv = [&]() -> bool {
+        if (pvn < 0) return true;
+        if (!mbar_wait(&p_full[g], pvn & 1)) return false;
+        if (pvfirst && !mbar_wait(&pv_empty[g], (pvuc & 1) ^ 1)) return false;
+        const int vs = g * ATT_V_STAGES + pvn % ATT_V_STAGES;
+        if (!mbar_wait(&v_full[vs], (pvn / ATT_V_STAGES) & 1)) return false;
         tc_fence_after();
-        const uint32_t pt = tmem + 384 + 64 * gs;  // P: 128 keys as bf16 pairs, 64 columns
+        const uint32_t pt = tmem + 384 + 64 * g;  // P: 128 keys as bf16 pairs, 64 columns
         const uint32_t v0 = smem_u32(sV + vs * ATT_TILE_BYTES);
-        const uint32_t d = tmem + 256 + 64 * gs;
+        const uint32_t d = tmem + 256 + 64 * g;
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
-        for (int k = 0; k < sp.pv_k16 / 16; ++k)  // keys 16k..16k+15: P columns 8k..8k+7
+        for (int k = 0; k < pvk16 / 16; ++k)  // keys 16k..16k+15: P columns 8k..8k+7
           umma_bf16_ts(d, pt + 8 * k, umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv,
-                       k != 0 || !sp.pv_first);
-        umma_commit(&pv_done[gs]);
+                       k != 0 || !pvfirst);
+        umma_commit(&pv_done[g]);
         umma_commit(&v_empty[vs]);
-        sp.pv_n = sp.pv2_n;  // pop the queue
-        sp.pv_k16 = sp.pv2_k16;
-        sp.pv_uc = sp.pv2_uc;
-        sp.pv_first = sp.pv2_first;
-        sp.pv2_n = -1;
+        pvn = -1;
         return true;
       };
-      // S = Q K^T for the stream's next step; queues the step's PV
-      auto issue_s = [&](StreamPos& sp) -> bool {
-        const int g = sp.g;
+      while (ok && sp.live) {
         const AttnUnit a = sp.u;
         const int kb = sp.kb, nn = sp.n;
         const int st = nn % ATT_KV_STAGES, use = nn / ATT_KV_STAGES;
         const int qs = sp.uc & 1;
-        if (kb == 0 && !mbar_test_wait(&q_full[2 * g + qs], (sp.uc >> 1) & 1)) return false;
-        if (!mbar_test_wait(&k_full[g * ATT_KV_STAGES + st], use & 1)) return false;
-        if (!mbar_test_wait(&s_empty[g], (nn & 1) ^ 1)) return false;
+        if ((kb == 0 && !mbar_wait(&q_full[2 * g + qs], (sp.uc >> 1) & 1)) ||
+            !mbar_wait(&k_full[g * ATT_KV_STAGES + st], use & 1) || !mbar_wait(&s_empty[g], (nn & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const int k16 = keys16(a.L, kb);
         const uint32_t q0 = smem_u32(sQ + (2 * g + qs) * ATT_TILE_BYTES);
@@ -343,51 +348,27 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         umma_commit(&s_full[g]);
         umma_commit(&k_empty[g * ATT_KV_STAGES + st]);
         if (kb == a.b) umma_commit(&q_empty[2 * g + qs]);
-        if (sp.pv_n < 0) {
-          sp.pv_n = nn;
-          sp.pv_k16 = k16;
-          sp.pv_first = kb == 0;
-          sp.pv_uc = sp.uc;
-        } else {
-          sp.pv2_n = nn;
-          sp.pv2_k16 = k16;
-          sp.pv2_first = kb == 0;
-          sp.pv2_uc = sp.uc;
-        }
-        gen.step(sp);
-        return true;
-      };
-      // a stream's next QK^T needs no PV of it issued first: the softmax of
-      // that step waits for the previous PV before it writes P, so at most
-      // two PVs are ever queued
-      auto serve = [&](StreamPos& sp) -> bool {
-        bool prog = false;
-        if (sp.pv_n >= 0 && issue_pv(sp)) prog = true;
-        if (sp.pv2_n < 0 && sp.live && issue_s(sp)) prog = true;
-        return prog;
-      };
-      uint64_t t_prog = globaltimer_ns();
-      while (gen.a.live || gen.a.pv_n >= 0 || gen.b.live || gen.b.pv_n >= 0) {
-        bool prog = serve(gen.a);
-        prog |= serve(gen.b);
-        if (prog) {
-          t_prog = globaltimer_ns();
-        } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
-          set_error(err, PTL_ERR_TIMEOUT);
+        if (!issue_pv()) {
+          ok = false;
           break;
-        } else {
-          __nanosleep(20);  // leave issue slots to the softmax warps while idle
         }
+        pvn = nn;
+        pvk16 = k16;
+        pvfirst = kb == 0;
+        pvuc = sp.uc;
+        gen.step(sp);
       }
+      if (ok) ok = issue_pv();
+      if (!ok) set_error(err, PTL_ERR_TIMEOUT);
     }
   } else {
     // Softmax: four warpgroups, two per stream.  Warpgroup (g, h) (warps
-    // 2 + 8g + 4h .. +3) handles keys 64h .. 64h + 63 of every S row of stream
+    // 3 + 8g + 4h .. +3) handles keys 64h .. 64h + 63 of every S row of stream
     // g, column block h of P and columns 32h .. 32h + 31 of O; thread r <->
     // query row r <-> TMEM lane r.  The two halves of a row combine their
     // maxima (every step) and their sums (at a unit's end) through spare TMEM
     // columns, synchronised by a per-stream mbarrier (bounded waits).
-    const int sw = (warp - 2) >> 2;
+    const int sw = (warp - 3) >> 2;
     const int g = sw >> 1, h = sw & 1;
     const int wq = warp & 3;
     const int r = 32 * wq + lane;
