@@ -118,15 +118,6 @@ __device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile
   }
 }
 
-// Release / acquire on a GPU-scope counter (MOE12 tile dependencies).
-__device__ __forceinline__ void red_release_gpu_add(int32_t* p, int32_t v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int32_t ld_acquire_gpu_s32(const int32_t* p) {
-  int32_t v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
@@ -220,17 +211,11 @@ __global__ void __launch_bounds__(192, 1)
         if (MODE == G_MOE12 && second) {
           // the tile's A rows (H) come from every first-GEMM tile of this M
           // tile, each stored by both CTAs of its pair
-          const int need = 2 * (p.N_total / BN);
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_gpu_s32(p.done + mt) < need) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-              set_error(p.err, PTL_ERR_TIMEOUT);
-              ok = false;
-              break;
-            }
-            __nanosleep(64);
+          if (!wait_flag_at_least(p.done + mt, 2 * (p.N_total / BN))) {
+            set_error(p.err, PTL_ERR_TIMEOUT);
+            ok = false;
+            break;
           }
-          if (!ok) break;
           fence_proxy_async_global();  // the H rows were written by TMA stores
         }
         for (int kb = 0; kb < nkb; ++kb, ++it) {

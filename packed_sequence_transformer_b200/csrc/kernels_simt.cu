@@ -404,15 +404,6 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
   }
 }
 
-// Flag store / load with release / acquire semantics at GPU scope.
-__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
-  int32_t v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
 // ------------------------------------------------------- gate + route
 // The layer path's gate and route builder in one kernel (bf16 build).  A
@@ -491,21 +482,13 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
     __threadfence();
   }
   __syncthreads();
-  if (threadIdx.x == 0) st_release_gpu(me, 1);
+  if (threadIdx.x == 0) sm100::st_release_gpu(me, 1);
   int part[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) part[e] = 0;
   for (int pc = threadIdx.x; pc < c; pc += blockDim.x) {
     const int32_t* pf = lb + 32 + 32 * pc;
-    int f = ld_acquire_gpu(pf);
-    if (f == 0) {
-      const uint64_t t0 = sm100::globaltimer_ns();
-      while ((f = ld_acquire_gpu(pf)) == 0) {
-        if (sm100::globaltimer_ns() - t0 > sm100::kWaitLimitNs) break;
-        __nanosleep(64);
-      }
-    }
-    if (f == 0) {
+    if (!sm100::wait_flag_at_least(pf, 1)) {
       set_error(err, PTL_ERR_TIMEOUT);
       break;
     }
@@ -1191,6 +1174,35 @@ int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLay
   if (launch_k(attn_f32_kernel, dim3(unsigned(L.max_items * H)), dim3(128), 0, st, 
       qkv, out, cu, reinterpret_cast<const int2*>(ws + L.items),
       reinterpret_cast<const int32_t*>(ws + L.item_count), reinterpret_cast<const int32_t*>(ws + L.err))) return -1;
+  return PTL_LAUNCH_CHECK();
+}
+
+// ------------------------------------------------------- wait self-test
+// Waits on something that never happens, with the same bounded waits the
+// layer's kernels use on their producers, so that the give-up path itself can
+// be run: which == 0 waits on an mbarrier phase that no thread completes,
+// which == 1 on a global flag (zeroed by the caller) that nothing raises.
+// Each of the 32 threads gives up after limit_ns and the kernel records
+// PTL_ERR_TIMEOUT in the error word; the context stays usable.
+__global__ void __launch_bounds__(32) wait_selftest_kernel(int32_t* err, const int32_t* flag,
+                                                           int which, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = which == 0 ? sm100::mbar_wait(&bar, 0, limit_ns)
+                             : sm100::wait_flag_at_least(flag, 1, limit_ns);
+  if (!ok) set_error(err, PTL_ERR_TIMEOUT);
+}
+
+int launch_wait_selftest(int32_t* err, const int32_t* flag, int which, uint64_t limit_ns,
+                         cudaStream_t st) {
+  if (launch_k(wait_selftest_kernel, dim3(1), dim3(32), 0, st, err, flag, which,
+               static_cast<unsigned long long>(limit_ns))) return -1;
   return PTL_LAUNCH_CHECK();
 }
 

@@ -35,6 +35,9 @@ constexpr int MOE1_BN = 256;
 
 // kernels_simt.cu
 int num_sms();  // of the current device (148 when it cannot be queried)
+// A kernel whose bounded wait runs out (which: 0 mbarrier, 1 global flag).
+int launch_wait_selftest(int32_t* err, const int32_t* flag, int which, uint64_t limit_ns,
+                         cudaStream_t st);
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st);
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st);
