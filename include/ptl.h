@@ -263,6 +263,79 @@ ptl_status ptl_attention_noalloc(const void* qkv, void* attn, const int32_t* cu_
                                  int32_t num_users, int64_t total_tokens, ptl_dtype dt,
                                  int32_t* device_status, void* stream);
 
+/* ---- The stack as one CUDA graph per token bucket. ----
+ * Serving issues the stack batch after batch with a different packing each
+ * time.  Issued kernel by kernel that loop is bound by launch overhead
+ * (README, CUDA Graph section: about 211 launches per batch); the remedy
+ * there is to pad every batch to a bucket of the token count (512-token
+ * steps), capture one graph per bucket lazily or ahead of time over static
+ * buffers, pad a short batch's user offsets on the GPU with zero-length
+ * users, and never synchronise the host.  A runner does that:
+ *   - ptl_runner_create allocates, once, a workspace and static input /
+ *     output buffers for batches of up to max_tokens tokens and max_users
+ *     users (device memory of the current device; the only allocation).
+ *     `layers` (num_layers entries) and `head` (nullable) are copied by value;
+ *     the device weights they point to must outlive the runner.  stride is
+ *     the bucket granule in tokens, a multiple of 128 (0 = PTL_RUNNER_STRIDE).
+ *   - ptl_runner_forward computes what ptl_stack_forward computes for the
+ *     batch (x [T][512] of the runner's dtype, cu_seqlens [U+1] int32,
+ *     pred_mask [T] uint8) with T rounded up to the bucket Tb: it copies the
+ *     inputs into the
+ *     static buffers (x, cu_seqlens and pred_mask may be host or device
+ *     pointers; host memory should be pinned for the copies to be
+ *     asynchronous), zero-fills the padding tokens, appends padding users of
+ *     at most 128 tokens over T .. Tb and zero-length users up to the
+ *     runner's fixed user count (ptl_runner_bucket), launches the bucket's
+ *     graph and copies out[T][512] (nullable when there is a head),
+ *     probs[0 .. T-1] (entries past *n_pred undefined) and *n_pred (nullable)
+ *     to host or device memory.  Real rows equal those of a direct
+ *     ptl_stack_forward call on the unpadded batch bit for bit (users are
+ *     independent, every other step is per token).  The first batch of a
+ *     bucket captures and instantiates its graph (host work, no device
+ *     synchronisation; ptl_runner_capture does it ahead of time).  All
+ *     work is enqueued on `stream`; a runner's calls must be ordered on one
+ *     stream (its buffers are reused by the next batch).  T == 0 returns
+ *     PTL_OK without work; T > max_tokens, U > max_users or a call from
+ *     another device return PTL_ERR_SHAPE.  Malformed offsets (including
+ *     cu_seqlens[U] != T) are reported by ptl_runner_last_device_error as
+ *     PTL_ERR_BAD_OFFSETS.
+ *   - ptl_runner_destroy frees everything (cudaFree waits for the device).
+ * ptl_runner_bucket is host arithmetic only: the bucket of a token count and
+ * the runner's padded user count. */
+#define PTL_RUNNER_STRIDE 512
+typedef struct ptl_stack_runner ptl_stack_runner;
+ptl_status ptl_runner_bucket(int64_t total_tokens, int32_t max_users, int32_t stride,
+                             int64_t* bucket, int32_t* padded_users);
+ptl_status ptl_runner_create(int64_t max_tokens, int32_t max_users, int32_t num_layers, ptl_dtype dt,
+                             const ptl_layer_weights* layers, const ptl_head_weights* head,
+                             int32_t stride, ptl_stack_runner** runner);
+ptl_status ptl_runner_capture(ptl_stack_runner* runner, int64_t total_tokens);
+ptl_status ptl_runner_forward(ptl_stack_runner* runner, const void* x, void* out,
+                              const int32_t* cu_seqlens, int32_t num_users, int64_t total_tokens,
+                              const uint8_t* pred_mask, float* probs, int32_t* n_pred, void* stream);
+/* Synchronises `stream`, returns and clears the runner's device error word. */
+ptl_status ptl_runner_last_device_error(ptl_stack_runner* runner, void* stream);
+/* Number of buckets whose graph has been captured (-1 for NULL). */
+int32_t ptl_runner_graphs(const ptl_stack_runner* runner);
+void ptl_runner_destroy(ptl_stack_runner* runner);
+
+/* ---- Failure detection self-test. ----
+ * Every wait inside the library's kernels (on an mbarrier phase, or on a
+ * counter that another CTA of the same launch raises) is bounded: after a
+ * limit without progress the waiting thread records PTL_ERR_TIMEOUT in the
+ * workspace error word and its kernel unwinds, leaving the context usable.
+ * ptl_wait_selftest launches one 32-thread kernel that runs those same waits
+ * on something that never happens -- which = 0: an mbarrier phase that no
+ * thread completes; which = 1: a flag in the workspace's error block that is
+ * zeroed first and that nothing raises -- so that the give-up path can be run
+ * on purpose.  limit_ns (1e3 .. 1e9) replaces the library's one-second limit.
+ * Asynchronous on `stream`; afterwards ptl_last_device_error() reports
+ * PTL_ERR_TIMEOUT.  Returns PTL_ERR_SHAPE for another `which` or a limit
+ * outside the range, and the usual NULL / alignment / size statuses for the
+ * workspace (at least 256 bytes). */
+ptl_status ptl_wait_selftest(void* workspace, size_t ws_bytes, int32_t which, int64_t limit_ns,
+                             void* stream);
+
 /* Synchronises `stream`, returns the status recorded in the workspace error
  * word by earlier calls on that workspace (PTL_OK if none) and clears it. */
 ptl_status ptl_last_device_error(void* workspace, size_t ws_bytes, void* stream);

@@ -551,6 +551,22 @@ ptl_status ptl_head(const void* h, const ptl_head_weights* head, const uint8_t* 
   return PTL_OK;
 }
 
+ptl_status ptl_wait_selftest(void* workspace, size_t ws_bytes, int32_t which, int64_t limit_ns,
+                             void* stream) {
+  if (!workspace) return PTL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PTL_ERR_ALIGN;
+  if (ws_bytes < 256) return PTL_ERR_WORKSPACE;
+  if ((which != 0 && which != 1) || limit_ns < 1000 || limit_ns > 1000000000) return PTL_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  // the flag lives in the error block's spare bytes; nothing else writes it
+  int32_t* flag = reinterpret_cast<int32_t*>(ws + 128);
+  if (cudaMemsetAsync(flag, 0, sizeof(int32_t), st) != cudaSuccess) return PTL_ERR_CUDA;
+  if (launch_wait_selftest(reinterpret_cast<int32_t*>(ws), flag, which, uint64_t(limit_ns), st) != 0)
+    return PTL_ERR_CUDA;
+  return PTL_OK;
+}
+
 ptl_status ptl_last_device_error(void* workspace, size_t ws_bytes, void* stream) {
   if (!workspace) return PTL_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PTL_ERR_ALIGN;

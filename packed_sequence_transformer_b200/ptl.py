@@ -97,7 +97,22 @@ _SIGS = {
                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                   ctypes.c_void_p], ctypes.c_int),
     "ptl_last_device_error": ([ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
+    "ptl_wait_selftest": ([ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64,
+                           ctypes.c_void_p], ctypes.c_int),
     "ptl_set_trace": ([ctypes.POINTER(Trace)], None),
+    "ptl_runner_bucket": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                           ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32)],
+                          ctypes.c_int),
+    "ptl_runner_create": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int,
+                           ctypes.POINTER(LayerWeights), ctypes.POINTER(HeadWeights), ctypes.c_int32,
+                           ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+    "ptl_runner_capture": ([ctypes.c_void_p, ctypes.c_int64], ctypes.c_int),
+    "ptl_runner_forward": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                            ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                            ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "ptl_runner_last_device_error": ([ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "ptl_runner_graphs": ([ctypes.c_void_p], ctypes.c_int32),
+    "ptl_runner_destroy": ([ctypes.c_void_p], None),
     "ptl_attention_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
                               ctypes.c_int),
@@ -304,6 +319,68 @@ def attention_noalloc(qkv, attn, cu_seqlens, device_status=None, stream=None):
 def last_device_error(workspace, stream=None) -> int:
     """Synchronises the stream and returns (and clears) the device error word."""
     return int(lib().ptl_last_device_error(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def runner_bucket(total_tokens: int, max_users: int, stride: int = 0):
+    """(bucket tokens, padded user count) a runner uses for a batch of
+    ``total_tokens`` (host arithmetic only)."""
+    b, u = ctypes.c_int64(), ctypes.c_int32()
+    _check(lib().ptl_runner_bucket(int(total_tokens), int(max_users), int(stride), ctypes.byref(b),
+                                   ctypes.byref(u)), "ptl_runner_bucket")
+    return b.value, u.value
+
+
+class StackRunner:
+    """The layer stack (and optional head) as one CUDA graph per token
+    bucket (``ptl_runner_*``): inputs and outputs may be host (ideally
+    pinned) or device tensors; calls must be ordered on one stream."""
+
+    def __init__(self, max_tokens: int, max_users: int, layers: List[Dict], dtype, head=None,
+                 stride: int = 0):
+        self._keep = (layers, head)  # the device weights must outlive the runner
+        arr = (LayerWeights * len(layers))(*[layer_struct(w) for w in layers])
+        hs = head_struct(head) if head is not None else None
+        r = ctypes.c_void_p()
+        _check(lib().ptl_runner_create(int(max_tokens), int(max_users), len(layers), _dt(dtype), arr,
+                                       ctypes.byref(hs) if hs is not None else None, int(stride),
+                                       ctypes.byref(r)), "ptl_runner_create")
+        self._r = r
+        self.has_head = head is not None
+
+    def capture(self, total_tokens: int) -> None:
+        _check(lib().ptl_runner_capture(self._r, int(total_tokens)), "ptl_runner_capture")
+
+    def forward(self, x, cu_seqlens, out=None, pred_mask=None, probs=None, n_pred=None,
+                stream=None):
+        _check(lib().ptl_runner_forward(self._r, _ptr(x), _ptr(out), _ptr(cu_seqlens),
+                                        cu_seqlens.numel() - 1, x.shape[0], _ptr(pred_mask),
+                                        _ptr(probs), _ptr(n_pred), _stream(stream)),
+               "ptl_runner_forward")
+        return out
+
+    def last_device_error(self, stream=None) -> int:
+        return int(lib().ptl_runner_last_device_error(self._r, _stream(stream)))
+
+    def graphs(self) -> int:
+        return int(lib().ptl_runner_graphs(self._r))
+
+    def close(self) -> None:
+        if getattr(self, "_r", None):
+            lib().ptl_runner_destroy(self._r)
+            self._r = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def wait_selftest(workspace, which: int, limit_ns: int, stream=None) -> None:
+    """Launches a kernel whose bounded wait (0: mbarrier, 1: global flag) runs
+    out after ``limit_ns``; ``last_device_error`` then reports PTL_ERR_TIMEOUT."""
+    _check(lib().ptl_wait_selftest(_ptr(workspace), workspace.numel(), int(which), int(limit_ns),
+                                   _stream(stream)), "ptl_wait_selftest")
 
 
 class KernelTrace:

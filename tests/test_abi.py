@@ -108,3 +108,43 @@ def test_step_entry_points_validate(P):
     assert L.ptl_stack_forward(FAKE, FAKE + 4096, FAKE, 4, 64, 0, 1, arr, None, None, None, None,
                                FAKE, ws_b, None) == S["PTL_ERR_SHAPE"]
     assert L.ptl_last_device_error(None, 0, None) == S["PTL_ERR_NULL"]
+
+
+def test_wait_selftest_host_checks(P):
+    L = P.lib()
+    S = P.STATUS_CODE
+    assert L.ptl_wait_selftest(None, 256, 0, 10**6, None) == S["PTL_ERR_NULL"]
+    assert L.ptl_wait_selftest(FAKE + 16, 256, 0, 10**6, None) == S["PTL_ERR_ALIGN"]
+    assert L.ptl_wait_selftest(FAKE, 128, 0, 10**6, None) == S["PTL_ERR_WORKSPACE"]
+    assert L.ptl_wait_selftest(FAKE, 256, 2, 10**6, None) == S["PTL_ERR_SHAPE"]
+    assert L.ptl_wait_selftest(FAKE, 256, 1, 10, None) == S["PTL_ERR_SHAPE"]
+    assert L.ptl_wait_selftest(FAKE, 256, 1, 2 * 10**9, None) == S["PTL_ERR_SHAPE"]
+
+
+def test_runner_bucket_and_host_checks(P):
+    L = P.lib()
+    S = P.STATUS_CODE
+    # 512-token buckets; padding users of <= 128 tokens: ceil(511 / 128) = 4 extra users
+    assert P.runner_bucket(6823, 60) == (7168, 64)
+    assert P.runner_bucket(7168, 60) == (7168, 64)
+    assert P.runner_bucket(1, 1) == (512, 5)
+    assert P.runner_bucket(0, 1) == (0, 5)
+    assert P.runner_bucket(129, 3, 128) == (256, 4)
+    assert P.runner_bucket(1000, 3, 1024) == (1024, 11)
+    b, u = ctypes.c_int64(), ctypes.c_int32()
+    for bad in [(100, 4, 96), (100, 0, 0), (-1, 4, 0), (2**31 - 1, 4, 0)]:
+        assert L.ptl_runner_bucket(*bad, ctypes.byref(b), ctypes.byref(u)) == S["PTL_ERR_SHAPE"]
+    assert L.ptl_runner_bucket(100, 4, 0, None, ctypes.byref(u)) == S["PTL_ERR_NULL"]
+    w = _w(P)
+    arr = (P.LayerWeights * 1)(w)
+    r = ctypes.c_void_p()
+    assert L.ptl_runner_create(1000, 4, 1, 1, arr, None, 0, None) == S["PTL_ERR_NULL"]
+    assert L.ptl_runner_create(1000, 4, 1, 7, arr, None, 0, ctypes.byref(r)) == S["PTL_ERR_DTYPE"]
+    assert L.ptl_runner_create(1000, 4, 0, 1, arr, None, 0, ctypes.byref(r)) == S["PTL_ERR_SHAPE"]
+    assert L.ptl_runner_create(1000, 4, 1, 1, arr, None, 100, ctypes.byref(r)) == S["PTL_ERR_SHAPE"]
+    assert r.value is None
+    assert L.ptl_runner_forward(None, FAKE, FAKE, FAKE, 1, 10, None, None, None, None) == S["PTL_ERR_NULL"]
+    assert L.ptl_runner_capture(None, 10) == S["PTL_ERR_NULL"]
+    assert L.ptl_runner_last_device_error(None, None) == S["PTL_ERR_NULL"]
+    assert L.ptl_runner_graphs(None) == -1
+    L.ptl_runner_destroy(None)
