@@ -19,6 +19,9 @@ Sources (web pages, cited by title and section):
     token_id*top_k + k_idx, per-token weighted sum) and the Prediction Head
     section (Linear(512->1) -> clamp(-15, 15) -> sigmoid, pred_mask select).
   * "CTI-Inference-Opt" optimisation plan -- attention as softmax(QK^T/sqrt(d))V.
+  * "cry-daniel/recsys" README -- the HSTU attention mask logic (contextual,
+    historical and candidate segments; mask types none, local, causal,
+    context + causal, target + causal), for the masked-attention variants.
   * "CTI-Inference-Opt" AUC-recovery plan -- the dense block-diagonal causal
     mask built from user_offsets (same user AND lower triangle), the
     FlexAttention mask_mod restatement of it, and the vectorised SMoE that
@@ -168,6 +171,75 @@ def dense_masked_attention(q, k, v, cu_seqlens, scale=None):
         S = q[:, h, :] @ k[:, h, :].T * scale
         S = np.where(mask, S, -np.inf)
         out[:, h, :] = _softmax_rows(S) @ v[:, h, :]
+    return out
+
+
+# --------------------------------------------------------------------------
+# HSTU-style attention masks (cry-daniel/recsys README: HSTU attention mask
+# logic and the attention function's mask types).  Not on the encoder layer's
+# path; a second workload for the same jagged attention.
+# --------------------------------------------------------------------------
+def hstu_user_mask(L, causal=True, num_contexts=0, num_targets=0, target_group_size=1, window=0):
+    """[L, L] boolean visibility for one user's sequence laid out as
+    [contextual tokens][historical tokens][candidate tokens].
+
+    Readings of the README's segment picture (it gives no formulas):
+      * base: key j is visible to query i when j <= i (causal), or always
+        (causal=False, the 'no mask' type);
+      * contextual tokens (the first C = num_contexts) attend to one another
+        in both directions;
+      * candidate tokens (the last N = num_targets, starting at Hs = L - N)
+        form groups of target_group_size in order; a candidate sees every
+        non-candidate token and the candidates of its own group (subject to
+        the base rule), never another group; non-candidates never see a
+        candidate;
+      * the local (sliding-window) type: with window W > 0 only keys with
+        |i - j| < W are visible.
+    Every query sees itself."""
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    vis = (j <= i) if causal else np.ones((L, L), dtype=bool)
+    C = int(num_contexts)
+    if C > 0:
+        vis = vis | ((i < C) & (j < C))
+    N = int(num_targets)
+    if N > 0:
+        Hs = L - N
+        G = int(target_group_size)
+        cand_i, cand_j = i >= Hs, j >= Hs
+        same_group = ((i - Hs) // G) == ((j - Hs) // G)
+        vis = vis & ~(cand_j & ~cand_i)            # non-candidates never see candidates
+        vis = vis & ~(cand_i & cand_j & ~same_group)  # candidates see only their own group
+    if window > 0:
+        vis = vis & (np.abs(i - j) < window)
+    return vis
+
+
+def jagged_hstu_attention(q, k, v, cu_seqlens, causal=True, num_contexts=None, num_targets=None,
+                          target_group_size=1, window=0, scale=None):
+    """softmax(Q K^T * scale) V per user and head under hstu_user_mask.
+    num_contexts / num_targets: per-user counts ([U]) or None (all zero)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, H, Dh = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dh)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    U = len(cu) - 1
+    ctx = np.zeros(U, np.int64) if num_contexts is None else np.asarray(num_contexts, np.int64)
+    tgt = np.zeros(U, np.int64) if num_targets is None else np.asarray(num_targets, np.int64)
+    out = np.zeros_like(q)
+    for u in range(U):
+        s, e = int(cu[u]), int(cu[u + 1])
+        L = e - s
+        if L <= 0:
+            continue
+        if not (0 <= ctx[u] and 0 <= tgt[u] and ctx[u] + tgt[u] <= L):
+            raise ValueError(f"user {u}: contexts + targets exceed its length")
+        vis = hstu_user_mask(L, causal, ctx[u], tgt[u], target_group_size, window)
+        for h in range(H):
+            S = q[s:e, h, :] @ k[s:e, h, :].T * scale
+            S = np.where(vis, S, -np.inf)
+            out[s:e, h, :] = _softmax_rows(S) @ v[s:e, h, :]
     return out
 
 

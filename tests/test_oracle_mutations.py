@@ -110,3 +110,38 @@ def test_dropped_expert_bias_is_caught(monkeypatch):
 def test_missing_logit_clamp_is_caught(monkeypatch):
     monkeypatch.setattr(O, "LOGIT_CLAMP", 1e9)
     assert _fails(P.test_head_clamp_and_sigmoid_values)
+
+
+# ------------------------------------------------- HSTU-style masks
+import tests.test_oracle_hstu as PH  # noqa: E402
+
+
+def _mask_mutant(monkeypatch, edit):
+    orig = O.hstu_user_mask
+
+    def mutant(L, causal=True, num_contexts=0, num_targets=0, target_group_size=1, window=0):
+        return edit(orig, L, causal, int(num_contexts), int(num_targets), int(target_group_size),
+                    int(window))
+    monkeypatch.setattr(O, "hstu_user_mask", mutant)
+
+
+def test_context_rule_dropped_is_caught(monkeypatch):
+    _mask_mutant(monkeypatch, lambda f, L, c, C, N, G, W: f(L, c, 0, N, G, W))
+    assert _fails(PH.test_context_rows_are_bidirectional_over_the_context_only)
+
+
+def test_candidate_groups_off_by_one_is_caught(monkeypatch):
+    _mask_mutant(monkeypatch, lambda f, L, c, C, N, G, W: f(L, c, C, N, G + 1, W))
+    assert _fails(PH.test_candidate_groups)
+
+
+def test_candidates_leaking_into_history_is_caught(monkeypatch):
+    # candidates visible to every later row, as with a plain causal mask
+    _mask_mutant(monkeypatch, lambda f, L, c, C, N, G, W: f(L, c, C, 0, G, W))
+    assert _fails(PH.test_single_candidates_see_history_and_themselves)
+
+
+def test_window_off_by_one_is_caught(monkeypatch):
+    _mask_mutant(monkeypatch, lambda f, L, c, C, N, G, W: f(L, c, C, N, G, W + 1 if W > 0 else 0))
+    assert _fails(PH.test_window_one_gives_own_v_and_wide_window_is_causal)
+    assert _fails(lambda: PH.test_window_rows_see_their_neighbourhood(True))
