@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 METRIC = "packed tokens/s per layer fwd (attn+top-2 MoE), 6823 tok/60 users; % TC peak"
 GEMM_FLOPS_PER_TOKEN = 2 * 512 * 1536 + 2 * 512 * 512 + 2 * 512 * 8 + 2 * 2 * (2 * 512 * 1024)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+RUNNER_STRIDE = 128  # token granule of the graph runner's buckets in the end-to-end leg
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each
 # kernel kind, from one ncu --set full capture of this workload's layer 0
 # (profiles/*_stack8_6823tok.md; ncu flushes caches between replays, so these
@@ -379,7 +380,10 @@ def run_ours(args):
     step_flops = n_layers * (GEMM_FLOPS_PER_TOKEN * T + attn_fl)
     whole_step_tflops = step_flops / (ms_max / 1e3) / 1e12
 
-    # ---- end to end through the public API: host (pinned) inputs in, result out
+    # ---- end to end through the public API: the bucketed graph runner with
+    # host (pinned) buffers; each step copies the batch in, replays the
+    # bucket's graph and copies the result (head probabilities + count, or
+    # the hidden rows) out
     x_h = torch.as_tensor(case.x).to(torch.bfloat16).pin_memory()
     cu_h = torch.as_tensor(case.cu_seqlens).to(torch.int32).pin_memory()
     mask_h = torch.as_tensor(case.pred_mask).to(torch.uint8).pin_memory() if head is not None else None
@@ -388,27 +392,45 @@ def run_ours(args):
     n_h = torch.zeros(1, dtype=torch.int32).pin_memory()
     h2d = x_h.numel() * 2 + cu_h.numel() * 4 + (mask_h.numel() if mask_h is not None else 0)
     d2h = res_h.numel() * res_h.element_size() + (4 if head is not None else 0)
-    e2e_ms = []
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup + args.steps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            x.copy_(x_h, non_blocking=True)
-            cu.copy_(cu_h, non_blocking=True)
-            if mask is not None:
-                mask.copy_(mask_h, non_blocking=True)
-            graph.replay()
-            if head is not None:
-                res_h.copy_(probs, non_blocking=True)
-                n_h.copy_(n_pred, non_blocking=True)
-            else:
-                res_h.copy_(out, non_blocking=True)
-            b.record(stream)
-            b.synchronize()
-            if i >= args.warmup:
-                e2e_ms.append(a.elapsed_time(b))
-            flush.fill_(float(i))
-    e2e_value = job_value(T, n_layers, world, max_over_ranks(statistics.mean(e2e_ms), world, dev))
+    # 128-token buckets: a serving process holds one small graph per bucket,
+    # and the finer stride keeps the padding work to under 128 tokens
+    runner = ptl.StackRunner(T, U, layers, "bf16", head=head, stride=RUNNER_STRIDE)
+    bucket = ptl.runner_bucket(T, U, RUNNER_STRIDE)[0]
+    runner.capture(T)
+
+    def run_runner(src_x, src_cu, src_mask, dst, dst_n):
+        if head is not None:
+            runner.forward(src_x, src_cu, pred_mask=src_mask, probs=dst, n_pred=dst_n, stream=stream)
+        else:
+            runner.forward(src_x, src_cu, out=dst, stream=stream)
+
+    def timed(fn, n_warm, n_timed, host_sync):
+        ms = []
+        with torch.cuda.stream(stream):
+            for i in range(n_warm + n_timed):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                if host_sync:
+                    b.synchronize()
+                if i >= n_warm:
+                    ms.append((a, b))
+                flush.fill_(float(i))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ms)
+
+    e2e_ms = timed(lambda: run_runner(x_h, cu_h, mask_h, res_h, n_h), args.warmup, args.steps, True)
+    st = runner.last_device_error(stream)
+    if st != 0:
+        raise RuntimeError(f"device error {ptl.STATUS.get(st)} in the runner")
+    e2e_value = job_value(T, n_layers, world, max_over_ranks(e2e_ms, world, dev))
+    # the same runner on device-resident buffers (device copies + graph), and
+    # the stack issued kernel by kernel from the host without a graph
+    res_d = probs if head is not None else torch.empty_like(out)
+    runner_ms = timed(lambda: run_runner(x, cu, mask, res_d, n_pred), 2, args.steps, False)
+    eager_ms = timed(step, 2, args.steps, False)
+    runner.close()
 
     cpu = None
     if rank == 0 and world == 1:
@@ -438,6 +460,9 @@ def run_ours(args):
             "detail": {"step_tflops": whole_step_tflops,
                        "step_frac_of_peak": whole_step_tflops / float(peaks.get("bf16_tflops", 1590.0)),
                        "us_per_layer": ms_max * 1e3 / n_layers,
+                       "runner": {"stride": RUNNER_STRIDE, "bucket_tokens": bucket, "device_buffers_ms_per_step": runner_ms,
+                                  "host_buffers_ms_per_step": e2e_ms},
+                       "eager_ms_per_step": eager_ms,
                        "kernels": kinds, "attention_flops_per_layer": attn_fl,
                        "gemm_flops_per_layer": GEMM_FLOPS_PER_TOKEN * T},
         }

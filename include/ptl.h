@@ -80,7 +80,8 @@ typedef enum {
   PTL_ERR_DTYPE = 6,       /* unknown ptl_dtype */
   PTL_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed */
   PTL_ERR_TIMEOUT = 8,     /* a bounded device-side wait ran out (kernel returned early) */
-  PTL_ERR_UNSUPPORTED = 9  /* no sm_100 device, or a feature not built */
+  PTL_ERR_UNSUPPORTED = 9, /* no sm_100 device, or a feature not built */
+  PTL_ERR_BAD_MASK = 10    /* attention mask out of range (ptl_attention_masked) */
 } ptl_status;
 
 typedef enum { PTL_F32 = 0, PTL_BF16 = 1 } ptl_dtype;
@@ -193,6 +194,38 @@ ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w
 ptl_status ptl_head(const void* h, const ptl_head_weights* head, const uint8_t* pred_mask,
                     float* probs, int32_t* n_pred, int64_t total_tokens, ptl_dtype dt,
                     void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- HSTU-style attention masks over the same jagged layout. ----
+ * The cry-daniel/recsys README (HSTU attention mask logic) lays a user's
+ * sequence out as [contextual tokens][historical tokens][candidate tokens]:
+ * contextual tokens (user profile) attend to one another in both
+ * directions, history is causal, candidates are grouped by
+ * target_group_size; its attention function also offers no mask and a local
+ * (sliding-window) mask.  For the user with L tokens, C = num_contexts[u]
+ * and N = num_targets[u] (candidates from Hs = L - N), key j is visible to
+ * query i when
+ *   (causal ? j <= i : 1)  or  (i < C and j < C),
+ *   and, if j >= Hs: i >= Hs and (i - Hs) / G == (j - Hs) / G,
+ *   and, if window > 0: |i - j| < window.
+ * Every query sees itself.  ptl_attention_masked computes softmax(Q K^T / 8) V
+ * per user and head over the visible keys, reading Q/K/V from qkv[T][1536]
+ * like ptl_attention; with causal = 1 and no contexts, candidates or window
+ * it equals ptl_attention.  num_contexts / num_targets: device int32 [U],
+ * NULL = all zero.  Host checks: target_group_size >= 1 and causal 0 or 1
+ * (else PTL_ERR_BAD_MASK), plus the usual ones; on the device, a user with
+ * C < 0, N < 0 or C + N > L sets PTL_ERR_BAD_MASK in the workspace error
+ * word (the attention then computes nothing). */
+typedef struct {
+  int32_t causal;             /* 1: causal base rule; 0: every key of the user (no mask) */
+  const int32_t* num_contexts; /* device [U] or NULL */
+  const int32_t* num_targets;  /* device [U] or NULL */
+  int32_t target_group_size;  /* candidates per group, >= 1 */
+  int32_t window;             /* > 0: sliding window |i - j| < window; <= 0: none */
+} ptl_attn_mask;
+ptl_status ptl_attention_masked(const void* qkv, void* attn, const int32_t* cu_seqlens,
+                                int32_t num_users, int64_t total_tokens, ptl_dtype dt,
+                                const ptl_attn_mask* mask, void* workspace, size_t ws_bytes,
+                                void* stream);
 
 /* ---- Per-kernel tracing (for profiling; off by default). ----
  * While a trace is installed on the calling host thread, every entry point

@@ -191,16 +191,17 @@ ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_wei
   return PTL_OK;
 }
 
-ptl_status step_attention(const Call& c, const void* qkv, void* attn, const int32_t* cu) {
+ptl_status step_attention(const Call& c, const void* qkv, void* attn, const int32_t* cu,
+                          const AttnMask* mask = nullptr) {
   if (c.dt == PTL_BF16) {
     CUtensorMap m;
     if (!map_bf16(&m, qkv, QKV_N, c.T, QKV_N * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_ATTENTION);
-    PTL_TRY(launch_attn_tc(m, attn, cu, c.L, c.ws, c.st));
+    PTL_TRY(launch_attn_tc(m, attn, cu, c.L, c.ws, c.st, mask));
   } else {
     mark(c.st, PTL_KERNEL_ATTENTION);
     PTL_TRY(launch_attn_f32(static_cast<const float*>(qkv), static_cast<float*>(attn), cu, c.L, c.ws,
-                            c.st));
+                            c.st, mask));
   }
   return PTL_OK;
 }
@@ -362,6 +363,7 @@ const char* ptl_status_string(ptl_status s) {
     case PTL_ERR_DTYPE: return "unknown dtype";
     case PTL_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case PTL_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case PTL_ERR_BAD_MASK: return "attention mask: target_group_size < 1, causal not 0/1, or a user's contextual + candidate counts outside 0 .. its length";
     case PTL_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
   }
   return "unknown status";
@@ -462,6 +464,30 @@ ptl_status ptl_attention(const void* qkv, void* attn, const int32_t* cu_seqlens,
   mark(c.st, PTL_KERNEL_WORKLIST);
   PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
   return step_attention(c, qkv, attn, cu_seqlens);
+}
+
+ptl_status ptl_attention_masked(const void* qkv, void* attn, const int32_t* cu_seqlens,
+                                int32_t num_users, int64_t total_tokens, ptl_dtype dt,
+                                const ptl_attn_mask* mask, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  Call c;
+  ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
+  if (s != PTL_OK) return s;
+  if (!mask) return PTL_ERR_NULL;
+  if (mask->target_group_size < 1 || (mask->causal != 0 && mask->causal != 1)) return PTL_ERR_BAD_MASK;
+  if (total_tokens == 0) return PTL_OK;
+  if (!qkv || !attn || !cu_seqlens) return PTL_ERR_NULL;
+  if (!a16(qkv) || !a16(attn) || !a4(cu_seqlens) || (mask->num_contexts && !a4(mask->num_contexts)) ||
+      (mask->num_targets && !a4(mask->num_targets)))
+    return PTL_ERR_ALIGN;
+  if ((s = device_ok()) != PTL_OK) return s;
+  if ((s = begin(c)) != PTL_OK) return s;
+  const AttnMask m{mask->num_contexts, mask->num_targets, mask->causal, mask->target_group_size,
+                   mask->window};
+  EndMark end_mark{c.st};
+  mark(c.st, PTL_KERNEL_WORKLIST);
+  PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st, &m));
+  return step_attention(c, qkv, attn, cu_seqlens, &m);
 }
 
 ptl_status ptl_out_projection(const void* attn, const void* x, void* x1, int64_t total_tokens,

@@ -67,11 +67,33 @@ constexpr int ATT_THREADS = 608;  // producer, two MMA issuers, four softmax war
 
 struct AttnUnit {
   int s0, L, b, h;
+  int lo, hi;  // first and last key block the unit walks
+  int C, Hs;   // masked variant: contextual tokens, first candidate (0 and L otherwise)
 };
 
-// One unit of a (CTA, stream) list written by the work-list kernel:
-// (first token of the user, its length, query block, head).
-__device__ __forceinline__ AttnUnit unit_from(const int4 d) { return AttnUnit{d.x, d.y, d.z, d.w}; }
+// One unit of a (CTA, stream) list written by the work-list kernel: (first
+// token of the user, its length, query block, head); with a mask, (first
+// token, length, block | head << 24, user), the user's contextual and
+// candidate counts read from the mask and the key blocks derived from them.
+template <bool MASKED>
+__device__ __forceinline__ AttnUnit unit_from(const int4 d, const AttnMask& mk) {
+  if constexpr (!MASKED) {
+    return AttnUnit{d.x, d.y, d.z, d.w, 0, d.z, 0, d.y};
+  } else {
+    AttnUnit a;
+    a.s0 = d.x;
+    a.L = d.y;
+    a.b = d.z & 0xFFFFFF;
+    a.h = d.z >> 24;
+    a.C = mk.ctx ? mk.ctx[d.w] : 0;
+    a.Hs = a.L - (mk.tgt ? mk.tgt[d.w] : 0);
+    int lo_key, hi_key;
+    mask_key_range(a.b, a.L, a.C, a.Hs, mk, lo_key, hi_key);
+    a.lo = lo_key / ATT_BLK;
+    a.hi = hi_key / ATT_BLK;
+    return a;
+  }
+}
 
 // keys of block kb that exist for this user, rounded up to the MMA's 16
 __device__ __forceinline__ int keys16(int L, int kb) {
@@ -106,15 +128,17 @@ struct StreamPos {
 // Both streams' step sequences as the producer and the MMA issuer walk them
 // (`a` = stream 0, `b` = stream 1); each role advances a stream when that
 // stream's next step can proceed.
+template <bool MASKED>
 struct AttnStepGen {
+  const AttnMask& mk;
+  __device__ explicit AttnStepGen(const AttnMask& m) : mk(m) {}
   __device__ void fetch_next(StreamPos& sp) {
     sp.nxt_live = sp.k_list < sp.n_list;
-    if (sp.nxt_live) sp.nxt = unit_from(sp.list[sp.k_list++]);
+    if (sp.nxt_live) sp.nxt = unit_from<MASKED>(sp.list[sp.k_list++], mk);
   }
   __device__ void init_stream(const int4* ulist, const int32_t* uoff, const int32_t* ucnt, int n_ok,
                               StreamPos& sp, int g) {
     sp.g = g;
-    sp.kb = 0;
     sp.n = 0;
     sp.uc = 0;
     sp.list = ulist + uoff[2 * blockIdx.x + g];
@@ -128,6 +152,7 @@ struct AttnStepGen {
     fetch_next(sp);
     sp.live = sp.nxt_live;
     sp.u = sp.nxt;
+    sp.kb = sp.u.lo;
     if (sp.live) fetch_next(sp);
   }
   StreamPos a, b;
@@ -138,22 +163,25 @@ struct AttnStepGen {
   // advances stream `sp` by one step
   __device__ void step(StreamPos& sp) {
     ++sp.n;
-    if (++sp.kb > sp.u.b) {
+    if (++sp.kb > sp.u.hi) {
       ++sp.uc;
-      sp.kb = 0;
       sp.q_sent = false;
       sp.live = sp.nxt_live;
       sp.u = sp.nxt;
+      sp.kb = sp.u.lo;
       if (sp.live) fetch_next(sp);
     }
   }
 };
 
 
+// MASKED: the HSTU-style variant (key blocks and visibility from the mask);
+// otherwise block-diagonal causal.
+template <bool MASKED>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int4* __restrict__ ulist,
                    const int32_t* __restrict__ uoff, const int32_t* __restrict__ ucnt,
-                   __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err) {
+                   __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err, const AttnMask mask) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // per stream: Q[2 units], K[ATT_KV_STAGES steps], V[1 step], P[2 column blocks]
@@ -229,7 +257,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // They give up (PTL_ERR_TIMEOUT) after a second without progress.
   if (warp == 0) {
     if (lane == 0) {
-      AttnStepGen gen;  // a = stream 0, b = stream 1 (never swapped here)
+      AttnStepGen<MASKED> gen(mask);  // a = stream 0, b = stream 1 (never swapped here)
       gen.init(ulist, uoff, ucnt, n_ok);
       // V tiles wait in a small per-stream queue (row of the step's keys,
       // head): V of step n loads once the stream's PV of step n - 1 is done
@@ -252,7 +280,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (!sp.live || vq_len[g] == 2) return prog;
         const AttnUnit a = sp.u;
         const int qs = sp.uc & 1;  // the unit's Q slot
-        if (sp.kb == 0 && !sp.q_sent) {  // a new unit of stream g: its Q tile
+        if (sp.kb == a.lo && !sp.q_sent) {  // a new unit of stream g: its Q tile
           if (!mbar_test_wait(&q_empty[2 * g + qs], ((sp.uc >> 1) & 1) ^ 1)) return prog;
           mbar_arrive_expect_tx(&q_full[2 * g + qs], ATT_TILE_BYTES);
           tma_load_2d(sQ + (2 * g + qs) * ATT_TILE_BYTES, &tm_qkv, &q_full[2 * g + qs], a.h * DH,
@@ -301,7 +329,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // (both wait for the end of softmax step n - 1).
     if (lane == 0) {
       const int g = warp - 1;
-      AttnStepGen gen;
+      AttnStepGen<MASKED> gen(mask);
       StreamPos& sp = g == 0 ? gen.a : gen.b;
       gen.init_stream(ulist, uoff, ucnt, n_ok, sp, g);
       bool ok = true;
@@ -331,7 +359,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int kb = sp.kb, nn = sp.n;
         const int st = nn % ATT_KV_STAGES, use = nn / ATT_KV_STAGES;
         const int qs = sp.uc & 1;
-        if ((kb == 0 && !mbar_wait(&q_full[2 * g + qs], (sp.uc >> 1) & 1)) ||
+        if ((kb == a.lo && !mbar_wait(&q_full[2 * g + qs], (sp.uc >> 1) & 1)) ||
             !mbar_wait(&k_full[g * ATT_KV_STAGES + st], use & 1) || !mbar_wait(&s_empty[g], (nn & 1) ^ 1)) {
           ok = false;
           break;
@@ -347,14 +375,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                        idesc_qk, k != 0);
         umma_commit(&s_full[g]);
         umma_commit(&k_empty[g * ATT_KV_STAGES + st]);
-        if (kb == a.b) umma_commit(&q_empty[2 * g + qs]);
+        if (kb == a.hi) umma_commit(&q_empty[2 * g + qs]);
         if (!issue_pv()) {
           ok = false;
           break;
         }
         pvn = nn;
         pvk16 = k16;
-        pvfirst = kb == 0;
+        pvfirst = kb == a.lo;
         pvuc = sp.uc;
         gen.step(sp);
       }
@@ -433,14 +461,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int4* list = ulist + uoff[2 * blockIdx.x + g];
     const int n_list = n_ok ? ucnt[2 * blockIdx.x + g] : 0;
     int k_list = 0;
-    AttnUnit nxt = k_list < n_list ? unit_from(list[k_list]) : AttnUnit{0, 0, 0, 0};
+    AttnUnit nxt = k_list < n_list ? unit_from<MASKED>(list[k_list], mask) : AttnUnit{0, 0, 0, 0, 0, 0, 0, 0};
     while (k_list < n_list && ok) {
       const AttnUnit a = nxt;
       ++k_list;
-      if (k_list < n_list) nxt = unit_from(list[k_list]);  // prefetch the next unit
+      if (k_list < n_list) nxt = unit_from<MASKED>(list[k_list], mask);  // prefetch the next unit
       const int qi = a.b * ATT_BLK + r;   // query position inside the user
       const int qlim = min(qi, a.L - 1);  // keys 0..qlim are visible
-      for (int kb = 0; kb <= a.b; ++kb, ++n) {
+      for (int kb = a.lo; kb <= a.hi; ++kb, ++n) {
         if (!mbar_wait(&s_full[g], n & 1)) { ok = false; break; }
         tc_fence_after();
         const int k16 = keys16(a.L, kb);
@@ -449,11 +477,25 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // and on the diagonal block only chunks not wholly above the warp's
         // rows; this half owns chunks 2h and 2h + 1 (keys past qlim masked)
         const int nch = (k16 + 31) >> 5;
-        const int nuse = (kb == a.b) ? min(nch, wq + 1) : nch;
+        const int nuse = (!MASKED && kb == a.b) ? min(nch, wq + 1) : nch;
         const bool mine = 2 * h < nuse;
         const int lim = qlim - (kbase + 64 * h);  // this half's keys i <= lim are visible
         // pass 1: this half's row maximum over the visible keys
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // masked variant: visibility of this half's 64 keys, one bit per key
+        uint32_t vbits[2] = {0u, 0u};
+        if constexpr (MASKED) {
+          if (mine) {
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+              uint32_t bits = 0u;
+              const int j0 = kbase + 64 * h + 32 * c;
+              for (int i = 0; i < 32; ++i)
+                if (j0 + i < a.L && mask_visible(qi, j0 + i, a.C, a.Hs, mask)) bits |= 1u << i;
+              vbits[c] = bits;
+            }
+          }
+        }
         if (mine) {
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {  // 32 columns per TMEM load
@@ -461,7 +503,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             tmem_ld32(tS + 32 * c, raw);
             tmem_ld_wait();
             const int lc = lim - 32 * c;
-            if (lc >= 31) {
+            if constexpr (MASKED) {
+              const uint32_t bits = vbits[c];
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if ((bits >> i) & 1u) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
+            } else if (lc >= 31) {
 #pragma unroll
               for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
             } else {
@@ -480,12 +527,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const float mblk = fmaxf(mx, xo) * c2;
         // the previous PV must be done before O is touched or P rewritten
         if (pn >= 0 && !finish_prev(pl + lo)) { ok = false; break; }
-        if (kb == 0) {
+        if (kb == a.lo) {
           m = mblk;  // the unit's first PV overwrites O
           l = 0.f;
         } else if (__any_sync(0xffffffffu, mblk > m + RESCALE_LOG2)) {
           const float m_new = fmaxf(m, mblk);
-          const float alpha = ex2_approx(m - m_new);
+          // masked variant: a row may have seen no visible key yet (m = -inf)
+          const float alpha = (MASKED && m_new == -INFINITY) ? 1.f : ex2_approx(m - m_new);
           uint32_t o[32];
           tmem_ld32(tO, o);
           tmem_ld_wait();
@@ -512,7 +560,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             for (int i = 0; i < 32; i += 2) {
               float p0 = ex2_approx(__uint_as_float(raw[i]) * c2 - m);
               float p1 = ex2_approx(__uint_as_float(raw[i + 1]) * c2 - m);
-              if (lc < 31) {
+              if constexpr (MASKED) {
+                p0 = ((vbits[c] >> i) & 1u) ? p0 : 0.f;
+                p1 = ((vbits[c] >> (i + 1)) & 1u) ? p1 : 0.f;
+              } else if (lc < 31) {
                 p0 = (i <= lc_eff) ? p0 : 0.f;
                 p1 = (i + 1 <= lc_eff) ? p1 : 0.f;
               }
@@ -538,7 +589,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         mbar_arrive(&p_full[g]);
         pn = n;
         pl = l;
-        plast = kb == a.b;
+        plast = kb == a.hi;
         pdst = qi < a.L ? (a.s0 + qi) * D + a.h * DH : -1;
       }
     }
@@ -557,23 +608,31 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   }
 }
 
-int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
-                   char* ws, cudaStream_t st) {
+template <bool MASKED>
+static int launch_attn_tc_t(const CUtensorMap& qkv_map, void* out, const WsLayout& L, char* ws,
+                            cudaStream_t st, const AttnMask& mask) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_tc_kernel<MASKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ATT_SMEM) != cudaSuccess)
       return -1;
     configured = true;
   }
   // the work-list kernel laid out each CTA's units for this grid
   const int grid = attn_grid(L.max_items, num_sms());
-  if (launch_k(attn_tc_kernel, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map,
+  if (launch_k(attn_tc_kernel<MASKED>, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map,
                reinterpret_cast<const int4*>(ws + L.ulist), reinterpret_cast<const int32_t*>(ws + L.uoff),
                reinterpret_cast<const int32_t*>(ws + L.ucnt),
-               static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err)) != 0)
+               static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err), mask) != 0)
     return -1;
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
+                   char* ws, cudaStream_t st, const AttnMask* mask) {
+  (void)cu;
+  if (mask) return launch_attn_tc_t<true>(qkv_map, out, L, ws, st, *mask);
+  return launch_attn_tc_t<false>(qkv_map, out, L, ws, st, AttnMask{nullptr, nullptr, 1, 1, 0});
 }
 
 }  // namespace ptl

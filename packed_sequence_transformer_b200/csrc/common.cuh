@@ -138,6 +138,50 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   return true;
 }
 
+// ---------------------------------------------------------------- masks
+// HSTU-style attention masks (cry-daniel/recsys README, HSTU attention mask
+// logic).  A user's L tokens are laid out [contextual][historical][candidate]:
+// the first C are contextual, the candidates start at Hs = L - N.  Key j is
+// visible to query i (positions inside the user, j < L) when
+//   - causal ? j <= i : always, or both are contextual (i < C and j < C);
+//   - and, for a candidate key (j >= Hs), i is a candidate of the same group
+//     (groups of `group` candidates counted from Hs);
+//   - and, with window > 0, |i - j| < window.
+// Every query sees itself, so no row of a valid batch is fully masked.
+struct AttnMask {
+  const int32_t* ctx;  // [U] contextual tokens per user, or nullptr (none)
+  const int32_t* tgt;  // [U] candidate tokens per user, or nullptr (none)
+  int32_t causal;      // 1: causal base rule; 0: every key of the user
+  int32_t group;       // candidates per group (>= 1)
+  int32_t window;      // > 0: sliding window; <= 0: none
+};
+
+__device__ __forceinline__ bool mask_visible(int i, int j, int C, int Hs, const AttnMask& m) {
+  bool v = m.causal ? j <= i : true;
+  v = v || (i < C && j < C);
+  if (j >= Hs) v = v && i >= Hs && (i - Hs) / m.group == (j - Hs) / m.group;
+  if (m.window > 0) v = v && (i > j ? i - j : j - i) < m.window;
+  return v;
+}
+
+// Keys [lo_key, hi_key] that hold every key visible to some query of block b
+// (queries q0 .. q1 of the user): the range the key loop walks.
+__device__ __forceinline__ void mask_key_range(int b, int L, int C, int Hs, const AttnMask& m,
+                                               int& lo_key, int& hi_key) {
+  const int q0 = b * ATT_BLK;
+  const int q1 = q0 + ATT_BLK - 1 < L - 1 ? q0 + ATT_BLK - 1 : L - 1;
+  int hi = m.causal ? q1 : L - 1;
+  if (q0 < C && C - 1 > hi) hi = C - 1;    // contextual rows see the whole context
+  if (q1 < Hs && Hs - 1 < hi) hi = Hs - 1;  // no candidate row: no candidate key
+  int lo = 0;
+  if (m.window > 0) {
+    lo = q0 - m.window + 1 > 0 ? q0 - m.window + 1 : 0;
+    if (q1 + m.window - 1 < hi) hi = q1 + m.window - 1;
+  }
+  lo_key = lo;
+  hi_key = hi;
+}
+
 // ---------------------------------------------------------------- device
 // Programmatic dependent launch.  Every kernel of the library is launched so
 // that the next kernel in the stream may start its prologue while this one

@@ -148,7 +148,8 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
                                                         int32_t* lvl_hist, int32_t* lvl_start,
                                                         int32_t* lvl_fill, int max_levels, int G,
                                                         int4* __restrict__ ulist, int32_t* __restrict__ uoff,
-                                                        int32_t* __restrict__ ucnt, int32_t* err) {
+                                                        int32_t* __restrict__ ucnt, int32_t* err,
+                                                        const AttnMask mask, const int masked) {
   pdl_wait();
   pdl_trigger();
   __shared__ int s_bad;
@@ -166,10 +167,18 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
   for (int u = tid; u < U; u += blockDim.x)
     if (cu[u + 1] < cu[u]) s_bad = 1;
   __syncthreads();
+  if (!s_bad && masked) {
+    // contextual and candidate counts must fit in their user
+    for (int u = tid; u < U; u += blockDim.x) {
+      const int C = mask.ctx ? mask.ctx[u] : 0, N = mask.tgt ? mask.tgt[u] : 0;
+      if (C < 0 || N < 0 || int64_t(C) + N > int64_t(cu[u + 1]) - cu[u]) s_bad = 2;
+    }
+    __syncthreads();
+  }
   if (s_bad) {
     if (tid == 0) {
       *item_count = 0;
-      set_error(err, PTL_ERR_BAD_OFFSETS);
+      set_error(err, s_bad == 2 ? PTL_ERR_BAD_MASK : PTL_ERR_BAD_OFFSETS);
     }
     for (int i = tid; i < 2 * G; i += blockDim.x) ucnt[i] = 0;
     return;
@@ -202,7 +211,9 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
   // G-1..0, ...: a mix of heavy and light units, the list being heaviest
   // first) and gives each to the stream (of two) with fewer key-block steps
   // so far.  Each (CTA, stream) list holds (s0, L, block, head) per unit in
-  // order, so the kernel reads one independent descriptor per unit.
+  // order, so the kernel reads one independent descriptor per unit; with a
+  // mask, (s0, L, block | head << 24, user) and a unit's steps are the key
+  // blocks its mask leaves to walk.
   const int nunits = s_total * H;
   __shared__ int32_t s_off[2 * ATT_MAX_CTAS];
   for (int pass = 0; pass < 2; ++pass) {
@@ -212,11 +223,21 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restric
         const int u = k * G + ((k & 1) ? G - 1 - c : c);
         if (u >= nunits) break;
         const int2 it = items[u >> 3];
-        const int steps = it.y + 1;
+        int steps = it.y + 1;
+        if (masked) {
+          const int Lu = cu[it.x + 1] - cu[it.x];
+          const int C = mask.ctx ? mask.ctx[it.x] : 0;
+          const int Hs = Lu - (mask.tgt ? mask.tgt[it.x] : 0);
+          int lo_key, hi_key;
+          mask_key_range(it.y, Lu, C, Hs, mask, lo_key, hi_key);
+          steps = hi_key / ATT_BLK - lo_key / ATT_BLK + 1;
+        }
         const int to = acc0 <= acc1 ? 0 : 1;
         if (pass == 1) {
           const int s0 = cu[it.x];
-          ulist[s_off[2 * c + to] + (to == 0 ? n0 : n1)] = make_int4(s0, cu[it.x + 1] - s0, it.y, u & 7);
+          ulist[s_off[2 * c + to] + (to == 0 ? n0 : n1)] =
+              masked ? make_int4(s0, cu[it.x + 1] - s0, it.y | ((u & 7) << 24), it.x)
+                     : make_int4(s0, cu[it.x + 1] - s0, it.y, u & 7);
         }
         if (to == 0) {
           acc0 += steps;
@@ -960,12 +981,15 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const float* __restric
 // threads per (user, query block, head) work item; thread i owns query row
 // i of the block and runs an fp32 online softmax over the user's keys
 // 0..q, staged 64 at a time in shared memory.
+// MASKED: the keys walked and the keys visible follow the AttnMask (HSTU-style
+// variants); otherwise keys 0 .. qi of the user (causal).
+template <bool MASKED>
 __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__ qkv,
                                                        float* __restrict__ out,
                                                        const int32_t* __restrict__ cu,
                                                        const int2* __restrict__ items,
                                                        const int32_t* __restrict__ item_count,
-                                                       const int32_t* err) {
+                                                       const int32_t* err, const AttnMask mask) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sK[64][DH + 1];
@@ -985,8 +1009,17 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
     o[d] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
-  const int kend = min(L, (it.y + 1) * ATT_BLK);
-  for (int k0 = 0; k0 < kend; k0 += 64) {
+  int kbeg = 0, kend = min(L, (it.y + 1) * ATT_BLK);
+  int C = 0, Hs = L;
+  if (MASKED) {
+    C = mask.ctx ? mask.ctx[it.x] : 0;
+    Hs = L - (mask.tgt ? mask.tgt[it.x] : 0);
+    int lo_key, hi_key;
+    mask_key_range(it.y, L, C, Hs, mask, lo_key, hi_key);
+    kbeg = lo_key / 64 * 64;
+    kend = hi_key + 1;
+  }
+  for (int k0 = kbeg; k0 < kend; k0 += 64) {
     __syncthreads();
     for (int i = threadIdx.x; i < 64 * DH; i += 128) {
       const int r = i / DH, d = i % DH;
@@ -996,7 +1029,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
     }
     __syncthreads();
     if (!valid) continue;
-    for (int r = 0; r < 64 && k0 + r <= qi; ++r) {
+    for (int r = 0; r < 64 && (MASKED ? k0 + r < kend : k0 + r <= qi); ++r) {
+      if (MASKED && !mask_visible(qi, k0 + r, C, Hs, mask)) continue;
       float s = 0.f;
 #pragma unroll
       for (int d = 0; d < DH; ++d) s = fmaf(q[d], sK[r][d], s);
@@ -1029,7 +1063,9 @@ int num_sms() {
   return n;
 }
 
-int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st) {
+int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st,
+                    const AttnMask* mask) {
+  const AttnMask m = mask ? *mask : AttnMask{nullptr, nullptr, 1, 1, 0};
   if (launch_k(worklist_kernel, dim3(1), dim3(1024), 0, st, cu, U, T, reinterpret_cast<int2*>(ws + L.items),
                                       reinterpret_cast<int32_t*>(ws + L.item_count),
                                       reinterpret_cast<int32_t*>(ws + L.lvl_hist),
@@ -1037,7 +1073,7 @@ int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws
                                       reinterpret_cast<int32_t*>(ws + L.lvl_fill), int(L.max_levels),
                                       attn_grid(L.max_items, num_sms()), reinterpret_cast<int4*>(ws + L.ulist),
                                       reinterpret_cast<int32_t*>(ws + L.uoff), reinterpret_cast<int32_t*>(ws + L.ucnt),
-                                      reinterpret_cast<int32_t*>(ws + L.err))) return -1;
+                                      reinterpret_cast<int32_t*>(ws + L.err), m, mask ? 1 : 0)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 
@@ -1170,10 +1206,15 @@ int launch_combine_f32(const float* y, const float* w, const float* x1, float* o
 }
 
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
-                    const char* ws, cudaStream_t st) {
-  if (launch_k(attn_f32_kernel, dim3(unsigned(L.max_items * H)), dim3(128), 0, st, 
-      qkv, out, cu, reinterpret_cast<const int2*>(ws + L.items),
-      reinterpret_cast<const int32_t*>(ws + L.item_count), reinterpret_cast<const int32_t*>(ws + L.err))) return -1;
+                    const char* ws, cudaStream_t st, const AttnMask* mask) {
+  const AttnMask m = mask ? *mask : AttnMask{nullptr, nullptr, 1, 1, 0};
+  const auto args = [&](auto kern) {
+    return launch_k(kern, dim3(unsigned(L.max_items * H)), dim3(128), 0, st, qkv, out, cu,
+                    reinterpret_cast<const int2*>(ws + L.items),
+                    reinterpret_cast<const int32_t*>(ws + L.item_count),
+                    reinterpret_cast<const int32_t*>(ws + L.err), m);
+  };
+  if (mask ? args(attn_f32_kernel<true>) : args(attn_f32_kernel<false>)) return -1;
   return PTL_LAUNCH_CHECK();
 }
 

@@ -38,7 +38,10 @@ int num_sms();  // of the current device (148 when it cannot be queried)
 // A kernel whose bounded wait runs out (which: 0 mbarrier, 1 global flag).
 int launch_wait_selftest(int32_t* err, const int32_t* flag, int which, uint64_t limit_ns,
                          cudaStream_t st);
-int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st);
+// mask (nullable): HSTU-style variant; validates the per-user counts and
+// lists the units for the masked attention
+int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st,
+                    const AttnMask* mask = nullptr);
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st);
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
@@ -68,7 +71,7 @@ int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, co
 int launch_combine_f32(const float* y, const float* w, const float* x1, float* out, int T,
                        const int32_t* err, cudaStream_t st);
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
-                    const char* ws, cudaStream_t st);
+                    const char* ws, cudaStream_t st, const AttnMask* mask = nullptr);
 
 // gemm_tc.cu (bf16, tcgen05).  QKV and the output projection run on CTA
 // pairs: their B (weight) tensor maps have boxes of BN/2 rows.
@@ -88,7 +91,9 @@ int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUten
                      const float* b2, const WsLayout& L, char* ws, cudaStream_t st);
 
 // attn_tc.cu (bf16, tcgen05)
+// mask (nullable): the HSTU-style variant, over a work list built with the
+// same mask
 int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
-                   char* ws, cudaStream_t st);
+                   char* ws, cudaStream_t st, const AttnMask* mask = nullptr);
 
 }  // namespace ptl

@@ -30,15 +30,27 @@
 
 namespace ptl {
 
-// Writes the padding users' offsets cu[U + 1 .. Ub] for a batch of T tokens
-// in a bucket of Tb tokens.  The real offsets cu[0 .. U] were copied in
+// Pads a batch of T tokens / U users to the bucket of Tb tokens / Ub users
+// in the static buffers: zero-fills the padding rows of x (row_bytes each)
+// and of the prediction mask (nullable), and (block 0) writes the padding
+// users' offsets cu[U + 1 .. Ub].  The real offsets cu[0 .. U] were copied in
 // before; if cu[U] is not T the batch is malformed, and the kernel makes the
 // offsets end below Tb so that the stack's offset validator reports
-// PTL_ERR_BAD_OFFSETS (the runner's own error word is cleared by the stack
-// call, so the fault has to travel through the offsets).
-__global__ void pad_offsets_kernel(int32_t* cu, int U, int T, int Tb, int Ub) {
+// PTL_ERR_BAD_OFFSETS (the error word itself is cleared by the stack call,
+// so the fault has to travel through the offsets).
+__global__ void pad_batch_kernel(int32_t* cu, int U, int T, int Tb, int Ub, char* x,
+                                 int row_bytes, uint8_t* mask) {
   pdl_wait();
   pdl_trigger();
+  const size_t n16 = size_t(Tb - T) * size_t(row_bytes) / 16;
+  int4* xp = reinterpret_cast<int4*>(x + size_t(T) * size_t(row_bytes));
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += size_t(gridDim.x) * blockDim.x)
+    xp[i] = make_int4(0, 0, 0, 0);
+  if (mask)
+    for (int i = T + int(blockIdx.x * blockDim.x + threadIdx.x); i < Tb; i += gridDim.x * blockDim.x)
+      mask[i] = 0;
+  if (blockIdx.x != 0) return;
   const bool bad = cu[U] != T;
   for (int i = U + 1 + int(threadIdx.x); i <= Ub; i += blockDim.x) {
     const int64_t v = int64_t(T) + int64_t(i - U) * ATT_BLK;
@@ -244,27 +256,28 @@ ptl_status ptl_runner_forward(ptl_stack_runner* r, const void* x, void* out, con
   ptl_status s = graph_for(r, b, &g);
   if (s != PTL_OK) return s;
   const size_t row = size_t(ptl::D) * r->es;
-  // inputs into the static buffers (host or device sources), padding zeroed
+  // inputs into the static buffers (host or device sources), then one
+  // kernel for the padding rows, mask entries and users
   if (cudaMemcpyAsync(r->x_s, x, size_t(T) * row, cudaMemcpyDefault, st) != cudaSuccess)
-    return PTL_ERR_CUDA;
-  if (Tb > T && cudaMemsetAsync(r->x_s + size_t(T) * row, 0, size_t(Tb - T) * row, st) != cudaSuccess)
     return PTL_ERR_CUDA;
   if (cudaMemcpyAsync(r->cu_s, cu_seqlens, 4 * (size_t(num_users) + 1), cudaMemcpyDefault, st) !=
       cudaSuccess)
     return PTL_ERR_CUDA;
+  if (r->has_head &&
+      cudaMemcpyAsync(r->mask_s, pred_mask, size_t(T), cudaMemcpyDefault, st) != cudaSuccess)
+    return PTL_ERR_CUDA;
   {
+    const size_t n16 = size_t(Tb - T) * row / 16;
+    size_t blocks = (n16 + 255) / 256;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 64) blocks = 64;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(1);
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3(unsigned(blocks));
+    cfg.blockDim = dim3(256);
     cfg.stream = st;
-    if (cudaLaunchKernelEx(&cfg, ptl::pad_offsets_kernel, r->cu_s, int(num_users), int(T), int(Tb),
-                           int(r->ub)) != cudaSuccess)
-      return PTL_ERR_CUDA;
-  }
-  if (r->has_head) {
-    if (cudaMemcpyAsync(r->mask_s, pred_mask, size_t(T), cudaMemcpyDefault, st) != cudaSuccess)
-      return PTL_ERR_CUDA;
-    if (Tb > T && cudaMemsetAsync(r->mask_s + T, 0, size_t(Tb - T), st) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, ptl::pad_batch_kernel, r->cu_s, int(num_users), int(T), int(Tb),
+                           int(r->ub), r->x_s, int(row), r->has_head ? r->mask_s : nullptr) !=
+        cudaSuccess)
       return PTL_ERR_CUDA;
   }
   if (cudaGraphLaunch(g, st) != cudaSuccess) return PTL_ERR_CUDA;

@@ -22,7 +22,7 @@ PTL_F32, PTL_BF16 = 0, 1
 STATUS = {
     0: "PTL_OK", 1: "PTL_ERR_NULL", 2: "PTL_ERR_ALIGN", 3: "PTL_ERR_SHAPE",
     4: "PTL_ERR_BAD_OFFSETS", 5: "PTL_ERR_WORKSPACE", 6: "PTL_ERR_DTYPE", 7: "PTL_ERR_CUDA",
-    8: "PTL_ERR_TIMEOUT", 9: "PTL_ERR_UNSUPPORTED",
+    8: "PTL_ERR_TIMEOUT", 9: "PTL_ERR_UNSUPPORTED", 10: "PTL_ERR_BAD_MASK",
 }
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
@@ -51,6 +51,12 @@ class HeadWeights(ctypes.Structure):
 class DebugOut(ctypes.Structure):
     _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
                 ("perm", ctypes.c_void_p), ("expert_off", ctypes.c_void_p)]
+
+
+class AttnMaskStruct(ctypes.Structure):
+    _fields_ = [("causal", ctypes.c_int32), ("num_contexts", ctypes.c_void_p),
+                ("num_targets", ctypes.c_void_p), ("target_group_size", ctypes.c_int32),
+                ("window", ctypes.c_int32)]
 
 
 class Trace(ctypes.Structure):
@@ -82,6 +88,9 @@ _SIGS = {
     "ptl_attention": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                        ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                        ctypes.c_void_p], ctypes.c_int),
+    "ptl_attention_masked": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                              ctypes.c_int64, ctypes.c_int, ctypes.POINTER(AttnMaskStruct),
+                              ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
     "ptl_out_projection": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                             ctypes.c_int, ctypes.POINTER(LayerWeights), ctypes.c_void_p,
                             ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
@@ -262,6 +271,18 @@ def attention(qkv, attn, cu_seqlens, workspace, stream=None):
     _check(lib().ptl_attention(_ptr(qkv), _ptr(attn), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
                                qkv.shape[0], _dt(qkv.dtype), _ptr(workspace), workspace.numel(),
                                _stream(stream)), "ptl_attention")
+    return attn
+
+
+def attention_masked(qkv, attn, cu_seqlens, workspace, causal=True, num_contexts=None,
+                     num_targets=None, target_group_size=1, window=0, stream=None):
+    """HSTU-style masked attention (``ptl_attention_masked``); num_contexts /
+    num_targets: device int32 tensors [U] or None."""
+    m = AttnMaskStruct(int(bool(causal)), _ptr(num_contexts), _ptr(num_targets),
+                       int(target_group_size), int(window))
+    _check(lib().ptl_attention_masked(_ptr(qkv), _ptr(attn), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                      qkv.shape[0], _dt(qkv.dtype), ctypes.byref(m), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "ptl_attention_masked")
     return attn
 
 

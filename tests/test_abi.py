@@ -148,3 +148,23 @@ def test_runner_bucket_and_host_checks(P):
     assert L.ptl_runner_last_device_error(None, None) == S["PTL_ERR_NULL"]
     assert L.ptl_runner_graphs(None) == -1
     L.ptl_runner_destroy(None)
+
+
+def test_attention_masked_host_checks(P):
+    L = P.lib()
+    S = P.STATUS_CODE
+    ws_b = P.workspace_size(64, 4, 1)
+    m = P.AttnMaskStruct(1, None, None, 1, 0)
+    assert L.ptl_attention_masked(FAKE, FAKE, FAKE, 4, 64, 1, None, FAKE, ws_b, None) == S["PTL_ERR_NULL"]
+    bad_group = P.AttnMaskStruct(1, None, None, 0, 0)
+    assert L.ptl_attention_masked(FAKE, FAKE, FAKE, 4, 64, 1, ctypes.byref(bad_group), FAKE, ws_b,
+                                  None) == S["PTL_ERR_BAD_MASK"]
+    bad_causal = P.AttnMaskStruct(2, None, None, 1, 0)
+    assert L.ptl_attention_masked(FAKE, FAKE, FAKE, 4, 64, 1, ctypes.byref(bad_causal), FAKE, ws_b,
+                                  None) == S["PTL_ERR_BAD_MASK"]
+    assert L.ptl_attention_masked(FAKE, FAKE, FAKE, 4, 0, 1, ctypes.byref(m), FAKE, ws_b,
+                                  None) == S["PTL_OK"]
+    mis = P.AttnMaskStruct(1, FAKE + 2, None, 1, 0)
+    assert L.ptl_attention_masked(FAKE, FAKE, FAKE, 4, 64, 1, ctypes.byref(mis), FAKE, ws_b,
+                                  None) == S["PTL_ERR_ALIGN"]
+    assert P.status_string(S["PTL_ERR_BAD_MASK"]).startswith("attention mask")
