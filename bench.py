@@ -107,6 +107,81 @@ def attention_flops(lengths):
     return 2048 * int((L * (L + 1) // 2).sum())
 
 
+# HSTU-style mask of the masked-attention leg: per user, a tenth of the
+# tokens contextual, a tenth of the rest candidates in groups of four
+MASKED_LEG = {"ctx_frac": 0.1, "tgt_frac": 0.1, "group": 4, "window": 0, "causal": True}
+
+
+def masked_counts(lengths):
+    L = np.asarray(lengths, np.int64)
+    ctx = (L * MASKED_LEG["ctx_frac"]).astype(np.int32)
+    tgt = ((L - ctx) * MASKED_LEG["tgt_frac"]).astype(np.int32)
+    return ctx, tgt
+
+
+def visible_pairs(lengths, ctx, tgt):
+    """(query, key) pairs the masked leg's mask leaves visible, counted per
+    user: the algorithmic work of the masked attention is 2048 FLOPs per
+    visible pair (QK^T and PV over 8 heads of 64)."""
+    total = 0
+    for L, C, N in zip(lengths, ctx, tgt):
+        L, C, N = int(L), int(C), int(N)
+        if L == 0:
+            continue
+        i = np.arange(L)[:, None]
+        j = np.arange(L)[None, :]
+        v = (j <= i) if MASKED_LEG["causal"] else np.ones((L, L), bool)
+        v |= (i < C) & (j < C)
+        Hs, G = L - N, MASKED_LEG["group"]
+        v &= (j < Hs) | ((i >= Hs) & ((i - Hs) // G == (j - Hs) // G))
+        if MASKED_LEG["window"] > 0:
+            v &= np.abs(i - j) < MASKED_LEG["window"]
+        total += int(v.sum())
+    return total
+
+
+def time_attention_legs(case, dev, stream, flush, reps=20):
+    """Device time (CUDA events, L2 flushed between launches) of the causal
+    attention and of the masked variant on the workload's packing."""
+    import torch
+
+    from packed_sequence_transformer_b200 import ptl
+    T, U = case.total_tokens, case.num_users
+    g = torch.Generator(device="cpu").manual_seed(5)
+    qkv = torch.randn(T, 1536, generator=g).to(dev, torch.bfloat16)
+    cu = torch.as_tensor(case.cu_seqlens).to(dev, torch.int32)
+    ctx_h, tgt_h = masked_counts(case.lengths)
+    ctx, tgt = torch.as_tensor(ctx_h).to(dev), torch.as_tensor(tgt_h).to(dev)
+    out = torch.empty(T, 512, dtype=torch.bfloat16, device=dev)
+    ws = ptl.alloc_workspace(T, U, "bf16", dev)
+    calls = {
+        "causal": lambda: ptl.attention(qkv, out, cu, ws, stream=stream),
+        "masked": lambda: ptl.attention_masked(qkv, out, cu, ws, causal=MASKED_LEG["causal"],
+                                               num_contexts=ctx, num_targets=tgt,
+                                               target_group_size=MASKED_LEG["group"],
+                                               window=MASKED_LEG["window"], stream=stream),
+    }
+    res = {}
+    for name, fn in calls.items():
+        kt = ptl.KernelTrace(capacity=8)
+        times = []
+        with torch.cuda.stream(stream):
+            for i in range(reps + 3):
+                with kt:
+                    fn()
+                torch.cuda.synchronize()
+                if i >= 3:
+                    times.extend(t for k, t in kt.launches() if k == "attention")
+                flush.fill_(float(i))
+        torch.cuda.synchronize()
+        st = ptl.last_device_error(ws, stream)
+        if st != 0:
+            raise RuntimeError(f"device error {ptl.STATUS.get(st)} in the {name} attention leg")
+        res[name] = 1e3 * statistics.mean(times)
+    pairs = visible_pairs(case.lengths, ctx_h, tgt_h)
+    return res, pairs
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples (every 200 ms) while the timed region runs."""
@@ -432,6 +507,16 @@ def run_ours(args):
     eager_ms = timed(step, 2, args.steps, False)
     runner.close()
 
+    attn_us, masked_pairs = time_attention_legs(case, dev, stream, flush)
+    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    masked_leg = {
+        "mask": dict(MASKED_LEG), "visible_pairs": masked_pairs,
+        "causal_us": attn_us["causal"], "masked_us": attn_us["masked"],
+        "causal_tflops": attn_fl / attn_us["causal"] / 1e6,
+        "masked_tflops": 2048 * masked_pairs / attn_us["masked"] / 1e6,
+    }
+    masked_leg["masked_frac"] = masked_leg["masked_tflops"] / bf16_peak
+
     cpu = None
     if rank == 0 and world == 1:
         sec, reps = time_oracle_layers(case, budget_s=15.0, max_reps=6, min_reps=2)
@@ -463,6 +548,7 @@ def run_ours(args):
                        "runner": {"stride": RUNNER_STRIDE, "bucket_tokens": bucket, "device_buffers_ms_per_step": runner_ms,
                                   "host_buffers_ms_per_step": e2e_ms},
                        "eager_ms_per_step": eager_ms,
+                       "attention_legs": masked_leg,
                        "kernels": kinds, "attention_flops_per_layer": attn_fl,
                        "gemm_flops_per_layer": GEMM_FLOPS_PER_TOKEN * T},
         }

@@ -468,6 +468,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       if (k_list < n_list) nxt = unit_from<MASKED>(list[k_list], mask);  // prefetch the next unit
       const int qi = a.b * ATT_BLK + r;   // query position inside the user
       const int qlim = min(qi, a.L - 1);  // keys 0..qlim are visible
+      // masked variant: the row's visible keys as two intervals
+      int va0 = 0, vb0 = -1, va1 = 0, vb1 = -1;
+      if constexpr (MASKED) {
+        if (qi < a.L) mask_row_intervals(qi, a.L, a.C, a.Hs, mask, va0, vb0, va1, vb1);
+      }
       for (int kb = a.lo; kb <= a.hi; ++kb, ++n) {
         if (!mbar_wait(&s_full[g], n & 1)) { ok = false; break; }
         tc_fence_after();
@@ -478,24 +483,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // rows; this half owns chunks 2h and 2h + 1 (keys past qlim masked)
         const int nch = (k16 + 31) >> 5;
         const int nuse = (!MASKED && kb == a.b) ? min(nch, wq + 1) : nch;
-        const bool mine = 2 * h < nuse;
+        // masked variant: visibility of this half's 64 keys, one bit per key;
+        // a warp whose rows see none of them skips the half (P written as 0)
+        uint32_t vbits[2] = {0u, 0u};
+        if constexpr (MASKED) {
+          const int j0 = kbase + 64 * h;
+          vbits[0] = interval_bits32(va0, vb0, j0) | interval_bits32(va1, vb1, j0);
+          vbits[1] = interval_bits32(va0, vb0, j0 + 32) | interval_bits32(va1, vb1, j0 + 32);
+        }
+        const bool mine = 2 * h < nuse && (!MASKED || __any_sync(0xffffffffu, (vbits[0] | vbits[1]) != 0u));
         const int lim = qlim - (kbase + 64 * h);  // this half's keys i <= lim are visible
         // pass 1: this half's row maximum over the visible keys
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        // masked variant: visibility of this half's 64 keys, one bit per key
-        uint32_t vbits[2] = {0u, 0u};
-        if constexpr (MASKED) {
-          if (mine) {
-#pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-              uint32_t bits = 0u;
-              const int j0 = kbase + 64 * h + 32 * c;
-              for (int i = 0; i < 32; ++i)
-                if (j0 + i < a.L && mask_visible(qi, j0 + i, a.C, a.Hs, mask)) bits |= 1u << i;
-              vbits[c] = bits;
-            }
-          }
-        }
         if (mine) {
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {  // 32 columns per TMEM load
@@ -504,7 +503,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             tmem_ld_wait();
             const int lc = lim - 32 * c;
             if constexpr (MASKED) {
-              const uint32_t bits = vbits[c];
+              const uint32_t bits = c ? vbits[1] : vbits[0];
 #pragma unroll
               for (int i = 0; i < 32; ++i)
                 if ((bits >> i) & 1u) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
@@ -556,13 +555,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const int lc = lim - 32 * c;
             const int lc_eff = lc >= 31 ? 31 : lc;
             uint32_t pk[16];
+            const uint32_t bits = c ? vbits[1] : vbits[0];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
               float p0 = ex2_approx(__uint_as_float(raw[i]) * c2 - m);
               float p1 = ex2_approx(__uint_as_float(raw[i + 1]) * c2 - m);
               if constexpr (MASKED) {
-                p0 = ((vbits[c] >> i) & 1u) ? p0 : 0.f;
-                p1 = ((vbits[c] >> (i + 1)) & 1u) ? p1 : 0.f;
+                p0 = ((bits >> i) & 1u) ? p0 : 0.f;
+                p1 = ((bits >> (i + 1)) & 1u) ? p1 : 0.f;
               } else if (lc < 31) {
                 p0 = (i <= lc_eff) ? p0 : 0.f;
                 p1 = (i + 1 <= lc_eff) ? p1 : 0.f;

@@ -164,6 +164,46 @@ __device__ __forceinline__ bool mask_visible(int i, int j, int C, int Hs, const 
   return v;
 }
 
+// The keys visible to query i under the mask, as two intervals [a0, b0] and
+// [a1, b1] of positions (an interval with a > b is empty): a non-candidate
+// row sees [0 .. (causal ? (contextual ? C - 1 : i) : L - 1)] below the
+// first candidate; a candidate row sees [0, Hs - 1] and, second, its own
+// group up to itself (causal) or to the group's end.  Both are then cut to
+// the window.  The same set as mask_visible, for every i < L.
+__device__ __forceinline__ void mask_row_intervals(int i, int L, int C, int Hs, const AttnMask& m,
+                                                   int& a0, int& b0, int& a1, int& b1) {
+  a0 = 0;
+  a1 = 1;
+  b1 = 0;  // empty
+  if (i < Hs) {
+    int hi = m.causal ? (i < C ? C - 1 : i) : L - 1;
+    b0 = hi < Hs - 1 ? hi : Hs - 1;
+  } else {
+    b0 = Hs - 1;
+    const int g0 = Hs + (i - Hs) / m.group * m.group;
+    const int rest = L - 1 - g0;  // keys of the user from g0 on, less one
+    a1 = g0;
+    b1 = m.causal ? i : g0 + (m.group - 1 < rest ? m.group - 1 : rest);
+  }
+  if (m.window > 0) {
+    const int wl = i - m.window + 1, wh = i + m.window - 1;
+    if (wl > a0) a0 = wl;
+    if (wh < b0) b0 = wh;
+    if (wl > a1) a1 = wl;
+    if (wh < b1) b1 = wh;
+  }
+}
+
+// Bits k (0..31) set where j0 + k lies in [a, b].
+__device__ __forceinline__ uint32_t interval_bits32(int a, int b, int j0) {
+  int lo = a - j0, hi = b - j0 + 1;  // bits [lo, hi)
+  lo = lo > 0 ? lo : 0;
+  hi = hi < 32 ? hi : 32;
+  if (hi <= lo) return 0u;
+  const uint32_t below_hi = hi >= 32 ? 0xFFFFFFFFu : ((1u << hi) - 1u);
+  return below_hi & ~((1u << lo) - 1u);
+}
+
 // Keys [lo_key, hi_key] that hold every key visible to some query of block b
 // (queries q0 .. q1 of the user): the range the key loop walks.
 __device__ __forceinline__ void mask_key_range(int b, int L, int C, int Hs, const AttnMask& m,

@@ -52,6 +52,8 @@ MASKS = {
     "window_200_no_mask": dict(window=200, causal=False),
     "combined": dict(ctx=(0.3, 0.3), group=4, window=150),
     "combined_no_mask": dict(ctx=(0.3, 0.3), group=2, window=300, causal=False),
+    "targets_small_window": dict(ctx=(0.2, 0.5), group=3, window=7),
+    "targets_no_mask_g2": dict(ctx=(0.0, 0.6), group=2, causal=False),
 }
 
 

@@ -75,3 +75,17 @@ def test_reference_arm_only_on_rank_zero(monkeypatch, capsys):
     monkeypatch.setattr(bench, "time_oracle_layers", lambda *a, **k: called.append(1) or (1.0, 1))
     assert bench.run_reference(Args) == 0
     assert called == [] and capsys.readouterr().out == ""
+
+
+def test_masked_leg_pair_count_matches_the_oracle_mask():
+    from oracle import ptl_oracle as O
+    lengths = [0, 1, 7, 40, 129, 300]
+    ctx, tgt = bench.masked_counts(lengths)
+    want = sum(int(O.hstu_user_mask(L, bench.MASKED_LEG["causal"], C, N, bench.MASKED_LEG["group"],
+                                    bench.MASKED_LEG["window"]).sum())
+               for L, C, N in zip(lengths, ctx, tgt) if L > 0)
+    assert bench.visible_pairs(lengths, ctx, tgt) == want
+    assert (ctx + tgt <= np.asarray(lengths)).all()
+    # with no contexts or candidates the count is the causal one
+    zero = np.zeros(len(lengths), np.int32)
+    assert bench.visible_pairs(lengths, zero, zero) == sum(L * (L + 1) // 2 for L in lengths)
