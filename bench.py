@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import faulthandler
 import json
 import os
 import statistics
@@ -560,6 +561,10 @@ def run_ours(args):
 
 def main():
     args = parse()
+    # watchdog: a run that has not finished after this many seconds prints
+    # every thread's Python stack to stderr and exits (the default run takes
+    # well under a minute of GPU time)
+    faulthandler.dump_traceback_later(float(os.environ.get("PTL_BENCH_WATCHDOG_S", "600")), exit=True)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
