@@ -17,7 +17,9 @@ Sources (web pages, cited by title and section):
     + Linear(1024->512); each token weighted over its 2 experts), the fused
     MoE routing notes (per-expert counts, token reordering, route-major rows
     token_id*top_k + k_idx, per-token weighted sum) and the Prediction Head
-    section (Linear(512->1) -> clamp(-15, 15) -> sigmoid, pred_mask select).
+    section (Linear(512->1) -> clamp(-15, 15) -> sigmoid, pred_mask select),
+    and the RepEncoder section (28-slot embedding bag with sum pooling,
+    LayerNorm over the 14336 concatenated values, Linear(14336->512)).
   * "CTI-Inference-Opt" optimisation plan -- attention as softmax(QK^T/sqrt(d))V.
   * "cry-daniel/recsys" README -- the HSTU attention mask logic (contextual,
     historical and candidate segments; mask types none, local, causal,
@@ -241,6 +243,41 @@ def jagged_hstu_attention(q, k, v, cu_seqlens, causal=True, num_contexts=None, n
             S = np.where(vis, S, -np.inf)
             out[s:e, h, :] = _softmax_rows(S) @ v[s:e, h, :]
     return out
+
+
+# --------------------------------------------------------------------------
+# RepEncoder front end (cti2026 README, RepEncoder section: a batched
+# embedding bag over 28 slots with sum pooling, the [tokens, 28, 512] result
+# flattened to [tokens, 14336], LayerNorm over the 14336 values, then
+# Linear(14336 -> 512) into the encoder's input rows)
+# --------------------------------------------------------------------------
+REP_SLOTS = 28
+
+
+def embedding_bags(tables, ids, bag_offsets, num_tokens):
+    """Sum pooling per (token, slot): bag (t, s) holds ids[off[t*28+s] ..
+    off[t*28+s+1]) of slot s's table; an empty bag gives zeros.  Returns
+    [T, 28*dim] with slot s in columns s*dim .. s*dim+dim-1."""
+    off = np.asarray(bag_offsets, np.int64)
+    ids = np.asarray(ids, np.int64)
+    dim = np.asarray(tables[0]).shape[1]
+    out = np.zeros((num_tokens, REP_SLOTS * dim))
+    for t in range(num_tokens):
+        for sl in range(REP_SLOTS):
+            b = t * REP_SLOTS + sl
+            rows = ids[off[b]:off[b + 1]]
+            if rows.size:
+                out[t, sl * dim:(sl + 1) * dim] = _f64(np.asarray(tables[sl])[rows]).sum(axis=0)
+    return out
+
+
+def rep_encoder(tables, ids, bag_offsets, num_tokens, ln_g, ln_b, w, b=None, storage=None):
+    """The front end: embedding bags -> LayerNorm(28*512) -> Linear to 512.
+    storage='bf16' rounds the normalised rows as a bf16 pipeline stores them."""
+    st = _storage(storage)
+    bags = embedding_bags(tables, ids, bag_offsets, num_tokens)
+    normed = st(layer_norm(bags, ln_g, ln_b))
+    return linear(normed, w, b)
 
 
 # --------------------------------------------------------------------------

@@ -241,3 +241,57 @@ CONFIGS = {0: config0, 1: config1, 2: config2, 3: config3, 4: config4}
 def random_bf16_array(rng: np.random.Generator, shape, std=1.0) -> np.ndarray:
     """N(0, std^2) float32 values rounded to the bfloat16 grid."""
     return round_to_bf16(_normal(rng, shape, std))
+
+
+# ------------------------------------------------------------ RepEncoder
+REP_SLOTS = 28
+REP_DIM = 512
+
+
+@dataclass
+class RepCase:
+    """Inputs of the RepEncoder front end: 28 embedding tables, the id bags
+    (bag (t, s) = ids[bag_offsets[t*28+s] .. bag_offsets[t*28+s+1])) and the
+    LayerNorm / Linear parameters."""
+    name: str
+    dtype: str
+    num_tokens: int
+    tables: List[np.ndarray]   # 28 x [vocab_s, 512]
+    ids: np.ndarray            # int64 [n_ids]
+    bag_offsets: np.ndarray    # int64 [T*28 + 1]
+    ln_g: np.ndarray           # [14336] f32
+    ln_b: np.ndarray
+    w: np.ndarray              # [512, 14336]
+    b: Optional[np.ndarray]    # [512] or None
+
+
+def make_rep_case(name: str, num_tokens: int, *, vocab=1000, max_bag=4, empty_p=0.1, seed=0,
+                  dtype="bf16", table_std=1.0, w_std=0.02, random_affine=False) -> RepCase:
+    """Seeded synthetic front-end inputs: per slot a table of `vocab` rows
+    (a slot index that differs per slot, so that mixing up slots shows),
+    bag sizes uniform in 1..max_bag with a share `empty_p` of empty bags,
+    ids uniform over the slot's table."""
+    rng = np.random.default_rng(seed)
+    vocabs = [int(vocab) + 7 * s for s in range(REP_SLOTS)]
+    tables = [_normal(rng, (v, REP_DIM), table_std) for v in vocabs]
+    n_bags = num_tokens * REP_SLOTS
+    sizes = rng.integers(1, max_bag + 1, size=n_bags)
+    sizes[rng.random(n_bags) < empty_p] = 0
+    off = np.zeros(n_bags + 1, np.int64)
+    np.cumsum(sizes, out=off[1:])
+    slot_of_bag = np.arange(n_bags) % REP_SLOTS
+    ids = np.concatenate([rng.integers(0, vocabs[s], size=int(n)) for s, n in zip(slot_of_bag, sizes)]
+                         if n_bags else [np.zeros(0, np.int64)]).astype(np.int64)
+    width = REP_SLOTS * REP_DIM
+    ln_g = np.ones(width, np.float32)
+    ln_b = np.zeros(width, np.float32)
+    b = None
+    if random_affine:
+        ln_g = (1.0 + 0.1 * rng.standard_normal(width)).astype(np.float32)
+        ln_b = (0.1 * rng.standard_normal(width)).astype(np.float32)
+        b = (0.02 * rng.standard_normal(REP_DIM)).astype(np.float32)
+    w = _normal(rng, (REP_DIM, width), w_std)
+    if dtype == "bf16":
+        tables = [round_to_bf16(t) for t in tables]
+        w = round_to_bf16(w)
+    return RepCase(name, dtype, num_tokens, tables, ids, off, ln_g, ln_b, w, b)

@@ -145,3 +145,29 @@ def test_window_off_by_one_is_caught(monkeypatch):
     _mask_mutant(monkeypatch, lambda f, L, c, C, N, G, W: f(L, c, C, N, G, W + 1 if W > 0 else 0))
     assert _fails(PH.test_window_one_gives_own_v_and_wide_window_is_causal)
     assert _fails(lambda: PH.test_window_rows_see_their_neighbourhood(True))
+
+
+# ------------------------------------------------- RepEncoder front end
+import tests.test_oracle_rep as PR  # noqa: E402
+
+
+def test_slot_mix_up_is_caught(monkeypatch):
+    # each slot's sum written one slot block to the right
+    orig = O.embedding_bags
+    monkeypatch.setattr(O, "embedding_bags",
+                        lambda tables, ids, off, T: np.roll(orig(tables, ids, off, T), 512, axis=1))
+    assert _fails(PR.test_bags_match_torch_embedding_bag_per_slot)
+
+
+def test_layer_norm_per_slot_instead_of_whole_row_is_caught(monkeypatch):
+    orig_ln = O.layer_norm
+
+    def per_slot(x, g, b, eps=O.LN_EPS):
+        x = np.asarray(x, np.float64)
+        if x.shape[-1] != 14336:
+            return orig_ln(x, g, b, eps)
+        parts = [orig_ln(x[..., s * 512:(s + 1) * 512], np.asarray(g)[s * 512:(s + 1) * 512],
+                         np.asarray(b)[s * 512:(s + 1) * 512], eps) for s in range(28)]
+        return np.concatenate(parts, axis=-1)
+    monkeypatch.setattr(O, "layer_norm", per_slot)
+    assert _fails(PR.test_front_end_is_torch_layer_norm_and_linear)
