@@ -183,6 +183,53 @@ def time_attention_legs(case, dev, stream, flush, reps=20):
     return res, pairs
 
 
+def time_rep_leg(T, dev, stream, flush, reps=10, vocab=50_000, max_bag=4, seed=9):
+    """The RepEncoder front end on T tokens: 28 device tables of `vocab` rows
+    (1.4 GB in bf16, beyond L2), bags of 1..max_bag ids (a tenth empty);
+    device time of the embedding-bag + LayerNorm kernel and of the Linear."""
+    import torch
+
+    from packed_sequence_transformer_b200 import ptl
+    rng = np.random.default_rng(seed)
+    g = torch.Generator(device=dev).manual_seed(seed)
+    tables = [torch.randn(vocab, 512, device=dev, generator=g).to(torch.bfloat16) for _ in range(28)]
+    sizes = rng.integers(1, max_bag + 1, size=T * 28)
+    sizes[rng.random(T * 28) < 0.1] = 0
+    off_h = np.zeros(T * 28 + 1, np.int64)
+    np.cumsum(sizes, out=off_h[1:])
+    ids = torch.as_tensor(rng.integers(0, vocab, size=int(off_h[-1])), dtype=torch.int64).to(dev)
+    off = torch.as_tensor(off_h).to(dev)
+    ln_g = torch.ones(14336, device=dev)
+    ln_b = torch.zeros(14336, device=dev)
+    w = (0.02 * torch.randn(512, 14336, device=dev, generator=g)).to(torch.bfloat16)
+    b = torch.zeros(512, device=dev)
+    st = ptl.rep_weights_struct(tables, ln_g, ln_b, w, b)
+    out = torch.empty(T, 512, dtype=torch.bfloat16, device=dev)
+    ws = ptl.rep_encoder_workspace(T, "bf16", dev)
+    kt = ptl.KernelTrace(capacity=8)
+    t_bag, t_gemm = [], []
+    with torch.cuda.stream(stream):
+        for i in range(reps + 3):
+            with kt:
+                ptl.rep_encoder(ids, off, T, st, out, ws, stream=stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ks = kt.launches()
+                t_bag += [t for k, t in ks if k == "layernorm"]
+                t_gemm += [t for k, t in ks if k == "gemm_qkv"]
+            flush.fill_(float(i))
+    torch.cuda.synchronize()
+    if ptl.last_device_error(ws, stream) != 0:
+        raise RuntimeError("device error in the RepEncoder leg")
+    n_ids = int(off_h[-1])
+    bag_bytes = n_ids * (1024 + 8) + T * 28 * 8 + T * 14336 * 2  # rows + ids + offsets, normalised rows out
+    flops = 2 * T * 14336 * 512
+    bag_us, gemm_us = 1e3 * statistics.mean(t_bag), 1e3 * statistics.mean(t_gemm)
+    return {"tokens": T, "ids": n_ids, "vocab_per_slot": vocab, "embag_ln_us": bag_us,
+            "embag_ln_gbs": bag_bytes / bag_us / 1e3, "linear_us": gemm_us,
+            "linear_tflops": flops / gemm_us / 1e6}
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples (every 200 ms) while the timed region runs."""
@@ -517,6 +564,9 @@ def run_ours(args):
         "masked_tflops": 2048 * masked_pairs / attn_us["masked"] / 1e6,
     }
     masked_leg["masked_frac"] = masked_leg["masked_tflops"] / bf16_peak
+    rep_leg = time_rep_leg(T, dev, stream, flush)
+    rep_leg["embag_ln_frac"] = rep_leg["embag_ln_gbs"] / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    rep_leg["linear_frac"] = rep_leg["linear_tflops"] / bf16_peak
 
     cpu = None
     if rank == 0 and world == 1:
@@ -550,6 +600,7 @@ def run_ours(args):
                                   "host_buffers_ms_per_step": e2e_ms},
                        "eager_ms_per_step": eager_ms,
                        "attention_legs": masked_leg,
+                       "rep_encoder": rep_leg,
                        "kernels": kinds, "attention_flops_per_layer": attn_fl,
                        "gemm_flops_per_layer": GEMM_FLOPS_PER_TOKEN * T},
         }

@@ -81,7 +81,8 @@ typedef enum {
   PTL_ERR_CUDA = 7,        /* a CUDA runtime call or launch failed */
   PTL_ERR_TIMEOUT = 8,     /* a bounded device-side wait ran out (kernel returned early) */
   PTL_ERR_UNSUPPORTED = 9, /* no sm_100 device, or a feature not built */
-  PTL_ERR_BAD_MASK = 10    /* attention mask out of range (ptl_attention_masked) */
+  PTL_ERR_BAD_MASK = 10,   /* attention mask out of range (ptl_attention_masked) */
+  PTL_ERR_BAD_IDS = 11     /* embedding id outside its table or bad bag offsets (ptl_rep_encoder) */
 } ptl_status;
 
 typedef enum { PTL_F32 = 0, PTL_BF16 = 1 } ptl_dtype;
@@ -351,6 +352,38 @@ ptl_status ptl_runner_last_device_error(ptl_stack_runner* runner, void* stream);
 /* Number of buckets whose graph has been captured (-1 for NULL). */
 int32_t ptl_runner_graphs(const ptl_stack_runner* runner);
 void ptl_runner_destroy(ptl_stack_runner* runner);
+
+/* ---- RepEncoder front end. ----
+ * The encoder's input rows come from a RepEncoder (cti2026 README,
+ * RepEncoder section): for every token, 28 slots each look up a bag of
+ * feature ids in their own embedding table and sum the rows (sum pooling;
+ * one launch for all slots, the tables passed as 28 pointers, 64-bit row
+ * offsets), the [28][512] sums are flattened to 14336 values, normalised by
+ * one LayerNorm over those 14336 values (eps 1e-5, biased variance), and
+ * Linear(14336 -> 512) gives the token's row:
+ *   out[t] = LN(concat_s sum_{i in bag(t, s)} tables[s][ids[i]]) W^T + b.
+ * Bag (t, s) holds ids[bag_offsets[t*28 + s] .. bag_offsets[t*28 + s + 1]);
+ * an empty bag gives zeros.  ids: device int64 [num_ids]; bag_offsets:
+ * device int64 [T*28 + 1], non-decreasing within 0 .. num_ids; out: device
+ * [T][512] of dt.  Tables and W in dt, LayerNorm parameters and b in fp32.
+ * Device checks: an id outside 0 .. vocab[s]-1, or a bag range outside
+ * 0 .. num_ids or decreasing, sets PTL_ERR_BAD_IDS in the workspace error
+ * word (read with ptl_last_device_error); the output is then undefined.
+ * workspace: ptl_rep_encoder_workspace_size(T, dt) bytes, 256-byte aligned
+ * (the error word and the normalised rows).  Asynchronous on `stream`. */
+#define PTL_REP_SLOTS 28
+typedef struct {
+  const void* tables[PTL_REP_SLOTS]; /* device [vocab[s]][512] dt (NULL allowed when vocab[s] == 0) */
+  int64_t vocab[PTL_REP_SLOTS];      /* rows of each table */
+  const float* ln_g;                 /* [14336] f32 */
+  const float* ln_b;                 /* [14336] f32 */
+  const void* w;                     /* [512][14336] dt */
+  const float* b;                    /* [512] f32 or NULL */
+} ptl_rep_encoder_weights;
+size_t ptl_rep_encoder_workspace_size(int64_t max_tokens, ptl_dtype dt);
+ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* bag_offsets,
+                           int64_t total_tokens, ptl_dtype dt, const ptl_rep_encoder_weights* w,
+                           void* out, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---- Failure detection self-test. ----
  * Every wait inside the library's kernels (on an mbarrier phase, or on a

@@ -363,6 +363,7 @@ const char* ptl_status_string(ptl_status s) {
     case PTL_ERR_DTYPE: return "unknown dtype";
     case PTL_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case PTL_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    case PTL_ERR_BAD_IDS: return "an embedding id outside its table, or bag offsets not within 0 .. num_ids and non-decreasing";
     case PTL_ERR_BAD_MASK: return "attention mask: target_group_size < 1, causal not 0/1, or a user's contextual + candidate counts outside 0 .. its length";
     case PTL_ERR_UNSUPPORTED: return "unsupported device (needs sm_100)";
   }
@@ -574,6 +575,60 @@ ptl_status ptl_head(const void* h, const ptl_head_weights* head, const uint8_t* 
   EndMark end_mark{c.st};
   mark(c.st, PTL_KERNEL_HEAD);
   PTL_TRY(launch_head(h, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st));
+  return PTL_OK;
+}
+
+size_t ptl_rep_encoder_workspace_size(int64_t max_tokens, ptl_dtype dt) {
+  if (max_tokens < 0 || max_tokens >= (int64_t(1) << 31) || (dt != PTL_F32 && dt != PTL_BF16)) return 0;
+  const size_t es = dt == PTL_BF16 ? 2 : 4;
+  return 256 + align_up(size_t(max_tokens) * REP_W * es, 256);
+}
+
+ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* bag_offsets,
+                           int64_t total_tokens, ptl_dtype dt, const ptl_rep_encoder_weights* w,
+                           void* out, void* workspace, size_t ws_bytes, void* stream) {
+  if (dt != PTL_F32 && dt != PTL_BF16) return PTL_ERR_DTYPE;
+  if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31) || num_ids < 0) return PTL_ERR_SHAPE;
+  if (!w || !workspace || !bag_offsets || !out) return PTL_ERR_NULL;
+  if (num_ids > 0 && !ids) return PTL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PTL_ERR_ALIGN;
+  if (ws_bytes < ptl_rep_encoder_workspace_size(total_tokens, dt)) return PTL_ERR_WORKSPACE;
+  if (!w->ln_g || !w->ln_b || !w->w) return PTL_ERR_NULL;
+  if (!a16(out) || !a16(w->w) || !a16(w->ln_g) || !a16(w->ln_b) || !a4(bag_offsets) || (ids && !a4(ids)))
+    return PTL_ERR_ALIGN;
+  RepTables tb;
+  for (int s = 0; s < REP_SLOTS; ++s) {
+    if (w->vocab[s] < 0) return PTL_ERR_SHAPE;
+    if (w->vocab[s] > 0 && !w->tables[s]) return PTL_ERR_NULL;
+    if (!a16(w->tables[s])) return PTL_ERR_ALIGN;
+    tb.t[s] = w->tables[s];
+    tb.vocab[s] = w->vocab[s];
+  }
+  if (total_tokens == 0) return PTL_OK;
+  ptl_status s;
+  if ((s = device_ok()) != PTL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* err = reinterpret_cast<int32_t*>(ws);
+  char* normed = ws + 256;
+  const int T = int(total_tokens);
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), st) != cudaSuccess) return PTL_ERR_CUDA;
+  mark(st, PTL_KERNEL_LAYERNORM);
+  PTL_TRY(launch_embag_ln(tb, ids, bag_offsets, num_ids, T, w->ln_g, w->ln_b, normed, dt, err, st));
+  EndMark end_mark{st};
+  if (dt == PTL_BF16) {
+    CUtensorMap ma, mb, mo;
+    if (!map_bf16(&ma, normed, REP_W, uint64_t(T), REP_W * 2, 64, 128)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mb, w->w, REP_W, D, REP_W * 2, 64, 128)) return PTL_ERR_CUDA;
+    if (!map_bf16(&mo, out, D, uint64_t(T), D * 2, 64, 128)) return PTL_ERR_CUDA;
+    mark(st, PTL_KERNEL_GEMM_QKV);
+    PTL_TRY(launch_gemm_rep(ma, mb, mo, w->b, T, err, st));
+  } else {
+    WsLayout L{};  // the fp32 GEMM reads only the error word (offset 0) in this mode
+    mark(st, PTL_KERNEL_GEMM_QKV);
+    PTL_TRY(launch_gemm_f32(0, reinterpret_cast<const float*>(normed), REP_W, F32(w->w), w->b, nullptr,
+                            static_cast<float*>(out), D, T, D, REP_W, L, ws, st));
+  }
   return PTL_OK;
 }
 

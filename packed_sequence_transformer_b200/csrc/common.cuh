@@ -138,6 +138,16 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   return true;
 }
 
+// ---------------------------------------------------------------- RepEncoder
+constexpr int REP_SLOTS = 28;
+constexpr int REP_W = REP_SLOTS * D;  // 14336 values per token
+// The 28 embedding tables (device pointers, [vocab][512] in the build dtype)
+// and their row counts, passed by value to the embedding-bag kernel.
+struct RepTables {
+  const void* t[REP_SLOTS];
+  int64_t vocab[REP_SLOTS];
+};
+
 // ---------------------------------------------------------------- masks
 // HSTU-style attention masks (cry-daniel/recsys README, HSTU attention mask
 // logic).  A user's L tokens are laid out [contextual][historical][candidate]:

@@ -476,6 +476,19 @@ int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorM
   return launch_pair<QKV_BN, G_QKV>(xn, w, qkv_out, p, p.n_tiles_dense, st);
 }
 
+int launch_gemm_rep(const CUtensorMap& normed, const CUtensorMap& w, const CUtensorMap& out_map,
+                    const float* bias, int T, int32_t* err, cudaStream_t st) {
+  GemmTcParams p{};
+  p.M = T;
+  p.N_total = D;
+  p.num_kb = REP_W / 64;
+  p.n_tiles_dense = ((T + 255) / 256) * (D / 256);  // 256-row pair tiles
+  p.bias = bias;
+  p.ldo = D;
+  p.err = err;
+  return launch_pair<256, G_QKV>(normed, w, out_map, p, p.n_tiles_dense, st);
+}
+
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
                     const float* bias, const void* x, void* x1, int T, int32_t* err, cudaStream_t st) {
   GemmTcParams p{};

@@ -1049,6 +1049,102 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
   for (int d = 0; d < DH; ++d) out[size_t(s0 + qi) * D + h * DH + d] = o[d] * inv;
 }
 
+// ------------------------------------------------------ RepEncoder front end
+// The batched embedding bag of the RepEncoder (cti2026 README, RepEncoder
+// section) with its LayerNorm: one block per token, 14 warps; warp w sums
+// (in fp32) the bags of slots w and w + 14, one 512-wide table row per id
+// (each lane two 16-byte pieces of the row, so a warp reads whole rows),
+// then the block takes the mean and the biased variance of the token's
+// 28 x 512 = 14336 sums (two passes over registers) and stores the
+// normalised row in the output dtype.  An id outside its table or a
+// malformed bag range sets PTL_ERR_BAD_IDS and contributes nothing.
+constexpr int REP_WARPS = 14;
+
+template <typename T>
+__global__ void __launch_bounds__(REP_WARPS * 32)
+    embag_ln_kernel(const __grid_constant__ RepTables tb, const int64_t* __restrict__ ids,
+                    const int64_t* __restrict__ off, int64_t n_ids, const float* __restrict__ g,
+                    const float* __restrict__ b, T* __restrict__ out, int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_red[REP_WARPS];
+  __shared__ float s_stat;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t t = blockIdx.x;
+  float v[2][16];
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int sl = warp + REP_WARPS * k;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[k][j] = 0.f;
+    const int64_t b0 = off[t * REP_SLOTS + sl], b1 = off[t * REP_SLOTS + sl + 1];
+    if (b0 < 0 || b1 < b0 || b1 > n_ids) {
+      bad = true;
+      continue;
+    }
+    const T* table = static_cast<const T*>(tb.t[sl]);
+    for (int64_t i = b0; i < b1; ++i) {
+      const int64_t id = __ldg(ids + i);
+      if (id < 0 || id >= tb.vocab[sl]) {
+        bad = true;
+        continue;
+      }
+      float r[16];
+      Row16<T>::load(table + size_t(id) * D, lane, r);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[k][j] += r[j];
+    }
+  }
+  if (bad && lane == 0) set_error(err, PTL_ERR_BAD_IDS);
+  // mean, then the biased variance of the centred values, over 14336
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sum += v[k][j];
+  sum = warp_sum(sum);
+  if (lane == 0) s_red[warp] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = 0.f;
+    for (int w = 0; w < REP_WARPS; ++w) a += s_red[w];
+    s_stat = a * (1.0f / REP_W);
+  }
+  __syncthreads();
+  const float mean = s_stat;
+  float sq = 0.f;
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      v[k][j] -= mean;
+      sq += v[k][j] * v[k][j];
+    }
+  sq = warp_sum(sq);
+  __syncthreads();  // s_stat read by every thread before it is reused
+  if (lane == 0) s_red[warp] = sq;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float a = 0.f;
+    for (int w = 0; w < REP_WARPS; ++w) a += s_red[w];
+    s_stat = rsqrtf(a * (1.0f / REP_W) + LN_EPS);
+  }
+  __syncthreads();
+  const float rstd = s_stat;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int c0 = (warp + REP_WARPS * k) * D;
+    float y[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = c0 + Row16<T>::elem(lane, j);
+      y[j] = v[k][j] * rstd * __ldg(g + c) + __ldg(b + c);
+    }
+    Row16<T>::store(out + t * REP_W + c0, lane, y);
+  }
+}
+
 // ------------------------------------------------------------- launchers
 #define PTL_LAUNCH_CHECK() (cudaPeekAtLastError() == cudaSuccess ? 0 : -1)
 
@@ -1202,6 +1298,19 @@ int launch_combine_f32(const float* y, const float* w, const float* x1, float* o
                        const int32_t* err, cudaStream_t st) {
   const size_t n = size_t(T) * D;
   if (launch_k(combine_f32_kernel, dim3(unsigned((n + 255) / 256)), dim3(256), 0, st, y, w, x1, out, T, err)) return -1;
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_embag_ln(const RepTables& tb, const int64_t* ids, const int64_t* off, int64_t n_ids, int T,
+                    const float* g, const float* b, void* out, ptl_dtype dt, int32_t* err,
+                    cudaStream_t st) {
+  if (dt == PTL_BF16) {
+    if (launch_k(embag_ln_kernel<__nv_bfloat16>, dim3(T), dim3(REP_WARPS * 32), 0, st, tb, ids, off, n_ids, g,
+                 b, static_cast<__nv_bfloat16*>(out), err)) return -1;
+  } else {
+    if (launch_k(embag_ln_kernel<float>, dim3(T), dim3(REP_WARPS * 32), 0, st, tb, ids, off, n_ids, g, b,
+                 static_cast<float*>(out), err)) return -1;
+  }
   return PTL_LAUNCH_CHECK();
 }
 

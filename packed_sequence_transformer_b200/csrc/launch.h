@@ -73,12 +73,20 @@ int launch_combine_f32(const float* y, const float* w, const float* x1, float* o
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
                     const char* ws, cudaStream_t st, const AttnMask* mask = nullptr);
 
+// RepEncoder: embedding bags + LayerNorm(14336) into out [T][14336] (dt)
+int launch_embag_ln(const RepTables& tb, const int64_t* ids, const int64_t* off, int64_t n_ids, int T,
+                    const float* g, const float* b, void* out, ptl_dtype dt, int32_t* err,
+                    cudaStream_t st);
+
 // gemm_tc.cu (bf16, tcgen05).  QKV and the output projection run on CTA
 // pairs: their B (weight) tensor maps have boxes of BN/2 rows.
 int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorMap& qkv_out,
                     const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st);
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
                     const float* bias, const void* x, void* x1, int T, int32_t* err, cudaStream_t st);
+// RepEncoder Linear: out [T][512] = normed [T][14336] W^T + b (256 x 256 pair tiles)
+int launch_gemm_rep(const CUtensorMap& normed, const CUtensorMap& w, const CUtensorMap& out_map,
+                    const float* bias, int T, int32_t* err, cudaStream_t st);
 int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf_out,
                      const float* b1, const WsLayout& L, char* ws, cudaStream_t st);
 // Both expert GEMMs in one persistent launch (first-GEMM tiles, then

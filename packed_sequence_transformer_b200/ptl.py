@@ -22,7 +22,7 @@ PTL_F32, PTL_BF16 = 0, 1
 STATUS = {
     0: "PTL_OK", 1: "PTL_ERR_NULL", 2: "PTL_ERR_ALIGN", 3: "PTL_ERR_SHAPE",
     4: "PTL_ERR_BAD_OFFSETS", 5: "PTL_ERR_WORKSPACE", 6: "PTL_ERR_DTYPE", 7: "PTL_ERR_CUDA",
-    8: "PTL_ERR_TIMEOUT", 9: "PTL_ERR_UNSUPPORTED", 10: "PTL_ERR_BAD_MASK",
+    8: "PTL_ERR_TIMEOUT", 9: "PTL_ERR_UNSUPPORTED", 10: "PTL_ERR_BAD_MASK", 11: "PTL_ERR_BAD_IDS",
 }
 STATUS_CODE = {v: k for k, v in STATUS.items()}
 
@@ -59,6 +59,12 @@ class AttnMaskStruct(ctypes.Structure):
                 ("window", ctypes.c_int32)]
 
 
+class RepWeightsStruct(ctypes.Structure):
+    _fields_ = [("tables", ctypes.c_void_p * 28), ("vocab", ctypes.c_int64 * 28),
+                ("ln_g", ctypes.c_void_p), ("ln_b", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("b", ctypes.c_void_p)]
+
+
 class Trace(ctypes.Structure):
     _fields_ = [("events", ctypes.POINTER(ctypes.c_void_p)), ("kinds", ctypes.POINTER(ctypes.c_int32)),
                 ("capacity", ctypes.c_int32), ("count", ctypes.c_int32)]
@@ -91,6 +97,10 @@ _SIGS = {
     "ptl_attention_masked": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                               ctypes.c_int64, ctypes.c_int, ctypes.POINTER(AttnMaskStruct),
                               ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
+    "ptl_rep_encoder_workspace_size": ([ctypes.c_int64, ctypes.c_int], ctypes.c_size_t),
+    "ptl_rep_encoder": ([ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                         ctypes.POINTER(RepWeightsStruct), ctypes.c_void_p, ctypes.c_void_p,
+                         ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
     "ptl_out_projection": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                             ctypes.c_int, ctypes.POINTER(LayerWeights), ctypes.c_void_p,
                             ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
@@ -284,6 +294,35 @@ def attention_masked(qkv, attn, cu_seqlens, workspace, causal=True, num_contexts
                                       qkv.shape[0], _dt(qkv.dtype), ctypes.byref(m), _ptr(workspace),
                                       workspace.numel(), _stream(stream)), "ptl_attention_masked")
     return attn
+
+
+def rep_encoder_workspace(max_tokens: int, dtype, device="cuda") -> torch.Tensor:
+    n = int(lib().ptl_rep_encoder_workspace_size(int(max_tokens), _dt(dtype)))
+    if n == 0:
+        raise ValueError("invalid RepEncoder workspace request")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def rep_weights_struct(tables, ln_g, ln_b, w, b=None) -> RepWeightsStruct:
+    """28 device tables [vocab_s, 512] (dt), LN params [14336] (f32), W [512, 14336] (dt), b [512] (f32)."""
+    if len(tables) != 28:
+        raise ValueError("the RepEncoder has 28 slots")
+    st = RepWeightsStruct()
+    for i, t in enumerate(tables):
+        st.tables[i] = t.data_ptr() if t.numel() else 0
+        st.vocab[i] = t.shape[0]
+    st.ln_g, st.ln_b, st.w = ln_g.data_ptr(), ln_b.data_ptr(), w.data_ptr()
+    st.b = b.data_ptr() if b is not None else None
+    return st
+
+
+def rep_encoder(ids, bag_offsets, num_tokens, weights: RepWeightsStruct, out, workspace, stream=None):
+    """RepEncoder front end (``ptl_rep_encoder``): embedding bags, LayerNorm
+    over 14336, Linear to 512 into out [T, 512] (dt of out)."""
+    _check(lib().ptl_rep_encoder(_ptr(ids), ids.numel(), _ptr(bag_offsets), int(num_tokens), _dt(out.dtype),
+                                 ctypes.byref(weights), _ptr(out), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "ptl_rep_encoder")
+    return out
 
 
 def out_projection(attn, x, x1, weights, workspace, stream=None):

@@ -168,3 +168,28 @@ def test_attention_masked_host_checks(P):
     assert L.ptl_attention_masked(FAKE, FAKE, FAKE, 4, 64, 1, ctypes.byref(mis), FAKE, ws_b,
                                   None) == S["PTL_ERR_ALIGN"]
     assert P.status_string(S["PTL_ERR_BAD_MASK"]).startswith("attention mask")
+
+
+def test_rep_encoder_host_checks(P):
+    L = P.lib()
+    S = P.STATUS_CODE
+    assert L.ptl_rep_encoder_workspace_size(100, 1) == 256 + ((100 * 14336 * 2 + 255) // 256) * 256
+    assert L.ptl_rep_encoder_workspace_size(-1, 1) == 0
+    assert L.ptl_rep_encoder_workspace_size(10, 5) == 0
+    w = P.RepWeightsStruct()
+    for i in range(28):
+        w.tables[i] = FAKE
+        w.vocab[i] = 10
+    w.ln_g = w.ln_b = w.w = FAKE
+    ws_b = L.ptl_rep_encoder_workspace_size(64, 1)
+    ok = ctypes.byref(w)
+    assert L.ptl_rep_encoder(FAKE, 10, FAKE, 64, 7, ok, FAKE, FAKE, ws_b, None) == S["PTL_ERR_DTYPE"]
+    assert L.ptl_rep_encoder(FAKE, 10, None, 64, 1, ok, FAKE, FAKE, ws_b, None) == S["PTL_ERR_NULL"]
+    assert L.ptl_rep_encoder(FAKE, 10, FAKE, 64, 1, ok, FAKE, FAKE, 16, None) == S["PTL_ERR_WORKSPACE"]
+    assert L.ptl_rep_encoder(FAKE, 10, FAKE, 64, 1, ok, FAKE + 8, FAKE, ws_b, None) == S["PTL_ERR_ALIGN"]
+    assert L.ptl_rep_encoder(FAKE, 10, FAKE, 0, 1, ok, FAKE, FAKE, ws_b, None) == S["PTL_OK"]
+    w.vocab[3] = -1
+    assert L.ptl_rep_encoder(FAKE, 10, FAKE, 64, 1, ok, FAKE, FAKE, ws_b, None) == S["PTL_ERR_SHAPE"]
+    w.vocab[3] = 10
+    w.tables[4] = None
+    assert L.ptl_rep_encoder(FAKE, 10, FAKE, 64, 1, ok, FAKE, FAKE, ws_b, None) == S["PTL_ERR_NULL"]
