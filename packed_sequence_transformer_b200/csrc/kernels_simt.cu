@@ -1051,98 +1051,131 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__
 
 // ------------------------------------------------------ RepEncoder front end
 // The batched embedding bag of the RepEncoder (cti2026 README, RepEncoder
-// section) with its LayerNorm: one block per token, 14 warps; warp w sums
-// (in fp32) the bags of slots w and w + 14, one 512-wide table row per id
-// (each lane two 16-byte pieces of the row, so a warp reads whole rows),
-// then the block takes the mean and the biased variance of the token's
-// 28 x 512 = 14336 sums (two passes over registers) and stores the
-// normalised row in the output dtype.  An id outside its table or a
-// malformed bag range sets PTL_ERR_BAD_IDS and contributes nothing.
-constexpr int REP_WARPS = 14;
+// section) with its LayerNorm.  Blocks of 28 warps, one warp per slot, loop
+// over tokens (token t = block, block + grid, ...), so each warp keeps its
+// slot's LayerNorm scale and shift (its lane's 16 columns) in registers for
+// the whole launch instead of re-reading 14336 x 8 bytes per token.  Per
+// token a warp loads up to 32 of its bag's ids at once (coalesced), shuffles
+// them to every lane and keeps DEPTH table rows in flight (each lane two
+// 16-byte pieces of a 512-wide row, so a warp reads whole rows), summing in
+// fp32 in bag order; the block then takes the mean and the biased variance
+// of the token's 28 x 512 = 14336 sums (two passes over registers) and
+// stores the normalised row in the output dtype.  An id outside its table or
+// a malformed bag range sets PTL_ERR_BAD_IDS and contributes nothing.
+constexpr int REP_WARPS = REP_SLOTS;
 
 template <typename T>
 __global__ void __launch_bounds__(REP_WARPS * 32)
     embag_ln_kernel(const __grid_constant__ RepTables tb, const int64_t* __restrict__ ids,
-                    const int64_t* __restrict__ off, int64_t n_ids, const float* __restrict__ g,
+                    const int64_t* __restrict__ off, int64_t n_ids, int T_, const float* __restrict__ g,
                     const float* __restrict__ b, T* __restrict__ out, int32_t* err) {
   pdl_wait();
   pdl_trigger();
   __shared__ float s_red[REP_WARPS];
   __shared__ float s_stat;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t t = blockIdx.x;
-  float v[2][16];
+  const int sl = threadIdx.x >> 5, lane = threadIdx.x & 31;  // warp = slot
+  constexpr int NP = sizeof(T) == 2 ? 2 : 4;      // 16-byte pieces of a lane's 16 values
+  constexpr int DEPTH = 1;                        // rows per step (the token loop keeps many warps busy)
+  constexpr int ROW16 = D * int(sizeof(T)) / 16;  // 16-byte pieces per table row
+  const int c0 = sl * D;
+  float gs[16], bs[16];  // this lane's LayerNorm scale and shift, for every token
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int c = c0 + Row16<T>::elem(lane, j);
+    gs[j] = __ldg(g + c);
+    bs[j] = __ldg(b + c);
+  }
+  const uint4* table = static_cast<const uint4*>(tb.t[sl]);
+  const int64_t vocab = tb.vocab[sl];
   bool bad = false;
+  for (int t = blockIdx.x; t < T_; t += gridDim.x) {
+    float v[16];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int sl = warp + REP_WARPS * k;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[k][j] = 0.f;
-    const int64_t b0 = off[t * REP_SLOTS + sl], b1 = off[t * REP_SLOTS + sl + 1];
+    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+    const int64_t b0 = off[size_t(t) * REP_SLOTS + sl], b1 = off[size_t(t) * REP_SLOTS + sl + 1];
     if (b0 < 0 || b1 < b0 || b1 > n_ids) {
       bad = true;
-      continue;
-    }
-    const T* table = static_cast<const T*>(tb.t[sl]);
-    for (int64_t i = b0; i < b1; ++i) {
-      const int64_t id = __ldg(ids + i);
-      if (id < 0 || id >= tb.vocab[sl]) {
-        bad = true;
-        continue;
-      }
-      float r[16];
-      Row16<T>::load(table + size_t(id) * D, lane, r);
+    } else {
+      for (int64_t base = b0; base < b1; base += 32) {
+        const int64_t i = base + lane;
+        int64_t my = i < b1 ? __ldg(ids + i) : 0;
+        const bool my_bad = i < b1 && (my < 0 || my >= vocab);
+        if (__any_sync(0xffffffffu, my_bad)) bad = true;
+        if (my_bad) my = -1;
+        const int cnt = b1 - base < 32 ? int(b1 - base) : 32;
+        for (int j = 0; j < cnt; j += DEPTH) {
+          int64_t idq[DEPTH];
+          uint4 raw[DEPTH][NP];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[k][j] += r[j];
+          for (int q = 0; q < DEPTH; ++q) idq[q] = __shfl_sync(0xffffffffu, my, j + q);
+#pragma unroll
+          for (int q = 0; q < DEPTH; ++q)
+            if (j + q < cnt && idq[q] >= 0) {
+              const uint4* row = table + size_t(idq[q]) * ROW16;
+#pragma unroll
+              for (int pc = 0; pc < NP; ++pc) raw[q][pc] = __ldg(row + pc * 32 + lane);
+            }
+#pragma unroll
+          for (int q = 0; q < DEPTH; ++q)
+            if (j + q < cnt && idq[q] >= 0) {
+#pragma unroll
+              for (int pc = 0; pc < NP; ++pc) {
+                if constexpr (sizeof(T) == 2) {
+                  const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[q][pc]);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    v[pc * 8 + 2 * e] += f.x;
+                    v[pc * 8 + 2 * e + 1] += f.y;
+                  }
+                } else {
+                  v[pc * 4 + 0] += __uint_as_float(raw[q][pc].x);
+                  v[pc * 4 + 1] += __uint_as_float(raw[q][pc].y);
+                  v[pc * 4 + 2] += __uint_as_float(raw[q][pc].z);
+                  v[pc * 4 + 3] += __uint_as_float(raw[q][pc].w);
+                }
+              }
+            }
+        }
+      }
     }
+    // mean, then the biased variance of the centred values, over 14336
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sum += v[j];
+    sum = warp_sum(sum);
+    if (lane == 0) s_red[sl] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float a = 0.f;
+      for (int w = 0; w < REP_WARPS; ++w) a += s_red[w];
+      s_stat = a * (1.0f / REP_W);
+    }
+    __syncthreads();
+    const float mean = s_stat;
+    float sq = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      v[j] -= mean;
+      sq += v[j] * v[j];
+    }
+    sq = warp_sum(sq);
+    __syncthreads();  // s_stat and s_red read by every thread before they are reused
+    if (lane == 0) s_red[sl] = sq;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float a = 0.f;
+      for (int w = 0; w < REP_WARPS; ++w) a += s_red[w];
+      s_stat = rsqrtf(a * (1.0f / REP_W) + LN_EPS);
+    }
+    __syncthreads();
+    const float rstd = s_stat;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = v[j] * rstd * gs[j] + bs[j];
+    Row16<T>::store(out + size_t(t) * REP_W + c0, lane, v);
+    __syncthreads();  // s_stat is rewritten by the next token
   }
   if (bad && lane == 0) set_error(err, PTL_ERR_BAD_IDS);
-  // mean, then the biased variance of the centred values, over 14336
-  float sum = 0.f;
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-#pragma unroll
-    for (int j = 0; j < 16; ++j) sum += v[k][j];
-  sum = warp_sum(sum);
-  if (lane == 0) s_red[warp] = sum;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float a = 0.f;
-    for (int w = 0; w < REP_WARPS; ++w) a += s_red[w];
-    s_stat = a * (1.0f / REP_W);
-  }
-  __syncthreads();
-  const float mean = s_stat;
-  float sq = 0.f;
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      v[k][j] -= mean;
-      sq += v[k][j] * v[k][j];
-    }
-  sq = warp_sum(sq);
-  __syncthreads();  // s_stat read by every thread before it is reused
-  if (lane == 0) s_red[warp] = sq;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float a = 0.f;
-    for (int w = 0; w < REP_WARPS; ++w) a += s_red[w];
-    s_stat = rsqrtf(a * (1.0f / REP_W) + LN_EPS);
-  }
-  __syncthreads();
-  const float rstd = s_stat;
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int c0 = (warp + REP_WARPS * k) * D;
-    float y[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int c = c0 + Row16<T>::elem(lane, j);
-      y[j] = v[k][j] * rstd * __ldg(g + c) + __ldg(b + c);
-    }
-    Row16<T>::store(out + t * REP_W + c0, lane, y);
-  }
 }
 
 // ------------------------------------------------------------- launchers
@@ -1304,11 +1337,13 @@ int launch_combine_f32(const float* y, const float* w, const float* x1, float* o
 int launch_embag_ln(const RepTables& tb, const int64_t* ids, const int64_t* off, int64_t n_ids, int T,
                     const float* g, const float* b, void* out, ptl_dtype dt, int32_t* err,
                     cudaStream_t st) {
+  // blocks loop over tokens: one resident block per SM
+  const int grid = T < num_sms() ? T : num_sms();
   if (dt == PTL_BF16) {
-    if (launch_k(embag_ln_kernel<__nv_bfloat16>, dim3(T), dim3(REP_WARPS * 32), 0, st, tb, ids, off, n_ids, g,
-                 b, static_cast<__nv_bfloat16*>(out), err)) return -1;
+    if (launch_k(embag_ln_kernel<__nv_bfloat16>, dim3(grid), dim3(REP_WARPS * 32), 0, st, tb, ids, off, n_ids, T,
+                 g, b, static_cast<__nv_bfloat16*>(out), err)) return -1;
   } else {
-    if (launch_k(embag_ln_kernel<float>, dim3(T), dim3(REP_WARPS * 32), 0, st, tb, ids, off, n_ids, g, b,
+    if (launch_k(embag_ln_kernel<float>, dim3(grid), dim3(REP_WARPS * 32), 0, st, tb, ids, off, n_ids, T, g, b,
                  static_cast<float*>(out), err)) return -1;
   }
   return PTL_LAUNCH_CHECK();
