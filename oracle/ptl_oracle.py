@@ -281,6 +281,50 @@ def rep_encoder(tables, ids, bag_offsets, num_tokens, ln_g, ln_b, w, b=None, sto
 
 
 # --------------------------------------------------------------------------
+# FP8 (e4m3) GEMM operands (cry-daniel/recsys README: FP8 among the listed
+# optimisations; CTI-Inference-Opt optimisation plan, INT8 quantisation
+# section, as the motivation for low-precision expert and QKV GEMMs)
+# --------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x):
+    """Nearest e4m3 value (1 sign, 4 exponent bits with bias 7, 3 mantissa
+    bits, no infinities: largest finite 448), ties to even, saturating at
+    +-448.  Normal binade [2^E, 2^(E+1)) for E >= -6 has spacing 2^(E-3);
+    below 2^-6 the subnormal spacing is 2^-9."""
+    x = _f64(x)
+    a = np.abs(x)
+    with np.errstate(divide="ignore"):
+        E = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    quantum = np.where(a >= 2.0 ** -6, 2.0 ** (np.maximum(E, -6) - 3), 2.0 ** -9)
+    q = np.round(a / quantum) * quantum  # numpy rounds half to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.sign(x) * q
+
+
+def quantize_rows_e4m3(x):
+    """Per-row scaled e4m3: s = max|row| / 448 (1 for an all-zero row),
+    codes = quantize_e4m3(row / s); returns (codes, s) with row ~ codes * s."""
+    x = _f64(x)
+    amax = np.abs(x).max(axis=-1, keepdims=True)
+    s = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    return quantize_e4m3(x / s), s[..., 0]
+
+
+def linear_fp8(x, weight, bias=None):
+    """y = x W^T + b with both operands quantised per row (rows of x = tokens,
+    rows of W = output channels) to e4m3; the products of the codes are summed
+    exactly (fp64 here; fp32 on the tensor cores) and scaled by s_x[i] s_w[j]."""
+    qx, sx = quantize_rows_e4m3(x)
+    qw, sw = quantize_rows_e4m3(weight)
+    y = (qx @ qw.T) * sx[:, None] * sw[None, :]
+    if bias is not None:
+        y = y + _f64(bias)
+    return y
+
+
+# --------------------------------------------------------------------------
 # Gate (cti2026 README, SMoE structure: softmax -> top-2 -> renormalise)
 # --------------------------------------------------------------------------
 def gate_probs(xn2, w_gate, b_gate):

@@ -171,3 +171,33 @@ def test_layer_norm_per_slot_instead_of_whole_row_is_caught(monkeypatch):
         return np.concatenate(parts, axis=-1)
     monkeypatch.setattr(O, "layer_norm", per_slot)
     assert _fails(PR.test_front_end_is_torch_layer_norm_and_linear)
+
+
+# ------------------------------------------------- FP8 (e4m3) operands
+import tests.test_oracle_fp8 as P8  # noqa: E402
+
+
+def _e4m3_mutant(mant_bits=3, tie_even=True, saturate=True, sub_exp=-9):
+    def q(x):
+        x = np.asarray(x, np.float64)
+        a = np.abs(x)
+        with np.errstate(divide="ignore"):
+            E = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+        quantum = np.where(a >= 2.0 ** -6, 2.0 ** (np.maximum(E, -6) - mant_bits), 2.0 ** sub_exp)
+        r = np.round(a / quantum) if tie_even else np.floor(a / quantum + 0.5)
+        r = r * quantum
+        if saturate:
+            r = np.minimum(r, 448.0)
+        return np.sign(x) * r
+    return q
+
+
+@pytest.mark.parametrize("kw", [dict(mant_bits=4), dict(tie_even=False), dict(sub_exp=-10)])
+def test_e4m3_rounding_slips_are_caught(monkeypatch, kw):
+    monkeypatch.setattr(O, "quantize_e4m3", _e4m3_mutant(**kw))
+    assert _fails(P8.test_rounding_matches_torch_float8_e4m3fn)
+
+
+def test_missing_saturation_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "quantize_e4m3", _e4m3_mutant(saturate=False))
+    assert _fails(P8.test_value_set_and_extremes)
