@@ -145,7 +145,7 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
                              float* probs, int32_t* n_pred, void* workspace, size_t ws_bytes,
                              void* stream);
 
-/* ---- The layer's steps, one entry point each (the pages' operator
+/* ---- The layer's steps, one entry point each (the cti2026 README's operator
  * interface: Linear_qkv, FlashAttention_Varlen(qkv, user_offsets),
  * Linear_out + residual, Gate(x) -> (topk_idx, topk_weight),
  * FusedMoE(x, topk_idx, topk_weight) + residual, Prediction Head). ---- */

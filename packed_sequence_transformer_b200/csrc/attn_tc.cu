@@ -101,13 +101,12 @@ __device__ __forceinline__ int keys16(int L, int kb) {
   return (k + 15) & ~15;
 }
 
-// The interleaved step sequence both the producer and the MMA issuer walk.
+// One stream's position in the step sequence that the producer and the MMA
+// issuers walk, plus (for the producer) whether the unit's Q load is issued.
 // Each stream's next unit is looked up one unit ahead, so switching units
-// does not wait on the work-list and offset loads.
-// One stream's position in its step sequence, plus (for the MMA issuer) its
-// deferred PV and (for the producer) whether the unit's Q load is issued.
-// The two streams are held in named registers, never indexed by the stream
-// number, so nothing lands in local memory.
+// does not wait on the unit list.  The two streams are held in named
+// registers, never indexed by the stream number, so nothing lands in local
+// memory.
 struct StreamPos {
   int g;             // the stream (softmax warpgroup)
   int kb, n, uc;     // key block of the current unit, steps so far, units started
@@ -115,14 +114,7 @@ struct StreamPos {
   AttnUnit u, nxt;   // current unit, the next one (looked up one unit ahead)
   const int4* list;  // this stream's units, in order
   int n_list, k_list;  // list length, next entry to read
-  // the MMA issuer's queue of steps whose PV is still to be issued (oldest
-  // first; -1: none): a step's QK^T may go ahead of the previous step's PV
-  int pv_n, pv_k16, pv_uc;
-  bool pv_first;
-  int pv2_n, pv2_k16, pv2_uc;
-  bool pv2_first;
   bool q_sent;       // producer: the current unit's Q tile load is issued
-  bool k_sent;       // producer: the current step's K tile load is issued
 };
 
 // Both streams' step sequences as the producer and the MMA issuer walk them
@@ -144,11 +136,7 @@ struct AttnStepGen {
     sp.list = ulist + uoff[2 * blockIdx.x + g];
     sp.n_list = n_ok ? ucnt[2 * blockIdx.x + g] : 0;
     sp.k_list = 0;
-    sp.pv_n = sp.pv2_n = -1;
-    sp.pv_k16 = sp.pv_uc = sp.pv2_k16 = sp.pv2_uc = 0;
-    sp.pv_first = sp.pv2_first = false;
     sp.q_sent = false;
-    sp.k_sent = false;
     fetch_next(sp);
     sp.live = sp.nxt_live;
     sp.u = sp.nxt;

@@ -9,7 +9,7 @@ Workload shapes follow the cti2026 README (Days-gone/cti2026): d_model 512,
 8 heads x 64, QKV 512->1536, 8 ReLU experts 512->1024->512, top-2 gating,
 many users packed end to end with ``user_offsets`` boundaries, 1221-10793
 tokens per batch and about 44k tokens as the point where a dense [S,S] mask
-no longer fits.  The competition data the pages measured on is not
+no longer fits.  The competition data the README measured on is not
 available; these generators stand in for it.
 
 Draw order for one case (all from ``numpy.random.default_rng(seed)``, PCG64,
