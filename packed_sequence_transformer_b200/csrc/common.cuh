@@ -166,7 +166,7 @@ struct AttnMask {
   int32_t window;      // > 0: sliding window; <= 0: none
 };
 
-__device__ __forceinline__ bool mask_visible(int i, int j, int C, int Hs, const AttnMask& m) {
+__host__ __device__ __forceinline__ bool mask_visible(int i, int j, int C, int Hs, const AttnMask& m) {
   bool v = m.causal ? j <= i : true;
   v = v || (i < C && j < C);
   if (j >= Hs) v = v && i >= Hs && (i - Hs) / m.group == (j - Hs) / m.group;
@@ -180,7 +180,7 @@ __device__ __forceinline__ bool mask_visible(int i, int j, int C, int Hs, const 
 // first candidate; a candidate row sees [0, Hs - 1] and, second, its own
 // group up to itself (causal) or to the group's end.  Both are then cut to
 // the window.  The same set as mask_visible, for every i < L.
-__device__ __forceinline__ void mask_row_intervals(int i, int L, int C, int Hs, const AttnMask& m,
+__host__ __device__ __forceinline__ void mask_row_intervals(int i, int L, int C, int Hs, const AttnMask& m,
                                                    int& a0, int& b0, int& a1, int& b1) {
   a0 = 0;
   a1 = 1;
@@ -205,7 +205,7 @@ __device__ __forceinline__ void mask_row_intervals(int i, int L, int C, int Hs, 
 }
 
 // Bits k (0..31) set where j0 + k lies in [a, b].
-__device__ __forceinline__ uint32_t interval_bits32(int a, int b, int j0) {
+__host__ __device__ __forceinline__ uint32_t interval_bits32(int a, int b, int j0) {
   int lo = a - j0, hi = b - j0 + 1;  // bits [lo, hi)
   lo = lo > 0 ? lo : 0;
   hi = hi < 32 ? hi : 32;
@@ -216,7 +216,7 @@ __device__ __forceinline__ uint32_t interval_bits32(int a, int b, int j0) {
 
 // Keys [lo_key, hi_key] that hold every key visible to some query of block b
 // (queries q0 .. q1 of the user): the range the key loop walks.
-__device__ __forceinline__ void mask_key_range(int b, int L, int C, int Hs, const AttnMask& m,
+__host__ __device__ __forceinline__ void mask_key_range(int b, int L, int C, int Hs, const AttnMask& m,
                                                int& lo_key, int& hi_key) {
   const int q0 = b * ATT_BLK;
   const int q1 = q0 + ATT_BLK - 1 < L - 1 ? q0 + ATT_BLK - 1 : L - 1;
