@@ -7,7 +7,11 @@ helpers are host-callable, so this test compiles a small host program against
 the library's own header and compares, for every small user shape and mask
 setting, (a) the interval words with the key-by-key predicate `mask_visible`,
 (b) that predicate with the oracle's mask, and (c) that every visible key of
-a query block lies inside the block's key range.  No GPU needed (nvcc only)."""
+a query block lies inside the block's key range.  A second host program
+checks the workspace layout (`make_layout`) over many batch shapes: every
+region 256-byte aligned and disjoint, the no-alloc scratch and the per-call
+clear ending where the kernels expect, the fused expert rows fitting.  No GPU
+needed (nvcc only)."""
 import os
 import shutil
 import subprocess
@@ -105,3 +109,71 @@ def test_interval_words_predicate_and_key_ranges_agree_with_the_oracle(harness):
         assert np.array_equal(got, want), c
         n_checked += 1
     assert n_checked == len(cases) > 500
+
+
+LAYOUT_HARNESS = r'''
+#include <cstdio>
+#include <vector>
+#include <algorithm>
+#include "common.cuh"
+using namespace ptl;
+// For each (T, U, dtype): print "OK" or the first broken invariant of the
+// workspace layout.
+int main() {
+  long long T; int U, dt;
+  while (scanf("%lld %d %d", &T, &U, &dt) == 3) {
+    WsLayout L;
+    if (!make_layout(T, U, dt ? PTL_BF16 : PTL_F32, &L)) { printf("REJECT\n"); continue; }
+    const size_t es = dt ? 2 : 4;
+    struct R { size_t off, bytes; const char* name; };
+    std::vector<R> r = {
+      {L.err, 4, "err"}, {L.items, 8 * (size_t)L.max_items, "items"}, {L.item_count, 4, "item_count"},
+      {L.lvl_hist, 4 * (size_t)(L.max_levels + 1), "lvl_hist"}, {L.lvl_start, 4 * (size_t)(L.max_levels + 1), "lvl_start"},
+      {L.lvl_fill, 4 * (size_t)(L.max_levels + 1), "lvl_fill"}, {L.ulist, 16 * (size_t)L.max_items * H, "ulist"},
+      {L.uoff, 8 * ATT_MAX_CTAS, "uoff"}, {L.ucnt, 8 * ATT_MAX_CTAS, "ucnt"},
+      {L.chunk_cnt, 4 * (size_t)L.n_chunks * E, "chunk_cnt"}, {L.lb, 4 * (32 + 32 * (size_t)L.n_gchunks), "lb"},
+      {L.moe_done, 4 * (size_t)L.max_tiles, "moe_done"},
+      {L.xn, es * T * D, "xn"}, {L.qkv, es * T * QKV_N, "qkv"}, {L.attn, es * T * D, "attn"},
+      {L.x1, 4 * T * D, "x1"}, {L.xn2, es * T * D, "xn2"}, {L.act0, es * T * D, "act0"}, {L.act1, es * T * D, "act1"},
+      {L.idx, 4 * T * K, "idx"}, {L.wgt, 4 * T * K, "wgt"}, {L.perm, 8 * T, "perm"}, {L.pos, 8 * T, "pos"},
+      {L.rowroute, 4 * (size_t)L.padded_rows, "rowroute"}, {L.tiles, 8 * (size_t)L.max_tiles, "tiles"},
+      {L.route_meta, 128, "route_meta"}, {L.hbuf, es * (size_t)L.padded_rows * F, "hbuf"},
+      {L.ybuf, dt ? 2 * (size_t)L.padded_rows * D : 4 * 2 * T * D, "ybuf"}, {L.head_p, 4 * T, "head_p"}};
+    if (dt) r.push_back({L.xperm, 2 * (size_t)L.padded_rows * D, "xperm"});
+    const char* bad = nullptr;
+    for (auto& x : r) {
+      if (x.off % 256 != 0) bad = x.name;
+      if (x.off + x.bytes > L.total) bad = x.name;
+    }
+    std::sort(r.begin(), r.end(), [](const R& a, const R& b) { return a.off < b.off; });
+    for (size_t i = 1; i < r.size(); ++i)
+      if (r[i - 1].bytes && r[i - 1].off + r[i - 1].bytes > r[i].off) bad = r[i].name;
+    // the no-alloc scratch holds [0, wl_end): the error word and the work list
+    if (L.wl_end < L.ucnt + 8 * ATT_MAX_CTAS || L.wl_end > L.chunk_cnt) bad = "wl_end";
+    // one memset per call clears [0, clear_end): up to the fused path's counters
+    if (L.clear_end < L.moe_done + 4 * (size_t)L.max_tiles || L.clear_end > L.xn) bad = "clear_end";
+    // the fused expert path puts expert e's rows at e * cap
+    if ((int64_t)E * L.cap > L.padded_rows || L.cap < T || L.cap % MOE_BM) bad = "cap";
+    // work-list bound: every user's query blocks fit
+    if (L.max_items < (T + ATT_BLK - 1) / ATT_BLK + std::min<long long>(U, T)) bad = "max_items";
+    printf(bad ? "BAD %s\n" : "OK\n", bad);
+  }
+  return 0;
+}
+'''
+
+
+def test_workspace_layout_invariants(tmp_path):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    src = tmp_path / "layout.cu"
+    src.write_text(LAYOUT_HARNESS)
+    exe = tmp_path / "layout"
+    subprocess.check_call([nvcc, "-std=c++17", "-O1", "-I", CSRC, "-o", str(exe), str(src)])
+    shapes = [(T, U, dt) for T in (0, 1, 2, 127, 128, 129, 255, 256, 257, 1000, 6823, 6912, 44000, 65536, 1 << 20)
+              for U in (1, 2, 60, 390, 4096) for dt in (0, 1)]
+    inp = "\n".join(f"{T} {U} {dt}" for T, U, dt in shapes) + "\n"
+    out = subprocess.run([str(exe)], input=inp, capture_output=True, text=True, check=True).stdout.split("\n")
+    bad = [(s, o) for s, o in zip(shapes, out) if o != "OK"]
+    assert not bad, bad[:5]
