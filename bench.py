@@ -44,10 +44,11 @@ RUNNER_STRIDE = 128  # token granule of the graph runner's buckets in the end-to
 # (profiles/*_stack8_6823tok.md; ncu flushes caches between replays, so these
 # are cold-cache figures).  A kernel changed since its capture must be
 # recaptured or dropped from this table.
+# The expert GEMM launch, the gate + route kernel and the attention changed
+# after their capture (the first two now wait through the shared bounded-wait
+# helper, the attention is templated on the mask), so they report no traffic
+# until they are captured again.
 NCU_DRAM_BYTES = {
-    "gemm_expert1": 31.801856e6 + 3.954432e6,  # both expert GEMMs in one launch
-    "attention": 21.015040e6,
-    "gate": 14.079488e6 + 0.037376e6,          # gate + route builder
     "gemm_qkv": 8.589312e6,
     "gemm_out": 14.527488e6,
     "combine": 28.068096e6 + 0.002048e6,
