@@ -409,7 +409,11 @@ ptl_status ptl_last_device_error(void* workspace, size_t ws_bytes, void* stream)
 /* Static text for a status code. */
 const char* ptl_status_string(ptl_status s);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor); PTL_VERSION is the value this
+ * header describes.  Minor 1 added the graph runner, the masked attention, the
+ * RepEncoder front end, the wait self-test and the PTL_ERR_BAD_MASK /
+ * PTL_ERR_BAD_IDS codes. */
+#define PTL_VERSION 101
 int32_t ptl_version(void);
 
 #ifdef __cplusplus

@@ -348,7 +348,7 @@ ptl_status setup(Call* c, int64_t T, int32_t U, ptl_dtype dt, void* ws, size_t w
 
 extern "C" {
 
-int32_t ptl_version(void) { return 100; }
+int32_t ptl_version(void) { return PTL_VERSION; }
 
 void ptl_set_trace(ptl_trace* trace) { g_trace = trace; }
 

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(P):
 
 
 def test_status_strings_and_version(P):
-    assert P.version() == 100
+    assert P.version() == 101
     for code in range(10):
         assert P.status_string(code)
     assert P.status_string(99) == "unknown status"
@@ -193,3 +193,8 @@ def test_rep_encoder_host_checks(P):
     w.vocab[3] = 10
     w.tables[4] = None
     assert L.ptl_rep_encoder(FAKE, 10, FAKE, 64, 1, ok, FAKE, FAKE, ws_b, None) == S["PTL_ERR_NULL"]
+
+
+def test_version_matches_header(P):
+    hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ptl.h")).read()
+    assert P.lib().ptl_version() == int(re.search(r"#define PTL_VERSION (\d+)", hdr).group(1)) == 101
