@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/ptl.h"
 #include "common.cuh"
@@ -115,7 +116,9 @@ ptl_status check_head(const ptl_head_weights* h) {
 thread_local ptl_trace* g_trace = nullptr;
 
 // Records the trace event that opens a launch of `kind` (no-op without a trace).
+void nvtx_kernel(int kind);
 inline void mark(cudaStream_t st, int kind) {
+  nvtx_kernel(kind);
   ptl_trace* t = g_trace;
   if (!t || !t->events || t->count >= t->capacity) return;
   // inside a stream capture only an external record becomes an event node
@@ -129,6 +132,47 @@ inline void mark(cudaStream_t st, int kind) {
   if (t->kinds) t->kinds[t->count] = kind;
   ++t->count;
 }
+
+// NVTX annotations (NVTX3, header-only: each call is a no-op unless a
+// profiler is attached).  Every entry point opens a range named after itself
+// and, nested in it, one range per kernel launch named by the launch's kind,
+// so a profiler can attribute and filter the library's kernels; the
+// entry point's guard closes both on every return path.
+const char* kind_name(int kind) {
+  switch (kind) {
+    case PTL_KERNEL_CLEAR: return "clear";
+    case PTL_KERNEL_WORKLIST: return "worklist";
+    case PTL_KERNEL_LAYERNORM: return "layernorm";
+    case PTL_KERNEL_GEMM_QKV: return "gemm_qkv";
+    case PTL_KERNEL_ATTENTION: return "attention";
+    case PTL_KERNEL_GEMM_OUT: return "gemm_out";
+    case PTL_KERNEL_GATE: return "gate";
+    case PTL_KERNEL_ROUTE: return "route";
+    case PTL_KERNEL_GEMM_EXPERT1: return "gemm_expert1";
+    case PTL_KERNEL_GEMM_EXPERT2: return "gemm_expert2";
+    case PTL_KERNEL_HEAD: return "head";
+    case PTL_KERNEL_COPY: return "copy";
+    case PTL_KERNEL_COMBINE: return "combine";
+    default: return "ptl";
+  }
+}
+thread_local bool g_nvtx_kernel_open = false;
+void nvtx_kernel(int kind) {
+  if (kind == PTL_KERNEL_END) return;
+  if (g_nvtx_kernel_open) nvtxRangePop();
+  nvtxRangePushA(kind_name(kind));
+  g_nvtx_kernel_open = true;
+}
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() {
+    if (g_nvtx_kernel_open) nvtxRangePop();
+    g_nvtx_kernel_open = false;
+    nvtxRangePop();
+  }
+  ApiRange(const ApiRange&) = delete;
+  ApiRange& operator=(const ApiRange&) = delete;
+};
 
 // Records the closing PTL_KERNEL_END event when an entry point returns.
 struct EndMark {
@@ -379,6 +423,7 @@ size_t ptl_workspace_size(int64_t max_tokens, int32_t max_users, ptl_dtype dt) {
 ptl_status ptl_layer_forward(const void* x, void* out, const int32_t* cu_seqlens, int32_t num_users,
                              int64_t total_tokens, ptl_dtype dt, const ptl_layer_weights* w,
                              void* workspace, size_t ws_bytes, const ptl_debug_out* dbg, void* stream) {
+  ApiRange nvtx_range{"ptl_layer_forward"};
   Call c;
   ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -400,6 +445,7 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
                              const ptl_layer_weights* layers, const ptl_head_weights* head,
                              const uint8_t* pred_mask, float* probs, int32_t* n_pred, void* workspace,
                              size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_stack_forward"};
   Call c;
   ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -437,6 +483,7 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
 
 ptl_status ptl_qkv_projection(const void* x, void* qkv, int64_t total_tokens, ptl_dtype dt,
                               const ptl_layer_weights* w, void* workspace, size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_qkv_projection"};
   Call c;
   ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -453,6 +500,7 @@ ptl_status ptl_qkv_projection(const void* x, void* qkv, int64_t total_tokens, pt
 ptl_status ptl_attention(const void* qkv, void* attn, const int32_t* cu_seqlens, int32_t num_users,
                          int64_t total_tokens, ptl_dtype dt, void* workspace, size_t ws_bytes,
                          void* stream) {
+  ApiRange nvtx_range{"ptl_attention"};
   Call c;
   ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -471,6 +519,7 @@ ptl_status ptl_attention_masked(const void* qkv, void* attn, const int32_t* cu_s
                                 int32_t num_users, int64_t total_tokens, ptl_dtype dt,
                                 const ptl_attn_mask* mask, void* workspace, size_t ws_bytes,
                                 void* stream) {
+  ApiRange nvtx_range{"ptl_attention_masked"};
   Call c;
   ptl_status s = setup(&c, total_tokens, num_users, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -494,6 +543,7 @@ ptl_status ptl_attention_masked(const void* qkv, void* attn, const int32_t* cu_s
 ptl_status ptl_out_projection(const void* attn, const void* x, void* x1, int64_t total_tokens,
                               ptl_dtype dt, const ptl_layer_weights* w, void* workspace, size_t ws_bytes,
                               void* stream) {
+  ApiRange nvtx_range{"ptl_out_projection"};
   Call c;
   ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -509,6 +559,7 @@ ptl_status ptl_out_projection(const void* attn, const void* x, void* x1, int64_t
 ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w, int64_t total_tokens,
                     ptl_dtype dt, const ptl_layer_weights* w, void* workspace, size_t ws_bytes,
                     void* stream) {
+  ApiRange nvtx_range{"ptl_gate"};
   Call c;
   ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -526,6 +577,7 @@ ptl_status ptl_gate(const void* x1, void* xn2, int32_t* topk_idx, float* topk_w,
 
 ptl_status ptl_route_build(const int32_t* topk_idx, int64_t total_tokens, int32_t* perm,
                            int32_t* expert_off, void* workspace, size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_route_build"};
   Call c;
   ptl_status s = setup(&c, total_tokens, 1, PTL_BF16, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -544,6 +596,7 @@ ptl_status ptl_route_build(const int32_t* topk_idx, int64_t total_tokens, int32_
 ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w, const void* residual,
                    void* out, int64_t total_tokens, ptl_dtype dt, const ptl_layer_weights* w,
                    void* workspace, size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_moe"};
   Call c;
   ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -563,6 +616,7 @@ ptl_status ptl_moe(const void* xn2, const int32_t* topk_idx, const float* topk_w
 ptl_status ptl_head(const void* h, const ptl_head_weights* head, const uint8_t* pred_mask, float* probs,
                     int32_t* n_pred, int64_t total_tokens, ptl_dtype dt, void* workspace,
                     size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_head"};
   Call c;
   ptl_status s = setup(&c, total_tokens, 1, dt, workspace, ws_bytes, stream);
   if (s != PTL_OK) return s;
@@ -587,6 +641,7 @@ size_t ptl_rep_encoder_workspace_size(int64_t max_tokens, ptl_dtype dt) {
 ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* bag_offsets,
                            int64_t total_tokens, ptl_dtype dt, const ptl_rep_encoder_weights* w,
                            void* out, void* workspace, size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_rep_encoder"};
   if (dt != PTL_F32 && dt != PTL_BF16) return PTL_ERR_DTYPE;
   if (total_tokens < 0 || total_tokens >= (int64_t(1) << 31) || num_ids < 0) return PTL_ERR_SHAPE;
   if (!w || !workspace || !bag_offsets || !out) return PTL_ERR_NULL;
@@ -634,6 +689,7 @@ ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* b
 
 ptl_status ptl_wait_selftest(void* workspace, size_t ws_bytes, int32_t which, int64_t limit_ns,
                              void* stream) {
+  ApiRange nvtx_range{"ptl_wait_selftest"};
   if (!workspace) return PTL_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PTL_ERR_ALIGN;
   if (ws_bytes < 256) return PTL_ERR_WORKSPACE;
