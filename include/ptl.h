@@ -275,13 +275,19 @@ void ptl_set_trace(ptl_trace* trace);
  * block) pairs and each attention CTA's unit lists), lives in one fixed
  * array of PTL_NOALLOC_SCRATCH_BYTES bytes in the library's device memory,
  * which every GPU that loads the library holds until the process exits.
- * It allocates nothing and calls no allocating routine.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Limits: total_tokens <= PTL_NOALLOC_MAX_TOKENS and num_users <=
  *     PTL_NOALLOC_MAX_USERS; larger requests return PTL_ERR_SHAPE and launch
  *     nothing.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *   - The first call on each device is its set-up: it looks up the array's
+ *     device address (cudaGetSymbolAddress, with that device current) and
+ *     caches it.  With lazy module loading (the CUDA 12 default) that lookup
+ *     is also what loads the library's kernels onto the device and backs the
+ *     array, which may reserve device memory and synchronise; every later
+ *     call reuses the cached address and reserves nothing.  Make the first
+ *     call before any stream capture.  The cached address belongs to the
+ *     device's current context: after cudaDeviceReset in the same process it
+ *     is stale, so do not call this entry point on a device that was reset.
  *   - Every call on a device uses the same array, which keeps the previous
  *     call's contents (each call clears what must start at zero).  Calls
  *     that can overlap on the GPU -- on different streams with no ordering

@@ -14,6 +14,65 @@
 #include "common.cuh"
 #include "launch.h"
 
+namespace ptl {
+
+thread_local ptl_trace* g_trace = nullptr;
+
+// NVTX annotations (NVTX3, header-only: each call is a no-op unless a
+// profiler is attached).  Every entry point opens a range named after itself
+// and, nested in it, one range per kernel launch named by the launch's kind,
+// so a profiler can attribute and filter the library's kernels; the
+// entry point's guard closes both on every return path.
+static const char* kind_name(int kind) {
+  switch (kind) {
+    case PTL_KERNEL_CLEAR: return "clear";
+    case PTL_KERNEL_WORKLIST: return "worklist";
+    case PTL_KERNEL_LAYERNORM: return "layernorm";
+    case PTL_KERNEL_GEMM_QKV: return "gemm_qkv";
+    case PTL_KERNEL_ATTENTION: return "attention";
+    case PTL_KERNEL_GEMM_OUT: return "gemm_out";
+    case PTL_KERNEL_GATE: return "gate";
+    case PTL_KERNEL_ROUTE: return "route";
+    case PTL_KERNEL_GEMM_EXPERT1: return "gemm_expert1";
+    case PTL_KERNEL_GEMM_EXPERT2: return "gemm_expert2";
+    case PTL_KERNEL_HEAD: return "head";
+    case PTL_KERNEL_COPY: return "copy";
+    case PTL_KERNEL_COMBINE: return "combine";
+    default: return "ptl";
+  }
+}
+static thread_local bool g_nvtx_kernel_open = false;
+static void nvtx_kernel(int kind) {
+  if (kind == PTL_KERNEL_END) return;
+  if (g_nvtx_kernel_open) nvtxRangePop();
+  nvtxRangePushA(kind_name(kind));
+  g_nvtx_kernel_open = true;
+}
+void api_range_push(const char* name) { nvtxRangePushA(name); }
+void api_range_pop() {
+  if (g_nvtx_kernel_open) nvtxRangePop();
+  g_nvtx_kernel_open = false;
+  nvtxRangePop();
+}
+
+void trace_mark(cudaStream_t st, int kind) {
+  nvtx_kernel(kind);
+  ptl_trace* t = g_trace;
+  if (!t || !t->events || t->count >= t->capacity) return;
+  // inside a stream capture only an external record becomes an event node
+  // that can be timed after the graph runs
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cap);
+  if (cap == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(t->events[t->count]), st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(static_cast<cudaEvent_t>(t->events[t->count]), st);
+  if (t->kinds) t->kinds[t->count] = kind;
+  ++t->count;
+}
+
+}  // namespace ptl
+
 namespace {
 using namespace ptl;
 
@@ -113,72 +172,7 @@ ptl_status check_head(const ptl_head_weights* h) {
   return PTL_OK;
 }
 
-thread_local ptl_trace* g_trace = nullptr;
-
-// Records the trace event that opens a launch of `kind` (no-op without a trace).
-void nvtx_kernel(int kind);
-inline void mark(cudaStream_t st, int kind) {
-  nvtx_kernel(kind);
-  ptl_trace* t = g_trace;
-  if (!t || !t->events || t->count >= t->capacity) return;
-  // inside a stream capture only an external record becomes an event node
-  // that can be timed after the graph runs
-  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  cudaStreamIsCapturing(st, &cap);
-  if (cap == cudaStreamCaptureStatusActive)
-    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(t->events[t->count]), st, cudaEventRecordExternal);
-  else
-    cudaEventRecord(static_cast<cudaEvent_t>(t->events[t->count]), st);
-  if (t->kinds) t->kinds[t->count] = kind;
-  ++t->count;
-}
-
-// NVTX annotations (NVTX3, header-only: each call is a no-op unless a
-// profiler is attached).  Every entry point opens a range named after itself
-// and, nested in it, one range per kernel launch named by the launch's kind,
-// so a profiler can attribute and filter the library's kernels; the
-// entry point's guard closes both on every return path.
-const char* kind_name(int kind) {
-  switch (kind) {
-    case PTL_KERNEL_CLEAR: return "clear";
-    case PTL_KERNEL_WORKLIST: return "worklist";
-    case PTL_KERNEL_LAYERNORM: return "layernorm";
-    case PTL_KERNEL_GEMM_QKV: return "gemm_qkv";
-    case PTL_KERNEL_ATTENTION: return "attention";
-    case PTL_KERNEL_GEMM_OUT: return "gemm_out";
-    case PTL_KERNEL_GATE: return "gate";
-    case PTL_KERNEL_ROUTE: return "route";
-    case PTL_KERNEL_GEMM_EXPERT1: return "gemm_expert1";
-    case PTL_KERNEL_GEMM_EXPERT2: return "gemm_expert2";
-    case PTL_KERNEL_HEAD: return "head";
-    case PTL_KERNEL_COPY: return "copy";
-    case PTL_KERNEL_COMBINE: return "combine";
-    default: return "ptl";
-  }
-}
-thread_local bool g_nvtx_kernel_open = false;
-void nvtx_kernel(int kind) {
-  if (kind == PTL_KERNEL_END) return;
-  if (g_nvtx_kernel_open) nvtxRangePop();
-  nvtxRangePushA(kind_name(kind));
-  g_nvtx_kernel_open = true;
-}
-struct ApiRange {
-  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
-  ~ApiRange() {
-    if (g_nvtx_kernel_open) nvtxRangePop();
-    g_nvtx_kernel_open = false;
-    nvtxRangePop();
-  }
-  ApiRange(const ApiRange&) = delete;
-  ApiRange& operator=(const ApiRange&) = delete;
-};
-
-// Records the closing PTL_KERNEL_END event when an entry point returns.
-struct EndMark {
-  cudaStream_t st;
-  ~EndMark() { mark(st, PTL_KERNEL_END); }
-};
+inline void mark(cudaStream_t st, int kind) { trace_mark(st, kind); }
 
 struct Call {
   WsLayout L;
@@ -394,7 +388,7 @@ extern "C" {
 
 int32_t ptl_version(void) { return PTL_VERSION; }
 
-void ptl_set_trace(ptl_trace* trace) { g_trace = trace; }
+void ptl_set_trace(ptl_trace* trace) { ptl::g_trace = trace; }
 
 const char* ptl_status_string(ptl_status s) {
   switch (s) {

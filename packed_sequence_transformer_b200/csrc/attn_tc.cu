@@ -599,13 +599,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 template <bool MASKED>
 static int launch_attn_tc_t(const CUtensorMap& qkv_map, void* out, const WsLayout& L, char* ws,
                             cudaStream_t st, const AttnMask& mask) {
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(attn_tc_kernel<MASKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ATT_SMEM) != cudaSuccess)
-      return -1;
-    configured = true;
-  }
+  static PerDevice configured;  // the shared-memory limit is a per-device kernel attribute
+  if (configured.get([] {
+        return cudaFuncSetAttribute(attn_tc_kernel<MASKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    ATT_SMEM) == cudaSuccess
+                   ? 1
+                   : -1;
+      }) < 0)
+    return -1;
   // the work-list kernel laid out each CTA's units for this grid
   const int grid = attn_grid(L.max_items, num_sms());
   if (launch_k(attn_tc_kernel<MASKED>, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map,

@@ -427,7 +427,9 @@ template <int BN, int MODE>
 static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& out,
                        const GemmTcParams& p, int tiles_bound, cudaStream_t st, const CUtensorMap* a2 = nullptr,
                        const CUtensorMap* b2 = nullptr, const CUtensorMap* out2 = nullptr) {
-  static int max_pairs = 0;  // co-resident clusters of two (one CTA per SM)
+  // co-resident clusters of two (one CTA per SM) on the current device,
+  // found once per device together with the kernel's shared-memory limit
+  static PerDevice max_pairs_dev;
   const int smem = PairCfg<BN, MODE>::SMEM;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(192);
@@ -442,16 +444,18 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (max_pairs == 0) {
+  const int max_pairs = max_pairs_dev.get([&] {
     if (cudaFuncSetAttribute(gemm_pair_kernel<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return -1;
-    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2 * (num_sms() / 2));
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, MODE>, &cfg) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<BN, MODE>, &q) != cudaSuccess || n < 1)
       n = num_sms() / 2;
-    max_pairs = n;
-  }
+    return n;
+  });
+  if (max_pairs < 1) return -1;
   int pairs = max_pairs;
   if (tiles_bound < pairs) pairs = tiles_bound;
   if (pairs < 1) pairs = 1;

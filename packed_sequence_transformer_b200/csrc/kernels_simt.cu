@@ -1182,14 +1182,15 @@ __global__ void __launch_bounds__(REP_WARPS * 32)
 #define PTL_LAUNCH_CHECK() (cudaPeekAtLastError() == cudaSuccess ? 0 : -1)
 
 int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
+  static PerDevice sms;
+  const int n = sms.get([] {
+    int dev = 0, v = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  }
-  return n;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return -1;
+    return v;
+  });
+  return n > 0 ? n : 148;
 }
 
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st,

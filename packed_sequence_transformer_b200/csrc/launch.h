@@ -3,12 +3,55 @@
 // failed.  All launches are asynchronous on `st`.
 #pragma once
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 
 namespace ptl {
+
+// A value set up once per device (kernel attributes such as the dynamic
+// shared-memory limit, and launch-shape queries, belong to a device, not to
+// the process).  get() returns the current device's value, running init()
+// on the first call for that device (under a lock); a failed init (<= 0) is
+// not remembered, so the next call tries again.  Returns -1 on failure.
+constexpr int kMaxDevices = 64;
+struct PerDevice {
+  std::mutex mu;
+  int v[kMaxDevices] = {};
+  template <typename F>
+  int get(F&& init) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    if (v[dev] <= 0) {
+      const int r = init();
+      if (r <= 0) return -1;
+      v[dev] = r;
+    }
+    return v[dev];
+  }
+};
+
+// Tracing hooks (api.cu): trace_mark opens the NVTX range of a kernel launch
+// of `kind` and records the calling thread's trace event for it (no-ops
+// without a profiler or an installed trace); ApiRange is the NVTX range of an
+// entry point, closing both on every return path; EndMark records the
+// closing PTL_KERNEL_END event when the entry point returns.
+void trace_mark(cudaStream_t st, int kind);
+void api_range_push(const char* name);
+void api_range_pop();
+struct ApiRange {
+  explicit ApiRange(const char* name) { api_range_push(name); }
+  ~ApiRange() { api_range_pop(); }
+  ApiRange(const ApiRange&) = delete;
+  ApiRange& operator=(const ApiRange&) = delete;
+};
+struct EndMark {
+  cudaStream_t st;
+  ~EndMark() { trace_mark(st, PTL_KERNEL_END); }
+};
 
 // Launches `kernel` on `st` with programmatic stream serialization, so a
 // captured graph gets programmatic edges and the kernel may launch while its

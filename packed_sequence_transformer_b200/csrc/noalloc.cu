@@ -27,7 +27,6 @@ using namespace ptl;
 // PTL_NOALLOC_MAX_TOKENS tokens and PTL_NOALLOC_MAX_USERS users.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PTL_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_addr_mu;
 void* g_addr[kMaxDevices];
 
@@ -80,6 +79,7 @@ bool qkv_map(CUtensorMap* m, const void* qkv, int T) {
 extern "C" ptl_status ptl_attention_noalloc(const void* qkv, void* attn, const int32_t* cu_seqlens,
                                             int32_t num_users, int64_t total_tokens, ptl_dtype dt,
                                             int32_t* device_status, void* stream) {
+  ApiRange nvtx_range{"ptl_attention_noalloc"};
   if (dt != PTL_F32 && dt != PTL_BF16) return PTL_ERR_DTYPE;
   if (num_users < 1 || total_tokens < 0) return PTL_ERR_SHAPE;
   if (total_tokens > PTL_NOALLOC_MAX_TOKENS || num_users > PTL_NOALLOC_MAX_USERS) return PTL_ERR_SHAPE;
@@ -104,17 +104,22 @@ extern "C" ptl_status ptl_attention_noalloc(const void* qkv, void* attn, const i
   const int T = int(total_tokens);
   // The array keeps the previous call's contents: the error word must start
   // at zero (the work-list kernel clears its own counters).
+  trace_mark(st, PTL_KERNEL_CLEAR);
   if (cudaMemsetAsync(ws + L.err, 0, sizeof(int32_t), st) != cudaSuccess) return PTL_ERR_CUDA;
+  EndMark end_mark{st};
+  trace_mark(st, PTL_KERNEL_WORKLIST);
   if (launch_worklist(cu_seqlens, num_users, T, L, ws, st) != 0) return PTL_ERR_CUDA;
+  CUtensorMap m;
+  if (dt == PTL_BF16 && !qkv_map(&m, qkv, T)) return PTL_ERR_CUDA;
+  trace_mark(st, PTL_KERNEL_ATTENTION);
   if (dt == PTL_BF16) {
-    CUtensorMap m;
-    if (!qkv_map(&m, qkv, T)) return PTL_ERR_CUDA;
     if (launch_attn_tc(m, attn, cu_seqlens, L, ws, st) != 0) return PTL_ERR_CUDA;
   } else {
     if (launch_attn_f32(static_cast<const float*>(qkv), static_cast<float*>(attn), cu_seqlens, L, ws,
                         st) != 0)
       return PTL_ERR_CUDA;
   }
+  if (device_status) trace_mark(st, PTL_KERNEL_COPY);
   if (device_status &&
       cudaMemcpyAsync(device_status, ws + L.err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
           cudaSuccess)

@@ -110,6 +110,18 @@ def test_config1_bf16_layer():
     assert followed < 0.01 * c.total_tokens
 
 
+def test_config1_packing_fp32_layer_at_the_stated_margin():
+    """The 60-user / 6823-token packing of the bf16 workload in the fp32
+    build, against the plain fp64 oracle (no storage mode in between): top-2
+    bit-exact wherever the 2nd-vs-3rd probability gap exceeds 1e-3, the route
+    permutation bit-exact, the layer output within 1e-4."""
+    c = S.make_case("config1_fp32", num_users=60, total=6823, median=80.0, sigma=1.0, lmax=1024,
+                    seed=1, dtype="fp32", gate_std=0.1)
+    out, dbg = run_layer(c)
+    followed = check_layer(c, out, dbg, LAYER_F32)
+    assert followed < 0.001 * c.total_tokens
+
+
 def test_config1_random_biases():
     c = S.make_case("c1bias", lengths=S.config1_lengths(), seed=11, dtype="bf16", gate_std=0.1,
                     random_bias=True)

@@ -154,6 +154,10 @@ int main() {
     if (L.clear_end < L.moe_done + 4 * (size_t)L.max_tiles || L.clear_end > L.xn) bad = "clear_end";
     // the fused expert path puts expert e's rows at e * cap
     if ((int64_t)E * L.cap > L.padded_rows || L.cap < T || L.cap % MOE_BM) bad = "cap";
+    // the no-alloc entry point's fixed array holds the scratch of every
+    // batch within its stated limits
+    if (T <= PTL_NOALLOC_MAX_TOKENS && U <= PTL_NOALLOC_MAX_USERS && L.wl_end > PTL_NOALLOC_SCRATCH_BYTES)
+      bad = "noalloc";
     // work-list bound: every user's query blocks fit
     if (L.max_items < (T + ATT_BLK - 1) / ATT_BLK + std::min<long long>(U, T)) bad = "max_items";
     printf(bad ? "BAD %s\n" : "OK\n", bad);
@@ -171,8 +175,8 @@ def test_workspace_layout_invariants(tmp_path):
     src.write_text(LAYOUT_HARNESS)
     exe = tmp_path / "layout"
     subprocess.check_call([nvcc, "-std=c++17", "-O1", "-I", CSRC, "-o", str(exe), str(src)])
-    shapes = [(T, U, dt) for T in (0, 1, 2, 127, 128, 129, 255, 256, 257, 1000, 6823, 6912, 44000, 65536, 1 << 20)
-              for U in (1, 2, 60, 390, 4096) for dt in (0, 1)]
+    shapes = [(T, U, dt) for T in (0, 1, 2, 127, 128, 129, 255, 256, 257, 1000, 6823, 6912, 44000, 65535, 65536, 65537, 1 << 20)
+              for U in (1, 2, 60, 390, 4095, 4096, 4097) for dt in (0, 1)]
     inp = "\n".join(f"{T} {U} {dt}" for T, U, dt in shapes) + "\n"
     out = subprocess.run([str(exe)], input=inp, capture_output=True, text=True, check=True).stdout.split("\n")
     bad = [(s, o) for s, o in zip(shapes, out) if o != "OK"]

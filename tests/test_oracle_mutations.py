@@ -201,3 +201,107 @@ def test_e4m3_rounding_slips_are_caught(monkeypatch, kw):
 def test_missing_saturation_is_caught(monkeypatch):
     monkeypatch.setattr(O, "quantize_e4m3", _e4m3_mutant(saturate=False))
     assert _fails(P8.test_value_set_and_extremes)
+
+
+# ------------------------------------------------- top-2 margins
+def test_gap_measured_from_the_first_expert_is_caught(monkeypatch):
+    """p_(1) - p_(3) in place of p_(2) - p_(3): the margin of the routing bar
+    would widen silently."""
+    def wrong(p):
+        ps = -np.sort(-np.asarray(p, np.float64), axis=-1)
+        return ps[:, 0] - ps[:, 2]
+    monkeypatch.setattr(O, "top2_gap", wrong)
+    assert _fails(P.test_top2_gaps_golden)
+    assert _fails(P.test_top2_gaps_are_the_distance_to_another_choice)
+
+
+def test_slot_gap_measured_to_the_third_is_caught(monkeypatch):
+    def wrong(p):
+        ps = -np.sort(-np.asarray(p, np.float64), axis=-1)
+        return ps[:, 0] - ps[:, 2]
+    monkeypatch.setattr(O, "top1_gap", wrong)
+    assert _fails(P.test_top2_gaps_golden)
+    assert _fails(P.test_top2_gaps_are_the_distance_to_another_choice)
+
+
+# ------------------------------------------------- bf16 storage points
+def _skip_nth_rounding(monkeypatch, n):
+    """The bf16 storage mode with its n-th rounding call (in layer order:
+    LayerNorm1, qkv, attention, LayerNorm2, then per expert hidden and output,
+    then the layer output; -1 = the last) left out."""
+    orig = O._storage
+
+    def storage(kind):
+        rnd = orig(kind)
+        if kind != "bf16":
+            return rnd
+        calls = []
+
+        def mutant(a):
+            calls.append(1)
+            if len(calls) == n:
+                return O._f64(a)
+            return rnd(a)
+        return mutant
+    monkeypatch.setattr(O, "_storage", storage)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4, 5])
+def test_each_dropped_bf16_rounding_point_is_caught(monkeypatch, n):
+    _skip_nth_rounding(monkeypatch, n)
+    assert _fails(P.test_bf16_storage_rounding_points)
+
+
+def test_dropped_expert_output_rounding_is_caught(monkeypatch):
+    orig = O.moe_routed
+
+    def no_y_round(xn2, idx, w, w1, b1, w2, b2, hidden_round=None):
+        out, y, hidden = orig(xn2, idx, w, w1, b1, w2, b2, hidden_round=None)
+        if hidden_round is not None:
+            hidden = hidden_round(hidden)
+        return out, y, hidden
+    monkeypatch.setattr(O, "moe_routed", no_y_round)
+    assert _fails(P.test_bf16_storage_rounding_points)
+
+
+def _patch_bf16_intermediate(monkeypatch, name, fn):
+    """The bf16 storage mode with intermediate `name` replaced by fn(it)."""
+    orig_layer = O.layer_forward
+
+    def layer(x, cu, wts, return_intermediates=False, storage=None, choose=None):
+        out, it = orig_layer(x, cu, wts, True, storage, choose)
+        if storage == "bf16":
+            it = dict(it)
+            it[name] = fn(it)
+            out = it["out"]
+        return (out, it) if return_intermediates else out
+    monkeypatch.setattr(O, "layer_forward", layer)
+
+
+def test_dropped_layer_output_rounding_is_caught(monkeypatch):
+    """The layer output left unrounded (x1 + moe stored in fp64)."""
+    _patch_bf16_intermediate(monkeypatch, "out", lambda it: it["x1"] + it["moe"])
+    assert _fails(P.test_bf16_storage_rounding_points)
+
+
+def test_rounded_residual_is_caught(monkeypatch):
+    """x1 rounded to bf16 (a bf16 residual buffer) instead of kept exact."""
+    _patch_bf16_intermediate(monkeypatch, "x1", lambda it: O.round_bf16(it["x1"]))
+    assert _fails(P.test_bf16_storage_rounding_points)
+
+
+def test_gate_on_the_stored_layernorm2_row_is_caught(monkeypatch):
+    """The gate fed the bf16-rounded LayerNorm2 row instead of the row before
+    it is stored."""
+    def p_rounded(it):
+        return O.gate_probs(it["xn2"], W["w_gate"], W["b_gate"])
+    W = {}
+    orig_case = P._bf16_storage_case
+
+    def case():
+        c, res = orig_case()
+        W.update(c.layers[0])
+        res[1]["p"] = p_rounded(res[1])
+        return c, res
+    monkeypatch.setattr(P, "_bf16_storage_case", case)
+    assert _fails(P.test_bf16_storage_rounding_points)

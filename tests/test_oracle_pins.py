@@ -144,6 +144,39 @@ def test_top2_golden_ties_and_weights():
     np.testing.assert_allclose(w, _frac(g["w"]), atol=1e-15)
 
 
+def test_top2_gaps_golden():
+    """top2_gap = p_(2) - p_(3) and top1_gap = p_(1) - p_(2), hand-read off the
+    sorted golden rows (a tie inside the pair in row 0, a tie at the pair's
+    edge in row 1)."""
+    g = _golden("moe_route_closed_form.json")["top2"]
+    p = np.array(g["p"])
+    np.testing.assert_allclose(O.top2_gap(p), [float(Fraction(v)) for v in g["gap23"]], atol=1e-15)
+    np.testing.assert_allclose(O.top1_gap(p), [float(Fraction(v)) for v in g["gap12"]], atol=1e-15)
+
+
+def test_top2_gaps_are_the_distance_to_another_choice():
+    """What the gaps mean for top2 (itself pinned by brute force): raising the
+    best left-out expert by less than top2_gap keeps the chosen pair, by more
+    changes it; raising the slot-1 expert by less than top1_gap keeps the slot
+    order, by more swaps it.  A gap measured between the wrong ranks moves one
+    of these thresholds."""
+    rng = np.random.default_rng(170)
+    p = rng.dirichlet(np.ones(8), size=200)
+    idx, _ = O.top2(p)
+    g23, g12 = O.top2_gap(p), O.top1_gap(p)
+    assert np.all(g23 >= 0) and np.all(g12 >= 0)
+    for t in range(p.shape[0]):
+        left_out = [e for e in range(8) if e not in idx[t]]
+        third = max(left_out, key=lambda e: (p[t, e], -e))
+        for frac, same in ((0.99, True), (1.01, False)):
+            q = p[t:t + 1].copy()
+            q[0, third] += frac * g23[t] + (0.0 if same else 1e-12)
+            assert (set(O.top2(q)[0][0]) == set(idx[t])) == same
+            q = p[t:t + 1].copy()
+            q[0, idx[t, 1]] += frac * g12[t] + (0.0 if same else 1e-12)
+            assert (O.top2(q)[0][0, 0] == idx[t, 0]) == same
+
+
 def test_top2_brute_force_and_weight_invariants():
     rng = np.random.default_rng(17)
     xn2 = rng.standard_normal((64, 512))
@@ -382,3 +415,38 @@ def test_bf16_storage_mode_stays_within_bf16_error_of_exact():
     assert np.max(np.abs(bf[same] - ex[same])) < 3e-2
     assert np.array_equal(bf, O.round_bf16(bf))          # stored output is on the bf16 grid
     assert not np.array_equal(bf, ex)
+
+
+BF16_STORED = ("xn", "qkv", "attn", "xn2", "hidden", "y", "out")
+
+
+def _bf16_storage_case():
+    c = S.make_case("st_pts", lengths=[9, 1, 20], seed=43, dtype="bf16", gate_std=0.1, random_bias=True)
+    return c, O.layer_forward(c.x, c.cu_seqlens, c.layers[0], return_intermediates=True,
+                              storage="bf16")
+
+
+def test_bf16_storage_rounding_points():
+    """Reading of bf16 inference with fp32 accumulation (cti2026 README: bf16
+    activations, fp32 softmax statistics): every activation the layer stores
+    -- LayerNorm1 output, q/k/v, attention output, LayerNorm2 output, expert
+    hidden rows, each route's expert output and the layer output -- lies on
+    the bf16 grid; the residual x1 = x + attn Wo^T + b_o is kept exact (an
+    fp32 buffer, not a bf16 one); the gate reads the LayerNorm2 row before it
+    is stored, so p is the softmax of the unrounded LayerNorm2 output."""
+    c, (out, it) = _bf16_storage_case()
+    w = c.layers[0]
+    for name in BF16_STORED:
+        a = np.asarray(it[name])
+        if name in ("hidden", "y"):
+            a = a[np.any(a != 0, axis=1)]
+        assert np.array_equal(a, O.round_bf16(a)), f"{name} is stored in bf16"
+    x1 = np.asarray(c.x, np.float64) + np.asarray(it["attn"]) @ np.asarray(w["w_o"], np.float64).T
+    if w.get("b_o") is not None:
+        x1 = x1 + np.asarray(w["b_o"], np.float64)
+    np.testing.assert_allclose(it["x1"], x1, rtol=0, atol=1e-12)
+    assert not np.array_equal(it["x1"], O.round_bf16(it["x1"]))
+    xn2_exact = O.layer_norm(it["x1"], w["ln2_g"], w["ln2_b"])
+    p = torch.softmax(torch.from_numpy(xn2_exact @ np.asarray(w["w_gate"], np.float64).T
+                                       + np.asarray(w["b_gate"], np.float64)), dim=-1).numpy()
+    np.testing.assert_allclose(it["p"], p, rtol=0, atol=1e-14)
