@@ -12,8 +12,11 @@ prediction head.  value = tokens x layers / step time, summed over ranks.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload stack8|layer]
 
-N > 1 runs under torch.distributed.run: every rank processes its own batch
-of the same shape (weak scaling, no collective on the data path); the step
+N > 1 runs under torch.distributed.run: the job's batch is N copies of the
+packing (N x 60 users), split into contiguous user ranges balanced by cost
+(ptl_partition_users), one per rank; each rank runs the stack on its range
+and the head probabilities are all-gathered over NCCL at the end of every
+step (weak scaling: per-rank work stays one packing's worth).  The step
 time is the max over ranks.  --impl reference times the CPU oracle (numpy
 fp64) on this host on a bounded sample of the same workload.
 """
@@ -41,13 +44,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 RUNNER_STRIDE = 128  # token granule of the graph runner's buckets in the end-to-end leg
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each
 # kernel kind, from one ncu --set full capture of this workload's layer 0
-# (profiles/*_stack8_6823tok.md; ncu flushes caches between replays, so these
-# are cold-cache figures).  A kernel changed since its capture must be
-# recaptured or dropped from this table.
-# The expert GEMM launch, the gate + route kernel and the attention changed
-# after their capture (the first two now wait through the shared bounded-wait
-# helper, the attention is templated on the mask), so they report no traffic
-# until they are captured again.
+# (ncu flushes caches between replays, so these are cold-cache figures).  A
+# kernel changed since its capture is dropped from this table until it is
+# captured again.
 NCU_DRAM_BYTES = {
     "gemm_qkv": 8.589312e6,
     "gemm_out": 14.527488e6,
@@ -74,16 +73,53 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def make_workload(name, rank):
+def make_workload(name, world=1):
+    """The job's batch: the 60-user / 6823-token packing (stack: 8 layers +
+    head, weights from seed 2; layer: one layer, gate std 0.1, seed 1), as
+    `world` copies laid end to end with their own activations and one set of
+    weights when world > 1."""
     from packed_sequence_transformer_b200 import synthetic as S
     lengths = S.config1_lengths()
     if name == "stack8":
-        c = S.make_case("stack8_6823tok_60u", lengths=lengths, seed=2 + 1000 * rank, dtype="bf16",
+        c = S.make_case("stack8_6823tok_60u", lengths=lengths, seed=2, dtype="bf16",
                         num_layers=8, with_head=True)
     else:
-        c = S.make_case("layer_6823tok_60u", lengths=lengths, seed=1 + 1000 * rank, dtype="bf16",
+        c = S.make_case("layer_6823tok_60u", lengths=lengths, seed=1, dtype="bf16",
                         gate_std=0.1)
-    return c
+    return S.replicate_batch(c, world, seed=1000)
+
+
+def rank_part(case, world, rank):
+    """This rank's share of the job's batch: contiguous users balanced by cost
+    (ptl_partition_users).  Returns (t0, t1, rebased int32 offsets)."""
+    from packed_sequence_transformer_b200 import ptl
+    begin = ptl.partition_users(case.cu_seqlens, world)
+    t0, t1, _, _, cu = ptl.part_of_batch(case.cu_seqlens, begin, rank)
+    return t0, t1, cu
+
+
+def gather_parts(local, count, world, cap):
+    """All-gather of every rank's first `count` entries of `local` (1-D,
+    padded to `cap` entries on every rank): returns (gathered [world * cap],
+    counts [world]) on local's device.  Collectives only; no host sync."""
+    import torch
+    import torch.distributed as dist
+    buf = torch.empty(world * cap, dtype=local.dtype, device=local.device)
+    cnt = torch.empty(world, dtype=count.dtype, device=count.device)
+    dist.all_gather_into_tensor(buf, local[:cap].contiguous())
+    dist.all_gather_into_tensor(cnt, count.reshape(1))
+    return buf, cnt
+
+
+def concat_parts(buf, cnt, cap):
+    """The gathered parts' entries in rank order (host numpy): the whole
+    batch's result, since each part is a contiguous range of users."""
+    buf = buf.cpu().numpy()
+    return np.concatenate([buf[r * cap:r * cap + int(c)] for r, c in enumerate(cnt.cpu().tolist())])
+
+
+def pct(xs, q):
+    return float(np.percentile(np.asarray(xs, np.float64), q))
 
 
 def max_over_ranks(x, world, device="cpu"):
@@ -142,9 +178,10 @@ def visible_pairs(lengths, ctx, tgt):
     return total
 
 
-def time_attention_legs(case, dev, stream, flush, reps=20):
+def time_attention_legs(case, dev, stream, flush, reps=20, masked=True):
     """Device time (CUDA events, L2 flushed between launches) of the causal
-    attention and of the masked variant on the workload's packing."""
+    attention and (masked=True) of the masked variant on the workload's
+    packing."""
     import torch
 
     from packed_sequence_transformer_b200 import ptl
@@ -163,6 +200,8 @@ def time_attention_legs(case, dev, stream, flush, reps=20):
                                                target_group_size=MASKED_LEG["group"],
                                                window=MASKED_LEG["window"], stream=stream),
     }
+    if not masked:
+        calls.pop("masked")
     res = {}
     for name, fn in calls.items():
         kt = ptl.KernelTrace(capacity=8)
@@ -179,8 +218,8 @@ def time_attention_legs(case, dev, stream, flush, reps=20):
         st = ptl.last_device_error(ws, stream)
         if st != 0:
             raise RuntimeError(f"device error {ptl.STATUS.get(st)} in the {name} attention leg")
-        res[name] = 1e3 * statistics.mean(times)
-    pairs = visible_pairs(case.lengths, ctx_h, tgt_h)
+        res[name] = 1e3 * statistics.median(times)
+    pairs = visible_pairs(case.lengths, ctx_h, tgt_h) if masked else None
     return res, pairs
 
 
@@ -299,37 +338,71 @@ def blas_threads():
         return os.cpu_count()
 
 
-def time_oracle_layers(case, budget_s=12.0, max_reps=8, min_reps=1, layer_offset=0):
-    """Time the oracle's full-batch layer forward (layers of the case in turn);
-    returns (seconds per layer, reps)."""
+def blas_name():
+    try:
+        from threadpoolctl import threadpool_info
+        libs = [f"{i.get('internal_api')} {i.get('version')}" for i in threadpool_info()
+                if i.get("user_api") == "blas"]
+        return ", ".join(libs) if libs else "unknown"
+    except Exception:
+        return "unknown"
+
+
+def time_oracle_layers(case, budget_s=12.0, max_reps=8, min_reps=1, layer_offset=0, threads=None):
+    """Time the oracle's full-batch layer forward (layers of the case in turn),
+    with the BLAS pool limited to `threads` (None: as configured); returns
+    (seconds per layer: median, p10, p90; reps)."""
     from oracle import ptl_oracle as O
-    times = []
-    h = case.x
-    t_all = time.perf_counter()
-    i = 0
-    while i < max_reps and (i < min_reps or time.perf_counter() - t_all < budget_s):
-        w = case.layers[(layer_offset + i) % len(case.layers)]
-        t0 = time.perf_counter()
-        O.layer_forward(h, case.cu_seqlens, w)
-        times.append(time.perf_counter() - t0)
-        i += 1
-    return statistics.mean(times), len(times)
+    ctx = None
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(limits=threads, user_api="blas")
+    try:
+        times = []
+        h = case.x
+        t_all = time.perf_counter()
+        i = 0
+        while i < max_reps and (i < min_reps or time.perf_counter() - t_all < budget_s):
+            w = case.layers[(layer_offset + i) % len(case.layers)]
+            t0 = time.perf_counter()
+            O.layer_forward(h, case.cu_seqlens, w)
+            times.append(time.perf_counter() - t0)
+            i += 1
+    finally:
+        if ctx is not None:
+            ctx.unregister()
+    return (statistics.median(times), pct(times, 10), pct(times, 90)), len(times)
+
+
+def cpu_baseline(case, budget_all=8.0, budget_one=10.0):
+    """The oracle on this host's cores: full-batch layers with every BLAS
+    thread, then with one; tokens/s from the median layer time."""
+    T = case.total_tokens
+    (med, p10, p90), reps = time_oracle_layers(case, budget_s=budget_all, max_reps=6, min_reps=2)
+    (med1, p10_1, p90_1), reps1 = time_oracle_layers(case, budget_s=budget_one, max_reps=4, min_reps=1,
+                                                     threads=1)
+    return {"value": T / med, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"numpy fp64 oracle, {reps} full-batch layers of this workload ({T} tokens each) "
+                      f"on all BLAS threads and {reps1} on one; median layer time",
+            "blas": blas_name(), "layer_s_median": med, "layer_s_p10": p10, "layer_s_p90": p90,
+            "one_thread": {"value": T / med1, "layer_s_median": med1, "layer_s_p10": p10_1,
+                           "layer_s_p90": p90_1, "reps": reps1}}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    case = make_workload(args.workload, 0)
+    case = make_workload(args.workload)
     T = case.total_tokens
     # warm-up and timed steps: one oracle layer over the full batch each
     for i in range(args.warmup):
         time_oracle_layers(case, max_reps=1, layer_offset=i)
     secs = []
     for i in range(args.steps):
-        s, _ = time_oracle_layers(case, max_reps=1, layer_offset=i)
+        (s, _, _), _ = time_oracle_layers(case, max_reps=1, layer_offset=i)
         secs.append(s)
-    sec = statistics.mean(secs)
+    sec = statistics.median(secs)
     value = T / sec
     cores = blas_threads()
     line = {
@@ -340,7 +413,8 @@ def run_reference(args):
         "config": {"workload": case.name + (" (one layer per step)" if args.workload == "stack8" else ""),
                    "tokens": T, "users": case.num_users, "layers_per_step": 1},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"numpy fp64 oracle, one full-batch layer ({T} tokens) per step"},
+                         "sample": f"numpy fp64 oracle, one full-batch layer ({T} tokens) per step; median step",
+                         "blas": blas_name()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -348,6 +422,174 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------- ours
+# Algorithmic work per launch of each kernel kind on T tokens: FLOPs for the
+# tensor-core kernels, bytes for the bandwidth-bound ones (bf16 build, fp32
+# residual x1: gate + route reads x1 and writes the LayerNorm2 row to both of
+# its expert rows plus ids / weights / positions; the combine reads two
+# per-route rows, x1 and the weights, writes the output and the next layer's
+# LayerNorm1 row; LayerNorm reads and writes one row).
+def kernel_work(T, attn_fl, separate_expert2):
+    return {
+        "gemm_qkv": ("tensor", 2 * T * 512 * 1536),
+        "attention": ("tensor", attn_fl),
+        "gemm_out": ("tensor", 2 * T * 512 * 512),
+        # both expert GEMMs run in one launch (traced as gemm_expert1) unless
+        # gemm_expert2 shows up as a launch of its own
+        "gemm_expert1": ("tensor", 2 * (2 * T) * 512 * 1024 * (1 if separate_expert2 else 2)),
+        "gemm_expert2": ("tensor", 2 * (2 * T) * 1024 * 512),
+        "combine": ("hbm", T * (2 * 1024 + 2048 + 1024 + 1024 + 16)),
+        "gate": ("hbm", T * (2048 + 2 * 1024 + 24)),
+        "layernorm": ("hbm", T * 2048),
+        "route": ("hbm", T * 24),
+    }
+
+
+def trace_kernels(step, stream, flush, n_launch_cap, reps):
+    """Per-kernel device times: the step captured with a CUDA event before
+    every launch (event nodes inside the graph), replayed `reps` times with
+    the L2 flushed in between; launch i takes events[i] -> events[i + 1].
+    An event node stops the next launch from starting early (programmatic
+    dependent launch), so each time includes its launch gap and prologue.
+    Returns {kind: {launches_per_step, avg_us, share}} and the sum of the
+    per-step times (ms)."""
+    import torch
+
+    from packed_sequence_transformer_b200 import ptl
+    kt = ptl.KernelTrace(capacity=n_launch_cap)
+    tgraph = torch.cuda.CUDAGraph()
+    with kt:
+        with torch.cuda.graph(tgraph, stream=stream):
+            step()
+    torch.cuda.synchronize()
+    recorded = []
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            tgraph.replay()
+            torch.cuda.synchronize()
+            recorded.extend(kt.launches())
+            flush.fill_(float(i))
+    torch.cuda.synchronize()
+    tgraph.reset()
+    per_kind = {}
+    for kind, t_ms in recorded:
+        d = per_kind.setdefault(kind, [0.0, 0])
+        d[0] += t_ms
+        d[1] += 1
+    kinds = {k: {"launches_per_step": v[1] / reps, "avg_us": 1e3 * v[0] / v[1], "share": 0.0}
+             for k, v in per_kind.items()}
+    tot = sum(v[0] for v in per_kind.values())
+    for k, v in per_kind.items():
+        kinds[k]["share"] = v[0] / tot if tot else 0.0
+    return kinds, tot / reps
+
+
+def apportion(kinds, step_ms):
+    """Each kind's per-launch time with the event-node times scaled so that a
+    step's launches add up to the measured step time (the event nodes' launch
+    gaps, which programmatic launch hides in the real step, spread in
+    proportion)."""
+    tot_us = sum(v["avg_us"] * v["launches_per_step"] for v in kinds.values())
+    f = 1e3 * step_ms / tot_us if tot_us else 0.0
+    for v in kinds.values():
+        v["apportioned_us"] = v["avg_us"] * f
+    return kinds
+
+
+def fractions(kinds, T, attn_fl, peaks):
+    """Achieved throughput and fraction of the measured peak per kernel kind
+    (event-node time; apportioned time in parentheses of the key names)."""
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    work = kernel_work(T, attn_fl, "gemm_expert2" in kinds)
+    out = {}
+    for k, v in kinds.items():
+        if k not in work:
+            continue
+        bound, w = work[k]
+        scale, peak = (1e12, bf16) if bound == "tensor" else (1e9, hbm)
+        a = w / (v["avg_us"] / 1e6) / scale
+        out[k] = {"bound": bound, "achieved": a, "frac": a / peak}
+        if v.get("apportioned_us"):
+            out[k]["frac_apportioned"] = w / (v["apportioned_us"] / 1e6) / scale / peak
+    return out
+
+
+def time_graph_steps(graph, stream, flush, steps, warmup):
+    """Median, p10 and p90 (ms) of `steps` replays of `graph`, CUDA events on
+    `stream` around each, the L2 flushed (256 MiB write) in between."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+            flush.fill_(1.0)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            evs[i][0].record(stream)
+            graph.replay()
+            evs[i][1].record(stream)
+            flush.fill_(float(i))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return statistics.median(ms), pct(ms, 10), pct(ms, 90)
+
+
+def time_workload_leg(case, dev, stream, flush, peaks, steps=10, attention_alone=False):
+    """A larger packing through the same entry points: the stack (or layer)
+    captured in a graph and replayed with the L2 flushed in between; packed
+    tokens/s per layer, the per-kernel fractions of the measured peaks and,
+    optionally, the attention alone on its packing."""
+    import torch
+
+    from packed_sequence_transformer_b200 import ptl
+    T, U = case.total_tokens, case.num_users
+    n_layers = len(case.layers)
+    layers = [ptl.to_device_layer(w, "bf16", dev) for w in case.layers]
+    x = torch.as_tensor(case.x).to(dev, torch.bfloat16).contiguous()
+    cu = torch.as_tensor(case.cu_seqlens).to(dev, torch.int32)
+    out = torch.empty_like(x)
+    ws = ptl.alloc_workspace(T, U, "bf16", dev)
+
+    def step():
+        if n_layers > 1:
+            ptl.stack_forward(x, out, cu, layers, ws)
+        else:
+            ptl.layer_forward(x, out, cu, layers[0], ws)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    st = ptl.last_device_error(ws, stream)
+    if st != 0:
+        raise RuntimeError(f"device error {ptl.STATUS.get(st)} in the {case.name} leg")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    torch.cuda.synchronize()
+    med, p10, p90 = time_graph_steps(graph, stream, flush, steps, 3)
+    graph.reset()
+    kinds, _ = trace_kernels(step, stream, flush, 8 * n_layers + 16, min(steps, 5))
+    apportion(kinds, med)
+    attn_fl = attention_flops(case.lengths)
+    step_flops = n_layers * (GEMM_FLOPS_PER_TOKEN * T + attn_fl)
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    leg = {"workload": case.name, "tokens": T, "users": U, "layers": n_layers,
+           "ms_per_step": med, "ms_p10": p10, "ms_p90": p90,
+           "tokens_per_s_per_layer": T * n_layers / (med / 1e3),
+           "us_per_layer": 1e3 * med / n_layers,
+           "step_frac_of_peak": step_flops / (med / 1e3) / 1e12 / bf16,
+           "kernels": kinds, "fractions": fractions(kinds, T, attn_fl, peaks)}
+    if attention_alone:
+        a_us, _ = time_attention_legs(case, dev, stream, flush, reps=10, masked=False)
+        leg["attention_alone_us"] = a_us["causal"]
+        leg["attention_alone_tflops"] = attn_fl / a_us["causal"] / 1e6
+        leg["attention_alone_frac"] = leg["attention_alone_tflops"] / bf16
+    del ws
+    torch.cuda.empty_cache()
+    return leg
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -369,19 +611,33 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    case = make_workload(args.workload, rank)
-    T, U = case.total_tokens, case.num_users
-    n_layers = len(case.layers)
-    layers = [ptl.to_device_layer(w, "bf16", dev) for w in case.layers]
-    head = ptl.to_device_head(case.head, dev) if case.head is not None else None
-    x = torch.as_tensor(case.x).to(dev, torch.bfloat16).contiguous()
-    cu = torch.as_tensor(case.cu_seqlens).to(dev, torch.int32)
-    mask = torch.as_tensor(case.pred_mask).to(dev, torch.uint8) if head is not None else None
+    # the job's batch, and this rank's contiguous share of its users
+    job = make_workload(args.workload, world)
+    t0, t1, cu_part = rank_part(job, world, rank)
+    T, U = t1 - t0, len(cu_part) - 1
+    if T == 0:
+        raise RuntimeError(f"rank {rank} received no tokens")
+    n_layers = len(job.layers)
+    layers = [ptl.to_device_layer(w, "bf16", dev) for w in job.layers]
+    head = ptl.to_device_head(job.head, dev) if job.head is not None else None
+    x_part = job.x[t0:t1]
+    mask_part = job.pred_mask[t0:t1] if head is not None else None
+    x = torch.as_tensor(x_part).to(dev, torch.bfloat16).contiguous()
+    cu = torch.as_tensor(cu_part).to(dev, torch.int32)
+    mask = torch.as_tensor(mask_part).to(dev, torch.uint8) if head is not None else None
     out = torch.empty_like(x)
     probs = torch.empty(T, dtype=torch.float32, device=dev) if head is not None else None
     n_pred = torch.zeros(1, dtype=torch.int32, device=dev) if head is not None else None
     ws = ptl.alloc_workspace(T, U, "bf16", dev)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MiB > L2
+    # N > 1: the head probabilities (or output rows) of every rank are
+    # all-gathered at the end of each step, padded to the largest part
+    cap = int(max_over_ranks(T, world, dev))
+    if world > 1:
+        res_local = (torch.zeros(cap, dtype=torch.float32, device=dev) if head is not None
+                     else torch.zeros(cap * 512, dtype=torch.bfloat16, device=dev))
+        res_count = n_pred if head is not None else torch.tensor([T * 512], dtype=torch.int32, device=dev)
+        res_cap = cap if head is not None else cap * 512
 
     stream = torch.cuda.Stream(device=dev)
 
@@ -391,6 +647,15 @@ def run_ours(args):
                               n_pred=n_pred)
         else:
             ptl.layer_forward(x, out, cu, layers[0], ws)
+
+    def gather():
+        if world > 1:
+            if head is not None:
+                res_local[:T].copy_(probs)
+            else:
+                res_local[:T * 512].copy_(out.reshape(-1))
+            return gather_parts(res_local, res_count, world, res_cap)
+        return None
 
     # eager warm-up (configures kernels), error check, then graph capture
     with torch.cuda.stream(stream):
@@ -412,10 +677,12 @@ def run_ours(args):
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
             graph.replay()
+            gather()
             flush.fill_(1.0)
     torch.cuda.synchronize()
 
-    # ---- timed region: K graph replays, L2 flushed between them
+    # ---- timed region: K graph replays (+ the all-gather at N > 1), L2
+    # flushed between them
     gpu_index = torch.cuda.current_device()
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
@@ -431,61 +698,31 @@ def run_ours(args):
         for i in range(args.steps):
             evs[i][0].record(stream)
             graph.replay()
+            gathered = gather()
             evs[i][1].record(stream)
             flush.fill_(float(i))
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    ms_max = max_over_ranks(statistics.mean(step_ms), world, dev)
-    value = job_value(T, n_layers, world, ms_max)
+    med_ms = statistics.median(step_ms)
+    ms_max = max_over_ranks(med_ms, world, dev)
+    p10_max = max_over_ranks(pct(step_ms, 10), world, dev)
+    p90_max = max_over_ranks(pct(step_ms, 90), world, dev)
+    value = job.total_tokens * n_layers / (ms_max / 1e3)
+    if world > 1 and head is not None:
+        # the gathered probabilities are the whole batch's, in token order
+        n_all = int(sum(gathered[1].cpu().tolist()))
+        assert n_all == int(job.pred_mask.sum())
 
-    # ---- per-kernel device times: the same step captured with a CUDA event
-    # before every launch (event nodes inside the graph), replayed with the
-    # L2 flushed in between; launch i takes events[i] -> events[i + 1].
-    trace_steps = min(args.steps, 10)
-    kt = ptl.KernelTrace(capacity=2 * launches_per_step + 16)
-    tgraph = torch.cuda.CUDAGraph()
-    with kt:
-        with torch.cuda.graph(tgraph, stream=stream):
-            step()
-    torch.cuda.synchronize()
-    recorded = []
-    with torch.cuda.stream(stream):
-        for i in range(trace_steps):
-            tgraph.replay()
-            torch.cuda.synchronize()
-            recorded.extend(kt.launches())
-            flush.fill_(float(i))
-    torch.cuda.synchronize()
-    tgraph.reset()
-    per_kind = {}
-    for kind, t_ms in recorded:
-        d = per_kind.setdefault(kind, [0.0, 0])
-        d[0] += t_ms
-        d[1] += 1
-    kinds = {k: {"launches_per_step": v[1] / trace_steps, "avg_us": 1e3 * v[0] / v[1],
-                 "share": 0.0} for k, v in per_kind.items()}
-    tot = sum(v[0] for v in per_kind.values())
-    for k, v in per_kind.items():
-        kinds[k]["share"] = v[0] / tot if tot else 0.0
+    # ---- per-kernel device times (event nodes in a second captured graph)
+    kinds, trace_ms = trace_kernels(step, stream, flush, 2 * launches_per_step + 16, min(args.steps, 10))
+    apportion(kinds, med_ms)
 
     peaks, peak_src = load_peaks()
-    lengths = case.lengths
+    lengths = np.diff(cu_part)
     attn_fl = attention_flops(lengths)
-    alg = {
-        "gemm_qkv": ("tensor", 2 * T * 512 * 1536),
-        "attention": ("tensor", attn_fl),
-        "gemm_out": ("tensor", 2 * T * 512 * 512),
-        # both expert GEMMs run in one launch (traced as gemm_expert1) unless
-        # gemm_expert2 shows up as a launch of its own
-        "gemm_expert1": ("tensor", 2 * (2 * T) * 512 * 1024 * (1 if "gemm_expert2" in kinds else 2)),
-        "gemm_expert2": ("tensor", 2 * (2 * T) * 1024 * 512),
-        "combine": ("hbm", T * (2 * 1024 + 2048 + 1024 + 1024 + 16)),
-        "gate": ("hbm", T * (2048 + 2 * 1024 + 24)),
-        "layernorm": ("hbm", T * 2048),
-        "route": ("hbm", T * 24),
-    }
+    alg = kernel_work(T, attn_fl, "gemm_expert2" in kinds)
     dom = max((k for k in kinds if k in alg), key=lambda k: kinds[k]["avg_us"] * kinds[k]["launches_per_step"])
     bound, work = alg[dom]
     t_s = kinds[dom]["avg_us"] / 1e6
@@ -500,7 +737,10 @@ def run_ours(args):
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": NCU_DRAM_BYTES.get(dom), "kernel": dom,
                 "peak_source": f"{peak_src} ({'bf16_tflops burst' if bound == 'tensor' else 'hbm_gbs'})",
-                "algorithmic_per_launch": work}
+                "algorithmic_per_launch": work,
+                "time": "event nodes around each launch (includes the launch gap that programmatic "
+                        "launch hides in the step); frac_apportioned scales them to the step time",
+                "frac_apportioned": work / (kinds[dom]["apportioned_us"] / 1e6) / (1e12 if bound == "tensor" else 1e9) / peak}
     step_flops = n_layers * (GEMM_FLOPS_PER_TOKEN * T + attn_fl)
     whole_step_tflops = step_flops / (ms_max / 1e3) / 1e12
 
@@ -508,9 +748,9 @@ def run_ours(args):
     # host (pinned) buffers; each step copies the batch in, replays the
     # bucket's graph and copies the result (head probabilities + count, or
     # the hidden rows) out
-    x_h = torch.as_tensor(case.x).to(torch.bfloat16).pin_memory()
-    cu_h = torch.as_tensor(case.cu_seqlens).to(torch.int32).pin_memory()
-    mask_h = torch.as_tensor(case.pred_mask).to(torch.uint8).pin_memory() if head is not None else None
+    x_h = torch.as_tensor(x_part).to(torch.bfloat16).pin_memory()
+    cu_h = torch.as_tensor(cu_part).to(torch.int32).pin_memory()
+    mask_h = torch.as_tensor(mask_part).to(torch.uint8).pin_memory() if head is not None else None
     res_h = (torch.empty(T, dtype=torch.float32).pin_memory() if head is not None
              else torch.empty(T, 512, dtype=torch.bfloat16).pin_memory())
     n_h = torch.zeros(1, dtype=torch.int32).pin_memory()
@@ -542,13 +782,13 @@ def run_ours(args):
                     ms.append((a, b))
                 flush.fill_(float(i))
         torch.cuda.synchronize()
-        return statistics.mean(a.elapsed_time(b) for a, b in ms)
+        return statistics.median(a.elapsed_time(b) for a, b in ms)
 
     e2e_ms = timed(lambda: run_runner(x_h, cu_h, mask_h, res_h, n_h), args.warmup, args.steps, True)
     st = runner.last_device_error(stream)
     if st != 0:
         raise RuntimeError(f"device error {ptl.STATUS.get(st)} in the runner")
-    e2e_value = job_value(T, n_layers, world, max_over_ranks(e2e_ms, world, dev))
+    e2e_value = job.total_tokens * n_layers / (max_over_ranks(e2e_ms, world, dev) / 1e3)
     # the same runner on device-resident buffers (device copies + graph), and
     # the stack issued kernel by kernel from the host without a graph
     res_d = probs if head is not None else torch.empty_like(out)
@@ -556,24 +796,39 @@ def run_ours(args):
     eager_ms = timed(step, 2, args.steps, False)
     runner.close()
 
-    attn_us, masked_pairs = time_attention_legs(case, dev, stream, flush)
-    bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    masked_leg = {
-        "mask": dict(MASKED_LEG), "visible_pairs": masked_pairs,
-        "causal_us": attn_us["causal"], "masked_us": attn_us["masked"],
-        "causal_tflops": attn_fl / attn_us["causal"] / 1e6,
-        "masked_tflops": 2048 * masked_pairs / attn_us["masked"] / 1e6,
-    }
-    masked_leg["masked_frac"] = masked_leg["masked_tflops"] / bf16_peak
-    rep_leg = time_rep_leg(T, dev, stream, flush)
-    rep_leg["embag_ln_frac"] = rep_leg["embag_ln_gbs"] / float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    rep_leg["linear_frac"] = rep_leg["linear_tflops"] / bf16_peak
-
+    detail = {"step_tflops": whole_step_tflops,
+              "step_frac_of_peak": whole_step_tflops / float(peaks.get("bf16_tflops", 1590.0)),
+              "us_per_layer": ms_max * 1e3 / n_layers,
+              "ms_p10": p10_max, "ms_p90": p90_max,
+              "runner": {"stride": RUNNER_STRIDE, "bucket_tokens": bucket,
+                         "device_buffers_ms_per_step": runner_ms, "host_buffers_ms_per_step": e2e_ms},
+              "eager_ms_per_step": eager_ms,
+              "kernels": kinds, "kernel_fractions": fractions(kinds, T, attn_fl, peaks),
+              "traced_step_ms": trace_ms,
+              "attention_flops_per_layer": attn_fl, "gemm_flops_per_layer": GEMM_FLOPS_PER_TOKEN * T}
     cpu = None
     if rank == 0 and world == 1:
-        sec, reps = time_oracle_layers(case, budget_s=15.0, max_reps=6, min_reps=2)
-        cpu = {"value": T / sec, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"numpy fp64 oracle, {reps} full-batch layers of this workload ({T} tokens each)"}
+        bf16_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        attn_us, masked_pairs = time_attention_legs(job, dev, stream, flush)
+        masked_leg = {
+            "mask": dict(MASKED_LEG), "visible_pairs": masked_pairs,
+            "causal_us": attn_us["causal"], "masked_us": attn_us["masked"],
+            "causal_tflops": attn_fl / attn_us["causal"] / 1e6,
+            "masked_tflops": 2048 * masked_pairs / attn_us["masked"] / 1e6,
+        }
+        masked_leg["masked_frac"] = masked_leg["masked_tflops"] / bf16_peak
+        rep_leg = time_rep_leg(T, dev, stream, flush)
+        rep_leg["embag_ln_frac"] = rep_leg["embag_ln_gbs"] / hbm_peak
+        rep_leg["linear_frac"] = rep_leg["linear_tflops"] / bf16_peak
+        detail["attention_legs"] = masked_leg
+        detail["rep_encoder"] = rep_leg
+        if os.environ.get("PTL_BENCH_LARGE", "1") != "0":
+            from packed_sequence_transformer_b200 import synthetic as S
+            detail["config3_stack8_44000tok"] = time_workload_leg(S.config3(), dev, stream, flush, peaks)
+            detail["config4_16x4096_skewed"] = time_workload_leg(S.config4(), dev, stream, flush, peaks,
+                                                                 attention_alone=True)
+        cpu = cpu_baseline(job)
 
     graph.reset()
     if world > 1:
@@ -584,26 +839,20 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; lognormal user lengths, random-init weights)",
-            "config": {"workload": case.name, "tokens": T, "users": U, "layers": n_layers,
-                       "head": head is not None, "parallelism": f"dp{world} (independent batches)",
+            "config": {"workload": job.name, "tokens": job.total_tokens, "users": job.num_users,
+                       "layers": n_layers, "head": head is not None,
+                       "parallelism": (f"users split by cost over {world} GPUs, head outputs all-gathered (NCCL)"
+                                       if world > 1 else "1 GPU"),
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "timing": "CUDA graph replay, CUDA events per step; per-kernel times from event nodes in a second captured graph"},
+                       "timing": "CUDA graph replay, CUDA events per step, median of the steps (max over ranks); "
+                                 "per-kernel times from event nodes in a second captured graph"},
             "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
-            "detail": {"step_tflops": whole_step_tflops,
-                       "step_frac_of_peak": whole_step_tflops / float(peaks.get("bf16_tflops", 1590.0)),
-                       "us_per_layer": ms_max * 1e3 / n_layers,
-                       "runner": {"stride": RUNNER_STRIDE, "bucket_tokens": bucket, "device_buffers_ms_per_step": runner_ms,
-                                  "host_buffers_ms_per_step": e2e_ms},
-                       "eager_ms_per_step": eager_ms,
-                       "attention_legs": masked_leg,
-                       "rep_encoder": rep_leg,
-                       "kernels": kinds, "attention_flops_per_layer": attn_fl,
-                       "gemm_flops_per_layer": GEMM_FLOPS_PER_TOKEN * T},
+            "detail": detail,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -391,6 +391,31 @@ ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* b
                            int64_t total_tokens, ptl_dtype dt, const ptl_rep_encoder_weights* w,
                            void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- One batch split across GPUs. ----
+ * Users are independent (a token attends only to its own user's tokens, and
+ * every other step works token by token: cti2026 README, packed batch with
+ * user_offsets and the FlashAttention_Varlen design), so one batch splits
+ * into contiguous user ranges, one per GPU; each GPU runs the single-GPU
+ * entry points on its range with rebased offsets cu_seqlens[b .. e] -
+ * cu_seqlens[b] and rows cu_seqlens[b] .. cu_seqlens[e] - 1, and the parts'
+ * outputs (rows, or compacted head probabilities, both in ascending token
+ * order) concatenated in part order equal the whole batch's.
+ * ptl_partition_users chooses the ranges: part r gets users user_begin[r] ..
+ * user_begin[r + 1] - 1.  A user of L tokens costs 6,299,648 L (one layer's
+ * GEMM FLOPs per token) + 1024 L (L + 1) (its attention FLOPs); the split
+ * minimises the largest part's cost over all contiguous splits (the smallest
+ * feasible bound, found by bisection over a greedy fill), then fills parts
+ * left to right up to that bound, so trailing parts may be empty when there
+ * are more parts than users.  Host arithmetic only (no GPU, no allocation).
+ *   cu_seqlens: HOST int32 [num_users + 1], 0-based and non-decreasing
+ *               (PTL_ERR_BAD_OFFSETS otherwise);
+ *   user_begin: HOST int32 [num_parts + 1], written: user_begin[0] = 0,
+ *               user_begin[num_parts] = num_users, non-decreasing.
+ * PTL_ERR_NULL for a NULL pointer, PTL_ERR_SHAPE for num_users < 1 or
+ * num_parts < 1. */
+ptl_status ptl_partition_users(const int32_t* cu_seqlens, int32_t num_users, int32_t num_parts,
+                               int32_t* user_begin);
+
 /* ---- Failure detection self-test. ----
  * Every wait inside the library's kernels (on an mbarrier phase, or on a
  * counter that another CTA of the same launch raises) is bounded: after a
@@ -418,8 +443,8 @@ const char* ptl_status_string(ptl_status s);
 /* Library ABI version (major * 100 + minor); PTL_VERSION is the value this
  * header describes.  Minor 1 added the graph runner, the masked attention, the
  * RepEncoder front end, the wait self-test and the PTL_ERR_BAD_MASK /
- * PTL_ERR_BAD_IDS codes. */
-#define PTL_VERSION 101
+ * PTL_ERR_BAD_IDS codes; minor 2 the user partitioner. */
+#define PTL_VERSION 102
 int32_t ptl_version(void);
 
 #ifdef __cplusplus

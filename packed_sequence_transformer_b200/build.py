@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libptl.so")
-SOURCES = ["api.cu", "kernels_simt.cu", "gemm_tc.cu", "attn_tc.cu", "noalloc.cu", "runner.cu"]
+SOURCES = ["api.cu", "kernels_simt.cu", "gemm_tc.cu", "attn_tc.cu", "noalloc.cu", "runner.cu", "partition.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-Xptxas", "-v"]

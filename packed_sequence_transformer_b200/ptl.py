@@ -135,6 +135,8 @@ _SIGS = {
     "ptl_attention_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
                               ctypes.c_int),
+    "ptl_partition_users": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, ctypes.c_int32,
+                             ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
 }
 
 
@@ -374,6 +376,28 @@ def attention_noalloc(qkv, attn, cu_seqlens, device_status=None, stream=None):
                                        _ptr(device_status), _stream(stream)),
            "ptl_attention_noalloc")
     return attn
+
+
+def partition_users(cu_seqlens, num_parts: int):
+    """ptl_partition_users: contiguous user ranges, one per part, balanced by
+    cost (host offsets in, host int32 [num_parts + 1] user boundaries out)."""
+    import numpy as np
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens), dtype=np.int32)
+    begin = np.zeros(num_parts + 1, dtype=np.int32)
+    _check(lib().ptl_partition_users(cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cu.size - 1,
+                                     num_parts, begin.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))),
+           "ptl_partition_users")
+    return begin
+
+
+def part_of_batch(cu_seqlens, user_begin, part: int):
+    """The slice of a batch that part `part` runs: (first token, end token,
+    first user, end user, rebased offsets int32 [users + 1])."""
+    import numpy as np
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    b, e = int(user_begin[part]), int(user_begin[part + 1])
+    t0, t1 = int(cu[b]), int(cu[e])
+    return t0, t1, b, e, (cu[b:e + 1] - t0).astype(np.int32)
 
 
 def last_device_error(workspace, stream=None) -> int:

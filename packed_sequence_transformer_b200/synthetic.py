@@ -195,6 +195,29 @@ def make_case(name: str, *, lengths=None, num_users=None, total=None, median=Non
     return _round_case(c)
 
 
+def replicate_batch(case: Case, copies: int, seed: int) -> Case:
+    """One batch of `copies` copies of the case's packing laid end to end:
+    copy 0 is the case's own activations (and prediction mask), copy r > 0
+    draws them afresh from ``default_rng(seed + r)`` with the same
+    distributions; the layer weights and the head are shared (a replicated
+    model serving a larger batch)."""
+    if copies == 1:
+        return case
+    xs, masks = [case.x], [case.pred_mask]
+    T = case.total_tokens
+    for r in range(1, copies):
+        rng = np.random.default_rng(seed + r)
+        x = rng.standard_normal(size=(T, D_MODEL), dtype=np.float32)
+        xs.append(round_to_bf16(x) if case.dtype == "bf16" else x)
+        if case.pred_mask is not None:
+            masks.append((rng.random(T) < 0.3).astype(np.uint8))
+    lengths = np.tile(case.lengths, copies)
+    return Case(name=f"{case.name}_x{copies}", dtype=case.dtype, cu_seqlens=offsets_from_lengths(lengths),
+                x=np.concatenate(xs), layers=case.layers, head=case.head,
+                pred_mask=None if case.pred_mask is None else np.concatenate(masks),
+                meta=dict(case.meta, copies=copies))
+
+
 # The five workloads.  Sizes, seeds and distributions as stated for each.
 def config0() -> Case:
     """fp32, 1 layer, 4 users of {3,7,12,20} tokens (42), seed 0."""

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(P):
 
 
 def test_status_strings_and_version(P):
-    assert P.version() == 101
+    assert P.version() == 102
     for code in range(10):
         assert P.status_string(code)
     assert P.status_string(99) == "unknown status"
@@ -197,4 +197,4 @@ def test_rep_encoder_host_checks(P):
 
 def test_version_matches_header(P):
     hdr = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ptl.h")).read()
-    assert P.lib().ptl_version() == int(re.search(r"#define PTL_VERSION (\d+)", hdr).group(1)) == 101
+    assert P.lib().ptl_version() == int(re.search(r"#define PTL_VERSION (\d+)", hdr).group(1)) == 102

@@ -1,10 +1,13 @@
-"""The N > 1 benchmark path on CPU: two gloo ranks, each with its own batch.
+"""The N > 1 benchmark path on CPU: two gloo ranks splitting one batch.
 
-The data path shards by batch (every rank runs the whole layer stack on its
-own packed batch; no collective touches activations), so what there is to
-test across ranks is the host logic: the slowest rank's step time decides
-the whole-job throughput, each rank draws a distinct batch of the same
-shape, and the reference arm runs on rank 0 alone.
+Users are independent, so the job's batch (N copies of the packing, one set
+of weights) is split into contiguous user ranges balanced by cost
+(ptl_partition_users); each rank runs the stack on its range with rebased
+offsets and the head probabilities are all-gathered at the end.  Here the
+oracle stands in for the GPU stack on a small batch, and the test checks that
+the gathered result equals the whole batch run on one rank, that the slowest
+rank's step time decides the whole-job throughput, and that the reference arm
+runs on rank 0 alone.
 """
 import json
 import os
@@ -23,10 +26,19 @@ def _free_port():
         return s.getsockname()[1]
 
 
+def _small_job(world):
+    from packed_sequence_transformer_b200 import synthetic as S
+    base = S.make_case("split", lengths=[3, 40, 0, 7, 129, 12, 1, 20], seed=5, dtype="bf16",
+                       num_layers=2, with_head=True)
+    return S.replicate_batch(base, world, seed=50)
+
+
 def _worker(rank, world, port, out_dir):
     import datetime
 
+    import torch
     import torch.distributed as dist
+    from oracle import ptl_oracle as O
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world,
@@ -35,10 +47,22 @@ def _worker(rank, world, port, out_dir):
         local_ms = 1.0 + 0.5 * rank  # the last rank is the slowest
         ms_max = bench.max_over_ranks(local_ms, world, "cpu")
         value = bench.job_value(6823, 8, world, ms_max)
-        case = bench.make_workload("layer", rank)
-        res = {"rank": rank, "ms_max": ms_max, "value": value, "T": case.total_tokens,
-               "x_sum": float(np.asarray(case.x, np.float64).sum()),
-               "cu": [int(v) for v in case.cu_seqlens]}
+        # one batch split by users: this rank's part through the oracle stack
+        job = _small_job(world)
+        t0, t1, cu = bench.rank_part(job, world, rank)
+        h, probs = O.stack_forward(job.x[t0:t1], cu, job.layers, head=job.head,
+                                   pred_mask=job.pred_mask[t0:t1])
+        cap = int(bench.max_over_ranks(t1 - t0, world, "cpu"))
+        loc = torch.zeros(cap, dtype=torch.float64)
+        loc[:probs.size] = torch.from_numpy(probs)
+        buf, cnt = bench.gather_parts(loc, torch.tensor([probs.size], dtype=torch.int64), world, cap)
+        rows = torch.zeros(cap * 512, dtype=torch.float64)
+        rows[:h.size] = torch.from_numpy(h.reshape(-1))
+        rbuf, rcnt = bench.gather_parts(rows, torch.tensor([h.size], dtype=torch.int64), world, cap * 512)
+        res = {"rank": rank, "ms_max": ms_max, "value": value, "tokens": [t0, t1],
+               "probs": bench.concat_parts(buf, cnt, cap).tolist(),
+               "rows_sum": float(bench.concat_parts(rbuf, rcnt, cap * 512).sum()),
+               "rows_n": int(bench.concat_parts(rbuf, rcnt, cap * 512).size)}
         with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
             json.dump(res, f)
         dist.barrier()
@@ -46,20 +70,44 @@ def _worker(rank, world, port, out_dir):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_max_time_and_distinct_batches(tmp_path):
+def test_two_gloo_ranks_split_one_batch_and_gather(tmp_path):
+    from oracle import ptl_oracle as O
     world = 2
     mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
     res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
     slowest = 1.0 + 0.5 * (world - 1)
+    job = _small_job(world)
+    h_all, p_all = O.stack_forward(job.x, job.cu_seqlens, job.layers, head=job.head,
+                                   pred_mask=job.pred_mask)
     for r in res:
         assert r["ms_max"] == pytest.approx(slowest)
         # whole-job tokens x layers over the slowest rank's time
         assert r["value"] == pytest.approx(6823 * 8 * world / (slowest / 1e3))
-        assert r["T"] == 6823
-    # same packing (weak scaling: per-rank work fixed), different data
-    assert res[0]["cu"] == res[1]["cu"]
-    assert res[0]["x_sum"] != res[1]["x_sum"]
+        # every rank gathers the whole batch's result, in token order
+        np.testing.assert_allclose(r["probs"], p_all, rtol=0, atol=1e-12)
+        assert r["rows_n"] == h_all.size
+        assert r["rows_sum"] == pytest.approx(float(h_all.sum()), abs=1e-9)
+    # the parts are contiguous, disjoint and cover the batch
+    assert res[0]["tokens"][0] == 0 and res[0]["tokens"][1] == res[1]["tokens"][0]
+    assert res[1]["tokens"][1] == job.total_tokens
+
+
+def test_job_batch_copies_share_weights_not_data():
+    one = bench.make_workload("layer", 1)
+    two = bench.make_workload("layer", 2)
+    T = one.total_tokens
+    assert two.total_tokens == 2 * T and two.num_users == 2 * one.num_users
+    np.testing.assert_array_equal(two.x[:T], one.x)
+    assert not np.array_equal(two.x[T:], one.x)
+    for a, b in zip(two.layers, one.layers):
+        for k in a:
+            np.testing.assert_array_equal(a[k], b[k])
+    # the cost-balanced split gives each rank one copy of the packing
+    for rank in range(2):
+        t0, t1, cu = bench.rank_part(two, 2, rank)
+        assert (t0, t1) == (rank * T, (rank + 1) * T)
+        np.testing.assert_array_equal(cu, one.cu_seqlens)
 
 
 def test_single_rank_helpers_need_no_process_group():
