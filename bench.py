@@ -270,6 +270,59 @@ def time_rep_leg(T, dev, stream, flush, reps=10, vocab=50_000, max_bag=4, seed=9
             "linear_tflops": flops / gemm_us / 1e6}
 
 
+def time_fp8_leg(T, dev, stream, flush, peaks, reps=10, seed=12):
+    """The FP8 (e4m3) linear layers on T tokens: per-row quantisation of the
+    activations, then the tcgen05 kind::f8f6f4 GEMM at the QKV shape
+    (512 -> 1536) and the expert GEMM1 shape (512 -> 1024), against an e4m3
+    dense peak taken as the measured bf16 peak times the nominal e4m3 / bf16
+    ratio (4.5 / 2.25 PFLOP/s)."""
+    import torch
+
+    from packed_sequence_transformer_b200 import ptl
+    g = torch.Generator(device=dev).manual_seed(seed)
+    x = torch.randn(T, 512, device=dev, generator=g).to(torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    fp8_peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    res = {"tokens": T, "fp8_peak_tflops": fp8_peak,
+           "fp8_peak_source": "measured bf16_tflops burst x 2 (nominal e4m3 / bf16 dense ratio 4.5 / 2.25)"}
+    with torch.cuda.stream(stream):
+        xq, sx = ptl.quantize_rows_e4m3(x, stream=stream)
+        for name, n_out in (("qkv_512x1536", 1536), ("expert1_512x1024", 1024)):
+            w = (0.02 * torch.randn(n_out, 512, device=dev, generator=g)).to(torch.bfloat16)
+            wq, sw = ptl.quantize_rows_e4m3(w, stream=stream)
+            out = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
+            ms = []
+            for i in range(reps + 3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                ptl.linear_fp8(xq, sx, wq, sw, None, out, ws, stream=stream)
+                b.record(stream)
+                if i >= 3:
+                    ms.append((a, b))
+                flush.fill_(float(i))
+            torch.cuda.synchronize()
+            us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ms)
+            tf = 2 * T * 512 * n_out / us / 1e6
+            res[name] = {"us": us, "tflops": tf, "frac_of_fp8_peak": tf / fp8_peak}
+        qs = []
+        for i in range(reps + 3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ptl.quantize_rows_e4m3(x, xq, sx, stream=stream)
+            b.record(stream)
+            if i >= 3:
+                qs.append((a, b))
+            flush.fill_(float(i))
+        torch.cuda.synchronize()
+        q_us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in qs)
+    if ptl.last_device_error(ws, stream) != 0:
+        raise RuntimeError("device error in the FP8 leg")
+    qbytes = T * 512 * (2 + 1) + 4 * T
+    res["quantize_rows_us"] = q_us
+    res["quantize_rows_gbs"] = qbytes / q_us / 1e3
+    return res
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples (every 200 ms) while the timed region runs."""
@@ -823,6 +876,7 @@ def run_ours(args):
         rep_leg["linear_frac"] = rep_leg["linear_tflops"] / bf16_peak
         detail["attention_legs"] = masked_leg
         detail["rep_encoder"] = rep_leg
+        detail["fp8_linear"] = time_fp8_leg(T, dev, stream, flush, peaks)
         if os.environ.get("PTL_BENCH_LARGE", "1") != "0":
             from packed_sequence_transformer_b200 import synthetic as S
             detail["config3_stack8_44000tok"] = time_workload_leg(S.config3(), dev, stream, flush, peaks)

@@ -391,6 +391,35 @@ ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* b
                            int64_t total_tokens, ptl_dtype dt, const ptl_rep_encoder_weights* w,
                            void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- FP8 (e4m3) linear layers. ----
+ * Low-precision GEMMs for the layer's projections (cry-daniel/recsys README:
+ * FP8 in its feature list; the CTI-Inference-Opt optimisation plan's INT8
+ * section as the motivation).  The pages fix no recipe; the reading taken is
+ * e4m3 codes (4 exponent bits, bias 7, 3 mantissa bits, largest finite 448)
+ * with one float32 scale per row of each operand: rows of the activations
+ * (tokens) and rows of the weight (output channels).
+ * ptl_quantize_rows_e4m3: scales[r] = max_c |x[r][c]| / 448 (1 for an
+ *   all-zero row) and codes[r][c] = e4m3(x[r][c] / scales[r]), both the scale
+ *   and the quotient IEEE float32 operations (correctly rounded), the code
+ *   rounded to the nearest e4m3 value, ties to even, saturating at +-448.
+ *   x: device [rows][cols] in dt; codes: device uint8 [rows][cols]; scales:
+ *   device float [rows].  cols a multiple of 16 (>= 16), x and codes 16-byte
+ *   aligned, scales 4-byte aligned.  Asynchronous on `stream`.
+ * ptl_linear_fp8: out[m][n] = bf16((sum_k xq[m][k] wq[n][k]) * sx[m] * sw[n]
+ *   + b[n]): the code products summed in float32 on the tensor cores
+ *   (tcgen05 kind::f8f6f4, 256 x 256 tiles on CTA pairs), then scaled.
+ *   xq [M][K] with sx [M] and wq [N][K] with sw [N] as ptl_quantize_rows_e4m3
+ *   writes them; bias (nullable) float [N]; out device bf16 [M][N].  K a
+ *   multiple of 128, N a multiple of 256, M < 2^31; codes and out 16-byte
+ *   aligned.  workspace: >= 256 bytes, 256-byte aligned (its error word, read
+ *   by ptl_last_device_error: PTL_ERR_TIMEOUT if a bounded wait ran out).
+ *   PTL_ERR_SHAPE for other sizes; M == 0 returns PTL_OK with no launch. */
+ptl_status ptl_quantize_rows_e4m3(const void* x, ptl_dtype dt, int64_t rows, int32_t cols, uint8_t* codes,
+                                  float* scales, void* stream);
+ptl_status ptl_linear_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                          const float* bias, void* out, int64_t rows, int32_t in_features,
+                          int32_t out_features, void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- One batch split across GPUs. ----
  * Users are independent (a token attends only to its own user's tokens, and
  * every other step works token by token: cti2026 README, packed batch with
@@ -443,7 +472,7 @@ const char* ptl_status_string(ptl_status s);
 /* Library ABI version (major * 100 + minor); PTL_VERSION is the value this
  * header describes.  Minor 1 added the graph runner, the masked attention, the
  * RepEncoder front end, the wait self-test and the PTL_ERR_BAD_MASK /
- * PTL_ERR_BAD_IDS codes; minor 2 the user partitioner. */
+ * PTL_ERR_BAD_IDS codes; minor 2 the user partitioner and the FP8 linear layers. */
 #define PTL_VERSION 102
 int32_t ptl_version(void);
 

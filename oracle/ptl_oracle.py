@@ -303,21 +303,34 @@ def quantize_e4m3(x):
     return np.sign(x) * q
 
 
-def quantize_rows_e4m3(x):
+def quantize_rows_e4m3(x, precision=None):
     """Per-row scaled e4m3: s = max|row| / 448 (1 for an all-zero row),
-    codes = quantize_e4m3(row / s); returns (codes, s) with row ~ codes * s."""
+    codes = quantize_e4m3(row / s); returns (codes, s) with row ~ codes * s.
+
+    precision=None computes s and the quotient in float64.  precision='f32'
+    computes both as IEEE float32 operations (numpy's float32 division is
+    correctly rounded): the code is an integer decided by floating point, and
+    this is the precision a float32 kernel decides it in, so both sides pick
+    the same code (the float64 quotient can fall on the other side of an e4m3
+    rounding boundary when it lies within a float32 rounding of it)."""
+    if precision == "f32":
+        x32 = np.asarray(x, dtype=np.float32)
+        amax = np.abs(x32).max(axis=-1, keepdims=True)
+        s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        return quantize_e4m3((x32 / s).astype(np.float32)), s[..., 0].astype(np.float64)
     x = _f64(x)
     amax = np.abs(x).max(axis=-1, keepdims=True)
     s = np.where(amax > 0, amax / E4M3_MAX, 1.0)
     return quantize_e4m3(x / s), s[..., 0]
 
 
-def linear_fp8(x, weight, bias=None):
+def linear_fp8(x, weight, bias=None, precision=None):
     """y = x W^T + b with both operands quantised per row (rows of x = tokens,
     rows of W = output channels) to e4m3; the products of the codes are summed
-    exactly (fp64 here; fp32 on the tensor cores) and scaled by s_x[i] s_w[j]."""
-    qx, sx = quantize_rows_e4m3(x)
-    qw, sw = quantize_rows_e4m3(weight)
+    exactly (fp64 here; fp32 on the tensor cores) and scaled by s_x[i] s_w[j].
+    precision: where the codes are decided (see quantize_rows_e4m3)."""
+    qx, sx = quantize_rows_e4m3(x, precision)
+    qw, sw = quantize_rows_e4m3(weight, precision)
     y = (qx @ qw.T) * sx[:, None] * sw[None, :]
     if bias is not None:
         y = y + _f64(bias)

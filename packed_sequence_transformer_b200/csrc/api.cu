@@ -125,6 +125,20 @@ bool map_f32(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uin
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D byte tensor map (e4m3 codes): box = box_rows x 128 bytes (the swizzle span).
+bool map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t stride_bytes,
+            uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 ptl_status device_ok() {
   static int cache[64];  // 0 unknown, 1 ok, 2 unsupported
   int dev = 0;
@@ -678,6 +692,54 @@ ptl_status ptl_rep_encoder(const int64_t* ids, int64_t num_ids, const int64_t* b
     PTL_TRY(launch_gemm_f32(0, reinterpret_cast<const float*>(normed), REP_W, F32(w->w), w->b, nullptr,
                             static_cast<float*>(out), D, T, D, REP_W, L, ws, st));
   }
+  return PTL_OK;
+}
+
+ptl_status ptl_quantize_rows_e4m3(const void* x, ptl_dtype dt, int64_t rows, int32_t cols, uint8_t* codes,
+                                  float* scales, void* stream) {
+  ApiRange nvtx_range{"ptl_quantize_rows_e4m3"};
+  if (dt != PTL_F32 && dt != PTL_BF16) return PTL_ERR_DTYPE;
+  if (rows < 0 || cols < 16 || cols % 16 != 0) return PTL_ERR_SHAPE;
+  if (rows == 0) return PTL_OK;
+  if (!x || !codes || !scales) return PTL_ERR_NULL;
+  if (!a16(x) || !a16(codes) || !a4(scales)) return PTL_ERR_ALIGN;
+  ptl_status s;
+  if ((s = device_ok()) != PTL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  EndMark end_mark{st};
+  mark(st, PTL_KERNEL_LAYERNORM);
+  PTL_TRY(launch_quant_rows_e4m3(x, dt, rows, cols, codes, scales, st));
+  return PTL_OK;
+}
+
+ptl_status ptl_linear_fp8(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                          const float* bias, void* out, int64_t rows, int32_t in_features,
+                          int32_t out_features, void* workspace, size_t ws_bytes, void* stream) {
+  ApiRange nvtx_range{"ptl_linear_fp8"};
+  if (rows < 0 || rows >= (int64_t(1) << 31) || in_features < 128 || in_features % 128 != 0 ||
+      out_features < 256 || out_features % 256 != 0)
+    return PTL_ERR_SHAPE;
+  if (!workspace) return PTL_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return PTL_ERR_ALIGN;
+  if (ws_bytes < 256) return PTL_ERR_WORKSPACE;
+  if (rows == 0) return PTL_OK;
+  if (!xq || !sx || !wq || !sw || !out) return PTL_ERR_NULL;
+  if (!a16(xq) || !a16(wq) || !a16(out) || !a4(sx) || !a4(sw) || !opt16(bias)) return PTL_ERR_ALIGN;
+  ptl_status s;
+  if ((s = device_ok()) != PTL_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* err = static_cast<int32_t*>(workspace);
+  CUtensorMap ma, mb, mo;
+  if (!map_u8(&ma, xq, uint64_t(in_features), uint64_t(rows), uint64_t(in_features), 128)) return PTL_ERR_CUDA;
+  if (!map_u8(&mb, wq, uint64_t(in_features), uint64_t(out_features), uint64_t(in_features), 128))
+    return PTL_ERR_CUDA;
+  if (!map_bf16(&mo, out, uint64_t(out_features), uint64_t(rows), uint64_t(out_features) * 2, 64, 128))
+    return PTL_ERR_CUDA;
+  mark(st, PTL_KERNEL_CLEAR);
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), st) != cudaSuccess) return PTL_ERR_CUDA;
+  EndMark end_mark{st};
+  mark(st, PTL_KERNEL_GEMM_QKV);
+  PTL_TRY(launch_gemm_fp8(ma, mb, mo, sx, sw, bias, int(rows), out_features, in_features, err, st));
   return PTL_OK;
 }
 

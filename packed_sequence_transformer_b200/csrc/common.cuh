@@ -20,9 +20,12 @@ constexpr int QKV_N = 3 * D;       // 1536
 constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
 constexpr int MOE_BM = 256;        // rows per expert tile (padding granule; one CTA pair's M)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
-constexpr int GR_TOK = 16;         // tokens per block of the fused gate + route kernel
+constexpr int GR_WARPS = 16;       // warps per block of the fused gate + route kernel
+constexpr int GR_TPW = 4;          // tokens per warp of that kernel
+constexpr int GR_TOK = GR_WARPS * GR_TPW;  // tokens per block (one chunk of routes)
 constexpr int ATT_MAX_CTAS = 1024;  // bound on the persistent attention grid
 constexpr int GEMM2_BN = 256;      // expert GEMM2 output columns per tile
+constexpr int MOE1_NT = F / 256;   // expert GEMM1 column tiles per M tile (256 wide)
 constexpr float LN_EPS = 1e-5f;
 constexpr float LOGIT_CLAMP = 15.0f;
 
@@ -47,7 +50,7 @@ struct WsLayout {
   size_t wgt;         // f32 [T][2]
   size_t chunk_cnt;   // int32 [n_chunks][8]
   size_t lb;          // int32 [32 + 32 * n_gchunks]  fused gate + route: ticket, per-chunk look-back state
-  size_t moe_done;    // int32 [max_tiles]  fused expert GEMMs: first-GEMM tiles done per M tile
+  size_t moe_done;    // int32 [max_tiles][MOE1_NT]  fused expert GEMMs: first-GEMM tiles done (CTAs)
   size_t perm;        // int32 [2T]
   size_t pos;         // int32 [2T]          route -> padded expert row
   size_t rowroute;    // int32 [padded_rows]   padded expert rows -> route (or -1)
@@ -114,7 +117,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->wl_end = o;  // error word + attention work list
   L->chunk_cnt = take(4 * L->n_chunks * E);
   L->lb = take(4 * (32 + 32 * L->n_gchunks));
-  L->moe_done = take(4 * L->max_tiles);
+  L->moe_done = take(4 * L->max_tiles * MOE1_NT);
   L->clear_end = o;  // [0, clear_end) is cleared by one memset per call
   L->xn = take(es * T * D);
   L->qkv = take(es * T * QKV_N);

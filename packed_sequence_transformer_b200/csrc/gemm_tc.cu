@@ -16,10 +16,12 @@
 //   warp 1      allocates TMEM (both CTAs); in CTA 0 one thread issues the
 //               MMAs (M=256, N=BN, K=16), commits each ring stage back to both
 //               producers and each finished accumulator to both epilogues;
-//   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane),
-//               reads it with tcgen05.ld, releases the accumulator on CTA 0
-//               (one arrival per warp), applies the fused epilogue and stages
-//               the tile for a TMA bulk-tensor store.
+//   warps 2..9  epilogue: each thread owns one accumulator row (TMEM lane)
+//               and one half of the tile's columns (two warps per TMEM lane
+//               quarter), reads them with tcgen05.ld, releases the
+//               accumulator on CTA 0 (one arrival per warp), applies the
+//               fused epilogue and stages the tile for a TMA bulk-tensor
+//               store.
 // Sharing B across the pair halves B's shared-memory traffic per output: at
 // this problem size the GEMMs are bound by L2 -> SM operand traffic, so the
 // tile shape is chosen for bytes per FLOP.
@@ -29,6 +31,8 @@
 //   MOE1  H[row] = ReLU(xperm[row] W1[e]^T + b1[e])       (A by TMA: the route
 //         builder copies each route's LayerNorm2 row to its padded row)
 //   MOE2  Y[row] = H[row] W2[e]^T + b2[e]                 (A by TMA)
+//   FP8   out = (xq wq^T) * sx[row] * sw[col] + b         (e4m3 codes, kind::f8f6f4;
+//         a 128-byte K slice holds 128 codes, so K steps by 128)
 //         (per-route expert outputs in padded row order, bf16; the top-2
 //         weighted combine + residual runs in combine_bf16_kernel)
 // The expert GEMMs' rows are padded per expert to 256 (one pair tile never
@@ -66,9 +70,20 @@ struct GemmTcParams {
   const float* bias2;
   int32_t* done;
   int32_t* err;
+  // FP8: per-row scales of A (rows of the output) and of B (its columns)
+  const float* sx;
+  const float* sw;
 };
 
-enum { G_QKV = 0, G_OUT = 1, G_MOE1 = 2, G_MOE2 = 3, G_MOE12 = 4 };
+enum { G_QKV = 0, G_OUT = 1, G_MOE1 = 2, G_MOE2 = 3, G_MOE12 = 4, G_FP8 = 5 };
+// expert modes: rows padded per expert, tiles from the route builder's list
+__host__ __device__ constexpr bool is_moe(int mode) { return mode == G_MOE1 || mode == G_MOE2 || mode == G_MOE12; }
+
+// Warps per CTA: producer, MMA issuer, and 8 epilogue warps (two per TMEM
+// lane quarter, each taking half of the tile's columns).
+constexpr int GEMM_EPI_WARPS = 8;
+constexpr int GEMM_STORE_WARP = 2 + GEMM_EPI_WARPS;  // issues the bf16 tiles' TMA stores
+constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS + 32;
 
 // Shared-memory plan: the operand ring, the output staging tile and the
 // tile's bias slice.
@@ -82,7 +97,8 @@ struct PairCfg {
   static constexpr int STAGING = 128 * PART * OUT_ELEM;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = (BN / 2) * 64 * 2;
-  static constexpr int BIAS = BN * 4;
+  // bias (+ FP8: the weight rows' scales), double-buffered by tile
+  static constexpr int BIAS = 2 * (MODE == G_FP8 ? 2 : 1) * BN * 4;
   static constexpr int USABLE = 232448 - 1024 - 256 - 64;
   static constexpr int STAGES_FIT = (USABLE - STAGING - BIAS) / (A_BYTES + B_BYTES);
   static constexpr int STAGES = STAGES_FIT > 10 ? 10 : STAGES_FIT;
@@ -108,7 +124,7 @@ __device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile
   }
   mt = tile / nN;
   n0 = (tile - mt * nN) * BN;
-  if (MODE >= G_MOE1) {
+  if (is_moe(MODE)) {
     const int2 tl = p.tiles[mt];
     expert = tl.x;
     m0 = tl.y;
@@ -123,7 +139,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 
 template <int BN, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut2,
@@ -139,8 +155,10 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg::STAGING + Cfg::BIAS);  // [stage] (CTA 0's counts)
   uint64_t* empty = full + STAGES;    // [stage] ring slot free (both CTAs)
   uint64_t* tfull = empty + STAGES;   // [2] accumulator ready (both CTAs)
-  uint64_t* tempty = tfull + 2;       // [2] accumulator drained (CTA 0's counts: 8 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tempty = tfull + 2;       // [2] accumulator drained (CTA 0's counts: every epilogue warp of both CTAs)
+  uint64_t* stg_full = tempty + 2;    // staging tile written (epilogue warps)
+  uint64_t* stg_empty = stg_full + 1;  // staging tile read by its TMA store (store thread)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stg_empty + 1);
   __shared__ int s_ntiles;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -153,8 +171,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);
+      mbar_init(&tempty[a], 2 * GEMM_EPI_WARPS);
     }
+    mbar_init(stg_full, GEMM_EPI_WARPS);
+    mbar_init(stg_empty, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -178,8 +198,8 @@ __global__ void __launch_bounds__(192, 1)
   pdl_trigger();  // dependents launch once this grid has passed its own wait
   __shared__ int s_nmt;
   if (threadIdx.x == 0) {
-    const int nmt = MODE >= G_MOE1 ? p.meta[0] : 0;
-    int nt = MODE >= G_MOE1 ? nmt * (p.N_total / BN) : p.n_tiles_dense;
+    const int nmt = is_moe(MODE) ? p.meta[0] : 0;
+    int nt = is_moe(MODE) ? nmt * (p.N_total / BN) : p.n_tiles_dense;
     if (MODE == G_MOE12) nt += nmt * (p.N2 / BN);
     s_ntiles = has_error(p.err) ? 0 : nt;
     s_nmt = nmt;
@@ -208,17 +228,18 @@ __global__ void __launch_bounds__(192, 1)
         const int nkb = second ? p.N_total / 64 : p.num_kb;
         const CUtensorMap* ma = second ? &tmA2 : &tmA;
         const CUtensorMap* mb = second ? &tmB2 : &tmB;
-        if (MODE == G_MOE12 && second) {
-          // the tile's A rows (H) come from every first-GEMM tile of this M
-          // tile, each stored by both CTAs of its pair
-          if (!wait_flag_at_least(p.done + mt, 2 * (p.N_total / BN))) {
-            set_error(p.err, PTL_ERR_TIMEOUT);
-            ok = false;
-            break;
-          }
-          fence_proxy_async_global();  // the H rows were written by TMA stores
-        }
         for (int kb = 0; kb < nkb; ++kb, ++it) {
+          if (MODE == G_MOE12 && second && kb % (BN / 64) == 0) {
+            // this K slice of the tile's A rows (H) is one first-GEMM column
+            // tile of this M tile, stored by both CTAs of its pair: start on
+            // it as soon as that tile is done, not the whole row
+            if (!wait_flag_at_least(p.done + mt * MOE1_NT + kb / (BN / 64), 2)) {
+              set_error(p.err, PTL_ERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();  // the H rows were written by TMA stores
+          }
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1)) {
             set_error(p.err, PTL_ERR_TIMEOUT);
@@ -227,14 +248,16 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (cr == 0) mbar_arrive_expect_tx(&full[s], tx);
           const uint32_t fb = full0 + uint32_t(s) * 8u;
-          tma_load_2d_pair(sA + s * Cfg::A_BYTES, ma, fb, kb * 64, arow);
-          tma_load_2d_pair(sB + s * Cfg::B_BYTES, mb, fb, kb * 64, brow);
+          // a K slice is one 128-byte swizzle row: 64 bf16 or 128 e4m3 elements
+          constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;
+          tma_load_2d_pair(sA + s * Cfg::A_BYTES, ma, fb, kb * KSLICE, arow);
+          tma_load_2d_pair(sB + s * Cfg::B_BYTES, mb, fb, kb * KSLICE, brow);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && cr == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(256, BN);
+      constexpr uint32_t idesc = MODE == G_FP8 ? umma_idesc_e4m3(256, BN) : umma_idesc_bf16(256, BN);
       int it = 0, j = 0;
       bool ok = true;
       for (int tile = pair; tile < ntiles && ok; tile += npairs, ++j) {
@@ -259,33 +282,62 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * Cfg::A_BYTES);
           const uint32_t b0 = smem_u32(sB + s * Cfg::B_BYTES);
+          // four MMAs per 128-byte K slice: K = 16 bf16 or 32 e4m3 each
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16_ss_pair(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
-                              (kb | k) != 0);
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (MODE == G_FP8)
+              umma_e4m3_ss_pair(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
+                                (kb | k) != 0);
+            else
+              umma_bf16_ss_pair(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
+                                (kb | k) != 0);
+          }
           umma_commit_pair(&empty[s], 0x3);
         }
         umma_commit_pair(&tfull[acc], 0x3);
       }
     }
+  } else if (warp == GEMM_STORE_WARP) {
+    // Store thread (bf16 outputs): per tile, once the epilogue warps have
+    // staged it, issue its TMA stores, free the staging tile as soon as the
+    // stores have read it, and -- first expert GEMM -- once they are
+    // complete, count the tile for the second GEMM's producers.  Its waits
+    // for the stores keep the epilogue warps and the tensor core running.
+    if (MODE != G_OUT && lane == 0) {
+      int jj = 0;
+      for (int tile = pair; tile < ntiles; tile += npairs, ++jj) {
+        int expert, m0, n0, mt;
+        bool second;
+        decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt);
+        m0 += 128 * int(cr);
+        if (!mbar_wait(stg_full, jj & 1)) {
+          set_error(p.err, PTL_ERR_TIMEOUT);
+          break;
+        }
+        const CUtensorMap* mo = second ? &tmOut2 : &tmOut;
+#pragma unroll 1
+        for (int bx = 0; bx < BN / Cfg::BOX_COLS; ++bx) tma_store_2d(mo, sOut + bx * 16384, n0 + bx * Cfg::BOX_COLS, m0);
+        tma_store_commit();
+        tma_store_wait_read();
+        mbar_arrive(stg_empty);
+        if (MODE == G_MOE12 && !second) {
+          tma_store_wait_all();
+          fence_proxy_async_global();
+          red_release_gpu_add(p.done + mt * MOE1_NT + n0 / BN, 1);
+        }
+      }
+      tma_store_wait_all();
+    }
   } else {
-    // Epilogue warps 2..5 of each CTA: row r of this CTA's 128 rows.
+    // Epilogue warps 2..9 of each CTA: row r of this CTA's 128 rows (a warp
+    // reads the TMEM lanes of its quarter, warp % 4), column half eg of the
+    // tile (warps 2..5 the first half, 6..9 the second).
     const int r = 32 * (warp & 3) + lane;
+    const int eg = (warp - 2) >> 2;
+    const int et = int(threadIdx.x) - 64;  // 0 .. 255 over the epilogue threads
     const uint32_t lane_off = uint32_t(32 * (warp & 3)) << 16;
     const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);
     int j = 0;
-    int pending_mt = -1;  // MOE12: M tile of the first-GEMM tile whose store is in flight
-    // MOE12: once this CTA's store of a first-GEMM tile is complete, count it
-    // for the second GEMM's producers (leader thread, right after the store:
-    // a pair's own later second-GEMM tiles may be the ones waiting for it)
-    auto publish = [&]() {
-      if (MODE == G_MOE12 && pending_mt >= 0) {
-        tma_store_wait_all();
-        fence_proxy_async_global();
-        red_release_gpu_add(p.done + pending_mt, 1);
-        pending_mt = -1;
-      }
-    };
     for (int tile = pair; tile < ntiles; tile += npairs, ++j) {
       int expert, m0, n0, mt;
       bool second;
@@ -294,123 +346,176 @@ __global__ void __launch_bounds__(192, 1)
       const int acc = j & 1;
       const int row = m0 + r;
       const float* bias_base = second ? p.bias2 : p.bias;
-      const float* bb = bias_base ? bias_base + (MODE >= G_MOE1 ? expert * (second ? p.N2 : p.N_total) : 0) + n0
+      const float* bb = bias_base ? bias_base + (is_moe(MODE) ? expert * (second ? p.N2 : p.N_total) : 0) + n0
                                   : nullptr;
       const bool relu = MODE == G_MOE1 || (MODE == G_MOE12 && !second);
-      float bv[(BN + 127) / 128];
-#pragma unroll
-      for (int i = 0; i < (BN + 127) / 128; ++i)
-        bv[i] = (bb && r + 128 * i < BN) ? __ldg(bb + r + 128 * i) : 0.f;
+      static_assert(BN <= 32 * 2 * GEMM_EPI_WARPS, "one bias value per epilogue thread");
+      const float bv = (bb && et < BN) ? __ldg(bb + et) : 0.f;
+      const float swv = (MODE == G_FP8 && et < BN) ? __ldg(p.sw + n0 + et) : 0.f;
+      const float sxr = (MODE == G_FP8 && row < p.M) ? __ldg(p.sx + row) : 0.f;
       constexpr int PART = Cfg::PART, NPART = BN / PART;
-      constexpr int NRES = MODE == G_OUT ? PART / 8 : 1;
-      uint4 res[NRES];  // this thread's residual row, one part at a time
+      constexpr int CPG = PART / 64;  // 32-column chunks of a part per column half
+      static_assert(PART % 64 == 0, "a part splits into two halves of whole chunks");
+      constexpr int NRES = MODE == G_OUT ? PART / 16 : 1;
+      uint4 res[NRES];  // this thread's half of its residual row, one part at a time
       auto load_res = [&](int pt) {
         if (MODE == G_OUT) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0 + pt * PART);
+          const uint4* src = reinterpret_cast<const uint4*>(p.resid + size_t(row < p.M ? row : 0) * D + n0 + pt * PART +
+                                                            eg * (PART / 2));
 #pragma unroll
           for (int q = 0; q < NRES; ++q) res[q] = row < p.M ? __ldg(src + q) : make_uint4(0, 0, 0, 0);
         }
       };
       load_res(0);
       const bool leader = warp == 2 && lane == 0;
-      if (j > 0 && leader) {
-        tma_store_wait_read();
-        publish();
-      }
-#pragma unroll
-      for (int i = 0; i < (BN + 127) / 128; ++i)
-        if (r + 128 * i < BN) s_bias[r + 128 * i] = bv[i];
-      named_barrier(1, 128);
+      // the fp32 output stages in parts through the leader's own stores; the
+      // bf16 outputs go through the store thread
+      if (MODE == G_OUT && j > 0 && leader) tma_store_wait_read();
+      // this tile's bias (+ scales) in buffer j % 2: the barrier below is
+      // passed only once every thread has finished tile j - 1, which read
+      // the other buffer
+      float* const sb = s_bias + (j & 1) * (Cfg::BIAS / 8);
+      if (et < BN) sb[et] = bv;
+      if (MODE == G_FP8 && et < BN) sb[BN + et] = swv;
+      named_barrier(1, 32 * GEMM_EPI_WARPS);
       if (!mbar_wait(&tfull[acc], (j >> 1) & 1)) {
         set_error(p.err, PTL_ERR_TIMEOUT);
         break;
       }
       tc_fence_after();
       const uint32_t taddr = tmem + uint32_t(acc * BN) + lane_off;
-#pragma unroll 1
-      for (int pt = 0; pt < NPART; ++pt) {
-        if (pt > 0) {  // the previous part's store must have read the staging tile
-          load_res(pt);
-          if (leader) tma_store_wait_read();
-          named_barrier(1, 128);
+      // bias (+ FP8 scales, + ReLU) on 32 accumulator columns starting at `col`
+      auto finish32 = [&](float (&v)[32], int col) {
+        if (MODE == G_FP8) {  // code products times the row's and the column's scales
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 s4 = *reinterpret_cast<const float4*>(sb + BN + col + 4 * q);
+            v[4 * q] = v[4 * q] * sxr * s4.x;
+            v[4 * q + 1] = v[4 * q + 1] * sxr * s4.y;
+            v[4 * q + 2] = v[4 * q + 2] * sxr * s4.z;
+            v[4 * q + 3] = v[4 * q + 3] * sxr * s4.w;
+          }
         }
 #pragma unroll
-        for (int c = 0; c < PART / 32; ++c) {
-          const int col = pt * PART + 32 * c;  // column within the tile
+        for (int q = 0; q < 8; ++q) {
+          const float4 b4 = *reinterpret_cast<const float4*>(sb + col + 4 * q);
+          v[4 * q] += b4.x;
+          v[4 * q + 1] += b4.y;
+          v[4 * q + 2] += b4.z;
+          v[4 * q + 3] += b4.w;
+        }
+        if (relu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
+        }
+      };
+      if constexpr (MODE != G_OUT) {
+        // bf16 output: this thread's columns go through registers first, so
+        // the accumulator is released (and the tensor core can start the
+        // tile after next) before the staging tile is waited for
+        uint32_t pk[CPG][16];
+#pragma unroll
+        for (int cc = 0; cc < CPG; ++cc) {
+          const int col = 32 * (eg * CPG + cc);  // column within the tile
           uint32_t raw[32];
           tmem_ld32(taddr + col, raw);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(raw);
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+          finish32(v, col);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 b4 = *reinterpret_cast<const float4*>(s_bias + col + 4 * q);
-            v[4 * q] += b4.x;
-            v[4 * q + 1] += b4.y;
-            v[4 * q + 2] += b4.z;
-            v[4 * q + 3] += b4.w;
-          }
-          if (relu) {
+          for (int i = 0; i < 16; ++i) pk[cc][i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        }
+        // this warp's rows of the accumulator are read: release it on CTA 0
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+        // the previous tile's stores have read the staging tile
+        if (j > 0 && !mbar_wait(stg_empty, (j - 1) & 1)) {
+          set_error(p.err, PTL_ERR_TIMEOUT);
+          break;
+        }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
-          }
-          if (MODE == G_OUT) {
+        for (int cc = 0; cc < CPG; ++cc) {
+          // 32 bf16 = half a box row: box c/2, 16-byte chunks (c%2)*4 .. +3
+          const int c = eg * CPG + cc;
+          const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 u = res[4 * c + q];
-              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(h2[i]);
-                v[8 * q + 2 * i] += f.x;
-                v[8 * q + 2 * i + 1] += f.y;
-              }
-            }
-            // 32 fp32 = one 128-byte box row: box c of the part, chunks 0..7
-            const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                           __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
-          } else {
-            // 32 bf16 = half a box row: box c/2, chunks (c%2)*4 .. +3
-            const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int chunk = (c & 1) * 4 + q;
-              st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pack_bf16x2(v[8 * q], v[8 * q + 1]),
-                           pack_bf16x2(v[8 * q + 2], v[8 * q + 3]), pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                           pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-            }
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (c & 1) * 4 + q;
+            st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pk[cc][4 * q], pk[cc][4 * q + 1], pk[cc][4 * q + 2],
+                         pk[cc][4 * q + 3]);
           }
         }
-        if (pt == NPART - 1) {
-          // this warp's rows of the accumulator are read: release it on CTA 0
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
-        }
+        // staged: hand the tile to the store thread (one arrival per warp)
         fence_proxy_async_smem();
-        named_barrier(1, 128);
-        if (leader) {
-          const CUtensorMap* mo = second ? &tmOut2 : &tmOut;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(stg_full);
+      } else {
 #pragma unroll 1
-          for (int bx = 0; bx < PART / Cfg::BOX_COLS; ++bx)
-            tma_store_2d(mo, sOut + bx * 16384, n0 + pt * PART + bx * Cfg::BOX_COLS, m0);
-          tma_store_commit();
+        for (int pt = 0; pt < NPART; ++pt) {
+          if (pt > 0) {  // the previous part's store must have read the staging tile
+            load_res(pt);
+            if (leader) tma_store_wait_read();
+            named_barrier(1, 32 * GEMM_EPI_WARPS);
+          }
+          // the accumulator chunks of this thread, one TMEM load ahead: chunk
+          // cc + 1 loads while chunk cc is converted and staged
+          uint32_t rawA[32], rawB[32];
+          tmem_ld32(taddr + pt * PART + 32 * (eg * CPG), rawA);
+          tmem_ld_wait_regs(rawA);
+#pragma unroll
+          for (int cc = 0; cc < CPG; ++cc) {
+            const int c = eg * CPG + cc;  // chunk within the part
+            const int col = pt * PART + 32 * c;  // column within the tile
+            uint32_t(&raw)[32] = (cc & 1) ? rawB : rawA;
+            uint32_t(&nxt)[32] = (cc & 1) ? rawA : rawB;
+            if (cc + 1 < CPG) tmem_ld32(taddr + col + 32, nxt);
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+            finish32(v, col);
+            {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 u = res[4 * cc + q];
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float2 f = __bfloat1622float2(h2[i]);
+                  v[8 * q + 2 * i] += f.x;
+                  v[8 * q + 2 * i + 1] += f.y;
+                }
+              }
+              // 32 fp32 = one 128-byte box row: box c of the part, chunks 0..7
+              const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                             __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+            }
+            if (cc + 1 < CPG) tmem_ld_wait_regs(nxt);
+          }
+          if (pt == NPART - 1) {
+            // this warp's rows of the accumulator are read: release it on CTA 0
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+          }
+          fence_proxy_async_smem();
+          named_barrier(1, 32 * GEMM_EPI_WARPS);
+          if (leader) {
+            const CUtensorMap* mo = second ? &tmOut2 : &tmOut;
+#pragma unroll 1
+            for (int bx = 0; bx < PART / Cfg::BOX_COLS; ++bx)
+              tma_store_2d(mo, sOut + bx * 16384, n0 + pt * PART + bx * Cfg::BOX_COLS, m0);
+            tma_store_commit();
+          }
         }
       }
-      if (leader && MODE == G_MOE12 && !second) {
-        // publish right away: this pair's own second-GEMM tiles may wait on it
-        pending_mt = mt;
-        publish();
-      }
     }
-    if (warp == 2 && lane == 0) {
-      tma_store_wait_all();
-      publish();
-    }
+    if (MODE == G_OUT && warp == 2 && lane == 0) tma_store_wait_all();
   }
   tc_fence_before();
   cluster_sync();  // no MMA, TMEM read or remote arrival of either CTA is outstanding
@@ -432,7 +537,7 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   static PerDevice max_pairs_dev;
   const int smem = PairCfg<BN, MODE>::SMEM;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(GEMM_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -506,6 +611,21 @@ int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtenso
   p.ldo = D;
   p.err = err;
   return launch_pair<OUT_BN, G_OUT>(attn, w, x1_out, p, p.n_tiles_dense, st);
+}
+
+int launch_gemm_fp8(const CUtensorMap& xq, const CUtensorMap& wq, const CUtensorMap& out_map, const float* sx,
+                    const float* sw, const float* bias, int M, int N, int Kd, int32_t* err, cudaStream_t st) {
+  GemmTcParams p{};
+  p.M = M;
+  p.N_total = N;
+  p.num_kb = Kd / 128;  // 128 e4m3 per 128-byte swizzle row
+  p.n_tiles_dense = ((M + 255) / 256) * (N / 256);
+  p.bias = bias;
+  p.ldo = N;
+  p.err = err;
+  p.sx = sx;
+  p.sw = sw;
+  return launch_pair<256, G_FP8>(xq, wq, out_map, p, p.n_tiles_dense, st);
 }
 
 int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUtensorMap& hbuf_out,

@@ -429,29 +429,35 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
 // ------------------------------------------------------- gate + route
 // The layer path's gate and route builder in one kernel (bf16 build).  A
 // block takes the next chunk of GR_TOK tokens (a ticket, so chunks start in
-// order), runs the gate for one token per warp, ranks the chunk's 2*GR_TOK
-// routes per expert (stable: ascending route id r = 2t + k), publishes the
-// chunk's counts (flag 1) and sums the published counts of every earlier
-// chunk (one thread per earlier chunk, in parallel; an earlier chunk's block
-// took its ticket first, so it is running and will publish).  Expert e's rows start at e * cap (cap = T
-// rounded up to 256 >= any expert's route count), so a route's row
-// e * cap + (routes of e before it) needs no global totals: each warp writes
-// pos[r] and stores its token's LayerNorm2 row (bf16) straight into both of
-// its rows of xperm.  The last chunk also writes the expert tile list and
-// the offsets.  Waits on predecessors are bounded (PTL_ERR_TIMEOUT).
+// order); each warp runs the gate for GR_TPW consecutive tokens at once (the
+// x1 rows of all of them in flight together; each gate-weight load, read
+// through L1, serves all of them): LayerNorm2 in fp32, the 8 logits in fp32,
+// the top-2 logits (ties to the lower index) and the renormalised weights.
+// The chunk's 2*GR_TOK routes are then ranked per expert (stable: ascending
+// route id r = 2t + k), the chunk publishes its counts (flag 1) and sums the
+// published counts of every earlier chunk (one thread per earlier chunk, in
+// parallel; an earlier chunk's block took its ticket first, so it is running
+// or done and will publish).  Expert e's rows start at e * cap (cap = T
+// rounded up to 256 >= any expert's route count), so a route's row e * cap +
+// (routes of e before it) needs no global totals: each warp writes pos[r]
+// and stores each token's LayerNorm2 row (bf16) straight into both of its
+// rows of xperm.  The last chunk also writes the expert tile list and the
+// offsets.  Waits on predecessors are bounded (PTL_ERR_TIMEOUT).
 // lb: [0] ticket, then per chunk 32 ints: [0] flag, [4..11] counts; all
 // zero before the kernel.
-__global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
+constexpr int GR_ROUTES = 2 * GR_TOK;
+constexpr int GR_GROUPS = GR_ROUTES / 32;  // 32-route groups ranked by one warp each
+static_assert(GR_ROUTES % 32 == 0 && GR_GROUPS <= GR_WARPS, "route groups");
+
+__global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
     const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
     const float* __restrict__ wg, const float* __restrict__ bg, int32_t* __restrict__ idx,
     float* __restrict__ wout, int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ xperm, int cap,
     int32_t* __restrict__ lb, int2* __restrict__ tiles, int32_t* __restrict__ meta,
     int32_t* __restrict__ moe_done, int T_, int32_t* err) {
-  __shared__ __align__(16) float s_wg[E * D];
-  __shared__ int s_chunk, s_e[2 * GR_TOK], s_rank[2 * GR_TOK], s_cnt[E], s_excl[E], s_tot[E];
-  __shared__ int s_red[GR_TOK][E];
-  stage_gate_weights(s_wg, wg);
-  __syncthreads();
+  __shared__ int s_chunk, s_e[GR_ROUTES], s_rank[GR_ROUTES], s_gcnt[GR_GROUPS][E];
+  __shared__ int s_cnt[E], s_excl[E], s_tot[E];
+  __shared__ int s_red[GR_WARPS][E];
   pdl_wait();  // x1 comes from the previous kernel
   pdl_trigger();  // dependents launch once this grid has passed its own wait
   if (has_error(err)) return;
@@ -461,45 +467,109 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
   __syncthreads();
   const int c = s_chunk;
   const int nchunks = (T_ + GR_TOK - 1) / GR_TOK;
-  const int t = c * GR_TOK + warp;
-  const bool valid = t < T_;
-  uint32_t vp[8];  // the token's LN2 values, packed bf16 pairs (fp32 lane layout)
-  int e0 = E, e1 = E;
-  if (valid) {
-    float v[16], w0, w1;
-    gate_token(x1 + size_t(t) * D, g, b, s_wg, bg, lane, v, e0, e1, w0, w1);
+  const int t0 = c * GR_TOK + warp * GR_TPW;  // this warp's first token
+  // the x1 rows of the warp's tokens (fp32 lane layout: 4 groups of 4
+  // consecutive columns at q*128 + lane*4), all loads issued together
+  float v[GR_TPW][16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) vp[i] = sm_pack_bf16x2(v[2 * i], v[2 * i + 1]);
-    if (lane == 0) {
+  for (int j = 0; j < GR_TPW; ++j) {
+    const int t = t0 + j;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 f = t < T_ ? __ldg(reinterpret_cast<const float4*>(x1 + size_t(t) * D + q * 128 + lane * 4))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[j][4 * q] = f.x;
+      v[j][4 * q + 1] = f.y;
+      v[j][4 * q + 2] = f.z;
+      v[j][4 * q + 3] = f.w;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < GR_TPW; ++j) layer_norm16<float>(v[j], g, b, lane);
+  // the 8 logits of every token: each weight load serves the warp's tokens
+  float acc[GR_TPW][E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    float4 w4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w4[q] = __ldg(reinterpret_cast<const float4*>(wg + e * D + q * 128 + lane * 4));
+#pragma unroll
+    for (int j = 0; j < GR_TPW; ++j) {
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        s += v[j][4 * q] * w4[q].x + v[j][4 * q + 1] * w4[q].y + v[j][4 * q + 2] * w4[q].z +
+             v[j][4 * q + 3] * w4[q].w;
+      acc[j][e] = s;
+    }
+  }
+  const float bias_mine = bg ? __ldg(bg + (lane >> 2)) : 0.f;
+  int e0s[GR_TPW], e1s[GR_TPW];
+#pragma unroll
+  for (int j = 0; j < GR_TPW; ++j) {
+    const int t = t0 + j;
+    const float mine = warp_reduce_scatter8(acc[j], lane) + bias_mine;
+    float lg[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) lg[e] = __shfl_sync(0xffffffffu, mine, 4 * e);
+    // softmax is monotonic: the top-2 of p are the top-2 logits (ties to the
+    // lower index); w0 = 1 / (1 + t), w1 = t / (1 + t), t = exp(l1 - l0)
+    int e0 = 0;
+    float l0 = lg[0];
+#pragma unroll
+    for (int e = 1; e < E; ++e)
+      if (lg[e] > l0) {
+        l0 = lg[e];
+        e0 = e;
+      }
+    int e1 = -1;
+    float l1 = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      if (e != e0 && (e1 < 0 || lg[e] > l1)) {
+        l1 = lg[e];
+        e1 = e;
+      }
+    const float tt = expf(l1 - l0);
+    const float w0 = 1.0f / (1.0f + tt);
+    const float w1 = tt * w0;
+    const bool valid = t < T_;
+    e0s[j] = valid ? e0 : E;
+    e1s[j] = valid ? e1 : E;
+    if (valid && lane == 0) {
       *reinterpret_cast<int2*>(idx + 2 * t) = make_int2(e0, e1);
       *reinterpret_cast<float2*>(wout + 2 * t) = make_float2(w0, w1);
     }
   }
   if (lane == 0) {
-    s_e[2 * warp] = e0;
-    s_e[2 * warp + 1] = e1;
+#pragma unroll
+    for (int j = 0; j < GR_TPW; ++j) {
+      s_e[2 * (warp * GR_TPW + j)] = e0s[j];
+      s_e[2 * (warp * GR_TPW + j) + 1] = e1s[j];
+    }
   }
   __syncthreads();
-  // chunk-local stable ranks and counts (the chunk's 2 * GR_TOK = 32 routes
-  // are one warp's lanes)
-  static_assert(2 * GR_TOK == 32, "one lane per route of the chunk");
-  if (warp == 0) {
-    const int e = s_e[lane];
+  // stable ranks inside each 32-route group and the groups' counts
+  if (warp < GR_GROUPS) {
+    const int q = 32 * warp + lane;
+    const int e = s_e[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
-    s_rank[lane] = __popc(same & ((1u << lane) - 1u));
+    s_rank[q] = __popc(same & ((1u << lane) - 1u));
 #pragma unroll
     for (int x = 0; x < E; ++x) {
       const unsigned bal = __ballot_sync(0xffffffffu, e == x);
-      if (lane == x) s_cnt[x] = __popc(bal);
+      if (lane == x) s_gcnt[warp][x] = __popc(bal);
     }
   }
   __syncthreads();
   // publish this chunk's counts, then sum the counts of every earlier chunk
-  // (one thread per earlier chunk, all read in parallel: no chain of
-  // prefixes to wait for)
   int32_t* me = lb + 32 + 32 * c;
   if (threadIdx.x < E) {
-    me[4 + threadIdx.x] = s_cnt[threadIdx.x];
+    int n = 0;
+#pragma unroll
+    for (int gq = 0; gq < GR_GROUPS; ++gq) n += s_gcnt[gq][threadIdx.x];
+    s_cnt[threadIdx.x] = n;
+    me[4 + threadIdx.x] = n;
     __threadfence();
   }
   __syncthreads();
@@ -535,22 +605,31 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
     const int e = threadIdx.x;
     int excl = 0;
 #pragma unroll
-    for (int w = 0; w < GR_TOK; ++w) excl += s_red[w][e];
+    for (int w = 0; w < GR_WARPS; ++w) excl += s_red[w][e];
     s_excl[e] = excl;
     s_tot[e] = excl + s_cnt[e];
   }
   __syncthreads();
-  if (valid) {
-    // this token's two routes: rows e * cap + (routes of e before it)
+  // each token's two routes: rows e * cap + (routes of e before it); the
+  // LayerNorm2 row goes out in bf16 (the layout of store_row16_groups)
+#pragma unroll
+  for (int j = 0; j < GR_TPW; ++j) {
+    if (t0 + j >= T_) break;
+    uint32_t vp[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) vp[i] = sm_pack_bf16x2(v[j][2 * i], v[j][2 * i + 1]);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      const int e = k == 0 ? e0 : e1;
-      const int row = e * cap + s_excl[e] + s_rank[2 * warp + k];
-      if (lane == 0) pos[2 * t + k] = row;
+      const int e = k == 0 ? e0s[j] : e1s[j];
+      const int q = 2 * (warp * GR_TPW + j) + k;
+      int rank = s_excl[e] + s_rank[q];
+      for (int gq = 0; gq < (q >> 5); ++gq) rank += s_gcnt[gq][e];
+      const int row = e * cap + rank;
+      if (lane == 0) pos[2 * (t0 + j) + k] = row;
       __nv_bfloat16* dst = xperm + size_t(row) * D;
 #pragma unroll
-      for (int q = 0; q < 4; ++q)  // the layout of store_row16_groups
-        *reinterpret_cast<uint2*>(dst + q * 128 + lane * 4) = make_uint2(vp[2 * q], vp[2 * q + 1]);
+      for (int qq = 0; qq < 4; ++qq)
+        *reinterpret_cast<uint2*>(dst + qq * 128 + lane * 4) = make_uint2(vp[2 * qq], vp[2 * qq + 1]);
     }
   }
   if (c == nchunks - 1) {
@@ -560,7 +639,9 @@ __global__ void __launch_bounds__(GR_TOK * 32, 3) gate_route_kernel(
       const int nt = (s_tot[e] + MOE_BM - 1) / MOE_BM;
       for (int j = threadIdx.x; j < nt; j += blockDim.x) {
         tiles[nt_before + j] = make_int2(e, e * cap + j * MOE_BM);
-        moe_done[nt_before + j] = 0;  // the fused expert GEMMs' per-tile counters
+#pragma unroll
+        for (int q = 0; q < MOE1_NT; ++q)  // the fused expert GEMMs' completion counters
+          moe_done[(nt_before + j) * MOE1_NT + q] = 0;
       }
       nt_before += nt;
     }
@@ -1178,6 +1259,55 @@ __global__ void __launch_bounds__(REP_WARPS * 32)
   if (bad && lane == 0) set_error(err, PTL_ERR_BAD_IDS);
 }
 
+// --------------------------------------------------- FP8 (e4m3) operands
+// Per-row e4m3 quantisation (one scale per row: s = max|row| / 448, 1 for an
+// all-zero row; codes = the row divided by s, rounded to the nearest e4m3
+// value, ties to even, saturating at +-448).  The scale and the quotient are
+// IEEE float32 operations (correctly rounded division), so the codes are
+// decided exactly as by a float32 restatement of the definition.  One warp
+// per row, 16-byte accesses; cols is a multiple of 16.
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const T* __restrict__ x, int64_t rows, int cols,
+                                                              uint8_t* __restrict__ codes,
+                                                              float* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  constexpr int VEC = 16 / sizeof(T);  // elements per 16-byte load
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+       r += int64_t(gridDim.x) * (blockDim.x >> 5)) {
+    const T* row = x + r * cols;
+    float amax = 0.f;
+    for (int c = lane * VEC; c < cols; c += 32 * VEC) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + c));
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) amax = fmaxf(amax, fabsf(to_f32<T>(e[i])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    if (lane == 0) scales[r] = s;
+    uint8_t* crow = codes + r * cols;
+    for (int c = lane * 16; c < cols; c += 32 * 16) {
+      float v[16];
+#pragma unroll
+      for (int h = 0; h < 16; h += VEC) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + c + h));
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) v[h + i] = to_f32<T>(e[i]);
+      }
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        w[q] = uint32_t(sm100::cvt_e4m3x2(__fdiv_rn(v[4 * q], s), __fdiv_rn(v[4 * q + 1], s))) |
+               (uint32_t(sm100::cvt_e4m3x2(__fdiv_rn(v[4 * q + 2], s), __fdiv_rn(v[4 * q + 3], s))) << 16);
+      *reinterpret_cast<uint4*>(crow + c) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 // ------------------------------------------------------------- launchers
 #define PTL_LAUNCH_CHECK() (cudaPeekAtLastError() == cudaSuccess ? 0 : -1)
 
@@ -1191,6 +1321,18 @@ int num_sms() {
     return v;
   });
   return n > 0 ? n : 148;
+}
+
+int launch_quant_rows_e4m3(const void* x, ptl_dtype dt, int64_t rows, int cols, uint8_t* codes, float* scales,
+                           cudaStream_t st) {
+  const int64_t want = (rows + 7) / 8;
+  const int blocks = int(want < 8 * num_sms() ? want : 8 * num_sms());
+  const int r = dt == PTL_BF16
+                    ? launch_k(quant_rows_e4m3_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                               static_cast<const __nv_bfloat16*>(x), rows, cols, codes, scales)
+                    : launch_k(quant_rows_e4m3_kernel<float>, dim3(blocks), dim3(256), 0, st,
+                               static_cast<const float*>(x), rows, cols, codes, scales);
+  return r != 0 ? -1 : PTL_LAUNCH_CHECK();
 }
 
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st,
@@ -1242,7 +1384,7 @@ int launch_gate(const void* x1, const float* g, const float* b, const float* wg,
 int launch_gate_route(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                       int T, const WsLayout& L, char* ws, cudaStream_t st) {
   const int blocks = (T + GR_TOK - 1) / GR_TOK;
-  if (launch_k(gate_route_kernel, dim3(blocks), dim3(GR_TOK * 32), 0, st, static_cast<const float*>(x1), g, b,
+  if (launch_k(gate_route_kernel, dim3(blocks), dim3(GR_WARPS * 32), 0, st, static_cast<const float*>(x1), g, b,
                wg, bg, reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<float*>(ws + L.wgt),
                reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<__nv_bfloat16*>(ws + L.xperm),
                int(L.cap), reinterpret_cast<int32_t*>(ws + L.lb), reinterpret_cast<int2*>(ws + L.tiles),

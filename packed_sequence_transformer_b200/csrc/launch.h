@@ -116,6 +116,10 @@ int launch_combine_f32(const float* y, const float* w, const float* x1, float* o
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
                     const char* ws, cudaStream_t st, const AttnMask* mask = nullptr);
 
+// Per-row e4m3 codes [rows][cols] and float32 scales [rows] of x (dt)
+int launch_quant_rows_e4m3(const void* x, ptl_dtype dt, int64_t rows, int cols, uint8_t* codes, float* scales,
+                           cudaStream_t st);
+
 // RepEncoder: embedding bags + LayerNorm(14336) into out [T][14336] (dt)
 int launch_embag_ln(const RepTables& tb, const int64_t* ids, const int64_t* off, int64_t n_ids, int T,
                     const float* g, const float* b, void* out, ptl_dtype dt, int32_t* err,
@@ -140,6 +144,11 @@ int launch_gemm_moe12(const CUtensorMap& xperm, const CUtensorMap& w1, const CUt
                       const WsLayout& L, char* ws, cudaStream_t st);
 int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUtensorMap& ybuf_out,
                      const float* b2, const WsLayout& L, char* ws, cudaStream_t st);
+
+// FP8: out [M][N] bf16 = (xq [M][K] wq [N][K]^T) * sx[m] * sw[n] + b[n], e4m3
+// codes with per-row scales, 256 x 256 pair tiles (K a multiple of 128, N of 256)
+int launch_gemm_fp8(const CUtensorMap& xq, const CUtensorMap& wq, const CUtensorMap& out_map, const float* sx,
+                    const float* sw, const float* bias, int M, int N, int Kd, int32_t* err, cudaStream_t st);
 
 // attn_tc.cu (bf16, tcgen05)
 // mask (nullable): the HSTU-style variant, over a work list built with the

@@ -135,6 +135,11 @@ _SIGS = {
     "ptl_attention_noalloc": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p],
                               ctypes.c_int),
+    "ptl_quantize_rows_e4m3": ([ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int32,
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p], ctypes.c_int),
+    "ptl_linear_fp8": ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                        ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                        ctypes.c_size_t, ctypes.c_void_p], ctypes.c_int),
     "ptl_partition_users": ([ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, ctypes.c_int32,
                              ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
 }
@@ -376,6 +381,26 @@ def attention_noalloc(qkv, attn, cu_seqlens, device_status=None, stream=None):
                                        _ptr(device_status), _stream(stream)),
            "ptl_attention_noalloc")
     return attn
+
+
+def quantize_rows_e4m3(x, codes=None, scales=None, stream=None):
+    """ptl_quantize_rows_e4m3: per-row e4m3 codes (uint8 tensor) and float32
+    scales of a 2-D bf16 / fp32 device tensor."""
+    rows, cols = x.shape
+    codes = codes if codes is not None else torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    scales = scales if scales is not None else torch.empty(rows, dtype=torch.float32, device=x.device)
+    _check(lib().ptl_quantize_rows_e4m3(_ptr(x), _dt(x.dtype), rows, cols, _ptr(codes), _ptr(scales),
+                                        _stream(stream)), "ptl_quantize_rows_e4m3")
+    return codes, scales
+
+
+def linear_fp8(xq, sx, wq, sw, bias, out, workspace, stream=None):
+    """ptl_linear_fp8: out (bf16 [M][N]) = (xq wq^T) * sx[m] * sw[n] + bias[n]."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    _check(lib().ptl_linear_fp8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias), _ptr(out), M, K, N,
+                                _ptr(workspace), workspace.numel(), _stream(stream)), "ptl_linear_fp8")
+    return out
 
 
 def partition_users(cu_seqlens, num_parts: int):

@@ -23,7 +23,7 @@ def P():
 def _declared():
     txt = open(os.path.join(ROOT, "include", "ptl.h")).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(ptl_[a-z_]+)\s*\(", txt)))
+    return sorted(set(re.findall(r"\b(ptl_[a-z0-9_]+)\s*\(", txt)))
 
 
 def test_exports_every_declared_symbol(P):

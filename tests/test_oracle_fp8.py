@@ -77,3 +77,32 @@ def test_fp8_linear_within_its_error_bound(K):
     assert np.all(np.abs(y8 - y) <= bound)
     # and it is a real approximation: far closer than the operands' size
     assert np.max(np.abs(y8 - y)) < 0.1 * np.max(np.abs(y - b))
+
+
+def test_float32_decided_codes():
+    """precision='f32': the scale is the float32 quotient max|row| / 448 and
+    each code is the e4m3 rounding of the float32 quotient x / s; it differs
+    from the float64-decided code only where the float64 quotient lies within
+    one float32 rounding of a point halfway between two e4m3 neighbours, and
+    then by exactly one e4m3 step."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((64, 512)) * 2.0 ** rng.integers(-8, 8, (64, 1))).astype(np.float32)
+    x[7] = 0.0
+    c32, s32 = O.quantize_rows_e4m3(x, precision="f32")
+    c64, s64 = O.quantize_rows_e4m3(x.astype(np.float64))
+    amax = np.abs(x).max(axis=1).astype(np.float32)
+    want_s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0))
+    np.testing.assert_array_equal(s32, want_s.astype(np.float64))
+    assert s32[7] == 1.0 and not c32[7].any()
+    np.testing.assert_allclose(s32, s64, rtol=2.0 ** -23, atol=0)
+    q32 = (x / want_s[:, None].astype(np.float32)).astype(np.float64)
+    np.testing.assert_array_equal(c32, O.quantize_e4m3(q32))
+    diff = c32 != c64
+    assert diff.mean() < 1e-3
+    # where they differ, the float64 quotient sits next to a rounding boundary
+    q64 = x.astype(np.float64) / s64[:, None]
+    a = np.abs(q64[diff])
+    step = np.where(a >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(a, 2.0 ** -6))) - 3), 2.0 ** -9)
+    frac = a / step - np.floor(a / step)
+    assert np.all(np.abs(frac - 0.5) <= 2.0 ** -20 * a / step + 1e-9)
+    assert np.all(np.abs(np.abs(c32[diff]) - np.abs(c64[diff])) <= step * (1 + 1e-12))
