@@ -48,9 +48,12 @@ RUNNER_STRIDE = 128  # token granule of the graph runner's buckets in the end-to
 # kernel changed since its capture is dropped from this table until it is
 # captured again.
 NCU_DRAM_BYTES = {
-    "gemm_qkv": 8.589312e6,
-    "gemm_out": 14.527488e6,
-    "combine": 28.068096e6 + 0.002048e6,
+    "gemm_qkv": 8.588032e6,
+    "gemm_out": 14.522880e6,
+    "gemm_expert1": 31.805184e6 + 6.673408e6,
+    "attention": 21.015296e6,
+    "gate": 14.058496e6,
+    "combine": 28.068352e6 + 0.00128e6,
 }
 
 
