@@ -444,6 +444,12 @@ ptl_status ptl_layer_forward(const void* x, void* out, const int32_t* cu_seqlens
   if ((s = begin(c)) != PTL_OK) return s;
   EndMark end_mark{c.st};
   mark(c.st, PTL_KERNEL_WORKLIST);
+  if (c.dt == PTL_BF16) {
+    // the work list and LayerNorm1 of x in one launch
+    PTL_TRY(launch_prologue(cu_seqlens, num_users, c.T, c.L, c.ws, x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn,
+                            c.st));
+    return layer_body(c, x, out, cu_seqlens, w, dbg, true);
+  }
   PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
   return layer_body(c, x, out, cu_seqlens, w, dbg);
 }
@@ -473,14 +479,21 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
   if ((s = begin(c)) != PTL_OK) return s;
   EndMark end_mark{c.st};
   mark(c.st, PTL_KERNEL_WORKLIST);
-  PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
+  const bool fuse = c.dt == PTL_BF16;
+  if (fuse) {
+    // the work list and layer 0's LayerNorm1 of x in one launch
+    PTL_TRY(launch_prologue(cu_seqlens, num_users, c.T, c.L, c.ws, x, F32(layers[0].ln1_g), F32(layers[0].ln1_b),
+                            c.ws + c.L.xn, c.st));
+  } else {
+    PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
+  }
   const void* h_in = x;
   for (int i = 0; i < num_layers; ++i) {
     void* h_out = (i == num_layers - 1) ? out : c.ws + ((i & 1) ? c.L.act1 : c.L.act0);
-    // bf16: layer i's combine also writes LayerNorm1 of its output for layer i + 1
-    const bool fuse = c.dt == PTL_BF16;
+    // bf16: layer i's combine also writes LayerNorm1 of its output for layer
+    // i + 1 (layer 0's comes from the prologue)
     const ptl_layer_weights* next = (fuse && i + 1 < num_layers) ? &layers[i + 1] : nullptr;
-    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr, fuse && i > 0, next)) != PTL_OK)
+    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr, fuse, next)) != PTL_OK)
       return s;
     h_in = h_out;
   }

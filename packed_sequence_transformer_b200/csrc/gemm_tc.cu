@@ -194,6 +194,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
+  if (!is_moe(MODE) && warp == 0 && lane == 0 && pair < p.n_tiles_dense) {
+    // the weights of this pair's first tile do not come from the previous
+    // kernel (its activations do): start pulling them into L2 while that
+    // kernel finishes, they are the loads that may have to come from HBM
+    int expert, m0, n0, mt;
+    bool second;
+    decode_pair_tile<BN, MODE>(p, pair, 0, expert, m0, n0, second, mt);
+    constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;
+    for (int kb = 0; kb < p.num_kb; ++kb) tma_prefetch_2d(&tmB, kb * KSLICE, n0 + int(cr) * (BN / 2));
+  }
   pdl_wait();  // inputs, route tables and the error word come from earlier kernels
   pdl_trigger();  // dependents launch once this grid has passed its own wait
   __shared__ int s_nmt;

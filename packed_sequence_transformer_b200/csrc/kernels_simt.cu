@@ -143,15 +143,64 @@ __device__ void block_suffix_exclusive(int32_t* a, int n) {
   }
 }
 
-__global__ void __launch_bounds__(1024) worklist_kernel(const int32_t* __restrict__ cu, int U, int T,
-                                                        int2* __restrict__ items, int32_t* item_count,
-                                                        int32_t* lvl_hist, int32_t* lvl_start,
-                                                        int32_t* lvl_fill, int max_levels, int G,
-                                                        int4* __restrict__ ulist, int32_t* __restrict__ uoff,
-                                                        int32_t* __restrict__ ucnt, int32_t* err,
-                                                        const AttnMask mask, const int masked) {
+// The work list's arguments (one struct, passed by value).
+struct WorklistArgs {
+  const int32_t* cu;
+  int U, T;
+  int2* items;
+  int32_t *item_count, *lvl_hist, *lvl_start, *lvl_fill;
+  int max_levels, G;
+  int4* ulist;
+  int32_t *uoff, *ucnt, *err;
+  AttnMask mask;
+  int masked;
+};
+
+__device__ void worklist_body(const WorklistArgs& w);
+
+__global__ void __launch_bounds__(1024) worklist_kernel(const WorklistArgs w) {
   pdl_wait();
   pdl_trigger();
+  worklist_body(w);
+}
+
+// The once-per-call prologue of the bf16 layer and stack: block 0 builds the
+// attention work list (one block of 1024 threads, as worklist_kernel) while
+// the other blocks apply the first layer's LayerNorm1 to the input rows, one
+// warp per row (the arithmetic of ln_rows_kernel); the two are independent.
+__global__ void __launch_bounds__(1024) prologue_kernel(const WorklistArgs w, const __nv_bfloat16* __restrict__ x,
+                                                        const float* __restrict__ g, const float* __restrict__ b,
+                                                        __nv_bfloat16* __restrict__ y, int T) {
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0) {
+    worklist_body(w);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int row = (blockIdx.x - 1) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= T) return;
+  float v[16];
+  Row16<__nv_bfloat16>::load(x + size_t(row) * D, lane, v);
+  layer_norm16<__nv_bfloat16>(v, g, b, lane);
+  Row16<__nv_bfloat16>::store(y + size_t(row) * D, lane, v);
+}
+
+__device__ void worklist_body(const WorklistArgs& w) {
+  const int32_t* __restrict__ cu = w.cu;
+  const int U = w.U, T = w.T;
+  int2* __restrict__ items = w.items;
+  int32_t* item_count = w.item_count;
+  int32_t* lvl_hist = w.lvl_hist;
+  int32_t* lvl_start = w.lvl_start;
+  int32_t* lvl_fill = w.lvl_fill;
+  const int max_levels = w.max_levels, G = w.G;
+  int4* __restrict__ ulist = w.ulist;
+  int32_t* __restrict__ uoff = w.uoff;
+  int32_t* __restrict__ ucnt = w.ucnt;
+  int32_t* err = w.err;
+  const AttnMask& mask = w.mask;
+  const int masked = w.masked;
   __shared__ int s_bad;
   __shared__ int s_total;
   const int tid = threadIdx.x;
@@ -866,34 +915,46 @@ __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, cons
   }
 }
 
-// Keeps p[t] for the tokens with pred_mask[t] != 0, in ascending t.
+// Keeps p[t] for the tokens with pred_mask[t] != 0, in ascending t.  One
+// block of 1024 threads in one pass: thread i owns the contiguous run of
+// tokens [i * run, (i + 1) * run), counts its kept tokens, the block takes
+// the exclusive prefix of the counts (warp shuffles, then the 32 warp totals),
+// and each thread writes its run's kept values in order.
 __global__ void __launch_bounds__(1024) head_compact_kernel(const float* __restrict__ p,
                                                             const uint8_t* __restrict__ mask,
                                                             float* __restrict__ probs,
                                                             int32_t* __restrict__ n_pred, int T_) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int32_t s_scan[1024];
-  __shared__ int32_t s_carry;
-  if (threadIdx.x == 0) s_carry = 0;
-  __syncthreads();
-  for (int base = 0; base < T_; base += 1024) {
-    const int t = base + threadIdx.x;
-    const int f = (t < T_ && mask[t]) ? 1 : 0;
-    s_scan[threadIdx.x] = f;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-      const int v = threadIdx.x >= unsigned(o) ? s_scan[threadIdx.x - o] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += v;
-      __syncthreads();
-    }
-    if (f) probs[s_carry + s_scan[threadIdx.x] - 1] = p[t];
-    __syncthreads();
-    if (threadIdx.x == 1023) s_carry += s_scan[1023];
-    __syncthreads();
+  __shared__ int32_t s_warp[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int run = (T_ + 1023) / 1024;
+  const int t0 = min(tid * run, T_), t1 = min(t0 + run, T_);
+  int cnt = 0;
+  for (int t = t0; t < t1; ++t) cnt += mask[t] ? 1 : 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
-  if (threadIdx.x == 0 && n_pred) *n_pred = s_carry;
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int tot = s_warp[lane];
+    int winc = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, winc, o);
+      if (lane >= o) winc += v;
+    }
+    s_warp[lane] = winc - tot;  // exclusive prefix of the warp totals
+    if (lane == 31 && n_pred) *n_pred = winc;
+  }
+  __syncthreads();
+  int o = s_warp[warp] + incl - cnt;
+  for (int t = t0; t < t1; ++t)
+    if (mask[t]) probs[o++] = p[t];
 }
 
 // ------------------------------------------------- fp32 build: CUDA cores
@@ -1335,17 +1396,40 @@ int launch_quant_rows_e4m3(const void* x, ptl_dtype dt, int64_t rows, int cols, 
   return r != 0 ? -1 : PTL_LAUNCH_CHECK();
 }
 
+static WorklistArgs worklist_args(const int32_t* cu, int U, int T, const WsLayout& L, char* ws,
+                                  const AttnMask* mask) {
+  WorklistArgs w;
+  w.cu = cu;
+  w.U = U;
+  w.T = T;
+  w.items = reinterpret_cast<int2*>(ws + L.items);
+  w.item_count = reinterpret_cast<int32_t*>(ws + L.item_count);
+  w.lvl_hist = reinterpret_cast<int32_t*>(ws + L.lvl_hist);
+  w.lvl_start = reinterpret_cast<int32_t*>(ws + L.lvl_start);
+  w.lvl_fill = reinterpret_cast<int32_t*>(ws + L.lvl_fill);
+  w.max_levels = int(L.max_levels);
+  w.G = attn_grid(L.max_items, num_sms());
+  w.ulist = reinterpret_cast<int4*>(ws + L.ulist);
+  w.uoff = reinterpret_cast<int32_t*>(ws + L.uoff);
+  w.ucnt = reinterpret_cast<int32_t*>(ws + L.ucnt);
+  w.err = reinterpret_cast<int32_t*>(ws + L.err);
+  w.mask = mask ? *mask : AttnMask{nullptr, nullptr, 1, 1, 0};
+  w.masked = mask ? 1 : 0;
+  return w;
+}
+
 int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, cudaStream_t st,
                     const AttnMask* mask) {
-  const AttnMask m = mask ? *mask : AttnMask{nullptr, nullptr, 1, 1, 0};
-  if (launch_k(worklist_kernel, dim3(1), dim3(1024), 0, st, cu, U, T, reinterpret_cast<int2*>(ws + L.items),
-                                      reinterpret_cast<int32_t*>(ws + L.item_count),
-                                      reinterpret_cast<int32_t*>(ws + L.lvl_hist),
-                                      reinterpret_cast<int32_t*>(ws + L.lvl_start),
-                                      reinterpret_cast<int32_t*>(ws + L.lvl_fill), int(L.max_levels),
-                                      attn_grid(L.max_items, num_sms()), reinterpret_cast<int4*>(ws + L.ulist),
-                                      reinterpret_cast<int32_t*>(ws + L.uoff), reinterpret_cast<int32_t*>(ws + L.ucnt),
-                                      reinterpret_cast<int32_t*>(ws + L.err), m, mask ? 1 : 0)) return -1;
+  if (launch_k(worklist_kernel, dim3(1), dim3(1024), 0, st, worklist_args(cu, U, T, L, ws, mask))) return -1;
+  return PTL_LAUNCH_CHECK();
+}
+
+int launch_prologue(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, const void* x, const float* g,
+                    const float* b, void* y, cudaStream_t st) {
+  const int ln_blocks = (T + 31) / 32;  // 32 rows (warps) per block
+  if (launch_k(prologue_kernel, dim3(1 + ln_blocks), dim3(1024), 0, st, worklist_args(cu, U, T, L, ws, nullptr),
+               static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T))
+    return -1;
   return PTL_LAUNCH_CHECK();
 }
 

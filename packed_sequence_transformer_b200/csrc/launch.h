@@ -87,6 +87,10 @@ int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws
                     const AttnMask* mask = nullptr);
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st);
+// bf16 layer / stack: the work list (block 0) and the first layer's
+// LayerNorm1 of x into y (the other blocks) in one launch
+int launch_prologue(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, const void* x, const float* g,
+                    const float* b, void* y, cudaStream_t st);
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
                 cudaStream_t st);
