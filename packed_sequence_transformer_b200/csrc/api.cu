@@ -232,7 +232,11 @@ ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_wei
     if (!map_bf16(&mb, w->w_qkv, D, QKV_N, D * 2, 64, QKV_BN / 2)) return PTL_ERR_CUDA;
     if (!map_bf16(&mo, qkv, QKV_N, T, QKV_N * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_GEMM_QKV);
-    PTL_TRY(launch_gemm_qkv(ma, mb, mo, F32(w->b_qkv), qkv, T, c.err, c.st));
+    // the expert weights (16 MB, read once per layer) start coming into L2
+    // while the attention and the gate run, which leave HBM mostly idle
+    const size_t expert_w_bytes = size_t(E) * F * D * 2;
+    PTL_TRY(launch_gemm_qkv(ma, mb, mo, F32(w->b_qkv), qkv, T, c.err, c.st, w->w1, expert_w_bytes, w->w2,
+                            expert_w_bytes));
   } else {
     mark(c.st, PTL_KERNEL_LAYERNORM);
     PTL_TRY(launch_layernorm(x, F32(w->ln1_g), F32(w->ln1_b), c.ws + c.L.xn, T, c.dt, c.st));

@@ -334,9 +334,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const uint32_t v0 = smem_u32(sV + vs * ATT_TILE_BYTES);
         const uint32_t d = tmem + 256 + 64 * g;
         constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 64, 0, 1);
-        for (int k = 0; k < pvk16 / 16; ++k)  // keys 16k..16k+15: P columns 8k..8k+7
-          umma_bf16_ts(d, pt + 8 * k, umma_desc_sw128(v0 + k * 2048, 1024, 8192), idesc_pv,
-                       k != 0 || !pvfirst);
+        // the descriptors of the K slices differ only in the start-address
+        // field (address / 16, no carry inside shared memory)
+        const uint64_t dv = umma_desc_sw128(v0, 1024, 8192);
+        const int nk = pvk16 / 16;
+        for (int k = 0; k < nk; ++k)  // keys 16k..16k+15: P columns 8k..8k+7, V rows 2048 bytes on
+          umma_bf16_ts(d, pt + 8 * k, dv + uint64_t(k * (2048 >> 4)), idesc_pv, k != 0 || !pvfirst);
         umma_commit(&pv_done[g]);
         umma_commit(&v_empty[vs]);
         pvn = -1;
@@ -357,10 +360,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const uint32_t q0 = smem_u32(sQ + (2 * g + qs) * ATT_TILE_BYTES);
         const uint32_t k0 = smem_u32(sK + (g * ATT_KV_STAGES + st) * ATT_TILE_BYTES);
         const uint32_t idesc_qk = umma_idesc_bf16(128, k16);
+        const uint64_t dq = umma_desc_sw128(q0, 1024), dk = umma_desc_sw128(k0, 1024);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16_ss(tmem + 128 * g, umma_desc_sw128(q0 + 32 * k, 1024), umma_desc_sw128(k0 + 32 * k, 1024),
-                       idesc_qk, k != 0);
+        for (int k = 0; k < 4; ++k)  // K slices 32 bytes apart: +2 in the address field
+          umma_bf16_ss(tmem + 128 * g, dq + uint64_t(2 * k), dk + uint64_t(2 * k), idesc_qk, k != 0);
         umma_commit(&s_full[g]);
         umma_commit(&k_empty[g * ATT_KV_STAGES + st]);
         if (kb == a.hi) umma_commit(&q_empty[2 * g + qs]);
@@ -588,6 +591,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     if (!ok) set_error(err, PTL_ERR_TIMEOUT);
   }
+  __syncwarp();  // the single-lane roles rejoin their warps before the block barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -20,7 +20,7 @@ constexpr int QKV_N = 3 * D;       // 1536
 constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
 constexpr int MOE_BM = 256;        // rows per expert tile (padding granule; one CTA pair's M)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
-constexpr int GR_WARPS = 16;       // warps per block of the fused gate + route kernel
+constexpr int GR_WARPS = 12;       // warps per block of the fused gate + route kernel
 constexpr int GR_TPW = 4;          // tokens per warp of that kernel
 constexpr int GR_TOK = GR_WARPS * GR_TPW;  // tokens per block (one chunk of routes)
 constexpr int ATT_MAX_CTAS = 1024;  // bound on the persistent attention grid

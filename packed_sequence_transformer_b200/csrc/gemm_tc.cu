@@ -62,6 +62,7 @@ struct GemmTcParams {
   int ldo;                       // output row stride (elements)
   const int2* tiles;             // (expert, first padded row) per 256-row M tile
   const int32_t* meta;           // [0] = number of M tiles
+  int max_mt;                    // capacity of `tiles` (entries)
   int32_t* zero_ptr;             // cleared by the grid once the predecessor is done (may be NULL)
   int zero_n;
   // MOE12 (both expert GEMMs in one launch): the second GEMM's width, bias
@@ -73,6 +74,10 @@ struct GemmTcParams {
   // FP8: per-row scales of A (rows of the output) and of B (its columns)
   const float* sx;
   const float* sw;
+  // weights of later kernels to bring into L2 while this one waits for its
+  // inputs (16-byte aligned, sizes multiples of 16; may be NULL)
+  const void* pf_ptr[2];
+  size_t pf_bytes[2];
 };
 
 enum { G_QKV = 0, G_OUT = 1, G_MOE1 = 2, G_MOE2 = 3, G_MOE12 = 4, G_FP8 = 5 };
@@ -114,7 +119,8 @@ struct PairCfg {
 // `mt` is the tile's M tile.
 template <int BN, int MODE>
 __device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile, int n_mt, int& expert,
-                                                 int& m0, int& n0, bool& second, int& mt) {
+                                                 int& m0, int& n0, bool& second, int& mt,
+                                                 const int2* tl_known = nullptr, int known_mt = -1) {
   second = false;
   int nN = p.N_total / BN;
   if (MODE == G_MOE12 && tile >= n_mt * nN) {
@@ -125,7 +131,7 @@ __device__ __forceinline__ void decode_pair_tile(const GemmTcParams& p, int tile
   mt = tile / nN;
   n0 = (tile - mt * nN) * BN;
   if (is_moe(MODE)) {
-    const int2 tl = p.tiles[mt];
+    const int2 tl = (tl_known && mt == known_mt) ? *tl_known : p.tiles[mt];
     expert = tl.x;
     m0 = tl.y;
   } else {
@@ -201,11 +207,46 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int expert, m0, n0, mt;
     bool second;
     decode_pair_tile<BN, MODE>(p, pair, 0, expert, m0, n0, second, mt);
-    constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;
-    for (int kb = 0; kb < p.num_kb; ++kb) tma_prefetch_2d(&tmB, kb * KSLICE, n0 + int(cr) * (BN / 2));
+    for (int kb = 0; kb < p.num_kb; ++kb) tma_prefetch_2d(&tmB, kb * (MODE == G_FP8 ? 128 : 64), n0 + int(cr) * (BN / 2));
+  }
+  if (warp == 0 && lane == 0) {
+    // this CTA's share of the later kernels' weights
+    for (int k = 0; k < 2; ++k) {
+      if (!p.pf_ptr[k]) continue;
+      const size_t share = ((p.pf_bytes[k] + gridDim.x - 1) / gridDim.x + 15) & ~size_t(15);
+      const size_t off = size_t(blockIdx.x) * share;
+      if (off < p.pf_bytes[k]) {
+        const size_t n = p.pf_bytes[k] - off < share ? p.pf_bytes[k] - off : share;
+        prefetch_l2_bulk(static_cast<const char*>(p.pf_ptr[k]) + off, uint32_t(n));
+      }
+    }
   }
   pdl_wait();  // inputs, route tables and the error word come from earlier kernels
   pdl_trigger();  // dependents launch once this grid has passed its own wait
+  constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;  // a K slice: one 128-byte swizzle row
+  // Dense modes: the first ring stages of the pair's first tile go out now,
+  // before the error word is read and the block synchronises (their operands
+  // are the caller's buffers, of sizes the host checked), so that the load
+  // latency overlaps that read.
+  int pre = 0;
+  if (!is_moe(MODE) && warp == 0 && lane == 0 && pair < p.n_tiles_dense) {
+    int expert, m0, n0, mt;
+    bool second;
+    decode_pair_tile<BN, MODE>(p, pair, 0, expert, m0, n0, second, mt);
+    pre = p.num_kb < STAGES ? p.num_kb : STAGES;
+    const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+    constexpr uint32_t tx = 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES);
+    for (int kb = 0; kb < pre; ++kb) {
+      if (cr == 0) mbar_arrive_expect_tx(&full[kb], tx);
+      tma_load_2d_pair(sA + kb * Cfg::A_BYTES, &tmA, full0 + uint32_t(kb) * 8u, kb * KSLICE, m0 + 128 * int(cr));
+      tma_load_2d_pair(sB + kb * Cfg::B_BYTES, &tmB, full0 + uint32_t(kb) * 8u, kb * KSLICE, n0 + int(cr) * (BN / 2));
+    }
+  }
+  // Expert modes: the pair's first tile entry is read together with the tile
+  // count (it is used only if the tile exists)
+  int2 first_tl = make_int2(0, 0);
+  const int first_mt = pair / (p.N_total / BN);
+  if (is_moe(MODE) && warp == 0 && lane == 0 && first_mt < p.max_mt) first_tl = p.tiles[first_mt];
   __shared__ int s_nmt;
   if (threadIdx.x == 0) {
     const int nmt = is_moe(MODE) ? p.meta[0] : 0;
@@ -226,19 +267,21 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (lane == 0) {
       // both CTAs: own halves of A and B, counted on CTA 0's full[s]
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);
-      int it = 0;
+      int it = pre;
       bool ok = true;
       constexpr uint32_t tx = 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES);
       for (int tile = pair; tile < ntiles && ok; tile += npairs) {
         int expert, m0, n0, mt;
         bool second;
-        decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt);
+        // the tile list is by M tile, the same entry for both expert GEMMs
+        decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt,
+                                   tile == pair && first_mt < p.max_mt ? &first_tl : nullptr, first_mt);
         const int arow = m0 + 128 * int(cr);
         const int brow = expert * (second ? p.N2 : p.N_total) + n0 + int(cr) * (BN / 2);
         const int nkb = second ? p.N_total / 64 : p.num_kb;
         const CUtensorMap* ma = second ? &tmA2 : &tmA;
         const CUtensorMap* mb = second ? &tmB2 : &tmB;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
+        for (int kb = tile == pair ? pre : 0; kb < nkb; ++kb, ++it) {
           if (MODE == G_MOE12 && second && kb % (BN / 64) == 0) {
             // this K slice of the tile's A rows (H) is one first-GEMM column
             // tile of this M tile, stored by both CTAs of its pair: start on
@@ -258,11 +301,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
           if (cr == 0) mbar_arrive_expect_tx(&full[s], tx);
           const uint32_t fb = full0 + uint32_t(s) * 8u;
-          // a K slice is one 128-byte swizzle row: 64 bf16 or 128 e4m3 elements
-          constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;
           tma_load_2d_pair(sA + s * Cfg::A_BYTES, ma, fb, kb * KSLICE, arow);
           tma_load_2d_pair(sB + s * Cfg::B_BYTES, mb, fb, kb * KSLICE, brow);
         }
+      }
+      if (ntiles == 0 && cr == 0) {
+        // an earlier kernel reported an error after the first stages went
+        // out: let them land (both CTAs' bytes count here) before the exit
+        for (int s = 0; s < pre; ++s)
+          if (!mbar_wait(&full[s], 0)) break;
       }
     }
   } else if (warp == 1) {
@@ -292,15 +339,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * Cfg::A_BYTES);
           const uint32_t b0 = smem_u32(sB + s * Cfg::B_BYTES);
-          // four MMAs per 128-byte K slice: K = 16 bf16 or 32 e4m3 each
+          // four MMAs per 128-byte K slice: K = 16 bf16 or 32 e4m3 each; the
+          // slices' descriptors differ by 32 bytes (+2) in the address field
+          const uint64_t da = umma_desc_sw128(a0, 1024), db = umma_desc_sw128(b0, 1024);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             if constexpr (MODE == G_FP8)
-              umma_e4m3_ss_pair(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
-                                (kb | k) != 0);
+              umma_e4m3_ss_pair(d, da + uint64_t(2 * k), db + uint64_t(2 * k), idesc, (kb | k) != 0);
             else
-              umma_bf16_ss_pair(d, umma_desc_sw128(a0 + 32 * k, 1024), umma_desc_sw128(b0 + 32 * k, 1024), idesc,
-                                (kb | k) != 0);
+              umma_bf16_ss_pair(d, da + uint64_t(2 * k), db + uint64_t(2 * k), idesc, (kb | k) != 0);
           }
           umma_commit_pair(&empty[s], 0x3);
         }
@@ -527,6 +574,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     if (MODE == G_OUT && warp == 2 && lane == 0) tma_store_wait_all();
   }
+  __syncwarp();  // the single-lane roles rejoin their warps before the cluster barrier
   tc_fence_before();
   cluster_sync();  // no MMA, TMEM read or remote arrival of either CTA is outstanding
   if (warp == 1) {
@@ -582,8 +630,13 @@ static int launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
 }
 
 int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorMap& qkv_out,
-                    const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st) {
+                    const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st, const void* pf0,
+                    size_t pf0_bytes, const void* pf1, size_t pf1_bytes) {
   GemmTcParams p{};
+  p.pf_ptr[0] = pf0;
+  p.pf_bytes[0] = pf0_bytes;
+  p.pf_ptr[1] = pf1;
+  p.pf_bytes[1] = pf1_bytes;
   p.M = T;
   p.N_total = QKV_N;
   p.num_kb = D / 64;
@@ -648,6 +701,7 @@ int launch_gemm_moe1(const CUtensorMap& xperm, const CUtensorMap& w1, const CUte
   p.ldo = F;
   p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
+  p.max_mt = int(L.max_tiles);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
   // the routing state of this layer (per-chunk expert counts, look-back
   // state, contiguous in the workspace) is consumed: clear it for the next
@@ -669,6 +723,7 @@ int launch_gemm_moe12(const CUtensorMap& xperm, const CUtensorMap& w1, const CUt
   p.bias2 = b2;
   p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
+  p.max_mt = int(L.max_tiles);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
   p.done = reinterpret_cast<int32_t*>(ws + L.moe_done);
   // the routing state of this layer is consumed: clear it for the next layer
@@ -688,6 +743,7 @@ int launch_gemm_moe2(const CUtensorMap& hbuf, const CUtensorMap& w2, const CUten
   p.ldo = D;
   p.tiles = reinterpret_cast<const int2*>(ws + L.tiles);
   p.meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
+  p.max_mt = int(L.max_tiles);
   p.err = reinterpret_cast<int32_t*>(ws + L.err);
   return launch_pair<GEMM2_BN, G_MOE2>(hbuf, w2, ybuf_out, p, int(L.max_tiles) * (D / GEMM2_BN), st);
 }

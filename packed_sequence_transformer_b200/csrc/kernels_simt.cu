@@ -71,7 +71,8 @@ struct Row16<float> {
 
 // LayerNorm of the lane's 16 values of a 512-element row (two passes over
 // registers: mean, then biased variance of the centred values).
-template <typename T>
+// SMEM: g and b point to shared memory (plain loads) instead of global memory.
+template <typename T, bool SMEM = false>
 __device__ __forceinline__ void layer_norm16(float (&v)[16], const float* __restrict__ g,
                                              const float* __restrict__ b, int lane) {
   float s = 0.f;
@@ -89,8 +90,8 @@ __device__ __forceinline__ void layer_norm16(float (&v)[16], const float* __rest
 #pragma unroll
   for (int qd = 0; qd < 4; ++qd) {
     const int c = Row16<T>::elem(lane, 4 * qd);
-    const float4 g4 = __ldg(reinterpret_cast<const float4*>(g + c));
-    const float4 b4 = __ldg(reinterpret_cast<const float4*>(b + c));
+    const float4 g4 = SMEM ? *reinterpret_cast<const float4*>(g + c) : __ldg(reinterpret_cast<const float4*>(g + c));
+    const float4 b4 = SMEM ? *reinterpret_cast<const float4*>(b + c) : __ldg(reinterpret_cast<const float4*>(b + c));
     v[4 * qd + 0] = v[4 * qd + 0] * rstd * g4.x + b4.x;
     v[4 * qd + 1] = v[4 * qd + 1] * rstd * g4.y + b4.y;
     v[4 * qd + 2] = v[4 * qd + 2] * rstd * g4.z + b4.z;
@@ -186,14 +187,20 @@ __global__ void __launch_bounds__(1024) prologue_kernel(const WorklistArgs w, co
   Row16<__nv_bfloat16>::store(y + size_t(row) * D, lane, v);
 }
 
+// Shared-memory capacities of the work-list build: up to these sizes the
+// offsets, the level counters and the items stay on chip (every count, scan
+// and deal step is then a shared-memory access); larger inputs use the
+// workspace arrays, with the same arithmetic.
+constexpr int WL_SMEM_USERS = 2048;
+constexpr int WL_SMEM_LEVELS = 1024;
+constexpr int WL_SMEM_ITEMS = 2048;
+
+
 __device__ void worklist_body(const WorklistArgs& w) {
-  const int32_t* __restrict__ cu = w.cu;
+  const int32_t* __restrict__ cu_g = w.cu;
   const int U = w.U, T = w.T;
   int2* __restrict__ items = w.items;
   int32_t* item_count = w.item_count;
-  int32_t* lvl_hist = w.lvl_hist;
-  int32_t* lvl_start = w.lvl_start;
-  int32_t* lvl_fill = w.lvl_fill;
   const int max_levels = w.max_levels, G = w.G;
   int4* __restrict__ ulist = w.ulist;
   int32_t* __restrict__ uoff = w.uoff;
@@ -203,14 +210,24 @@ __device__ void worklist_body(const WorklistArgs& w) {
   const int masked = w.masked;
   __shared__ int s_bad;
   __shared__ int s_total;
+  __shared__ int32_t s_cu[WL_SMEM_USERS + 1];
+  __shared__ int32_t s_lstart[WL_SMEM_LEVELS], s_lfill[WL_SMEM_LEVELS];
+  __shared__ int2 s_items[WL_SMEM_ITEMS];
   const int tid = threadIdx.x;
+  const bool cu_s = U <= WL_SMEM_USERS, lv_s = max_levels + 1 <= WL_SMEM_LEVELS;
+  // generic pointers: shared memory when the sizes fit, else the workspace
+  const int32_t* cu = cu_s ? s_cu : cu_g;
+  int32_t* lstart = lv_s ? s_lstart : w.lvl_start;
+  int32_t* lfill = lv_s ? s_lfill : w.lvl_fill;
   if (tid == 0) {
-    s_bad = (cu[0] != 0 || cu[U] != T) ? 1 : 0;
+    s_bad = (cu_g[0] != 0 || cu_g[U] != T) ? 1 : 0;
     s_total = 0;
   }
+  if (cu_s)
+    for (int i = tid; i <= U; i += blockDim.x) s_cu[i] = cu_g[i];
   for (int i = tid; i <= max_levels; i += blockDim.x) {
-    lvl_hist[i] = 0;
-    lvl_fill[i] = 0;
+    lstart[i] = 0;  // first the number of users with exactly i query blocks
+    lfill[i] = 0;
   }
   __syncthreads();
   for (int u = tid; u < U; u += blockDim.x)
@@ -235,22 +252,22 @@ __device__ void worklist_body(const WorklistArgs& w) {
   int local = 0;
   for (int u = tid; u < U; u += blockDim.x) {
     const int nb = (cu[u + 1] - cu[u] + ATT_BLK - 1) / ATT_BLK;
-    if (nb > 0) atomicAdd(&lvl_hist[nb], 1);
+    if (nb > 0) atomicAdd(&lstart[nb], 1);
     local += nb;
   }
   atomicAdd(&s_total, local);
   __syncthreads();
-  // lvl_start[b] <- #users with nb > b (pairs at level b) ...
-  for (int i = tid; i <= max_levels; i += blockDim.x) lvl_start[i] = lvl_hist[i];
-  __syncthreads();
-  block_suffix_exclusive(lvl_start, max_levels + 1);
+  // lstart[b] <- #users with nb > b (pairs at level b) ...
+  block_suffix_exclusive(lstart, max_levels + 1);
   // ... then the first slot of level b: sum over the deeper levels b' > b.
-  block_suffix_exclusive(lvl_start, max_levels + 1);
+  block_suffix_exclusive(lstart, max_levels + 1);
+  const bool it_s = s_total <= WL_SMEM_ITEMS;
   for (int u = tid; u < U; u += blockDim.x) {
     const int nb = (cu[u + 1] - cu[u] + ATT_BLK - 1) / ATT_BLK;
     for (int b = 0; b < nb; ++b) {
-      const int slot = lvl_start[b] + atomicAdd(&lvl_fill[b], 1);
+      const int slot = lstart[b] + atomicAdd(&lfill[b], 1);
       items[slot] = make_int2(u, b);
+      if (it_s) s_items[slot] = make_int2(u, b);
     }
   }
   if (tid == 0) *item_count = s_total;
@@ -271,7 +288,7 @@ __device__ void worklist_body(const WorklistArgs& w) {
       for (int k = 0;; ++k) {
         const int u = k * G + ((k & 1) ? G - 1 - c : c);
         if (u >= nunits) break;
-        const int2 it = items[u >> 3];
+        const int2 it = it_s ? s_items[u >> 3] : items[u >> 3];
         int steps = it.y + 1;
         if (masked) {
           const int Lu = cu[it.x + 1] - cu[it.x];
@@ -507,11 +524,22 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
   __shared__ int s_chunk, s_e[GR_ROUTES], s_rank[GR_ROUTES], s_gcnt[GR_GROUPS][E];
   __shared__ int s_cnt[E], s_excl[E], s_tot[E];
   __shared__ int s_red[GR_WARPS][E];
+  // the layer's LayerNorm2 and gate parameters, read before the wait for the
+  // previous kernel (they are not its outputs) so that their first reads on
+  // this SM do not sit on the path from x1 to the routes
+  __shared__ __align__(16) float s_wg[E * D], s_g[D], s_b[D];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < E * D / 4; i += blockDim.x)
+    reinterpret_cast<float4*>(s_wg)[i] = __ldg(reinterpret_cast<const float4*>(wg) + i);
+  for (int i = threadIdx.x; i < D / 4; i += blockDim.x) {
+    reinterpret_cast<float4*>(s_g)[i] = __ldg(reinterpret_cast<const float4*>(g) + i);
+    reinterpret_cast<float4*>(s_b)[i] = __ldg(reinterpret_cast<const float4*>(b) + i);
+  }
+  const float bias_mine = bg ? __ldg(bg + (lane >> 2)) : 0.f;
   pdl_wait();  // x1 comes from the previous kernel
   pdl_trigger();  // dependents launch once this grid has passed its own wait
   if (has_error(err)) return;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) s_chunk = atomicAdd(lb, 1);
   __syncthreads();
   const int c = s_chunk;
@@ -534,14 +562,14 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
     }
   }
 #pragma unroll
-  for (int j = 0; j < GR_TPW; ++j) layer_norm16<float>(v[j], g, b, lane);
+  for (int j = 0; j < GR_TPW; ++j) layer_norm16<float, true>(v[j], s_g, s_b, lane);
   // the 8 logits of every token: each weight load serves the warp's tokens
   float acc[GR_TPW][E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     float4 w4[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) w4[q] = __ldg(reinterpret_cast<const float4*>(wg + e * D + q * 128 + lane * 4));
+    for (int q = 0; q < 4; ++q) w4[q] = *reinterpret_cast<const float4*>(s_wg + e * D + q * 128 + lane * 4);
 #pragma unroll
     for (int j = 0; j < GR_TPW; ++j) {
       float s = 0.f;
@@ -552,7 +580,6 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
       acc[j][e] = s;
     }
   }
-  const float bias_mine = bg ? __ldg(bg + (lane >> 2)) : 0.f;
   int e0s[GR_TPW], e1s[GR_TPW];
 #pragma unroll
   for (int j = 0; j < GR_TPW; ++j) {

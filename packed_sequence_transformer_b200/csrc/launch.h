@@ -131,8 +131,12 @@ int launch_embag_ln(const RepTables& tb, const int64_t* ids, const int64_t* off,
 
 // gemm_tc.cu (bf16, tcgen05).  QKV and the output projection run on CTA
 // pairs: their B (weight) tensor maps have boxes of BN/2 rows.
+// pf0 / pf1 (nullable): weights of later kernels of the layer that the QKV
+// GEMM's CTAs bring into L2 before their inputs are ready
 int launch_gemm_qkv(const CUtensorMap& xn, const CUtensorMap& w, const CUtensorMap& qkv_out,
-                    const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st);
+                    const float* bias, void* qkv, int T, int32_t* err, cudaStream_t st,
+                    const void* pf0 = nullptr, size_t pf0_bytes = 0, const void* pf1 = nullptr,
+                    size_t pf1_bytes = 0);
 int launch_gemm_out(const CUtensorMap& attn, const CUtensorMap& w, const CUtensorMap& x1_out,
                     const float* bias, const void* x, void* x1, int T, int32_t* err, cudaStream_t st);
 // RepEncoder Linear: out [T][512] = normed [T][14336] W^T + b (256 x 256 pair tiles)
