@@ -20,9 +20,14 @@ constexpr int QKV_N = 3 * D;       // 1536
 constexpr int ATT_BLK = 128;       // query / key block of the jagged attention
 constexpr int MOE_BM = 256;        // rows per expert tile (padding granule; one CTA pair's M)
 constexpr int ROUTE_CHUNK = 256;   // routes per route-builder block (= 128 tokens)
-constexpr int GR_WARPS = 12;       // warps per block of the fused gate + route kernel
-constexpr int GR_TPW = 4;          // tokens per warp of that kernel
-constexpr int GR_TOK = GR_WARPS * GR_TPW;  // tokens per block (one chunk of routes)
+// The fused gate + route kernel: GR_TPW tokens per warp, blocks of
+// GR_WARPS_SMALL warps when every chunk fits one wave on the SMs (more SMs
+// busy), else GR_WARPS warps (fewer chunks to look back over).
+constexpr int GR_WARPS = 16;
+constexpr int GR_WARPS_SMALL = 12;
+constexpr int GR_TPW = 4;
+constexpr int GR_TOK = GR_WARPS * GR_TPW;              // tokens per chunk (large blocks)
+constexpr int GR_TOK_SMALL = GR_WARPS_SMALL * GR_TPW;  // tokens per chunk (small blocks)
 constexpr int ATT_MAX_CTAS = 1024;  // bound on the persistent attention grid
 constexpr int GEMM2_BN = 256;      // expert GEMM2 output columns per tile
 constexpr int MOE1_NT = F / 256;   // expert GEMM1 column tiles per M tile (256 wide)
@@ -68,7 +73,7 @@ struct WsLayout {
   int64_t T;
   int32_t U;
   int64_t max_items, max_levels, n_chunks, max_tiles, padded_rows;
-  int64_t n_gchunks;  // fused gate + route chunks (GR_TOK tokens each)
+  int64_t n_gchunks;  // fused gate + route chunks (at most, GR_TOK_SMALL tokens each)
   int64_t cap;        // fused path: expert e's rows start at e * cap (T rounded up to MOE_BM)
 };
 
@@ -94,7 +99,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->max_levels = (T + ATT_BLK - 1) / ATT_BLK + 1;
   L->n_chunks = (2 * T + ROUTE_CHUNK - 1) / ROUTE_CHUNK + 1;
   L->max_tiles = (2 * T + MOE_BM - 1) / MOE_BM + E + 1;
-  L->n_gchunks = (T + GR_TOK - 1) / GR_TOK + 1;
+  L->n_gchunks = (T + GR_TOK_SMALL - 1) / GR_TOK_SMALL + 1;  // the smaller chunks
   L->cap = (T + MOE_BM - 1) / MOE_BM * MOE_BM;
   // expert rows: compact-padded (route builder) or at fixed e * cap (fused path)
   L->padded_rows = 2 * T + E * MOE_BM;

@@ -99,11 +99,15 @@ struct PairCfg {
   // columns staged (and stored) at a time: the fp32 output of a wide tile
   // goes out in two 128-column parts through one 64 KB staging buffer
   static constexpr int PART = (MODE == G_OUT && BN > 128) ? 128 : BN;
-  static constexpr int STAGING = 128 * PART * OUT_ELEM;
+  // bf16 tiles 256 wide stage in two rounds of 128 columns (one 64-column
+  // box per column half) through a 32 KB buffer: two more operand stages fit
+  static constexpr bool HALF_STG = MODE != G_OUT && BN == 256;
+  static constexpr int STAGING = HALF_STG ? 128 * 128 * 2 : 128 * PART * OUT_ELEM;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = (BN / 2) * 64 * 2;
-  // bias (+ FP8: the weight rows' scales), double-buffered by tile
-  static constexpr int BIAS = 2 * (MODE == G_FP8 ? 2 : 1) * BN * 4;
+  // FP8: the bias and the weight rows' scales, double-buffered by tile (the
+  // other modes read the bias through L1)
+  static constexpr int BIAS = MODE == G_FP8 ? 2 * 2 * BN * 4 : 0;
   static constexpr int USABLE = 232448 - 1024 - 256 - 64;
   static constexpr int STAGES_FIT = (USABLE - STAGING - BIAS) / (A_BYTES + B_BYTES);
   static constexpr int STAGES = STAGES_FIT > 10 ? 10 : STAGES_FIT;
@@ -367,16 +371,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         bool second;
         decode_pair_tile<BN, MODE>(p, tile, n_mt, expert, m0, n0, second, mt);
         m0 += 128 * int(cr);
-        if (!mbar_wait(stg_full, jj & 1)) {
-          set_error(p.err, PTL_ERR_TIMEOUT);
-          break;
-        }
         const CUtensorMap* mo = second ? &tmOut2 : &tmOut;
+        constexpr int ROUNDS = Cfg::HALF_STG ? 2 : 1;
+        bool stored = true;
+        for (int rd = 0; rd < ROUNDS; ++rd) {
+          if (!mbar_wait(stg_full, (ROUNDS * jj + rd) & 1)) {
+            set_error(p.err, PTL_ERR_TIMEOUT);
+            stored = false;
+            break;
+          }
+          if constexpr (Cfg::HALF_STG) {
+            // slot s holds box 2 s + rd of the tile (64 columns each)
+            tma_store_2d(mo, sOut, n0 + rd * 64, m0);
+            tma_store_2d(mo, sOut + 16384, n0 + (2 + rd) * 64, m0);
+          } else {
 #pragma unroll 1
-        for (int bx = 0; bx < BN / Cfg::BOX_COLS; ++bx) tma_store_2d(mo, sOut + bx * 16384, n0 + bx * Cfg::BOX_COLS, m0);
-        tma_store_commit();
-        tma_store_wait_read();
-        mbar_arrive(stg_empty);
+            for (int bx = 0; bx < BN / Cfg::BOX_COLS; ++bx)
+              tma_store_2d(mo, sOut + bx * 16384, n0 + bx * Cfg::BOX_COLS, m0);
+          }
+          tma_store_commit();
+          tma_store_wait_read();
+          mbar_arrive(stg_empty);
+        }
+        if (!stored) break;
         if (MODE == G_MOE12 && !second) {
           tma_store_wait_all();
           fence_proxy_async_global();
@@ -407,7 +424,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                                   : nullptr;
       const bool relu = MODE == G_MOE1 || (MODE == G_MOE12 && !second);
       static_assert(BN <= 32 * 2 * GEMM_EPI_WARPS, "one bias value per epilogue thread");
-      const float bv = (bb && et < BN) ? __ldg(bb + et) : 0.f;
+      const float bv = (MODE == G_FP8 && bb && et < BN) ? __ldg(bb + et) : 0.f;
       const float swv = (MODE == G_FP8 && et < BN) ? __ldg(p.sw + n0 + et) : 0.f;
       const float sxr = (MODE == G_FP8 && row < p.M) ? __ldg(p.sx + row) : 0.f;
       constexpr int PART = Cfg::PART, NPART = BN / PART;
@@ -432,9 +449,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       // passed only once every thread has finished tile j - 1, which read
       // the other buffer
       float* const sb = s_bias + (j & 1) * (Cfg::BIAS / 8);
-      if (et < BN) sb[et] = bv;
-      if (MODE == G_FP8 && et < BN) sb[BN + et] = swv;
-      named_barrier(1, 32 * GEMM_EPI_WARPS);
+      if (MODE == G_FP8 && et < BN) {
+        sb[et] = bv;
+        sb[BN + et] = swv;
+      }
+      if (MODE == G_FP8 || MODE == G_OUT) named_barrier(1, 32 * GEMM_EPI_WARPS);
       if (!mbar_wait(&tfull[acc], (j >> 1) & 1)) {
         set_error(p.err, PTL_ERR_TIMEOUT);
         break;
@@ -455,7 +474,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 b4 = *reinterpret_cast<const float4*>(sb + col + 4 * q);
+          // the bias of 32 columns: the same addresses for the whole warp
+          // (16-byte aligned: the entry points check the bias pointers)
+          const float4 b4 = MODE == G_FP8 ? *reinterpret_cast<const float4*>(sb + col + 4 * q)
+                            : bb          ? __ldg(reinterpret_cast<const float4*>(bb + col + 4 * q))
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
           v[4 * q] += b4.x;
           v[4 * q + 1] += b4.y;
           v[4 * q + 2] += b4.z;
@@ -467,48 +490,63 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       };
       if constexpr (MODE != G_OUT) {
-        // bf16 output: this thread's columns go through registers first, so
-        // the accumulator is released (and the tensor core can start the
-        // tile after next) before the staging tile is waited for
-        uint32_t pk[CPG][16];
+        // bf16 output, staged in one round (the whole tile) or two of 128
+        // columns (a box from each column half; column half eg writes slot
+        // eg).  A round's columns go through registers first; after the last
+        // round's TMEM reads the accumulator is released (the tensor core can
+        // start the tile after next) before the staging tile is waited for.
+        constexpr int ROUNDS = Cfg::HALF_STG ? 2 : 1, CPR = CPG / ROUNDS;
+        static_assert(!Cfg::HALF_STG || CPG == 4, "half staging: two boxes per column half");
+        bool staged = true;
 #pragma unroll
-        for (int cc = 0; cc < CPG; ++cc) {
-          const int col = 32 * (eg * CPG + cc);  // column within the tile
-          uint32_t raw[32];
-          tmem_ld32(taddr + col, raw);
-          tmem_ld_wait_regs(raw);
-          float v[32];
+        for (int rd = 0; rd < ROUNDS; ++rd) {
+          uint32_t pk[CPR][16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-          finish32(v, col);
+          for (int k = 0; k < CPR; ++k) {
+            const int col = 32 * (eg * CPG + rd * CPR + k);  // column within the tile
+            uint32_t raw[32];
+            tmem_ld32(taddr + col, raw);
+            tmem_ld_wait_regs(raw);
+            float v[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[cc][i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        }
-        // this warp's rows of the accumulator are read: release it on CTA 0
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
-        // the previous tile's stores have read the staging tile
-        if (j > 0 && !mbar_wait(stg_empty, (j - 1) & 1)) {
-          set_error(p.err, PTL_ERR_TIMEOUT);
-          break;
-        }
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+            finish32(v, col);
 #pragma unroll
-        for (int cc = 0; cc < CPG; ++cc) {
-          // 32 bf16 = half a box row: box c/2, 16-byte chunks (c%2)*4 .. +3
-          const int c = eg * CPG + cc;
-          const uint32_t rowa = smem_u32(sOut + (c >> 1) * 16384) + r * 128;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = (c & 1) * 4 + q;
-            st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pk[cc][4 * q], pk[cc][4 * q + 1], pk[cc][4 * q + 2],
-                         pk[cc][4 * q + 3]);
+            for (int i = 0; i < 16; ++i) pk[k][i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
           }
+          if (rd == ROUNDS - 1) {
+            // this warp's rows of the accumulator are read: release it on CTA 0
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0 + uint32_t(acc) * 8u);
+          }
+          // the previous round's stores have read the staging tile
+          const int R = ROUNDS * j + rd;
+          if (R > 0 && !mbar_wait(stg_empty, (R - 1) & 1)) {
+            set_error(p.err, PTL_ERR_TIMEOUT);
+            staged = false;
+            break;
+          }
+#pragma unroll
+          for (int k = 0; k < CPR; ++k) {
+            // 32 bf16 = half a box row: 16-byte chunks (c%2)*4 .. +3 of box
+            // c/2 (whole tile) or of slot eg (half staging)
+            const int c = eg * CPG + rd * CPR + k;
+            const int box = Cfg::HALF_STG ? eg : (c >> 1);
+            const uint32_t rowa = smem_u32(sOut + box * 16384) + r * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int chunk = (c & 1) * 4 + q;
+              st_shared_v4(rowa + ((chunk ^ (r & 7)) << 4), pk[k][4 * q], pk[k][4 * q + 1], pk[k][4 * q + 2],
+                           pk[k][4 * q + 3]);
+            }
+          }
+          // staged: hand the round to the store thread (one arrival per warp)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(stg_full);
         }
-        // staged: hand the tile to the store thread (one arrival per warp)
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(stg_full);
+        if (!staged) break;
       } else {
 #pragma unroll 1
         for (int pt = 0; pt < NPART; ++pt) {

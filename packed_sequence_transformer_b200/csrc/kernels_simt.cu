@@ -494,12 +494,13 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
 
 // ------------------------------------------------------- gate + route
 // The layer path's gate and route builder in one kernel (bf16 build).  A
-// block takes the next chunk of GR_TOK tokens (a ticket, so chunks start in
-// order); each warp runs the gate for GR_TPW consecutive tokens at once (the
-// x1 rows of all of them in flight together; each gate-weight load, read
-// through L1, serves all of them): LayerNorm2 in fp32, the 8 logits in fp32,
+// block of WARPS warps takes the next chunk of WARPS * GR_TPW tokens (a
+// ticket, so chunks start in order); each warp runs the gate for GR_TPW
+// consecutive tokens at once (the x1 rows of all of them in flight together;
+// the LayerNorm2 and gate parameters, staged in shared memory before the
+// wait for x1, serve all of them): LayerNorm2 in fp32, the 8 logits in fp32,
 // the top-2 logits (ties to the lower index) and the renormalised weights.
-// The chunk's 2*GR_TOK routes are then ranked per expert (stable: ascending
+// The chunk's routes are then ranked per expert (stable: ascending
 // route id r = 2t + k), the chunk publishes its counts (flag 1) and sums the
 // published counts of every earlier chunk (one thread per earlier chunk, in
 // parallel; an earlier chunk's block took its ticket first, so it is running
@@ -511,19 +512,20 @@ __global__ void __launch_bounds__(GATE_WARPS * 32) gate_kernel(
 // offsets.  Waits on predecessors are bounded (PTL_ERR_TIMEOUT).
 // lb: [0] ticket, then per chunk 32 ints: [0] flag, [4..11] counts; all
 // zero before the kernel.
-constexpr int GR_ROUTES = 2 * GR_TOK;
-constexpr int GR_GROUPS = GR_ROUTES / 32;  // 32-route groups ranked by one warp each
-static_assert(GR_ROUTES % 32 == 0 && GR_GROUPS <= GR_WARPS, "route groups");
-
-__global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
     const float* __restrict__ x1, const float* __restrict__ g, const float* __restrict__ b,
     const float* __restrict__ wg, const float* __restrict__ bg, int32_t* __restrict__ idx,
     float* __restrict__ wout, int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ xperm, int cap,
     int32_t* __restrict__ lb, int2* __restrict__ tiles, int32_t* __restrict__ meta,
     int32_t* __restrict__ moe_done, int T_, int32_t* err) {
-  __shared__ int s_chunk, s_e[GR_ROUTES], s_rank[GR_ROUTES], s_gcnt[GR_GROUPS][E];
+  constexpr int TOK = WARPS * GR_TPW;      // tokens of a chunk
+  constexpr int ROUTES = 2 * TOK;
+  constexpr int GROUPS = ROUTES / 32;      // 32-route groups ranked by one warp each
+  static_assert(ROUTES % 32 == 0 && GROUPS <= WARPS, "route groups");
+  __shared__ int s_chunk, s_e[ROUTES], s_rank[ROUTES], s_gcnt[GROUPS][E];
   __shared__ int s_cnt[E], s_excl[E], s_tot[E];
-  __shared__ int s_red[GR_WARPS][E];
+  __shared__ int s_red[WARPS][E];
   // the layer's LayerNorm2 and gate parameters, read before the wait for the
   // previous kernel (they are not its outputs) so that their first reads on
   // this SM do not sit on the path from x1 to the routes
@@ -543,8 +545,8 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
   if (threadIdx.x == 0) s_chunk = atomicAdd(lb, 1);
   __syncthreads();
   const int c = s_chunk;
-  const int nchunks = (T_ + GR_TOK - 1) / GR_TOK;
-  const int t0 = c * GR_TOK + warp * GR_TPW;  // this warp's first token
+  const int nchunks = (T_ + TOK - 1) / TOK;
+  const int t0 = c * TOK + warp * GR_TPW;  // this warp's first token
   // the x1 rows of the warp's tokens (fp32 lane layout: 4 groups of 4
   // consecutive columns at q*128 + lane*4), all loads issued together
   float v[GR_TPW][16];
@@ -626,7 +628,7 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
   }
   __syncthreads();
   // stable ranks inside each 32-route group and the groups' counts
-  if (warp < GR_GROUPS) {
+  if (warp < GROUPS) {
     const int q = 32 * warp + lane;
     const int e = s_e[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
@@ -643,7 +645,7 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
   if (threadIdx.x < E) {
     int n = 0;
 #pragma unroll
-    for (int gq = 0; gq < GR_GROUPS; ++gq) n += s_gcnt[gq][threadIdx.x];
+    for (int gq = 0; gq < GROUPS; ++gq) n += s_gcnt[gq][threadIdx.x];
     s_cnt[threadIdx.x] = n;
     me[4 + threadIdx.x] = n;
     __threadfence();
@@ -681,7 +683,7 @@ __global__ void __launch_bounds__(GR_WARPS * 32, 1) gate_route_kernel(
     const int e = threadIdx.x;
     int excl = 0;
 #pragma unroll
-    for (int w = 0; w < GR_WARPS; ++w) excl += s_red[w][e];
+    for (int w = 0; w < WARPS; ++w) excl += s_red[w][e];
     s_excl[e] = excl;
     s_tot[e] = excl + s_cnt[e];
   }
@@ -1494,13 +1496,19 @@ int launch_gate(const void* x1, const float* g, const float* b, const float* wg,
 
 int launch_gate_route(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                       int T, const WsLayout& L, char* ws, cudaStream_t st) {
-  const int blocks = (T + GR_TOK - 1) / GR_TOK;
-  if (launch_k(gate_route_kernel, dim3(blocks), dim3(GR_WARPS * 32), 0, st, static_cast<const float*>(x1), g, b,
-               wg, bg, reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<float*>(ws + L.wgt),
-               reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<__nv_bfloat16*>(ws + L.xperm),
-               int(L.cap), reinterpret_cast<int32_t*>(ws + L.lb), reinterpret_cast<int2*>(ws + L.tiles),
-               reinterpret_cast<int32_t*>(ws + L.route_meta), reinterpret_cast<int32_t*>(ws + L.moe_done), T,
-               reinterpret_cast<int32_t*>(ws + L.err)))
+  // small chunks when they all fit one wave (one block per SM), so that
+  // more SMs share the work; otherwise larger chunks, fewer to look back over
+  const bool small = (T + GR_TOK_SMALL - 1) / GR_TOK_SMALL <= num_sms();
+  auto go = [&](auto kernel, int warps, int tok) {
+    return launch_k(kernel, dim3((T + tok - 1) / tok), dim3(warps * 32), 0, st, static_cast<const float*>(x1), g, b,
+                    wg, bg, reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<float*>(ws + L.wgt),
+                    reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<__nv_bfloat16*>(ws + L.xperm),
+                    int(L.cap), reinterpret_cast<int32_t*>(ws + L.lb), reinterpret_cast<int2*>(ws + L.tiles),
+                    reinterpret_cast<int32_t*>(ws + L.route_meta), reinterpret_cast<int32_t*>(ws + L.moe_done), T,
+                    reinterpret_cast<int32_t*>(ws + L.err));
+  };
+  if (small ? go(gate_route_kernel<GR_WARPS_SMALL>, GR_WARPS_SMALL, GR_TOK_SMALL)
+            : go(gate_route_kernel<GR_WARPS>, GR_WARPS, GR_TOK))
     return -1;
   return PTL_LAUNCH_CHECK();
 }
