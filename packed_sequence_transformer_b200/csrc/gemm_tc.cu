@@ -211,7 +211,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int expert, m0, n0, mt;
     bool second;
     decode_pair_tile<BN, MODE>(p, pair, 0, expert, m0, n0, second, mt);
-    for (int kb = 0; kb < p.num_kb; ++kb) tma_prefetch_2d(&tmB, kb * (MODE == G_FP8 ? 128 : 64), n0 + int(cr) * (BN / 2));
+    // the first K slices only: a long K (the RepEncoder's 14336) streams
+    // the rest behind them, and 108 CTAs prefetching all of it would flood L2
+    const int npf = p.num_kb < 16 ? p.num_kb : 16;
+    for (int kb = 0; kb < npf; ++kb) tma_prefetch_2d(&tmB, kb * (MODE == G_FP8 ? 128 : 64), n0 + int(cr) * (BN / 2));
   }
   if (warp == 0 && lane == 0) {
     // this CTA's share of the later kernels' weights
