@@ -725,11 +725,11 @@ def run_ours(args):
     with torch.cuda.graph(graph, stream=stream):
         step()
     torch.cuda.synchronize()
-    # work list + layer 0's LayerNorm1 in one launch, 6 kernels per layer (QKV,
-    # attention, out-projection, gate + route, both expert GEMMs in one launch,
-    # combine; each layer's combine writes the next layer's LayerNorm1), head
-    # and its compaction
-    launches_per_step = 1 + 6 * n_layers + (2 if head is not None else 0)
+    # the prologue (work list, the head's output slots, layer 0's LayerNorm1)
+    # in one launch, 6 kernels per layer (QKV, attention, out-projection,
+    # gate + route, both expert GEMMs in one launch, combine; each layer's
+    # combine writes the next layer's LayerNorm1), the head
+    launches_per_step = 1 + 6 * n_layers + (1 if head is not None else 0)
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):

@@ -486,8 +486,9 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
   const bool fuse = c.dt == PTL_BF16;
   if (fuse) {
     // the work list and layer 0's LayerNorm1 of x in one launch
+    // (with a head, also the head's output slots from the prediction mask)
     PTL_TRY(launch_prologue(cu_seqlens, num_users, c.T, c.L, c.ws, x, F32(layers[0].ln1_g), F32(layers[0].ln1_b),
-                            c.ws + c.L.xn, c.st));
+                            c.ws + c.L.xn, c.st, head ? pred_mask : nullptr, head ? n_pred : nullptr));
   } else {
     PTL_TRY(launch_worklist(cu_seqlens, num_users, c.T, c.L, c.ws, c.st));
   }
@@ -502,7 +503,7 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
     h_in = h_out;
   }
   if (head) mark(c.st, PTL_KERNEL_HEAD);
-  if (head) PTL_TRY(launch_head(out, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st));
+  if (head) PTL_TRY(launch_head(out, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st, fuse));
   return PTL_OK;
 }
 

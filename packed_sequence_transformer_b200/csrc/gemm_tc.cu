@@ -98,11 +98,13 @@ struct PairCfg {
   static constexpr int BOX_COLS = 128 / OUT_ELEM;
   // columns staged (and stored) at a time: the fp32 output of a wide tile
   // goes out in two 128-column parts through one 64 KB staging buffer
-  static constexpr int PART = (MODE == G_OUT && BN > 128) ? 128 : BN;
+  // the fp32 output goes out in parts of 64 columns through two 32 KB
+  // buffers, so that a part is staged while the previous one is stored
+  static constexpr int PART = MODE == G_OUT ? 64 : BN;
   // bf16 tiles 256 wide stage in two rounds of 128 columns (one 64-column
   // box per column half) through a 32 KB buffer: two more operand stages fit
   static constexpr bool HALF_STG = MODE != G_OUT && BN == 256;
-  static constexpr int STAGING = HALF_STG ? 128 * 128 * 2 : 128 * PART * OUT_ELEM;
+  static constexpr int STAGING = HALF_STG ? 128 * 128 * 2 : (MODE == G_OUT ? 2 : 1) * 128 * PART * OUT_ELEM;
   static constexpr int A_BYTES = 128 * 64 * 2;
   static constexpr int B_BYTES = (BN / 2) * 64 * 2;
   // FP8: the bias and the weight rows' scales, double-buffered by tile (the
@@ -447,7 +449,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool leader = warp == 2 && lane == 0;
       // the fp32 output stages in parts through the leader's own stores; the
       // bf16 outputs go through the store thread
-      if (MODE == G_OUT && j > 0 && leader) tma_store_wait_read();
       // this tile's bias (+ scales) in buffer j % 2: the barrier below is
       // passed only once every thread has finished tile j - 1, which read
       // the other buffer
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         sb[et] = bv;
         sb[BN + et] = swv;
       }
-      if (MODE == G_FP8 || MODE == G_OUT) named_barrier(1, 32 * GEMM_EPI_WARPS);
+      if (MODE == G_FP8) named_barrier(1, 32 * GEMM_EPI_WARPS);
       if (!mbar_wait(&tfull[acc], (j >> 1) & 1)) {
         set_error(p.err, PTL_ERR_TIMEOUT);
         break;
@@ -553,47 +554,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       } else {
 #pragma unroll 1
         for (int pt = 0; pt < NPART; ++pt) {
-          if (pt > 0) {  // the previous part's store must have read the staging tile
-            load_res(pt);
-            if (leader) tma_store_wait_read();
-            named_barrier(1, 32 * GEMM_EPI_WARPS);
-          }
-          // the accumulator chunks of this thread, one TMEM load ahead: chunk
-          // cc + 1 loads while chunk cc is converted and staged
-          uint32_t rawA[32], rawB[32];
-          tmem_ld32(taddr + pt * PART + 32 * (eg * CPG), rawA);
-          tmem_ld_wait_regs(rawA);
+          // buffer pt % 2 was last staged two parts ago (in this tile or the
+          // previous one): its store must have read it; the previous part's
+          // store may still be running
+          if (pt > 0) load_res(pt);
+          if (leader) tma_store_wait_read_but_one();
+          named_barrier(1, 32 * GEMM_EPI_WARPS);
+          uint8_t* const buf = sOut + (pt & 1) * (Cfg::STAGING / 2);
 #pragma unroll
           for (int cc = 0; cc < CPG; ++cc) {
             const int c = eg * CPG + cc;  // chunk within the part
             const int col = pt * PART + 32 * c;  // column within the tile
-            uint32_t(&raw)[32] = (cc & 1) ? rawB : rawA;
-            uint32_t(&nxt)[32] = (cc & 1) ? rawA : rawB;
-            if (cc + 1 < CPG) tmem_ld32(taddr + col + 32, nxt);
+            uint32_t raw[32];
+            tmem_ld32(taddr + col, raw);
+            tmem_ld_wait_regs(raw);
             float v[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
             finish32(v, col);
-            {
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint4 u = res[4 * cc + q];
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 u = res[4 * cc + q];
+              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float2 f = __bfloat1622float2(h2[i]);
-                  v[8 * q + 2 * i] += f.x;
-                  v[8 * q + 2 * i + 1] += f.y;
-                }
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h2[i]);
+                v[8 * q + 2 * i] += f.x;
+                v[8 * q + 2 * i + 1] += f.y;
               }
-              // 32 fp32 = one 128-byte box row: box c of the part, chunks 0..7
-              const uint32_t rowa = smem_u32(sOut + c * 16384) + r * 128;
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                             __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
             }
-            if (cc + 1 < CPG) tmem_ld_wait_regs(nxt);
+            // 32 fp32 = one 128-byte box row: box c of the part, chunks 0..7
+            const uint32_t rowa = smem_u32(buf + c * 16384) + r * 128;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              st_shared_v4(rowa + ((q ^ (r & 7)) << 4), __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                           __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
           }
           if (pt == NPART - 1) {
             // this warp's rows of the accumulator are read: release it on CTA 0
@@ -607,7 +602,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             const CUtensorMap* mo = second ? &tmOut2 : &tmOut;
 #pragma unroll 1
             for (int bx = 0; bx < PART / Cfg::BOX_COLS; ++bx)
-              tma_store_2d(mo, sOut + bx * 16384, n0 + pt * PART + bx * Cfg::BOX_COLS, m0);
+              tma_store_2d(mo, buf + bx * 16384, n0 + pt * PART + bx * Cfg::BOX_COLS, m0);
             tma_store_commit();
           }
         }

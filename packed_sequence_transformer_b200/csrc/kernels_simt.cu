@@ -165,21 +165,65 @@ __global__ void __launch_bounds__(1024) worklist_kernel(const WorklistArgs w) {
   worklist_body(w);
 }
 
+// Slot of each kept token (mask[t] != 0) in ascending t, -1 for the others,
+// and their count (n_pred, nullable): one block of 1024 threads in one pass,
+// thread i owning the run of tokens [i * run, (i + 1) * run), the block's
+// exclusive prefix of the runs' counts from warp shuffles and the 32 warp
+// totals.  The compaction of the prediction head, taken ahead of it.
+__device__ void head_slots_body(const uint8_t* __restrict__ mask, int32_t* __restrict__ slot,
+                                int32_t* __restrict__ n_pred, int T_) {
+  __shared__ int32_t s_warp[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int run = (T_ + 1023) / 1024;
+  const int t0 = min(tid * run, T_), t1 = min(t0 + run, T_);
+  int cnt = 0;
+  for (int t = t0; t < t1; ++t) cnt += mask[t] ? 1 : 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int tot = s_warp[lane];
+    int winc = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, winc, o);
+      if (lane >= o) winc += v;
+    }
+    s_warp[lane] = winc - tot;  // exclusive prefix of the warp totals
+    if (lane == 31 && n_pred) *n_pred = winc;
+  }
+  __syncthreads();
+  int o = s_warp[warp] + incl - cnt;
+  for (int t = t0; t < t1; ++t) slot[t] = mask[t] ? o++ : -1;
+}
+
 // The once-per-call prologue of the bf16 layer and stack: block 0 builds the
-// attention work list (one block of 1024 threads, as worklist_kernel) while
-// the other blocks apply the first layer's LayerNorm1 to the input rows, one
-// warp per row (the arithmetic of ln_rows_kernel); the two are independent.
+// attention work list (one block of 1024 threads, as worklist_kernel), block
+// 1 takes the prediction head's output slots (with a mask), and the other
+// blocks apply the first layer's LayerNorm1 to the input rows, one warp per row
+// (the arithmetic of ln_rows_kernel); the three are independent.
 __global__ void __launch_bounds__(1024) prologue_kernel(const WorklistArgs w, const __nv_bfloat16* __restrict__ x,
                                                         const float* __restrict__ g, const float* __restrict__ b,
-                                                        __nv_bfloat16* __restrict__ y, int T) {
+                                                        __nv_bfloat16* __restrict__ y, int T,
+                                                        const uint8_t* __restrict__ mask, int32_t* __restrict__ slot,
+                                                        int32_t* __restrict__ n_pred) {
   pdl_wait();
   pdl_trigger();
   if (blockIdx.x == 0) {
     worklist_body(w);
     return;
   }
+  if (blockIdx.x == 1) {
+    if (mask) head_slots_body(mask, slot, n_pred, T);
+    return;
+  }
   const int lane = threadIdx.x & 31;
-  const int row = (blockIdx.x - 1) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int row = (blockIdx.x - 2) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= T) return;
   float v[16];
   Row16<__nv_bfloat16>::load(x + size_t(row) * D, lane, v);
@@ -925,7 +969,8 @@ __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, cons
                                                    const float* __restrict__ b,
                                                    const float* __restrict__ w,
                                                    const float* __restrict__ bias,
-                                                   float* __restrict__ p, int T_) {
+                                                   float* __restrict__ p, int T_,
+                                                   const int32_t* __restrict__ slot) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -940,7 +985,13 @@ __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, cons
   s = warp_sum(s) + (bias ? __ldg(bias) : 0.f);
   if (lane == 0) {
     const float z = fminf(fmaxf(s, -LOGIT_CLAMP), LOGIT_CLAMP);
-    p[t] = 1.0f / (1.0f + expf(-z));
+    const float pr = 1.0f / (1.0f + expf(-z));
+    if (!slot) {
+      p[t] = pr;  // compacted afterwards
+    } else {
+      const int k = slot[t];  // the token's place in the compacted output, or -1
+      if (k >= 0) p[k] = pr;
+    }
   }
 }
 
@@ -1454,10 +1505,11 @@ int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws
 }
 
 int launch_prologue(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, const void* x, const float* g,
-                    const float* b, void* y, cudaStream_t st) {
+                    const float* b, void* y, cudaStream_t st, const uint8_t* pred_mask, int32_t* n_pred) {
   const int ln_blocks = (T + 31) / 32;  // 32 rows (warps) per block
-  if (launch_k(prologue_kernel, dim3(1 + ln_blocks), dim3(1024), 0, st, worklist_args(cu, U, T, L, ws, nullptr),
-               static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T))
+  if (launch_k(prologue_kernel, dim3(2 + ln_blocks), dim3(1024), 0, st, worklist_args(cu, U, T, L, ws, nullptr),
+               static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T, pred_mask,
+               reinterpret_cast<int32_t*>(ws + L.head_p), n_pred))
     return -1;
   return PTL_LAUNCH_CHECK();
 }
@@ -1545,8 +1597,12 @@ int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t
 }
 
 int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, float* probs,
-                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st) {
-  float* p = reinterpret_cast<float*>(ws + L.head_p);
+                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st,
+                bool slots_ready) {
+  // slots ready: each kept token's probability goes straight to its slot of
+  // probs (head_p holds the slots); otherwise into head_p, then compacted
+  float* p = slots_ready ? probs : reinterpret_cast<float*>(ws + L.head_p);
+  const int32_t* slot = slots_ready ? reinterpret_cast<const int32_t*>(ws + L.head_p) : nullptr;
   const int blocks = (T + 7) / 8;
   const float* g = static_cast<const float*>(hw->lnf_g);
   const float* b = static_cast<const float*>(hw->lnf_b);
@@ -1554,11 +1610,13 @@ int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, 
   const float* bias = static_cast<const float*>(hw->b);
   if (dt == PTL_BF16) {
     if (launch_k(head_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(h), g, b, w,
-                                                       bias, p, T)) return -1;
+                                                       bias, p, T, slot)) return -1;
   } else {
-    if (launch_k(head_kernel<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(h), g, b, w, bias, p, T)) return -1;
+    if (launch_k(head_kernel<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(h), g, b, w, bias, p, T,
+                 slot)) return -1;
   }
   if (PTL_LAUNCH_CHECK() != 0) return -1;
+  if (slots_ready) return 0;
   if (launch_k(head_compact_kernel, dim3(1), dim3(1024), 0, st, p, mask, probs, n_pred, T)) return -1;
   return PTL_LAUNCH_CHECK();
 }

@@ -87,10 +87,13 @@ int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws
                     const AttnMask* mask = nullptr);
 int launch_layernorm(const void* x, const float* g, const float* b, void* y, int T, ptl_dtype dt,
                      cudaStream_t st);
-// bf16 layer / stack: the work list (block 0) and the first layer's
+// bf16 layer / stack: the work list (block 0), with a prediction mask each
+// kept token's slot in the head's compacted output and their count (block
+// 1, into the workspace's head_p and *n_pred), and the first layer's
 // LayerNorm1 of x into y (the other blocks) in one launch
 int launch_prologue(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, const void* x, const float* g,
-                    const float* b, void* y, cudaStream_t st);
+                    const float* b, void* y, cudaStream_t st, const uint8_t* pred_mask = nullptr,
+                    int32_t* n_pred = nullptr);
 int launch_gate(const void* x1, const float* g, const float* b, const float* wg, const float* bg,
                 void* xn2, int32_t* idx, float* w, int32_t* chunk_cnt, int T, ptl_dtype dt,
                 cudaStream_t st);
@@ -106,8 +109,11 @@ int launch_route_debug(int T, const WsLayout& L, const char* ws, int32_t* perm, 
 // padded slot of the workspace's xperm
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
                  int32_t* dbg_off, const void* xn2, cudaStream_t st);
+// slots_ready: the prologue already put each kept token's output slot in
+// head_p and the count in *n_pred, so the head writes probs directly
 int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, float* probs,
-                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st);
+                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st,
+                bool slots_ready = false);
 int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const float* bias,
                     const float* R, float* C, int ldc, int M, int N, int Kd, const WsLayout& L,
                     const char* ws, cudaStream_t st);
