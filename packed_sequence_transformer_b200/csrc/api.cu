@@ -340,10 +340,14 @@ ptl_status step_experts(const Call& c, const float* wts, const void* resid, void
       PTL_TRY(launch_gemm_moe2(mh, m2, my, F32(w->b2), c.L, c.ws, c.st));
     }
     mark(c.st, PTL_KERNEL_COMBINE);
+    // after the fused launch, when the combine's blocks fit one wave at 8 per
+    // SM (its waiting blocks then stay few beside the expert launch), the
+    // combine starts on the finished tiles instead of waiting for the launch
+    const bool streamed = fused && (c.T + 7) / 8 <= 8 * num_sms();
     PTL_TRY(launch_combine_bf16(c.ws + c.L.ybuf, at<int32_t>(c, c.L.pos), wts,
                                 static_cast<const float*>(resid), out, c.T,
                                 next ? F32(next->ln1_g) : nullptr, next ? F32(next->ln1_b) : nullptr,
-                                next ? c.ws + c.L.xn : nullptr, c.err, c.st));
+                                next ? c.ws + c.L.xn : nullptr, c.err, c.st, streamed ? &c.L : nullptr, c.ws));
   }
   return PTL_OK;
 }

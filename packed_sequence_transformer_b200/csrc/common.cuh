@@ -31,6 +31,12 @@ constexpr int GR_TOK_SMALL = GR_WARPS_SMALL * GR_TPW;  // tokens per chunk (smal
 constexpr int ATT_MAX_CTAS = 1024;  // bound on the persistent attention grid
 constexpr int GEMM2_BN = 256;      // expert GEMM2 output columns per tile
 constexpr int MOE1_NT = F / 256;   // expert GEMM1 column tiles per M tile (256 wide)
+constexpr int MOE2_NT = D / 256;   // expert GEMM2 column tiles per M tile
+// route_meta (int32 [32], written by the route builder): [0] M tiles, [1..9]
+// expert route offsets, [10..18] expert row bases, [20..27] each expert's first
+// M tile, [31] set (release) once the fused expert GEMMs have their inputs
+constexpr int META_TILE0 = 20;
+constexpr int META_MOE_GO = 31;
 constexpr float LN_EPS = 1e-5f;
 constexpr float LOGIT_CLAMP = 15.0f;
 
@@ -55,7 +61,8 @@ struct WsLayout {
   size_t wgt;         // f32 [T][2]
   size_t chunk_cnt;   // int32 [n_chunks][8]
   size_t lb;          // int32 [32 + 32 * n_gchunks]  fused gate + route: ticket, per-chunk look-back state
-  size_t moe_done;    // int32 [max_tiles][MOE1_NT]  fused expert GEMMs: first-GEMM tiles done (CTAs)
+  size_t moe_done;    // int32 [max_tiles][MOE1_NT] first-GEMM tiles done (CTAs), then
+                      // int32 [max_tiles][MOE2_NT] second-GEMM tiles done (fused expert GEMMs)
   size_t perm;        // int32 [2T]
   size_t pos;         // int32 [2T]          route -> padded expert row
   size_t rowroute;    // int32 [padded_rows]   padded expert rows -> route (or -1)
@@ -122,7 +129,7 @@ __host__ inline bool make_layout(int64_t T, int32_t U, ptl_dtype dt, WsLayout* L
   L->wl_end = o;  // error word + attention work list
   L->chunk_cnt = take(4 * L->n_chunks * E);
   L->lb = take(4 * (32 + 32 * L->n_gchunks));
-  L->moe_done = take(4 * L->max_tiles * MOE1_NT);
+  L->moe_done = take(4 * L->max_tiles * (MOE1_NT + MOE2_NT));
   L->clear_end = o;  // [0, clear_end) is cleared by one memset per call
   L->xn = take(es * T * D);
   L->qkv = take(es * T * QKV_N);

@@ -257,6 +257,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int first_mt = pair / (p.N_total / BN);
   if (is_moe(MODE) && warp == 0 && lane == 0 && first_mt < p.max_mt) first_tl = p.tiles[first_mt];
   __shared__ int s_nmt;
+  if (MODE == G_MOE12 && blockIdx.x == 0 && threadIdx.x == 0) {
+    // the route builder's outputs are complete: the streamed combine that
+    // follows may read them (and wait for this launch's second-GEMM tiles)
+    st_release_gpu(const_cast<int32_t*>(p.meta) + META_MOE_GO, 1);
+  }
   if (threadIdx.x == 0) {
     const int nmt = is_moe(MODE) ? p.meta[0] : 0;
     int nt = is_moe(MODE) ? nmt * (p.N_total / BN) : p.n_tiles_dense;
@@ -399,10 +404,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           mbar_arrive(stg_empty);
         }
         if (!stored) break;
-        if (MODE == G_MOE12 && !second) {
+        if (MODE == G_MOE12) {
+          // count the tile (both CTAs of the pair) once its stores are
+          // complete: first-GEMM tiles for this launch's second GEMM,
+          // second-GEMM tiles for the combine that follows
           tma_store_wait_all();
           fence_proxy_async_global();
-          red_release_gpu_add(p.done + mt * MOE1_NT + n0 / BN, 1);
+          red_release_gpu_add(second ? p.done + p.max_mt * MOE1_NT + mt * MOE2_NT + n0 / BN
+                                     : p.done + mt * MOE1_NT + n0 / BN,
+                              1);
         }
       }
       tma_store_wait_all();

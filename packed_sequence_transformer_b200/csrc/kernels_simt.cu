@@ -562,7 +562,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
     const float* __restrict__ wg, const float* __restrict__ bg, int32_t* __restrict__ idx,
     float* __restrict__ wout, int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ xperm, int cap,
     int32_t* __restrict__ lb, int2* __restrict__ tiles, int32_t* __restrict__ meta,
-    int32_t* __restrict__ moe_done, int T_, int32_t* err) {
+    int32_t* __restrict__ moe_done, int max_tiles, int T_, int32_t* err) {
   constexpr int TOK = WARPS * GR_TPW;      // tokens of a chunk
   constexpr int ROUTES = 2 * TOK;
   constexpr int GROUPS = ROUTES / 32;      // 32-route groups ranked by one warp each
@@ -761,10 +761,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
       const int nt = (s_tot[e] + MOE_BM - 1) / MOE_BM;
       for (int j = threadIdx.x; j < nt; j += blockDim.x) {
         tiles[nt_before + j] = make_int2(e, e * cap + j * MOE_BM);
+        // the fused expert GEMMs' completion counters of both GEMMs
 #pragma unroll
-        for (int q = 0; q < MOE1_NT; ++q)  // the fused expert GEMMs' completion counters
-          moe_done[(nt_before + j) * MOE1_NT + q] = 0;
+        for (int q = 0; q < MOE1_NT; ++q) moe_done[(nt_before + j) * MOE1_NT + q] = 0;
+#pragma unroll
+        for (int q = 0; q < MOE2_NT; ++q) moe_done[max_tiles * MOE1_NT + (nt_before + j) * MOE2_NT + q] = 0;
       }
+      if (threadIdx.x == 0) meta[META_TILE0 + e] = nt_before;
       nt_before += nt;
     }
     if (threadIdx.x == 0) {
@@ -777,6 +780,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
       }
       meta[1 + E] = off;
       meta[10 + E] = E * cap;
+      meta[META_MOE_GO] = 0;
     }
   }
 }
@@ -1143,6 +1147,17 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__
 // (bf16).  One warp per token, 16-byte loads.  Inside a stack, the next
 // layer's LayerNorm1 is applied to the rounded row as well (ln_g != NULL):
 // xn = LN(out) with exactly the arithmetic of the standalone LayerNorm.
+// STREAMED (after the fused expert GEMMs): launched as soon as the expert
+// launch has started, the kernel does not wait for that grid to finish.  A
+// warp first waits for the expert launch to have its inputs (meta[31], set
+// by it once past its own dependency wait: pos and w, from the route
+// builder, are then complete), then for the second-GEMM column tiles of both
+// of its token's routes (their counters reach 2, one per CTA of the pair,
+// released once the tiles' stores are complete), so the combine runs on the
+// SMs the expert launch frees while its last tiles finish.  It waits for the
+// expert grid at its end, so that its own completion still implies that of
+// every earlier kernel.  Waits are bounded (PTL_ERR_TIMEOUT).
+template <bool STREAMED>
 __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* __restrict__ ybuf,
                                                            const int32_t* __restrict__ pos,
                                                            const float* __restrict__ w,
@@ -1151,36 +1166,97 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
                                                            const float* __restrict__ ln_g,
                                                            const float* __restrict__ ln_b,
                                                            __nv_bfloat16* __restrict__ xn,
-                                                           const int32_t* err) {
-  pdl_wait();
+                                                           int32_t* err, const int32_t* __restrict__ meta,
+                                                           const int32_t* __restrict__ done2) {
+  if (!STREAMED) pdl_wait();
   pdl_trigger();
-  if (has_error(err)) return;
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T_) return;
-  const int2 pr = __ldg(reinterpret_cast<const int2*>(pos) + t);
-  const float2 wt = __ldg(reinterpret_cast<const float2*>(w) + t);
-  float y0[16], y1[16], xr[16], o[16];
-  Row16<__nv_bfloat16>::load(ybuf + size_t(pr.x) * D, lane, y0);
-  Row16<__nv_bfloat16>::load(ybuf + size_t(pr.y) * D, lane, y1);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 f = __ldg(reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<__nv_bfloat16>::elem(lane, 4 * q)));
-    xr[4 * q] = f.x;
-    xr[4 * q + 1] = f.y;
-    xr[4 * q + 2] = f.z;
-    xr[4 * q + 3] = f.w;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  bool ok = true;
+  __shared__ int s_ok;
+  static_assert(MOE2_NT == 2, "warp 0's lanes: 8 tokens x 2 routes x 2 column tiles");
+  if (STREAMED) {
+    // warp 0 waits for the whole block (the other warps sleep at the block
+    // barrier, so that waiting blocks take few issue slots and little L2
+    // bandwidth from the expert launch): first for the launch to have its
+    // inputs, then lane l for column tile l % 2 of route (l / 2) % 2 of the
+    // block's token l / 4
+    if (warp == 0) {
+      const uint32_t nap = 256;
+      if (lane == 0 && !sm100::wait_flag_at_least(meta + META_MOE_GO, 1, sm100::kWaitLimitNs, nap)) ok = false;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok && !has_error(err)) {
+        const int tt = blockIdx.x * (blockDim.x >> 5) + (lane >> 2);
+        if (tt < T_) {
+          const int2 pr = __ldcg(reinterpret_cast<const int2*>(pos) + tt);
+          const int slot = (lane & 2) ? pr.y : pr.x;
+          const int cap = __ldcg(meta + 11) - __ldcg(meta + 10);  // expert e's rows start at e * cap
+          const int e = slot / cap;
+          const int mt = __ldcg(meta + META_TILE0 + e) + (slot - e * cap) / MOE_BM;
+          if (!sm100::wait_flag_at_least(done2 + mt * MOE2_NT + (lane & 1), 2, sm100::kWaitLimitNs, nap))
+            ok = false;
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (lane == 0) {
+        if (!ok) set_error(err, PTL_ERR_TIMEOUT);
+        s_ok = ok ? 1 : 0;
+      }
+    }
+    __syncthreads();
+    ok = s_ok != 0;
   }
+  if (ok && t < T_ && !has_error(err)) {
+    const int2 pr = STREAMED ? __ldcg(reinterpret_cast<const int2*>(pos) + t)
+                             : __ldg(reinterpret_cast<const int2*>(pos) + t);
+    const float2 wt = STREAMED ? __ldcg(reinterpret_cast<const float2*>(w) + t)
+                               : __ldg(reinterpret_cast<const float2*>(w) + t);
+    if (ok) {
+      float y0[16], y1[16], xr[16], o[16];
+      if (STREAMED) {
+        // the rows were written by another kernel still running: read them
+        // from L2 (the acquire loads above order these after the stores)
 #pragma unroll
-  for (int j = 0; j < 16; ++j) o[j] = (xr[j] + wt.x * y0[j]) + wt.y * y1[j];
-  Row16<__nv_bfloat16>::store(out + size_t(t) * D, lane, o);
-  if (ln_g != nullptr) {
-    // the values the next layer reads back: o rounded to bf16
+        for (int c = 0; c < 2; ++c) {
+          const uint4 u0 = __ldcg(reinterpret_cast<const uint4*>(ybuf + size_t(pr.x) * D + c * 256 + lane * 8));
+          const uint4 u1 = __ldcg(reinterpret_cast<const uint4*>(ybuf + size_t(pr.y) * D + c * 256 + lane * 8));
+          const __nv_bfloat162* p0 = reinterpret_cast<const __nv_bfloat162*>(&u0);
+          const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&u1);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
-    layer_norm16<__nv_bfloat16>(o, ln_g, ln_b, lane);
-    Row16<__nv_bfloat16>::store(xn + size_t(t) * D, lane, o);
+          for (int i = 0; i < 4; ++i) {
+            const float2 f0 = __bfloat1622float2(p0[i]), f1 = __bfloat1622float2(p1[i]);
+            y0[c * 8 + 2 * i] = f0.x;
+            y0[c * 8 + 2 * i + 1] = f0.y;
+            y1[c * 8 + 2 * i] = f1.x;
+            y1[c * 8 + 2 * i + 1] = f1.y;
+          }
+        }
+      } else {
+        Row16<__nv_bfloat16>::load(ybuf + size_t(pr.x) * D, lane, y0);
+        Row16<__nv_bfloat16>::load(ybuf + size_t(pr.y) * D, lane, y1);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4* src = reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<__nv_bfloat16>::elem(lane, 4 * q));
+        const float4 f = STREAMED ? __ldcg(src) : __ldg(src);
+        xr[4 * q] = f.x;
+        xr[4 * q + 1] = f.y;
+        xr[4 * q + 2] = f.z;
+        xr[4 * q + 3] = f.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) o[j] = (xr[j] + wt.x * y0[j]) + wt.y * y1[j];
+      Row16<__nv_bfloat16>::store(out + size_t(t) * D, lane, o);
+      if (ln_g != nullptr) {
+        // the values the next layer reads back: o rounded to bf16
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
+        layer_norm16<__nv_bfloat16>(o, ln_g, ln_b, lane);
+        Row16<__nv_bfloat16>::store(xn + size_t(t) * D, lane, o);
+      }
+    }
   }
+  if (STREAMED) pdl_wait();
 }
 
 // fp32 build: out[t] = (x1[t] + w[t][0] * y[2t]) + w[t][1] * y[2t+1].
@@ -1556,8 +1632,8 @@ int launch_gate_route(const void* x1, const float* g, const float* b, const floa
                     wg, bg, reinterpret_cast<int32_t*>(ws + L.idx), reinterpret_cast<float*>(ws + L.wgt),
                     reinterpret_cast<int32_t*>(ws + L.pos), reinterpret_cast<__nv_bfloat16*>(ws + L.xperm),
                     int(L.cap), reinterpret_cast<int32_t*>(ws + L.lb), reinterpret_cast<int2*>(ws + L.tiles),
-                    reinterpret_cast<int32_t*>(ws + L.route_meta), reinterpret_cast<int32_t*>(ws + L.moe_done), T,
-                    reinterpret_cast<int32_t*>(ws + L.err));
+                    reinterpret_cast<int32_t*>(ws + L.route_meta), reinterpret_cast<int32_t*>(ws + L.moe_done),
+                    int(L.max_tiles), T, reinterpret_cast<int32_t*>(ws + L.err));
   };
   if (small ? go(gate_route_kernel<GR_WARPS_SMALL>, GR_WARPS_SMALL, GR_TOK_SMALL)
             : go(gate_route_kernel<GR_WARPS>, GR_WARPS, GR_TOK))
@@ -1640,10 +1716,23 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
 }
 
 int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
-                        int T, const float* ln_g, const float* ln_b, void* xn, const int32_t* err,
-                        cudaStream_t st) {
-  if (launch_k(combine_bf16_kernel, dim3((T + 7) / 8), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(ybuf), pos, w, x1,
-               static_cast<__nv_bfloat16*>(out), T, ln_g, ln_b, static_cast<__nv_bfloat16*>(xn), err)) return -1;
+                        int T, const float* ln_g, const float* ln_b, void* xn, int32_t* err,
+                        cudaStream_t st, const WsLayout* streamed_after, const char* ws) {
+  const auto* y = static_cast<const __nv_bfloat16*>(ybuf);
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  auto* n = static_cast<__nv_bfloat16*>(xn);
+  int rc;
+  if (streamed_after) {
+    const WsLayout& L = *streamed_after;
+    const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
+    const int32_t* done2 = reinterpret_cast<const int32_t*>(ws + L.moe_done) + L.max_tiles * MOE1_NT;
+    rc = launch_k(combine_bf16_kernel<true>, dim3((T + 7) / 8), dim3(256), 0, st, y, pos, w, x1, o, T, ln_g, ln_b, n,
+                  err, meta, done2);
+  } else {
+    rc = launch_k(combine_bf16_kernel<false>, dim3((T + 7) / 8), dim3(256), 0, st, y, pos, w, x1, o, T, ln_g, ln_b, n,
+                  err, static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr));
+  }
+  if (rc) return -1;
   return PTL_LAUNCH_CHECK();
 }
 

@@ -117,10 +117,13 @@ int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, 
 int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const float* bias,
                     const float* R, float* C, int ldc, int M, int N, int Kd, const WsLayout& L,
                     const char* ws, cudaStream_t st);
-// ln_g / ln_b / xn: optional (all NULL or none) LayerNorm of the output row into xn
+// ln_g / ln_b / xn: optional (all NULL or none) LayerNorm of the output row into xn.
+// streamed_after (nullable): the fused expert GEMMs of that workspace layout run
+// just before; the combine starts on their finished tiles instead of waiting
+// for the whole launch
 int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
-                        int T, const float* ln_g, const float* ln_b, void* xn, const int32_t* err,
-                        cudaStream_t st);
+                        int T, const float* ln_g, const float* ln_b, void* xn, int32_t* err,
+                        cudaStream_t st, const WsLayout* streamed_after = nullptr, const char* ws = nullptr);
 int launch_combine_f32(const float* y, const float* w, const float* x1, float* out, int T,
                        const int32_t* err, cudaStream_t st);
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,

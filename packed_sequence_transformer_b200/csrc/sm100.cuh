@@ -97,12 +97,12 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
 // `limit_ns`.  Returns false when the limit ran out (the caller records the
 // timeout and unwinds); never spins forever.
 __device__ __forceinline__ bool wait_flag_at_least(const int32_t* flag, int32_t target,
-                                                   uint64_t limit_ns = kWaitLimitNs) {
+                                                   uint64_t limit_ns = kWaitLimitNs, uint32_t sleep_ns = 64) {
   if (ld_acquire_gpu(flag) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   while (ld_acquire_gpu(flag) < target) {
     if (globaltimer_ns() - t0 > limit_ns) return false;
-    __nanosleep(64);
+    __nanosleep(sleep_ns);
   }
   return true;
 }

@@ -118,6 +118,43 @@ def test_runner_host_buffers_and_replay(case):
     r.close()
 
 
+def test_two_runners_on_two_streams_overlap_and_agree(case):
+    """The serving loop of the bench: two runners on two streams, batches
+    alternating between them with no host synchronisation, so that one
+    runner's copies and graph run while the other's graph does.  Every batch's
+    rows and probabilities equal the direct call's bit for bit."""
+    c = case
+    layers = [ptl.to_device_layer(w, "bf16") for w in c.layers]
+    head = ptl.to_device_head(c.head)
+    x, cu, mask, _ = batch(c, 0, 16, "bf16")
+    T = x.shape[0]
+    d_out, d_probs, d_n = direct(c, x, cu, mask, layers, head)
+    k = int(d_n.item())
+    xh, cuh, mh = x.cpu().pin_memory(), cu.cpu().pin_memory(), mask.cpu().pin_memory()
+    lanes = []
+    for _ in range(2):
+        r = ptl.StackRunner(T, 16, layers, "bf16", head=head)
+        r.capture(T)
+        lanes.append((r, torch.cuda.Stream()))
+    results = []
+    for i in range(6):
+        r, s = lanes[i % 2]
+        out_h = torch.empty(T, 512, dtype=torch.bfloat16).pin_memory()
+        probs_h = torch.empty(T, dtype=torch.float32).pin_memory()
+        n_h = torch.zeros(1, dtype=torch.int32).pin_memory()
+        with torch.cuda.stream(s):
+            r.forward(xh, cuh, out=out_h, pred_mask=mh, probs=probs_h, n_pred=n_h, stream=s)
+        results.append((out_h, probs_h, n_h))
+    torch.cuda.synchronize()
+    for r, s in lanes:
+        assert r.last_device_error(s) == 0
+        r.close()
+    for out_h, probs_h, n_h in results:
+        assert int(n_h.item()) == k
+        assert torch.equal(out_h, d_out.cpu())
+        assert torch.equal(probs_h[:k], d_probs[:k].cpu())
+
+
 def test_runner_limits_and_bad_offsets(case):
     c = case
     layers = [ptl.to_device_layer(w, "bf16") for w in c.layers]

@@ -132,7 +132,7 @@ int main() {
       {L.lvl_fill, 4 * (size_t)(L.max_levels + 1), "lvl_fill"}, {L.ulist, 16 * (size_t)L.max_items * H, "ulist"},
       {L.uoff, 8 * ATT_MAX_CTAS, "uoff"}, {L.ucnt, 8 * ATT_MAX_CTAS, "ucnt"},
       {L.chunk_cnt, 4 * (size_t)L.n_chunks * E, "chunk_cnt"}, {L.lb, 4 * (32 + 32 * (size_t)L.n_gchunks), "lb"},
-      {L.moe_done, 4 * (size_t)L.max_tiles * MOE1_NT, "moe_done"},
+      {L.moe_done, 4 * (size_t)L.max_tiles * (MOE1_NT + MOE2_NT), "moe_done"},
       {L.xn, es * T * D, "xn"}, {L.qkv, es * T * QKV_N, "qkv"}, {L.attn, es * T * D, "attn"},
       {L.x1, 4 * T * D, "x1"}, {L.xn2, es * T * D, "xn2"}, {L.act0, es * T * D, "act0"}, {L.act1, es * T * D, "act1"},
       {L.idx, 4 * T * K, "idx"}, {L.wgt, 4 * T * K, "wgt"}, {L.perm, 8 * T, "perm"}, {L.pos, 8 * T, "pos"},
@@ -151,7 +151,8 @@ int main() {
     // the no-alloc scratch holds [0, wl_end): the error word and the work list
     if (L.wl_end < L.ucnt + 8 * ATT_MAX_CTAS || L.wl_end > L.chunk_cnt) bad = "wl_end";
     // one memset per call clears [0, clear_end): up to the fused path's counters
-    if (L.clear_end < L.moe_done + 4 * (size_t)L.max_tiles * MOE1_NT || L.clear_end > L.xn) bad = "clear_end";
+    if (L.clear_end < L.moe_done + 4 * (size_t)L.max_tiles * (MOE1_NT + MOE2_NT) || L.clear_end > L.xn)
+      bad = "clear_end";
     // the fused expert path puts expert e's rows at e * cap
     if ((int64_t)E * L.cap > L.padded_rows || L.cap < T || L.cap % MOE_BM) bad = "cap";
     // the no-alloc entry point's fixed array holds the scratch of every
