@@ -47,7 +47,10 @@
  *     `stream` is a cudaStream_t (NULL = the legacy default stream).
  *   - workspace: a device buffer of at least ptl_workspace_size(T, U, dt)
  *     bytes, 256-byte aligned, used only by the calls that receive it.  Two
- *     calls that run concurrently must not share a workspace.
+ *     calls that run concurrently must not share a workspace.  Its contents
+ *     need no initialisation for the calls (each clears the error word before
+ *     its first launch); ptl_last_device_error on a workspace that no call has
+ *     used reads whatever its first word holds, so zero a new one first.
  *   - Host-checkable problems (NULL pointers, misalignment, sizes, a too
  *     small workspace, an unknown dtype) return a status immediately and
  *     launch nothing.  total_tokens == 0 returns PTL_OK with no launches.

@@ -500,7 +500,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 if ((bits >> i) & 1u) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
             } else if (lc >= 31) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(raw[i]));
+              for (int i = 0; i < 32; i += 2)
+                mx4[(i >> 1) & 3] = fmax3(mx4[(i >> 1) & 3], __uint_as_float(raw[i]), __uint_as_float(raw[i + 1]));
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i)
@@ -537,7 +538,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // pass 2: this half's probabilities -> bf16 pairs in TMEM (P columns
         // 32h..32h+31); masked and skipped keys give p = 0
         if (mine) {
-          float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+          uint64_t ls2[2] = {0ull, 0ull};  // paired partial sums
+          const uint64_t c2x2 = f2_pack(c2, c2), negm = f2_pack(-m, -m);
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {  // keys 32c..32c+31 of the half: P columns 16c..16c+15
             uint32_t raw[32];
@@ -549,8 +551,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const uint32_t bits = c ? vbits[1] : vbits[0];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              float p0 = ex2_approx(__uint_as_float(raw[i]) * c2 - m);
-              float p1 = ex2_approx(__uint_as_float(raw[i + 1]) * c2 - m);
+              const uint64_t xs = f2_fma(f2_pack(__uint_as_float(raw[i]), __uint_as_float(raw[i + 1])), c2x2, negm);
+              float p0, p1;
+              f2_unpack(xs, p0, p1);
+              p0 = ex2_approx(p0);
+              p1 = ex2_approx(p1);
               if constexpr (MASKED) {
                 p0 = ((bits >> i) & 1u) ? p0 : 0.f;
                 p1 = ((bits >> (i + 1)) & 1u) ? p1 : 0.f;
@@ -558,12 +563,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                 p0 = (i <= lc_eff) ? p0 : 0.f;
                 p1 = (i + 1 <= lc_eff) ? p1 : 0.f;
               }
-              ls4[(i >> 1) & 3] += p0 + p1;
+              ls2[(i >> 1) & 1] = f2_add(ls2[(i >> 1) & 1], f2_pack(p0, p1));
               pk[i >> 1] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tP + 16 * c, pk);
           }
-          l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+          float s0, s1, s2, s3;
+          f2_unpack(ls2[0], s0, s1);
+          f2_unpack(ls2[1], s2, s3);
+          l += (s0 + s1) + (s2 + s3);
         } else if (2 * h < nch) {
           uint32_t z[16];
 #pragma unroll

@@ -244,7 +244,8 @@ def alloc_workspace(max_tokens: int, max_users: int, dtype, device="cuda") -> to
     n = workspace_size(max_tokens, max_users, dtype)
     if n == 0:
         raise ValueError("invalid workspace request")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    # zeroed so that the error word reads PTL_OK before any call has used it
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def layer_forward(x, out, cu_seqlens, weights, workspace, debug: Optional[Dict] = None, stream=None):
