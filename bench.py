@@ -60,7 +60,7 @@ NCU_DRAM_BYTES = {
     "gemm_qkv": 25.039616e6 + 0.002304e6,
     "gemm_out": 14.526976e6,
     "gemm_expert1": 31.808000e6 + 4.998912e6,
-    "attention": 21.015552e6 + 0.001024e6,
+    "attention": 21.014784e6,
     "gate": 14.065664e6,
     "combine": 28.072704e6 + 0.000512e6,
 }
