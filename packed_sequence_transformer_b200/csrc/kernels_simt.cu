@@ -120,28 +120,42 @@ __global__ void __launch_bounds__(256) ln_rows_kernel(const TI* __restrict__ x, 
 // so pairs are grouped by b in descending order (any order inside a group).
 // One block of 1024 threads.
 __device__ void block_suffix_exclusive(int32_t* a, int n) {
-  // a[i] <- sum_{j > i} a[j] for i in [0, n), done in chunks of blockDim from
-  // the top so that the running carry flows downward.
-  __shared__ int32_t s_scan[1024];
+  // a[i] <- sum_{j > i} a[j] for i in [0, n), in chunks of blockDim taken from
+  // the top so that the running carry flows downward; inside a chunk, thread
+  // k holds a[top - k] and the chunk is scanned with warp shuffles and one
+  // scan of the warp totals (three block barriers per chunk).
+  __shared__ int32_t s_wtot[32];
   __shared__ int32_t s_carry;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = (blockDim.x + 31) >> 5;
   if (threadIdx.x == 0) s_carry = 0;
-  __syncthreads();
-  for (int base = n - 1; base >= 0; base -= blockDim.x) {
-    const int i = base - int(threadIdx.x);
+  for (int top = n - 1; top >= 0; top -= blockDim.x) {
+    const int i = top - int(threadIdx.x);
     const int32_t v = i >= 0 ? a[i] : 0;
-    s_scan[threadIdx.x] = v;
-    __syncthreads();
-    for (int o = 1; o < int(blockDim.x); o <<= 1) {
-      int32_t t = threadIdx.x >= unsigned(o) ? s_scan[threadIdx.x - o] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += t;
-      __syncthreads();
+    int32_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
-    if (i >= 0) a[i] = s_carry + s_scan[threadIdx.x] - v;
+    if (lane == 31) s_wtot[warp] = incl;
+    __syncthreads();  // (also orders the carry's previous update)
+    if (warp == 0) {
+      const int32_t tot = lane < nwarps ? s_wtot[lane] : 0;
+      int32_t winc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, winc, o);
+        if (lane >= o) winc += t;
+      }
+      s_wtot[lane] = winc - tot;  // exclusive prefix of the warp totals
+    }
     __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) s_carry += s_scan[threadIdx.x];
+    const int32_t carry = s_carry;
+    if (i >= 0) a[i] = carry + s_wtot[warp] + incl - v;
     __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) s_carry = carry + s_wtot[warp] + incl;
   }
+  __syncthreads();
 }
 
 // The work list's arguments (one struct, passed by value).
