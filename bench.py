@@ -285,9 +285,11 @@ def time_rep_leg(T, dev, stream, flush, reps=10, vocab=50_000, max_bag=4, seed=9
 def time_fp8_leg(T, dev, stream, flush, peaks, reps=10, seed=12):
     """The FP8 (e4m3) linear layers on T tokens: per-row quantisation of the
     activations, then the tcgen05 kind::f8f6f4 GEMM at the QKV shape
-    (512 -> 1536) and the expert GEMM1 shape (512 -> 1024), against an e4m3
-    dense peak taken as the measured bf16 peak times the nominal e4m3 / bf16
-    ratio (4.5 / 2.25 PFLOP/s)."""
+    (512 -> 1536), the expert GEMM1 shape (512 -> 1024) and the RepEncoder
+    projection's shape (14336 -> 512, where the contraction is long enough
+    for the MMA rate to show), against an e4m3 dense peak taken as the
+    measured bf16 peak times the nominal e4m3 / bf16 ratio (4.5 / 2.25
+    PFLOP/s)."""
     import torch
 
     from packed_sequence_transformer_b200 import ptl
@@ -299,22 +301,29 @@ def time_fp8_leg(T, dev, stream, flush, peaks, reps=10, seed=12):
            "fp8_peak_source": "measured bf16_tflops burst x 2 (nominal e4m3 / bf16 dense ratio 4.5 / 2.25)"}
     with torch.cuda.stream(stream):
         xq, sx = ptl.quantize_rows_e4m3(x, stream=stream)
-        for name, n_out in (("qkv_512x1536", 1536), ("expert1_512x1024", 1024)):
-            w = (0.02 * torch.randn(n_out, 512, device=dev, generator=g)).to(torch.bfloat16)
+        for name, k_in, n_out in (("qkv_512x1536", 512, 1536), ("expert1_512x1024", 512, 1024),
+                                  ("rep_14336x512", 14336, 512)):
+            if k_in == 512:
+                aq, sa = xq, sx
+            else:
+                xa = torch.randn(T, k_in, device=dev, generator=g).to(torch.bfloat16)
+                aq, sa = ptl.quantize_rows_e4m3(xa, stream=stream)
+                del xa
+            w = (0.02 * torch.randn(n_out, k_in, device=dev, generator=g)).to(torch.bfloat16)
             wq, sw = ptl.quantize_rows_e4m3(w, stream=stream)
             out = torch.empty(T, n_out, dtype=torch.bfloat16, device=dev)
             ms = []
             for i in range(reps + 3):
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                ptl.linear_fp8(xq, sx, wq, sw, None, out, ws, stream=stream)
+                ptl.linear_fp8(aq, sa, wq, sw, None, out, ws, stream=stream)
                 b.record(stream)
                 if i >= 3:
                     ms.append((a, b))
                 flush.fill_(float(i))
             torch.cuda.synchronize()
             us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ms)
-            tf = 2 * T * 512 * n_out / us / 1e6
+            tf = 2 * T * k_in * n_out / us / 1e6
             res[name] = {"us": us, "tflops": tf, "frac_of_fp8_peak": tf / fp8_peak}
         qs = []
         for i in range(reps + 3):

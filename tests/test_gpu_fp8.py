@@ -43,7 +43,8 @@ def test_quantize_rows_bit_exact(dt, rows, cols):
     np.testing.assert_array_equal(_codes_host(codes), want_c)
 
 
-@pytest.mark.parametrize("M,K,N", [(6823, 512, 1536), (300, 512, 1024), (257, 1024, 512), (1, 128, 256)])
+@pytest.mark.parametrize("M,K,N", [(6823, 512, 1536), (300, 512, 1024), (257, 1024, 512), (1, 128, 256),
+                                   (300, 14336, 512)])
 def test_linear_fp8_against_the_oracle(M, K, N):
     rng = np.random.default_rng(M + K + N)
     x = rng.standard_normal((M, K)).astype(np.float32)
