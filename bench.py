@@ -746,7 +746,7 @@ def run_ours(args):
     # in one launch, 6 kernels per layer (QKV, attention, out-projection,
     # gate + route, both expert GEMMs in one launch, combine; each layer's
     # combine writes the next layer's LayerNorm1), the head
-    launches_per_step = 1 + 6 * n_layers + (1 if head is not None else 0)
+    launches_per_step = 1 + 6 * n_layers  # the head runs in the last layer's combine
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):

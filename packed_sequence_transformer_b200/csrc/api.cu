@@ -290,7 +290,8 @@ ptl_status step_gate(const Call& c, const void* x1, void* xn2, int32_t* idx, flo
 // Routes + both expert GEMMs + combine + residual.  The per-chunk expert
 // counts must already be in the workspace.
 ptl_status step_experts(const Call& c, const float* wts, const void* resid, void* out,
-                        const ptl_layer_weights* w, const ptl_layer_weights* next, bool fused = false);
+                        const ptl_layer_weights* w, const ptl_layer_weights* next, bool fused = false,
+                        const HeadArgs* head = nullptr);
 
 // next (bf16 build, nullable): the following layer, whose LayerNorm1 of `out`
 // the combine also writes into the workspace.
@@ -320,9 +321,11 @@ ptl_status step_moe(const Call& c, const void* xn2, const int32_t* idx, const fl
 // (xperm, tiles, meta, pos), then the combine + residual (+ the next layer's
 // LayerNorm1 inside a stack).
 // fused: both expert GEMMs in one launch (the layer path, whose gate +
-// route kernel cleared the per-tile counters).
+// route kernel cleared the per-tile counters).  head (nullable): the last
+// layer of a bf16 stack, whose combine also computes the prediction head.
 ptl_status step_experts(const Call& c, const float* wts, const void* resid, void* out,
-                        const ptl_layer_weights* w, const ptl_layer_weights* next, bool fused) {
+                        const ptl_layer_weights* w, const ptl_layer_weights* next, bool fused,
+                        const HeadArgs* head) {
   {
     CUtensorMap mx, m1, m2, mh, my;
     if (!map_bf16(&mx, c.ws + c.L.xperm, D, c.L.padded_rows, D * 2, 64, 128)) return PTL_ERR_CUDA;
@@ -347,17 +350,19 @@ ptl_status step_experts(const Call& c, const float* wts, const void* resid, void
     PTL_TRY(launch_combine_bf16(c.ws + c.L.ybuf, at<int32_t>(c, c.L.pos), wts,
                                 static_cast<const float*>(resid), out, c.T,
                                 next ? F32(next->ln1_g) : nullptr, next ? F32(next->ln1_b) : nullptr,
-                                next ? c.ws + c.L.xn : nullptr, c.err, c.st, streamed ? &c.L : nullptr, c.ws));
+                                next ? c.ws + c.L.xn : nullptr, c.err, c.st, streamed ? &c.L : nullptr, c.ws,
+                                head));
   }
   return PTL_OK;
 }
 
 // xn_ready: LayerNorm1 of x is already in the workspace; next (nullable,
 // bf16 build): the following layer of a stack, whose LayerNorm1 the combine
-// computes on the way out.
+// computes on the way out; head (nullable, bf16 build): the prediction head,
+// computed by the combine of the stack's last layer.
 ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu,
                       const ptl_layer_weights* w, const ptl_debug_out* dbg, bool xn_ready = false,
-                      const ptl_layer_weights* next = nullptr) {
+                      const ptl_layer_weights* next = nullptr, const HeadArgs* head = nullptr) {
   ptl_status s;
   if ((s = step_qkv(c, x, c.ws + c.L.qkv, w, xn_ready)) != PTL_OK) return s;
   if ((s = step_attention(c, c.ws + c.L.qkv, c.ws + c.L.attn, cu)) != PTL_OK) return s;
@@ -373,7 +378,7 @@ ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu
       mark(c.st, PTL_KERNEL_ROUTE);
       PTL_TRY(launch_route_debug(c.T, c.L, c.ws, dbg->perm, dbg->expert_off, c.st));
     }
-    if ((s = step_experts(c, wts, c.ws + c.L.x1, out, w, next, true)) != PTL_OK) return s;
+    if ((s = step_experts(c, wts, c.ws + c.L.x1, out, w, next, true, head)) != PTL_OK) return s;
   } else {
     if ((s = step_gate(c, c.ws + c.L.x1, c.ws + c.L.xn2, idx, wts, w)) != PTL_OK) return s;
     if ((s = step_moe(c, c.ws + c.L.xn2, idx, wts, c.ws + c.L.x1, out, w, dbg ? dbg->perm : nullptr,
@@ -502,12 +507,21 @@ ptl_status ptl_stack_forward(const void* x, void* out, const int32_t* cu_seqlens
     // bf16: layer i's combine also writes LayerNorm1 of its output for layer
     // i + 1 (layer 0's comes from the prologue)
     const ptl_layer_weights* next = (fuse && i + 1 < num_layers) ? &layers[i + 1] : nullptr;
-    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr, fuse, next)) != PTL_OK)
+    // bf16 with a head: the last layer's combine computes it, each kept
+    // token's probability going to the slot the prologue gave it
+    const HeadArgs hd{head ? F32(head->lnf_g) : nullptr, head ? F32(head->lnf_b) : nullptr,
+                      head ? F32(head->w) : nullptr, head ? F32(head->b) : nullptr, probs,
+                      reinterpret_cast<const int32_t*>(c.ws + c.L.head_p)};
+    const bool head_here = fuse && head && i == num_layers - 1;
+    if ((s = layer_body(c, h_in, h_out, cu_seqlens, &layers[i], nullptr, fuse, next, head_here ? &hd : nullptr)) !=
+        PTL_OK)
       return s;
     h_in = h_out;
   }
-  if (head) mark(c.st, PTL_KERNEL_HEAD);
-  if (head) PTL_TRY(launch_head(out, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st, fuse));
+  if (head && !fuse) {
+    mark(c.st, PTL_KERNEL_HEAD);
+    PTL_TRY(launch_head(out, head, pred_mask, probs, n_pred, c.T, c.dt, c.L, c.ws, c.st));
+  }
   return PTL_OK;
 }
 

@@ -597,10 +597,16 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
     reinterpret_cast<float4*>(s_b)[i] = __ldg(reinterpret_cast<const float4*>(b) + i);
   }
   const float bias_mine = bg ? __ldg(bg + (lane >> 2)) : 0.f;
+  // The chunk ticket is taken before the wait for the previous kernel: the
+  // counter was zeroed by a kernel (or the call's clear) that finished before
+  // this grid could start, and the ticket orders only this grid's blocks
+  // (every block that holds a ticket is resident and will publish, or
+  // returns before any block looks back: on an error from earlier kernels
+  // all of them do).
+  if (threadIdx.x == 0) s_chunk = atomicAdd(lb, 1);
   pdl_wait();  // x1 comes from the previous kernel
   pdl_trigger();  // dependents launch once this grid has passed its own wait
   if (has_error(err)) return;
-  if (threadIdx.x == 0) s_chunk = atomicAdd(lb, 1);
   __syncthreads();
   const int c = s_chunk;
   const int nchunks = (T_ + TOK - 1) / TOK;
@@ -982,13 +988,27 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_kernel(
 }
 
 // ------------------------------------------------------------------ head
+// The prediction head on one row held as 16 fp32 values per lane (the
+// Row16 layout): LayerNorm_f, the dot product with w, + bias, clamp to
+// +-LOGIT_CLAMP, sigmoid; lane 0 writes p[k].
+__device__ __forceinline__ void head_row(float (&v)[16], const HeadArgs& hd, int lane, int k) {
+  layer_norm16<__nv_bfloat16>(v, hd.g, hd.b, lane);
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) s += v[j] * __ldg(hd.w + Row16<__nv_bfloat16>::elem(lane, j));
+  s = warp_sum(s) + (hd.bias ? __ldg(hd.bias) : 0.f);
+  if (lane == 0) {
+    const float z = fminf(fmaxf(s, -LOGIT_CLAMP), LOGIT_CLAMP);
+    hd.probs[k] = 1.0f / (1.0f + expf(-z));
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, const float* __restrict__ g,
                                                    const float* __restrict__ b,
                                                    const float* __restrict__ w,
                                                    const float* __restrict__ bias,
-                                                   float* __restrict__ p, int T_,
-                                                   const int32_t* __restrict__ slot) {
+                                                   float* __restrict__ p, int T_) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
@@ -1003,13 +1023,7 @@ __global__ void __launch_bounds__(256) head_kernel(const T* __restrict__ h, cons
   s = warp_sum(s) + (bias ? __ldg(bias) : 0.f);
   if (lane == 0) {
     const float z = fminf(fmaxf(s, -LOGIT_CLAMP), LOGIT_CLAMP);
-    const float pr = 1.0f / (1.0f + expf(-z));
-    if (!slot) {
-      p[t] = pr;  // compacted afterwards
-    } else {
-      const int k = slot[t];  // the token's place in the compacted output, or -1
-      if (k >= 0) p[k] = pr;
-    }
+    p[t] = 1.0f / (1.0f + expf(-z));  // compacted afterwards
   }
 }
 
@@ -1181,7 +1195,7 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
                                                            const float* __restrict__ ln_b,
                                                            __nv_bfloat16* __restrict__ xn,
                                                            int32_t* err, const int32_t* __restrict__ meta,
-                                                           const int32_t* __restrict__ done2) {
+                                                           const int32_t* __restrict__ done2, const HeadArgs hd) {
   if (!STREAMED) pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1267,6 +1281,15 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
         for (int j = 0; j < 16; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
         layer_norm16<__nv_bfloat16>(o, ln_g, ln_b, lane);
         Row16<__nv_bfloat16>::store(xn + size_t(t) * D, lane, o);
+      } else if (hd.w != nullptr) {
+        // the last layer of a stack: the prediction head on the stored
+        // (bf16-rounded) row, for the tokens the prologue gave a slot
+        const int k = __ldg(hd.slot + t);
+        if (k >= 0) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
+          head_row(o, hd, lane, k);
+        }
       }
     }
   }
@@ -1687,12 +1710,9 @@ int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t
 }
 
 int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, float* probs,
-                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st,
-                bool slots_ready) {
-  // slots ready: each kept token's probability goes straight to its slot of
-  // probs (head_p holds the slots); otherwise into head_p, then compacted
-  float* p = slots_ready ? probs : reinterpret_cast<float*>(ws + L.head_p);
-  const int32_t* slot = slots_ready ? reinterpret_cast<const int32_t*>(ws + L.head_p) : nullptr;
+                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st) {
+  // every token's probability into head_p, then the kept ones compacted
+  float* p = reinterpret_cast<float*>(ws + L.head_p);
   const int blocks = (T + 7) / 8;
   const float* g = static_cast<const float*>(hw->lnf_g);
   const float* b = static_cast<const float*>(hw->lnf_b);
@@ -1700,13 +1720,12 @@ int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, 
   const float* bias = static_cast<const float*>(hw->b);
   if (dt == PTL_BF16) {
     if (launch_k(head_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(h), g, b, w,
-                                                       bias, p, T, slot)) return -1;
+                 bias, p, T)) return -1;
   } else {
-    if (launch_k(head_kernel<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(h), g, b, w, bias, p, T,
-                 slot)) return -1;
+    if (launch_k(head_kernel<float>, dim3(blocks), dim3(256), 0, st, static_cast<const float*>(h), g, b, w, bias, p, T))
+      return -1;
   }
   if (PTL_LAUNCH_CHECK() != 0) return -1;
-  if (slots_ready) return 0;
   if (launch_k(head_compact_kernel, dim3(1), dim3(1024), 0, st, p, mask, probs, n_pred, T)) return -1;
   return PTL_LAUNCH_CHECK();
 }
@@ -1731,7 +1750,8 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
 
 int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
                         int T, const float* ln_g, const float* ln_b, void* xn, int32_t* err,
-                        cudaStream_t st, const WsLayout* streamed_after, const char* ws) {
+                        cudaStream_t st, const WsLayout* streamed_after, const char* ws, const HeadArgs* head) {
+  const HeadArgs hd = head ? *head : HeadArgs{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   const auto* y = static_cast<const __nv_bfloat16*>(ybuf);
   auto* o = static_cast<__nv_bfloat16*>(out);
   auto* n = static_cast<__nv_bfloat16*>(xn);
@@ -1741,10 +1761,10 @@ int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, co
     const int32_t* meta = reinterpret_cast<const int32_t*>(ws + L.route_meta);
     const int32_t* done2 = reinterpret_cast<const int32_t*>(ws + L.moe_done) + L.max_tiles * MOE1_NT;
     rc = launch_k(combine_bf16_kernel<true>, dim3((T + 7) / 8), dim3(256), 0, st, y, pos, w, x1, o, T, ln_g, ln_b, n,
-                  err, meta, done2);
+                  err, meta, done2, hd);
   } else {
     rc = launch_k(combine_bf16_kernel<false>, dim3((T + 7) / 8), dim3(256), 0, st, y, pos, w, x1, o, T, ln_g, ln_b, n,
-                  err, static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr));
+                  err, static_cast<const int32_t*>(nullptr), static_cast<const int32_t*>(nullptr), hd);
   }
   if (rc) return -1;
   return PTL_LAUNCH_CHECK();

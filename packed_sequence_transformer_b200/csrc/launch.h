@@ -109,11 +109,10 @@ int launch_route_debug(int T, const WsLayout& L, const char* ws, int32_t* perm, 
 // padded slot of the workspace's xperm
 int launch_route(const int32_t* idx, int T, const WsLayout& L, char* ws, int32_t* dbg_perm,
                  int32_t* dbg_off, const void* xn2, cudaStream_t st);
-// slots_ready: the prologue already put each kept token's output slot in
-// head_p and the count in *n_pred, so the head writes probs directly
+// The prediction head as its own launches (the fp32 stack and ptl_head):
+// every token's probability into head_p, then the kept ones compacted
 int launch_head(const void* h, const ptl_head_weights* hw, const uint8_t* mask, float* probs,
-                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st,
-                bool slots_ready = false);
+                int32_t* n_pred, int T, ptl_dtype dt, const WsLayout& L, char* ws, cudaStream_t st);
 int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const float* bias,
                     const float* R, float* C, int ldc, int M, int N, int Kd, const WsLayout& L,
                     const char* ws, cudaStream_t st);
@@ -121,9 +120,18 @@ int launch_gemm_f32(int mode, const float* A, int lda, const float* W, const flo
 // streamed_after (nullable): the fused expert GEMMs of that workspace layout run
 // just before; the combine starts on their finished tiles instead of waiting
 // for the whole launch
+// The prediction head computed by the last layer's combine (bf16 stack):
+// LayerNorm_f parameters g, b, the weight row w, bias (nullable), the output
+// probs and each token's slot in it (-1: not predicted).
+struct HeadArgs {
+  const float *g, *b, *w, *bias;
+  float* probs;
+  const int32_t* slot;
+};
 int launch_combine_bf16(const void* ybuf, const int32_t* pos, const float* w, const float* x1, void* out,
                         int T, const float* ln_g, const float* ln_b, void* xn, int32_t* err,
-                        cudaStream_t st, const WsLayout* streamed_after = nullptr, const char* ws = nullptr);
+                        cudaStream_t st, const WsLayout* streamed_after = nullptr, const char* ws = nullptr,
+                        const HeadArgs* head = nullptr);
 int launch_combine_f32(const float* y, const float* w, const float* x1, float* out, int T,
                        const int32_t* err, cudaStream_t st);
 int launch_attn_f32(const float* qkv, float* out, const int32_t* cu, const WsLayout& L,
