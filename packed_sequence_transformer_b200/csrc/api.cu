@@ -247,13 +247,15 @@ ptl_status step_qkv(const Call& c, const void* x, void* qkv, const ptl_layer_wei
   return PTL_OK;
 }
 
+// list_early: a kernel (the QKV projection) runs between the work list and
+// the attention
 ptl_status step_attention(const Call& c, const void* qkv, void* attn, const int32_t* cu,
-                          const AttnMask* mask = nullptr) {
+                          const AttnMask* mask = nullptr, bool list_early = false) {
   if (c.dt == PTL_BF16) {
     CUtensorMap m;
     if (!map_bf16(&m, qkv, QKV_N, c.T, QKV_N * 2, 64, 128)) return PTL_ERR_CUDA;
     mark(c.st, PTL_KERNEL_ATTENTION);
-    PTL_TRY(launch_attn_tc(m, attn, cu, c.L, c.ws, c.st, mask));
+    PTL_TRY(launch_attn_tc(m, attn, cu, c.L, c.ws, c.st, mask, list_early));
   } else {
     mark(c.st, PTL_KERNEL_ATTENTION);
     PTL_TRY(launch_attn_f32(static_cast<const float*>(qkv), static_cast<float*>(attn), cu, c.L, c.ws,
@@ -365,7 +367,7 @@ ptl_status layer_body(const Call& c, const void* x, void* out, const int32_t* cu
                       const ptl_layer_weights* next = nullptr, const HeadArgs* head = nullptr) {
   ptl_status s;
   if ((s = step_qkv(c, x, c.ws + c.L.qkv, w, xn_ready)) != PTL_OK) return s;
-  if ((s = step_attention(c, c.ws + c.L.qkv, c.ws + c.L.attn, cu)) != PTL_OK) return s;
+  if ((s = step_attention(c, c.ws + c.L.qkv, c.ws + c.L.attn, cu, nullptr, true)) != PTL_OK) return s;
   if ((s = step_out(c, c.ws + c.L.attn, x, c.ws + c.L.x1, w)) != PTL_OK) return s;
   int32_t* idx = at<int32_t>(c, c.L.idx);
   float* wts = at<float>(c, c.L.wgt);

@@ -113,8 +113,19 @@ struct StreamPos {
   bool live, nxt_live;
   AttnUnit u, nxt;   // current unit, the next one (looked up one unit ahead)
   const int4* list;  // this stream's units, in order
+  const int4* first;  // its first two entries, read before the dependency wait (shared memory)
   int n_list, k_list;  // list length, next entry to read
   bool q_sent;       // producer: the current unit's Q tile load is issued
+};
+
+// The head of each stream's unit list: its offset, length and first two
+// entries, read into shared memory before the kernel waits for the QKV
+// projection (the work list was complete before this grid could start), so
+// that no chain of dependent loads sits between that wait and the first tile
+// loads.
+struct AttnListHead {
+  int off[2], cnt[2];
+  int4 first[2][2];
 };
 
 // Both streams' step sequences as the producer and the MMA issuer walk them
@@ -126,15 +137,19 @@ struct AttnStepGen {
   __device__ explicit AttnStepGen(const AttnMask& m) : mk(m) {}
   __device__ void fetch_next(StreamPos& sp) {
     sp.nxt_live = sp.k_list < sp.n_list;
-    if (sp.nxt_live) sp.nxt = unit_from<MASKED>(sp.list[sp.k_list++], mk);
+    if (sp.nxt_live) {
+      const int4 d = sp.k_list < 2 ? sp.first[sp.k_list] : sp.list[sp.k_list];
+      ++sp.k_list;
+      sp.nxt = unit_from<MASKED>(d, mk);
+    }
   }
-  __device__ void init_stream(const int4* ulist, const int32_t* uoff, const int32_t* ucnt, int n_ok,
-                              StreamPos& sp, int g) {
+  __device__ void init_stream(const int4* ulist, const AttnListHead& lh, int n_ok, StreamPos& sp, int g) {
     sp.g = g;
     sp.n = 0;
     sp.uc = 0;
-    sp.list = ulist + uoff[2 * blockIdx.x + g];
-    sp.n_list = n_ok ? ucnt[2 * blockIdx.x + g] : 0;
+    sp.list = ulist + lh.off[g];
+    sp.first = lh.first[g];
+    sp.n_list = n_ok ? lh.cnt[g] : 0;
     sp.k_list = 0;
     sp.q_sent = false;
     fetch_next(sp);
@@ -144,9 +159,9 @@ struct AttnStepGen {
     if (sp.live) fetch_next(sp);
   }
   StreamPos a, b;
-  __device__ void init(const int4* ulist, const int32_t* uoff, const int32_t* ucnt, int n_ok) {
-    init_stream(ulist, uoff, ucnt, n_ok, a, 0);
-    init_stream(ulist, uoff, ucnt, n_ok, b, 1);
+  __device__ void init(const int4* ulist, const AttnListHead& lh, int n_ok) {
+    init_stream(ulist, lh, n_ok, a, 0);
+    init_stream(ulist, lh, n_ok, b, 1);
   }
   // advances stream `sp` by one step
   __device__ void step(StreamPos& sp) {
@@ -169,7 +184,8 @@ template <bool MASKED>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const int4* __restrict__ ulist,
                    const int32_t* __restrict__ uoff, const int32_t* __restrict__ ucnt,
-                   __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err, const AttnMask mask) {
+                   __nv_bfloat16* __restrict__ out, int32_t* __restrict__ err, const AttnMask mask,
+                   const int list_early) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // per stream: Q[2 units], K[ATT_KV_STAGES steps], V[1 step], P[2 column blocks]
@@ -196,6 +212,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* x_bar = s_full + 10;                  // [stream] the two softmax halves meet
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 12);
   __shared__ int s_units;
+  __shared__ AttnListHead s_lh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -226,11 +243,25 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  // this CTA's list heads (L2 reads).  list_early: the work list was written
+  // by a kernel that had completed before the one this grid depends on
+  // passed its own wait (the layer path: work list, QKV projection,
+  // attention), so it is read before this grid's wait; otherwise after it.
+  auto read_list_heads = [&]() {
+    const int g = lane;
+    const int off = __ldcg(uoff + 2 * blockIdx.x + g), cnt = __ldcg(ucnt + 2 * blockIdx.x + g);
+    s_lh.off[g] = off;
+    s_lh.cnt[g] = cnt;
+    s_lh.first[g][0] = cnt > 0 ? __ldcg(ulist + off) : make_int4(0, 0, 0, 0);
+    s_lh.first[g][1] = cnt > 1 ? __ldcg(ulist + off + 1) : make_int4(0, 0, 0, 0);
+  };
+  if (list_early && warp == 2 && lane < 2) read_list_heads();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();  // qkv, the work list and the error word come from earlier kernels
+  pdl_wait();  // qkv and the error word come from earlier kernels (and the work list unless list_early)
   pdl_trigger();  // dependents launch once this grid has passed its own wait
+  if (!list_early && warp == 2 && lane < 2) read_list_heads();
   if (threadIdx.x == 0) s_units = has_error(err) ? 0 : 1;
   __syncthreads();
   const int n_ok = s_units;  // 0: an earlier kernel reported an error, no units
@@ -246,7 +277,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       AttnStepGen<MASKED> gen(mask);  // a = stream 0, b = stream 1 (never swapped here)
-      gen.init(ulist, uoff, ucnt, n_ok);
+      gen.init(ulist, s_lh, n_ok);
       // V tiles wait in a small per-stream queue (row of the step's keys,
       // head): V of step n loads once the stream's PV of step n - 1 is done
       int vq0_row[2], vq0_col[2], vq1_row[2], vq1_col[2];  // [queue entry][stream]
@@ -319,7 +350,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int g = warp - 1;
       AttnStepGen<MASKED> gen(mask);
       StreamPos& sp = g == 0 ? gen.a : gen.b;
-      gen.init_stream(ulist, uoff, ucnt, n_ok, sp, g);
+      gen.init_stream(ulist, s_lh, n_ok, sp, g);
       bool ok = true;
       int pvn = -1, pvk16 = 0, pvuc = 0;
       bool pvfirst = false;
@@ -449,14 +480,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       return true;
     };
     int n = 0;  // steps of this stream
-    const int4* list = ulist + uoff[2 * blockIdx.x + g];
-    const int n_list = n_ok ? ucnt[2 * blockIdx.x + g] : 0;
+    const int4* list = ulist + s_lh.off[g];
+    const int n_list = n_ok ? s_lh.cnt[g] : 0;
     int k_list = 0;
-    AttnUnit nxt = k_list < n_list ? unit_from<MASKED>(list[k_list], mask) : AttnUnit{0, 0, 0, 0, 0, 0, 0, 0};
+    AttnUnit nxt = k_list < n_list ? unit_from<MASKED>(s_lh.first[g][0], mask) : AttnUnit{0, 0, 0, 0, 0, 0, 0, 0};
     while (k_list < n_list && ok) {
       const AttnUnit a = nxt;
       ++k_list;
-      if (k_list < n_list) nxt = unit_from<MASKED>(list[k_list], mask);  // prefetch the next unit
+      if (k_list < n_list)  // look the next unit up
+        nxt = unit_from<MASKED>(k_list < 2 ? s_lh.first[g][k_list] : list[k_list], mask);
       const int qi = a.b * ATT_BLK + r;   // query position inside the user
       const int qlim = min(qi, a.L - 1);  // keys 0..qlim are visible
       // masked variant: the row's visible keys as two intervals
@@ -610,7 +642,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
 template <bool MASKED>
 static int launch_attn_tc_t(const CUtensorMap& qkv_map, void* out, const WsLayout& L, char* ws,
-                            cudaStream_t st, const AttnMask& mask) {
+                            cudaStream_t st, const AttnMask& mask, bool list_early) {
   static PerDevice configured;  // the shared-memory limit is a per-device kernel attribute
   if (configured.get([] {
         return cudaFuncSetAttribute(attn_tc_kernel<MASKED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -624,16 +656,17 @@ static int launch_attn_tc_t(const CUtensorMap& qkv_map, void* out, const WsLayou
   if (launch_k(attn_tc_kernel<MASKED>, dim3(grid), dim3(ATT_THREADS), ATT_SMEM, st, qkv_map,
                reinterpret_cast<const int4*>(ws + L.ulist), reinterpret_cast<const int32_t*>(ws + L.uoff),
                reinterpret_cast<const int32_t*>(ws + L.ucnt),
-               static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err), mask) != 0)
+               static_cast<__nv_bfloat16*>(out), reinterpret_cast<int32_t*>(ws + L.err), mask,
+               list_early ? 1 : 0) != 0)
     return -1;
   return cudaPeekAtLastError() == cudaSuccess ? 0 : -1;
 }
 
 int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
-                   char* ws, cudaStream_t st, const AttnMask* mask) {
+                   char* ws, cudaStream_t st, const AttnMask* mask, bool list_early) {
   (void)cu;
-  if (mask) return launch_attn_tc_t<true>(qkv_map, out, L, ws, st, *mask);
-  return launch_attn_tc_t<false>(qkv_map, out, L, ws, st, AttnMask{nullptr, nullptr, 1, 1, 0});
+  if (mask) return launch_attn_tc_t<true>(qkv_map, out, L, ws, st, *mask, list_early);
+  return launch_attn_tc_t<false>(qkv_map, out, L, ws, st, AttnMask{nullptr, nullptr, 1, 1, 0}, list_early);
 }
 
 }  // namespace ptl

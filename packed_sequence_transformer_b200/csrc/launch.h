@@ -178,7 +178,10 @@ int launch_gemm_fp8(const CUtensorMap& xq, const CUtensorMap& wq, const CUtensor
 // attn_tc.cu (bf16, tcgen05)
 // mask (nullable): the HSTU-style variant, over a work list built with the
 // same mask
+// list_early: the work list was written by a kernel that completed before
+// the attention's own predecessor passed its dependency wait (the layer
+// path), so the kernel reads its list heads before its own wait.
 int launch_attn_tc(const CUtensorMap& qkv_map, void* out, const int32_t* cu, const WsLayout& L,
-                   char* ws, cudaStream_t st, const AttnMask* mask = nullptr);
+                   char* ws, cudaStream_t st, const AttnMask* mask = nullptr, bool list_early = false);
 
 }  // namespace ptl
