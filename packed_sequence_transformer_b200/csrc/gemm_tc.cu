@@ -206,17 +206,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   tc_fence_before();
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
+  constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;  // a K slice: one 128-byte swizzle row
+  // Dense modes: the weights of this pair's first tile do not come from the
+  // previous kernel (its activations do), so the first ring stages' B halves
+  // go into shared memory while that kernel finishes (each stage's barrier
+  // expects its A and B bytes now; A follows after the wait) and the next K
+  // slices into L2 (the first 16 only: a long K, the RepEncoder's 14336,
+  // streams the rest behind them, and 108 CTAs prefetching all of it would
+  // flood L2).
+  int pre = 0, pre_m0 = 0;
   if (!is_moe(MODE) && warp == 0 && lane == 0 && pair < p.n_tiles_dense) {
-    // the weights of this pair's first tile do not come from the previous
-    // kernel (its activations do): start pulling them into L2 while that
-    // kernel finishes, they are the loads that may have to come from HBM
     int expert, m0, n0, mt;
     bool second;
     decode_pair_tile<BN, MODE>(p, pair, 0, expert, m0, n0, second, mt);
-    // the first K slices only: a long K (the RepEncoder's 14336) streams
-    // the rest behind them, and 108 CTAs prefetching all of it would flood L2
+    pre = p.num_kb < STAGES ? p.num_kb : STAGES;
+    pre_m0 = m0;
+    const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+    constexpr uint32_t tx = 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES);
+    for (int kb = 0; kb < pre; ++kb) {
+      if (cr == 0) mbar_arrive_expect_tx(&full[kb], tx);
+      tma_load_2d_pair(sB + kb * Cfg::B_BYTES, &tmB, full0 + uint32_t(kb) * 8u, kb * KSLICE, n0 + int(cr) * (BN / 2));
+    }
     const int npf = p.num_kb < 16 ? p.num_kb : 16;
-    for (int kb = 0; kb < npf; ++kb) tma_prefetch_2d(&tmB, kb * (MODE == G_FP8 ? 128 : 64), n0 + int(cr) * (BN / 2));
+    for (int kb = pre; kb < npf; ++kb) tma_prefetch_2d(&tmB, kb * KSLICE, n0 + int(cr) * (BN / 2));
   }
   if (warp == 0 && lane == 0) {
     // this CTA's share of the later kernels' weights
@@ -232,24 +244,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
   pdl_wait();  // inputs, route tables and the error word come from earlier kernels
   pdl_trigger();  // dependents launch once this grid has passed its own wait
-  constexpr int KSLICE = MODE == G_FP8 ? 128 : 64;  // a K slice: one 128-byte swizzle row
-  // Dense modes: the first ring stages of the pair's first tile go out now,
-  // before the error word is read and the block synchronises (their operands
-  // are the caller's buffers, of sizes the host checked), so that the load
-  // latency overlaps that read.
-  int pre = 0;
-  if (!is_moe(MODE) && warp == 0 && lane == 0 && pair < p.n_tiles_dense) {
-    int expert, m0, n0, mt;
-    bool second;
-    decode_pair_tile<BN, MODE>(p, pair, 0, expert, m0, n0, second, mt);
-    pre = p.num_kb < STAGES ? p.num_kb : STAGES;
+  // Dense modes: the A halves of the first ring stages go out now, before the
+  // error word is read and the block synchronises (their operands are the
+  // caller's buffers, of sizes the host checked), so that the load latency
+  // overlaps that read.
+  if (pre > 0) {
     const uint32_t full0 = mapa_shared(smem_u32(full), 0);
-    constexpr uint32_t tx = 2u * uint32_t(Cfg::A_BYTES + Cfg::B_BYTES);
-    for (int kb = 0; kb < pre; ++kb) {
-      if (cr == 0) mbar_arrive_expect_tx(&full[kb], tx);
-      tma_load_2d_pair(sA + kb * Cfg::A_BYTES, &tmA, full0 + uint32_t(kb) * 8u, kb * KSLICE, m0 + 128 * int(cr));
-      tma_load_2d_pair(sB + kb * Cfg::B_BYTES, &tmB, full0 + uint32_t(kb) * 8u, kb * KSLICE, n0 + int(cr) * (BN / 2));
-    }
+    for (int kb = 0; kb < pre; ++kb)
+      tma_load_2d_pair(sA + kb * Cfg::A_BYTES, &tmA, full0 + uint32_t(kb) * 8u, kb * KSLICE, pre_m0 + 128 * int(cr));
   }
   // Expert modes: the pair's first tile entry is read together with the tile
   // count (it is used only if the tile exists)
