@@ -57,12 +57,12 @@ RUNNER_STRIDE = 128  # token granule of the graph runner's buckets in the end-to
 # captured again.
 NCU_DRAM_BYTES = {
     # the QKV launch also brings the layer's expert weights (16.8 MB) into L2
-    "gemm_qkv": 25.039616e6 + 0.002304e6,
-    "gemm_out": 14.526976e6,
-    "gemm_expert1": 31.808000e6 + 4.998912e6,
-    "attention": 21.014784e6,
-    "gate": 14.065664e6,
-    "combine": 28.072704e6 + 0.000512e6,
+    "gemm_qkv": 25.023232e6 + 0.001280e6,
+    "gemm_out": 14.528256e6,
+    "gemm_expert1": 31.805440e6 + 5.067776e6,
+    "attention": 21.017088e6,
+    "gate": 14.062592e6,
+    "combine": 28.080640e6,
 }
 
 
