@@ -1196,34 +1196,33 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
                                                            __nv_bfloat16* __restrict__ xn,
                                                            int32_t* err, const int32_t* __restrict__ meta,
                                                            const int32_t* __restrict__ done2, const HeadArgs hd) {
-  if (!STREAMED) pdl_wait();
-  pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   bool ok = true;
   __shared__ int s_ok;
   static_assert(MOE2_NT == 2, "warp 0's lanes: 8 tokens x 2 routes x 2 column tiles");
-  // streamed: the token's route rows, weights and x1 row come from kernels
-  // that completed before the expert launch passed its dependency wait, so
-  // warps 1..7 read them while warp 0 waits for the expert tiles
+  // The token's route rows, weights and x1 row come from kernels that
+  // completed before the expert launch passed its dependency wait (this
+  // grid starts only after that): every warp reads them first, before this
+  // grid's own wait (or, streamed, while warp 0 waits for the expert tiles).
   int2 pr = make_int2(0, 0);
   float2 wt = make_float2(0.f, 0.f);
   float xr[16];
-  auto load_token = [&]() {
-    pr = STREAMED ? __ldcg(reinterpret_cast<const int2*>(pos) + t) : __ldg(reinterpret_cast<const int2*>(pos) + t);
-    wt = STREAMED ? __ldcg(reinterpret_cast<const float2*>(w) + t) : __ldg(reinterpret_cast<const float2*>(w) + t);
+  if (t < T_) {
+    pr = __ldcg(reinterpret_cast<const int2*>(pos) + t);
+    wt = __ldcg(reinterpret_cast<const float2*>(w) + t);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4* src = reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<__nv_bfloat16>::elem(lane, 4 * q));
-      const float4 f = STREAMED ? __ldcg(src) : __ldg(src);
+      const float4 f =
+          __ldcg(reinterpret_cast<const float4*>(x1 + size_t(t) * D + Row16<__nv_bfloat16>::elem(lane, 4 * q)));
       xr[4 * q] = f.x;
       xr[4 * q + 1] = f.y;
       xr[4 * q + 2] = f.z;
       xr[4 * q + 3] = f.w;
     }
-  };
-  const bool early = STREAMED && warp != 0 && t < T_;
-  if (early) load_token();
+  }
+  if (!STREAMED) pdl_wait();
+  pdl_trigger();
   if (STREAMED) {
     // warp 0 waits for the whole block (the other warps sleep at the block
     // barrier, so that waiting blocks take few issue slots and little L2
@@ -1256,7 +1255,6 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
     ok = s_ok != 0;
   }
   if (ok && t < T_ && !has_error(err)) {
-    if (!early) load_token();
     if (ok) {
       float y0[16], y1[16], o[16];
       if (STREAMED) {
