@@ -606,13 +606,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
   if (threadIdx.x == 0) s_chunk = atomicAdd(lb, 1);
   pdl_wait();  // x1 comes from the previous kernel
   pdl_trigger();  // dependents launch once this grid has passed its own wait
-  if (has_error(err)) return;
   __syncthreads();
   const int c = s_chunk;
   const int nchunks = (T_ + TOK - 1) / TOK;
   const int t0 = c * TOK + warp * GR_TPW;  // this warp's first token
   // the x1 rows of the warp's tokens (fp32 lane layout: 4 groups of 4
-  // consecutive columns at q*128 + lane*4), all loads issued together
+  // consecutive columns at q*128 + lane*4), all loads issued together, and
+  // the error word read beside them (they are in the workspace, valid to
+  // read whatever an earlier kernel reported); the whole block then leaves
+  // together if an earlier kernel reported an error
   float v[GR_TPW][16];
 #pragma unroll
   for (int j = 0; j < GR_TPW; ++j) {
@@ -627,6 +629,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
       v[j][4 * q + 3] = f.w;
     }
   }
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = has_error(err) ? 1 : 0;
+  __syncthreads();
+  if (s_bad) return;
 #pragma unroll
   for (int j = 0; j < GR_TPW; ++j) layer_norm16<float, true>(v[j], s_g, s_b, lane);
   // the 8 logits of every token: each weight load serves the warp's tokens
@@ -712,8 +718,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
     for (int gq = 0; gq < GROUPS; ++gq) n += s_gcnt[gq][threadIdx.x];
     s_cnt[threadIdx.x] = n;
     me[4 + threadIdx.x] = n;
-    __threadfence();
   }
+  // the block barrier orders the eight counts before thread 0's release
+  // store, which makes them visible with the flag (cumulative release)
   __syncthreads();
   if (threadIdx.x == 0) sm100::st_release_gpu(me, 1);
   int part[E];
@@ -1248,13 +1255,15 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const __nv_bfloat16* 
       ok = __all_sync(0xffffffffu, ok);
       if (lane == 0) {
         if (!ok) set_error(err, PTL_ERR_TIMEOUT);
-        s_ok = ok ? 1 : 0;
+        // (an error from an earlier kernel also stops the block, read here
+        // once for all its warps)
+        s_ok = ok && !has_error(err) ? 1 : 0;
       }
     }
     __syncthreads();
     ok = s_ok != 0;
   }
-  if (ok && t < T_ && !has_error(err)) {
+  if (ok && t < T_ && (STREAMED || !has_error(err))) {
     if (ok) {
       float y0[16], y1[16], o[16];
       if (STREAMED) {
