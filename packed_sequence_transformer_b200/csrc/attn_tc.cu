@@ -261,10 +261,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   tc_fence_after();
   pdl_wait();  // qkv and the error word come from earlier kernels (and the work list unless list_early)
   pdl_trigger();  // dependents launch once this grid has passed its own wait
-  if (!list_early && warp == 2 && lane < 2) read_list_heads();
-  if (threadIdx.x == 0) s_units = has_error(err) ? 0 : 1;
-  __syncthreads();
-  const int n_ok = s_units;  // 0: an earlier kernel reported an error, no units
+  // n_ok = 0: an earlier kernel reported an error, no units.  On the layer
+  // path (list_early) the error word is not read here: the lists are either
+  // empty (the work list found bad offsets) or describe valid rows, so the
+  // units run (on whatever an earlier failed kernel left) and the first
+  // tile loads do not wait for that read.
+  if (!list_early) {
+    if (warp == 2 && lane < 2) read_list_heads();
+    if (threadIdx.x == 0) s_units = has_error(err) ? 0 : 1;
+    __syncthreads();
+  }
+  const int n_ok = list_early ? 1 : s_units;
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S[0] 0..127, S[1] 128..255, O[0] 256..319, O[1] 320..383,
   // P[0] 384..447, P[1] 448..511 (bf16 pairs)
