@@ -60,9 +60,9 @@ NCU_DRAM_BYTES = {
     "gemm_qkv": 25.023232e6 + 0.001280e6,
     "gemm_out": 14.528256e6,
     "gemm_expert1": 31.805440e6 + 5.067776e6,
-    "attention": 21.017088e6,
-    "gate": 14.062592e6,
-    "combine": 28.081152e6 + 0.001280e6,
+    "attention": 21.016832e6,
+    "gate": 14.062848e6,
+    "combine": 28.080896e6 + 0.004352e6,
 }
 
 
