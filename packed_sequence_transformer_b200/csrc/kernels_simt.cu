@@ -635,7 +635,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
   if (s_bad) return;
 #pragma unroll
   for (int j = 0; j < GR_TPW; ++j) layer_norm16<float, true>(v[j], s_g, s_b, lane);
-  // the 8 logits of every token: each weight load serves the warp's tokens
+  // the 8 logits of every token: each weight load serves the warp's tokens;
+  // the lane's 16 products summed as two interleaved fp32 partial sums (even
+  // and odd columns) with paired FMAs, then added
   float acc[GR_TPW][E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -644,12 +646,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gate_route_kernel(
     for (int q = 0; q < 4; ++q) w4[q] = *reinterpret_cast<const float4*>(s_wg + e * D + q * 128 + lane * 4);
 #pragma unroll
     for (int j = 0; j < GR_TPW; ++j) {
-      float s = 0.f;
+      uint64_t s2 = 0ull;
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        s += v[j][4 * q] * w4[q].x + v[j][4 * q + 1] * w4[q].y + v[j][4 * q + 2] * w4[q].z +
-             v[j][4 * q + 3] * w4[q].w;
-      acc[j][e] = s;
+      for (int q = 0; q < 4; ++q) {
+        s2 = sm100::f2_fma(sm100::f2_pack(v[j][4 * q], v[j][4 * q + 1]), sm100::f2_pack(w4[q].x, w4[q].y), s2);
+        s2 = sm100::f2_fma(sm100::f2_pack(v[j][4 * q + 2], v[j][4 * q + 3]), sm100::f2_pack(w4[q].z, w4[q].w), s2);
+      }
+      float lo, hi;
+      sm100::f2_unpack(s2, lo, hi);
+      acc[j][e] = lo + hi;
     }
   }
   int e0s[GR_TPW], e1s[GR_TPW];
