@@ -61,7 +61,7 @@ NCU_DRAM_BYTES = {
     "gemm_out": 14.528256e6,
     "gemm_expert1": 31.805440e6 + 5.067776e6,
     "attention": 21.016832e6,
-    "gate": 14.062848e6,
+    "gate": 14.056960e6,
     "combine": 28.080896e6 + 0.004352e6,
 }
 
