@@ -745,8 +745,9 @@ def run_ours(args):
     # the prologue (work list, the head's output slots, layer 0's LayerNorm1)
     # in one launch, 6 kernels per layer (QKV, attention, out-projection,
     # gate + route, both expert GEMMs in one launch, combine; each layer's
-    # combine writes the next layer's LayerNorm1), the head
-    launches_per_step = 1 + 6 * n_layers  # the head runs in the last layer's combine
+    # combine writes the next layer's LayerNorm1, the last one computes the
+    # head)
+    launches_per_step = 1 + 6 * n_layers
 
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
