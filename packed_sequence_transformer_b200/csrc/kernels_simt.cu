@@ -236,13 +236,45 @@ __global__ void __launch_bounds__(1024) prologue_kernel(const WorklistArgs w, co
     if (mask) head_slots_body(mask, slot, n_pred, T);
     return;
   }
+  // LayerNorm1 rows: one grid-wide warp stride (one wave of blocks, so no SM
+  // runs two blocks back to back); each warp keeps its next P rows' loads in
+  // flight as raw bf16 (8 registers a row) while it normalises the current one.
+  constexpr int P = 3;
   const int lane = threadIdx.x & 31;
+  const int W = (gridDim.x - 2) * (blockDim.x >> 5);
   const int row = (blockIdx.x - 2) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= T) return;
-  float v[16];
-  Row16<__nv_bfloat16>::load(x + size_t(row) * D, lane, v);
-  layer_norm16<__nv_bfloat16>(v, g, b, lane);
-  Row16<__nv_bfloat16>::store(y + size_t(row) * D, lane, v);
+  auto load_raw = [&](int r, uint4 (&u)[2]) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + size_t(r) * D);
+    u[0] = __ldg(src + lane);
+    u[1] = __ldg(src + 32 + lane);
+  };
+  uint4 raw[P][2];
+#pragma unroll
+  for (int i = 0; i < P; ++i)
+    if (row + i * W < T) load_raw(row + i * W, raw[i]);
+  for (int base = row; base < T; base += P * W) {
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const int r = base + i * W;
+      if (r < T) {
+        float v[16];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[i][c]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(h[k]);
+            v[c * 8 + 2 * k] = f.x;
+            v[c * 8 + 2 * k + 1] = f.y;
+          }
+        }
+        if (r + P * W < T) load_raw(r + P * W, raw[i]);
+        layer_norm16<__nv_bfloat16>(v, g, b, lane);
+        Row16<__nv_bfloat16>::store(y + size_t(r) * D, lane, v);
+      }
+    }
+  }
 }
 
 // Shared-memory capacities of the work-list build: up to these sizes the
@@ -1640,7 +1672,9 @@ int launch_worklist(const int32_t* cu, int U, int T, const WsLayout& L, char* ws
 
 int launch_prologue(const int32_t* cu, int U, int T, const WsLayout& L, char* ws, const void* x, const float* g,
                     const float* b, void* y, cudaStream_t st, const uint8_t* pred_mask, int32_t* n_pred) {
-  const int ln_blocks = (T + 31) / 32;  // 32 rows (warps) per block
+  // one block per SM (1024 threads of this kernel's register count fill
+  // one): the work list, the head slots and up to SMs - 2 LayerNorm blocks
+  const int ln_blocks = std::min((T + 31) / 32, std::max(1, num_sms() - 2));
   if (launch_k(prologue_kernel, dim3(2 + ln_blocks), dim3(1024), 0, st, worklist_args(cu, U, T, L, ws, nullptr),
                static_cast<const __nv_bfloat16*>(x), g, b, static_cast<__nv_bfloat16*>(y), T, pred_mask,
                reinterpret_cast<int32_t*>(ws + L.head_p), n_pred))
