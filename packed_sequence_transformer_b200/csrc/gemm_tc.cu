@@ -96,9 +96,8 @@ template <int BN, int MODE>
 struct PairCfg {
   static constexpr int OUT_ELEM = MODE == G_OUT ? 4 : 2;
   static constexpr int BOX_COLS = 128 / OUT_ELEM;
-  // columns staged (and stored) at a time: the fp32 output of a wide tile
-  // goes out in two 128-column parts through one 64 KB staging buffer
-  // the fp32 output goes out in parts of 64 columns through two 32 KB
+  // columns staged (and stored) at a time: the fp32 output goes out in
+  // parts of 64 columns through two 32 KB
   // buffers, so that a part is staged while the previous one is stored
   static constexpr int PART = MODE == G_OUT ? 64 : BN;
   // bf16 tiles 256 wide stage in two rounds of 128 columns (one 64-column
