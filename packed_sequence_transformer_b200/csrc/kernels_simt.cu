@@ -238,11 +238,18 @@ __global__ void __launch_bounds__(1024) prologue_kernel(const WorklistArgs w, co
   }
   // LayerNorm1 rows: one grid-wide warp stride (one wave of blocks, so no SM
   // runs two blocks back to back); each warp keeps its next P rows' loads in
-  // flight as raw bf16 (8 registers a row) while it normalises the current one.
-  constexpr int P = 3;
+  // flight as raw bf16 (8 registers a row) while it normalises the current
+  // one, with gamma and beta read from shared memory.
+  constexpr int P = 2;
   const int lane = threadIdx.x & 31;
   const int W = (gridDim.x - 2) * (blockDim.x >> 5);
   const int row = (blockIdx.x - 2) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  __shared__ __align__(16) float s_lg[D], s_lb[D];
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    s_lg[i] = g[i];
+    s_lb[i] = b[i];
+  }
+  __syncthreads();
   if (row >= T) return;
   auto load_raw = [&](int r, uint4 (&u)[2]) {
     const uint4* src = reinterpret_cast<const uint4*>(x + size_t(r) * D);
@@ -270,7 +277,7 @@ __global__ void __launch_bounds__(1024) prologue_kernel(const WorklistArgs w, co
           }
         }
         if (r + P * W < T) load_raw(r + P * W, raw[i]);
-        layer_norm16<__nv_bfloat16>(v, g, b, lane);
+        layer_norm16<__nv_bfloat16, true>(v, s_lg, s_lb, lane);
         Row16<__nv_bfloat16>::store(y + size_t(r) * D, lane, v);
       }
     }
